@@ -1,0 +1,382 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other than
+itself — brute force, a closed form, an invariant, or a library routine
+(torch) computing the same mathematical object a different way."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from dropless_top_mixture_b200.workloads import (WORKLOADS, adversarial_logits, make_inputs)
+
+
+# ---------------------------------------------------------------- router logits
+
+def _bf16(shape, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+
+
+def test_router_logits_bf16_matches_unfused_fp32_sum():
+    # bf16 x bf16 products are exact in fp32, so sequential fmaf equals the
+    # sequential fp32 sum of exact products, computed here with numpy.
+    x = _bf16((37, 96), 1)
+    W = _bf16((11, 96), 2, 0.02)
+    got = O.router_logits(x, W)
+    xf = x.float().numpy()
+    wf = W.float().numpy()
+    acc = np.zeros((37, 11), dtype=np.float32)
+    for j in range(96):
+        acc = (acc + np.outer(xf[:, j], wf[:, j]).astype(np.float32)).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), acc.view(np.uint32))
+
+
+def test_router_logits_error_bound_vs_fp64():
+    # Sequential fp32 accumulation error is at most gamma_d * sum|x_j w_j|.
+    x = torch.randn(64, 128, generator=torch.Generator().manual_seed(3))
+    W = torch.randn(8, 128, generator=torch.Generator().manual_seed(4)) * 0.02
+    got = O.router_logits(x, W).astype(np.float64)
+    ref = x.double().numpy() @ W.double().numpy().T
+    absdot = np.abs(x.double().numpy()) @ np.abs(W.double().numpy()).T
+    u = 2.0 ** -24
+    gamma = 128 * u / (1 - 128 * u)
+    assert np.all(np.abs(got - ref) <= gamma * absdot + 1e-30)
+
+
+def test_router_logits_one_hot_picks_weight_column():
+    W = _bf16((5, 64), 7)
+    x = torch.zeros(64, 64, dtype=torch.bfloat16)
+    x[torch.arange(64), torch.arange(64)] = 1.0
+    got = O.router_logits(x, W)
+    assert np.array_equal(got, W.float().numpy().T)
+
+
+def test_router_logits_fp32_small_integers_exact():
+    g = torch.Generator().manual_seed(9)
+    x = torch.randint(-8, 8, (10, 50), generator=g).float()
+    W = torch.randint(-8, 8, (6, 50), generator=g).float()
+    got = O.router_logits(x, W)
+    assert np.array_equal(got, (x.double() @ W.double().T).float().numpy())
+
+
+# ---------------------------------------------------------------- softmax + top-k
+
+def _brute_topk(row, k):
+    keyed = sorted(range(len(row)), key=lambda e: (-float(row[e]), e))
+    return keyed[:k]
+
+
+@pytest.mark.parametrize("kind", ["constant", "dups", "signed_zero", "normal"])
+@pytest.mark.parametrize("E,k", [(1, 1), (8, 2), (8, 8), (33, 5), (64, 8)])
+def test_topk_matches_brute_force(kind, E, k):
+    lg = adversarial_logits(40, E, kind, seed=E * 10 + k).numpy()
+    idx = O.topk_select(lg, k)
+    for t in range(lg.shape[0]):
+        assert list(idx[t]) == _brute_topk(lg[t], k)
+
+
+def test_topk_matches_torch_topk_without_ties():
+    lg = torch.randn(200, 64, generator=torch.Generator().manual_seed(5))
+    assert len(set(lg.flatten().tolist())) == lg.numel()
+    v, i = torch.topk(lg, 8, dim=1, largest=True, sorted=True)
+    assert np.array_equal(O.topk_select(lg.numpy(), 8), i.numpy())
+
+
+def test_constant_logits_closed_form():
+    E, k = 16, 4
+    idx, gate, probs = O.route(np.full((3, E), 1.5, np.float32), k)
+    assert (idx == np.arange(k)).all()
+    assert np.allclose(gate, 1.0 / E, rtol=0, atol=1e-15)
+
+
+def test_nan_logit_ranks_last():
+    lg = np.array([[np.nan, -100.0, 3.0, -np.inf]], np.float32)
+    assert list(O.topk_select(lg, 4)[0]) == [2, 1, 0, 3]
+
+
+def test_softmax_matches_torch():
+    lg = torch.randn(50, 40, generator=torch.Generator().manual_seed(6)) * 3
+    p = O.softmax_fp64(lg.numpy())
+    assert np.allclose(p, torch.softmax(lg.double(), dim=1).numpy(), rtol=1e-14, atol=0)
+
+
+def test_gates_are_probs_of_selected_and_renorm():
+    lg = torch.randn(30, 12, generator=torch.Generator().manual_seed(8)).numpy()
+    idx, gate, probs = O.route(lg, 3)
+    for t in range(30):
+        for j in range(3):
+            assert gate[t, j] == probs[t, idx[t, j]]
+    assert np.all(np.diff(gate, axis=1) <= 0)  # descending
+    _, g2, _ = O.route(lg, 3, renorm=True)
+    assert np.allclose(g2.sum(1), 1.0, atol=1e-15)
+    _, gall, _ = O.route(lg, 12)
+    assert np.allclose(gall.sum(1), 1.0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- routing metadata
+
+def _brute_slots(idx, E):
+    T, k = idx.shape
+    counts = [0] * E
+    for t in range(T):
+        for j in range(k):
+            counts[idx[t, j]] += 1
+    offs = [0]
+    for e in range(E):
+        offs.append(offs[-1] + counts[e])
+    seen = [0] * E
+    slot = np.zeros_like(idx)
+    for t in range(T):           # token-major walk = stable order
+        for j in range(k):
+            e = idx[t, j]
+            slot[t, j] = offs[e] + seen[e]
+            seen[e] += 1
+    return counts, offs, slot
+
+
+@pytest.mark.parametrize("E,k,T", [(8, 2, 64), (33, 5, 50), (128, 4, 300), (3, 3, 7), (1, 1, 5)])
+def test_metadata_brute_force_and_invariants(E, k, T):
+    lg = adversarial_logits(T, E, "normal", seed=E + T).numpy()
+    # skew: make some experts empty
+    lg[:, E // 2:] -= 5.0 if E > k + 1 else 0.0
+    idx = O.topk_select(lg, k)
+    m = O.routing_metadata(idx, E)
+    counts, offs, slot = _brute_slots(idx, E)
+    assert list(m["counts"]) == counts
+    assert list(m["offsets"]) == offs
+    assert np.array_equal(m["slot"], slot)
+    assert m["counts"].sum() == T * k and m["offsets"][-1] == T * k
+    assert np.all(np.diff(m["offsets"]) >= 0)
+    assert sorted(m["slot"].reshape(-1).tolist()) == list(range(T * k))
+    for e in range(E):  # within an expert, slots increase with t
+        rows = [(t, m["slot"][t, j]) for t in range(T) for j in range(k) if idx[t, j] == e]
+        assert [s for _, s in rows] == sorted(s for _, s in rows)
+    tiles = [(c + 127) // 128 for c in counts]
+    assert list(m["tile_offsets"]) == [0] + list(itertools.accumulate(tiles))
+    assert all(m["row_token"][m["slot"][t, j]] == t for t in range(T) for j in range(k))
+
+
+def test_dispatch_is_bitwise_copy_and_combine_identity_experts():
+    T, E, k, d = 50, 8, 3, 24
+    x = _bf16((T, d), 11)
+    lg = adversarial_logits(T, E, "dups", seed=3).numpy()
+    idx, gate, _ = O.route(lg, k)
+    m = O.routing_metadata(idx, E)
+    xb = x.view(torch.int16).numpy()
+    Xe = O.dispatch(xb, m["slot"])
+    for t in range(T):
+        for j in range(k):
+            assert np.array_equal(Xe[m["slot"][t, j]], xb[t])
+    # identity experts: Ye := Xe gives (sum_j gate) * x
+    x64 = x.double().numpy()
+    out = O.combine(O.dispatch(x64, m["slot"]), m["slot"], gate)
+    assert np.allclose(out, gate.sum(1, keepdims=True) * x64, rtol=1e-14, atol=1e-14)
+
+
+# ---------------------------------------------------------------- expert FFN / layer
+
+def _torch_swiglu(x, w1, w3, w2):
+    return (torch.nn.functional.silu(x @ w1.T) * (x @ w3.T)) @ w2.T
+
+
+def test_single_expert_top1_is_dense_swiglu():
+    T, d, F = 20, 16, 24
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(1, F, d, generator=g, dtype=torch.float64) * 0.3
+    W3 = torch.randn(1, F, d, generator=g, dtype=torch.float64) * 0.3
+    W2 = torch.randn(1, d, F, generator=g, dtype=torch.float64) * 0.3
+    r = O.moe_layer(x, 1, W1, W3, W2, logits=np.zeros((T, 1), np.float32))
+    ref = _torch_swiglu(x, W1[0], W3[0], W2[0]).numpy()
+    assert np.allclose(r["gate"], 1.0)
+    assert np.allclose(r["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_k_equals_E_is_dense_softmax_mixture():
+    T, d, F, E = 9, 8, 12, 5
+    g = torch.Generator().manual_seed(13)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W3 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W2 = torch.randn(E, d, F, generator=g, dtype=torch.float64) * 0.3
+    lg = torch.randn(T, E, generator=g).numpy()
+    r = O.moe_layer(x, E, W1, W3, W2, logits=lg)
+    p = torch.softmax(torch.from_numpy(lg).double(), dim=1)
+    ref = sum(p[:, e:e + 1] * _torch_swiglu(x, W1[e], W3[e], W2[e]) for e in range(E))
+    assert np.allclose(r["out"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_per_expert_layer_matches_per_token_formula_and_torch_index_add():
+    T, d, F, E, k = 33, 16, 24, 6, 2
+    g = torch.Generator().manual_seed(14)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W3 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W2 = torch.randn(E, d, F, generator=g, dtype=torch.float64) * 0.3
+    lg = torch.randn(T, E, generator=g).numpy()
+    lg[:, 4] -= 20  # expert 4 receives nothing
+    r = O.moe_layer(x, k, W1, W3, W2, logits=lg)
+    assert r["counts"][4] == 0
+    per_tok = O.moe_layer_tokens(x, np.arange(T), r["idx"], r["gate"], W1, W3, W2)
+    assert np.allclose(r["out"], per_tok, rtol=1e-12, atol=1e-12)
+    # the same layer via torch's index_add_ over a hit mask (library routine)
+    idx = torch.from_numpy(r["idx"]).long()
+    gate = torch.from_numpy(r["gate"])
+    ref = torch.zeros(T, d, dtype=torch.float64)
+    for e in range(E):
+        tok, j = torch.nonzero(idx == e, as_tuple=True)
+        if tok.numel():
+            y = _torch_swiglu(x[tok], W1[e], W3[e], W2[e]) * gate[tok, j, None]
+            ref.index_add_(0, tok, y)
+    assert np.allclose(r["out"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_workload_generator_is_deterministic_and_shaped():
+    w = WORKLOADS["tiny_fp32"]
+    a = make_inputs(w)
+    b = make_inputs(w)
+    for key in a:
+        assert torch.equal(a[key], b[key])
+    assert a["x"].shape == (256, 128) and a["Wr"].shape == (8, 128)
+    assert a["W1"].shape == (8, 256, 128) and a["W2"].shape == (8, 128, 256)
+    assert a["x"].dtype == torch.float32
+    assert abs(a["W1"].std().item() - 0.02) < 0.002
+
+
+# ---------------------------------------------------------------- E4M3 / MXFP8
+
+ALL = np.arange(256, dtype=np.uint8)
+
+
+def test_e4m3_decode_matches_torch_float8():
+    ref = torch.from_numpy(ALL.copy()).view(torch.float8_e4m3fn).float().numpy()
+    got = O.e4m3_decode(ALL)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan].astype(np.float64))
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_e4m3_roundtrip_every_code():
+    vals = O.e4m3_decode(ALL).astype(np.float32)
+    ok = ~np.isnan(vals)
+    assert np.array_equal(O.e4m3_encode(vals[ok]), ALL[ok])
+
+
+def test_e4m3_encode_matches_torch_cast_in_range():
+    g = torch.Generator().manual_seed(21)
+    v = torch.cat([torch.randn(1 << 18, generator=g) * s for s in (1e-3, 0.05, 1.0, 30.0, 150.0)])
+    v = v[v.abs() < 464]
+    ref = v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(v.numpy()), ref)
+
+
+def test_e4m3_rounding_and_saturation_closed_forms():
+    f = lambda x: int(O.e4m3_encode(np.array([x], np.float32))[0])
+    assert f(1.0625) == 0x38          # midpoint of 1.0 / 1.125 -> even
+    assert f(1.1875) == 0x3A          # midpoint of 1.125 / 1.25 -> even
+    assert f(2.0 ** -10) == 0x00      # half the smallest subnormal -> 0
+    assert f(3 * 2.0 ** -10) == 0x02  # midpoint of 1 and 2 units -> even
+    for big in (448.0, 460.0, 464.0, 1e6, np.inf):
+        assert f(big) == 0x7E and f(-big) == 0xFE
+    assert f(-0.0) == 0x80 and f(np.nan) & 0x7F == 0x7F
+
+
+@pytest.mark.parametrize("mode", ["f32", "e8m0"])
+def test_mxfp8_roundtrip_bound_and_zero_block(mode):
+    g = torch.Generator().manual_seed(22)
+    v = torch.randn(64, 256, generator=g) * torch.logspace(-3, 3, 64).unsqueeze(1)
+    v[3, 32:64] = 0.0
+    v = v.to(torch.bfloat16).float().numpy()
+    q, s = O.mxfp8_quantize(v, mode)
+    back = O.mxfp8_dequantize_f32(q, s, mode).astype(np.float64)
+    sc = np.repeat(O.mxfp8_scales_to_f32(s, mode).astype(np.float64), 32, axis=1)
+    err = np.abs(back - v)
+    bound = np.maximum(2.0 ** -4 * np.abs(v), 2.0 ** -10 * sc) * (1 + 2.0 ** -20)
+    assert np.all(err <= bound)
+    assert np.all(q[3, 32:64] == 0)
+    zero_scale = s[3, 1]
+    assert (zero_scale == 1.0) if mode == "f32" else (zero_scale == 127)
+    amax = np.abs(v.reshape(64, 8, 32)).max(2)
+    if mode == "e8m0":
+        s32 = O.mxfp8_scales_to_f32(s, mode)
+        nz = amax > 0
+        # the smallest power of two at or above amax/448
+        assert np.all(s32[nz] >= (amax[nz] / np.float32(448)).astype(np.float32))
+        assert np.all(s32[nz] / 2 < (amax[nz] / np.float32(448)).astype(np.float32))
+        assert np.all(np.abs(O.e4m3_decode(q)).max() <= 448)
+    else:
+        assert np.all(np.abs(O.e4m3_decode(q.reshape(64, 8, 32))).max(2)[amax > 0] >= 416)
+
+
+def test_mxfp8_dequantize_bf16_rounds_fp32_product():
+    v = torch.randn(4, 64, generator=torch.Generator().manual_seed(23)).numpy()
+    q, s = O.mxfp8_quantize(v, "f32")
+    b = O.mxfp8_dequantize(q, s, "f32")
+    f = torch.from_numpy(O.mxfp8_dequantize_f32(q, s, "f32"))
+    assert torch.equal(b, f.to(torch.bfloat16))
+
+
+# ---------------------------------------------------------------- backward
+
+def _tiny_problem(seed, T=12, d=6, F=8, E=4, k=2):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.5
+    W3 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.5
+    W2 = torch.randn(E, d, F, generator=g, dtype=torch.float64) * 0.5
+    lg = torch.randn(T, E, generator=g).numpy()
+    lg[:, E - 1] -= 30.0  # one expert with zero rows
+    dOut = torch.randn(T, d, generator=g, dtype=torch.float64)
+    return x, W1, W3, W2, lg, dOut
+
+
+def test_backward_matches_torch_autograd():
+    x, W1, W3, W2, lg, dOut = _tiny_problem(31)
+    k = 2
+    r = O.moe_layer_bwd(x, dOut, k, W1, W3, W2, lg)
+    xs = x.clone().requires_grad_(True)
+    ws = [w.clone().requires_grad_(True) for w in (W1, W3, W2)]
+    idx = torch.from_numpy(r["idx"]).long()
+    gate = torch.from_numpy(r["gate"])
+    out = torch.zeros_like(x)
+    for t in range(x.shape[0]):
+        for j in range(k):
+            e = int(idx[t, j])
+            out[t] = out[t] + gate[t, j] * _torch_swiglu(xs[t:t + 1], ws[0][e], ws[1][e], ws[2][e])[0]
+    out.backward(dOut)
+    assert np.allclose(r["dx"], xs.grad.numpy(), rtol=1e-11, atol=1e-12)
+    for name, w in zip(("dW1", "dW3", "dW2"), ws):
+        assert np.allclose(r[name], w.grad.numpy(), rtol=1e-11, atol=1e-12)
+    assert np.all(r["dW1"][3] == 0) and np.all(r["dW2"][3] == 0)
+
+
+def test_backward_finite_differences():
+    x, W1, W3, W2, lg, dOut = _tiny_problem(32, T=6, d=4, F=5, E=3, k=2)
+    k = 2
+    r = O.moe_layer_bwd(x, dOut, k, W1, W3, W2, lg)
+
+    def loss(xv, w1, w3, w2):
+        o = O.moe_layer(xv, k, w1, w3, w2, logits=lg)["out"]
+        return float((o * dOut.numpy()).sum())
+
+    h = 1e-6
+    for (t, j) in [(0, 0), (3, 2), (5, 3)]:
+        xp, xm = x.clone(), x.clone()
+        xp[t, j] += h
+        xm[t, j] -= h
+        fd = (loss(xp, W1, W3, W2) - loss(xm, W1, W3, W2)) / (2 * h)
+        assert math.isclose(fd, r["dx"][t, j], rel_tol=1e-6, abs_tol=1e-8)
+    for (e, a, b) in [(0, 1, 2), (1, 4, 0)]:
+        Wp, Wm = W2.clone(), W2.clone()
+        Wp[e, b, a] += h
+        Wm[e, b, a] -= h
+        fd = (loss(x, W1, W3, Wp) - loss(x, W1, W3, Wm)) / (2 * h)
+        assert math.isclose(fd, r["dW2"][e, b, a], rel_tol=1e-6, abs_tol=1e-8)
+        Wp, Wm = W1.clone(), W1.clone()
+        Wp[e, a, b] += h
+        Wm[e, a, b] -= h
+        fd = (loss(x, Wp, W3, W2) - loss(x, Wm, W3, W2)) / (2 * h)
+        assert math.isclose(fd, r["dW1"][e, a, b], rel_tol=1e-6, abs_tol=1e-8)
