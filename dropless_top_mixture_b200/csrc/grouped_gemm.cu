@@ -1,0 +1,617 @@
+// Grouped SwiGLU expert FFN on 5th-generation tensor cores (sm_100a).
+//
+// "Transformers 中的 OLMoE" (blog.gitcode.com) §3: every expert is a SwiGLU
+// FFN, Ye = W2 (silu(W1 x) * W3 x), over the rows routed to it. "olmoforge"
+// README, capability table (grouped GEMM): the many small per-expert matmuls
+// run as one kernel. Here one persistent kernel walks a device-side tile
+// table built from the routing offsets, so the host never learns the
+// per-expert row counts.
+//
+// Two instantiations:
+//   gate_up  H[r]  = silu(Xe[r] W1_eᵀ) * (Xe[r] W3_eᵀ)   B tile = [W1 rows; W3 rows]
+//   down     Ye[r] = H[r] W2_eᵀ
+//
+// Tile = 128 rows (one expert's rows; the last tile of an expert overlaps the
+// next expert's rows, which are computed and masked at the store) x MMA_N
+// columns of B. One 128xMMA_Nx16 MMA per 32 bytes of K; K is staged 128
+// bytes at a time by TMA with the 128-byte swizzle the MMA descriptors read.
+//
+// Warp roles (192 threads, one CTA per SM):
+//   warp 0, lane 0   TMA producer over a STAGES-deep shared-memory ring
+//   warp 1           allocates TMEM; lane 0 issues tcgen05.mma
+//   warps 2..5       epilogue: tcgen05.ld from TMEM (warp w reads lanes
+//                    32*(w%4)..), SwiGLU / conversion, row-masked stores
+// The accumulator is double-buffered in TMEM (2 x MMA_N columns), so the
+// epilogue of tile i overlaps the main loop of tile i+1.
+//
+// Every wait is bounded: after WAIT_LIMIT_NS the waiting thread sets
+// MOE_DEVERR_TIMEOUT and an abort flag, all roles leave their loops, the MMA
+// issuer drains its outstanding MMAs, the producer waits (again bounded) for
+// its copies in flight, and TMEM is released before the CTA exits.
+#include <cudaTypedefs.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // 0.1 s
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity. Returns false if the wait
+// timed out (status bit + abort flag set here) or another role aborted.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* status, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                set_status(status, MOE_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+template <bool TF32>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accum) {
+    if constexpr (TF32) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+            : "memory");
+    }
+}
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets row
+// (lane base + i), columns taddr.col .. +31.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: fp32 accumulator, A/B format (bf16 = 1, tf32 = 2),
+// both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt, int M, int N) {
+    return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ config
+
+template <typename TIn, bool SWIGLU, int MMA_N_>
+struct Cfg {
+    static constexpr bool TF32 = std::is_same<TIn, float>::value;
+    static constexpr int ES = (int)sizeof(TIn);
+    static constexpr int BK = 128 / ES;           // elements per 128-byte K slab
+    static constexpr int UMMA_K = 32 / ES;        // elements per MMA (32 bytes)
+    static constexpr int KSTEPS = BK / UMMA_K;    // 4
+    static constexpr int MMA_N = MMA_N_;          // B rows per tile
+    static constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = MMA_N * 128;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = 2 * MMA_N;   // two accumulator buffers
+    static constexpr int TMEM_ALLOC = TMEM_COLS <= 256 ? 256 : 512;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    static constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + META_BYTES;
+    static constexpr uint32_t IDESC = make_idesc(TF32 ? 2u : 1u, BM, MMA_N);
+    static_assert(OUT_N % 32 == 0, "epilogue works in 32-column chunks");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct Tile {
+    int e, row0, row_end, n0;
+};
+
+// Tile t -> (expert, rows, columns). Tiles are ordered expert by expert;
+// inside an expert, n-block major and m-tile minor, so CTAs running at the
+// same time share B (weight) tiles and A row blocks through L2.
+__device__ __forceinline__ Tile decode_tile(int t, int NB, int E, int out_n, const int* s_toff,
+                                            const int* s_off) {
+    const int q = t / NB;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_toff[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    Tile tl;
+    tl.e = lo;
+    const int Me = s_toff[lo + 1] - s_toff[lo];
+    const int l = t - s_toff[lo] * NB;
+    const int nb = l / Me, m = l - nb * Me;
+    tl.row0 = s_off[lo] + m * BM;
+    tl.row_end = s_off[lo + 1];
+    tl.n0 = nb * out_n;
+    return tl;
+}
+
+template <typename TOut>
+struct Store32;
+
+template <>
+struct Store32<__nv_bfloat16> {
+    __device__ static void run(__nv_bfloat16* dst, const float* v) {
+        uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[i] = pack8(v + 8 * i);
+    }
+};
+
+template <>
+struct Store32<float> {
+    __device__ static void run(float* dst, const float* v) {
+        float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+};
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+template <typename TIn, bool SWIGLU, int MMA_N>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const int32_t* __restrict__ offsets, int E, int R, int K, int N,
+                        TIn* __restrict__ out, int64_t ldo, int* status) {
+    using C = Cfg<TIn, SWIGLU, MMA_N>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* meta = smem + STAGES * C::STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + C::NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + C::NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // --- device-side tile table from the routing offsets (validated) -------
+    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int m = 0;
+            if (e < E) {
+                const int cnt = s_off[e + 1] - s_off[e];
+                if (cnt < 0) bad = true;
+                else m = (cnt + BM - 1) / BM;
+            }
+            int tot;
+            const int ex = warp_exclusive_scan(m, &tot);
+            if (e < E) s_toff[e] = carry + ex;
+            carry += tot;
+        }
+        bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
+        if (lane == 0) {
+            s_toff[E] = carry;
+            *s_bad = bad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    if (*s_bad) {
+        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+        return;
+    }
+    const int NB = N / C::OUT_N;
+    const int total = s_toff[E] * NB;
+    if ((int)blockIdx.x >= total) return;
+    const int KB = K / C::BK;
+
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(tfull + b), 1);
+            mbar_init(smem_u32(tempty + b), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmA);
+        prefetch_map(&tmB0);
+        if (SWIGLU) prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s_tmem), C::TMEM_ALLOC);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(full + stage);
+                const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+                const uint32_t sb = sa + C::A_BYTES;
+                mbar_expect_tx(fb, C::STAGE_BYTES);
+                tma_load_2d(sa, &tmA, fb, kb * C::BK, tl.row0);
+                if (SWIGLU) {
+                    tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
+                    tma_load_3d(sb + C::B_BYTES / 2, &tmB1, fb, kb * C::BK, tl.n0, tl.e);
+                } else {
+                    tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
+                }
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            // wait (bounded) for the copies this thread put in flight
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued_mask >> s) & 1u) {
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                              DRAIN_LIMIT_NS);
+                }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int i = 0;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+                const uint64_t ad = sw128_desc(sa);
+                const uint64_t bd = sw128_desc(sa + C::A_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks)
+                    tc_mma<C::TF32>(dt, ad + 2 * ks, bd + 2 * ks, C::IDESC, (kb | ks) != 0);
+                tc_commit(smem_u32(empty + stage));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit(smem_u32(tfull + buf));
+        }
+        if (!ok) {
+            // make sure every MMA this thread issued has finished with TMEM
+            tc_commit(smem_u32(drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int r_in_tile = q * 32 + lane;
+        int i = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+            const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
+            const int grow = tl.row0 + r_in_tile;
+            const bool valid = grow < tl.row_end;
+            TIn* orow = out + (size_t)(valid ? grow : 0) * ldo + tl.n0;
+#pragma unroll 1
+            for (int c = 0; c < C::OUT_N / 32; ++c) {
+                uint32_t a[32];
+                float v[32];
+                tmem_ld32(ta + c * 32, a);
+                if constexpr (SWIGLU) {
+                    uint32_t b[32];
+                    tmem_ld32(ta + C::OUT_N + c * 32, b);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v[j] = silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j]));
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                }
+                if (valid) Store32<TIn>::run(orow + c * 32, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, C::TMEM_ALLOC);
+    }
+}
+
+// ------------------------------------------------------------------ host
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major [rows, cols] matrix; box = 128 bytes x box_rows.
+static bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
+                        uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)es};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over E matrices [rows, cols] spaced `estride` elements apart.
+static bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
+                        uint64_t cols, uint64_t rows, uint64_t E, uint64_t estride,
+                        uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cols, rows, E};
+    cuuint64_t strides[2] = {cols * (uint64_t)es, estride * (uint64_t)es};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / es), box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TIn, bool SWIGLU, int MMA_N>
+static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                  const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, void* out,
+                  int64_t ldo, cudaStream_t st) {
+    using C = Cfg<TIn, SWIGLU, MMA_N>;
+    auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t max_tiles = (R / BM + E) * (N / C::OUT_N);
+    const int64_t sms = num_sms();
+    const int grid = (int)(max_tiles < sms ? max_tiles : sms);
+    if (grid <= 0) return MOE_OK;
+    kern<<<grid, THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K, (int)N,
+                                              static_cast<TIn*>(out), ldo, status_ptr());
+    return launch_status();
+}
+
+static int check_common(const void* A, const void* B, const int32_t* offsets, int64_t E,
+                        int64_t R, int64_t d, int64_t F, int dtype) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
+    if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (R > INT32_MAX - 2 * BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+    if (!offsets || !A || !B || !aligned16(A) || !aligned16(B)) return MOE_ERR_INVALID;
+    return MOE_OK;
+}
+
+}  // namespace gg
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
+                                   int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
+                                   int64_t R, int64_t d, int64_t F, int dtype, void* H,
+                                   void* stream) {
+    int rc = gg::check_common(Xe, W1, offsets, E, R, d, F, dtype);
+    if (rc != MOE_OK) return rc;
+    if (!W3 || !H || !aligned16(W3) || !aligned16(H)) return MOE_ERR_INVALID;
+    if (w13_expert_stride < F * d && E > 1) return MOE_ERR_INVALID;
+    if (w13_expert_stride % 8 != 0) return MOE_ERR_INVALID;
+    if (R == 0) return MOE_OK;
+    const int es = dtype == MOE_F32 ? 4 : 2;
+    const CUtensorMapDataType dt =
+        dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap a, b0, b1;
+    if (!gg::make_map_2d(&a, Xe, dt, es, d, R, gg::BM) ||
+        !gg::make_map_3d(&b0, W1, dt, es, d, F, E, w13_expert_stride, 128) ||
+        !gg::make_map_3d(&b1, W3, dt, es, d, F, E, w13_expert_stride, 128))
+        return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (dtype == MOE_BF16)
+        return gg::launch<__nv_bfloat16, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st);
+    return gg::launch<float, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st);
+}
+
+extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
+                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                int64_t F, int dtype, void* Ye, void* stream) {
+    int rc = gg::check_common(H, W2, offsets, E, R, d, F, dtype);
+    if (rc != MOE_OK) return rc;
+    if (!Ye || !aligned16(Ye)) return MOE_ERR_INVALID;
+    if (w2_expert_stride < F * d && E > 1) return MOE_ERR_INVALID;
+    if (w2_expert_stride % 8 != 0) return MOE_ERR_INVALID;
+    if (R == 0) return MOE_OK;
+    const int es = dtype == MOE_F32 ? 4 : 2;
+    const CUtensorMapDataType dt =
+        dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int mma_n = (d % 256 == 0) ? 256 : 128;
+    CUtensorMap a, b0;
+    if (!gg::make_map_2d(&a, H, dt, es, F, R, gg::BM) ||
+        !gg::make_map_3d(&b0, W2, dt, es, F, d, E, w2_expert_stride, mma_n))
+        return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (dtype == MOE_BF16) {
+        if (mma_n == 256)
+            return gg::launch<__nv_bfloat16, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+        return gg::launch<__nv_bfloat16, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+    }
+    if (mma_n == 256) return gg::launch<float, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+    return gg::launch<float, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+}
+
+extern "C" int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, const void* W2,
+                                  int64_t w13_expert_stride, int64_t w2_expert_stride,
+                                  const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                  int64_t F, int dtype, void* H, void* Ye, void* stream) {
+    int rc = moe_grouped_gate_up(Xe, W1, W3, w13_expert_stride, offsets, E, R, d, F, dtype, H,
+                                 stream);
+    if (rc != MOE_OK) return rc;
+    return moe_grouped_down(H, W2, w2_expert_stride, offsets, E, R, d, F, dtype, Ye, stream);
+}

@@ -1,0 +1,113 @@
+// The whole expert layer and the library-wide entry points.
+//
+// moe_layer_fwd enqueues route -> dispatch -> grouped gate/up -> grouped
+// down -> combine on one stream ("Transformers 中的 OLMoE" §2-§3). Every size
+// the kernels need is known on the host from (T, k, d, F, E): dropless
+// routing means exactly R = T*k expert rows, so per-expert counts never come
+// back to the host and nothing synchronises.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ int g_status_word;
+
+int* status_ptr() {
+    static int* cached[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cached[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) cached[dev] = static_cast<int*>(p);
+    }
+    return cached[dev];
+}
+
+namespace layer {
+
+inline size_t a256(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct Carve {
+    void* Xe;
+    void* H;
+    void* Ye;
+    void* route_ws;
+    size_t route_bytes;
+    size_t total;
+};
+
+inline Carve carve(void* base, int64_t T, int64_t d, int64_t E, int64_t F, int k, int dtype,
+                   int logits_given) {
+    const size_t es = dtype == MOE_F32 ? 4 : 2;
+    const size_t R = (size_t)T * (size_t)k;
+    char* p = static_cast<char*>(base);
+    Carve c;
+    size_t off = 0;
+    c.Xe = p + off;
+    off += a256(R * d * es);
+    c.H = p + off;
+    off += a256(R * F * es);
+    c.Ye = p + off;
+    off += a256(R * d * es);
+    c.route_ws = p + off;
+    c.route_bytes = moe_route_workspace_size(T, E, logits_given ? 0 : 1);
+    off += a256(c.route_bytes);
+    c.total = off;
+    return c;
+}
+
+}  // namespace layer
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" const char* moe_version(void) { return "dropless_top_mixture_b200 0.1 sm_100a"; }
+
+extern "C" int moe_get_status(int32_t* host_status, int clear, void* stream) {
+    if (!host_status) return MOE_ERR_INVALID;
+    int* p = status_ptr();
+    if (!p) return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(host_status, p, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (clear && cudaMemsetAsync(p, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+extern "C" size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
+                                           int dtype, int logits_given) {
+    if (T < 0 || d <= 0 || E <= 0 || F <= 0 || k <= 0) return 0;
+    return layer::carve(nullptr, T, d, E, F, k, dtype, logits_given).total;
+}
+
+extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
+    if (!a) return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->dtype != MOE_BF16 && a->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return MOE_ERR_INVALID;
+    const int logits_given = a->logits != nullptr;
+    layer::Carve c = layer::carve(a->workspace, a->T, a->d, a->E, a->F, a->k, a->dtype, logits_given);
+    if (a->workspace_bytes < c.total) return MOE_ERR_INVALID;
+    if (a->T == 0) {
+        return moe_route(a->logits, a->x, a->Wr, a->dtype, 0, a->d, a->E, a->k, a->renorm,
+                         nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
+                         c.route_ws, c.route_bytes, stream);
+    }
+    const int64_t R = a->T * a->k;
+    int rc = moe_route(a->logits, a->x, a->Wr, a->dtype, a->T, a->d, a->E, a->k, a->renorm,
+                       nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
+                       c.route_ws, c.route_bytes, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, c.Xe, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_grouped_swiglu(c.Xe, a->W1, a->W3, a->W2, a->w13_expert_stride, a->w2_expert_stride,
+                            a->offsets, a->E, R, a->d, a->F, a->dtype, c.H, c.Ye, stream);
+    if (rc != MOE_OK) return rc;
+    return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
+}

@@ -1,0 +1,471 @@
+// Route step of the dropless top-k MoE layer on sm_100a.
+//
+//   a0  router logits  logits[t,e] = fmaf-chain over j of x[t,j]*Wr[e,j]
+//   a1  fp32 softmax + top-k (ties to the lower expert index)
+//   a2  routing metadata: counts, offsets, slots, tile offsets
+//
+// "Transformers 中的 OLMoE" (blog.gitcode.com) §2: softmax over the expert
+// logits in fp32, then top-k, optional renormalisation; bias-free (E, d)
+// router weight. "olmoforge" README, capability table: the routing table is
+// built and kept on the device, so nothing is copied back to the host.
+//
+// Routing metadata is a stable counting sort of the token-major (t, j) list
+// by expert, built in three launches:
+//   1. topk_chunk: one warp per chunk of CHUNK consecutive tokens. It selects
+//      the k experts of each token in order and keeps, per expert, a running
+//      count inside the chunk; the count before a token's hit is that
+//      token's rank among the chunk's rows of the expert (stable by token).
+//      Per-chunk counts go to ws_count[e][c].
+//   2. scan: one block per expert scans ws_count[e][:] over chunks (exclusive,
+//      in place) and writes counts[e]; the last block to finish (ticket
+//      counter) scans counts into offsets and tile_offsets.
+//   3. finalize: slot = offsets[e] + chunk_base[e][c] + rank.
+// Integer work only after the top-k, so the result is bit-exact and
+// independent of scheduling.
+#include "common.cuh"
+
+namespace moe {
+namespace route {
+
+constexpr int CHUNK = 8;           // tokens per warp in topk_chunk
+constexpr int LOGIT_TT = 64;       // tokens per router-logits tile
+constexpr int LOGIT_TE = 64;       // experts per router-logits tile
+constexpr int LOGIT_TK = 32;       // contraction chunk staged in shared memory
+constexpr int LOGIT_LD = 68;       // padded row of the staged chunk (floats)
+
+// ------------------------------------------------------------------ a0
+
+template <typename TX>
+struct Stage8;  // loads 8 consecutive elements as fp32
+
+template <>
+struct Stage8<__nv_bfloat16> {
+    __device__ static void load(const __nv_bfloat16* p, bool ok, float* f) {
+        if (ok) {
+            uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+            unpack8(u, f);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        }
+    }
+};
+
+template <>
+struct Stage8<float> {
+    __device__ static void load(const float* p, bool ok, float* f) {
+        if (ok) {
+            float4 a = __ldg(reinterpret_cast<const float4*>(p));
+            float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+            f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        }
+    }
+};
+
+// One CTA computes a 64-token x 64-expert tile. Thread (ty, tx) owns tokens
+// 4ty..4ty+3 and experts 4tx..4tx+3, each with its own fp32 accumulator
+// updated in ascending j, so every logit is the same sequential fmaf chain
+// the definition states. Rows of x and Wr are staged 32 columns at a time,
+// transposed into k-major shared memory; the next chunk is prefetched into
+// registers while the current one is consumed.
+template <typename TX>
+__global__ void __launch_bounds__(256) router_logits_kernel(const TX* __restrict__ x,
+                                                            const TX* __restrict__ Wr, int T,
+                                                            int d, int E,
+                                                            float* __restrict__ logits) {
+    __shared__ __align__(16) float xs[LOGIT_TK][LOGIT_LD];
+    __shared__ __align__(16) float ws[LOGIT_TK][LOGIT_LD];
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.x * LOGIT_TT;
+    const int e0 = blockIdx.y * LOGIT_TE;
+    // staging role: row = tid / 4 (token or expert), columns (tid % 4) * 8 .. +7
+    const int srow = tid >> 2;
+    const int scol = (tid & 3) * 8;
+    const bool xok = (t0 + srow) < T;
+    const bool wok = (e0 + srow) < E;
+    const TX* xp = x + (size_t)(t0 + srow) * d + scol;
+    const TX* wp = Wr + (size_t)(e0 + srow) * d + scol;
+    // compute role
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    float fx[8], fw[8];
+    Stage8<TX>::load(xp, xok, fx);
+    Stage8<TX>::load(wp, wok, fw);
+    for (int k0 = 0; k0 < d; k0 += LOGIT_TK) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            xs[scol + i][srow] = fx[i];
+            ws[scol + i][srow] = fw[i];
+        }
+        __syncthreads();
+        if (k0 + LOGIT_TK < d) {
+            Stage8<TX>::load(xp + k0 + LOGIT_TK, xok, fx);
+            Stage8<TX>::load(wp + k0 + LOGIT_TK, wok, fw);
+        }
+#pragma unroll 8
+        for (int kk = 0; kk < LOGIT_TK; ++kk) {
+            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + ty * 4 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + tx * 4 + j;
+            if (e < E) logits[(size_t)t * E + e] = acc[i][j];
+        }
+    }
+}
+
+// ------------------------------------------------------------------ a1
+
+// Total order used by the top-k: larger logit first, then lower index.
+__device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
+    if (ai < 0) return false;
+    if (bi < 0) return true;
+    return av > bv || (av == bv && ai < bi);
+}
+
+// EPL = experts per lane (ceil(E/32)); expert e lives in lane e%32, slot e/32.
+template <int EPL>
+__global__ void __launch_bounds__(128) topk_chunk_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int renorm, int nchunks,
+    int32_t* __restrict__ idx, float* __restrict__ gate, int32_t* __restrict__ rank,
+    int32_t* __restrict__ ws_count) {
+    const int lane = threadIdx.x & 31;
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (c >= nchunks) return;
+    int cnt[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) cnt[q] = 0;
+
+    for (int i = 0; i < CHUNK; ++i) {
+        const int t = c * CHUNK + i;
+        if (t >= T) break;
+        const float* row = logits + (size_t)t * E;
+        float v[EPL];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane + 32 * q;
+            float a = (e < E) ? __ldg(row + e) : -INFINITY;
+            if (isnan(a)) a = -INFINITY;
+            v[q] = a;
+            mx = fmaxf(mx, a);
+        }
+        mx = warp_max(mx);
+        float s = 0.f;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const int e = lane + 32 * q;
+            if (e < E) s += expf(v[q] - mx);
+        }
+        s = warp_sum(s);
+
+        uint32_t taken = 0;
+        int my_e = 0, my_r = 0;
+        float my_g = 0.f;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int be = -1;
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = lane + 32 * q;
+                if (e < E && !((taken >> q) & 1u) && beats(v[q], e, bv, be)) {
+                    bv = v[q];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (beats(ov, oe, bv, be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            // be is the same in every lane; its owner marks it and hands out
+            // the in-chunk rank (count before this hit).
+            int r = 0;
+            if ((be & 31) == lane) {
+                const int qq = be >> 5;
+#pragma unroll
+                for (int q = 0; q < EPL; ++q)
+                    if (q == qq) {
+                        r = cnt[q];
+                        cnt[q] = r + 1;
+                        taken |= 1u << q;
+                    }
+            }
+            r = __shfl_sync(0xffffffffu, r, be & 31);
+            const float g = expf(bv - mx) / s;
+            if (lane == j) {
+                my_e = be;
+                my_g = g;
+                my_r = r;
+            }
+        }
+        if (renorm) {
+            float gs = 0.f;
+            for (int j = 0; j < k; ++j) gs += __shfl_sync(0xffffffffu, my_g, j);
+            my_g = my_g / gs;
+        }
+        if (lane < k) {
+            idx[(size_t)t * k + lane] = my_e;
+            gate[(size_t)t * k + lane] = my_g;
+            rank[(size_t)t * k + lane] = my_r;
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+        const int e = lane + 32 * q;
+        if (e < E) ws_count[(size_t)e * nchunks + c] = cnt[q];
+    }
+}
+
+// ------------------------------------------------------------------ a2
+
+constexpr int SCAN_THREADS = 256;
+constexpr int SCAN_ITEMS = 4;
+
+// Block-wide exclusive scan of one int per thread (SCAN_THREADS threads).
+__device__ int block_exclusive_scan(int v, int* total, int* sh /*[32]*/) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int wt;
+    int ex = warp_exclusive_scan(v, &wt);
+    if (lane == 0) sh[w] = wt;
+    __syncthreads();
+    if (w == 0) {
+        int x = lane < SCAN_THREADS / 32 ? sh[lane] : 0;
+        int tt;
+        int e2 = warp_exclusive_scan(x, &tt);
+        if (lane < SCAN_THREADS / 32) sh[lane] = e2;
+        if (lane == 0) sh[31] = tt;
+    }
+    __syncthreads();
+    const int r = ex + sh[w];
+    *total = sh[31];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int E, int nchunks,
+                                                            int32_t* __restrict__ ws_count,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ tile_offsets,
+                                                            int32_t* __restrict__ ticket) {
+    __shared__ int sh[32];
+    __shared__ int is_last;
+    const int e = blockIdx.x;
+    int32_t* row = ws_count + (size_t)e * nchunks;
+    int carry = 0;
+    for (int base = 0; base < nchunks; base += SCAN_THREADS * SCAN_ITEMS) {
+        int v[SCAN_ITEMS];
+        int local = 0;
+        const int b0 = base + threadIdx.x * SCAN_ITEMS;
+#pragma unroll
+        for (int i = 0; i < SCAN_ITEMS; ++i) {
+            v[i] = (b0 + i < nchunks) ? row[b0 + i] : 0;
+            local += v[i];
+        }
+        int tot;
+        int ex = block_exclusive_scan(local, &tot, sh) + carry;
+#pragma unroll
+        for (int i = 0; i < SCAN_ITEMS; ++i) {
+            if (b0 + i < nchunks) row[b0 + i] = ex;
+            ex += v[i];
+        }
+        carry += tot;
+    }
+    if (threadIdx.x == 0) {
+        counts[e] = carry;
+        __threadfence();
+        const int prev = atomicAdd(ticket, 1);
+        is_last = (prev == (int)gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    // last block: offsets and tile offsets over E <= 512 experts, 2 per thread
+    int c0 = 0, c1 = 0;
+    const int i0 = threadIdx.x * 2;
+    if (i0 < E) c0 = __ldcg(counts + i0);
+    if (i0 + 1 < E) c1 = __ldcg(counts + i0 + 1);
+    int tot;
+    int ex = block_exclusive_scan(c0 + c1, &tot, sh);
+    if (i0 < E) offsets[i0] = ex;
+    if (i0 + 1 < E) offsets[i0 + 1] = ex + c0;
+    if (threadIdx.x == 0) offsets[E] = tot;
+    if (tile_offsets) {
+        const int m0 = (c0 + MOE_TILE_M - 1) / MOE_TILE_M, m1 = (c1 + MOE_TILE_M - 1) / MOE_TILE_M;
+        int mt;
+        int mex = block_exclusive_scan(m0 + m1, &mt, sh);
+        if (i0 < E) tile_offsets[i0] = mex;
+        if (i0 + 1 < E) tile_offsets[i0 + 1] = mex + m0;
+        if (threadIdx.x == 0) tile_offsets[E] = mt;
+    }
+    if (threadIdx.x == 0) *ticket = 0;
+}
+
+__global__ void finalize_kernel(int T, int k, int E, int nchunks, const int32_t* __restrict__ idx,
+                                const int32_t* __restrict__ offsets,
+                                const int32_t* __restrict__ ws_count, int32_t* __restrict__ slot,
+                                int* status) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n = (int64_t)T * k;
+    if (i >= n) return;
+    const int t = (int)(i / k);
+    const int e = idx[i];
+    if (e < 0 || e >= E) {
+        set_status(status, MOE_DEVERR_BAD_INDEX);
+        return;
+    }
+    const int c = t / CHUNK;
+    slot[i] = offsets[e] + ws_count[(size_t)e * nchunks + c] + slot[i];
+}
+
+// ------------------------------------------------------------------ host
+
+inline int64_t nchunks_of(int64_t T) { return (T + CHUNK - 1) / CHUNK; }
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct RouteWs {
+    int32_t* count;
+    int32_t* ticket;
+    float* logits;
+};
+
+inline size_t workspace_bytes(int64_t T, int64_t E, bool need_logits) {
+    size_t b = align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
+    b += 256;  // ticket
+    if (need_logits) b += align256(sizeof(float) * (size_t)T * (size_t)E);
+    return b;
+}
+
+inline RouteWs carve(void* ws, int64_t T, int64_t E, bool need_logits) {
+    char* p = static_cast<char*>(ws);
+    RouteWs r;
+    r.count = reinterpret_cast<int32_t*>(p);
+    p += align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
+    r.ticket = reinterpret_cast<int32_t*>(p);
+    p += 256;
+    r.logits = need_logits ? reinterpret_cast<float*>(p) : nullptr;
+    return r;
+}
+
+template <int EPL>
+static void launch_topk(const float* logits, int T, int E, int k, int renorm, int nch,
+                        int32_t* idx, float* gate, int32_t* rank, int32_t* wsc,
+                        cudaStream_t st) {
+    const int warps_per_block = 4;
+    const int blocks = (nch + warps_per_block - 1) / warps_per_block;
+    topk_chunk_kernel<EPL><<<blocks, 32 * warps_per_block, 0, st>>>(logits, T, E, k, renorm, nch,
+                                                                    idx, gate, rank, wsc);
+}
+
+}  // namespace route
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_route_workspace_size(int64_t T, int64_t E, int need_logits_buffer) {
+    if (T < 0 || E <= 0) return 0;
+    return route::workspace_bytes(T, E, need_logits_buffer != 0);
+}
+
+extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int dtype, int64_t T,
+                         int64_t d, int64_t E, int k, int renorm, float* logits_out, int32_t* idx,
+                         float* gate, int32_t* counts, int32_t* offsets, int32_t* slot,
+                         int32_t* tile_offsets, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || k < 1 || k > MOE_MAX_TOPK || k > E)
+        return MOE_ERR_INVALID;
+    if (T * k > INT32_MAX || T > INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    if (!counts || !offsets) return MOE_ERR_INVALID;
+    if (T == 0) {
+        // empty batch (an empty logits tensor may well be a null pointer): all
+        // counts, offsets and tile offsets are zero
+        cudaStream_t st0 = as_stream(stream);
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st0) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (tile_offsets &&
+            cudaMemsetAsync(tile_offsets, 0, sizeof(int32_t) * (E + 1), st0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    const bool from_x = (logits == nullptr);
+    if (from_x) {
+        if (!x || !Wr || d <= 0 || (d % route::LOGIT_TK) != 0) return MOE_ERR_INVALID;
+        if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+        if (!aligned16(x) || !aligned16(Wr)) return MOE_ERR_INVALID;
+    }
+    if (T > 0 && (!idx || !gate || !slot)) return MOE_ERR_INVALID;
+    const bool need_logits = from_x && logits_out == nullptr;
+    if (!workspace || workspace_bytes < route::workspace_bytes(T, E, need_logits))
+        return MOE_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    route::RouteWs ws = route::carve(workspace, T, E, need_logits);
+
+    const float* lg = logits;
+    if (from_x) {
+        float* dst = logits_out ? logits_out : ws.logits;
+        dim3 grid((unsigned)((T + route::LOGIT_TT - 1) / route::LOGIT_TT),
+                  (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE));
+        if (dtype == MOE_BF16)
+            route::router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
+                (int)T, (int)d, (int)E, dst);
+        else
+            route::router_logits_kernel<float><<<grid, 256, 0, st>>>(
+                static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d,
+                (int)E, dst);
+        lg = dst;
+    }
+    const int nch = (int)route::nchunks_of(T);
+    // the in-chunk ranks are parked in `slot` and completed by finalize_kernel
+    switch ((E + 31) / 32) {
+#define MOE_TOPK_CASE(n)                                                                       \
+    case n:                                                                                    \
+        route::launch_topk<n>(lg, (int)T, (int)E, k, renorm, nch, idx, gate, slot, ws.count, \
+                              st);                                                             \
+        break;
+        MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4)
+        MOE_TOPK_CASE(5) MOE_TOPK_CASE(6) MOE_TOPK_CASE(7) MOE_TOPK_CASE(8)
+        MOE_TOPK_CASE(9) MOE_TOPK_CASE(10) MOE_TOPK_CASE(11) MOE_TOPK_CASE(12)
+        MOE_TOPK_CASE(13) MOE_TOPK_CASE(14) MOE_TOPK_CASE(15) MOE_TOPK_CASE(16)
+#undef MOE_TOPK_CASE
+        default:
+            return MOE_ERR_UNSUPPORTED;
+    }
+    if (cudaMemsetAsync(ws.ticket, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    route::scan_kernel<<<(unsigned)E, route::SCAN_THREADS, 0, st>>>(
+        (int)E, nch, ws.count, counts, offsets, tile_offsets, ws.ticket);
+    const int64_t n = T * k;
+    route::finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        (int)T, k, (int)E, nch, idx, offsets, ws.count, slot, status_ptr());
+    return launch_status();
+}

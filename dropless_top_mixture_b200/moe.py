@@ -1,0 +1,321 @@
+"""Python binding of the C ABI in include/moe.h.
+
+Argument marshalling only: tensors become ``data_ptr()`` values, the stream
+is torch's current stream on the tensors' device, and a non-zero return code
+raises :class:`MoeError`. Every step of the layer runs in the sm_100a
+library ``lib/libdtm_b200.so``; if it is missing, importing this module
+fails — there is no other implementation behind these names.
+
+Output tensors may be passed in; when omitted they are allocated with
+``torch.empty`` on the input's device (allocation only, no compute).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libdtm_b200.so")
+
+MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, -1, -2, -3
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+MOE_SCALE_F32, MOE_SCALE_E8M0 = 0, 1
+MOE_DEVERR_TIMEOUT, MOE_DEVERR_BAD_OFFSETS, MOE_DEVERR_BAD_INDEX = 1, 2, 4
+TILE_M = 128
+
+_ERRNAMES = {MOE_ERR_INVALID: "MOE_ERR_INVALID", MOE_ERR_UNSUPPORTED: "MOE_ERR_UNSUPPORTED",
+             MOE_ERR_CUDA: "MOE_ERR_CUDA"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {_ERRNAMES.get(code, code)}")
+        self.code = code
+
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m dropless_top_mixture_b200.build`")
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int
+_sz = ctypes.c_size_t
+
+
+class LayerArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i64), ("d", _i64), ("E", _i64), ("F", _i64),
+        ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("renorm", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
+        ("x", _p), ("logits", _p), ("Wr", _p), ("W1", _p), ("W3", _p), ("W2", _p),
+        ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
+        ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
+        ("workspace", _p), ("workspace_bytes", _sz),
+    ]
+
+
+_SIGS = {
+    "moe_route_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "moe_route": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _p, _p, _p, _p, _p,
+                         _p, _p, _sz, _p]),
+    "moe_dispatch": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
+    "moe_grouped_gate_up": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
+    "moe_grouped_down": (_i32, [_p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
+    "moe_grouped_swiglu": (_i32, [_p, _p, _p, _p, _i64, _i64, _p, _i64, _i64, _i64, _i64, _i32,
+                                  _p, _p, _p]),
+    "moe_combine": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
+    "mxfp8_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _p, _p, _p]),
+    "mxfp8_dequantize": (_i32, [_p, _p, _i32, _i64, _i64, _p, _p]),
+    "moe_layer_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32, _i32]),
+    "moe_layer_fwd": (_i32, [ctypes.POINTER(LayerArgs), _p]),
+    "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
+    "moe_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+# ----------------------------------------------------------------- helpers
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(t: torch.Tensor):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return MOE_BF16
+    if dt == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _alloc_ws(nbytes: int, device) -> torch.Tensor:
+    # 256-byte aligned: torch's caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------- API
+
+@dataclass
+class Route:
+    idx: torch.Tensor
+    gate: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    slot: torch.Tensor
+    tile_offsets: torch.Tensor
+    logits: Optional[torch.Tensor] = None
+
+
+def moe_route(k: int, *, logits: Optional[torch.Tensor] = None, x: Optional[torch.Tensor] = None,
+              Wr: Optional[torch.Tensor] = None, renorm: bool = False, E: Optional[int] = None,
+              keep_logits: bool = False, out: Optional[Route] = None,
+              workspace: Optional[torch.Tensor] = None) -> Route:
+    if logits is not None:
+        _need(logits, "logits")
+        T, E = logits.shape
+        dev = logits.device
+        dtype, d = MOE_F32, 0
+    else:
+        _need(x, "x"); _need(Wr, "Wr")
+        T, d = x.shape
+        E = Wr.shape[0]
+        dev = x.device
+        dtype = _dtype_code(x.dtype)
+    i32 = dict(dtype=torch.int32, device=dev)
+    if out is None:
+        out = Route(idx=torch.empty((T, k), **i32), gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                    counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                    slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
+        if logits is None and keep_logits:
+            out.logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    need_buf = logits is None and out.logits is None
+    ws_bytes = lib.moe_route_workspace_size(T, E, int(need_buf))
+    if workspace is None:
+        workspace = _alloc_ws(ws_bytes, dev)
+    rc = lib.moe_route(_ptr(logits), _ptr(x), _ptr(Wr), dtype, T, d, E, k, int(renorm),
+                       _ptr(out.logits), _ptr(out.idx), _ptr(out.gate), _ptr(out.counts),
+                       _ptr(out.offsets), _ptr(out.slot), _ptr(out.tile_offsets),
+                       _ptr(workspace), workspace.numel(), _stream(workspace))
+    _check("moe_route", rc)
+    return out
+
+
+def moe_dispatch(x: torch.Tensor, slot: torch.Tensor, gate: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(x, "x"); _need(slot, "slot")
+    T, d = x.shape
+    k = slot.shape[1]
+    if out is None:
+        out = torch.empty((T * k, d), dtype=x.dtype, device=x.device)
+    rc = lib.moe_dispatch(_ptr(x), _ptr(slot), _ptr(gate), T, d, k, _dtype_code(x.dtype),
+                          _ptr(out), _stream(x))
+    _check("moe_dispatch", rc)
+    return out
+
+
+def _w13(W1: torch.Tensor, W3: torch.Tensor):
+    # [E,F,d] tensors, or views into a fused [E,2F,d] gate/up tensor
+    E, F, d = W1.shape
+    stride = W1.stride(0)
+    if W3.stride(0) != stride or W1.stride(1) != d or W1.stride(2) != 1:
+        raise ValueError("W1/W3 must be [E,F,d] with rows contiguous and a common expert stride")
+    return E, F, d, stride
+
+
+def moe_grouped_gate_up(Xe, W1, W3, offsets, H: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(Xe, "Xe"); _need(offsets, "offsets")
+    E, F, d, s13 = _w13(W1, W3)
+    R = Xe.shape[0]
+    if H is None:
+        H = torch.empty((R, F), dtype=Xe.dtype, device=Xe.device)
+    rc = lib.moe_grouped_gate_up(_ptr(Xe), _ptr(W1), _ptr(W3), s13, _ptr(offsets), E, R, d, F,
+                                 _dtype_code(Xe.dtype), _ptr(H), _stream(Xe))
+    _check("moe_grouped_gate_up", rc)
+    return H
+
+
+def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(H, "H"); _need(W2, "W2"); _need(offsets, "offsets")
+    E, d, F = W2.shape
+    R = H.shape[0]
+    if Ye is None:
+        Ye = torch.empty((R, d), dtype=H.dtype, device=H.device)
+    rc = lib.moe_grouped_down(_ptr(H), _ptr(W2), W2.stride(0), _ptr(offsets), E, R, d, F,
+                              _dtype_code(H.dtype), _ptr(Ye), _stream(H))
+    _check("moe_grouped_down", rc)
+    return Ye
+
+
+def moe_grouped_swiglu(Xe, W1, W3, W2, offsets, H: Optional[torch.Tensor] = None,
+                       Ye: Optional[torch.Tensor] = None):
+    _need(Xe, "Xe"); _need(W2, "W2"); _need(offsets, "offsets")
+    E, F, d, s13 = _w13(W1, W3)
+    R = Xe.shape[0]
+    if H is None:
+        H = torch.empty((R, F), dtype=Xe.dtype, device=Xe.device)
+    if Ye is None:
+        Ye = torch.empty((R, d), dtype=Xe.dtype, device=Xe.device)
+    rc = lib.moe_grouped_swiglu(_ptr(Xe), _ptr(W1), _ptr(W3), _ptr(W2), s13, W2.stride(0),
+                                _ptr(offsets), E, R, d, F, _dtype_code(Xe.dtype), _ptr(H),
+                                _ptr(Ye), _stream(Xe))
+    _check("moe_grouped_swiglu", rc)
+    return H, Ye
+
+
+def moe_combine(Ye, slot, gate: Optional[torch.Tensor], out: Optional[torch.Tensor] = None):
+    _need(Ye, "Ye"); _need(slot, "slot")
+    T, k = slot.shape
+    d = Ye.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=Ye.dtype, device=Ye.device)
+    rc = lib.moe_combine(_ptr(Ye), _ptr(slot), _ptr(gate), T, d, k, _dtype_code(Ye.dtype),
+                         _ptr(out), _stream(Ye))
+    _check("moe_combine", rc)
+    return out
+
+
+def mxfp8_quantize(v: torch.Tensor, scale_mode: int = MOE_SCALE_E8M0, q=None, scales=None):
+    _need(v, "v")
+    rows, cols = v.shape
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=v.device)
+    if scales is None:
+        sdt = torch.float32 if scale_mode == MOE_SCALE_F32 else torch.uint8
+        scales = torch.empty((rows, cols // 32), dtype=sdt, device=v.device)
+    rc = lib.mxfp8_quantize(_ptr(v), _dtype_code(v.dtype), rows, cols, scale_mode, _ptr(q),
+                            _ptr(scales), _stream(v))
+    _check("mxfp8_quantize", rc)
+    return q, scales
+
+
+def mxfp8_dequantize(q: torch.Tensor, scales: torch.Tensor, scale_mode: int = MOE_SCALE_E8M0,
+                     out=None) -> torch.Tensor:
+    _need(q, "q"); _need(scales, "scales")
+    rows, cols = q.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=q.device)
+    rc = lib.mxfp8_dequantize(_ptr(q), _ptr(scales), scale_mode, rows, cols, _ptr(out), _stream(q))
+    _check("mxfp8_dequantize", rc)
+    return out
+
+
+def moe_layer_workspace_size(T, d, E, F, k, dtype: torch.dtype, logits_given: bool) -> int:
+    return lib.moe_layer_workspace_size(T, d, E, F, k, _dtype_code(dtype), int(logits_given))
+
+
+@dataclass
+class LayerOut:
+    out: torch.Tensor
+    idx: torch.Tensor
+    gate: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    slot: torch.Tensor
+    workspace: torch.Tensor
+
+
+def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool = False,
+                  out: Optional[LayerOut] = None) -> LayerOut:
+    _need(x, "x")
+    T, d = x.shape
+    E, F, _, s13 = _w13(W1, W3)
+    dev = x.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        ws = _alloc_ws(moe_layer_workspace_size(T, d, E, F, k, x.dtype, logits is not None), dev)
+        out = LayerOut(out=torch.empty((T, d), dtype=x.dtype, device=dev),
+                       idx=torch.empty((T, k), **i32),
+                       gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                       counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                       slot=torch.empty((T, k), **i32), workspace=ws)
+    a = LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(x.dtype), renorm=int(renorm),
+                  reserved0=0, x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1=_ptr(W1),
+                  W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13, w2_expert_stride=W2.stride(0),
+                  out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
+                  counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
+                  workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    rc = lib.moe_layer_fwd(ctypes.byref(a), _stream(x))
+    _check("moe_layer_fwd", rc)
+    return out
+
+
+def moe_get_status(clear: bool = True, device=None) -> int:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    v = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        rc = lib.moe_get_status(ctypes.byref(v), int(clear), torch.cuda.current_stream(dev).cuda_stream)
+    _check("moe_get_status", rc)
+    return int(v.value)
+
+
+def moe_version() -> str:
+    return lib.moe_version().decode()

@@ -1,0 +1,236 @@
+/*
+ * dropless top-k Mixture-of-Experts expert layer for NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument named as "device" is caller-owned device
+ * memory; the library never allocates, frees or synchronises (except
+ * moe_get_status, which reads the device status word). All work is enqueued
+ * on the caller's stream, passed as a `void*` holding a cudaStream_t
+ * (NULL = legacy default stream).
+ *
+ * Notation: T tokens, d hidden size, E experts, k experts per token, F expert
+ * FFN width, R = T*k rows of the expert-sorted buffers.
+ *
+ * Sources (page title, section) for what each call computes:
+ *   [HF]  "Transformers 中的 OLMoE：稀疏 MoE 语言模型架构解析与推理实践"
+ *         (blog.gitcode.com), §2 router, §3 experts, OlmoeConfig table.
+ *   [OF]  "olmoforge" README (git.onestrm.cn/huzjie/olmoforge), capability
+ *         table and MXFP8 block-quantisation sketch.
+ *   [NEWS] "专家池 8→128 只慢 5%：Ai2 开源万亿参数 MoE 训练框架 Olmo-core 3"
+ *         (xxqk.cn), section "三招拆分、三项优化、一个精度开关".
+ *   [REL] "OLMo-core 3 发布：主攻混合专家训练与导出校验" (wedoingai.com),
+ *         section "主要功能".
+ *
+ * Error behaviour (all calls): arguments are validated on the host before
+ * anything is enqueued. MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED mean nothing was
+ * launched. MOE_ERR_CUDA means a launch failed (the CUDA error is left for
+ * cudaGetLastError). Faults found on the device (a metadata value out of
+ * range, a pipeline wait that exceeded its time limit) set bits in a
+ * per-process device status word instead of trapping; the kernel that finds
+ * one skips the bad access and returns. Read it with moe_get_status.
+ * T == 0 is a valid no-op.
+ */
+#ifndef DROPLESS_TOP_MIXTURE_B200_MOE_H
+#define DROPLESS_TOP_MIXTURE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID (-1)     /* bad argument, nothing launched            */
+#define MOE_ERR_UNSUPPORTED (-2) /* shape/dtype outside what the build serves */
+#define MOE_ERR_CUDA (-3)        /* a CUDA call or launch failed              */
+
+/* element types */
+#define MOE_F32 0
+#define MOE_BF16 1
+#define MOE_E4M3 2
+
+/* MXFP8 scale encodings */
+#define MOE_SCALE_F32 0  /* fp32 scale = amax/448 (1.0 for an all-zero block)      */
+#define MOE_SCALE_E8M0 1 /* that value rounded up to a power of two, stored as the
+                            biased exponent byte (e + 127)                       */
+
+/* device status bits (moe_get_status) */
+#define MOE_DEVERR_TIMEOUT 1      /* a bounded pipeline wait gave up           */
+#define MOE_DEVERR_BAD_OFFSETS 2  /* offsets not monotone / not ending at R    */
+#define MOE_DEVERR_BAD_INDEX 4    /* an expert index or slot out of range      */
+
+/* limits of this build */
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 32
+#define MOE_TILE_M 128 /* rows per M-tile of the grouped GEMM and tile table */
+
+/* ------------------------------------------------------------------------
+ * moe_route — router logits (optional), fp32 softmax, top-k, and the
+ * GPU-resident routing metadata.
+ *
+ * [HF §2]: softmax over the E expert logits in fp32, torch.topk, optional
+ * norm_topk_prob renormalisation (off by default per the OlmoeConfig table);
+ * the router is a bias-free (E, d) weight. [OF capability table; NEWS]: the
+ * routing table stays on the device so the host never waits for it.
+ *
+ * Inputs (device):
+ *   logits   [T,E] fp32 row-major, or NULL to compute logits = x·Wrᵀ from
+ *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). The logit
+ *            of (t,e) is one fp32 accumulator updated by fused multiply-add
+ *            over j = 0..d-1 in ascending order, starting from +0.0.
+ *   renorm   0: gates are the softmax probabilities; 1: divided by their sum.
+ * Outputs (device, caller-allocated):
+ *   logits_out  [T,E] fp32, or NULL (used only when logits == NULL)
+ *   idx      [T,k] int32: expert indices by descending logit, ties to the
+ *            lower index (selection on the fp32 logits; NaN ranks as -inf)
+ *   gate     [T,k] fp32: softmax probability of idx[t,j] (fp32 arithmetic)
+ *   counts   [E]   int32 rows per expert
+ *   offsets  [E+1] int32 exclusive prefix sum of counts; offsets[E] = R
+ *   slot     [T,k] int32 row of (t,j) in the expert-sorted buffers: rows of
+ *            expert e are offsets[e].., in ascending token order
+ *   tile_offsets [E+1] int32 exclusive prefix sum of ceil(counts/128), or NULL
+ * Workspace: `workspace_bytes` >= moe_route_workspace_size(T, E, logits==NULL
+ *            && logits_out==NULL); 256-byte aligned device memory. Its
+ *            contents need not be initialised.
+ * Limits: 1 <= k <= min(E, 32), E <= 512, d % 32 == 0 when computing logits.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_route_workspace_size(int64_t T, int64_t E, int need_logits_buffer);
+MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dtype, int64_t T,
+                      int64_t d, int64_t E, int k, int renorm, float* logits_out, int32_t* idx,
+                      float* gate, int32_t* counts, int32_t* offsets, int32_t* slot,
+                      int32_t* tile_offsets, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_dispatch — row-wise dispatch: Xe[slot[t,j], :] = x[t, :].
+ *
+ * [OF capability table, row-wise expert parallelism]: each (token, k) row is
+ * written straight into its expert's contiguous input buffer; there is no
+ * separate permute. With `gate` non-NULL each copy is scaled:
+ * Xe[slot[t,j]] = round_dtype(fp32(gate[t,j]) * x[t]) (used to form the
+ * upstream gradient of the backward pass).
+ *   x [T,d], Xe [R,d] in `dtype` (MOE_F32 or MOE_BF16), rows contiguous,
+ *   16-byte aligned, d*elem_size % 16 == 0. slot [T,k] from moe_route.
+ * A slot outside [0,R) is skipped and sets MOE_DEVERR_BAD_INDEX.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_dispatch(const void* x, const int32_t* slot, const float* gate, int64_t T,
+                         int64_t d, int k, int dtype, void* Xe, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN over variable per-expert row counts.
+ *
+ * [HF §3]: per expert e, rows r in [offsets[e], offsets[e+1]):
+ *   H[r]  = silu(Xe[r]·W1_eᵀ) * (Xe[r]·W3_eᵀ)        (moe_grouped_gate_up)
+ *   Ye[r] = H[r]·W2_eᵀ                                (moe_grouped_down)
+ * [OF; NEWS]: all experts' small matmuls run as one grouped kernel.
+ * Tensor-core (tcgen05) products with fp32 accumulation; MOE_BF16 operands
+ * use bf16 MMA, MOE_F32 operands use tf32 MMA. H and Ye are stored in the
+ * same dtype.
+ *   Xe  [R,d]                      row-major
+ *   W1, W3  expert e at W + e*w13_expert_stride elements, each [F,d]
+ *           row-major (d contiguous). Separate [E,F,d] tensors use stride
+ *           F*d; the fused gate/up layout [E,2F,d] of [HF §3] uses W1 =
+ *           base, W3 = base + F*d, stride 2*F*d.
+ *   W2  expert e at W2 + e*w2_expert_stride elements, [d,F] row-major.
+ *   offsets [E+1] from moe_route (validated on the device: monotone, ending
+ *           at R; otherwise MOE_DEVERR_BAD_OFFSETS and nothing is written).
+ *   H   [R,F] device output/workspace; Ye [R,d] device output.
+ * Limits: d % 128 == 0, F % 128 == 0, E <= 512; every pointer 16-byte
+ * aligned; strides multiples of 8 elements.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
+                                int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
+                                int64_t R, int64_t d, int64_t F, int dtype, void* H,
+                                void* stream);
+MOE_API int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
+                             const int32_t* offsets, int64_t E, int64_t R, int64_t d, int64_t F,
+                             int dtype, void* Ye, void* stream);
+MOE_API int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, const void* W2,
+                               int64_t w13_expert_stride, int64_t w2_expert_stride,
+                               const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                               int64_t F, int dtype, void* H, void* Ye, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine — gate-weighted combine back to token order.
+ *
+ * [HF §3]: each expert output is multiplied by its top-k weight and added
+ * back at its token (index_add_). Here, per token, a gather:
+ *   out[t] = round_dtype( sum_{j=0..k-1} gate[t,j] * Ye[slot[t,j]] )
+ * accumulated in fp32 by fused multiply-add in ascending j, starting from 0.
+ * gate == NULL means unit gates (used for the input gradient in backward).
+ * No atomics: the result is deterministic.
+ *   Ye [R,d], out [T,d] in `dtype`; rows 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_combine(const void* Ye, const int32_t* slot, const float* gate, int64_t T,
+                        int64_t d, int k, int dtype, void* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 block quantisation [OF "MXFP8 分块量化"; NEWS].
+ *
+ * Blocks of 32 consecutive elements of each row share one scale:
+ *   s = fp32(amax/448) (1.0 if amax == 0); MOE_SCALE_E8M0 rounds s up to
+ *   the next power of two (exponent clamped to [-127,127]) and stores the
+ *   byte e+127. Codes: q = E4M3(fp32(v/s)), round-to-nearest-even,
+ *   saturating to ±448.
+ *   in [rows, cols] MOE_F32 or MOE_BF16; cols % 32 == 0
+ *   q [rows, cols] uint8 E4M3 codes; scales [rows, cols/32] fp32
+ *   (MOE_SCALE_F32) or uint8 (MOE_SCALE_E8M0).
+ * Dequantise: out_bf16 = bf16_rne(fp32(decode(q) * s)).
+ * ---------------------------------------------------------------------- */
+MOE_API int mxfp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols,
+                           int scale_mode, uint8_t* q, void* scales, void* stream);
+MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mode,
+                             int64_t rows, int64_t cols, void* out_bf16, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_layer_fwd — the whole layer: route -> dispatch -> grouped SwiGLU ->
+ * combine [HF §2-§3], enqueued on one stream with no host synchronisation.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_layer_args {
+    int64_t T, d, E, F;
+    int32_t k, dtype, renorm, reserved0;
+    /* inputs (device) */
+    const void* x;          /* [T,d]                                          */
+    const float* logits;    /* [T,E] fp32, or NULL to use Wr                  */
+    const void* Wr;         /* [E,d] (when logits == NULL)                    */
+    const void* W1;         /* see moe_grouped_gate_up                        */
+    const void* W3;
+    const void* W2;
+    int64_t w13_expert_stride, w2_expert_stride;
+    /* outputs (device) */
+    void* out;              /* [T,d]                                          */
+    int32_t* idx;           /* [T,k]                                          */
+    float* gate;            /* [T,k]                                          */
+    int32_t* counts;        /* [E]                                            */
+    int32_t* offsets;       /* [E+1]                                          */
+    int32_t* slot;          /* [T,k]                                          */
+    /* scratch (device): Xe [R,d], H [R,F], Ye [R,d] and the route workspace */
+    void* workspace;
+    size_t workspace_bytes;
+} moe_layer_args;
+
+MOE_API size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
+                                        int dtype, int logits_given);
+MOE_API int moe_layer_fwd(const moe_layer_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_get_status — read (and optionally clear) the device status word of the
+ * current device. Synchronises the given stream. *host_status receives an OR
+ * of MOE_DEVERR_* bits (0 = no fault seen).
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_get_status(int32_t* host_status, int clear, void* stream);
+
+/* library version string */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DROPLESS_TOP_MIXTURE_B200_MOE_H */

@@ -303,17 +303,22 @@ def moe_layer(x: torch.Tensor, k: int, W1, W3, W2, *, logits: Optional[np.ndarra
 
 def moe_layer_tokens(x: torch.Tensor, tokens: np.ndarray, idx: np.ndarray, gate: np.ndarray,
                      W1, W3, W2) -> np.ndarray:
-    """out[t] for a sample of tokens, one token at a time (for full-size
-    workloads where the whole layer would take too long on the CPU)."""
+    """out[t] for a sample of tokens (for full-size workloads where the whole
+    layer would take too long on the CPU): the per-token formula
+    out[t] = sum_j gate[t,j] W2_e(silu(W1_e x_t) * W3_e x_t), visiting each
+    needed expert once."""
+    tokens = np.asarray(tokens)
     xs = to64(x[torch.as_tensor(tokens, dtype=torch.long)])
-    d = xs.shape[1]
-    out = np.zeros((len(tokens), d))
-    for i, t in enumerate(tokens):
-        for j in range(idx.shape[1]):
-            e = int(idx[t, j])
-            w1, w3, w2 = to64(W1[e]), to64(W3[e]), to64(W2[e])
-            h = silu(w1 @ xs[i]) * (w3 @ xs[i])
-            out[i] += gate[t, j] * (w2 @ h)
+    out = np.zeros((len(tokens), xs.shape[1]))
+    sel = idx[tokens]
+    for e in np.unique(sel):
+        e = int(e)
+        rows, js = np.nonzero(sel == e)
+        w1, w3, w2 = to64(W1[e]), to64(W3[e]), to64(W2[e])
+        X = xs[rows]
+        h = silu(X @ w1.T) * (X @ w3.T)
+        y = h @ w2.T
+        out[rows] += gate[tokens[rows], js][:, None] * y
     return out
 
 

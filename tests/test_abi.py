@@ -1,0 +1,82 @@
+"""The C-ABI library loads, exports every symbol include/*.h declares, and
+rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dropless_top_mixture_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("moe_route", "moe_dispatch", "moe_grouped_swiglu", "moe_combine", "mxfp8_quantize",
+              "mxfp8_dequantize", "moe_layer_fwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_symbol():
+    from dropless_top_mixture_b200 import moe
+    assert set(_declared()) <= set(moe.exported_symbols())
+
+
+def test_host_validation_rejects_without_launch(lib):
+    from dropless_top_mixture_b200 import moe as m
+    L = m.lib
+    buf = ctypes.create_string_buffer(1 << 16)
+    p = ctypes.addressof(buf)
+    p16 = (p + 255) & ~255
+    # k > E
+    assert L.moe_route(p16, None, None, 0, 10, 0, 4, 5, 0, None, p16, p16, p16, p16, p16, None,
+                       p16, 4096, None) == m.MOE_ERR_INVALID
+    # E beyond the build limit
+    assert L.moe_route(p16, None, None, 0, 10, 0, 1000, 2, 0, None, p16, p16, p16, p16, p16, None,
+                       p16, 4096, None) == m.MOE_ERR_INVALID
+    # workspace too small
+    assert L.moe_route(p16, None, None, 0, 1000, 0, 64, 2, 0, None, p16, p16, p16, p16, p16, None,
+                       p16, 16, None) == m.MOE_ERR_INVALID
+    # d not a multiple of 128 for the grouped GEMM
+    assert L.moe_grouped_gate_up(p16, p16, p16, 96 * 128, p16, 4, 100, 96, 128, m.MOE_BF16, p16,
+                                 None) == m.MOE_ERR_UNSUPPORTED
+    # unsupported dtype
+    assert L.moe_dispatch(p16, p16, None, 4, 64, 2, 7, p16, None) == m.MOE_ERR_UNSUPPORTED
+    # misaligned pointer
+    assert L.moe_combine(p16 + 2, p16, None, 4, 64, 2, m.MOE_BF16, p16, None) == m.MOE_ERR_INVALID
+    # MXFP8 columns must be whole blocks
+    assert L.mxfp8_quantize(p16, m.MOE_BF16, 4, 48, m.MOE_SCALE_E8M0, p16, p16, None) == m.MOE_ERR_INVALID
+    # T == 0 is a no-op
+    assert L.moe_dispatch(p16, p16, None, 0, 64, 2, m.MOE_BF16, p16, None) == m.MOE_OK
+    assert L.moe_layer_fwd(None, None) == m.MOE_ERR_INVALID
+
+
+def test_workspace_sizes_are_consistent(lib):
+    from dropless_top_mixture_b200 import moe as m
+    a = m.lib.moe_route_workspace_size(16384, 64, 1)
+    b = m.lib.moe_route_workspace_size(16384, 64, 0)
+    assert a - b >= 16384 * 64 * 4
+    T, d, E, F, k = 16384, 2048, 64, 1024, 8
+    ws = m.lib.moe_layer_workspace_size(T, d, E, F, k, m.MOE_BF16, 0)
+    R = T * k
+    assert ws >= 2 * (R * d * 2 + R * F * 2 // 2) + b

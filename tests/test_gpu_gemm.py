@@ -1,0 +1,154 @@
+"""Grouped SwiGLU GEMMs (tcgen05) and the whole layer on the GPU against the
+oracle: small shapes that span several tiles with ragged tails and empty
+experts, then every workload at full size on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
+from tests._util import assert_close_layer, assert_close_scaled, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _moe():
+    from dropless_top_mixture_b200 import moe
+    return moe
+
+
+def _problem(T, d, F, E, k, dtype, seed, skew=True):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, d, generator=g).to(dtype)
+    s_in, s_mid = d ** -0.5, F ** -0.5
+    W1 = (torch.randn(E, F, d, generator=g) * s_in).to(dtype)
+    W3 = (torch.randn(E, F, d, generator=g) * s_in).to(dtype)
+    W2 = (torch.randn(E, d, F, generator=g) * s_mid).to(dtype)
+    lg = adversarial_logits(T, E, "normal", seed=seed).numpy()
+    if skew and E >= 4:
+        lg[:, 1] -= 40.0   # expert 1 empty
+        lg[:, 0] += 3.0    # expert 0 heavy (several tiles)
+    return x, W1, W3, W2, lg
+
+
+def _expert_ref(x, W1, W3, W2, lg, k):
+    E = W1.shape[0]
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    Xe = O.dispatch(x.double().numpy(), meta["slot"])
+    Ye, A, B, H = O.expert_ffn(Xe, meta["offsets"], np64(W1), np64(W3), np64(W2), keep=True)
+    return meta, gate, Xe, H, Ye
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,d,F,E,k", [(300, 256, 256, 5, 2), (129, 128, 384, 3, 1),
+                                       (700, 512, 128, 16, 4), (5, 256, 128, 4, 2),
+                                       (1000, 384, 256, 7, 3)])
+def test_grouped_swiglu_small(dtype, T, d, F, E, k):
+    moe = _moe()
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, dtype, seed=T + d + F)
+    meta, gate, Xe_ref, H_ref, Ye_ref = _expert_ref(x, W1, W3, W2, lg, k)
+    dev = "cuda"
+    Xe = torch.from_numpy(Xe_ref).to(dtype).to(dev)  # exact: Xe rows are rows of x
+    offs = torch.from_numpy(meta["offsets"]).to(dev)
+    H, Ye = moe.moe_grouped_swiglu(Xe, W1.to(dev), W3.to(dev), W2.to(dev), offs)
+    assert moe.moe_get_status() == 0
+    assert_close_scaled(np64(H), H_ref, "H")
+    assert_close_scaled(np64(Ye), Ye_ref, "Ye")
+
+
+def test_grouped_gate_up_fused_gate_up_layout():
+    """W1/W3 as the two halves of one [E, 2F, d] gate_up tensor."""
+    moe = _moe()
+    T, d, F, E, k = 400, 256, 256, 6, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=42)
+    meta, gate, Xe_ref, H_ref, Ye_ref = _expert_ref(x, W1, W3, W2, lg, k)
+    gate_up = torch.cat([W1, W3], dim=1).cuda()
+    Xe = torch.from_numpy(Xe_ref).to(torch.bfloat16).cuda()
+    H = moe.moe_grouped_gate_up(Xe, gate_up[:, :F], gate_up[:, F:],
+                                torch.from_numpy(meta["offsets"]).cuda())
+    assert_close_scaled(np64(H), H_ref, "H")
+
+
+def test_grouped_gemm_deterministic():
+    moe = _moe()
+    T, d, F, E, k = 600, 512, 256, 8, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=7)
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    Xe = moe.moe_dispatch(x.cuda(), torch.from_numpy(meta["slot"]).cuda())
+    offs = torch.from_numpy(meta["offsets"]).cuda()
+    a = moe.moe_grouped_swiglu(Xe, W1.cuda(), W3.cuda(), W2.cuda(), offs)
+    b = moe.moe_grouped_swiglu(Xe, W1.cuda(), W3.cuda(), W2.cuda(), offs)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_bad_offsets_flagged_not_faulted():
+    moe = _moe()
+    d, F, E = 128, 128, 4
+    Xe = torch.zeros(256, d, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(E, F, d, dtype=torch.bfloat16, device="cuda")
+    W2 = torch.zeros(E, d, F, dtype=torch.bfloat16, device="cuda")
+    offs = torch.tensor([0, 100, 50, 200, 256], dtype=torch.int32, device="cuda")  # not monotone
+    H = torch.full((256, F), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_grouped_gate_up(Xe, W, W, offs, H=H)
+    st = moe.moe_get_status(clear=True)
+    assert st & moe.MOE_DEVERR_BAD_OFFSETS
+    assert (H == 7.0).all()  # nothing written
+    assert moe.moe_get_status() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_layer_small_full_check(dtype):
+    moe = _moe()
+    T, d, F, E, k = 777, 256, 384, 12, 3
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, dtype, seed=99)
+    Wr = (torch.randn(E, d, generator=torch.Generator().manual_seed(5)) * 0.05).to(dtype)
+    r = moe.moe_layer_fwd(x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda(), Wr=Wr.cuda())
+    ref = O.moe_layer(x, k, W1, W3, W2, Wr=Wr)
+    assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
+    assert np.array_equal(r.slot.cpu().numpy(), ref["slot"])
+    assert np.array_equal(r.offsets.cpu().numpy(), ref["offsets"])
+    assert_close_scaled(np64(r.out), ref["out"], "out")
+    assert moe.moe_get_status() == 0
+
+
+def test_layer_tiny_fp32_workload_full():
+    moe = _moe()
+    w = WORKLOADS["tiny_fp32"]
+    inp = make_inputs(w, "cpu")
+    dev = {k_: v.cuda() for k_, v in inp.items()}
+    r = moe.moe_layer_fwd(dev["x"], w.k, dev["W1"], dev["W3"], dev["W2"], Wr=dev["Wr"])
+    ref = O.moe_layer(inp["x"], w.k, inp["W1"], inp["W3"], inp["W2"], Wr=inp["Wr"])
+    assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
+    assert np.array_equal(r.counts.cpu().numpy(), ref["counts"])
+    assert_close_layer(np64(r.out), ref["out"], "out")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["olmoe_1b7b", "sweep_e8", "sweep_e32", "sweep_e128",
+                                  "sweep_e128_zipf", "fine_grained_e384"])
+def test_layer_full_size_sampled(name):
+    """Full-size workload in the launch configuration the benchmark times;
+    routing checked in full, the output on 64 sampled tokens."""
+    moe = _moe()
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cuda")
+    kw = dict(Wr=inp["Wr"]) if w.logits == "router" else dict(logits=inp["logits"])
+    r = moe.moe_layer_fwd(inp["x"], w.k, inp["W1"], inp["W3"], inp["W2"], **kw)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    x_cpu = inp["x"].cpu()
+    lg = (O.router_logits(x_cpu, inp["Wr"].cpu()) if w.logits == "router"
+          else inp["logits"].cpu().numpy())
+    idx, gate, _ = O.route(lg, w.k)
+    meta = O.routing_metadata(idx, w.E)
+    assert np.array_equal(r.idx.cpu().numpy(), idx)
+    assert np.array_equal(r.slot.cpu().numpy(), meta["slot"])
+    assert np.array_equal(r.offsets.cpu().numpy(), meta["offsets"])
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(w.T, size=64, replace=False))
+    toks[0], toks[-1] = 0, w.T - 1
+    ref = O.moe_layer_tokens(x_cpu, toks, idx, gate, inp["W1"], inp["W3"], inp["W2"])
+    got = np64(r.out[torch.as_tensor(toks, device="cuda")])
+    assert_close_layer(got, ref, name)

@@ -1,0 +1,97 @@
+"""Route step on the GPU against the oracle: indices, counts, offsets, slots
+and tile offsets bit-exact; gates within the fp32 softmax bound."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
+from tests._util import gate_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+def _moe():
+    from dropless_top_mixture_b200 import moe
+    return moe
+
+
+def _check_route(r, lg_np, k, E, renorm=False):
+    idx, gate, _ = O.route(lg_np, k, renorm)
+    meta = O.routing_metadata(idx, E)
+    g_idx = r.idx.cpu().numpy()
+    assert np.array_equal(g_idx, idx), "top-k indices differ"
+    assert np.array_equal(r.counts.cpu().numpy(), meta["counts"])
+    assert np.array_equal(r.offsets.cpu().numpy(), meta["offsets"])
+    assert np.array_equal(r.slot.cpu().numpy(), meta["slot"])
+    assert np.array_equal(r.tile_offsets.cpu().numpy(), meta["tile_offsets"])
+    g = r.gate.cpu().numpy().astype(np.float64)
+    tol = gate_tolerance(lg_np, idx, renorm)
+    err = np.abs(g - gate) / np.maximum(np.abs(gate), 1e-300)
+    assert np.all((err <= tol) | (gate == 0)), f"gate rel err {err.max():.3e}"
+
+
+@pytest.mark.parametrize("kind", ["normal", "dups", "constant", "signed_zero"])
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (7, 8, 8), (37, 33, 5), (300, 64, 8), (1000, 128, 4),
+                                   (257, 384, 8), (64, 512, 32), (50, 1, 1)])
+def test_route_from_logits_bitexact(kind, T, E, k):
+    moe = _moe()
+    lg = adversarial_logits(T, E, kind, seed=T + E)
+    r = moe.moe_route(k, logits=lg.cuda())
+    _check_route(r, lg.numpy(), k, E)
+
+
+def test_route_renorm():
+    moe = _moe()
+    lg = adversarial_logits(333, 64, "normal", seed=5)
+    r = moe.moe_route(8, logits=lg.cuda(), renorm=True)
+    _check_route(r, lg.numpy(), 8, 64, renorm=True)
+
+
+def test_route_skewed_with_empty_experts():
+    moe = _moe()
+    T, E, k = 2000, 40, 3
+    lg = adversarial_logits(T, E, "normal", seed=11)
+    lg[:, 10:30] -= 50.0  # experts 10..29 never chosen
+    lg[:, 0] += 5.0       # expert 0 always chosen (> 128 rows: several tiles)
+    r = moe.moe_route(k, logits=lg.cuda())
+    _check_route(r, lg.numpy(), k, E)
+    assert (r.counts.cpu().numpy()[10:30] == 0).all()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T,d,E,k", [(5, 128, 8, 2), (130, 256, 64, 8), (77, 64, 33, 3)])
+def test_router_logits_bitexact(dtype, T, d, E, k):
+    moe = _moe()
+    g = torch.Generator().manual_seed(T * d + E)
+    x = torch.randn(T, d, generator=g).to(dtype)
+    Wr = (torch.randn(E, d, generator=g) * 0.02).to(dtype)
+    r = moe.moe_route(k, x=x.cuda(), Wr=Wr.cuda(), keep_logits=True)
+    ref = O.router_logits(x, Wr)
+    assert np.array_equal(r.logits.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    _check_route(r, ref, k, E)
+
+
+def test_route_empty_batch():
+    moe = _moe()
+    lg = torch.zeros((0, 16), device="cuda")
+    r = moe.moe_route(4, logits=lg)
+    assert (r.counts.cpu() == 0).all() and (r.offsets.cpu() == 0).all()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["tiny_fp32", "olmoe_1b7b", "sweep_e8", "sweep_e128_zipf",
+                                  "fine_grained_e384"])
+def test_route_full_size_workloads(name):
+    moe = _moe()
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cpu", weights=False)
+    if w.logits == "router":
+        r = moe.moe_route(w.k, x=inp["x"].cuda(), Wr=inp["Wr"].cuda(), keep_logits=True)
+        lg = O.router_logits(inp["x"], inp["Wr"])
+        assert np.array_equal(r.logits.cpu().numpy().view(np.uint32), lg.view(np.uint32))
+    else:
+        r = moe.moe_route(w.k, logits=inp["logits"].cuda())
+        lg = inp["logits"].numpy()
+    _check_route(r, lg, w.k, w.E)
+    assert moe.moe_get_status() == 0
