@@ -296,7 +296,7 @@ def run_ours(args):
         if ev is not None:
             ev[5].record()
 
-    sampler = ClockSampler(local) if rank == 0 else None
+    sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -437,6 +437,8 @@ def main(argv=None):
                     help="tokens per step of the CPU-oracle reference arm")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="skip nvidia-smi clock sampling (for runs under a profiler)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps; the line reports it
     if args.impl == "reference":
