@@ -64,6 +64,8 @@ _SIGS = {
     "moe_route_workspace_size": (_sz, [_i64, _i64, _i32]),
     "moe_route": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _p, _p, _p, _p, _p,
                          _p, _p, _sz, _p]),
+    "moe_route_noalloc": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _p, _p, _p,
+                                 _p, _p, _p, _p]),
     "moe_dispatch": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
     "moe_grouped_gate_up": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_grouped_down": (_i32, [_p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
@@ -166,6 +168,28 @@ def moe_route(k: int, *, logits: Optional[torch.Tensor] = None, x: Optional[torc
                        _ptr(out.offsets), _ptr(out.slot), _ptr(out.tile_offsets),
                        _ptr(workspace), workspace.numel(), _stream(workspace))
     _check("moe_route", rc)
+    return out
+
+
+def moe_route_noalloc(k: int, *, logits: Optional[torch.Tensor] = None,
+                      x: Optional[torch.Tensor] = None, Wr: Optional[torch.Tensor] = None,
+                      renorm: bool = False, out: Route) -> Route:
+    """moe_route with the library's own scratch: the caller passes every
+    output (``out``) and no workspace; nothing is allocated here either."""
+    if logits is not None:
+        _need(logits, "logits")
+        T, E = logits.shape
+        dtype, d, dev_t = MOE_F32, 0, logits
+    else:
+        _need(x, "x"); _need(Wr, "Wr")
+        T, d = x.shape
+        E = Wr.shape[0]
+        dtype, dev_t = _dtype_code(x.dtype), x
+    rc = lib.moe_route_noalloc(_ptr(logits), _ptr(x), _ptr(Wr), dtype, T, d, E, k, int(renorm),
+                               _ptr(out.logits), _ptr(out.idx), _ptr(out.gate), _ptr(out.counts),
+                               _ptr(out.offsets), _ptr(out.slot), _ptr(out.tile_offsets),
+                               _stream(dev_t))
+    _check("moe_route_noalloc", rc)
     return out
 
 

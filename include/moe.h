@@ -109,6 +109,38 @@ MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dt
                       void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_route_noalloc — moe_route without a caller workspace.
+ *
+ * No counterpart in the pages: this is an interface convenience of this
+ * library. It is for callers that cannot allocate device memory (an enqueue
+ * callback that is given only tensors and a stream, or a process whose memory
+ * pool owns the device, where cudaMalloc would synchronise or fail). It
+ * computes exactly what moe_route computes, with the same arguments minus
+ * `workspace`/`workspace_bytes`; its scratch is a library-owned device array
+ * of MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU loading the library
+ * keeps reserved until the process exits.
+ *   - Size limit: moe_route_workspace_size(T, E, logits == NULL &&
+ *     logits_out == NULL) must not exceed MOE_ROUTE_NOALLOC_SCRATCH_BYTES,
+ *     else MOE_ERR_UNSUPPORTED and nothing is launched. (E = 64 with logits
+ *     computed from x fits up to T = 29,121 tokens; E = 128 with logits
+ *     given up to T = 131,057; E = 384 with logits given up to T = 43,681.)
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture begins.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents; calls whose work can overlap on the GPU (different streams
+ *     without ordering, or different host threads) race on it and must be
+ *     serialised by the caller.
+ *   - It calls no cudaMalloc/cudaFree and allocates nothing.
+ * ---------------------------------------------------------------------- */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (8u << 20)
+MOE_API int moe_route_noalloc(const float* logits, const void* x, const void* Wr, int dtype,
+                              int64_t T, int64_t d, int64_t E, int k, int renorm,
+                              float* logits_out, int32_t* idx, float* gate, int32_t* counts,
+                              int32_t* offsets, int32_t* slot, int32_t* tile_offsets,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_dispatch — row-wise dispatch: Xe[slot[t,j], :] = x[t, :].
  *
  * [OF capability table, row-wise expert parallelism]: each (token, k) row is
