@@ -96,12 +96,16 @@ __global__ void __launch_bounds__(THREADS) dispatch_kernel(const uint4* __restri
 }
 
 // out[t] = sum_j gate[t,j] * Ye[slot[t,j]]  (UNIT: gate == 1)
+// Each thread owns one 16-byte column vector of a token and issues the loads
+// of up to JB rows before it accumulates them, so JB loads are in flight per
+// thread; the accumulation itself stays in ascending j.
 template <int DT, bool UNIT>
 __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restrict__ Ye,
                                                           const int32_t* __restrict__ slot,
                                                           const float* __restrict__ gate, int T,
                                                           int k, int vpr, int64_t R,
                                                           uint4* __restrict__ out, int* status) {
+    constexpr int JB = 8;
     __shared__ int s_slot[MOE_MAX_TOPK];
     __shared__ float s_gate[MOE_MAX_TOPK];
     constexpr int N = Vec<DT>::N;
@@ -117,38 +121,30 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
             s_gate[threadIdx.x] = UNIT ? 1.f : gate[(size_t)t * k + threadIdx.x];
         }
         __syncthreads();
-        for (int v0 = threadIdx.x; v0 < vpr; v0 += THREADS * UNROLL) {
-            float acc[UNROLL][N];
+        for (int v = threadIdx.x; v < vpr; v += THREADS) {
+            float acc[N];
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u)
+            for (int q = 0; q < N; ++q) acc[q] = 0.f;
+            for (int j0 = 0; j0 < k; j0 += JB) {
+                uint4 val[JB];
 #pragma unroll
-                for (int q = 0; q < N; ++q) acc[u][q] = 0.f;
-            for (int j = 0; j < k; ++j) {
-                const int s = s_slot[j];
-                if (s < 0) continue;
-                const uint4* src = Ye + (size_t)s * vpr;
-                const float g = s_gate[j];
-                uint4 val[UNROLL];
-#pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
-                    const int v = v0 + u * THREADS;
-                    if (v < vpr) val[u] = __ldcs(src + v);
+                for (int jj = 0; jj < JB; ++jj) {
+                    const int j = j0 + jj;
+                    const int s = (j < k) ? s_slot[j] : -1;
+                    if (s >= 0) val[jj] = __ldcs(Ye + (size_t)s * vpr + v);
                 }
 #pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
-                    const int v = v0 + u * THREADS;
-                    if (v >= vpr) continue;
+                for (int jj = 0; jj < JB; ++jj) {
+                    const int j = j0 + jj;
+                    if (j >= k || s_slot[j] < 0) continue;
+                    const float g = s_gate[j];
                     float f[N];
-                    Vec<DT>::load(val[u], f);
+                    Vec<DT>::load(val[jj], f);
 #pragma unroll
-                    for (int q = 0; q < N; ++q) acc[u][q] = fmaf(g, f[q], acc[u][q]);
+                    for (int q = 0; q < N; ++q) acc[q] = fmaf(g, f[q], acc[q]);
                 }
             }
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int v = v0 + u * THREADS;
-                if (v < vpr) out[(size_t)t * vpr + v] = Vec<DT>::store(acc[u]);
-            }
+            out[(size_t)t * vpr + v] = Vec<DT>::store(acc);
         }
     }
 }

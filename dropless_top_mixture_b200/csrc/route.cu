@@ -66,72 +66,87 @@ struct Stage8<float> {
     }
 };
 
-// One CTA computes a 64-token x 64-expert tile. Thread (ty, tx) owns tokens
-// 4ty..4ty+3 and experts 4tx..4tx+3, each with its own fp32 accumulator
-// updated in ascending j, so every logit is the same sequential fmaf chain
-// the definition states. Rows of x and Wr are staged 32 columns at a time,
-// transposed into k-major shared memory; the next chunk is prefetched into
-// registers while the current one is consumed.
+// One CTA (128 threads) computes a 64-token x 64-expert tile. Thread (ty, tx)
+// owns tokens 8ty..8ty+7 and experts 4tx..4tx+3, each with its own fp32
+// accumulator updated in ascending j, so every logit is the same sequential
+// fmaf chain the definition states. Rows of x and Wr are staged 32 columns at
+// a time, transposed into k-major shared memory (two buffers, one barrier per
+// chunk); the next chunk is prefetched into registers while the current
+// one is consumed. Per column: 3 shared loads feed 32 FMAs.
+constexpr int LOGIT_THREADS = 128;
+
 template <typename TX>
-__global__ void __launch_bounds__(256) router_logits_kernel(const TX* __restrict__ x,
-                                                            const TX* __restrict__ Wr, int T,
-                                                            int d, int E,
-                                                            float* __restrict__ logits) {
-    __shared__ __align__(16) float xs[LOGIT_TK][LOGIT_LD];
-    __shared__ __align__(16) float ws[LOGIT_TK][LOGIT_LD];
+__global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* __restrict__ x,
+                                                                      const TX* __restrict__ Wr,
+                                                                      int T, int d, int E,
+                                                                      float* __restrict__ logits) {
+    __shared__ __align__(16) float xs[2][LOGIT_TK][LOGIT_LD];
+    __shared__ __align__(16) float ws[2][LOGIT_TK][LOGIT_LD];
     const int tid = threadIdx.x;
     const int t0 = blockIdx.x * LOGIT_TT;
     const int e0 = blockIdx.y * LOGIT_TE;
-    // staging role: row = tid / 4 (token or expert), columns (tid % 4) * 8 .. +7
-    const int srow = tid >> 2;
-    const int scol = (tid & 3) * 8;
+    // staging role: row = tid / 2 (token or expert), columns (tid % 2) * 16 .. +15
+    const int srow = tid >> 1;
+    const int scol = (tid & 1) * 16;
     const bool xok = (t0 + srow) < T;
     const bool wok = (e0 + srow) < E;
     const TX* xp = x + (size_t)(t0 + srow) * d + scol;
     const TX* wp = Wr + (size_t)(e0 + srow) * d + scol;
     // compute role
     const int ty = tid >> 4, tx = tid & 15;
-    float acc[4][4];
+    float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-    float fx[8], fw[8];
+    float fx[16], fw[16];
     Stage8<TX>::load(xp, xok, fx);
+    Stage8<TX>::load(xp + 8, xok, fx + 8);
     Stage8<TX>::load(wp, wok, fw);
-    for (int k0 = 0; k0 < d; k0 += LOGIT_TK) {
-        __syncthreads();
+    Stage8<TX>::load(wp + 8, wok, fw + 8);
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += LOGIT_TK, buf ^= 1) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            xs[scol + i][srow] = fx[i];
-            ws[scol + i][srow] = fw[i];
+        for (int i = 0; i < 16; ++i) {
+            xs[buf][scol + i][srow] = fx[i];
+            ws[buf][scol + i][srow] = fw[i];
         }
         __syncthreads();
         if (k0 + LOGIT_TK < d) {
             Stage8<TX>::load(xp + k0 + LOGIT_TK, xok, fx);
+            Stage8<TX>::load(xp + k0 + LOGIT_TK + 8, xok, fx + 8);
             Stage8<TX>::load(wp + k0 + LOGIT_TK, wok, fw);
+            Stage8<TX>::load(wp + k0 + LOGIT_TK + 8, wok, fw + 8);
         }
-#pragma unroll 8
+#pragma unroll 4
         for (int kk = 0; kk < LOGIT_TK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8 + 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
+        // no second barrier: the next chunk goes to the other buffer, and the
+        // barrier after that write keeps any thread from overwriting this
+        // buffer before every thread has finished reading it
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + ty * 8 + i;
         if (t >= T) continue;
+        const int e = e0 + tx * 4;
+        if (e + 3 < E && (E & 3) == 0) {
+            *reinterpret_cast<float4*>(&logits[(size_t)t * E + e]) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + tx * 4 + j;
-            if (e < E) logits[(size_t)t * E + e] = acc[i][j];
+            for (int j = 0; j < 4; ++j)
+                if (e + j < E) logits[(size_t)t * E + e + j] = acc[i][j];
         }
     }
 }
@@ -436,11 +451,11 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
         dim3 grid((unsigned)((T + route::LOGIT_TT - 1) / route::LOGIT_TT),
                   (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE));
         if (dtype == MOE_BF16)
-            route::router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            route::router_logits_kernel<__nv_bfloat16><<<grid, route::LOGIT_THREADS, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
                 (int)T, (int)d, (int)E, dst);
         else
-            route::router_logits_kernel<float><<<grid, 256, 0, st>>>(
+            route::router_logits_kernel<float><<<grid, route::LOGIT_THREADS, 0, st>>>(
                 static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d,
                 (int)E, dst);
         lg = dst;
