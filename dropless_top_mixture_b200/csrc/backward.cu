@@ -1,0 +1,503 @@
+// Backward of the grouped SwiGLU expert FFN on tcgen05 (sm_100a).
+//
+// For each expert e and its rows r in [offsets[e], offsets[e+1]), with the
+// forward's pre-activations A = Xe W1_eᵀ, B = Xe W3_eᵀ, H = silu(A) * B and
+// the upstream rows dYe (= gate * dOut[token], formed by the scaled dispatch):
+//   dH  = dYe W2_e                               K = d
+//   dA  = dH * B * silu'(A),  dB = dH * silu(A)  (pairwise SwiGLU backward,
+//         fused into the dH epilogue; "OLMo-core 3 发布：主攻混合专家训练与导出校验",
+//         主要功能: optional pairwise SwiGLU backward)
+//   dXe = dA W1_e + dB W3_e                      K = 2F
+//   dW1_e = dAᵀ Xe,  dW3_e = dBᵀ Xe,  dW2_e = dYeᵀ H   K = rows of e
+// silu'(a) = s (1 + a (1 - s)), s = sigmoid(a). Weight gradients are written
+// in bf16 from fp32 accumulators (the same release notes: bf16 weight
+// gradients). The router and gate gradients are not part of this pass.
+//
+// One kernel template, three modes, the same pipeline as the forward grouped
+// GEMM (TMA producer warp, single-thread tcgen05.mma issue, 4 epilogue warps,
+// 4-stage shared-memory ring, double-buffered 128x256 fp32 TMEM accumulator):
+//   DH  A = dYe rows (K-major), B = W2_e read as [F x d] (MN-major, F
+//       contiguous); epilogue loads A,B of the same rows/columns and writes dA, dB.
+//   DX  A = dA then dB rows (K-major), B = W1_e then W3_e read as [d x F]
+//       (MN-major, d contiguous); epilogue writes dXe.
+//   DW  per expert a 128 x 256 tile of the [M x N] gradient; A and B are the
+//       expert's rows of two [R x M] / [R x N] matrices, both MN-major, with K
+//       running over the rows. The last K slab of an expert can reach into the
+//       next expert's rows: those rows are zeroed in shared memory before the
+//       MMA reads them. An expert with no rows writes zeros.
+#include "tc_sm100.cuh"
+
+namespace moe {
+namespace bwd {
+
+using namespace tc;
+
+constexpr int BM = 128;
+constexpr int MMA_N = 256;
+constexpr int BK = 64;  // bf16 elements per 128-byte slab
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * 128;
+constexpr int B_BYTES = MMA_N * 128;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BOX_BYTES = 64 * 128;  // one MN-major box: 64 K rows x 64 elements
+constexpr int TMEM_ALLOC = 512;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + META_BYTES;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+enum Mode { DH = 0, DX = 1, DW = 2 };
+
+template <int MODE>
+struct ModeCfg {
+    static constexpr bool A_MN = (MODE == DW);
+    static constexpr uint32_t IDESC = make_idesc_major(1u, BM, MMA_N, A_MN, true);
+};
+
+struct Tile {
+    int e, row0, row_end, m0, n0, kb0, nkb;
+};
+
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + __expf(-a)); }
+
+template <int MODE>
+__device__ __forceinline__ Tile decode(int t, int E, int NB, int MB, int K, const int* s_toff,
+                                       const int* s_off) {
+    Tile tl;
+    if (MODE == DW) {
+        const int tpe = MB * NB;
+        const int e = t / tpe;
+        const int l = t - e * tpe;
+        const int nb = l / MB, mb = l - nb * MB;
+        tl.e = e;
+        tl.row0 = s_off[e];
+        tl.row_end = s_off[e + 1];
+        tl.m0 = mb * BM;
+        tl.n0 = nb * MMA_N;
+        tl.kb0 = 0;
+        tl.nkb = (tl.row_end - tl.row0 + BK - 1) / BK;
+    } else {
+        const int q = t / NB;
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_toff[mid] <= q) lo = mid;
+            else hi = mid - 1;
+        }
+        const int Me = s_toff[lo + 1] - s_toff[lo];
+        const int l = t - s_toff[lo] * NB;
+        const int nb = l / Me, m = l - nb * Me;
+        tl.e = lo;
+        tl.row0 = s_off[lo] + m * BM;
+        tl.row_end = s_off[lo + 1];
+        tl.m0 = 0;
+        tl.n0 = nb * MMA_N;
+        tl.kb0 = 0;
+        tl.nkb = K / BK;
+    }
+    return tl;
+}
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = pack8(v + 8 * i);
+}
+
+__device__ __forceinline__ void load32_bf16(const __nv_bfloat16* src, float* v) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack8(__ldg(s + i), v + 8 * i);
+}
+
+// tmA0/tmA1/tmB0/tmB1: see the mode table at the top of the file.
+//   K      DH: d; DX: 2F (KF = K/2 slabs per operand pair); DW: unused
+//   Mdim   DW: rows of each expert's gradient (F or d)
+//   Ndim   DH: F; DX: d; DW: columns of each expert's gradient
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                    const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1,
+                    const int32_t* __restrict__ offsets, int E, int R, int K, int Mdim, int Ndim,
+                    __nv_bfloat16* __restrict__ out0, __nv_bfloat16* __restrict__ out1,
+                    int64_t ldo, const __nv_bfloat16* __restrict__ saveA,
+                    const __nv_bfloat16* __restrict__ saveB, int* status) {
+    using C = ModeCfg<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* meta = smem + STAGES * STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // --- routing offsets -> tile table (validated) -----------------------
+    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int m = 0;
+            if (e < E) {
+                const int cnt = s_off[e + 1] - s_off[e];
+                if (cnt < 0) bad = true;
+                else m = (cnt + BM - 1) / BM;
+            }
+            int tot;
+            const int ex = warp_exclusive_scan(m, &tot);
+            if (e < E) s_toff[e] = carry + ex;
+            carry += tot;
+        }
+        bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
+        if (lane == 0) {
+            s_toff[E] = carry;
+            *s_bad = bad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    if (*s_bad) {
+        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+        return;
+    }
+    const int NB = Ndim / MMA_N;
+    const int MB = (MODE == DW) ? Mdim / BM : 1;
+    const int total = (MODE == DW) ? E * MB * NB : s_toff[E] * NB;
+    if ((int)blockIdx.x >= total) return;
+    const int KF = K / 2 / BK;  // DX: slabs per operand pair
+
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(tfull + b), 1);
+            mbar_init(smem_u32(tempty + b), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmA0);
+        prefetch_map(&tmB0);
+        if (MODE == DX) {
+            prefetch_map(&tmA1);
+            prefetch_map(&tmB1);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s_tmem), TMEM_ALLOC);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
+            for (int kb = 0; kb < tl.nkb; ++kb) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(full + stage);
+                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                const uint32_t sb = sa + A_BYTES;
+                mbar_expect_tx(fb, STAGE_BYTES);
+                if (MODE == DH) {
+                    tma_load_2d(sa, &tmA0, fb, kb * BK, tl.row0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tma_load_3d(sb + j * BOX_BYTES, &tmB0, fb, tl.n0 + j * 64, kb * BK, tl.e);
+                } else if (MODE == DX) {
+                    const bool second = kb >= KF;
+                    const int kf = second ? kb - KF : kb;
+                    tma_load_2d(sa, second ? &tmA1 : &tmA0, fb, kf * BK, tl.row0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tma_load_3d(sb + j * BOX_BYTES, second ? &tmB1 : &tmB0, fb,
+                                    tl.n0 + j * 64, kf * BK, tl.e);
+                } else {
+                    const int r = tl.row0 + kb * BK;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        tma_load_2d(sa + i * BOX_BYTES, &tmA0, fb, tl.m0 + i * 64, r);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tma_load_2d(sb + j * BOX_BYTES, &tmB0, fb, tl.n0 + j * 64, r);
+                }
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued_mask >> s) & 1u) {
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                              DRAIN_LIMIT_NS);
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (whole warp;
+        // lane 0 issues, all lanes zero out-of-segment rows in DW mode)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int i = 0;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+            const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
+            for (int kb = 0; kb < tl.nkb; ++kb) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa_p = smem + stage * STAGE_BYTES;
+                const uint32_t sa = smem_u32(sa_p);
+                const uint32_t sb = sa + A_BYTES;
+                if (MODE == DW) {
+                    const int valid = tl.row_end - (tl.row0 + kb * BK);
+                    if (valid < BK) {
+                        // rows [valid, 64) of each of the 6 boxes belong to another
+                        // expert (or lie past R): zero them before the MMA reads them
+                        const int nrows = BK - valid;
+                        const int chunks = 6 * nrows * 8;  // 16-byte chunks
+                        for (int c = lane; c < chunks; c += 32) {
+                            const int box = c / (nrows * 8);
+                            const int rem = c - box * nrows * 8;
+                            const int row = valid + rem / 8;
+                            const int col = rem & 7;
+                            uint8_t* p = sa_p + box * BOX_BYTES + row * 128 + col * 16;
+                            *reinterpret_cast<uint4*>(p) = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = C::A_MN ? sw128_mn_desc(sa + ks * 2048, BOX_BYTES)
+                                                    : sw128_desc(sa) + 2 * ks;
+                        const uint64_t bd = sw128_mn_desc(sb + ks * 2048, BOX_BYTES);
+                        tc_mma<false>(dt, ad, bd, C::IDESC, (kb | ks) != 0);
+                    }
+                    tc_commit(smem_u32(empty + stage));
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok && lane == 0) tc_commit(smem_u32(tfull + buf));
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            tc_commit(smem_u32(drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+        __syncwarp();
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int r_in_tile = q * 32 + lane;
+        int i = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+            const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
+            if (MODE == DW) {
+                __nv_bfloat16* orow = out0 + (size_t)tl.e * Mdim * Ndim +
+                                      (size_t)(tl.m0 + r_in_tile) * Ndim + tl.n0;
+                const bool empty_k = tl.nkb == 0;
+#pragma unroll 1
+                for (int c = 0; c < MMA_N / 32; ++c) {
+                    float v[32];
+                    if (!empty_k) {
+                        uint32_t a[32];
+                        tmem_ld32(ta + c * 32, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                    }
+                    store32_bf16(orow + c * 32, v);
+                }
+            } else {
+                const int grow = tl.row0 + r_in_tile;
+                const bool valid = grow < tl.row_end;
+                const size_t rowoff = (size_t)(valid ? grow : 0) * ldo + tl.n0;
+#pragma unroll 1
+                for (int c = 0; c < MMA_N / 32; ++c) {
+                    uint32_t a[32];
+                    tmem_ld32(ta + c * 32, a);
+                    tmem_wait_ld();
+                    if (!valid) continue;
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                    if (MODE == DH) {
+                        float ga[32], ub[32], da[32], db[32];
+                        load32_bf16(saveA + rowoff + c * 32, ga);
+                        load32_bf16(saveB + rowoff + c * 32, ub);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float s = sigmoidf_(ga[j]);
+                            const float silu = ga[j] * s;
+                            const float dsilu = s * (1.0f + ga[j] * (1.0f - s));
+                            da[j] = v[j] * ub[j] * dsilu;
+                            db[j] = v[j] * silu;
+                        }
+                        store32_bf16(out0 + rowoff + c * 32, da);
+                        store32_bf16(out1 + rowoff + c * 32, db);
+                    } else {
+                        store32_bf16(out0 + rowoff + c * 32, v);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, TMEM_ALLOC);
+    }
+}
+
+template <int MODE>
+static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
+                  const CUtensorMap& b1, const int32_t* offsets, int64_t E, int64_t R, int64_t K,
+                  int64_t Mdim, int64_t Ndim, void* out0, void* out1, int64_t ldo,
+                  const void* saveA, const void* saveB, cudaStream_t st) {
+    auto kern = bwd_gemm_kernel<MODE>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t NB = Ndim / MMA_N;
+    const int64_t max_tiles = (MODE == DW) ? E * (Mdim / BM) * NB : (R / BM + E) * NB;
+    const int64_t sms = num_sms();
+    const int grid = (int)(max_tiles < sms ? max_tiles : sms);
+    if (grid <= 0) return MOE_OK;
+    kern<<<grid, THREADS, SMEM_BYTES, st>>>(
+        a0, a1, b0, b1, offsets, (int)E, (int)R, (int)K, (int)Mdim, (int)Ndim,
+        static_cast<__nv_bfloat16*>(out0), static_cast<__nv_bfloat16*>(out1), ldo,
+        static_cast<const __nv_bfloat16*>(saveA), static_cast<const __nv_bfloat16*>(saveB),
+        status_ptr());
+    return launch_status();
+}
+
+constexpr CUtensorMapDataType BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+}  // namespace bwd
+}  // namespace moe
+
+using namespace moe;
+using namespace moe::tc;
+
+extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void* B, const void* H,
+                                      const void* dYe, const void* W1, const void* W3,
+                                      const void* W2, int64_t w13_expert_stride,
+                                      int64_t w2_expert_stride, const int32_t* offsets, int64_t E,
+                                      int64_t R, int64_t d, int64_t F, int dtype, void* dA,
+                                      void* dB, void* dXe, void* dW1, void* dW3, void* dW2,
+                                      void* stream) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
+    if (dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (d % 256 != 0 || F % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if (R > INT32_MAX - 2 * bwd::BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+    const void* ptrs[] = {Xe, A, B, H, dYe, W1, W3, W2, dA, dB, dXe, dW1, dW3, dW2};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID;
+    if (!offsets) return MOE_ERR_INVALID;
+    if ((w13_expert_stride < F * d || w2_expert_stride < F * d) && E > 1) return MOE_ERR_INVALID;
+    if (w13_expert_stride % 8 != 0 || w2_expert_stride % 8 != 0) return MOE_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    int rc;
+    if (R > 0) {
+        // dH = dYe W2_e (+ pairwise SwiGLU backward) -> dA, dB
+        CUtensorMap mA, mW2;
+        if (!make_map_2d(&mA, dYe, bwd::BF16, 2, d, R, bwd::BM) ||
+            !make_map_3d(&mW2, W2, bwd::BF16, 2, F, d, E, w2_expert_stride, 64))
+            return MOE_ERR_CUDA;
+        rc = bwd::launch<bwd::DH>(mA, mA, mW2, mW2, offsets, E, R, d, 0, F, dA, dB, F, A, B, st);
+        if (rc != MOE_OK) return rc;
+        // dXe = dA W1_e + dB W3_e
+        CUtensorMap mdA, mdB, mW1, mW3;
+        if (!make_map_2d(&mdA, dA, bwd::BF16, 2, F, R, bwd::BM) ||
+            !make_map_2d(&mdB, dB, bwd::BF16, 2, F, R, bwd::BM) ||
+            !make_map_3d(&mW1, W1, bwd::BF16, 2, d, F, E, w13_expert_stride, 64) ||
+            !make_map_3d(&mW3, W3, bwd::BF16, 2, d, F, E, w13_expert_stride, 64))
+            return MOE_ERR_CUDA;
+        rc = bwd::launch<bwd::DX>(mdA, mdB, mW1, mW3, offsets, E, R, 2 * F, 0, d, dXe, nullptr, d,
+                                  nullptr, nullptr, st);
+        if (rc != MOE_OK) return rc;
+    }
+    // weight gradients (every expert's tile runs, so empty experts get zeros)
+    CUtensorMap gA, gB, gX, gY, gH;
+    const int64_t Rm = R > 0 ? R : 1;  // a map needs a non-empty extent; no rows are read when R == 0
+    if (!make_map_2d(&gA, dA, bwd::BF16, 2, F, Rm, 64) ||
+        !make_map_2d(&gB, dB, bwd::BF16, 2, F, Rm, 64) ||
+        !make_map_2d(&gX, Xe, bwd::BF16, 2, d, Rm, 64) ||
+        !make_map_2d(&gY, dYe, bwd::BF16, 2, d, Rm, 64) ||
+        !make_map_2d(&gH, H, bwd::BF16, 2, F, Rm, 64))
+        return MOE_ERR_CUDA;
+    rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, offsets, E, R, 0, F, d, dW1, nullptr, d, nullptr,
+                              nullptr, st);
+    if (rc != MOE_OK) return rc;
+    rc = bwd::launch<bwd::DW>(gB, gB, gX, gX, offsets, E, R, 0, F, d, dW3, nullptr, d, nullptr,
+                              nullptr, st);
+    if (rc != MOE_OK) return rc;
+    return bwd::launch<bwd::DW>(gY, gY, gH, gH, offsets, E, R, 0, d, F, dW2, nullptr, F, nullptr,
+                                nullptr, st);
+}

@@ -28,11 +28,9 @@
 // MOE_DEVERR_TIMEOUT and an abort flag, all roles leave their loops, the MMA
 // issuer drains its outstanding MMAs, the producer waits (again bounded) for
 // its copies in flight, and TMEM is released before the CTA exits.
-#include <cudaTypedefs.h>
-
 #include <type_traits>
 
-#include "common.cuh"
+#include "tc_sm100.cuh"
 
 namespace moe {
 namespace gg {
@@ -40,145 +38,7 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int STAGES = 4;
 constexpr int THREADS = 192;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
-constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // 0.1 s
-
-// ------------------------------------------------------------------ PTX
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for the phase with the given parity. Returns false if the wait
-// timed out (status bit + abort flag set here) or another role aborted.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int* status, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                set_status(status, MOE_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-template <bool TF32>
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accum) {
-    if constexpr (TF32) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-            : "memory");
-    } else {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-            : "memory");
-    }
-}
-// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets row
-// (lane base + i), columns taddr.col .. +31.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
-        "[%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
-           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor: fp32 accumulator, A/B format (bf16 = 1, tf32 = 2),
-// both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt, int M, int N) {
-    return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
-}
+using namespace tc;
 
 // ------------------------------------------------------------------ config
 
@@ -260,7 +120,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const int32_t* __restrict__ offsets, int E, int R, int K, int N,
-                        TIn* __restrict__ out, int64_t ldo, int* status) {
+                        TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
+                        TIn* __restrict__ save_b, int* status) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -450,6 +311,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         v[j] = silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j]));
+                    if (save_a != nullptr && valid) {
+                        // pre-activations kept for the backward pass
+                        const size_t off = (size_t)grow * ldo + tl.n0 + c * 32;
+                        Store32<TIn>::run(save_a + off, reinterpret_cast<const float*>(a));
+                        Store32<TIn>::run(save_b + off, reinterpret_cast<const float*>(b));
+                    }
                 } else {
                     tmem_wait_ld();
 #pragma unroll
@@ -474,52 +341,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------------------ host
 
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// 2-D map over a row-major [rows, cols] matrix; box = 128 bytes x box_rows.
-static bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
-                        uint64_t cols, uint64_t rows, uint32_t box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * (uint64_t)es};
-    cuuint32_t box[2] = {(cuuint32_t)(128 / es), box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3-D map over E matrices [rows, cols] spaced `estride` elements apart.
-static bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
-                        uint64_t cols, uint64_t rows, uint64_t E, uint64_t estride,
-                        uint32_t box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {cols, rows, E};
-    cuuint64_t strides[2] = {cols * (uint64_t)es, estride * (uint64_t)es};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / es), box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename TIn, bool SWIGLU, int MMA_N>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, void* out,
-                  int64_t ldo, cudaStream_t st) {
+                  int64_t ldo, cudaStream_t st, void* save_a = nullptr, void* save_b = nullptr) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N>;
     static bool attr_done[64] = {false};
@@ -536,7 +361,8 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
     kern<<<grid, THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K, (int)N,
-                                              static_cast<TIn*>(out), ldo, status_ptr());
+                                              static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a),
+                                              static_cast<TIn*>(save_b), status_ptr());
     return launch_status();
 }
 
@@ -555,10 +381,12 @@ static int check_common(const void* A, const void* B, const int32_t* offsets, in
 
 using namespace moe;
 
-extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
-                                   int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
-                                   int64_t R, int64_t d, int64_t F, int dtype, void* H,
-                                   void* stream) {
+extern "C" int moe_grouped_gate_up_save(const void* Xe, const void* W1, const void* W3,
+                                        int64_t w13_expert_stride, const int32_t* offsets,
+                                        int64_t E, int64_t R, int64_t d, int64_t F, int dtype,
+                                        void* H, void* A_out, void* B_out, void* stream) {
+    if ((A_out == nullptr) != (B_out == nullptr)) return MOE_ERR_INVALID;
+    if (A_out && (!aligned16(A_out) || !aligned16(B_out))) return MOE_ERR_INVALID;
     int rc = gg::check_common(Xe, W1, offsets, E, R, d, F, dtype);
     if (rc != MOE_OK) return rc;
     if (!W3 || !H || !aligned16(W3) || !aligned16(H)) return MOE_ERR_INVALID;
@@ -575,8 +403,17 @@ extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W
         return MOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     if (dtype == MOE_BF16)
-        return gg::launch<__nv_bfloat16, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st);
-    return gg::launch<float, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st);
+        return gg::launch<__nv_bfloat16, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st,
+                                                     A_out, B_out);
+    return gg::launch<float, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st, A_out, B_out);
+}
+
+extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
+                                   int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
+                                   int64_t R, int64_t d, int64_t F, int dtype, void* H,
+                                   void* stream) {
+    return moe_grouped_gate_up_save(Xe, W1, W3, w13_expert_stride, offsets, E, R, d, F, dtype, H,
+                                    nullptr, nullptr, stream);
 }
 
 extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,

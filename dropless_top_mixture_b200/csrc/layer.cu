@@ -104,10 +104,52 @@ extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
                        nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
                        c.route_ws, c.route_bytes, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, c.Xe, stream);
+    void* Xe = a->save_Xe ? a->save_Xe : c.Xe;
+    void* H = a->save_H ? a->save_H : c.H;
+    rc = moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, Xe, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_swiglu(c.Xe, a->W1, a->W3, a->W2, a->w13_expert_stride, a->w2_expert_stride,
-                            a->offsets, a->E, R, a->d, a->F, a->dtype, c.H, c.Ye, stream);
+    rc = moe_grouped_gate_up_save(Xe, a->W1, a->W3, a->w13_expert_stride, a->offsets, a->E, R,
+                                  a->d, a->F, a->dtype, H, a->save_A, a->save_B, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_grouped_down(H, a->W2, a->w2_expert_stride, a->offsets, a->E, R, a->d, a->F,
+                          a->dtype, c.Ye, stream);
     if (rc != MOE_OK) return rc;
     return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
+}
+
+extern "C" size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype) {
+    if (T < 0 || d <= 0 || F <= 0 || k <= 0) return 0;
+    const size_t es = dtype == MOE_F32 ? 4 : 2;
+    const size_t R = (size_t)T * (size_t)k;
+    return 2 * layer::a256(R * d * es) + 2 * layer::a256(R * F * es);
+}
+
+extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
+    if (!a) return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    const size_t need = moe_layer_bwd_workspace_size(a->T, a->d, a->F, a->k, a->dtype);
+    if (!a->workspace || a->workspace_bytes < need ||
+        (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return MOE_ERR_INVALID;
+    const int64_t R = a->T * a->k;
+    char* p = static_cast<char*>(a->workspace);
+    void* dYe = p;
+    p += layer::a256((size_t)R * a->d * 2);
+    void* dXe = p;
+    p += layer::a256((size_t)R * a->d * 2);
+    void* dA = p;
+    p += layer::a256((size_t)R * a->F * 2);
+    void* dB = p;
+    int rc;
+    if (a->T > 0) {
+        rc = moe_dispatch(a->dOut, a->slot, a->gate, a->T, a->d, a->k, a->dtype, dYe, stream);
+        if (rc != MOE_OK) return rc;
+    }
+    rc = moe_grouped_swiglu_bwd(a->Xe, a->A, a->B, a->H, dYe, a->W1, a->W3, a->W2,
+                                a->w13_expert_stride, a->w2_expert_stride, a->offsets, a->E, R,
+                                a->d, a->F, a->dtype, dA, dB, dXe, a->dW1, a->dW3, a->dW2, stream);
+    if (rc != MOE_OK) return rc;
+    if (a->T == 0) return MOE_OK;
+    return moe_combine(dXe, a->slot, nullptr, a->T, a->d, a->k, a->dtype, a->dx, stream);
 }

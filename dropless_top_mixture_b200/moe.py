@@ -57,6 +57,20 @@ class LayerArgs(ctypes.Structure):
         ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
         ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
         ("workspace", _p), ("workspace_bytes", _sz),
+        ("save_Xe", _p), ("save_H", _p), ("save_A", _p), ("save_B", _p),
+    ]
+
+
+class LayerBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i64), ("d", _i64), ("E", _i64), ("F", _i64),
+        ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("reserved1", ctypes.c_int32),
+        ("slot", _p), ("gate", _p), ("offsets", _p),
+        ("Xe", _p), ("A", _p), ("B", _p), ("H", _p), ("W1", _p), ("W3", _p), ("W2", _p),
+        ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
+        ("dOut", _p), ("dx", _p), ("dW1", _p), ("dW3", _p), ("dW2", _p),
+        ("workspace", _p), ("workspace_bytes", _sz),
     ]
 
 
@@ -71,11 +85,17 @@ _SIGS = {
     "moe_grouped_down": (_i32, [_p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_grouped_swiglu": (_i32, [_p, _p, _p, _p, _i64, _i64, _p, _i64, _i64, _i64, _i64, _i32,
                                   _p, _p, _p]),
+    "moe_grouped_gate_up_save": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p,
+                                        _p, _p, _p]),
+    "moe_grouped_swiglu_bwd": (_i32, [_p, _p, _p, _p, _p, _p, _p, _p, _i64, _i64, _p, _i64, _i64,
+                                      _i64, _i64, _i32, _p, _p, _p, _p, _p, _p, _p]),
     "moe_combine": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
     "mxfp8_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _p, _p, _p]),
     "mxfp8_dequantize": (_i32, [_p, _p, _i32, _i64, _i64, _p, _p]),
     "moe_layer_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32, _i32]),
     "moe_layer_fwd": (_i32, [ctypes.POINTER(LayerArgs), _p]),
+    "moe_layer_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32]),
+    "moe_layer_bwd": (_i32, [ctypes.POINTER(LayerBwdArgs), _p]),
     "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
     "moe_version": (ctypes.c_char_p, []),
 }
@@ -227,6 +247,51 @@ def moe_grouped_gate_up(Xe, W1, W3, offsets, H: Optional[torch.Tensor] = None) -
     return H
 
 
+def moe_grouped_gate_up_save(Xe, W1, W3, offsets, H=None, A=None, B=None):
+    _need(Xe, "Xe"); _need(offsets, "offsets")
+    E, F, d, s13 = _w13(W1, W3)
+    R = Xe.shape[0]
+    mk = lambda t: torch.empty((R, F), dtype=Xe.dtype, device=Xe.device) if t is None else t
+    H, A, B = mk(H), mk(A), mk(B)
+    rc = lib.moe_grouped_gate_up_save(_ptr(Xe), _ptr(W1), _ptr(W3), s13, _ptr(offsets), E, R, d,
+                                      F, _dtype_code(Xe.dtype), _ptr(H), _ptr(A), _ptr(B),
+                                      _stream(Xe))
+    _check("moe_grouped_gate_up_save", rc)
+    return H, A, B
+
+
+@dataclass
+class ExpertGrads:
+    dXe: torch.Tensor
+    dW1: torch.Tensor
+    dW3: torch.Tensor
+    dW2: torch.Tensor
+    dA: torch.Tensor
+    dB: torch.Tensor
+
+
+def moe_grouped_swiglu_bwd(Xe, A, B, H, dYe, W1, W3, W2, offsets,
+                           out: Optional[ExpertGrads] = None) -> ExpertGrads:
+    for t, n in ((Xe, "Xe"), (A, "A"), (B, "B"), (H, "H"), (dYe, "dYe"), (offsets, "offsets")):
+        _need(t, n)
+    E, F, d, s13 = _w13(W1, W3)
+    R = Xe.shape[0]
+    dev, dt = Xe.device, Xe.dtype
+    if out is None:
+        out = ExpertGrads(dXe=torch.empty((R, d), dtype=dt, device=dev),
+                          dW1=torch.empty((E, F, d), dtype=dt, device=dev),
+                          dW3=torch.empty((E, F, d), dtype=dt, device=dev),
+                          dW2=torch.empty((E, d, F), dtype=dt, device=dev),
+                          dA=torch.empty((R, F), dtype=dt, device=dev),
+                          dB=torch.empty((R, F), dtype=dt, device=dev))
+    rc = lib.moe_grouped_swiglu_bwd(_ptr(Xe), _ptr(A), _ptr(B), _ptr(H), _ptr(dYe), _ptr(W1),
+                                    _ptr(W3), _ptr(W2), s13, W2.stride(0), _ptr(offsets), E, R, d,
+                                    F, _dtype_code(dt), _ptr(out.dA), _ptr(out.dB), _ptr(out.dXe),
+                                    _ptr(out.dW1), _ptr(out.dW3), _ptr(out.dW2), _stream(Xe))
+    _check("moe_grouped_swiglu_bwd", rc)
+    return out
+
+
 def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need(H, "H"); _need(W2, "W2"); _need(offsets, "offsets")
     E, d, F = W2.shape
@@ -305,10 +370,14 @@ class LayerOut:
     offsets: torch.Tensor
     slot: torch.Tensor
     workspace: torch.Tensor
+    Xe: Optional[torch.Tensor] = None   # rows kept for the backward (save=True)
+    H: Optional[torch.Tensor] = None
+    A: Optional[torch.Tensor] = None
+    B: Optional[torch.Tensor] = None
 
 
 def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool = False,
-                  out: Optional[LayerOut] = None) -> LayerOut:
+                  out: Optional[LayerOut] = None, save: bool = False) -> LayerOut:
     _need(x, "x")
     T, d = x.shape
     E, F, _, s13 = _w13(W1, W3)
@@ -321,14 +390,55 @@ def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool =
                        gate=torch.empty((T, k), dtype=torch.float32, device=dev),
                        counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
                        slot=torch.empty((T, k), **i32), workspace=ws)
+        if save:
+            R = T * k
+            out.Xe = torch.empty((R, d), dtype=x.dtype, device=dev)
+            out.H, out.A, out.B = (torch.empty((R, F), dtype=x.dtype, device=dev) for _ in range(3))
     a = LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(x.dtype), renorm=int(renorm),
                   reserved0=0, x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1=_ptr(W1),
                   W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13, w2_expert_stride=W2.stride(0),
                   out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
                   counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
-                  workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+                  workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel(),
+                  save_Xe=_ptr(out.Xe), save_H=_ptr(out.H), save_A=_ptr(out.A), save_B=_ptr(out.B))
     rc = lib.moe_layer_fwd(ctypes.byref(a), _stream(x))
     _check("moe_layer_fwd", rc)
+    return out
+
+
+@dataclass
+class LayerGrads:
+    dx: torch.Tensor
+    dW1: torch.Tensor
+    dW3: torch.Tensor
+    dW2: torch.Tensor
+    workspace: torch.Tensor
+
+
+def moe_layer_bwd(fwd: LayerOut, dOut, k: int, W1, W3, W2,
+                  out: Optional[LayerGrads] = None) -> LayerGrads:
+    """Backward of moe_layer_fwd(save=True) with the gates held constant."""
+    _need(dOut, "dOut")
+    if fwd.Xe is None:
+        raise ValueError("moe_layer_bwd needs the forward run with save=True")
+    T, d = dOut.shape
+    E, F, _, s13 = _w13(W1, W3)
+    dev, dt = dOut.device, dOut.dtype
+    if out is None:
+        ws = _alloc_ws(lib.moe_layer_bwd_workspace_size(T, d, F, k, _dtype_code(dt)), dev)
+        out = LayerGrads(dx=torch.empty((T, d), dtype=dt, device=dev),
+                         dW1=torch.empty((E, F, d), dtype=dt, device=dev),
+                         dW3=torch.empty((E, F, d), dtype=dt, device=dev),
+                         dW2=torch.empty((E, d, F), dtype=dt, device=dev), workspace=ws)
+    a = LayerBwdArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(dt), reserved0=0, reserved1=0,
+                     slot=_ptr(fwd.slot), gate=_ptr(fwd.gate), offsets=_ptr(fwd.offsets),
+                     Xe=_ptr(fwd.Xe), A=_ptr(fwd.A), B=_ptr(fwd.B), H=_ptr(fwd.H), W1=_ptr(W1),
+                     W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13,
+                     w2_expert_stride=W2.stride(0), dOut=_ptr(dOut), dx=_ptr(out.dx),
+                     dW1=_ptr(out.dW1), dW3=_ptr(out.dW3), dW2=_ptr(out.dW2),
+                     workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    rc = lib.moe_layer_bwd(ctypes.byref(a), _stream(dOut))
+    _check("moe_layer_bwd", rc)
     return out
 
 

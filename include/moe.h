@@ -188,6 +188,38 @@ MOE_API int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, c
                                int64_t w13_expert_stride, int64_t w2_expert_stride,
                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
                                int64_t F, int dtype, void* H, void* Ye, void* stream);
+/* moe_grouped_gate_up with the pre-activations kept for the backward pass:
+ * A_out[r] = Xe[r]·W1_eᵀ and B_out[r] = Xe[r]·W3_eᵀ ([R,F], layer dtype),
+ * written by the same epilogue that writes H. Both NULL = moe_grouped_gate_up. */
+MOE_API int moe_grouped_gate_up_save(const void* Xe, const void* W1, const void* W3,
+                                     int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
+                                     int64_t R, int64_t d, int64_t F, int dtype, void* H,
+                                     void* A_out, void* B_out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_grouped_swiglu_bwd — backward of the grouped SwiGLU FFN.
+ *
+ * ["OLMo-core 3 发布：主攻混合专家训练与导出校验", 主要功能: pairwise SwiGLU
+ * backward and bf16 weight gradients.] Given the forward's saved rows Xe,
+ * A = Xe·W1ᵀ, B = Xe·W3ᵀ, H = silu(A)*B and the upstream rows dYe [R,d]
+ * (moe_dispatch of dOut with the gates), per expert e and its rows:
+ *   dH  = dYe·W2_e;  dA = dH*B*silu'(A);  dB = dH*silu(A)   (silu'(a) =
+ *         s(1 + a(1-s)), s = sigmoid(a); fused into the dH GEMM epilogue)
+ *   dXe = dA·W1_e + dB·W3_e
+ *   dW1_e = dAᵀ·Xe_e,  dW3_e = dBᵀ·Xe_e,  dW2_e = dYeᵀ·H_e
+ * tcgen05 bf16 MMA, fp32 accumulation, every output stored in bf16.
+ *   dA, dB [R,F] (outputs, also used as workspace), dXe [R,d];
+ *   dW1, dW3 [E,F,d] and dW2 [E,d,F], contiguous; an expert with no rows
+ *   gets zero gradients. Weights as in moe_grouped_gate_up/down.
+ * Limits: MOE_BF16 only; d % 256 == 0, F % 256 == 0, E <= 512. Router and
+ * gate gradients are not computed here.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void* B, const void* H,
+                                   const void* dYe, const void* W1, const void* W3,
+                                   const void* W2, int64_t w13_expert_stride,
+                                   int64_t w2_expert_stride, const int32_t* offsets, int64_t E,
+                                   int64_t R, int64_t d, int64_t F, int dtype, void* dA, void* dB,
+                                   void* dXe, void* dW1, void* dW3, void* dW2, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine — gate-weighted combine back to token order.
@@ -246,11 +278,53 @@ typedef struct moe_layer_args {
     /* scratch (device): Xe [R,d], H [R,F], Ye [R,d] and the route workspace */
     void* workspace;
     size_t workspace_bytes;
+    /* optional (device, NULL = not kept): rows kept for moe_layer_bwd. When
+     * save_Xe / save_H are given they replace the workspace copies; save_A and
+     * save_B (given together) receive the gate/up pre-activations. */
+    void* save_Xe;          /* [R,d] */
+    void* save_H;           /* [R,F] */
+    void* save_A;           /* [R,F] */
+    void* save_B;           /* [R,F] */
 } moe_layer_args;
 
 MOE_API size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
                                         int dtype, int logits_given);
 MOE_API int moe_layer_fwd(const moe_layer_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_layer_bwd — backward of moe_layer_fwd with the gates held constant:
+ *   dYe[slot[t,j]] = bf16(gate[t,j] * dOut[t])       (moe_dispatch, scaled)
+ *   moe_grouped_swiglu_bwd                          -> dXe, dW1, dW3, dW2
+ *   dx[t] = sum_j dXe[slot[t,j]]                    (moe_combine, unit gates)
+ * Needs the forward's routing (slot, gate, offsets) and saved rows (Xe, A,
+ * B, H: moe_layer_args.save_*). Workspace: moe_layer_bwd_workspace_size
+ * (dYe, dA, dB, dXe). bf16 only, same limits as moe_grouped_swiglu_bwd.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_layer_bwd_args {
+    int64_t T, d, E, F;
+    int32_t k, dtype, reserved0, reserved1;
+    const int32_t* slot;    /* [T,k] from the forward                          */
+    const float* gate;      /* [T,k]                                          */
+    const int32_t* offsets; /* [E+1]                                          */
+    const void* Xe;         /* [R,d] saved forward rows                       */
+    const void* A;          /* [R,F]                                          */
+    const void* B;          /* [R,F]                                          */
+    const void* H;          /* [R,F]                                          */
+    const void* W1;
+    const void* W3;
+    const void* W2;
+    int64_t w13_expert_stride, w2_expert_stride;
+    const void* dOut;       /* [T,d] upstream gradient                        */
+    void* dx;               /* [T,d]                                          */
+    void* dW1;              /* [E,F,d]                                        */
+    void* dW3;              /* [E,F,d]                                        */
+    void* dW2;              /* [E,d,F]                                        */
+    void* workspace;
+    size_t workspace_bytes;
+} moe_layer_bwd_args;
+
+MOE_API size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype);
+MOE_API int moe_layer_bwd(const moe_layer_bwd_args* args, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_get_status — read (and optionally clear) the device status word of the

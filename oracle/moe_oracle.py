@@ -519,6 +519,40 @@ def moe_layer_bwd(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W2,
     return dict(dx=dx, dW1=dW1, dW3=dW3, dW2=dW2, dYe=dYe, dXe=dXe, idx=idx, gate=gate, **meta)
 
 
+def moe_layer_bwd_sampled(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W2,
+                          logits: np.ndarray, tokens, experts) -> Dict[str, np.ndarray]:
+    """The same gradients as moe_layer_bwd, restricted to a sample: dx for the
+    given tokens (each (t, j) row's dXe from the per-row formula) and dW1,
+    dW3, dW2 for the given experts (from all of that expert's rows). For
+    full-size workloads whose whole backward would take too long on the CPU."""
+    E = W1.shape[0]
+    idx, gate, _ = route(logits, k)
+    meta = routing_metadata(idx, E)
+    tokens = np.asarray(tokens)
+    dx = np.zeros((len(tokens), x.shape[1]))
+    for i, t in enumerate(tokens):
+        xt = to64(x[int(t)])
+        dot = to64(dOut[int(t)])
+        for j in range(k):
+            e = int(idx[t, j])
+            w1, w3, w2 = to64(W1[e]), to64(W3[e]), to64(W2[e])
+            a, b = w1 @ xt, w3 @ xt
+            dh = w2.T @ (gate[t, j] * dot)
+            dx[i] += w1.T @ (dh * b * dsilu(a)) + w3.T @ (dh * silu(a))
+    dW = {}
+    for e in experts:
+        e = int(e)
+        toks, js = np.nonzero(idx == e)   # token-major order, as in the expert buffer
+        X = to64(x[torch.as_tensor(toks, dtype=torch.long)]) if len(toks) else np.zeros((0, x.shape[1]))
+        dY = (gate[toks, js][:, None] * to64(dOut[torch.as_tensor(toks, dtype=torch.long)])
+              if len(toks) else np.zeros((0, x.shape[1])))
+        off = np.array([0, len(toks)])
+        _, g1, g3, g2 = expert_ffn_bwd(X, off, to64(W1[e:e + 1]), to64(W3[e:e + 1]),
+                                       to64(W2[e:e + 1]), dY)
+        dW[e] = (g1[0], g3[0], g2[0])
+    return dict(dx=dx, dW=dW, idx=idx, gate=gate, tokens=tokens, **meta)
+
+
 # --------------------------------------------------------------------------
 # error measures used by the parity tests
 # --------------------------------------------------------------------------

@@ -380,3 +380,15 @@ def test_backward_finite_differences():
         Wm[e, a, b] -= h
         fd = (loss(x, Wp, W3, W2) - loss(x, Wm, W3, W2)) / (2 * h)
         assert math.isclose(fd, r["dW1"][e, a, b], rel_tol=1e-6, abs_tol=1e-8)
+
+
+def test_sampled_backward_matches_full_backward():
+    x, W1, W3, W2, lg, dOut = _tiny_problem(33, T=20, d=6, F=8, E=5, k=2)
+    full = O.moe_layer_bwd(x, dOut, 2, W1, W3, W2, lg)
+    toks = np.array([0, 7, 19])
+    smp = O.moe_layer_bwd_sampled(x, dOut, 2, W1, W3, W2, lg, toks, [0, 2, 4])
+    assert np.allclose(smp["dx"], full["dx"][toks], rtol=1e-12, atol=1e-13)
+    for e in (0, 2, 4):
+        for n, g in zip(("dW1", "dW3", "dW2"), smp["dW"][e]):
+            assert np.allclose(g, full[n][e], rtol=1e-12, atol=1e-13)
+    assert np.all(smp["dW"][4][0] == 0)  # expert 4 has no rows
