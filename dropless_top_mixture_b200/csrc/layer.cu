@@ -153,3 +153,73 @@ extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
     if (a->T == 0) return MOE_OK;
     return moe_combine(dXe, a->slot, nullptr, a->T, a->d, a->k, a->dtype, a->dx, stream);
 }
+
+namespace moe {
+namespace layer {
+
+struct CarveMx {
+    uint8_t* Xq;
+    uint8_t* Xs;
+    uint8_t* Hq;
+    uint8_t* Hs;
+    void* Ye;
+    void* route_ws;
+    size_t route_bytes;
+    size_t total;
+};
+
+inline CarveMx carve_mx(void* base, int64_t T, int64_t d, int64_t E, int64_t F, int k,
+                        int logits_given) {
+    const size_t R = (size_t)T * (size_t)k;
+    char* p = static_cast<char*>(base);
+    CarveMx c;
+    size_t off = 0;
+    c.Xq = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(R * d);
+    c.Xs = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(R * d / 32);
+    c.Hq = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(R * F);
+    c.Hs = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(R * F / 32);
+    c.Ye = p + off;
+    off += a256(R * d * 2);
+    c.route_ws = p + off;
+    c.route_bytes = moe_route_workspace_size(T, E, logits_given ? 0 : 1);
+    off += a256(c.route_bytes);
+    c.total = off;
+    return c;
+}
+
+}  // namespace layer
+}  // namespace moe
+
+extern "C" size_t moe_layer_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
+                                                 int logits_given) {
+    if (T < 0 || d <= 0 || E <= 0 || F <= 0 || k <= 0) return 0;
+    return layer::carve_mx(nullptr, T, d, E, F, k, logits_given).total;
+}
+
+extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) {
+    if (!a) return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
+    if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return MOE_ERR_INVALID;
+    const int logits_given = a->logits != nullptr;
+    layer::CarveMx c = layer::carve_mx(a->workspace, a->T, a->d, a->E, a->F, a->k, logits_given);
+    if (a->workspace_bytes < c.total) return MOE_ERR_INVALID;
+    int rc = moe_route(a->logits, a->x, a->Wr, MOE_BF16, a->T, a->d, a->E, a->k, a->renorm,
+                       nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
+                       c.route_ws, c.route_bytes, stream);
+    if (rc != MOE_OK || a->T == 0) return rc;
+    const int64_t R = a->T * a->k;
+    rc = moe_dispatch_mxfp8(a->x, a->slot, a->T, a->d, a->k, c.Xq, c.Xs, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xs, a->W1q, a->W1s, a->W3q, a->W3s, a->w13_expert_stride,
+                                   a->offsets, a->E, R, a->d, a->F, c.Hq, c.Hs, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_grouped_down_mxfp8(c.Hq, c.Hs, a->W2q, a->W2s, a->w2_expert_stride, a->offsets, a->E, R,
+                                a->d, a->F, c.Ye, stream);
+    if (rc != MOE_OK) return rc;
+    return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, MOE_BF16, a->out, stream);
+}

@@ -10,36 +10,15 @@
 //
 // One thread per 32-element block: it reads the block (64 or 128 bytes),
 // finds amax, derives the scale and writes 32 code bytes plus one scale.
-#include <cuda_fp8.h>
-
-#include "common.cuh"
+#include "mx_common.cuh"
 
 namespace moe {
 namespace mx {
 
 constexpr int THREADS = 256;
 
-// Smallest e with 2^e >= s for a positive finite fp32 s, clamped to
-// [-127, 127]. Works from the bit pattern so no rounding is involved.
-__device__ __forceinline__ int pow2_ceil_exp(float s) {
-    const uint32_t u = __float_as_uint(s);
-    const int be = (int)((u >> 23) & 0xFF);
-    const uint32_t man = u & 0x7FFFFFu;
-    int e;
-    if (be == 0) {
-        // subnormal: s = man * 2^-149, man in [1, 2^23)
-        const int msb = 31 - __clz((int)man);
-        e = msb - 149 + ((man & (man - 1)) ? 1 : 0);
-    } else {
-        e = be - 127 + (man ? 1 : 0);
-    }
-    return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
-__device__ __forceinline__ float exp2_exact(int e) {
-    // 2^e for e in [-127, 127] as an fp32 bit pattern (2^-127 is subnormal)
-    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
-}
+using mxc::exp2_exact;
+using mxc::pow2_ceil_exp;
 
 template <int DT>
 __device__ __forceinline__ void load32(const void* in, int64_t blk, float* v) {

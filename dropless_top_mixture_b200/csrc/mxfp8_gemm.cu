@@ -1,0 +1,504 @@
+// MXFP8 variant of the layer: dispatch that quantises each token row once,
+// and the grouped SwiGLU FFN on block-scaled FP8 tensor cores (sm_100a).
+//
+// "olmoforge" README, capability table and "MXFP8 分块量化": 32-value blocks
+// share one scale, E4M3 payload; the Olmo-core 3 news article (xxqk.cn),
+// "三招拆分、三项优化、一个精度开关": MXFP8 as the low-precision switch, its
+// gain coming from the FFN and the expert data movement. Operands here:
+//   x  -> Xq [R,d] e4m3 + UE8M0 scales [R,d/32]   (moe_dispatch_mxfp8)
+//   W1, W3 [E,F,d], W2 [E,d,F] quantised offline along their K dimension
+//   H  -> Hq [R,F] e4m3 + scales [R,F/32], quantised from the fp32 SwiGLU
+//         output in the gate/up epilogue
+//   Ye = Hq W2q (block-scaled), fp32 accumulate, bf16 out; combine as in bf16.
+//
+// Kernel: tcgen05.mma kind::mxf8f6f4.block_scale, M = 128, N = 128, K = 32 per
+// instruction, 128-byte K slabs staged by TMA with the same 128-byte swizzle
+// as the bf16 kernels. Per slab every row carries 4 UE8M0 scales (one 32-bit
+// word); the producer warp gathers the 128 A words and 128 B words into the
+// 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4 copies into TMEM
+// (lane m%32 of every sub-partition, column m/32, byte = K block), and the
+// MMA selects the byte with the scale-factor id of each of the 4 MMAs.
+// Accumulators: two 128-column TMEM buffers; the scale factors follow them.
+#include "mx_common.cuh"
+#include "tc_sm100.cuh"
+
+namespace moe {
+namespace mxg {
+
+using namespace tc;
+
+constexpr int BM = 128;
+constexpr int MMA_N = 128;
+constexpr int BK = 128;  // e4m3 elements per 128-byte slab
+constexpr int STAGES = 6;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * 128;
+constexpr int B_BYTES = MMA_N * 128;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SF_STAGE_BYTES = 1024;  // 512 B of A scale words + 512 B of B scale words
+constexpr int TMEM_ALLOC = 512;
+constexpr int SFA_COL = 2 * MMA_N;    // 256
+constexpr int SFB_COL = SFA_COL + 4;  // 260
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + META_BYTES;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// Block-scaled instruction descriptor: E4M3 A and B (format 0), K-major,
+// N >> 3 at bit 17, UE8M0 scales (bit 23), M >> 4 at bit 24, scale-factor
+// ids of A (bits 29-30) and B (bits 4-5) select the byte of the scale word.
+__host__ __device__ constexpr uint32_t mx_idesc(int sf_id) {
+    return ((uint32_t)sf_id << 4) | ((uint32_t)(MMA_N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(BM >> 4) << 24) | ((uint32_t)sf_id << 29);
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// 32 rows x 16 bytes, contiguous, no swizzle: 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(128 >> 4) << 32) |
+           ((uint64_t)1 << 46);
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+struct Tile {
+    int e, row0, row_end, n0;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, int NB, int E, int out_n, const int* s_toff,
+                                            const int* s_off) {
+    const int q = t / NB;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_toff[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    Tile tl;
+    tl.e = lo;
+    const int Me = s_toff[lo + 1] - s_toff[lo];
+    const int l = t - s_toff[lo] * NB;
+    const int nb = l / Me, m = l - nb * Me;
+    tl.row0 = s_off[lo] + m * BM;
+    tl.row_end = s_off[lo + 1];
+    tl.n0 = nb * out_n;
+    return tl;
+}
+
+__device__ __forceinline__ uint32_t ld_word(const uint8_t* p) {
+    return __ldg(reinterpret_cast<const uint32_t*>(p));
+}
+
+// SWIGLU: B tile = 64 rows of W1 then 64 rows of W3 at the same n0; the
+// epilogue writes Hq/Hs (64 output columns per tile). Otherwise B = 128 rows
+// of W2 and the epilogue writes bf16 Ye (128 columns).
+template <bool SWIGLU>
+__global__ void __launch_bounds__(THREADS, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, const uint8_t* __restrict__ sfA,
+                   const uint8_t* __restrict__ sfB0, const uint8_t* __restrict__ sfB1,
+                   int64_t sfb_expert_stride, const int32_t* __restrict__ offsets, int E, int R,
+                   int K, int N, uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_s,
+                   __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status) {
+    constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sf_smem = smem + STAGES * STAGE_BYTES;
+    uint8_t* meta = sf_smem + STAGES * SF_STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int m = 0;
+            if (e < E) {
+                const int cnt = s_off[e + 1] - s_off[e];
+                if (cnt < 0) bad = true;
+                else m = (cnt + BM - 1) / BM;
+            }
+            int tot;
+            const int ex = warp_exclusive_scan(m, &tot);
+            if (e < E) s_toff[e] = carry + ex;
+            carry += tot;
+        }
+        bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
+        if (lane == 0) {
+            s_toff[E] = carry;
+            *s_bad = bad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    if (*s_bad) {
+        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+        return;
+    }
+    const int NB = N / OUT_N;
+    const int total = s_toff[E] * NB;
+    if ((int)blockIdx.x >= total) return;
+    const int KB = K / BK;
+    const int sf_row = K / 32;  // scale bytes per row
+
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 2);  // TMA bytes + the scale words
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(tfull + b), 1);
+            mbar_init(smem_u32(tempty + b), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmA);
+        prefetch_map(&tmB0);
+        if (SWIGLU) prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s_tmem), TMEM_ALLOC);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer warp:
+        // lane 0 issues the TMA copies, all lanes gather the scale words
+        int stage = 0;
+        uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(full + stage);
+                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                const uint32_t sb = sa + A_BYTES;
+                if (lane == 0) {
+                    mbar_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, fb, kb * BK, tl.row0);
+                    if (SWIGLU) {
+                        tma_load_3d(sb, &tmB0, fb, kb * BK, tl.n0, tl.e);
+                        tma_load_3d(sb + B_BYTES / 2, &tmB1, fb, kb * BK, tl.n0, tl.e);
+                    } else {
+                        tma_load_3d(sb, &tmB0, fb, kb * BK, tl.n0, tl.e);
+                    }
+                }
+                uint32_t* sfw = reinterpret_cast<uint32_t*>(sf_smem + stage * SF_STAGE_BYTES);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int m = lane + 32 * j;  // A row within the tile
+                    const int grow = tl.row0 + m;
+                    const uint32_t wa =
+                        grow < R ? ld_word(sfA + (size_t)grow * sf_row + 4 * kb) : 0u;
+                    sfw[lane * 4 + j] = wa;
+                    const uint8_t* bsrc;
+                    if (SWIGLU) {
+                        bsrc = (m < 64 ? sfB0 + (size_t)(tl.n0 + m) * sf_row
+                                       : sfB1 + (size_t)(tl.n0 + m - 64) * sf_row);
+                    } else {
+                        bsrc = sfB0 + (size_t)(tl.n0 + m) * sf_row;
+                    }
+                    sfw[128 + lane * 4 + j] = ld_word(bsrc + (size_t)tl.e * sfb_expert_stride + 4 * kb);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fb);
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued_mask >> s) & 1u) {
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                              DRAIN_LIMIT_NS);
+                }
+        }
+        __syncwarp();
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int i = 0;
+        const uint32_t sfa_t = tmem_base + SFA_COL;
+        const uint32_t sfb_t = tmem_base + SFB_COL;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
+                tmem_cp_sf(sfa_t, sf_desc(sfs));
+                tmem_cp_sf(sfb_t, sf_desc(sfs + 512));
+                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                const uint64_t ad = sw128_desc(sa);
+                const uint64_t bd = sw128_desc(sa + A_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_mx(dt, ad + 2 * ks, bd + 2 * ks, mx_idesc(ks), sfa_t | ((uint32_t)ks << 30),
+                           sfb_t | ((uint32_t)ks << 30), (kb | ks) != 0);
+                tc_commit(smem_u32(empty + stage));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit(smem_u32(tfull + buf));
+        }
+        if (!ok) {
+            tc_commit(smem_u32(drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int r_in_tile = q * 32 + lane;
+        int i = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+            const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
+            const int grow = tl.row0 + r_in_tile;
+            const bool valid = grow < tl.row_end;
+            const size_t grow_c = (size_t)(valid ? grow : 0);
+#pragma unroll 1
+            for (int c = 0; c < OUT_N / 32; ++c) {
+                uint32_t a[32];
+                float v[32];
+                tmem_ld32(ta + c * 32, a);
+                if constexpr (SWIGLU) {
+                    uint32_t b[32];
+                    tmem_ld32(ta + OUT_N + c * 32, b);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float g = __uint_as_float(a[j]);
+                        v[j] = g / (1.0f + __expf(-g)) * __uint_as_float(b[j]);
+                    }
+                    if (valid) {
+                        float sc;
+                        const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
+                        uint32_t w[8];
+                        mxc::encode32(v, sc, w);
+                        uint4* dq = reinterpret_cast<uint4*>(out_q + grow_c * ldo + tl.n0 + c * 32);
+                        dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        out_s[grow_c * (ldo / 32) + (tl.n0 + c * 32) / 32] = sbyte;
+                    }
+                } else {
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                        uint4* d = reinterpret_cast<uint4*>(out_bf16 + grow_c * ldo + tl.n0 + c * 32);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) d[u] = pack8(v + 8 * u);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, TMEM_ALLOC);
+    }
+}
+
+// Quantise each token row once (blocks of 32 along d, UE8M0 scales) and
+// write the codes and scales to its k slots. One thread per 32-value block.
+__global__ void __launch_bounds__(256) mx_dispatch_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const int32_t* __restrict__ slot, int T,
+                                                          int d, int k, int64_t R,
+                                                          uint8_t* __restrict__ Xq,
+                                                          uint8_t* __restrict__ Xs, int* status) {
+    const int bpr = d / 32;
+    const int64_t n = (int64_t)T * bpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / bpr);
+        const int b = (int)(i - (int64_t)t * bpr);
+        float v[32];
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d + b * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) unpack8(__ldcs(src + u), v + 8 * u);
+        float sc;
+        const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
+        uint32_t w[8];
+        mxc::encode32(v, sc, w);
+        const uint4 c0 = make_uint4(w[0], w[1], w[2], w[3]);
+        const uint4 c1 = make_uint4(w[4], w[5], w[6], w[7]);
+        for (int j = 0; j < k; ++j) {
+            const int s = slot[(size_t)t * k + j];
+            if (s < 0 || s >= R) {
+                set_status(status, MOE_DEVERR_BAD_INDEX);
+                continue;
+            }
+            uint4* dq = reinterpret_cast<uint4*>(Xq + (size_t)s * d + b * 32);
+            dq[0] = c0;
+            dq[1] = c1;
+            Xs[(size_t)s * bpr + b] = sbyte;
+        }
+    }
+}
+
+template <bool SWIGLU>
+static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                  const uint8_t* sfA, const uint8_t* sfB0, const uint8_t* sfB1, int64_t sfb_stride,
+                  const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, uint8_t* oq,
+                  uint8_t* os, __nv_bfloat16* ob, int64_t ldo, cudaStream_t st) {
+    auto kern = mx_gemm_kernel<SWIGLU>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int out_n = SWIGLU ? MMA_N / 2 : MMA_N;
+    const int64_t max_tiles = (R / BM + E) * (N / out_n);
+    const int64_t sms = num_sms();
+    const int grid = (int)(max_tiles < sms ? max_tiles : sms);
+    if (grid <= 0) return MOE_OK;
+    kern<<<grid, THREADS, SMEM_BYTES, st>>>(a, b0, b1, sfA, sfB0, sfB1, sfb_stride, offsets, (int)E,
+                                           (int)R, (int)K, (int)N, oq, os, ob, ldo, status_ptr());
+    return launch_status();
+}
+
+constexpr CUtensorMapDataType U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+
+}  // namespace mxg
+}  // namespace moe
+
+using namespace moe;
+using namespace moe::tc;
+
+extern "C" int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T, int64_t d, int k,
+                                  uint8_t* Xq, uint8_t* Xs, void* stream) {
+    if (T < 0 || d <= 0 || d % 32 != 0 || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID;
+    if (T == 0) return MOE_OK;
+    if (!x || !slot || !Xq || !Xs || !aligned16(x) || !aligned16(Xq)) return MOE_ERR_INVALID;
+    if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    const int64_t n = T * (d / 32);
+    int64_t g = (n + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (g > cap) g = cap;
+    mxg::mx_dispatch_kernel<<<(int)g, 256, 0, as_stream(stream)>>>(
+        static_cast<const __nv_bfloat16*>(x), slot, (int)T, (int)d, k, T * k, Xq, Xs, status_ptr());
+    return launch_status();
+}
+
+static int mx_check(const void* A, const void* As, const void* B, const void* Bs,
+                    const int32_t* offsets, int64_t E, int64_t R, int64_t d, int64_t F) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
+    if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (R > INT32_MAX - 2 * mxg::BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+    if (!offsets || !A || !As || !B || !Bs) return MOE_ERR_INVALID;
+    if (!aligned16(A) || !aligned16(B)) return MOE_ERR_INVALID;
+    // scale words are read as aligned 32-bit loads
+    if ((reinterpret_cast<uintptr_t>(As) & 3u) || (reinterpret_cast<uintptr_t>(Bs) & 3u))
+        return MOE_ERR_INVALID;
+    return MOE_OK;
+}
+
+extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
+                                         const uint8_t* W1s, const uint8_t* W3q,
+                                         const uint8_t* W3s, int64_t w13_expert_stride,
+                                         const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                         int64_t F, uint8_t* Hq, uint8_t* Hs, void* stream) {
+    int rc = mx_check(Xq, Xs, W1q, W1s, offsets, E, R, d, F);
+    if (rc != MOE_OK) return rc;
+    if (!W3q || !W3s || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq)) return MOE_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(W3s) & 3u)) return MOE_ERR_INVALID;
+    if ((w13_expert_stride < F * d && E > 1) || w13_expert_stride % 128 != 0) return MOE_ERR_INVALID;
+    if (R == 0) return MOE_OK;
+    CUtensorMap a, b0, b1;
+    if (!make_map_2d(&a, Xq, mxg::U8, 1, d, R, mxg::BM) ||
+        !make_map_3d(&b0, W1q, mxg::U8, 1, d, F, E, w13_expert_stride, 64) ||
+        !make_map_3d(&b1, W3q, mxg::U8, 1, d, F, E, w13_expert_stride, 64))
+        return MOE_ERR_CUDA;
+    return mxg::launch<true>(a, b0, b1, Xs, W1s, W3s, w13_expert_stride / 32, offsets, E, R, d, F,
+                             Hq, Hs, nullptr, F, as_stream(stream));
+}
+
+extern "C" int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const uint8_t* W2q,
+                                      const uint8_t* W2s, int64_t w2_expert_stride,
+                                      const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                      int64_t F, void* Ye, void* stream) {
+    int rc = mx_check(Hq, Hs, W2q, W2s, offsets, E, R, d, F);
+    if (rc != MOE_OK) return rc;
+    if (!Ye || !aligned16(Ye)) return MOE_ERR_INVALID;
+    if ((w2_expert_stride < F * d && E > 1) || w2_expert_stride % 128 != 0) return MOE_ERR_INVALID;
+    if (R == 0) return MOE_OK;
+    CUtensorMap a, b0;
+    if (!make_map_2d(&a, Hq, mxg::U8, 1, F, R, mxg::BM) ||
+        !make_map_3d(&b0, W2q, mxg::U8, 1, F, d, E, w2_expert_stride, mxg::MMA_N))
+        return MOE_ERR_CUDA;
+    return mxg::launch<false>(a, b0, b0, Hs, W2s, W2s, w2_expert_stride / 32, offsets, E, R, F, d,
+                              nullptr, nullptr, static_cast<__nv_bfloat16*>(Ye), d,
+                              as_stream(stream));
+}

@@ -74,6 +74,19 @@ class LayerBwdArgs(ctypes.Structure):
     ]
 
 
+class LayerMxArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i64), ("d", _i64), ("E", _i64), ("F", _i64),
+        ("k", ctypes.c_int32), ("renorm", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("reserved1", ctypes.c_int32),
+        ("x", _p), ("logits", _p), ("Wr", _p),
+        ("W1q", _p), ("W1s", _p), ("W3q", _p), ("W3s", _p), ("W2q", _p), ("W2s", _p),
+        ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
+        ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
+        ("workspace", _p), ("workspace_bytes", _sz),
+    ]
+
+
 _SIGS = {
     "moe_route_workspace_size": (_sz, [_i64, _i64, _i32]),
     "moe_route": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _p, _p, _p, _p, _p,
@@ -92,6 +105,12 @@ _SIGS = {
     "moe_combine": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
     "mxfp8_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _p, _p, _p]),
     "mxfp8_dequantize": (_i32, [_p, _p, _i32, _i64, _i64, _p, _p]),
+    "moe_dispatch_mxfp8": (_i32, [_p, _p, _i64, _i64, _i32, _p, _p, _p]),
+    "moe_grouped_gate_up_mxfp8": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64,
+                                         _p, _p, _p]),
+    "moe_grouped_down_mxfp8": (_i32, [_p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _p]),
+    "moe_layer_mxfp8_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
+    "moe_layer_fwd_mxfp8": (_i32, [ctypes.POINTER(LayerMxArgs), _p]),
     "moe_layer_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32, _i32]),
     "moe_layer_fwd": (_i32, [ctypes.POINTER(LayerArgs), _p]),
     "moe_layer_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32]),
@@ -453,3 +472,93 @@ def moe_get_status(clear: bool = True, device=None) -> int:
 
 def moe_version() -> str:
     return lib.moe_version().decode()
+
+
+# ----------------------------------------------------------------- MXFP8 path
+
+@dataclass
+class MxWeights:
+    """E4M3 codes and UE8M0 scales of W1, W3 [E,F,d] and W2 [E,d,F]."""
+    W1q: torch.Tensor
+    W1s: torch.Tensor
+    W3q: torch.Tensor
+    W3s: torch.Tensor
+    W2q: torch.Tensor
+    W2s: torch.Tensor
+
+
+def mxfp8_quantize_weights(W1, W3, W2) -> MxWeights:
+    """Offline quantisation of the expert weights along their contraction
+    dimension (d for W1/W3, F for W2) with UE8M0 block scales."""
+    E, F, d = W1.shape
+    q1, s1 = mxfp8_quantize(W1.reshape(E * F, d), MOE_SCALE_E8M0)
+    q3, s3 = mxfp8_quantize(W3.reshape(E * F, d), MOE_SCALE_E8M0)
+    q2, s2 = mxfp8_quantize(W2.reshape(E * d, F), MOE_SCALE_E8M0)
+    return MxWeights(q1.view(E, F, d), s1.view(E, F, d // 32), q3.view(E, F, d),
+                     s3.view(E, F, d // 32), q2.view(E, d, F), s2.view(E, d, F // 32))
+
+
+def moe_dispatch_mxfp8(x, slot, Xq=None, Xs=None):
+    _need(x, "x"); _need(slot, "slot")
+    T, d = x.shape
+    k = slot.shape[1]
+    if Xq is None:
+        Xq = torch.empty((T * k, d), dtype=torch.uint8, device=x.device)
+    if Xs is None:
+        Xs = torch.empty((T * k, d // 32), dtype=torch.uint8, device=x.device)
+    rc = lib.moe_dispatch_mxfp8(_ptr(x), _ptr(slot), T, d, k, _ptr(Xq), _ptr(Xs), _stream(x))
+    _check("moe_dispatch_mxfp8", rc)
+    return Xq, Xs
+
+
+def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None):
+    _need(Xq, "Xq"); _need(Xs, "Xs"); _need(offsets, "offsets")
+    E, F, d = w.W1q.shape
+    R = Xq.shape[0]
+    if Hq is None:
+        Hq = torch.empty((R, F), dtype=torch.uint8, device=Xq.device)
+    if Hs is None:
+        Hs = torch.empty((R, F // 32), dtype=torch.uint8, device=Xq.device)
+    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xs), _ptr(w.W1q), _ptr(w.W1s), _ptr(w.W3q),
+                                       _ptr(w.W3s), w.W1q.stride(0), _ptr(offsets), E, R, d, F,
+                                       _ptr(Hq), _ptr(Hs), _stream(Xq))
+    _check("moe_grouped_gate_up_mxfp8", rc)
+    return Hq, Hs
+
+
+def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None):
+    _need(Hq, "Hq"); _need(Hs, "Hs"); _need(offsets, "offsets")
+    E, d, F = w.W2q.shape
+    R = Hq.shape[0]
+    if Ye is None:
+        Ye = torch.empty((R, d), dtype=torch.bfloat16, device=Hq.device)
+    rc = lib.moe_grouped_down_mxfp8(_ptr(Hq), _ptr(Hs), _ptr(w.W2q), _ptr(w.W2s), w.W2q.stride(0),
+                                    _ptr(offsets), E, R, d, F, _ptr(Ye), _stream(Hq))
+    _check("moe_grouped_down_mxfp8", rc)
+    return Ye
+
+
+def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm: bool = False,
+                        out: Optional[LayerOut] = None) -> LayerOut:
+    _need(x, "x")
+    T, d = x.shape
+    E, F, _ = w.W1q.shape
+    dev = x.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        ws = _alloc_ws(lib.moe_layer_mxfp8_workspace_size(T, d, E, F, k, int(logits is not None)), dev)
+        out = LayerOut(out=torch.empty((T, d), dtype=torch.bfloat16, device=dev),
+                       idx=torch.empty((T, k), **i32),
+                       gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                       counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                       slot=torch.empty((T, k), **i32), workspace=ws)
+    a = LayerMxArgs(T=T, d=d, E=E, F=F, k=k, renorm=int(renorm), reserved0=0, reserved1=0,
+                    x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1q=_ptr(w.W1q), W1s=_ptr(w.W1s),
+                    W3q=_ptr(w.W3q), W3s=_ptr(w.W3s), W2q=_ptr(w.W2q), W2s=_ptr(w.W2s),
+                    w13_expert_stride=w.W1q.stride(0), w2_expert_stride=w.W2q.stride(0),
+                    out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
+                    counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
+                    workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    rc = lib.moe_layer_fwd_mxfp8(ctypes.byref(a), _stream(x))
+    _check("moe_layer_fwd_mxfp8", rc)
+    return out

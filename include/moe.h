@@ -254,6 +254,65 @@ MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mod
                              int64_t rows, int64_t cols, void* out_bf16, void* stream);
 
 /* ------------------------------------------------------------------------
+ * MXFP8 path ["olmoforge" README, capability table and "MXFP8 分块量化";
+ * "专家池 8→128 只慢 5%…", "三招拆分、三项优化、一个精度开关"].
+ *
+ * moe_dispatch_mxfp8: quantise each token row of x [T,d] (bf16) once, in
+ *   blocks of 32 along d with UE8M0 scales (as mxfp8_quantize with
+ *   MOE_SCALE_E8M0), and write codes and scales to its k slots:
+ *   Xq [R,d] uint8 E4M3, Xs [R,d/32] uint8. d % 32 == 0.
+ * moe_grouped_gate_up_mxfp8 / moe_grouped_down_mxfp8: the grouped SwiGLU
+ *   FFN on block-scaled FP8 MMA (tcgen05 kind::mxf8f6f4, fp32 accumulate).
+ *   Weights are E4M3 codes with UE8M0 scales along their contraction
+ *   dimension (mxfp8_quantize of W1/W3 as [E*F, d] and W2 as [E*d, F]):
+ *   W1q/W3q [E,F,d] + W1s/W3s [E,F,d/32]; W2q [E,d,F] + W2s [E,d,F/32];
+ *   expert strides in elements of the code tensors (scale strides are /32).
+ *   gate/up writes H quantised from its fp32 value: Hq [R,F] + Hs [R,F/32];
+ *   down writes Ye [R,d] bf16. Limits: d % 128 == 0, F % 128 == 0; code
+ *   pointers 16-byte aligned, scale pointers 4-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T, int64_t d, int k,
+                               uint8_t* Xq, uint8_t* Xs, void* stream);
+MOE_API int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
+                                      const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                      int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
+                                      int64_t R, int64_t d, int64_t F, uint8_t* Hq, uint8_t* Hs,
+                                      void* stream);
+MOE_API int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const uint8_t* W2q,
+                                   const uint8_t* W2s, int64_t w2_expert_stride,
+                                   const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                   int64_t F, void* Ye, void* stream);
+
+/* moe_layer_fwd_mxfp8 — route -> moe_dispatch_mxfp8 -> gate/up (MXFP8) ->
+ * down (MXFP8) -> moe_combine (bf16), on one stream. x, Wr and out are bf16. */
+typedef struct moe_layer_mxfp8_args {
+    int64_t T, d, E, F;
+    int32_t k, renorm, reserved0, reserved1;
+    const void* x;          /* [T,d] bf16                                     */
+    const float* logits;    /* [T,E] fp32, or NULL to use Wr                  */
+    const void* Wr;         /* [E,d] bf16                                     */
+    const uint8_t* W1q;
+    const uint8_t* W1s;
+    const uint8_t* W3q;
+    const uint8_t* W3s;
+    const uint8_t* W2q;
+    const uint8_t* W2s;
+    int64_t w13_expert_stride, w2_expert_stride;
+    void* out;              /* [T,d] bf16                                     */
+    int32_t* idx;
+    float* gate;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* slot;
+    void* workspace;        /* Xq, Xs, Hq, Hs, Ye and the route workspace     */
+    size_t workspace_bytes;
+} moe_layer_mxfp8_args;
+
+MOE_API size_t moe_layer_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
+                                              int logits_given);
+MOE_API int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_layer_fwd — the whole layer: route -> dispatch -> grouped SwiGLU ->
  * combine [HF §2-§3], enqueued on one stream with no host synchronisation.
  * ---------------------------------------------------------------------- */

@@ -1,0 +1,139 @@
+"""MXFP8 path on the GPU against the oracle: the quantising dispatch
+(codes and scales bit-exact), the block-scaled grouped GEMMs on operands the
+oracle quantised, and the whole MXFP8 layer against the MXFP8 oracle, with
+its distance to the bf16 oracle measured."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
+from tests._util import assert_close_layer, assert_close_scaled, np64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _moe():
+    from dropless_top_mixture_b200 import moe
+    return moe
+
+
+def _deq(q, s):
+    return O.mxfp8_dequantize_f32(q, s, "e8m0").astype(np.float64)
+
+
+def _quant_w(W):
+    """Oracle quantisation of [E, N, K] weights along K -> codes, scales."""
+    E, N, K = W.shape
+    q, s = O.mxfp8_quantize(W.reshape(E * N, K).float().numpy(), "e8m0")
+    return q.reshape(E, N, K), s.reshape(E, N, K // 32)
+
+
+def _problem(T, d, F, E, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn(T, d, generator=g).to(bf)
+    W1 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(bf)
+    W3 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(bf)
+    W2 = (torch.randn(E, d, F, generator=g) * F ** -0.5).to(bf)
+    lg = adversarial_logits(T, E, "normal", seed=seed).numpy()
+    if E >= 4:
+        lg[:, 1] -= 40.0
+        lg[:, 0] += 3.0
+    return x, W1, W3, W2, lg
+
+
+def test_dispatch_mxfp8_bitexact():
+    moe = _moe()
+    T, d, E, k = 300, 512, 8, 3
+    x, *_ , lg = _problem(T, d, 128, E, k, seed=3)
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    Xq, Xs = moe.moe_dispatch_mxfp8(x.cuda(), torch.from_numpy(meta["slot"]).cuda())
+    q, s = O.mxfp8_quantize(x.float().numpy(), "e8m0")
+    assert np.array_equal(Xq.cpu().numpy(), O.dispatch(q, meta["slot"]))
+    assert np.array_equal(Xs.cpu().numpy(), O.dispatch(s, meta["slot"]))
+
+
+@pytest.mark.parametrize("T,d,F,E,k", [(300, 256, 256, 5, 2), (700, 512, 384, 16, 4),
+                                       (37, 128, 128, 4, 2)])
+def test_grouped_mxfp8_gemms(T, d, F, E, k):
+    moe = _moe()
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, seed=T + d + F)
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    offs = meta["offsets"]
+    xq, xs = O.mxfp8_quantize(x.float().numpy(), "e8m0")
+    Xq, Xs = O.dispatch(xq, meta["slot"]), O.dispatch(xs, meta["slot"])
+    (w1q, w1s), (w3q, w3s), (w2q, w2s) = _quant_w(W1), _quant_w(W3), _quant_w(W2)
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    w = moe.MxWeights(t(w1q), t(w1s), t(w3q), t(w3s), t(w2q), t(w2s))
+    Hq, Hs = moe.moe_grouped_gate_up_mxfp8(t(Xq), t(Xs), w, t(offs))
+    # oracle: exact products of the dequantised operands, then SwiGLU
+    Xd = _deq(Xq, Xs)
+    H = np.zeros((T * k, F))
+    for e in range(E):
+        r0, r1 = offs[e], offs[e + 1]
+        if r1 > r0:
+            a = Xd[r0:r1] @ _deq(w1q[e], w1s[e]).T
+            b = Xd[r0:r1] @ _deq(w3q[e], w3s[e]).T
+            H[r0:r1] = O.silu(a) * b
+    Hq_g, Hs_g = Hq.cpu().numpy(), Hs.cpu().numpy()
+    Hd_g = _deq(Hq_g, Hs_g)
+    hq_ref, hs_ref = O.mxfp8_quantize(H.astype(np.float32), "e8m0")
+    # fp32 accumulation on the GPU moves a few values across a rounding
+    # boundary of the E4M3 grid; almost every code and scale is identical
+    assert np.mean(Hq_g == hq_ref) > 0.99 and np.mean(Hs_g == hs_ref) > 0.99
+    assert rel_l2(Hd_g, _deq(hq_ref, hs_ref)) < 1e-2
+    # down GEMM on the oracle's own quantised H
+    Ye = moe.moe_grouped_down_mxfp8(t(hq_ref), t(hs_ref), w, t(offs))
+    Hd = _deq(hq_ref, hs_ref)
+    Ye_ref = np.zeros((T * k, d))
+    for e in range(E):
+        r0, r1 = offs[e], offs[e + 1]
+        if r1 > r0:
+            Ye_ref[r0:r1] = Hd[r0:r1] @ _deq(w2q[e], w2s[e]).T
+    assert moe.moe_get_status() == 0
+    assert_close_scaled(np64(Ye), Ye_ref, "Ye")
+
+
+def test_layer_mxfp8_small():
+    moe = _moe()
+    T, d, F, E, k = 500, 256, 256, 8, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, seed=11)
+    dev = "cuda"
+    w = moe.mxfp8_quantize_weights(W1.to(dev), W3.to(dev), W2.to(dev))
+    r = moe.moe_layer_fwd_mxfp8(x.to(dev), k, w, logits=torch.from_numpy(lg).to(dev))
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    ref = O.mxfp8_layer(x, k, W1, W3, W2, lg)
+    assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
+    assert_close_scaled(np64(r.out), ref["out"], "out vs MXFP8 oracle")
+
+
+@pytest.mark.slow
+def test_layer_mxfp8_full_size_sampled():
+    """The MXFP8 variant of the 128-expert sweep workload (T=8192, d=4096,
+    F=2048, top-4): the output on sampled tokens against the MXFP8 oracle
+    (bar: rel-L2 1e-2) and, measured, against the bf16 oracle."""
+    moe = _moe()
+    wl = WORKLOADS["mxfp8_e128"]
+    inp = make_inputs(wl, "cuda")
+    w = moe.mxfp8_quantize_weights(inp["W1"], inp["W3"], inp["W2"])
+    r = moe.moe_layer_fwd_mxfp8(inp["x"], wl.k, w, logits=inp["logits"])
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    rng = np.random.default_rng(2)
+    toks = np.sort(rng.choice(wl.T, size=16, replace=False))
+    lg = inp["logits"].cpu().numpy()
+    x_cpu = inp["x"].cpu()
+    ref = O.mxfp8_layer(x_cpu, wl.k, inp["W1"], inp["W3"], inp["W2"], lg, tokens=toks)
+    got = np64(r.out[torch.as_tensor(toks, device="cuda")])
+    assert_close_layer(got, ref["out"], "MXFP8 layer vs MXFP8 oracle")
+    idx, gate, _ = O.route(lg, wl.k)
+    bf = O.moe_layer_tokens(x_cpu, toks, idx, gate, inp["W1"], inp["W3"], inp["W2"])
+    gap = rel_l2(got, bf)
+    print(f"\nMXFP8 layer vs bf16 oracle: rel-L2 {gap:.4f}; "
+          f"MXFP8 oracle vs bf16 oracle: rel-L2 {rel_l2(ref['out'], bf):.4f}")
+    assert gap < 0.1
