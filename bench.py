@@ -184,9 +184,11 @@ def blas_threads():
 
 # ---------------------------------------------------------------- CPU oracle arm
 
-def oracle_sample(w, inp_cpu, S: int):
+def oracle_sample(w, inp_cpu, S: int, backward: bool = False):
     """Run the CPU oracle on the first S tokens of the workload; returns
-    seconds. Routing of the sample, then the per-token SwiGLU mixture."""
+    seconds. Routing of the sample, then the per-token SwiGLU mixture (the
+    MXFP8 oracle for the MXFP8 workload; plus the input gradient of those
+    tokens when the step includes the backward)."""
     from oracle import moe_oracle as O
     x = inp_cpu["x"][:S]
     t0 = time.perf_counter()
@@ -194,21 +196,30 @@ def oracle_sample(w, inp_cpu, S: int):
         lg = O.router_logits(x, inp_cpu["Wr"])
     else:
         lg = inp_cpu["logits"][:S].numpy()
+    if w.mxfp8:
+        O.mxfp8_layer(x, w.k, inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"], lg)
+        return time.perf_counter() - t0
     idx, gate, _ = O.route(lg, w.k)
     O.routing_metadata(idx, w.E)
     O.moe_layer_tokens(x, list(range(S)), idx, gate, inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"])
+    if backward:
+        O.moe_layer_bwd_sampled(x, inp_cpu["dOut"][:S], w.k, inp_cpu["W1"], inp_cpu["W3"],
+                                inp_cpu["W2"], lg, list(range(S)), [])
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, inp_cpu, target_s: float = 12.0):
-    S = 64
-    dt = oracle_sample(w, inp_cpu, S)
+def cpu_baseline(w, inp_cpu, target_s: float = 12.0, backward: bool = False):
+    S = 16 if (w.mxfp8 or backward) else 64
+    dt = oracle_sample(w, inp_cpu, S, backward)
     if dt < target_s / 4 and S < w.T:
         S = int(min(w.T, max(S + 1, S * target_s / max(dt, 1e-3))))
-        dt = oracle_sample(w, inp_cpu, S)
+        dt = oracle_sample(w, inp_cpu, S, backward)
+    what = ("router logits, top-k, routing metadata and the per-token "
+            + ("MXFP8 SwiGLU mixture" if w.mxfp8 else "SwiGLU mixture")
+            + (" plus the input gradient of those tokens (no weight gradients)" if backward else "")
+            + " in float64")
     return {"value": S / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {S} of {w.T} tokens of {w.name}: router logits, top-k, routing "
-                      f"metadata and the per-token SwiGLU mixture in float64 ({dt:.1f} s)"}
+            "sample": f"first {S} of {w.T} tokens of {w.name}: {what} ({dt:.1f} s)"}
 
 
 def run_reference(args):
@@ -219,8 +230,8 @@ def run_reference(args):
     inp = make_inputs(w, "cpu")
     S = args.ref_tokens
     for _ in range(args.warmup):
-        oracle_sample(w, inp, S)
-    times = [oracle_sample(w, inp, S) for _ in range(args.steps)]
+        oracle_sample(w, inp, S, args.backward)
+    times = [oracle_sample(w, inp, S, args.backward) for _ in range(args.steps)]
     tot = sum(times)
     value = S * args.steps / tot
     line = {
@@ -237,8 +248,10 @@ def run_reference(args):
     return 0
 
 
-def config_of(w, world):
+def config_of(w, world, backward=False):
     return {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F,
+            "pass": "forward + backward" if backward else "forward",
+            "precision": "MXFP8 (E4M3, UE8M0 block scales)" if w.mxfp8 else w.dtype,
             "routing": {"router": "logits = x·Wrᵀ", "normal": "logits ~ N(0,1)",
                         "zipf": "logits ~ N(0,1) + ln Zipf(1.1)"}[w.logits],
             "global_batch": w.T * world, "parallelism": f"replicas x{world}",
@@ -246,6 +259,103 @@ def config_of(w, world):
 
 
 # ---------------------------------------------------------------- GPU arm
+
+def _steps(moe, w, inp, dev, backward):
+    """Buffers and the step of one workload. Returns (parts, step,
+    kernels_per_step, work) where work[part] = (flop, algorithmic bytes)."""
+    T, d, E, k, F, R = w.T, w.d, w.E, w.k, w.F, w.R
+    dt = w.torch_dtype
+    es = w.esize
+    i32 = dict(dtype=torch.int32, device=dev)
+    use_router = w.logits == "router"
+    x, Wr, logits = inp["x"], inp.get("Wr"), inp.get("logits")
+    W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
+    rt = moe.Route(idx=torch.empty((T, k), **i32),
+                   gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                   counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                   slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
+    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router)), dtype=torch.uint8,
+                      device=dev)
+    out = torch.empty((T, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
+    Ye = torch.empty((R, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
+
+    def route():
+        if use_router:
+            moe.moe_route(k, x=x, Wr=Wr, out=rt, workspace=rws)
+        else:
+            moe.moe_route(k, logits=logits, out=rt, workspace=rws)
+
+    if w.mxfp8:
+        mw = moe.mxfp8_quantize_weights(W1, W3, W2)  # offline, outside the timed region
+        Xq = torch.empty((R, d), dtype=torch.uint8, device=dev)
+        Xs = torch.empty((R, d // 32), dtype=torch.uint8, device=dev)
+        Hq = torch.empty((R, F), dtype=torch.uint8, device=dev)
+        Hs = torch.empty((R, F // 32), dtype=torch.uint8, device=dev)
+        fns = [("route", route),
+               ("dispatch", lambda: moe.moe_dispatch_mxfp8(x, rt.slot, Xq, Xs)),
+               ("gate_up", lambda: moe.moe_grouped_gate_up_mxfp8(Xq, Xs, mw, rt.offsets, Hq, Hs)),
+               ("down", lambda: moe.moe_grouped_down_mxfp8(Hq, Hs, mw, rt.offsets, Ye)),
+               ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
+        sx, sw, sh = 1 + 1 / 32, 1 + 1 / 32, 1 + 1 / 32
+    else:
+        Xe = torch.empty((R, d), dtype=dt, device=dev)
+        H = torch.empty((R, F), dtype=dt, device=dev)
+        A = torch.empty((R, F), dtype=dt, device=dev) if backward else None
+        B = torch.empty((R, F), dtype=dt, device=dev) if backward else None
+
+        def gate_up():
+            if backward:
+                moe.moe_grouped_gate_up_save(Xe, W1, W3, rt.offsets, H, A, B)
+            else:
+                moe.moe_grouped_gate_up(Xe, W1, W3, rt.offsets, H=H)
+
+        fns = [("route", route),
+               ("dispatch", lambda: moe.moe_dispatch(x, rt.slot, out=Xe)),
+               ("gate_up", gate_up),
+               ("down", lambda: moe.moe_grouped_down(H, W2, rt.offsets, Ye=Ye)),
+               ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
+        sx, sw, sh = es, es, es
+        if backward:
+            dOut = inp["dOut"]
+            dYe = torch.empty((R, d), dtype=dt, device=dev)
+            grads = moe.ExpertGrads(dXe=torch.empty((R, d), dtype=dt, device=dev),
+                                    dW1=torch.empty((E, F, d), dtype=dt, device=dev),
+                                    dW3=torch.empty((E, F, d), dtype=dt, device=dev),
+                                    dW2=torch.empty((E, d, F), dtype=dt, device=dev),
+                                    dA=torch.empty((R, F), dtype=dt, device=dev),
+                                    dB=torch.empty((R, F), dtype=dt, device=dev))
+            dx = torch.empty((T, d), dtype=dt, device=dev)
+            fns += [("bwd_dispatch", lambda: moe.moe_dispatch(dOut, rt.slot, gate=rt.gate, out=dYe)),
+                    ("bwd_gemms", lambda: moe.moe_grouped_swiglu_bwd(Xe, A, B, H, dYe, W1, W3, W2,
+                                                                     rt.offsets, out=grads)),
+                    ("bwd_combine", lambda: moe.moe_combine(grads.dXe, rt.slot, None, out=dx))]
+
+    def step(ev=None):
+        for j, (_, fn) in enumerate(fns):
+            if ev is not None:
+                ev[j].record()
+            fn()
+        if ev is not None:
+            ev[len(fns)].record()
+
+    step()
+    torch.cuda.synchronize(dev)
+    e_act = int((rt.counts > 0).sum().item())
+    wbytes = e_act * F * d * sw
+    work = {
+        "route": (0.0, T * (d * es if use_router else E * 4) + R * 12),
+        "dispatch": (0.0, T * d * es + R * d * sx + R * 4),
+        "gate_up": (4.0 * R * d * F, R * d * sx + 2 * wbytes + R * F * sh),
+        "down": (2.0 * R * d * F, R * F * sh + wbytes + R * d * 2),
+        "combine": (0.0, R * d * 2 + T * d * 2 + R * 8),
+    }
+    if backward:
+        work["bwd_dispatch"] = (0.0, T * d * es + R * d * es + R * 8)
+        work["bwd_gemms"] = (12.0 * R * d * F, 6 * wbytes + R * (5 * d + 5 * F) * es)
+        work["bwd_combine"] = (0.0, R * d * es + T * d * es + R * 4)
+    kernels = (4 if use_router else 3) + 4 + (7 if backward else 0)
+    return [n for n, _ in fns], step, kernels, work, e_act
+
 
 def run_ours(args):
     rank, world, local = dist_env()
@@ -255,46 +365,12 @@ def run_ours(args):
     from dropless_top_mixture_b200 import moe
 
     w = WORKLOADS[args.workload]
+    backward = bool(args.backward)
+    if backward and (w.mxfp8 or w.dtype != "bf16"):
+        raise SystemExit("--backward runs on the bf16 workloads")
     inp = make_inputs(w, dev)
     T, d, E, k, F, R = w.T, w.d, w.E, w.k, w.F, w.R
-    dt = w.torch_dtype
-    i32 = dict(dtype=torch.int32, device=dev)
-    use_router = w.logits == "router"
-    x = inp["x"]
-    Wr = inp.get("Wr")
-    logits = inp.get("logits")
-    W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
-    rt = moe.Route(idx=torch.empty((T, k), **i32), gate=torch.empty((T, k), dtype=torch.float32, device=dev),
-                   counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
-                   slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
-    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router)), dtype=torch.uint8, device=dev)
-    Xe = torch.empty((R, d), dtype=dt, device=dev)
-    H = torch.empty((R, F), dtype=dt, device=dev)
-    Ye = torch.empty((R, d), dtype=dt, device=dev)
-    out = torch.empty((T, d), dtype=dt, device=dev)
-    kernels_per_step = (4 if use_router else 3) + 4
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record()
-        if use_router:
-            moe.moe_route(k, x=x, Wr=Wr, out=rt, workspace=rws)
-        else:
-            moe.moe_route(k, logits=logits, out=rt, workspace=rws)
-        if ev is not None:
-            ev[1].record()
-        moe.moe_dispatch(x, rt.slot, out=Xe)
-        if ev is not None:
-            ev[2].record()
-        moe.moe_grouped_gate_up(Xe, W1, W3, rt.offsets, H=H)
-        if ev is not None:
-            ev[3].record()
-        moe.moe_grouped_down(H, W2, rt.offsets, Ye=Ye)
-        if ev is not None:
-            ev[4].record()
-        moe.moe_combine(Ye, rt.slot, rt.gate, out=out)
-        if ev is not None:
-            ev[5].record()
+    parts, step, kernels_per_step, work, e_act = _steps(moe, w, inp, dev, backward)
 
     sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     for _ in range(args.warmup):
@@ -303,7 +379,8 @@ def run_ours(args):
     if moe.moe_get_status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+           for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -316,23 +393,21 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     w1 = time.monotonic()
     barrier(world)
-    ms_local = start.elapsed_time(end)
-    ms_total = max_over_ranks(ms_local, world, dev)
+    ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
     ms_step = ms_total / args.steps
     value = T * world * args.steps / (ms_total / 1e3)
-
-    parts = ["route", "dispatch", "gate_up", "down", "combine"]
     per = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, p in enumerate(parts)}
 
     # clocks: the timed window; if it held too few samples, keep running
     # untimed steps of the same workload while sampling
-    extra_s = 0.0
+    clocks = None
     if sampler is not None:
         lines = sampler.window(w0, w1)
+        extra_s = 0.0
         if len(lines) < 10:
             t_ext0 = time.monotonic()
             while time.monotonic() - t_ext0 < 1.0:
-                for _ in range(20):
+                for _ in range(5):
                     step()
                 torch.cuda.synchronize(dev)
             extra_s = time.monotonic() - t_ext0
@@ -340,90 +415,130 @@ def run_ours(args):
         clocks = ClockSampler.summarize(lines)
         if clocks is not None and extra_s:
             clocks["note"] = f"timed window plus {extra_s:.1f} s of untimed steps of the same workload"
-    else:
-        clocks = None
 
-    # end to end through the public call with host buffers
+    # end to end through the public layer calls with host buffers
     e2e = None
     if not args.no_e2e:
-        x_h = x.cpu().pin_memory()
-        lg_h = logits.cpu().pin_memory() if logits is not None else None
-        out_h = torch.empty((T, d), dtype=dt).pin_memory()
-        x_d = torch.empty_like(x)
-        lg_d = torch.empty_like(logits) if logits is not None else None
-        lo = moe.moe_layer_fwd(x, k, W1, W3, W2, logits=logits, Wr=Wr)
-
-        def e2e_step():
-            x_d.copy_(x_h, non_blocking=True)
-            if lg_d is not None:
-                lg_d.copy_(lg_h, non_blocking=True)
-            moe.moe_layer_fwd(x_d, k, W1, W3, W2, logits=lg_d, Wr=Wr, out=lo)
-            out_h.copy_(lo.out, non_blocking=True)
-
-        for _ in range(args.warmup):
-            e2e_step()
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        s2 = torch.cuda.Event(enable_timing=True)
-        e2 = torch.cuda.Event(enable_timing=True)
-        s2.record()
-        for _ in range(args.steps):
-            e2e_step()
-        e2.record()
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
-        h2d = x.numel() * x.element_size() + (logits.numel() * 4 if logits is not None else 0)
-        e2e = {"value": T * world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size()}
+        e2e = _e2e(moe, w, inp, dev, world, args, backward)
 
     if moe.moe_get_status() != 0:
         raise RuntimeError("device status word set during the timed region")
     if sampler is not None:
         sampler.stop()
-
     if rank != 0:
         return 0
 
     peaks, peak_src = measured_peaks()
-    es = w.esize
-    gemm1_flops = 4.0 * R * d * F
-    gemm2_flops = 2.0 * R * d * F
-    tf_gate_up = gemm1_flops / (per["gate_up"] / 1e3) / 1e12
-    tf_down = gemm2_flops / (per["down"] / 1e3) / 1e12
-    tf_ffn = (gemm1_flops + gemm2_flops) / ((per["gate_up"] + per["down"]) / 1e3) / 1e12
-    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    disp_bytes = T * d * es + R * d * es + R * 4
-    comb_bytes = R * d * es + T * d * es + R * 8
     hbm = peaks["hbm_gbs"]
+    bf16_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_tf = bf16_tf * (2.0 if w.mxfp8 else 1.0)
+    tf_src = (f"{peak_src} bf16 sustained x 2 (dense FP8/BF16 nominal ratio 4.5/2.25)" if w.mxfp8
+              else f"{peak_src} bf16 sustained (kernel timed inside a long step)")
+    rates = {}
+    for p in parts:
+        flop, byts = work[p]
+        t = per[p] / 1e3
+        rates[p] = {"ms": per[p], "gbs": byts / t / 1e9}
+        if flop:
+            rates[p]["tflops"] = flop / t / 1e12
+            rates[p]["intensity_flop_per_byte"] = flop / byts
+    gemm_parts = [p for p in parts if work[p][0] > 0]
+    dom = max(gemm_parts, key=lambda p: per[p])
+    flop, byts = work[dom]
+    ridge = peak_tf * 1e12 / (hbm * 1e9)
+    if flop / byts >= ridge:
+        roof = {"bound": "tensor", "achieved": rates[dom]["tflops"], "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": rates[dom]["tflops"] / peak_tf, "peak_source": tf_src,
+                "algorithmic_per_launch": f"{flop:.4g} flop"}
+    else:
+        roof = {"bound": "hbm", "achieved": rates[dom]["gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": rates[dom]["gbs"] / hbm, "peak_source": f"{peak_src} HBM copy bandwidth",
+                "algorithmic_per_launch": f"{byts:.4g} bytes (operands once, outputs once)"}
+    roof["kernel"] = {"gate_up": "grouped gate_up GEMM + SwiGLU (tcgen05)",
+                      "down": "grouped down GEMM (tcgen05)",
+                      "bwd_gemms": "grouped backward GEMMs dH/dX/dW (tcgen05)"}[dom]
+    roof["ridge_flop_per_byte"] = ridge
+    roof["traffic"] = recorded_traffic(dom, w.name) if not w.mxfp8 else None
+    ffn_t = (per["gate_up"] + per["down"]) / 1e3
+    ffn_tf = (work["gate_up"][0] + work["down"][0]) / ffn_t / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
-        "data": "synthetic", "config": config_of(w, world),
-        "roofline": {"kernel": "grouped gate_up GEMM + SwiGLU (tcgen05)", "bound": "tensor",
-                     "achieved": tf_gate_up, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": tf_gate_up / peak_tf,
-                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                     "algorithmic_per_launch": f"{gemm1_flops:.4g} flop = 4*R*d*F",
-                     "traffic": recorded_traffic("gate_up", w.name)},
-        "breakdown_ms": per,
-        "grouped_gemm": {"gate_up_tflops": tf_gate_up, "down_tflops": tf_down,
-                         "ffn_tflops": tf_ffn, "ffn_frac_of_peak": tf_ffn / peak_tf},
-        "hbm": {"dispatch_gbs": disp_bytes / (per["dispatch"] / 1e3) / 1e9,
-                "combine_gbs": comb_bytes / (per["combine"] / 1e3) / 1e9,
-                "dispatch_frac": disp_bytes / (per["dispatch"] / 1e3) / 1e9 / hbm,
-                "combine_frac": comb_bytes / (per["combine"] / 1e3) / 1e9 / hbm,
-                "peak_gbs": hbm},
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if w.mxfp8 else ("bf16" if w.dtype == "bf16" else "f32"),
+        "data": "synthetic", "config": config_of(w, world, backward), "roofline": roof,
+        "breakdown": rates,
+        "grouped_gemm": {"ffn_tflops": ffn_tf, "ffn_frac_of_peak": ffn_tf / peak_tf,
+                         "peak_tflops": peak_tf, "experts_with_rows": e_act},
+        "hbm": {"dispatch_frac": rates["dispatch"]["gbs"] / hbm,
+                "combine_frac": rates["combine"]["gbs"] / hbm, "peak_gbs": hbm},
         "e2e": e2e, "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
         inp_cpu = {kk: v.cpu() for kk, v in inp.items()}
-        line["cpu_baseline"] = cpu_baseline(w, inp_cpu)
+        line["cpu_baseline"] = cpu_baseline(w, inp_cpu, backward=backward)
     else:
         line["cpu_baseline"] = None
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _e2e(moe, w, inp, dev, world, args, backward):
+    """Same metric through the public layer calls, with the step's inputs
+    copied from pinned host memory and its result copied back, per step."""
+    T, k = w.T, w.k
+    x, Wr, logits = inp["x"], inp.get("Wr"), inp.get("logits")
+    W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
+    x_h = x.cpu().pin_memory()
+    lg_h = logits.cpu().pin_memory() if logits is not None else None
+    x_d = torch.empty_like(x)
+    lg_d = torch.empty_like(logits) if logits is not None else None
+    h2d = x.numel() * x.element_size() + (logits.numel() * 4 if logits is not None else 0)
+    if w.mxfp8:
+        mw = moe.mxfp8_quantize_weights(W1, W3, W2)
+        lo = moe.moe_layer_fwd_mxfp8(x, k, mw, logits=logits, Wr=Wr)
+        res = lo.out
+        run = lambda: moe.moe_layer_fwd_mxfp8(x_d, k, mw, logits=lg_d, Wr=Wr, out=lo)
+    elif backward:
+        dO_h = inp["dOut"].cpu().pin_memory()
+        dO_d = torch.empty_like(inp["dOut"])
+        h2d += dO_d.numel() * dO_d.element_size()
+        lo = moe.moe_layer_fwd(x, k, W1, W3, W2, logits=logits, Wr=Wr, save=True)
+        gr = moe.moe_layer_bwd(lo, inp["dOut"], k, W1, W3, W2)
+        res = gr.dx
+
+        def run():
+            dO_d.copy_(dO_h, non_blocking=True)
+            moe.moe_layer_fwd(x_d, k, W1, W3, W2, logits=lg_d, Wr=Wr, out=lo, save=True)
+            moe.moe_layer_bwd(lo, dO_d, k, W1, W3, W2, out=gr)
+    else:
+        lo = moe.moe_layer_fwd(x, k, W1, W3, W2, logits=logits, Wr=Wr)
+        res = lo.out
+        run = lambda: moe.moe_layer_fwd(x_d, k, W1, W3, W2, logits=lg_d, Wr=Wr, out=lo)
+    res_h = torch.empty(res.shape, dtype=res.dtype).pin_memory()
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        if lg_d is not None:
+            lg_d.copy_(lg_h, non_blocking=True)
+        run()
+        res_h.copy_(res, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
+    return {"value": T * world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": res.numel() * res.element_size()}
 
 
 def main(argv=None):
@@ -435,6 +550,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the CPU-oracle reference arm")
+    ap.add_argument("--backward", action="store_true",
+                    help="time forward + backward (bf16 workloads; the fine-grained workload's pass)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",
