@@ -365,6 +365,11 @@ def run_ours(args):
     from dropless_top_mixture_b200 import moe
 
     w = WORKLOADS[args.workload]
+    if args.shrink > 1:
+        # the same shape per expert (T and E divided together) on a smaller
+        # problem, for profiler captures that must stay small
+        w = w.scaled(name=f"{w.name}/shrink{args.shrink}", T=max(1, w.T // args.shrink),
+                     E=max(w.k, w.E // args.shrink))
     backward = bool(args.backward)
     if backward and (w.mxfp8 or w.dtype != "bf16"):
         raise SystemExit("--backward runs on the bf16 workloads")
@@ -552,6 +557,8 @@ def main(argv=None):
                     help="tokens per step of the CPU-oracle reference arm")
     ap.add_argument("--backward", action="store_true",
                     help="time forward + backward (bf16 workloads; the fine-grained workload's pass)")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide T and E by this factor (profiling a small case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",

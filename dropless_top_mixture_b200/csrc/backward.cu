@@ -15,7 +15,9 @@
 //
 // One kernel template, three modes, the same pipeline as the forward grouped
 // GEMM (TMA producer warp, single-thread tcgen05.mma issue, 4 epilogue warps,
-// 4-stage shared-memory ring, double-buffered 128x256 fp32 TMEM accumulator):
+// 4-stage shared-memory ring, double-buffered 128x256 fp32 TMEM accumulator,
+// 8 epilogue warps: each TMEM lane quarter is drained by two warps, one per
+// half of the columns):
 //   DH  A = dYe rows (K-major), B = W2_e read as [F x d] (MN-major, F
 //       contiguous); epilogue loads A,B of the same rows/columns and writes dA, dB.
 //   DX  A = dA then dB rows (K-major), B = W1_e then W3_e read as [d x F]
@@ -23,8 +25,9 @@
 //   DW  per expert a 128 x 256 tile of the [M x N] gradient; A and B are the
 //       expert's rows of two [R x M] / [R x N] matrices, both MN-major, with K
 //       running over the rows. The last K slab of an expert can reach into the
-//       next expert's rows: those rows are zeroed in shared memory before the
-//       MMA reads them. An expert with no rows writes zeros.
+//       next expert's rows: only its 16-row MMA steps that hold valid rows run,
+//       and the few foreign rows inside the last of them are zeroed in shared
+//       memory before the MMA reads them. An expert with no rows writes zeros.
 #include "tc_sm100.cuh"
 
 namespace moe {
@@ -35,24 +38,30 @@ using namespace tc;
 constexpr int BM = 128;
 constexpr int MMA_N = 256;
 constexpr int BK = 64;  // bf16 elements per 128-byte slab
-constexpr int STAGES = 4;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, one per column half
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int A_BYTES = BM * 128;
 constexpr int B_BYTES = MMA_N * 128;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BOX_BYTES = 64 * 128;  // one MN-major box: 64 K rows x 64 elements
 constexpr int TMEM_ALLOC = 512;
-constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + META_BYTES;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+constexpr int STG_BYTES = 32 * 128;  // dW store staging: 32 rows x 64 bf16, one per buffer
 
 enum Mode { DH = 0, DX = 1, DW = 2 };
 
+// DW tiles have a short K (an expert's rows) and a large output, so they use
+// fewer pipeline stages and spend the shared memory on store staging
+// (4 epilogue warps x 2 buffers) for TMA tensor stores.
 template <int MODE>
 struct ModeCfg {
     static constexpr bool A_MN = (MODE == DW);
     static constexpr uint32_t IDESC = make_idesc_major(1u, BM, MMA_N, A_MN, true);
+    static constexpr int STAGES = (MODE == DW) ? 3 : 4;
+    static constexpr int STAGING = (MODE == DW) ? EPI_WARPS * 2 * STG_BYTES : 0;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    static constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING + META_BYTES;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
 struct Tile {
@@ -115,12 +124,14 @@ __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* src, float* v) 
 //   K      DH: d; DX: 2F (KF = K/2 slabs per operand pair); DW: unused
 //   Mdim   DW: rows of each expert's gradient (F or d)
 //   Ndim   DH: F; DX: d; DW: columns of each expert's gradient
+//   tmOut  DW: the gradient viewed as [E*Mdim, Ndim] bf16, box 64 x 32 (TMA store)
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmOut,
                     const int32_t* __restrict__ offsets, int E, int R, int K, int Mdim, int Ndim,
                     __nv_bfloat16* __restrict__ out0, __nv_bfloat16* __restrict__ out1,
                     int64_t ldo, const __nv_bfloat16* __restrict__ saveA,
@@ -129,7 +140,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* meta = smem + STAGES * STAGE_BYTES;
+    constexpr int STAGES = C::STAGES;
+    constexpr int NUM_BARS = C::NUM_BARS;
+    uint8_t* staging = smem + STAGES * STAGE_BYTES;
+    uint8_t* meta = staging + C::STAGING;
     uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
@@ -186,7 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(tfull + b), 1);
-            mbar_init(smem_u32(tempty + b), 4);
+            mbar_init(smem_u32(tempty + b), EPI_WARPS);
         }
         mbar_init(smem_u32(drain), 1);
         *s_abort = 0;
@@ -286,22 +300,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint8_t* sa_p = smem + stage * STAGE_BYTES;
                 const uint32_t sa = smem_u32(sa_p);
                 const uint32_t sb = sa + A_BYTES;
+                int nks = 4;  // 16-row K steps of this slab the MMAs consume
                 if (MODE == DW) {
                     const int valid = tl.row_end - (tl.row0 + kb * BK);
                     if (valid < BK) {
-                        // rows [valid, 64) of each of the 6 boxes belong to another
-                        // expert (or lie past R): zero them before the MMA reads them
-                        const int nrows = BK - valid;
-                        const int chunks = 6 * nrows * 8;  // 16-byte chunks
-                        for (int c = lane; c < chunks; c += 32) {
-                            const int box = c / (nrows * 8);
-                            const int rem = c - box * nrows * 8;
-                            const int row = valid + rem / 8;
-                            const int col = rem & 7;
-                            uint8_t* p = sa_p + box * BOX_BYTES + row * 128 + col * 16;
-                            *reinterpret_cast<uint4*>(p) = make_uint4(0, 0, 0, 0);
+                        // The slab ends inside the expert's last rows: only the K
+                        // steps holding valid rows run, and the rows between the
+                        // last valid row and the end of its 16-row step (another
+                        // expert's rows, or past R) are zeroed in all 6 boxes first.
+                        nks = (valid + 15) >> 4;
+                        const int nz = nks * 16 - valid;
+                        if (nz > 0) {
+#pragma unroll 1
+                            for (int box = 0; box < 6; ++box)
+                                for (int c = lane; c < nz * 8; c += 32) {
+                                    uint8_t* p = sa_p + box * BOX_BYTES + (valid + (c >> 3)) * 128 +
+                                                 ((c & 7) << 4);
+                                    *reinterpret_cast<uint4*>(p) = make_uint4(0, 0, 0, 0);
+                                }
+                            fence_proxy_async_smem();
                         }
-                        fence_proxy_async_smem();
                         __syncwarp();
                     }
                 }
@@ -309,6 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
+                        if (ks >= nks) break;
                         const uint64_t ad = C::A_MN ? sw128_mn_desc(sa + ks * 2048, BOX_BYTES)
                                                     : sw128_desc(sa) + 2 * ks;
                         const uint64_t bd = sw128_mn_desc(sb + ks * 2048, BOX_BYTES);
@@ -333,8 +352,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;
+        const int q = warp & 3;                       // TMEM lane quarter
+        const int col0 = ((warp - 2) >> 2) * (MMA_N / 2);  // this warp's column half
         const int r_in_tile = q * 32 + lane;
+        int stg_count = 0;
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
@@ -344,30 +365,49 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
             if (MODE == DW) {
-                __nv_bfloat16* orow = out0 + (size_t)tl.e * Mdim * Ndim +
-                                      (size_t)(tl.m0 + r_in_tile) * Ndim + tl.n0;
+                // 64-column groups: TMEM -> bf16 -> 128-byte-swizzled staging
+                // (chunk c of row r at c ^ (r % 8), conflict-free) -> TMA store
+                // of the warp's 32 x 64 box; two staging buffers per warp
                 const bool empty_k = tl.nkb == 0;
+                const int ybase = tl.e * Mdim + tl.m0 + q * 32;
+                uint8_t* stg = staging + (warp - 2) * 2 * STG_BYTES;
 #pragma unroll 1
-                for (int c = 0; c < MMA_N / 32; ++c) {
-                    float v[32];
+                for (int cc = col0 / 64; cc < (col0 + MMA_N / 2) / 64; ++cc) {
+                    uint8_t* sbuf = stg + (stg_count & 1) * STG_BYTES;
+                    ++stg_count;
+                    if (lane == 0) bulk_wait_read<1>();  // this buffer's previous store has read it
+                    __syncwarp();
+                    uint32_t a[2][32];
                     if (!empty_k) {
-                        uint32_t a[32];
-                        tmem_ld32(ta + c * 32, a);
+                        tmem_ld32(ta + cc * 64, a[0]);
+                        tmem_ld32(ta + cc * 64 + 32, a[1]);
                         tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                        for (int j = 0; j < 32; ++j) a[0][j] = a[1][j] = 0u;
                     }
-                    store32_bf16(orow + c * 32, v);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int chunk = h * 4 + j;
+                            *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                                pack8(reinterpret_cast<const float*>(a[h]) + 8 * j);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmOut, smem_u32(sbuf), tl.n0 + cc * 64, ybase);
+                        bulk_commit();
+                    }
                 }
             } else {
                 const int grow = tl.row0 + r_in_tile;
                 const bool valid = grow < tl.row_end;
                 const size_t rowoff = (size_t)(valid ? grow : 0) * ldo + tl.n0;
 #pragma unroll 1
-                for (int c = 0; c < MMA_N / 32; ++c) {
+                for (int c = col0 / 32; c < (col0 + MMA_N / 2) / 32; ++c) {
                     uint32_t a[32];
                     tmem_ld32(ta + c * 32, a);
                     tmem_wait_ld();
@@ -398,6 +438,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
         }
+        if (MODE == DW && lane == 0) bulk_wait<0>();  // stores done before the CTA leaves
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -411,10 +453,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 template <int MODE>
 static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                  const CUtensorMap& b1, const int32_t* offsets, int64_t E, int64_t R, int64_t K,
-                  int64_t Mdim, int64_t Ndim, void* out0, void* out1, int64_t ldo,
-                  const void* saveA, const void* saveB, cudaStream_t st) {
+                  const CUtensorMap& b1, const CUtensorMap& om, const int32_t* offsets, int64_t E,
+                  int64_t R, int64_t K, int64_t Mdim, int64_t Ndim, void* out0, void* out1,
+                  int64_t ldo, const void* saveA, const void* saveB, cudaStream_t st) {
     auto kern = bwd_gemm_kernel<MODE>;
+    constexpr int SMEM_BYTES = ModeCfg<MODE>::SMEM_BYTES;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -430,7 +473,7 @@ static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMa
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
     kern<<<grid, THREADS, SMEM_BYTES, st>>>(
-        a0, a1, b0, b1, offsets, (int)E, (int)R, (int)K, (int)Mdim, (int)Ndim,
+        a0, a1, b0, b1, om, offsets, (int)E, (int)R, (int)K, (int)Mdim, (int)Ndim,
         static_cast<__nv_bfloat16*>(out0), static_cast<__nv_bfloat16*>(out1), ldo,
         static_cast<const __nv_bfloat16*>(saveA), static_cast<const __nv_bfloat16*>(saveB),
         status_ptr());
@@ -470,7 +513,8 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
         if (!make_map_2d(&mA, dYe, bwd::BF16, 2, d, R, bwd::BM) ||
             !make_map_3d(&mW2, W2, bwd::BF16, 2, F, d, E, w2_expert_stride, 64))
             return MOE_ERR_CUDA;
-        rc = bwd::launch<bwd::DH>(mA, mA, mW2, mW2, offsets, E, R, d, 0, F, dA, dB, F, A, B, st);
+        rc = bwd::launch<bwd::DH>(mA, mA, mW2, mW2, mA, offsets, E, R, d, 0, F, dA, dB, F, A, B,
+                                  st);
         if (rc != MOE_OK) return rc;
         // dXe = dA W1_e + dB W3_e
         CUtensorMap mdA, mdB, mW1, mW3;
@@ -479,8 +523,8 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
             !make_map_3d(&mW1, W1, bwd::BF16, 2, d, F, E, w13_expert_stride, 64) ||
             !make_map_3d(&mW3, W3, bwd::BF16, 2, d, F, E, w13_expert_stride, 64))
             return MOE_ERR_CUDA;
-        rc = bwd::launch<bwd::DX>(mdA, mdB, mW1, mW3, offsets, E, R, 2 * F, 0, d, dXe, nullptr, d,
-                                  nullptr, nullptr, st);
+        rc = bwd::launch<bwd::DX>(mdA, mdB, mW1, mW3, mdA, offsets, E, R, 2 * F, 0, d, dXe,
+                                  nullptr, d, nullptr, nullptr, st);
         if (rc != MOE_OK) return rc;
     }
     // weight gradients (every expert's tile runs, so empty experts get zeros)
@@ -492,12 +536,17 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
         !make_map_2d(&gY, dYe, bwd::BF16, 2, d, Rm, 64) ||
         !make_map_2d(&gH, H, bwd::BF16, 2, F, Rm, 64))
         return MOE_ERR_CUDA;
-    rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, offsets, E, R, 0, F, d, dW1, nullptr, d, nullptr,
+    CUtensorMap o1, o3, o2;  // the gradients as [E*M, N] for the TMA stores
+    if (!make_map_2d(&o1, dW1, bwd::BF16, 2, d, E * F, 32) ||
+        !make_map_2d(&o3, dW3, bwd::BF16, 2, d, E * F, 32) ||
+        !make_map_2d(&o2, dW2, bwd::BF16, 2, F, E * d, 32))
+        return MOE_ERR_CUDA;
+    rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, o1, offsets, E, R, 0, F, d, dW1, nullptr, d, nullptr,
                               nullptr, st);
     if (rc != MOE_OK) return rc;
-    rc = bwd::launch<bwd::DW>(gB, gB, gX, gX, offsets, E, R, 0, F, d, dW3, nullptr, d, nullptr,
+    rc = bwd::launch<bwd::DW>(gB, gB, gX, gX, o3, offsets, E, R, 0, F, d, dW3, nullptr, d, nullptr,
                               nullptr, st);
     if (rc != MOE_OK) return rc;
-    return bwd::launch<bwd::DW>(gY, gY, gH, gH, offsets, E, R, 0, d, F, dW2, nullptr, F, nullptr,
-                                nullptr, st);
+    return bwd::launch<bwd::DW>(gY, gY, gH, gH, o2, offsets, E, R, 0, d, F, dW2, nullptr, F,
+                                nullptr, nullptr, st);
 }

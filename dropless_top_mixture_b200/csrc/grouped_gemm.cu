@@ -16,11 +16,12 @@
 // columns of B. One 128xMMA_Nx16 MMA per 32 bytes of K; K is staged 128
 // bytes at a time by TMA with the 128-byte swizzle the MMA descriptors read.
 //
-// Warp roles (192 threads, one CTA per SM):
+// Warp roles (320 threads, one CTA per SM):
 //   warp 0, lane 0   TMA producer over a STAGES-deep shared-memory ring
 //   warp 1           allocates TMEM; lane 0 issues tcgen05.mma
-//   warps 2..5       epilogue: tcgen05.ld from TMEM (warp w reads lanes
-//                    32*(w%4)..), SwiGLU / conversion, row-masked stores
+//   warps 2..9       epilogue: tcgen05.ld from TMEM (warp w reads lanes
+//                    32*(w%4).., two warps per quarter split the columns),
+//                    SwiGLU / conversion, row-masked stores
 // The accumulator is double-buffered in TMEM (2 x MMA_N columns), so the
 // epilogue of tile i overlaps the main loop of tile i+1.
 //
@@ -37,7 +38,8 @@ namespace gg {
 
 constexpr int BM = 128;
 constexpr int STAGES = 4;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, one per column half
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 using namespace tc;
 
 // ------------------------------------------------------------------ config
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(tfull + b), 1);
-            mbar_init(smem_u32(tempty + b), 4);
+            mbar_init(smem_u32(tempty + b), EPI_WARPS);
         }
         mbar_init(smem_u32(drain), 1);
         *s_abort = 0;
@@ -287,6 +289,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int c_lo = ((warp - 2) >> 2) * (C::OUT_N / 64);  // this warp's half of the
+        const int c_hi = c_lo + C::OUT_N / 64;                  // 32-column chunks
         const int r_in_tile = q * 32 + lane;
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool valid = grow < tl.row_end;
             TIn* orow = out + (size_t)(valid ? grow : 0) * ldo + tl.n0;
 #pragma unroll 1
-            for (int c = 0; c < C::OUT_N / 32; ++c) {
+            for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t a[32];
                 float v[32];
                 tmem_ld32(ta + c * 32, a);

@@ -14,8 +14,8 @@
 // Kernel: tcgen05.mma kind::mxf8f6f4.block_scale, M = 128, N = 128, K = 32 per
 // instruction, 128-byte K slabs staged by TMA with the same 128-byte swizzle
 // as the bf16 kernels. Per slab every row carries 4 UE8M0 scales (one 32-bit
-// word); the producer warp gathers the 128 A words and 128 B words into the
-// 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4 copies into TMEM
+// word); the producer warp gathers the 128 A words and 128 B words (cp.async,
+// tracked by the stage's mbarrier) into the 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4 copies into TMEM
 // (lane m%32 of every sub-partition, column m/32, byte = K block), and the
 // MMA selects the byte with the scale-factor id of each of the 4 MMAs.
 // Accumulators: two 128-column TMEM buffers; the scale factors follow them.
@@ -98,8 +98,16 @@ __device__ __forceinline__ Tile decode_tile(int t, int NB, int E, int out_n, con
     return tl;
 }
 
-__device__ __forceinline__ uint32_t ld_word(const uint8_t* p) {
-    return __ldg(reinterpret_cast<const uint32_t*>(p));
+// 4-byte asynchronous global->shared copy; src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async_word(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// The mbarrier counts one arrival once all of this thread's earlier cp.async
+// copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // SWIGLU: B tile = 64 rows of W1 then 64 rows of W3 at the same n0; the
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* drain = bars + 2 * STAGES + 4;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(full + s), 2);  // TMA bytes + the scale words
+            mbar_init(smem_u32(full + s), 1 + 32);  // TMA bytes + each lane's scale words
             mbar_init(smem_u32(empty + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -219,14 +227,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_3d(sb, &tmB0, fb, kb * BK, tl.n0, tl.e);
                     }
                 }
-                uint32_t* sfw = reinterpret_cast<uint32_t*>(sf_smem + stage * SF_STAGE_BYTES);
+                // scale words, copied asynchronously: the stage's barrier
+                // completes only once they have landed, so the producer never
+                // waits on their latency
+                const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int m = lane + 32 * j;  // A row within the tile
                     const int grow = tl.row0 + m;
-                    const uint32_t wa =
-                        grow < R ? ld_word(sfA + (size_t)grow * sf_row + 4 * kb) : 0u;
-                    sfw[lane * 4 + j] = wa;
+                    const bool in = grow < R;
+                    cp_async_word(sfs + (uint32_t)(lane * 4 + j) * 4u,
+                                  sfA + (size_t)(in ? grow : 0) * sf_row + 4 * kb, in ? 4u : 0u);
                     const uint8_t* bsrc;
                     if (SWIGLU) {
                         bsrc = (m < 64 ? sfB0 + (size_t)(tl.n0 + m) * sf_row
@@ -234,11 +245,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     } else {
                         bsrc = sfB0 + (size_t)(tl.n0 + m) * sf_row;
                     }
-                    sfw[128 + lane * 4 + j] = ld_word(bsrc + (size_t)tl.e * sfb_expert_stride + 4 * kb);
+                    cp_async_word(sfs + 512u + (uint32_t)(lane * 4 + j) * 4u,
+                                  bsrc + (size_t)tl.e * sfb_expert_stride + 4 * kb, 4u);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(fb);
+                cp_async_arrive(fb);
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) {
@@ -279,6 +289,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                fence_proxy_async_smem();  // scale words came through the generic proxy
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 tmem_cp_sf(sfa_t, sf_desc(sfs));
                 tmem_cp_sf(sfb_t, sf_desc(sfs + 512));
