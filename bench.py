@@ -463,7 +463,7 @@ def run_ours(args):
                       "down": "grouped down GEMM (tcgen05)",
                       "bwd_gemms": "grouped backward GEMMs dH/dX/dW (tcgen05)"}[dom]
     roof["ridge_flop_per_byte"] = ridge
-    roof["traffic"] = recorded_traffic(dom, w.name) if not w.mxfp8 else None
+    roof["traffic"] = recorded_traffic(dom, w.name)
     ffn_t = (per["gate_up"] + per["down"]) / 1e3
     ffn_tf = (work["gate_up"][0] + work["down"][0]) / ffn_t / 1e12
     line = {
