@@ -370,6 +370,323 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     return launch_status();
 }
 
+// ---------------------------------------------------------------- CTA pairs
+//
+// The same computation on a 256-row x 256-column tile shared by a cluster of
+// two CTAs (tcgen05 cta_group::2, M = 256). CTA r of the pair keeps rows
+// row0 + 128 r .. + 127 of A and one half of the B tile in its own shared
+// memory (SwiGLU: CTA 0 the W1 block, CTA 1 the W3 block; down: the two
+// 128-row halves of the W2 block), so each CTA streams half the B bytes of
+// the single-CTA tile for the same work. Both CTAs' TMA copies complete on
+// the leader's (rank 0) stage barrier; the leader's elected thread issues
+// the MMAs and its commits arrive on the stage-empty and accumulator-full
+// barriers of both CTAs; each CTA drains its own 128 TMEM lanes and both
+// arrive on the leader's accumulator-empty barrier. Cluster barriers bracket
+// set-up and tear-down, so no CTA signals a barrier that is not live.
+namespace pr {
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * 128;   // this CTA's 128 rows of a 128-byte K slab
+constexpr int BH_BYTES = 128 * 128; // this CTA's 128 of the 256 B rows
+constexpr int STAGE_BYTES = A_BYTES + BH_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + META_BYTES;
+constexpr int PM = 2 * BM;          // rows per pair tile
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+}  // namespace pr
+
+template <typename TIn, bool SWIGLU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1,
+                             const int32_t* __restrict__ offsets, int E, int R, int K, int N,
+                             TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
+                             TIn* __restrict__ save_b, int* status) {
+    constexpr bool TF32 = std::is_same<TIn, float>::value;
+    constexpr int BK = 128 / (int)sizeof(TIn);
+    constexpr int MMA_N = 256;
+    constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
+    constexpr uint32_t IDESC = make_idesc(TF32 ? 2u : 1u, pr::PM, MMA_N);
+    constexpr int STAGES = pr::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* meta = smem + STAGES * pr::STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + pr::NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + pr::NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cid = (int)cluster_id_x(), ncl = (int)ncluster_x();
+
+    // --- tile table of 256-row pair tiles from the routing offsets ---------
+    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int m = 0;
+            if (e < E) {
+                const int cnt = s_off[e + 1] - s_off[e];
+                if (cnt < 0) bad = true;
+                else m = (cnt + pr::PM - 1) / pr::PM;
+            }
+            int tot;
+            const int ex = warp_exclusive_scan(m, &tot);
+            if (e < E) s_toff[e] = carry + ex;
+            carry += tot;
+        }
+        bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
+        if (lane == 0) {
+            s_toff[E] = carry;
+            *s_bad = bad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    // both CTAs of a pair see the same offsets, so they leave here together
+    if (*s_bad) {
+        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+        return;
+    }
+    const int NB = N / OUT_N;
+    const int total = s_toff[E] * NB;
+    if (cid >= total) return;
+    const int KB = K / BK;
+
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(tfull + b), 1);
+            mbar_init(smem_u32(tempty + b), 2 * EPI_WARPS);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmA);
+        prefetch_map(&tmB0);
+        if (SWIGLU) prefetch_map(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(s_tmem), 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const uint32_t leader_full = map_to_cta(smem_u32(full), 0);
+    const uint32_t leader_tempty = map_to_cta(smem_u32(tempty), 0);
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int t = cid; t < total && ok; t += ncl) {
+            const int q = t / NB;
+            int lo = 0, hi = E - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_toff[mid] <= q) lo = mid;
+                else hi = mid - 1;
+            }
+            const int Me = s_toff[lo + 1] - s_toff[lo];
+            const int l = t - s_toff[lo] * NB;
+            const int nb = l / Me, m = l - nb * Me;
+            const int arow = s_off[lo] + m * pr::PM + (int)rank * BM;
+            const int n0 = nb * OUT_N;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = leader_full + (uint32_t)stage * 8u;
+                if (rank == 0) mbar_expect_tx(smem_u32(full + stage), 2 * pr::STAGE_BYTES);
+                const uint32_t sa = smem_u32(smem + stage * pr::STAGE_BYTES);
+                tma_load_2d_pair(sa, &tmA, fb, kb * BK, arow);
+                if (SWIGLU)
+                    tma_load_3d_pair(sa + pr::A_BYTES, rank == 0 ? &tmB0 : &tmB1, fb, kb * BK, n0, lo);
+                else
+                    tma_load_3d_pair(sa + pr::A_BYTES, &tmB0, fb, kb * BK, n0 + (int)rank * 128, lo);
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            // the leader's stage barriers count both CTAs' copies: wait there
+            // (bounded); the partner gives its copies a bounded grace period
+            if (rank == 0) {
+                for (int s = 0; s < STAGES; ++s)
+                    if ((issued_mask >> s) & 1u) {
+                        volatile int no_abort = 0;
+                        mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                                  DRAIN_LIMIT_NS);
+                    }
+            } else {
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 1000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------ MMA issuer (leader)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int i = 0;
+        for (int t = cid; t < total && ok; t += ncl, ++i) {
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + stage * pr::STAGE_BYTES);
+                const uint64_t ad = sw128_desc(sa);
+                const uint64_t bd = sw128_desc(sa + pr::A_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc_mma_pair(dt, ad + 2 * ks, bd + 2 * ks, IDESC, (kb | ks) != 0);
+                tc_commit_pair(smem_u32(empty + stage), 0x3);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit_pair(smem_u32(tfull + buf), 0x3);
+        }
+        if (!ok) {
+            tc_commit_pair(smem_u32(drain), 0x1);
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int qd = warp & 3;
+        const int c_lo = ((warp - 2) >> 2) * (OUT_N / 64);
+        const int c_hi = c_lo + OUT_N / 64;
+        const int r_in_tile = qd * 32 + lane;
+        int i = 0;
+        for (int t = cid; t < total; t += ncl, ++i) {
+            const int q = t / NB;
+            int lo = 0, hi = E - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_toff[mid] <= q) lo = mid;
+                else hi = mid - 1;
+            }
+            const int Me = s_toff[lo + 1] - s_toff[lo];
+            const int l = t - s_toff[lo] * NB;
+            const int nb = l / Me, m = l - nb * Me;
+            const int row_end = s_off[lo + 1];
+            const int n0 = nb * OUT_N;
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * MMA_N);
+            const int grow = s_off[lo] + m * pr::PM + (int)rank * BM + r_in_tile;
+            const bool valid = grow < row_end;
+            TIn* orow = out + (size_t)(valid ? grow : 0) * ldo + n0;
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; ++c) {
+                uint32_t a[32];
+                float v[32];
+                tmem_ld32(ta + c * 32, a);
+                if constexpr (SWIGLU) {
+                    uint32_t b[32];
+                    tmem_ld32(ta + OUT_N + c * 32, b);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v[j] = silu_mul(__uint_as_float(a[j]), __uint_as_float(b[j]));
+                    if (save_a != nullptr && valid) {
+                        const size_t off = (size_t)grow * ldo + n0 + c * 32;
+                        Store32<TIn>::run(save_a + off, reinterpret_cast<const float*>(a));
+                        Store32<TIn>::run(save_b + off, reinterpret_cast<const float*>(b));
+                    }
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                }
+                if (valid) Store32<TIn>::run(orow + c * 32, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty + (uint32_t)buf * 8u);
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+template <typename TIn, bool SWIGLU>
+static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N,
+                       void* out, int64_t ldo, cudaStream_t st, void* save_a = nullptr,
+                       void* save_b = nullptr) {
+    auto kern = grouped_gemm_pair_kernel<TIn, SWIGLU>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pr::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int out_n = SWIGLU ? 128 : 256;
+    const int64_t max_pairs = (R / pr::PM + E) * (N / out_n);
+    const int64_t pairs = num_sms() / 2;
+    const int npairs = (int)(max_pairs < pairs ? max_pairs : pairs);
+    if (npairs <= 0) return MOE_OK;
+    kern<<<2 * npairs, THREADS, pr::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K,
+                                                      (int)N, static_cast<TIn*>(out), ldo,
+                                                      static_cast<TIn*>(save_a),
+                                                      static_cast<TIn*>(save_b), status_ptr());
+    return launch_status();
+}
+
+// Measured on B200: the pair tile speeds up the down GEMM (olmoe-shaped layer
+// 1071 -> 1143 TFLOP/s) but not gate/up, which already runs at the
+// power-capped clock; with about 256 rows per expert the pair's second half
+// computes many rows it then masks (128-expert sweep: slower). So it is
+// used for the down GEMM when experts average at least 512 rows.
+inline bool use_pair(int64_t R, int64_t E) { return R >= 512 * E; }
+
 static int check_common(const void* A, const void* B, const int32_t* offsets, int64_t E,
                         int64_t R, int64_t d, int64_t F, int dtype) {
     if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
@@ -433,11 +750,17 @@ extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert
     const CUtensorMapDataType dt =
         dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int mma_n = (d % 256 == 0) ? 256 : 128;
+    const bool pair = mma_n == 256 && gg::use_pair(R, E);
     CUtensorMap a, b0;
     if (!gg::make_map_2d(&a, H, dt, es, F, R, gg::BM) ||
-        !gg::make_map_3d(&b0, W2, dt, es, F, d, E, w2_expert_stride, mma_n))
+        !gg::make_map_3d(&b0, W2, dt, es, F, d, E, w2_expert_stride, pair ? 128 : mma_n))
         return MOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
+    if (pair) {
+        if (dtype == MOE_BF16)
+            return gg::launch_pair<__nv_bfloat16, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+        return gg::launch_pair<float, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+    }
     if (dtype == MOE_BF16) {
         if (mma_n == 256)
             return gg::launch<__nv_bfloat16, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);

@@ -43,7 +43,11 @@ def _expert_ref(x, W1, W3, W2, lg, k):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("T,d,F,E,k", [(300, 256, 256, 5, 2), (129, 128, 384, 3, 1),
                                        (700, 512, 128, 16, 4), (5, 256, 128, 4, 2),
-                                       (1000, 384, 256, 7, 3)])
+                                       (1000, 384, 256, 7, 3),
+                                       # at least 512 rows per expert on average: the
+                                       # down GEMM on 256-row CTA-pair tiles (with an
+                                       # empty and a heavy expert, ragged tails)
+                                       (1500, 256, 256, 2, 2), (2100, 512, 384, 4, 3)])
 def test_grouped_swiglu_small(dtype, T, d, F, E, k):
     moe = _moe()
     x, W1, W3, W2, lg = _problem(T, d, F, E, k, dtype, seed=T + d + F)
