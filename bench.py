@@ -517,17 +517,22 @@ def _e2e(moe, w, inp, dev, world, args, backward):
             moe.moe_layer_fwd(x_d, k, W1, W3, W2, logits=lg_d, Wr=Wr, out=lo, save=True)
             moe.moe_layer_bwd(lo, dO_d, k, W1, W3, W2, out=gr)
     else:
-        lo = moe.moe_layer_fwd(x, k, W1, W3, W2, logits=logits, Wr=Wr)
-        res = lo.out
-        run = lambda: moe.moe_layer_fwd(x_d, k, W1, W3, W2, logits=lg_d, Wr=Wr, out=lo)
+        # token slices whose copies overlap the compute (moe_layer_fwd_host)
+        hl = moe.HostLayer(T, w.d, w.E, w.F, k, x.dtype, dev, logits_given=logits is not None,
+                           chunks=args.e2e_chunks)
+        res = hl.res.out
     res_h = torch.empty(res.shape, dtype=res.dtype).pin_memory()
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        if lg_d is not None:
-            lg_d.copy_(lg_h, non_blocking=True)
-        run()
-        res_h.copy_(res, non_blocking=True)
+    if not w.mxfp8 and not backward:
+        def e2e_step():
+            hl(x_h, W1, W3, W2, logits_host=lg_h, Wr=Wr, out_host=res_h)
+    else:
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            if lg_d is not None:
+                lg_d.copy_(lg_h, non_blocking=True)
+            run()
+            res_h.copy_(res, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -542,8 +547,11 @@ def _e2e(moe, w, inp, dev, world, args, backward):
     torch.cuda.synchronize(dev)
     barrier(world)
     ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
-    return {"value": T * world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": res.numel() * res.element_size()}
+    r = {"value": T * world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": res.numel() * res.element_size()}
+    if not w.mxfp8 and not backward:
+        r["pipeline_chunks"] = args.e2e_chunks
+    return r
 
 
 def main(argv=None):
@@ -560,6 +568,8 @@ def main(argv=None):
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide T and E by this factor (profiling a small case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=2,
+                    help="token slices of the host-buffer forward (copies overlap compute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",
                     help="skip nvidia-smi clock sampling (for runs under a profiler)")

@@ -117,6 +117,93 @@ extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
     return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
 }
 
+namespace moe {
+namespace layer {
+
+constexpr int MAX_CHUNKS = 64;
+
+// Events of the host pipeline, created once per device and kept.
+static cudaEvent_t* pipeline_events() {
+    static cudaEvent_t ev[64][2 * MAX_CHUNKS + 2];
+    static bool made[64] = {false};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!made[dev]) {
+        for (int i = 0; i < 2 * MAX_CHUNKS + 2; ++i)
+            if (cudaEventCreateWithFlags(&ev[dev][i], cudaEventDisableTiming) != cudaSuccess)
+                return nullptr;
+        made[dev] = true;
+    }
+    return ev[dev];
+}
+
+}  // namespace layer
+}  // namespace moe
+
+extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
+                                  const float* logits_host, void* out_host, int chunks,
+                                  void* stream, void* stream_h2d, void* stream_d2h) {
+    if (!a || !x_host || !out_host || chunks < 1 || chunks > layer::MAX_CHUNKS) return MOE_ERR_INVALID;
+    if ((a->logits == nullptr) != (logits_host == nullptr)) return MOE_ERR_INVALID;
+    if (a->save_Xe || a->save_H || a->save_A || a->save_B) return MOE_ERR_INVALID;
+    if (stream == stream_h2d || stream == stream_d2h || stream_h2d == stream_d2h)
+        return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->dtype != MOE_BF16 && a->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (a->T == 0) return moe_layer_fwd(a, stream);
+    cudaEvent_t* ev = layer::pipeline_events();
+    if (!ev) return MOE_ERR_CUDA;
+    cudaStream_t sc = as_stream(stream), si = as_stream(stream_h2d), so = as_stream(stream_d2h);
+    const size_t es = a->dtype == MOE_F32 ? 4 : 2;
+    const int64_t T = a->T, d = a->d, E = a->E, k = a->k;
+    const int64_t Tc = (T + chunks - 1) / chunks;
+    // the staging buffers may still be in use by work enqueued on `stream`
+    // before this call: the copy-ins wait for it
+    if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS + 1], sc) != cudaSuccess ||
+        cudaStreamWaitEvent(si, ev[2 * layer::MAX_CHUNKS + 1], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int n = 0;
+    for (int64_t t0 = 0; t0 < T; t0 += Tc, ++n) {
+        const int64_t tn = (T - t0 < Tc) ? T - t0 : Tc;
+        const size_t xoff = (size_t)t0 * d * es, xbytes = (size_t)tn * d * es;
+        char* xd = static_cast<char*>(const_cast<void*>(a->x)) + xoff;
+        if (cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + xoff, xbytes,
+                            cudaMemcpyHostToDevice, si) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        float* ld = nullptr;
+        if (a->logits) {
+            ld = const_cast<float*>(a->logits) + (size_t)t0 * E;
+            if (cudaMemcpyAsync(ld, logits_host + (size_t)t0 * E, (size_t)tn * E * sizeof(float),
+                                cudaMemcpyHostToDevice, si) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
+        if (cudaEventRecord(ev[2 * n], si) != cudaSuccess || cudaStreamWaitEvent(sc, ev[2 * n], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        moe_layer_args s = *a;
+        s.T = tn;
+        s.x = xd;
+        s.logits = ld;
+        s.out = static_cast<char*>(a->out) + xoff;
+        s.idx = a->idx + (size_t)t0 * k;
+        s.gate = a->gate + (size_t)t0 * k;
+        s.slot = a->slot + (size_t)t0 * k;
+        const int rc = moe_layer_fwd(&s, stream);
+        if (rc != MOE_OK) return rc;
+        if (cudaEventRecord(ev[2 * n + 1], sc) != cudaSuccess ||
+            cudaStreamWaitEvent(so, ev[2 * n + 1], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaMemcpyAsync(static_cast<char*>(out_host) + xoff, s.out, xbytes,
+                            cudaMemcpyDeviceToHost, so) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS], so) != cudaSuccess ||
+        cudaStreamWaitEvent(sc, ev[2 * layer::MAX_CHUNKS], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 extern "C" size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype) {
     if (T < 0 || d <= 0 || F <= 0 || k <= 0) return 0;
     const size_t es = dtype == MOE_F32 ? 4 : 2;

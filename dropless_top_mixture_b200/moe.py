@@ -113,6 +113,7 @@ _SIGS = {
     "moe_layer_fwd_mxfp8": (_i32, [ctypes.POINTER(LayerMxArgs), _p]),
     "moe_layer_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32, _i32]),
     "moe_layer_fwd": (_i32, [ctypes.POINTER(LayerArgs), _p]),
+    "moe_layer_fwd_host": (_i32, [ctypes.POINTER(LayerArgs), _p, _p, _p, _i32, _p, _p, _p]),
     "moe_layer_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32]),
     "moe_layer_bwd": (_i32, [ctypes.POINTER(LayerBwdArgs), _p]),
     "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
@@ -423,6 +424,61 @@ def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool =
     rc = lib.moe_layer_fwd(ctypes.byref(a), _stream(x))
     _check("moe_layer_fwd", rc)
     return out
+
+
+class HostLayer:
+    """moe_layer_fwd_host: the layer from pinned host x (and logits) to
+    pinned host out, cut into `chunks` token slices whose copy-in, compute
+    and copy-out overlap. Holds the device staging buffers, the routing
+    outputs (idx, gate, slot for every token) and the two copy streams, so
+    repeated calls of one shape allocate nothing."""
+
+    def __init__(self, T: int, d: int, E: int, F: int, k: int, dtype: torch.dtype, device,
+                 *, logits_given: bool, chunks: int = 2):
+        if not 1 <= chunks <= 64:
+            raise ValueError("chunks must be in [1, 64]")
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.T, self.d, self.E, self.F, self.k, self.dtype = T, d, E, F, k, dtype
+        self.chunks = chunks
+        self.x = torch.empty((T, d), dtype=dtype, device=dev)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_given else None
+        self.res = LayerOut(out=torch.empty((T, d), dtype=dtype, device=dev),
+                            idx=torch.empty((T, k), **i32),
+                            gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                            counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                            slot=torch.empty((T, k), **i32),
+                            workspace=_alloc_ws(moe_layer_workspace_size(
+                                T, d, E, F, k, dtype, logits_given), dev))
+        self.s_h2d = torch.cuda.Stream(dev)
+        self.s_d2h = torch.cuda.Stream(dev)
+
+    def __call__(self, x_host: torch.Tensor, W1, W3, W2, *, logits_host=None, Wr=None,
+                 renorm: bool = False, out_host: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if x_host.is_cuda or tuple(x_host.shape) != (self.T, self.d) or x_host.dtype != self.dtype:
+            raise ValueError("x_host must be a [T, d] host tensor of the layer's dtype")
+        if (logits_host is None) != (self.logits is None):
+            raise ValueError("logits_host must be given exactly when the layer was built for it")
+        if logits_host is not None and (logits_host.is_cuda or logits_host.dtype != torch.float32
+                                        or tuple(logits_host.shape) != (self.T, self.E)):
+            raise ValueError("logits_host must be a [T, E] fp32 host tensor")
+        if out_host is None:
+            out_host = torch.empty((self.T, self.d), dtype=self.dtype, pin_memory=True)
+        E, F, _, s13 = _w13(W1, W3)
+        r = self.res
+        a = LayerArgs(T=self.T, d=self.d, E=E, F=F, k=self.k, dtype=_dtype_code(self.dtype),
+                      renorm=int(renorm), reserved0=0, x=_ptr(self.x), logits=_ptr(self.logits),
+                      Wr=_ptr(Wr), W1=_ptr(W1), W3=_ptr(W3), W2=_ptr(W2),
+                      w13_expert_stride=s13, w2_expert_stride=W2.stride(0), out=_ptr(r.out),
+                      idx=_ptr(r.idx), gate=_ptr(r.gate), counts=_ptr(r.counts),
+                      offsets=_ptr(r.offsets), slot=_ptr(r.slot), workspace=_ptr(r.workspace),
+                      workspace_bytes=r.workspace.numel(), save_Xe=None, save_H=None,
+                      save_A=None, save_B=None)
+        rc = lib.moe_layer_fwd_host(ctypes.byref(a), x_host.data_ptr(), _ptr(logits_host),
+                                    out_host.data_ptr(), self.chunks, _stream(self.x),
+                                    self.s_h2d.cuda_stream, self.s_d2h.cuda_stream)
+        _check("moe_layer_fwd_host", rc)
+        return out_host
 
 
 @dataclass

@@ -351,6 +351,30 @@ MOE_API size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int64_t
 MOE_API int moe_layer_fwd(const moe_layer_args* args, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_layer_fwd_host — moe_layer_fwd from and to host memory, with the
+ * copies overlapped with compute. The layer is token-wise, so the batch is
+ * cut into `chunks` consecutive token slices (<= 64): slice c is copied in
+ * on `stream_h2d`, computed on `stream`, and copied out on `stream_d2h`, so
+ * the copy-in of slice c+1 and the copy-out of slice c-1 run while slice c
+ * computes. Every token's output equals moe_layer_fwd's bit for bit.
+ *   args        as for moe_layer_fwd; args->x (and args->logits) and
+ *               args->out are device staging buffers for the whole batch
+ *               ([T,d], [T,E], [T,d]); idx, gate and slot receive the
+ *               per-token results (slot indexes the slice's own buffers);
+ *               counts and offsets hold the last slice's.
+ *   x_host      [T,d] host (pinned for asynchronous copies)
+ *   logits_host [T,E] fp32 host, or NULL when args->logits is NULL
+ *   out_host    [T,d] host
+ *   stream, stream_h2d, stream_d2h  three distinct streams; when the call
+ *               returns, `stream` is ordered after the last copy-out.
+ * The first call on a device creates the events the pipeline uses (kept
+ * for the life of the process). No save_* buffers in this mode.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_layer_fwd_host(const moe_layer_args* args, const void* x_host,
+                               const float* logits_host, void* out_host, int chunks,
+                               void* stream, void* stream_h2d, void* stream_d2h);
+
+/* ------------------------------------------------------------------------
  * moe_layer_bwd — backward of moe_layer_fwd with the gates held constant:
  *   dYe[slot[t,j]] = bf16(gate[t,j] * dOut[t])       (moe_dispatch, scaled)
  *   moe_grouped_swiglu_bwd                          -> dXe, dW1, dW3, dW2
