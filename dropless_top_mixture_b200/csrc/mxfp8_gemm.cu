@@ -13,7 +13,8 @@
 //
 // Kernel: tcgen05.mma kind::mxf8f6f4.block_scale, M = 128, N = 128, K = 32 per
 // instruction, 128-byte K slabs staged by TMA with the same 128-byte swizzle
-// as the bf16 kernels. Per slab every row carries 4 UE8M0 scales (one 32-bit
+// as the bf16 kernels, two slabs (8 MMAs) per pipeline stage so the per-stage
+// barrier wait, proxy fence and scale copies are paid once per 256 K. Per slab every row carries 4 UE8M0 scales (one 32-bit
 // word); the producer warp gathers the 128 A words and 128 B words (cp.async,
 // tracked by the stage's mbarrier) into the 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4 copies into TMEM
 // (lane m%32 of every sub-partition, column m/32, byte = K block), and the
@@ -30,15 +31,18 @@ using namespace tc;
 constexpr int BM = 128;
 constexpr int MMA_N = 128;
 constexpr int BK = 128;  // e4m3 elements per 128-byte slab
-constexpr int STAGES = 6;
+constexpr int SLABS = 2; // slabs per pipeline stage (8 MMAs per stage wait)
+constexpr int STAGES = 3;
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * 128;
 constexpr int B_BYTES = MMA_N * 128;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SF_STAGE_BYTES = 1024;  // 512 B of A scale words + 512 B of B scale words
+constexpr int SLAB_BYTES = A_BYTES + B_BYTES;
+constexpr int STAGE_BYTES = SLABS * SLAB_BYTES;
+constexpr int SF_SLAB_BYTES = 1024;   // 512 B of A scale words + 512 B of B scale words
+constexpr int SF_STAGE_BYTES = SLABS * SF_SLAB_BYTES;
 constexpr int TMEM_ALLOC = 512;
-constexpr int SFA_COL = 2 * MMA_N;    // 256
-constexpr int SFB_COL = SFA_COL + 4;  // 260
+constexpr int SFA_COL = 2 * MMA_N;    // 256 (+8 per slab)
+constexpr int SFB_COL = SFA_COL + 4;  // 260 (+8 per slab)
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
 constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + META_BYTES;
@@ -168,8 +172,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int NB = N / OUT_N;
     const int total = s_toff[E] * NB;
     if ((int)blockIdx.x >= total) return;
-    const int KB = K / BK;
-    const int sf_row = K / 32;  // scale bytes per row
+    const int KS = K / BK;                   // 128-byte slabs
+    const int KB = (KS + SLABS - 1) / SLABS;  // pipeline stages per tile
+    const int sf_row = K / 32;               // scale bytes per row
 
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
@@ -215,38 +220,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 const uint32_t fb = smem_u32(full + stage);
-                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-                const uint32_t sb = sa + A_BYTES;
+                const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
                 if (lane == 0) {
-                    mbar_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, fb, kb * BK, tl.row0);
-                    if (SWIGLU) {
-                        tma_load_3d(sb, &tmB0, fb, kb * BK, tl.n0, tl.e);
-                        tma_load_3d(sb + B_BYTES / 2, &tmB1, fb, kb * BK, tl.n0, tl.e);
-                    } else {
-                        tma_load_3d(sb, &tmB0, fb, kb * BK, tl.n0, tl.e);
+                    mbar_expect_tx(fb, (uint32_t)(ns * SLAB_BYTES));
+                    for (int sl = 0; sl < ns; ++sl) {
+                        const int kc = (kb * SLABS + sl) * BK;
+                        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
+                        const uint32_t sb = sa + A_BYTES;
+                        tma_load_2d(sa, &tmA, fb, kc, tl.row0);
+                        if (SWIGLU) {
+                            tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
+                            tma_load_3d(sb + B_BYTES / 2, &tmB1, fb, kc, tl.n0, tl.e);
+                        } else {
+                            tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
+                        }
                     }
                 }
                 // scale words, copied asynchronously: the stage's barrier
                 // completes only once they have landed, so the producer never
                 // waits on their latency
-                const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
+                for (int sl = 0; sl < ns; ++sl) {
+                    const uint32_t sfs =
+                        smem_u32(sf_smem + stage * SF_STAGE_BYTES + sl * SF_SLAB_BYTES);
+                    const int kw = 4 * (kb * SLABS + sl);  // scale byte of the slab's first block
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int m = lane + 32 * j;  // A row within the tile
-                    const int grow = tl.row0 + m;
-                    const bool in = grow < R;
-                    cp_async_word(sfs + (uint32_t)(lane * 4 + j) * 4u,
-                                  sfA + (size_t)(in ? grow : 0) * sf_row + 4 * kb, in ? 4u : 0u);
-                    const uint8_t* bsrc;
-                    if (SWIGLU) {
-                        bsrc = (m < 64 ? sfB0 + (size_t)(tl.n0 + m) * sf_row
-                                       : sfB1 + (size_t)(tl.n0 + m - 64) * sf_row);
-                    } else {
-                        bsrc = sfB0 + (size_t)(tl.n0 + m) * sf_row;
+                    for (int j = 0; j < 4; ++j) {
+                        const int m = lane + 32 * j;  // A row within the tile
+                        const int grow = tl.row0 + m;
+                        const bool in = grow < R;
+                        cp_async_word(sfs + (uint32_t)(lane * 4 + j) * 4u,
+                                      sfA + (size_t)(in ? grow : 0) * sf_row + kw, in ? 4u : 0u);
+                        const uint8_t* bsrc;
+                        if (SWIGLU) {
+                            bsrc = (m < 64 ? sfB0 + (size_t)(tl.n0 + m) * sf_row
+                                           : sfB1 + (size_t)(tl.n0 + m - 64) * sf_row);
+                        } else {
+                            bsrc = sfB0 + (size_t)(tl.n0 + m) * sf_row;
+                        }
+                        cp_async_word(sfs + 512u + (uint32_t)(lane * 4 + j) * 4u,
+                                      bsrc + (size_t)tl.e * sfb_expert_stride + kw, 4u);
                     }
-                    cp_async_word(sfs + 512u + (uint32_t)(lane * 4 + j) * 4u,
-                                  bsrc + (size_t)tl.e * sfb_expert_stride + 4 * kb, 4u);
                 }
                 cp_async_arrive(fb);
                 issued_mask |= 1u << stage;
@@ -290,16 +303,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_after();
                 fence_proxy_async_smem();  // scale words came through the generic proxy
+                const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
-                tmem_cp_sf(sfa_t, sf_desc(sfs));
-                tmem_cp_sf(sfb_t, sf_desc(sfs + 512));
-                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-                const uint64_t ad = sw128_desc(sa);
-                const uint64_t bd = sw128_desc(sa + A_BYTES);
+                for (int sl = 0; sl < ns; ++sl) {
+                    tmem_cp_sf(sfa_t + 8u * sl, sf_desc(sfs + sl * SF_SLAB_BYTES));
+                    tmem_cp_sf(sfb_t + 8u * sl, sf_desc(sfs + sl * SF_SLAB_BYTES + 512));
+                }
+                for (int sl = 0; sl < ns; ++sl) {
+                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
+                    const uint64_t ad = sw128_desc(sa);
+                    const uint64_t bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_mx(dt, ad + 2 * ks, bd + 2 * ks, mx_idesc(ks), sfa_t | ((uint32_t)ks << 30),
-                           sfb_t | ((uint32_t)ks << 30), (kb | ks) != 0);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_mx(dt, ad + 2 * ks, bd + 2 * ks, mx_idesc(ks),
+                               (sfa_t + 8u * sl) | ((uint32_t)ks << 30),
+                               (sfb_t + 8u * sl) | ((uint32_t)ks << 30), (kb | sl | ks) != 0);
+                }
                 tc_commit(smem_u32(empty + stage));
                 if (++stage == STAGES) {
                     stage = 0;

@@ -61,6 +61,45 @@ def test_grouped_swiglu_small(dtype, T, d, F, E, k):
     assert_close_scaled(np64(Ye), Ye_ref, "Ye")
 
 
+# expert row counts whose last 128-row tile holds 1, 15, 16, 17, 31, 33, 64,
+# 127, 128 (full) or 0 (empty expert) rows, several experts spanning more
+# than one tile
+TAIL_COUNTS = [1, 15, 16, 17, 31, 33, 127, 128, 129, 200, 0, 255, 257, 64, 384, 3]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("d,F", [(256, 256), (384, 128), (512, 384)])
+def test_grouped_swiglu_every_tail_size(dtype, d, F):
+    """Expert segments given directly by offsets, so every ragged tail size
+    (the operand-swapped tail tiles) is met; A, B and H kept for the
+    backward are checked too."""
+    moe = _moe()
+    counts = np.array(TAIL_COUNTS, dtype=np.int64)
+    E, R = len(counts), int(counts.sum())
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    g = torch.Generator().manual_seed(d + F)
+    Xe = torch.randn(R, d, generator=g).to(dtype)
+    W1 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(dtype)
+    W3 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(dtype)
+    W2 = (torch.randn(E, d, F, generator=g) * F ** -0.5).to(dtype)
+    Ye_ref, A_ref, B_ref, H_ref = O.expert_ffn(np64(Xe), offsets, np64(W1), np64(W3), np64(W2),
+                                               keep=True)
+    dev = "cuda"
+    offs = torch.from_numpy(offsets).to(dev)
+    nan = lambda n: torch.full((R, n), float("nan"), dtype=dtype, device=dev)
+    H, A, B = moe.moe_grouped_gate_up_save(Xe.to(dev), W1.to(dev), W3.to(dev), offs,
+                                           H=nan(F), A=nan(F), B=nan(F))
+    Ye = moe.moe_grouped_down(H, W2.to(dev), offs, Ye=nan(d))
+    assert moe.moe_get_status() == 0
+    assert_close_scaled(np64(A), A_ref, "A")
+    assert_close_scaled(np64(B), B_ref, "B")
+    assert_close_scaled(np64(H), H_ref, "H")
+    assert_close_scaled(np64(Ye), Ye_ref, "Ye")
+    # every row of every expert was written (a missed row stays NaN)
+    for t in (H, A, B, Ye):
+        assert torch.isfinite(t.float()).all()
+
+
 def test_grouped_gate_up_fused_gate_up_layout():
     """W1/W3 as the two halves of one [E, 2F, d] gate_up tensor."""
     moe = _moe()
