@@ -149,6 +149,23 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
     }
 }
 
+// row_token[slot[t,j]] = t: the token whose copy each expert row holds (the
+// inverse of the slot permutation), so a GEMM can fetch its A rows from x.
+__global__ void __launch_bounds__(THREADS) row_token_kernel(const int32_t* __restrict__ slot,
+                                                            int64_t n, int k, int64_t R,
+                                                            int32_t* __restrict__ row_token,
+                                                            int* status) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int s = slot[i];
+        if (s < 0 || s >= R) {
+            set_status(status, MOE_DEVERR_BAD_INDEX);
+            continue;
+        }
+        row_token[s] = (int32_t)(i / k);
+    }
+}
+
 inline int grid_for(int64_t T) {
     const int64_t cap = (int64_t)num_sms() * 8;
     return (int)(T < cap ? T : cap);
@@ -214,5 +231,20 @@ extern "C" int moe_combine(const void* Ye, const int32_t* slot, const float* gat
         else
             dc::combine_kernel<MOE_F32, true><<<grid, dc::THREADS, 0, st>>>(ye, slot, gate, (int)T, k, vpr, R, o, status_ptr());
     }
+    return launch_status();
+}
+
+extern "C" int moe_row_token(const int32_t* slot, int64_t T, int k, int32_t* row_token,
+                             void* stream) {
+    if (T < 0 || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID;
+    if (T == 0) return MOE_OK;
+    if (!slot || !row_token) return MOE_ERR_INVALID;
+    if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    const int64_t n = T * k;
+    int64_t g = (n + dc::THREADS - 1) / dc::THREADS;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (g > cap) g = cap;
+    dc::row_token_kernel<<<(int)g, dc::THREADS, 0, as_stream(stream)>>>(slot, n, k, n, row_token,
+                                                                        status_ptr());
     return launch_status();
 }

@@ -16,8 +16,19 @@
 // columns of B. One 128xMMA_Nx16 MMA per 32 bytes of K; K is staged 128
 // bytes at a time by TMA with the 128-byte swizzle the MMA descriptors read.
 //
+// Gathered A (gate/up only). With GATHER the A operand is not a dispatched
+// Xe buffer: row r of the tile is token row_token[r] of x, fetched by TMA
+// tile::gather4 copies (four rows of one 128-byte K slab each; lane l of
+// the producer warp fetches tile rows 4l..4l+3), so the dispatch copy of x
+// into Xe and its re-read are never made ("olmoforge" README, row-wise
+// expert parallelism: tokens go straight into the expert's input without a
+// separate permutation). Measured on B200 this path is about 3x slower
+// than dispatch + tiled TMA (a 512-byte gather per lane per slab cannot
+// keep the tensor cores fed), so the layer does not use it.
+//
 // Warp roles (320 threads, one CTA per SM):
 //   warp 0, lane 0   TMA producer over a STAGES-deep shared-memory ring
+//                    (GATHER: all of warp 0)
 //   warp 1           allocates TMEM; lane 0 issues tcgen05.mma
 //   warps 2..9       epilogue: tcgen05.ld from TMEM (warp w reads lanes
 //                    32*(w%4).., two warps per quarter split the columns),
@@ -116,14 +127,15 @@ struct Store32<float> {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <typename TIn, bool SWIGLU, int MMA_N>
+template <typename TIn, bool SWIGLU, int MMA_N, bool GATHER = false>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const int32_t* __restrict__ offsets, int E, int R, int K, int N,
                         TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
-                        TIn* __restrict__ save_b, int* status) {
+                        TIn* __restrict__ save_b, int* status,
+                        const int32_t* __restrict__ row_token, int x_rows) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -204,7 +216,75 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
 
-    if (warp == 0 && lane == 0) {
+    if (GATHER && warp == 0) {
+        // ------------------------------------------------ TMA producer, A
+        // rows gathered from x by row_token (whole warp): lane l fetches tile
+        // rows 4l..4l+3 of each K slab with one tile::gather4 copy
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        // this lane's four token rows of the next tile, loaded one tile ahead
+        // so their latency hides behind the current tile's copies; rows past
+        // R (the last tile's overhang) fetch token 0, computed and masked;
+        // a token outside [0, x_rows) is flagged and read as token 0
+        int nxt[4];
+        auto load_rows = [&](int t) {
+            const Tile tn = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = tn.row0 + 4 * lane + j;
+                int tk = r < R ? __ldg(row_token + r) : 0;
+                if ((unsigned)tk >= (unsigned)x_rows) {
+                    set_status(status, MOE_DEVERR_BAD_INDEX);
+                    tk = 0;
+                }
+                nxt[j] = tk;
+            }
+        };
+        load_rows(blockIdx.x);
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
+            const int tok[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+            if (t + (int)gridDim.x < total) load_rows(t + (int)gridDim.x);
+            for (int kb = 0; kb < KB; ++kb) {
+                bool w = true;
+                if (lane == 0)
+                    w = mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status,
+                                  WAIT_LIMIT_NS);
+                if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(full + stage);
+                const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+                const uint32_t sb = sa + C::A_BYTES;
+                if (lane == 0) {
+                    mbar_expect_tx(fb, C::STAGE_BYTES);
+                    tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
+                    tma_load_3d(sb + C::B_BYTES / 2, &tmB1, fb, kb * C::BK, tl.n0, tl.e);
+                    issued_mask |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                }
+                __syncwarp();
+                tma_gather4(sa + (uint32_t)lane * 512u, &tmA, fb, kb * C::BK, tok[0], tok[1],
+                            tok[2], tok[3]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued_mask >> s) & 1u) {
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                              DRAIN_LIMIT_NS);
+                }
+        }
+        __syncwarp();
+    } else if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
         int stage = 0;
         uint32_t phase = 0;
@@ -345,12 +425,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------------------ host
 
-template <typename TIn, bool SWIGLU, int MMA_N>
+template <typename TIn, bool SWIGLU, int MMA_N, bool GATHER = false>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, void* out,
-                  int64_t ldo, cudaStream_t st, void* save_a = nullptr, void* save_b = nullptr) {
+                  int64_t ldo, cudaStream_t st, void* save_a = nullptr, void* save_b = nullptr,
+                  const int32_t* row_token = nullptr, int64_t x_rows = 0) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
-    auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N>;
+    auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N, GATHER>;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -366,7 +447,8 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     if (grid <= 0) return MOE_OK;
     kern<<<grid, THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K, (int)N,
                                               static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a),
-                                              static_cast<TIn*>(save_b), status_ptr());
+                                              static_cast<TIn*>(save_b), status_ptr(), row_token,
+                                              (int)x_rows);
     return launch_status();
 }
 
@@ -735,6 +817,35 @@ extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W
                                    void* stream) {
     return moe_grouped_gate_up_save(Xe, W1, W3, w13_expert_stride, offsets, E, R, d, F, dtype, H,
                                     nullptr, nullptr, stream);
+}
+
+extern "C" int moe_grouped_gate_up_gather(const void* x, const int32_t* row_token, int64_t T,
+                                          const void* W1, const void* W3,
+                                          int64_t w13_expert_stride, const int32_t* offsets,
+                                          int64_t E, int64_t R, int64_t d, int64_t F, int dtype,
+                                          void* H, void* stream) {
+    int rc = gg::check_common(x, W1, offsets, E, R, d, F, dtype);
+    if (rc != MOE_OK) return rc;
+    if (T < 0 || T > INT32_MAX || !row_token) return MOE_ERR_INVALID;
+    if (!W3 || !H || !aligned16(W3) || !aligned16(H)) return MOE_ERR_INVALID;
+    if (w13_expert_stride < F * d && E > 1) return MOE_ERR_INVALID;
+    if (w13_expert_stride % 8 != 0) return MOE_ERR_INVALID;
+    if (R == 0) return MOE_OK;
+    if (T == 0) return MOE_ERR_INVALID;  // R rows but no token to gather
+    const int es = dtype == MOE_F32 ? 4 : 2;
+    const CUtensorMapDataType dt =
+        dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap a, b0, b1;
+    if (!gg::make_map_2d(&a, x, dt, es, d, T, 1) ||  // one row high: gather4 boxes
+        !gg::make_map_3d(&b0, W1, dt, es, d, F, E, w13_expert_stride, 128) ||
+        !gg::make_map_3d(&b1, W3, dt, es, d, F, E, w13_expert_stride, 128))
+        return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (dtype == MOE_BF16)
+        return gg::launch<__nv_bfloat16, true, 256, true>(a, b0, b1, offsets, E, R, d, F, H, F, st,
+                                                           nullptr, nullptr, row_token, T);
+    return gg::launch<float, true, 256, true>(a, b0, b1, offsets, E, R, d, F, H, F, st, nullptr,
+                                              nullptr, row_token, T);
 }
 
 extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,

@@ -96,6 +96,9 @@ _SIGS = {
     "moe_dispatch": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
     "moe_grouped_gate_up": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_grouped_down": (_i32, [_p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
+    "moe_row_token": (_i32, [_p, _i64, _i32, _p, _p]),
+    "moe_grouped_gate_up_gather": (_i32, [_p, _p, _i64, _p, _p, _i64, _p, _i64, _i64, _i64, _i64,
+                                          _i32, _p, _p]),
     "moe_grouped_swiglu": (_i32, [_p, _p, _p, _p, _i64, _i64, _p, _i64, _i64, _i64, _i64, _i32,
                                   _p, _p, _p]),
     "moe_grouped_gate_up_save": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p,
@@ -264,6 +267,30 @@ def moe_grouped_gate_up(Xe, W1, W3, offsets, H: Optional[torch.Tensor] = None) -
     rc = lib.moe_grouped_gate_up(_ptr(Xe), _ptr(W1), _ptr(W3), s13, _ptr(offsets), E, R, d, F,
                                  _dtype_code(Xe.dtype), _ptr(H), _stream(Xe))
     _check("moe_grouped_gate_up", rc)
+    return H
+
+
+def moe_row_token(slot, row_token: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(slot, "slot")
+    T, k = slot.shape
+    if row_token is None:
+        row_token = torch.empty(T * k, dtype=torch.int32, device=slot.device)
+    rc = lib.moe_row_token(_ptr(slot), T, k, _ptr(row_token), _stream(slot))
+    _check("moe_row_token", rc)
+    return row_token
+
+
+def moe_grouped_gate_up_gather(x, row_token, W1, W3, offsets,
+                               H: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(x, "x"); _need(row_token, "row_token"); _need(offsets, "offsets")
+    E, F, d, s13 = _w13(W1, W3)
+    R = row_token.numel()
+    if H is None:
+        H = torch.empty((R, F), dtype=x.dtype, device=x.device)
+    rc = lib.moe_grouped_gate_up_gather(_ptr(x), _ptr(row_token), x.shape[0], _ptr(W1), _ptr(W3),
+                                        s13, _ptr(offsets), E, R, d, F, _dtype_code(x.dtype),
+                                        _ptr(H), _stream(x))
+    _check("moe_grouped_gate_up_gather", rc)
     return H
 
 

@@ -156,6 +156,20 @@ MOE_API int moe_dispatch(const void* x, const int32_t* slot, const float* gate, 
                          int64_t d, int k, int dtype, void* Xe, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_row_token — the inverse of the slot map: row_token[slot[t,j]] = t,
+ * i.e. the token whose copy expert row r holds.
+ *
+ * [OF capability table, row-wise expert parallelism, "免重排" (no separate
+ * permutation)]: with row_token a GEMM can fetch its expert rows straight
+ * from x (moe_grouped_gate_up_gather), so the dispatched copy Xe is never
+ * materialised.
+ *   slot [T,k] from moe_route; row_token [R = T*k] int32 output.
+ * A slot outside [0,R) is skipped and sets MOE_DEVERR_BAD_INDEX.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_row_token(const int32_t* slot, int64_t T, int k, int32_t* row_token,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
  * Grouped SwiGLU expert FFN over variable per-expert row counts.
  *
  * [HF §3]: per expert e, rows r in [offsets[e], offsets[e+1]):
@@ -188,6 +202,20 @@ MOE_API int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, c
                                int64_t w13_expert_stride, int64_t w2_expert_stride,
                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
                                int64_t F, int dtype, void* H, void* Ye, void* stream);
+/* moe_grouped_gate_up with the dispatch folded in: expert row r is token
+ * row_token[r] of x [T,d] (moe_row_token), fetched by TMA row gathers
+ * (tile::gather4, four 128-byte row pieces per copy) into the GEMM's A
+ * tiles, so Xe is never written. H equals moe_grouped_gate_up on
+ * moe_dispatch's Xe bit for bit. A row_token outside [0,T) is read as
+ * token 0 and sets MOE_DEVERR_BAD_INDEX. Limits as moe_grouped_gate_up;
+ * T >= 1 when R > 0. On B200 this is about 3x slower than moe_dispatch +
+ * moe_grouped_gate_up (the row gathers, not the bytes, limit it), so
+ * moe_layer_fwd does not use it. */
+MOE_API int moe_grouped_gate_up_gather(const void* x, const int32_t* row_token, int64_t T,
+                                       const void* W1, const void* W3,
+                                       int64_t w13_expert_stride, const int32_t* offsets,
+                                       int64_t E, int64_t R, int64_t d, int64_t F, int dtype,
+                                       void* H, void* stream);
 /* moe_grouped_gate_up with the pre-activations kept for the backward pass:
  * A_out[r] = Xe[r]·W1_eᵀ and B_out[r] = Xe[r]·W3_eᵀ ([R,F], layer dtype),
  * written by the same epilogue that writes H. Both NULL = moe_grouped_gate_up. */

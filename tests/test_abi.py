@@ -66,8 +66,15 @@ def test_host_validation_rejects_without_launch(lib):
     assert L.moe_combine(p16 + 2, p16, None, 4, 64, 2, m.MOE_BF16, p16, None) == m.MOE_ERR_INVALID
     # MXFP8 columns must be whole blocks
     assert L.mxfp8_quantize(p16, m.MOE_BF16, 4, 48, m.MOE_SCALE_E8M0, p16, p16, None) == m.MOE_ERR_INVALID
+    # gathered gate/up: no row_token, or rows to compute but no token to gather
+    assert L.moe_grouped_gate_up_gather(p16, None, 10, p16, p16, 128 * 128, p16, 4, 20, 128, 128,
+                                        m.MOE_BF16, p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_grouped_gate_up_gather(p16, p16, 0, p16, p16, 128 * 128, p16, 4, 20, 128, 128,
+                                        m.MOE_BF16, p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_row_token(p16, 4, 0, p16, None) == m.MOE_ERR_INVALID
     # T == 0 is a no-op
     assert L.moe_dispatch(p16, p16, None, 0, 64, 2, m.MOE_BF16, p16, None) == m.MOE_OK
+    assert L.moe_row_token(p16, 0, 2, p16, None) == m.MOE_OK
     assert L.moe_layer_fwd(None, None) == m.MOE_ERR_INVALID
 
 

@@ -100,6 +100,71 @@ def test_grouped_swiglu_every_tail_size(dtype, d, F):
         assert torch.isfinite(t.float()).all()
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,d,F,E,k", [(300, 256, 256, 5, 2), (5, 256, 128, 4, 2),
+                                       (1000, 384, 256, 7, 3), (129, 128, 384, 3, 1),
+                                       (2100, 512, 384, 4, 3)])
+def test_gate_up_gather_equals_dispatched(dtype, T, d, F, E, k):
+    """The fused path (row_token + A rows gathered from x by TMA) computes
+    exactly what the dispatch path does: same rows, same MMA order, so H is
+    identical bit for bit; and it matches the oracle."""
+    moe = _moe()
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, dtype, seed=3 * T + d)
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    dev = "cuda"
+    xd, W1d, W3d = x.to(dev), W1.to(dev), W3.to(dev)
+    slot = torch.from_numpy(meta["slot"]).to(dev)
+    offs = torch.from_numpy(meta["offsets"]).to(dev)
+    rt = moe.moe_row_token(slot)
+    want_rt = np.empty(T * k, np.int32)
+    want_rt[meta["slot"].reshape(-1)] = np.repeat(np.arange(T, dtype=np.int32), k)
+    assert np.array_equal(rt.cpu().numpy(), want_rt)
+    Hg = moe.moe_grouped_gate_up_gather(xd, rt, W1d, W3d, offs)
+    Hd = moe.moe_grouped_gate_up(moe.moe_dispatch(xd, slot), W1d, W3d, offs)
+    assert moe.moe_get_status() == 0
+    assert torch.equal(Hg, Hd)
+    Xe = O.dispatch(x.double().numpy(), meta["slot"])
+    _, _, _, H_ref = O.expert_ffn(Xe, meta["offsets"], np64(W1), np64(W3), np64(W2), keep=True)
+    assert_close_scaled(np64(Hg), H_ref, "H gathered")
+
+
+def test_gate_up_gather_flags_bad_token():
+    """A row_token outside [0, T) is never used as an address: that row is
+    computed from token 0 and the status word says so; the other rows are
+    unaffected."""
+    moe = _moe()
+    T, d, F, E, k = 64, 256, 128, 4, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=11)
+    idx, gate, _ = O.route(lg, k)
+    meta = O.routing_metadata(idx, E)
+    dev = "cuda"
+    xd, W1d, W3d = x.to(dev), W1.to(dev), W3.to(dev)
+    slot = torch.from_numpy(meta["slot"]).to(dev)
+    offs = torch.from_numpy(meta["offsets"]).to(dev)
+    rt = moe.moe_row_token(slot)
+    good = moe.moe_grouped_gate_up_gather(xd, rt, W1d, W3d, offs)
+    bad_rt = rt.clone()
+    bad_rt[5] = T + 5
+    bad_rt[9] = -1
+    H = moe.moe_grouped_gate_up_gather(xd, bad_rt, W1d, W3d, offs)
+    assert moe.moe_get_status(clear=True) & moe.MOE_DEVERR_BAD_INDEX
+    keep = torch.ones(T * k, dtype=torch.bool, device=dev)
+    keep[5] = keep[9] = False
+    assert torch.equal(H[keep], good[keep])
+    assert moe.moe_get_status() == 0
+
+
+def test_row_token_flags_bad_slot():
+    moe = _moe()
+    slot = torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda")  # 9 >= R = 4
+    rt = torch.full((4,), -7, dtype=torch.int32, device="cuda")
+    moe.moe_row_token(slot, rt)
+    assert moe.moe_get_status(clear=True) & moe.MOE_DEVERR_BAD_INDEX
+    assert rt.cpu().tolist() == [0, 0, 1, -7]
+    assert moe.moe_get_status() == 0
+
+
 def test_grouped_gate_up_fused_gate_up_layout():
     """W1/W3 as the two halves of one [E, 2F, d] gate_up tensor."""
     moe = _moe()
