@@ -554,6 +554,70 @@ def moe_layer_bwd_sampled(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W
 
 
 # --------------------------------------------------------------------------
+# f2: router backward and the load-balancing auxiliary loss
+#     [HF §2 router (fp32 softmax, top-k, optional norm_topk_prob);
+#      HF §4 "负载均衡辅助损失": Switch-Transformer-style loss from the
+#      per-expert assignment frequency and the routing probability
+#      distribution, multiplied and summed; router_aux_loss_coef (0.01 by
+#      default) scales it into the total loss]
+# --------------------------------------------------------------------------
+
+def aux_loss(logits: np.ndarray, idx: np.ndarray) -> float:
+    """aux = E * sum_e f_e * P_e with f_e = (number of (t, j) routed to e) / T
+    and P_e = mean over tokens of softmax(logits_t)_e. Reading: every one of a
+    token's k choices counts toward f (so a uniform router gives aux = k),
+    and the factor E is Switch Transformer's expert-count scaling."""
+    T, E = np.asarray(logits).shape
+    p = softmax_fp64(logits)
+    f = np.bincount(np.asarray(idx).reshape(-1), minlength=E).astype(np.float64) / T
+    P = p.mean(axis=0)
+    return float(E * (f * P).sum())
+
+
+def gate_grad(dOut: np.ndarray, Y: np.ndarray) -> np.ndarray:
+    """dgate[t, j] = <dOut[t], Y[t, j]>, Y[t, j] = the j-th chosen expert's
+    output for token t (before gating): the gradient of out[t] = sum_j
+    gate[t, j] Y[t, j] with respect to the gate."""
+    return np.einsum("td,tjd->tj", np.asarray(dOut, np.float64), np.asarray(Y, np.float64))
+
+
+def router_grad(logits: np.ndarray, idx: np.ndarray, dgate: np.ndarray, renorm: bool = False,
+                aux_coef: float = 0.0) -> np.ndarray:
+    """dlogits [T,E] for a loss L(gates) + aux_coef * aux_loss, with the top-k
+    choice and the counts held fixed (both are piecewise constant).
+
+    gate[t,j] = p[t, idx[t,j]] (renorm: divided by S_t = sum_j p[t, idx[t,j]]),
+    p = softmax(logits[t]). Chain rule: the gradient reaching p,
+      dp[t,e] = sum_j [idx[t,j] = e] dsel[t,j] + aux_coef * E * f_e / T,
+      dsel = dgate (renorm: (dgate - sum_i gate_i dgate_i) / S_t),
+    then the softmax Jacobian: dlogits = p * (dp - sum_e p dp)."""
+    p = softmax_fp64(logits)
+    T, E = p.shape
+    idx = np.asarray(idx).astype(np.int64)
+    dg = np.asarray(dgate, np.float64)
+    if renorm:
+        sel = np.take_along_axis(p, idx, axis=1)
+        S = sel.sum(axis=1, keepdims=True)
+        g = sel / S
+        dsel = (dg - (g * dg).sum(axis=1, keepdims=True)) / S
+    else:
+        dsel = dg
+    dp = np.zeros((T, E))
+    for j in range(idx.shape[1]):
+        dp[np.arange(T), idx[:, j]] += dsel[:, j]
+    if aux_coef:
+        f = np.bincount(idx.reshape(-1), minlength=E).astype(np.float64) / T
+        dp += aux_coef * E * f / T
+    return p * (dp - (p * dp).sum(axis=1, keepdims=True))
+
+
+def router_linear_grad(dlogits: np.ndarray, x, Wr):
+    """logits = x Wr^T: dx = dlogits Wr [T,d], dWr = dlogits^T x [E,d]."""
+    dl = np.asarray(dlogits, np.float64)
+    return dl @ to64(Wr), dl.T @ to64(x)
+
+
+# --------------------------------------------------------------------------
 # error measures used by the parity tests
 # --------------------------------------------------------------------------
 

@@ -392,3 +392,150 @@ def test_sampled_backward_matches_full_backward():
         for n, g in zip(("dW1", "dW3", "dW2"), smp["dW"][e]):
             assert np.allclose(g, full[n][e], rtol=1e-12, atol=1e-13)
     assert np.all(smp["dW"][4][0] == 0)  # expert 4 has no rows
+
+
+# ------------------------------------------- f2: router backward, aux loss
+
+def _grid_logits(T, E, seed):
+    """Logits on a 2^-10 grid in [-4, 4): exact in fp32, and so are their
+    perturbations by 2^-12, so finite differences see the fp32 softmax
+    input move by exactly eps."""
+    rng = np.random.default_rng(seed)
+    return (rng.integers(-4096, 4096, size=(T, E)) / 1024.0).astype(np.float32)
+
+
+def _expert_rows(x, idx, W1, W3, W2):
+    """Y[t, j] = FFN_{idx[t,j]}(x_t), the un-gated expert outputs."""
+    T, k = idx.shape
+    x64 = O.to64(x)
+    Y = np.zeros((T, k, x64.shape[1]))
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            a = O.to64(W1[e]) @ x64[t]
+            b = O.to64(W3[e]) @ x64[t]
+            Y[t, j] = O.to64(W2[e]) @ (O.silu(a) * b)
+    return Y
+
+
+def test_aux_loss_closed_forms():
+    T, E, k = 64, 8, 2
+    rng = np.random.default_rng(0)
+    # a uniform router gives aux = k whatever the counts (sum_e f_e = k)
+    flat = np.zeros((T, E), np.float32)
+    assert O.aux_loss(flat, O.topk_select(flat, k)) == pytest.approx(k, rel=1e-12)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    assert O.aux_loss(flat, idx) == pytest.approx(k, rel=1e-12)
+    # exactly balanced counts give aux = k whatever the probabilities
+    bal = np.array([[(2 * t) % E, (2 * t + 1) % E] for t in range(T)], np.int32)
+    assert np.all(np.bincount(bal.ravel(), minlength=E) == T * k // E)
+    assert O.aux_loss(rng.normal(size=(T, E)).astype(np.float32), bal) == pytest.approx(k, rel=1e-12)
+    # a collapsed router (every token picks the same k experts, probability
+    # 1/k on each) gives aux = E
+    col = np.zeros((T, E), np.float32)
+    col[:, :k] = 60.0
+    assert O.aux_loss(col, O.topk_select(col, k)) == pytest.approx(E, rel=1e-12)
+
+
+def test_gate_grad_finite_differences():
+    rng = np.random.default_rng(1)
+    T, k, d = 5, 3, 7
+    Y = rng.normal(size=(T, k, d))
+    dOut = rng.normal(size=(T, d))
+    g = rng.random((T, k))
+    L = lambda gg: float((dOut * np.einsum("tj,tjd->td", gg, Y)).sum())
+    got = O.gate_grad(dOut, Y)
+    for t, j in itertools.product(range(T), range(k)):
+        e = np.zeros((T, k)); e[t, j] = 1.0
+        assert got[t, j] == pytest.approx(L(g + e) - L(g), rel=1e-9, abs=1e-12)
+
+
+@pytest.mark.parametrize("renorm", [False, True])
+@pytest.mark.parametrize("aux_coef", [0.0, 0.37])
+def test_router_grad_finite_differences_through_the_layer(renorm, aux_coef):
+    """dlogits of <dOut, out(logits)> + aux_coef * aux(logits) by central
+    differences of the oracle layer itself (top-k choice and counts fixed:
+    the logits are far from ties, and eps is small)."""
+    T, d, E, k, F = 6, 8, 5, 2, 6
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W3 = torch.randn(E, F, d, generator=g, dtype=torch.float64) * 0.3
+    W2 = torch.randn(E, d, F, generator=g, dtype=torch.float64) * 0.3
+    dOut = np.random.default_rng(6).normal(size=(T, d))
+    lg = _grid_logits(T, E, 7)
+    idx0 = O.topk_select(lg, k)
+
+    def loss(l):
+        assert np.array_equal(O.topk_select(l, k), idx0)
+        out = O.moe_layer(x, k, W1, W3, W2, logits=l, renorm=renorm)["out"]
+        return float((dOut * out).sum()) + aux_coef * O.aux_loss(l, idx0)
+
+    Y = _expert_rows(x, idx0, W1, W3, W2)
+    got = O.router_grad(lg, idx0, O.gate_grad(dOut, Y), renorm=renorm, aux_coef=aux_coef)
+    eps = 2.0 ** -12
+    fd = np.zeros((T, E))
+    for t, e in itertools.product(range(T), range(E)):
+        lp, lm = lg.copy(), lg.copy()
+        lp[t, e] += eps
+        lm[t, e] -= eps
+        fd[t, e] = (loss(lp) - loss(lm)) / (2 * eps)
+    assert np.abs(got - fd).max() <= 1e-6 * max(1.0, np.abs(fd).max())
+    assert np.abs(got).max() > 1e-3   # not vacuous
+
+
+@pytest.mark.parametrize("renorm", [False, True])
+def test_router_grad_matches_torch_autograd(renorm):
+    T, E, k = 40, 9, 3
+    lg = np.random.default_rng(8).normal(size=(T, E)).astype(np.float32)
+    dg = np.random.default_rng(9).normal(size=(T, k))
+    idx = O.topk_select(lg, k)
+    c = 0.21
+    L = torch.tensor(lg.astype(np.float64), requires_grad=True)
+    p = torch.softmax(L, dim=1)
+    sel = torch.gather(p, 1, torch.as_tensor(idx, dtype=torch.long))
+    if renorm:
+        sel = sel / sel.sum(dim=1, keepdim=True)
+    f = torch.bincount(torch.as_tensor(idx.ravel(), dtype=torch.long), minlength=E).double() / T
+    total = (sel * torch.as_tensor(dg)).sum() + c * E * (f * p.mean(dim=0)).sum()
+    total.backward()
+    got = O.router_grad(lg, idx, dg, renorm=renorm, aux_coef=c)
+    assert np.allclose(got, L.grad.numpy(), rtol=1e-10, atol=1e-13)
+
+
+def test_router_grad_closed_forms():
+    T, E = 30, 6
+    rng = np.random.default_rng(10)
+    lg = rng.normal(size=(T, E)).astype(np.float32)
+    # k = E, the same upstream gradient on every gate: the gates are the whole
+    # softmax, whose outputs sum to 1, so the logits get no gradient
+    idx = O.topk_select(lg, E)
+    assert np.abs(O.router_grad(lg, idx, np.full((T, E), 0.7))).max() < 1e-15
+    # renormalised gates are invariant to a common shift of the chosen
+    # logits' probabilities' scale: k = E renorm equals plain softmax
+    dg = rng.normal(size=(T, E))
+    assert np.allclose(O.router_grad(lg, idx, dg, renorm=True), O.router_grad(lg, idx, dg),
+                       rtol=1e-12, atol=1e-15)
+    # the aux term alone vanishes for a uniform router with balanced counts
+    flat = np.zeros((T, E), np.float32)
+    bal = np.array([[t % E, (t + 1) % E] for t in range(T)], np.int32)
+    assert np.abs(O.router_grad(flat, bal, np.zeros((T, 2)), aux_coef=1.0)).max() < 1e-15
+
+
+def test_router_linear_grad_finite_differences():
+    """logits = x Wr^T is linear in each operand, so a unit step gives the
+    exact derivative (no truncation error)."""
+    T, d, E = 5, 7, 3
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(E, d))
+    G = rng.normal(size=(T, E))
+    L = lambda xx, ww: float((G * (xx @ ww.T)).sum())
+    dx, dWr = O.router_linear_grad(G, x, Wr)
+    assert dx.shape == (T, d) and dWr.shape == (E, d)
+    for t, c in itertools.product(range(T), range(d)):
+        e = np.zeros((T, d)); e[t, c] = 1.0
+        assert dx[t, c] == pytest.approx(L(x + e, Wr) - L(x, Wr), rel=1e-9, abs=1e-12)
+    for r, c in itertools.product(range(E), range(d)):
+        e = np.zeros((E, d)); e[r, c] = 1.0
+        assert dWr[r, c] == pytest.approx(L(x, Wr + e) - L(x, Wr), rel=1e-9, abs=1e-12)
