@@ -274,8 +274,10 @@ def _steps(moe, w, inp, dev, backward):
                    gate=torch.empty((T, k), dtype=torch.float32, device=dev),
                    counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
                    slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
-    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router)), dtype=torch.uint8,
-                      device=dev)
+    if use_router and backward:
+        rt.logits = torch.empty((T, E), dtype=torch.float32, device=dev)  # kept for the router bwd
+    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router and not backward)),
+                      dtype=torch.uint8, device=dev)
     out = torch.empty((T, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
     Ye = torch.empty((R, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
 
@@ -329,6 +331,26 @@ def _steps(moe, w, inp, dev, backward):
                     ("bwd_gemms", lambda: moe.moe_grouped_swiglu_bwd(Xe, A, B, H, dYe, W1, W3, W2,
                                                                      rt.offsets, out=grads)),
                     ("bwd_combine", lambda: moe.moe_combine(grads.dXe, rt.slot, None, out=dx))]
+            # router backward: the load-balancing loss (coefficient 0.01, the
+            # OLMoE default), the gates through the softmax, and the router
+            # GEMM when the logits come from x and Wr
+            lg_src = rt.logits if use_router else logits
+            aux = torch.empty(1, dtype=torch.float32, device=dev)
+            aux_ws = torch.empty(moe.lib.moe_aux_loss_workspace_size(T, E), dtype=torch.uint8,
+                                 device=dev)
+            rg = moe.RouterGrads(dgate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                                 dlogits=torch.empty((T, E), dtype=torch.float32, device=dev))
+            fns += [("aux_loss", lambda: moe.moe_aux_loss(lg_src, rt.counts, out=aux,
+                                                          workspace=aux_ws)),
+                    ("router_bwd", lambda: moe.moe_router_bwd(
+                        dOut, Ye, rt.slot, rt.idx, lg_src, rt.counts, aux_coef=0.01,
+                        dgate=rg.dgate, dlogits=rg.dlogits))]
+            if use_router:
+                dWr = torch.empty((E, d), dtype=dt, device=dev)
+                lin_ws = torch.empty(moe.lib.moe_router_linear_bwd_workspace_size(T, d, E),
+                                     dtype=torch.uint8, device=dev)
+                fns += [("router_linear_bwd", lambda: moe.moe_router_linear_bwd(
+                    rg.dlogits, x, Wr, dx=dx, dWr=dWr, workspace=lin_ws))]
 
     def step(ev=None):
         for j, (_, fn) in enumerate(fns):
@@ -353,7 +375,13 @@ def _steps(moe, w, inp, dev, backward):
         work["bwd_dispatch"] = (0.0, T * d * es + R * d * es + R * 8)
         work["bwd_gemms"] = (12.0 * R * d * F, 6 * wbytes + R * (5 * d + 5 * F) * es)
         work["bwd_combine"] = (0.0, R * d * es + T * d * es + R * 4)
-    kernels = (4 if use_router else 3) + 4 + (7 if backward else 0)
+        work["aux_loss"] = (0.0, T * E * 4 + E * 4)
+        work["router_bwd"] = (0.0, T * d * es + R * d * es + 2 * T * E * 4 + 3 * R * 4)
+        # dx += dlogits Wr and dWr = dlogits^T x: two T x E x d products
+        work["router_linear_bwd"] = (4.0 * T * E * d, T * E * 4 + E * d * es + 3 * T * d * es
+                                     + E * d * es)
+    kernels = ((4 if use_router else 3) + 4
+               + ((7 + 2 + 1 + (3 if use_router else 0)) if backward else 0))
     return [n for n, _ in fns], step, kernels, work, e_act
 
 
@@ -373,6 +401,8 @@ def run_ours(args):
     backward = bool(args.backward)
     if backward and (w.mxfp8 or w.dtype != "bf16"):
         raise SystemExit("--backward runs on the bf16 workloads")
+    if backward and not w.backward:
+        w = w.scaled(name=w.name, backward=True)  # adds the upstream gradient dOut
     inp = make_inputs(w, dev)
     T, d, E, k, F, R = w.T, w.d, w.E, w.k, w.F, w.R
     parts, step, kernels_per_step, work, e_act = _steps(moe, w, inp, dev, backward)
@@ -461,7 +491,8 @@ def run_ours(args):
                 "algorithmic_per_launch": f"{byts:.4g} bytes (operands once, outputs once)"}
     roof["kernel"] = {"gate_up": "grouped gate_up GEMM + SwiGLU (tcgen05)",
                       "down": "grouped down GEMM (tcgen05)",
-                      "bwd_gemms": "grouped backward GEMMs dH/dX/dW (tcgen05)"}[dom]
+                      "bwd_gemms": "grouped backward GEMMs dH/dX/dW (tcgen05)",
+                      "router_linear_bwd": "router GEMM backward (CUDA cores)"}[dom]
     roof["ridge_flop_per_byte"] = ridge
     roof["traffic"] = recorded_traffic(dom, w.name)
     ffn_t = (per["gate_up"] + per["down"]) / 1e3

@@ -101,20 +101,21 @@ extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
     }
     const int64_t R = a->T * a->k;
     int rc = moe_route(a->logits, a->x, a->Wr, a->dtype, a->T, a->d, a->E, a->k, a->renorm,
-                       nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
-                       c.route_ws, c.route_bytes, stream);
+                       a->logits ? nullptr : a->save_logits, a->idx, a->gate, a->counts,
+                       a->offsets, a->slot, nullptr, c.route_ws, c.route_bytes, stream);
     if (rc != MOE_OK) return rc;
     void* Xe = a->save_Xe ? a->save_Xe : c.Xe;
     void* H = a->save_H ? a->save_H : c.H;
+    void* Ye = a->save_Ye ? a->save_Ye : c.Ye;
     rc = moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, Xe, stream);
     if (rc != MOE_OK) return rc;
     rc = moe_grouped_gate_up_save(Xe, a->W1, a->W3, a->w13_expert_stride, a->offsets, a->E, R,
                                   a->d, a->F, a->dtype, H, a->save_A, a->save_B, stream);
     if (rc != MOE_OK) return rc;
     rc = moe_grouped_down(H, a->W2, a->w2_expert_stride, a->offsets, a->E, R, a->d, a->F,
-                          a->dtype, c.Ye, stream);
+                          a->dtype, Ye, stream);
     if (rc != MOE_OK) return rc;
-    return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
+    return moe_combine(Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
 }
 
 namespace moe {
@@ -147,7 +148,8 @@ extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
                                   void* stream, void* stream_h2d, void* stream_d2h) {
     if (!a || !x_host || !out_host || chunks < 1 || chunks > layer::MAX_CHUNKS) return MOE_ERR_INVALID;
     if ((a->logits == nullptr) != (logits_host == nullptr)) return MOE_ERR_INVALID;
-    if (a->save_Xe || a->save_H || a->save_A || a->save_B) return MOE_ERR_INVALID;
+    if (a->save_Xe || a->save_H || a->save_A || a->save_B || a->save_Ye || a->save_logits)
+        return MOE_ERR_INVALID;
     if (stream == stream_h2d || stream == stream_d2h || stream_h2d == stream_d2h)
         return MOE_ERR_INVALID;
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->k < 1) return MOE_ERR_INVALID;
@@ -215,6 +217,12 @@ extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
     if (!a) return MOE_ERR_INVALID;
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
     if (a->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (a->dlogits && (!a->logits || !a->idx || !a->Ye || (a->aux_coef != 0.f && !a->counts)))
+        return MOE_ERR_INVALID;
+    if (a->dlogits && a->Wr && a->dWr &&
+        (!a->x || !a->router_workspace ||
+         a->router_workspace_bytes < moe_router_linear_bwd_workspace_size(a->T, a->d, a->E)))
+        return MOE_ERR_INVALID;
     const size_t need = moe_layer_bwd_workspace_size(a->T, a->d, a->F, a->k, a->dtype);
     if (!a->workspace || a->workspace_bytes < need ||
         (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
@@ -238,7 +246,14 @@ extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
                                 a->d, a->F, a->dtype, dA, dB, dXe, a->dW1, a->dW3, a->dW2, stream);
     if (rc != MOE_OK) return rc;
     if (a->T == 0) return MOE_OK;
-    return moe_combine(dXe, a->slot, nullptr, a->T, a->d, a->k, a->dtype, a->dx, stream);
+    rc = moe_combine(dXe, a->slot, nullptr, a->T, a->d, a->k, a->dtype, a->dx, stream);
+    if (rc != MOE_OK || !a->dlogits) return rc;
+    // router backward: gates -> softmax (+ the load-balancing term) -> logits
+    rc = moe_router_bwd(a->dOut, a->Ye, a->slot, a->idx, a->logits, a->counts, a->T, a->d, a->E,
+                        a->k, a->dtype, a->renorm, a->aux_coef, a->dgate, a->dlogits, stream);
+    if (rc != MOE_OK || !a->Wr) return rc;
+    return moe_router_linear_bwd(a->dlogits, a->x, a->Wr, a->T, a->d, a->E, a->dtype, a->dx,
+                                 a->dWr, a->router_workspace, a->router_workspace_bytes, stream);
 }
 
 namespace moe {

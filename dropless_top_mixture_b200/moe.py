@@ -58,6 +58,7 @@ class LayerArgs(ctypes.Structure):
         ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
         ("workspace", _p), ("workspace_bytes", _sz),
         ("save_Xe", _p), ("save_H", _p), ("save_A", _p), ("save_B", _p),
+        ("save_Ye", _p), ("save_logits", _p),
     ]
 
 
@@ -71,6 +72,10 @@ class LayerBwdArgs(ctypes.Structure):
         ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
         ("dOut", _p), ("dx", _p), ("dW1", _p), ("dW3", _p), ("dW2", _p),
         ("workspace", _p), ("workspace_bytes", _sz),
+        ("logits", _p), ("idx", _p), ("counts", _p), ("Ye", _p), ("x", _p), ("Wr", _p),
+        ("aux_coef", ctypes.c_float), ("renorm", ctypes.c_int32),
+        ("dgate", _p), ("dlogits", _p), ("dWr", _p),
+        ("router_workspace", _p), ("router_workspace_bytes", _sz),
     ]
 
 
@@ -119,6 +124,12 @@ _SIGS = {
     "moe_layer_fwd_host": (_i32, [ctypes.POINTER(LayerArgs), _p, _p, _p, _i32, _p, _p, _p]),
     "moe_layer_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32, _i32]),
     "moe_layer_bwd": (_i32, [ctypes.POINTER(LayerBwdArgs), _p]),
+    "moe_aux_loss_workspace_size": (_sz, [_i64, _i64]),
+    "moe_aux_loss": (_i32, [_p, _p, _i64, _i64, _p, _p, _sz, _p]),
+    "moe_router_bwd": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _i32,
+                              ctypes.c_float, _p, _p, _p]),
+    "moe_router_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "moe_router_linear_bwd": (_i32, [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _p, _sz, _p]),
     "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
     "moe_version": (ctypes.c_char_p, []),
 }
@@ -421,6 +432,9 @@ class LayerOut:
     H: Optional[torch.Tensor] = None
     A: Optional[torch.Tensor] = None
     B: Optional[torch.Tensor] = None
+    Ye: Optional[torch.Tensor] = None   # expert outputs, for the router backward
+    logits: Optional[torch.Tensor] = None  # fp32 logits (computed or given)
+    renorm: bool = False
 
 
 def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool = False,
@@ -441,13 +455,21 @@ def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool =
             R = T * k
             out.Xe = torch.empty((R, d), dtype=x.dtype, device=dev)
             out.H, out.A, out.B = (torch.empty((R, F), dtype=x.dtype, device=dev) for _ in range(3))
+            out.Ye = torch.empty((R, d), dtype=x.dtype, device=dev)
+            if logits is None:
+                out.logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    if logits is not None:
+        out.logits = logits
+    out.renorm = bool(renorm)
+    save_logits = out.logits if (save and logits is None) else None
     a = LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(x.dtype), renorm=int(renorm),
                   reserved0=0, x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1=_ptr(W1),
                   W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13, w2_expert_stride=W2.stride(0),
                   out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
                   counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
                   workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel(),
-                  save_Xe=_ptr(out.Xe), save_H=_ptr(out.H), save_A=_ptr(out.A), save_B=_ptr(out.B))
+                  save_Xe=_ptr(out.Xe), save_H=_ptr(out.H), save_A=_ptr(out.A), save_B=_ptr(out.B),
+                  save_Ye=_ptr(out.Ye), save_logits=_ptr(save_logits))
     rc = lib.moe_layer_fwd(ctypes.byref(a), _stream(x))
     _check("moe_layer_fwd", rc)
     return out
@@ -515,14 +537,27 @@ class LayerGrads:
     dW3: torch.Tensor
     dW2: torch.Tensor
     workspace: torch.Tensor
+    dlogits: Optional[torch.Tensor] = None    # router backward (router=True)
+    dgate: Optional[torch.Tensor] = None
+    dWr: Optional[torch.Tensor] = None
+    router_workspace: Optional[torch.Tensor] = None
 
 
 def moe_layer_bwd(fwd: LayerOut, dOut, k: int, W1, W3, W2,
-                  out: Optional[LayerGrads] = None) -> LayerGrads:
-    """Backward of moe_layer_fwd(save=True) with the gates held constant."""
+                  out: Optional[LayerGrads] = None, *, router: bool = False, x=None, Wr=None,
+                  aux_coef: float = 0.0) -> LayerGrads:
+    """Backward of moe_layer_fwd(save=True). With router=False the gates are
+    held constant; with router=True the gates are differentiated through the
+    softmax too (plus aux_coef times the load-balancing loss), giving dlogits,
+    dgate and, when Wr is given, the router GEMM backward (dx += dlogits Wr,
+    dWr = dlogits^T x, which needs x)."""
     _need(dOut, "dOut")
     if fwd.Xe is None:
         raise ValueError("moe_layer_bwd needs the forward run with save=True")
+    if router and (fwd.Ye is None or fwd.logits is None):
+        raise ValueError("the router backward needs the forward's Ye and logits (save=True)")
+    if router and Wr is not None and x is None:
+        raise ValueError("dWr needs the forward input x")
     T, d = dOut.shape
     E, F, _, s13 = _w13(W1, W3)
     dev, dt = dOut.device, dOut.dtype
@@ -532,6 +567,14 @@ def moe_layer_bwd(fwd: LayerOut, dOut, k: int, W1, W3, W2,
                          dW1=torch.empty((E, F, d), dtype=dt, device=dev),
                          dW3=torch.empty((E, F, d), dtype=dt, device=dev),
                          dW2=torch.empty((E, d, F), dtype=dt, device=dev), workspace=ws)
+        if router:
+            out.dlogits = torch.empty((T, E), dtype=torch.float32, device=dev)
+            out.dgate = torch.empty((T, k), dtype=torch.float32, device=dev)
+            if Wr is not None:
+                out.dWr = torch.empty((E, d), dtype=dt, device=dev)
+                out.router_workspace = _alloc_ws(
+                    lib.moe_router_linear_bwd_workspace_size(T, d, E), dev)
+    rws = out.router_workspace
     a = LayerBwdArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(dt), reserved0=0, reserved1=0,
                      slot=_ptr(fwd.slot), gate=_ptr(fwd.gate), offsets=_ptr(fwd.offsets),
                      Xe=_ptr(fwd.Xe), A=_ptr(fwd.A), B=_ptr(fwd.B), H=_ptr(fwd.H), W1=_ptr(W1),
@@ -539,9 +582,77 @@ def moe_layer_bwd(fwd: LayerOut, dOut, k: int, W1, W3, W2,
                      w2_expert_stride=W2.stride(0), dOut=_ptr(dOut), dx=_ptr(out.dx),
                      dW1=_ptr(out.dW1), dW3=_ptr(out.dW3), dW2=_ptr(out.dW2),
                      workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    if router:
+        a.logits, a.idx, a.counts, a.Ye = (_ptr(fwd.logits), _ptr(fwd.idx), _ptr(fwd.counts),
+                                           _ptr(fwd.Ye))
+        a.x, a.Wr = _ptr(x), _ptr(Wr)
+        a.aux_coef, a.renorm = float(aux_coef), int(fwd.renorm)
+        a.dgate, a.dlogits, a.dWr = _ptr(out.dgate), _ptr(out.dlogits), _ptr(out.dWr)
+        a.router_workspace = _ptr(rws)
+        a.router_workspace_bytes = 0 if rws is None else rws.numel()
     rc = lib.moe_layer_bwd(ctypes.byref(a), _stream(dOut))
     _check("moe_layer_bwd", rc)
     return out
+
+
+def moe_aux_loss(logits, counts, out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Load-balancing loss E * sum_e (counts_e/T) * mean_t softmax(logits_t)_e,
+    as a one-element fp32 device tensor."""
+    _need(logits, "logits"); _need(counts, "counts")
+    T, E = logits.shape
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=logits.device)
+    if workspace is None:
+        workspace = _alloc_ws(lib.moe_aux_loss_workspace_size(T, E), logits.device)
+    rc = lib.moe_aux_loss(_ptr(logits), _ptr(counts), T, E, _ptr(out), _ptr(workspace),
+                          workspace.numel(), _stream(logits))
+    _check("moe_aux_loss", rc)
+    return out
+
+
+@dataclass
+class RouterGrads:
+    dgate: Optional[torch.Tensor]
+    dlogits: torch.Tensor
+
+
+def moe_router_bwd(dOut, Ye, slot, idx, logits, counts=None, *, renorm: bool = False,
+                   aux_coef: float = 0.0, dgate=None, dlogits=None,
+                   want_dgate: bool = True) -> RouterGrads:
+    """Gate and router-logit gradients (top-k choice and counts held fixed)."""
+    for t, n in ((dOut, "dOut"), (Ye, "Ye"), (slot, "slot"), (idx, "idx"), (logits, "logits")):
+        _need(t, n)
+    T, d = dOut.shape
+    k = slot.shape[1]
+    E = logits.shape[1]
+    if dgate is None and want_dgate:
+        dgate = torch.empty((T, k), dtype=torch.float32, device=dOut.device)
+    if dlogits is None:
+        dlogits = torch.empty((T, E), dtype=torch.float32, device=dOut.device)
+    rc = lib.moe_router_bwd(_ptr(dOut), _ptr(Ye), _ptr(slot), _ptr(idx), _ptr(logits),
+                            _ptr(counts), T, d, E, k, _dtype_code(dOut.dtype), int(renorm),
+                            float(aux_coef), _ptr(dgate), _ptr(dlogits), _stream(dOut))
+    _check("moe_router_bwd", rc)
+    return RouterGrads(dgate=dgate, dlogits=dlogits)
+
+
+def moe_router_linear_bwd(dlogits, x, Wr, dx=None, want_dWr: bool = True, dWr=None,
+                          workspace: Optional[torch.Tensor] = None):
+    """logits = x Wr^T backward: dx += dlogits Wr (in place, when dx is given)
+    and dWr = dlogits^T x. Returns (dx, dWr)."""
+    _need(dlogits, "dlogits"); _need(x, "x"); _need(Wr, "Wr")
+    T, d = x.shape
+    E = Wr.shape[0]
+    if dWr is None and want_dWr:
+        dWr = torch.empty((E, d), dtype=x.dtype, device=x.device)
+    if dWr is not None and workspace is None:
+        workspace = _alloc_ws(lib.moe_router_linear_bwd_workspace_size(T, d, E), x.device)
+    rc = lib.moe_router_linear_bwd(_ptr(dlogits), _ptr(x), _ptr(Wr), T, d, E,
+                                   _dtype_code(x.dtype), _ptr(dx), _ptr(dWr), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(x))
+    _check("moe_router_linear_bwd", rc)
+    return dx, dWr
 
 
 def moe_get_status(clear: bool = True, device=None) -> int:

@@ -372,6 +372,11 @@ typedef struct moe_layer_args {
     void* save_H;           /* [R,F] */
     void* save_A;           /* [R,F] */
     void* save_B;           /* [R,F] */
+    /* optional, for the router backward of moe_layer_bwd: the expert output
+     * rows Ye [R,d] (replacing the workspace copy) and, when the logits are
+     * computed from x and Wr, the fp32 logits [T,E] */
+    void* save_Ye;
+    float* save_logits;
 } moe_layer_args;
 
 MOE_API size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
@@ -410,6 +415,14 @@ MOE_API int moe_layer_fwd_host(const moe_layer_args* args, const void* x_host,
  * Needs the forward's routing (slot, gate, offsets) and saved rows (Xe, A,
  * B, H: moe_layer_args.save_*). Workspace: moe_layer_bwd_workspace_size
  * (dYe, dA, dB, dXe). bf16 only, same limits as moe_grouped_swiglu_bwd.
+ *
+ * With dlogits non-NULL the gates are differentiated too (router backward,
+ * see moe_router_bwd): dlogits [T,E] fp32 (and dgate [T,k] if non-NULL)
+ * from dOut, the forward's Ye (save_Ye), logits, idx and counts, with
+ * aux_coef times the load-balancing loss's gradient; when Wr is given the
+ * router GEMM backward follows: dx += dlogits·Wr and, if dWr is non-NULL,
+ * dWr = dlogitsᵀ·x ([E,d] bf16, router_workspace of
+ * moe_router_linear_bwd_workspace_size bytes).
  * ---------------------------------------------------------------------- */
 typedef struct moe_layer_bwd_args {
     int64_t T, d, E, F;
@@ -432,10 +445,75 @@ typedef struct moe_layer_bwd_args {
     void* dW2;              /* [E,d,F]                                        */
     void* workspace;
     size_t workspace_bytes;
+    /* optional router backward (dlogits == NULL: gates held constant) */
+    const float* logits;    /* [T,E] fp32 logits of the forward               */
+    const int32_t* idx;     /* [T,k]                                          */
+    const int32_t* counts;  /* [E]                                            */
+    const void* Ye;         /* [R,d] the forward's expert outputs (save_Ye)   */
+    const void* x;          /* [T,d] forward input (for dWr)                  */
+    const void* Wr;         /* [E,d], or NULL when the logits were an input   */
+    float aux_coef;         /* weight of the load-balancing loss              */
+    int32_t renorm;         /* the forward's renorm flag                      */
+    float* dgate;           /* [T,k] fp32, or NULL                            */
+    float* dlogits;         /* [T,E] fp32                                     */
+    void* dWr;              /* [E,d], or NULL                                 */
+    void* router_workspace;
+    size_t router_workspace_bytes;
 } moe_layer_bwd_args;
 
 MOE_API size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype);
 MOE_API int moe_layer_bwd(const moe_layer_bwd_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Router backward and the load-balancing auxiliary loss.
+ *
+ * ["Transformers 中的 OLMoE", §2 router; §4 "负载均衡辅助损失": a Switch-
+ * Transformer-style loss built from each expert's assignment frequency and
+ * its mean routing probability, multiplied and summed; the caller scales it
+ * into the total loss (router_aux_loss_coef, 0.01 by default).] p[t,:] is
+ * the fp32 softmax of logits[t,:]; f_e = counts[e]/T counts each of a
+ * token's k choices (a uniform router gives aux = k).
+ *
+ * moe_aux_loss: *aux_out (device fp32) = E * sum_e f_e * (1/T) sum_t p[t,e].
+ *   logits [T,E] fp32, counts [E] from moe_route. Workspace (16-byte
+ *   aligned, moe_aux_loss_workspace_size bytes) holds per-block partial
+ *   sums; the result is deterministic (fixed reduction order). T >= 1.
+ *
+ * moe_router_bwd: gradients of a loss L(out) + aux_coef * aux with respect
+ * to the gates and the router logits, the top-k choice and the counts held
+ * fixed (both piecewise constant):
+ *   dgate[t,j]   = <dOut[t], Ye[slot[t,j]]>   (fp32 sums of the layer-dtype
+ *                  rows; out[t] = sum_j gate[t,j] Ye[slot[t,j]])
+ *   dsel[t,j]    = dgate, or with renorm (gates p_sel/S, S = sum of the k
+ *                  chosen p): (dgate - sum_i gate_i dgate_i) / S
+ *   dp[t,e]      = sum_j [idx[t,j] = e] dsel[t,j] + aux_coef*E*counts[e]/T^2
+ *   dlogits[t,e] = p[t,e] * (dp[t,e] - sum_e' p[t,e'] dp[t,e'])
+ *   dOut [T,d], Ye [R,d] (the forward's expert outputs) in `dtype`, 16-byte
+ *   aligned rows; slot, idx [T,k], logits [T,E] fp32 and counts [E] from
+ *   the forward (counts may be NULL when aux_coef == 0). dgate [T,k] fp32
+ *   (NULL = not written), dlogits [T,E] fp32. A slot or idx out of range is
+ *   skipped and sets MOE_DEVERR_BAD_INDEX.
+ *
+ * moe_router_linear_bwd: the router GEMM logits = x Wr^T:
+ *   dx[t,:]  = round(dx[t,:] + sum_e dlogits[t,e] Wr[e,:])  (dx NULL: skip;
+ *              accumulates into the layer-dtype dx of moe_layer_bwd)
+ *   dWr[e,:] = round(sum_t dlogits[t,e] x[t,:])             (dWr NULL: skip)
+ *   fp32 sums (dWr over fixed token chunks, then the chunks in order, in the
+ *   workspace of moe_router_linear_bwd_workspace_size bytes). x [T,d],
+ *   Wr [E,d], dx, dWr in `dtype`; d % 4 == 0.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_aux_loss_workspace_size(int64_t T, int64_t E);
+MOE_API int moe_aux_loss(const float* logits, const int32_t* counts, int64_t T, int64_t E,
+                         float* aux_out, void* workspace, size_t workspace_bytes, void* stream);
+MOE_API int moe_router_bwd(const void* dOut, const void* Ye, const int32_t* slot,
+                           const int32_t* idx, const float* logits, const int32_t* counts,
+                           int64_t T, int64_t d, int64_t E, int k, int dtype, int renorm,
+                           float aux_coef, float* dgate, float* dlogits, void* stream);
+MOE_API size_t moe_router_linear_bwd_workspace_size(int64_t T, int64_t d, int64_t E);
+MOE_API int moe_router_linear_bwd(const float* dlogits, const void* x, const void* Wr,
+                                  int64_t T, int64_t d, int64_t E, int dtype, void* dx,
+                                  void* dWr, void* workspace, size_t workspace_bytes,
+                                  void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_get_status — read (and optionally clear) the device status word of the

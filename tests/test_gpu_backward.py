@@ -132,3 +132,48 @@ def test_fine_grained_backward_full_size_sampled():
         assert_close_scaled(np64(g.dW1[e]), r1, f"dW1[{e}]")
         assert_close_scaled(np64(g.dW3[e]), r3, f"dW3[{e}]")
         assert_close_scaled(np64(g.dW2[e]), r2, f"dW2[{e}]")
+
+
+@pytest.mark.parametrize("renorm", [False, True])
+@pytest.mark.parametrize("router_from_x", [True, False])
+def test_layer_backward_with_router(renorm, router_from_x):
+    """The whole training backward of the layer: expert path, the gates
+    through the softmax (and renorm) with the load-balancing term, and the
+    router GEMM backward (dx += dlogits Wr, dWr) when the logits come from
+    x and Wr; against the oracle at the layer tolerance."""
+    moe = _moe()
+    T, d, F, E, k = 384, 256, 256, 8, 2
+    x, W1, W3, W2, dOut, lg = _problem(T, d, F, E, k, seed=77, skew=False)
+    g = torch.Generator().manual_seed(78)
+    Wr = (torch.randn(E, d, generator=g) * 0.05).to(torch.bfloat16)
+    dev = "cuda"
+    W = [w.to(dev) for w in (W1, W3, W2)]
+    kw = dict(Wr=Wr.to(dev)) if router_from_x else dict(logits=torch.from_numpy(lg).to(dev))
+    fwd = moe.moe_layer_fwd(x.to(dev), k, *W, renorm=renorm, save=True, **kw)
+    gr = moe.moe_layer_bwd(fwd, dOut.to(dev), k, *W, router=True, x=x.to(dev),
+                           Wr=kw.get("Wr"), aux_coef=0.01)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    ref = (O.moe_layer(x, k, W1, W3, W2, Wr=Wr, renorm=renorm) if router_from_x
+           else O.moe_layer(x, k, W1, W3, W2, logits=lg, renorm=renorm))
+    idx = ref["idx"]
+    assert np.array_equal(gr.dgate.shape, (T, k))
+    assert np.array_equal(fwd.idx.cpu().numpy(), idx)
+    logits = ref["logits"]
+    # expert path with the gates held constant (its own oracle), plus the
+    # router path
+    eb = O.moe_layer_bwd(x, dOut, k, W1, W3, W2, logits) if not renorm else None
+    Y = ref["Ye"][ref["slot"]]
+    dg = O.gate_grad(np64(dOut), Y)
+    dlog = O.router_grad(logits, idx, dg, renorm=renorm, aux_coef=0.01)
+    assert_close_layer(np64(gr.dgate), dg, "dgate", max_abs=2e-2 * np.abs(dg).max())
+    assert_close_layer(np64(gr.dlogits), dlog, "dlogits", max_abs=2e-2 * np.abs(dlog).max())
+    if router_from_x:
+        gx, gW = O.router_linear_grad(dlog, x, Wr)
+        assert_close_layer(np64(gr.dWr), gW, "dWr", max_abs=2e-2 * np.abs(gW).max())
+        if eb is not None:
+            want = eb["dx"] + gx
+            assert_close_scaled(np64(gr.dx), want, "dx (experts + router)")
+    elif eb is not None:
+        assert gr.dWr is None
+        assert_close_scaled(np64(gr.dx), eb["dx"], "dx (experts only)")
