@@ -36,6 +36,9 @@ notes):
   * routing metadata is the stable counting sort of the token-major list of
     (token, j) pairs by expert: slot = offsets[e] + (number of earlier
     tokens routed to e). Offsets are unpadded.
+  * router logits x·Wrᵀ: four sequential fp32 fmaf chains over the
+    contiguous quarters of the hidden dimension, added in order (the
+    summation order decides the top-k bits, so it is fixed on both sides).
   * the expert FFN and the combine are evaluated without intermediate
     rounding (float64); the CUDA path stores H and Ye in the layer dtype.
   * MXFP8: blocks of 32 consecutive elements along the contraction axis;
@@ -104,11 +107,15 @@ def _load():
 # --------------------------------------------------------------------------
 
 def router_logits(x: torch.Tensor, Wr: torch.Tensor) -> np.ndarray:
-    """fp32 logits[t, e] = sequential fmaf over j of x[t, j] * Wr[e, j]."""
+    """fp32 logits[t, e]: four sequential fmaf chains over the contiguous
+    quarters of j (each from +0.0), the quarter sums added in order
+    ((c0 + c1) + c2) + c3. d must be a multiple of 4."""
     lib = _load()
     x = x.detach().cpu().contiguous()
     Wr = Wr.detach().cpu().contiguous()
     T, d = x.shape
+    if d % 4:
+        raise ValueError("the router's hidden size must be a multiple of 4")
     E = Wr.shape[0]
     out = np.empty((T, E), dtype=np.float32)
     if x.dtype == torch.float32:

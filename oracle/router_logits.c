@@ -11,14 +11,18 @@
  *
  * The pages leave the summation order of this dot product open. Because the
  * top-k decision is taken on these fp32 values, both sides must produce the
- * same bits, so the order is fixed to the plainest one: one fp32 accumulator
- * per (token, expert), started at +0.0 and updated with a fused multiply-add
- * for j = 0, 1, ..., d-1 in ascending order:
+ * same bits, so the order is fixed: d is cut into four contiguous quarters
+ * (d % 4 == 0); in each quarter one fp32 accumulator starts at +0.0 and is
+ * updated with a fused multiply-add for j ascending, and the four quarter
+ * sums are added in order:
  *
- *     acc <- fmaf(x[t][j], Wr[e][j], acc)
+ *     c_q    = fmaf-chain over j in [q d/4, (q+1) d/4):  acc <- fmaf(x, w, acc)
+ *     logit  = ((c_0 + c_1) + c_2) + c_3
  *
- * (For bf16 inputs the product is exact in fp32, so this equals the unfused
- * acc + x*w; for fp32 inputs the single rounding of fmaf is what is meant.)
+ * (Four independent chains per logit give the GPU four times the parallel
+ * work of a single chain; for bf16 inputs each product is exact in fp32, so
+ * fmaf equals the unfused acc + x*w; for fp32 inputs the single rounding of
+ * fmaf is what is meant.)
  *
  * Built with -ffp-contract=off so the compiler introduces no other fusion.
  */
@@ -37,13 +41,18 @@ static float bf16_to_f32(uint16_t h) {
 /* logits[t*E + e] for x [T,d] and Wr [E,d], both fp32, row-major. */
 void oracle_router_logits_f32(const float *x, const float *Wr, int64_t T, int64_t d,
                               int64_t E, float *logits) {
+    const int64_t dq = d / 4;
     #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int64_t e = 0; e < E; ++e) {
-            float acc = 0.0f;
-            for (int64_t j = 0; j < d; ++j)
-                acc = fmaf(x[t * d + j], Wr[e * d + j], acc);
-            logits[t * E + e] = acc;
+            float sum = 0.0f;
+            for (int q = 0; q < 4; ++q) {
+                float acc = 0.0f;
+                for (int64_t j = q * dq; j < (q + 1) * dq; ++j)
+                    acc = fmaf(x[t * d + j], Wr[e * d + j], acc);
+                sum = q == 0 ? acc : sum + acc;
+            }
+            logits[t * E + e] = sum;
         }
     }
 }
@@ -51,13 +60,18 @@ void oracle_router_logits_f32(const float *x, const float *Wr, int64_t T, int64_
 /* Same, for bf16 x and Wr given as raw 16-bit patterns. */
 void oracle_router_logits_bf16(const uint16_t *x, const uint16_t *Wr, int64_t T, int64_t d,
                                int64_t E, float *logits) {
+    const int64_t dq = d / 4;
     #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int64_t e = 0; e < E; ++e) {
-            float acc = 0.0f;
-            for (int64_t j = 0; j < d; ++j)
-                acc = fmaf(bf16_to_f32(x[t * d + j]), bf16_to_f32(Wr[e * d + j]), acc);
-            logits[t * E + e] = acc;
+            float sum = 0.0f;
+            for (int q = 0; q < 4; ++q) {
+                float acc = 0.0f;
+                for (int64_t j = q * dq; j < (q + 1) * dq; ++j)
+                    acc = fmaf(bf16_to_f32(x[t * d + j]), bf16_to_f32(Wr[e * d + j]), acc);
+                sum = q == 0 ? acc : sum + acc;
+            }
+            logits[t * E + e] = sum;
         }
     }
 }

@@ -20,28 +20,44 @@ def _bf16(shape, seed, std=1.0):
 
 
 def test_router_logits_bf16_matches_unfused_fp32_sum():
-    # bf16 x bf16 products are exact in fp32, so sequential fmaf equals the
-    # sequential fp32 sum of exact products, computed here with numpy.
+    # bf16 x bf16 products are exact in fp32, so each quarter's fmaf chain
+    # equals the sequential fp32 sum of its exact products (numpy here); the
+    # four quarter sums are then added in order.
     x = _bf16((37, 96), 1)
     W = _bf16((11, 96), 2, 0.02)
     got = O.router_logits(x, W)
     xf = x.float().numpy()
     wf = W.float().numpy()
-    acc = np.zeros((37, 11), dtype=np.float32)
-    for j in range(96):
-        acc = (acc + np.outer(xf[:, j], wf[:, j]).astype(np.float32)).astype(np.float32)
-    assert np.array_equal(got.view(np.uint32), acc.view(np.uint32))
+    total = None
+    for q in range(4):
+        acc = np.zeros((37, 11), dtype=np.float32)
+        for j in range(24 * q, 24 * q + 24):
+            acc = (acc + np.outer(xf[:, j], wf[:, j]).astype(np.float32)).astype(np.float32)
+        total = acc if total is None else (total + acc).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), total.view(np.uint32))
+
+
+def test_router_logits_quarter_order_closed_form():
+    # products [2^24, 0, 1, 1 | -2^24, 0, 0, 0] (d = 8, quarters of 2): a
+    # single sequential chain loses both 1s against 2^24 and gives 0; the
+    # quarter chains give (2^24 + 2) - 2^24 = 2 exactly
+    x = torch.tensor([[4096.0, 0, 1, 1, 4096.0, 0, 0, 0]], dtype=torch.bfloat16)
+    W = torch.tensor([[4096.0, 0, 1, 1, -4096.0, 0, 0, 0]], dtype=torch.bfloat16)
+    assert O.router_logits(x, W)[0, 0] == 2.0
+    assert O.router_logits(x.float(), W.float())[0, 0] == 2.0
 
 
 def test_router_logits_error_bound_vs_fp64():
-    # Sequential fp32 accumulation error is at most gamma_d * sum|x_j w_j|.
+    # Four chains of d/4 terms and three adds: the error is at most
+    # gamma_{d/4+3} * sum|x_j w_j|.
     x = torch.randn(64, 128, generator=torch.Generator().manual_seed(3))
     W = torch.randn(8, 128, generator=torch.Generator().manual_seed(4)) * 0.02
     got = O.router_logits(x, W).astype(np.float64)
     ref = x.double().numpy() @ W.double().numpy().T
     absdot = np.abs(x.double().numpy()) @ np.abs(W.double().numpy()).T
     u = 2.0 ** -24
-    gamma = 128 * u / (1 - 128 * u)
+    n = 128 // 4 + 3
+    gamma = n * u / (1 - n * u)
     assert np.all(np.abs(got - ref) <= gamma * absdot + 1e-30)
 
 
@@ -55,8 +71,8 @@ def test_router_logits_one_hot_picks_weight_column():
 
 def test_router_logits_fp32_small_integers_exact():
     g = torch.Generator().manual_seed(9)
-    x = torch.randint(-8, 8, (10, 50), generator=g).float()
-    W = torch.randint(-8, 8, (6, 50), generator=g).float()
+    x = torch.randint(-8, 8, (10, 52), generator=g).float()
+    W = torch.randint(-8, 8, (6, 52), generator=g).float()
     got = O.router_logits(x, W)
     assert np.array_equal(got, (x.double() @ W.double().T).float().numpy())
 
