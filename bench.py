@@ -276,8 +276,8 @@ def _steps(moe, w, inp, dev, backward):
                    slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
     if use_router and backward:
         rt.logits = torch.empty((T, E), dtype=torch.float32, device=dev)  # kept for the router bwd
-    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router and not backward)),
-                      dtype=torch.uint8, device=dev)
+    rws = torch.empty(moe.lib.moe_route_workspace_size(T, E, int(use_router)), dtype=torch.uint8,
+                      device=dev)
     out = torch.empty((T, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
     Ye = torch.empty((R, d), dtype=torch.bfloat16 if w.mxfp8 else dt, device=dev)
 

@@ -1,6 +1,7 @@
 // Route step of the dropless top-k MoE layer on sm_100a.
 //
-//   a0  router logits  logits[t,e] = fmaf-chain over j of x[t,j]*Wr[e,j]
+//   a0  router logits  logits[t,e] = four fmaf chains over the quarters of j
+//                      of x[t,j]*Wr[e,j], added in order
 //   a1  fp32 softmax + top-k (ties to the lower expert index)
 //   a2  routing metadata: counts, offsets, slots, tile offsets
 //
@@ -66,32 +67,41 @@ struct Stage8<float> {
     }
 };
 
-// One CTA (128 threads) computes a 64-token x 64-expert tile. Thread (ty, tx)
-// owns tokens 8ty..8ty+7 and experts 4tx..4tx+3, each with its own fp32
-// accumulator updated in ascending j, so every logit is the same sequential
-// fmaf chain the definition states. Rows of x and Wr are staged 32 columns at
-// a time, transposed into k-major shared memory (two buffers, one barrier per
-// chunk); the next chunk is prefetched into registers while the current
-// one is consumed. Per column: 3 shared loads feed 32 FMAs.
+// The logit of (t, e) is four fmaf chains, one per contiguous quarter of j,
+// each from +0.0 in ascending j, their sums added in order ((c0 + c1) + c2)
+// + c3. One CTA (128 threads) computes one quarter's chains for a 64-token x
+// 64-expert tile (grid z = quarter) and writes them to that quarter's plane;
+// sum_quarters_kernel adds the four planes. Thread (ty, tx) owns tokens
+// 8ty..8ty+7 and experts 4tx..4tx+3, each with its own fp32 accumulator.
+// Rows of x and Wr are staged 32 columns at a time, transposed into k-major
+// shared memory (two buffers, one barrier per chunk; a warp writes 32
+// consecutive rows of one column, so the transposing stores do not conflict);
+// the next chunk is prefetched into registers while the current one is
+// consumed. Per column: 3 shared loads feed 32 FMAs.
 constexpr int LOGIT_THREADS = 128;
+constexpr int LOGIT_SPLIT = 4;  // quarter chains per logit
 
 template <typename TX>
 __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* __restrict__ x,
                                                                       const TX* __restrict__ Wr,
                                                                       int T, int d, int E,
-                                                                      float* __restrict__ logits) {
+                                                                      float* __restrict__ planes,
+                                                                      int64_t pstride) {
     __shared__ __align__(16) float xs[2][LOGIT_TK][LOGIT_LD];
     __shared__ __align__(16) float ws[2][LOGIT_TK][LOGIT_LD];
     const int tid = threadIdx.x;
     const int t0 = blockIdx.x * LOGIT_TT;
     const int e0 = blockIdx.y * LOGIT_TE;
-    // staging role: row = tid / 2 (token or expert), columns (tid % 2) * 16 .. +15
-    const int srow = tid >> 1;
-    const int scol = (tid & 1) * 16;
+    const int dq = d / LOGIT_SPLIT;
+    const int kbeg = blockIdx.z * dq;
+    float* __restrict__ logits = planes + (size_t)blockIdx.z * pstride;
+    // staging role: row = tid % 64 (token or expert), columns (tid / 64) * 16 .. +15
+    const int srow = tid & 63;
+    const int scol = (tid >> 6) * 16;
     const bool xok = (t0 + srow) < T;
     const bool wok = (e0 + srow) < E;
-    const TX* xp = x + (size_t)(t0 + srow) * d + scol;
-    const TX* wp = Wr + (size_t)(e0 + srow) * d + scol;
+    const TX* xp = x + (size_t)(t0 + srow) * d + kbeg + scol;
+    const TX* wp = Wr + (size_t)(e0 + srow) * d + kbeg + scol;
     // compute role
     const int ty = tid >> 4, tx = tid & 15;
     float acc[8][4];
@@ -106,14 +116,14 @@ __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* 
     Stage8<TX>::load(wp, wok, fw);
     Stage8<TX>::load(wp + 8, wok, fw + 8);
     int buf = 0;
-    for (int k0 = 0; k0 < d; k0 += LOGIT_TK, buf ^= 1) {
+    for (int k0 = 0; k0 < dq; k0 += LOGIT_TK, buf ^= 1) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             xs[buf][scol + i][srow] = fx[i];
             ws[buf][scol + i][srow] = fw[i];
         }
         __syncthreads();
-        if (k0 + LOGIT_TK < d) {
+        if (k0 + LOGIT_TK < dq) {
             Stage8<TX>::load(xp + k0 + LOGIT_TK, xok, fx);
             Stage8<TX>::load(xp + k0 + LOGIT_TK + 8, xok, fx + 8);
             Stage8<TX>::load(wp + k0 + LOGIT_TK, wok, fw);
@@ -148,6 +158,34 @@ __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* 
             for (int j = 0; j < 4; ++j)
                 if (e + j < E) logits[(size_t)t * E + e + j] = acc[i][j];
         }
+    }
+}
+
+// logits[i] = ((p0[i] + p1[i]) + p2[i]) + p3[i] over the four quarter planes
+// (plane stride pstride floats, a multiple of 64; planes and logits 16-byte
+// aligned), four floats per thread step, the last n % 4 one at a time.
+__global__ void __launch_bounds__(256) sum_quarters_kernel(const float* __restrict__ planes,
+                                                           int64_t n, int64_t pstride,
+                                                           float* __restrict__ logits) {
+    const int64_t nv = n / 4, sv = pstride / 4;
+    const float4* p = reinterpret_cast<const float4*>(planes);
+    float4* o = reinterpret_cast<float4*>(logits);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = __ldcs(p + i);
+#pragma unroll
+        for (int q = 1; q < LOGIT_SPLIT; ++q) {
+            const float4 b = __ldcs(p + q * sv + i);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        o[i] = a;
+    }
+    for (int64_t i = nv * 4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float a = planes[i];
+#pragma unroll
+        for (int q = 1; q < LOGIT_SPLIT; ++q) a += planes[q * pstride + i];
+        logits[i] = a;
     }
 }
 
@@ -369,24 +407,36 @@ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 struct RouteWs {
     int32_t* count;
     int32_t* ticket;
-    float* logits;
+    float* logits;  // the [T,E] logits when computed and not returned
+    float* planes;  // the four [T,E] quarter planes when computed
 };
 
-inline size_t workspace_bytes(int64_t T, int64_t E, bool need_logits) {
+// from_x: the logits are computed from x and Wr. The workspace then holds the
+// four quarter planes and a [T,E] logits buffer (used when the caller does
+// not ask for the logits), whatever logits_out is, so the size is a function
+// of (T, E, from_x) alone.
+inline int64_t plane_stride(int64_t T, int64_t E) { return (T * E + 63) / 64 * 64; }
+
+inline size_t workspace_bytes(int64_t T, int64_t E, bool from_x) {
     size_t b = align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
     b += 256;  // ticket
-    if (need_logits) b += align256(sizeof(float) * (size_t)T * (size_t)E);
+    if (from_x) {
+        b += align256(sizeof(float) * (size_t)T * (size_t)E);
+        b += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
+    }
     return b;
 }
 
-inline RouteWs carve(void* ws, int64_t T, int64_t E, bool need_logits) {
+inline RouteWs carve(void* ws, int64_t T, int64_t E, bool from_x) {
     char* p = static_cast<char*>(ws);
     RouteWs r;
     r.count = reinterpret_cast<int32_t*>(p);
     p += align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
     r.ticket = reinterpret_cast<int32_t*>(p);
     p += 256;
-    r.logits = need_logits ? reinterpret_cast<float*>(p) : nullptr;
+    r.logits = from_x ? reinterpret_cast<float*>(p) : nullptr;
+    p += from_x ? align256(sizeof(float) * (size_t)T * (size_t)E) : 0;
+    r.planes = from_x ? reinterpret_cast<float*>(p) : nullptr;
     return r;
 }
 
@@ -405,9 +455,9 @@ static void launch_topk(const float* logits, int T, int E, int k, int renorm, in
 
 using namespace moe;
 
-extern "C" size_t moe_route_workspace_size(int64_t T, int64_t E, int need_logits_buffer) {
+extern "C" size_t moe_route_workspace_size(int64_t T, int64_t E, int logits_from_x) {
     if (T < 0 || E <= 0) return 0;
-    return route::workspace_bytes(T, E, need_logits_buffer != 0);
+    return route::workspace_bytes(T, E, logits_from_x != 0);
 }
 
 extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int dtype, int64_t T,
@@ -433,31 +483,40 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     }
     const bool from_x = (logits == nullptr);
     if (from_x) {
-        if (!x || !Wr || d <= 0 || (d % route::LOGIT_TK) != 0) return MOE_ERR_INVALID;
+        if (!x || !Wr || d <= 0 || (d % (route::LOGIT_SPLIT * route::LOGIT_TK)) != 0)
+            return MOE_ERR_INVALID;
         if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
         if (!aligned16(x) || !aligned16(Wr)) return MOE_ERR_INVALID;
     }
     if (T > 0 && (!idx || !gate || !slot)) return MOE_ERR_INVALID;
-    const bool need_logits = from_x && logits_out == nullptr;
-    if (!workspace || workspace_bytes < route::workspace_bytes(T, E, need_logits))
+    if (!workspace || workspace_bytes < route::workspace_bytes(T, E, from_x))
         return MOE_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID;
+    if (from_x && logits_out && (reinterpret_cast<uintptr_t>(logits_out) & 15u) != 0)
+        return MOE_ERR_INVALID;
     cudaStream_t st = as_stream(stream);
-    route::RouteWs ws = route::carve(workspace, T, E, need_logits);
+    route::RouteWs ws = route::carve(workspace, T, E, from_x);
 
     const float* lg = logits;
     if (from_x) {
         float* dst = logits_out ? logits_out : ws.logits;
         dim3 grid((unsigned)((T + route::LOGIT_TT - 1) / route::LOGIT_TT),
-                  (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE));
+                  (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE), route::LOGIT_SPLIT);
         if (dtype == MOE_BF16)
             route::router_logits_kernel<__nv_bfloat16><<<grid, route::LOGIT_THREADS, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
-                (int)T, (int)d, (int)E, dst);
+                (int)T, (int)d, (int)E, ws.planes, route::plane_stride(T, E));
         else
             route::router_logits_kernel<float><<<grid, route::LOGIT_THREADS, 0, st>>>(
                 static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d,
-                (int)E, dst);
+                (int)E, ws.planes, route::plane_stride(T, E));
+        const int64_t n = T * E;
+        int64_t g = (n / 4 + 255) / 256;
+        const int64_t cap = (int64_t)num_sms() * 8;
+        if (g > cap) g = cap;
+        if (g < 1) g = 1;
+        route::sum_quarters_kernel<<<(int)g, 256, 0, st>>>(ws.planes, n,
+                                                           route::plane_stride(T, E), dst);
         lg = dst;
     }
     const int nch = (int)route::nchunks_of(T);

@@ -49,8 +49,8 @@ extern "C" int moe_route_noalloc(const float* logits, const void* x, const void*
                                  int32_t* offsets, int32_t* slot, int32_t* tile_offsets,
                                  void* stream) {
     if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS) return MOE_ERR_INVALID;
-    const int need_logits_buffer = (logits == nullptr && logits_out == nullptr && T > 0) ? 1 : 0;
-    const size_t need = moe_route_workspace_size(T, E, need_logits_buffer);
+    const int from_x = (logits == nullptr && T > 0) ? 1 : 0;
+    const size_t need = moe_route_workspace_size(T, E, from_x);
     if (need > (size_t)MOE_ROUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
     void* scratch = noalloc::scratch_address();
     if (!scratch) return MOE_ERR_CUDA;

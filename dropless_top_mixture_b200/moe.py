@@ -213,8 +213,7 @@ def moe_route(k: int, *, logits: Optional[torch.Tensor] = None, x: Optional[torc
                     slot=torch.empty((T, k), **i32), tile_offsets=torch.empty(E + 1, **i32))
         if logits is None and keep_logits:
             out.logits = torch.empty((T, E), dtype=torch.float32, device=dev)
-    need_buf = logits is None and out.logits is None
-    ws_bytes = lib.moe_route_workspace_size(T, E, int(need_buf))
+    ws_bytes = lib.moe_route_workspace_size(T, E, int(logits is None))
     if workspace is None:
         workspace = _alloc_ws(ws_bytes, dev)
     rc = lib.moe_route(_ptr(logits), _ptr(x), _ptr(Wr), dtype, T, d, E, k, int(renorm),

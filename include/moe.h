@@ -83,8 +83,11 @@ extern "C" {
  * Inputs (device):
  *   logits   [T,E] fp32 row-major, or NULL to compute logits = x·Wrᵀ from
  *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). The logit
- *            of (t,e) is one fp32 accumulator updated by fused multiply-add
- *            over j = 0..d-1 in ascending order, starting from +0.0.
+ *            of (t,e) is four fp32 accumulators, one per contiguous quarter
+ *            of j, each starting from +0.0 and updated by fused multiply-add
+ *            in ascending j; the four are then added in order,
+ *            ((c0 + c1) + c2) + c3. (The pages leave the order open; it is
+ *            fixed because the top-k is taken on these bits.)
  *   renorm   0: gates are the softmax probabilities; 1: divided by their sum.
  * Outputs (device, caller-allocated):
  *   logits_out  [T,E] fp32, or NULL (used only when logits == NULL)
@@ -96,12 +99,14 @@ extern "C" {
  *   slot     [T,k] int32 row of (t,j) in the expert-sorted buffers: rows of
  *            expert e are offsets[e].., in ascending token order
  *   tile_offsets [E+1] int32 exclusive prefix sum of ceil(counts/128), or NULL
- * Workspace: `workspace_bytes` >= moe_route_workspace_size(T, E, logits==NULL
- *            && logits_out==NULL); 256-byte aligned device memory. Its
- *            contents need not be initialised.
- * Limits: 1 <= k <= min(E, 32), E <= 512, d % 32 == 0 when computing logits.
+ * Workspace: `workspace_bytes` >= moe_route_workspace_size(T, E,
+ *            logits == NULL); 256-byte aligned device memory (with logits
+ *            computed it holds the four quarter sums and, when logits_out
+ *            is NULL, the logits). Its contents need not be initialised.
+ * Limits: 1 <= k <= min(E, 32), E <= 512; when computing logits d % 128 == 0
+ *            and logits_out (if given) 16-byte aligned.
  * ---------------------------------------------------------------------- */
-MOE_API size_t moe_route_workspace_size(int64_t T, int64_t E, int need_logits_buffer);
+MOE_API size_t moe_route_workspace_size(int64_t T, int64_t E, int logits_from_x);
 MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dtype, int64_t T,
                       int64_t d, int64_t E, int k, int renorm, float* logits_out, int32_t* idx,
                       float* gate, int32_t* counts, int32_t* offsets, int32_t* slot,
@@ -119,11 +124,11 @@ MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dt
  * `workspace`/`workspace_bytes`; its scratch is a library-owned device array
  * of MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU loading the library
  * keeps reserved until the process exits.
- *   - Size limit: moe_route_workspace_size(T, E, logits == NULL &&
- *     logits_out == NULL) must not exceed MOE_ROUTE_NOALLOC_SCRATCH_BYTES,
- *     else MOE_ERR_UNSUPPORTED and nothing is launched. (E = 64 with logits
- *     computed from x fits up to T = 29,121 tokens; E = 128 with logits
- *     given up to T = 131,057; E = 384 with logits given up to T = 43,681.)
+ *   - Size limit: moe_route_workspace_size(T, E, logits == NULL) must not
+ *     exceed MOE_ROUTE_NOALLOC_SCRATCH_BYTES, else MOE_ERR_UNSUPPORTED and
+ *     nothing is launched. (E = 64 with logits computed from x fits up to
+ *     T = 6,393 tokens; E = 128 with logits given up to T = 131,064; E = 384
+ *     with logits given up to T = 43,688.)
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
  *     that first call before any stream capture begins.

@@ -54,6 +54,9 @@ def test_host_validation_rejects_without_launch(lib):
     # E beyond the build limit
     assert L.moe_route(p16, None, None, 0, 10, 0, 1000, 2, 0, None, p16, p16, p16, p16, p16, None,
                        p16, 4096, None) == m.MOE_ERR_INVALID
+    # logits from x need d % 128 == 0 (four quarters of whole 32-column chunks)
+    assert L.moe_route(None, p16, p16, m.MOE_BF16, 10, 96, 4, 2, 0, None, p16, p16, p16, p16,
+                       p16, None, p16, 1 << 15, None) == m.MOE_ERR_INVALID
     # workspace too small
     assert L.moe_route(p16, None, None, 0, 1000, 0, 64, 2, 0, None, p16, p16, p16, p16, p16, None,
                        p16, 16, None) == m.MOE_ERR_INVALID

@@ -60,7 +60,8 @@ def test_route_skewed_with_empty_experts():
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("T,d,E,k", [(5, 128, 8, 2), (130, 256, 64, 8), (77, 64, 33, 3)])
+@pytest.mark.parametrize("T,d,E,k", [(5, 128, 8, 2), (130, 256, 64, 8), (77, 128, 33, 3),
+                                     (64, 384, 17, 4)])
 def test_router_logits_bitexact(dtype, T, d, E, k):
     moe = _moe()
     g = torch.Generator().manual_seed(T * d + E)
