@@ -317,11 +317,11 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     const int64_t R = a->T * a->k;
     rc = moe_dispatch_mxfp8(a->x, a->slot, a->T, a->d, a->k, c.Xq, c.Xs, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xs, a->W1q, a->W1s, a->W3q, a->W3s, a->w13_expert_stride,
+    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xs, a->W1q, a->W3q, a->Ps13, a->w13_expert_stride,
                                    a->offsets, a->E, R, a->d, a->F, c.Hq, c.Hs, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_down_mxfp8(c.Hq, c.Hs, a->W2q, a->W2s, a->w2_expert_stride, a->offsets, a->E, R,
-                                a->d, a->F, c.Ye, stream);
+    rc = moe_grouped_down_mxfp8(c.Hq, c.Hs, a->W2q, a->Ps2, a->w2_expert_stride, a->offsets, a->E,
+                                R, a->d, a->F, c.Ye, stream);
     if (rc != MOE_OK) return rc;
     return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, MOE_BF16, a->out, stream);
 }

@@ -38,8 +38,10 @@ constexpr int A_BYTES = BM * 128;
 constexpr int B_BYTES = MMA_N * 128;
 constexpr int SLAB_BYTES = A_BYTES + B_BYTES;
 constexpr int STAGE_BYTES = SLABS * SLAB_BYTES;
-constexpr int SF_SLAB_BYTES = 1024;   // 512 B of A scale words + 512 B of B scale words
-constexpr int SF_STAGE_BYTES = SLABS * SF_SLAB_BYTES;
+constexpr int SF_BLOCK = 512;         // one operand's scale words for one slab
+// per stage: A blocks of the SLABS slabs, then their B blocks (contiguous, so
+// one bulk copy brings the packed weight scales of the whole stage)
+constexpr int SF_STAGE_BYTES = 2 * SLABS * SF_BLOCK;
 constexpr int TMEM_ALLOC = 512;
 constexpr int SFA_COL = 2 * MMA_N;    // 256 (+8 per slab)
 constexpr int SFB_COL = SFA_COL + 4;  // 260 (+8 per slab)
@@ -122,8 +124,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                    const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const uint8_t* __restrict__ sfA,
-                   const uint8_t* __restrict__ sfB0, const uint8_t* __restrict__ sfB1,
-                   int64_t sfb_expert_stride, const int32_t* __restrict__ offsets, int E, int R,
+                   const uint8_t* __restrict__ sfBp, const int32_t* __restrict__ offsets, int E, int R,
                    int K, int N, uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_s,
                    __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status) {
     constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
@@ -221,8 +222,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 const uint32_t fb = smem_u32(full + stage);
                 const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
+                const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 if (lane == 0) {
-                    mbar_expect_tx(fb, (uint32_t)(ns * SLAB_BYTES));
+                    mbar_expect_tx(fb, (uint32_t)(ns * (SLAB_BYTES + SF_BLOCK)));
+                    // packed B scales of this stage's slabs: one bulk copy
+                    const size_t blk = ((size_t)tl.e * NB + tl.n0 / OUT_N) * KS + kb * SLABS;
+                    bulk_load(sfs + SLABS * SF_BLOCK, sfBp + blk * SF_BLOCK,
+                              (uint32_t)(ns * SF_BLOCK), fb);
                     for (int sl = 0; sl < ns; ++sl) {
                         const int kc = (kb * SLABS + sl) * BK;
                         const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
@@ -236,29 +242,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                     }
                 }
-                // scale words, copied asynchronously: the stage's barrier
-                // completes only once they have landed, so the producer never
-                // waits on their latency
+                // activation scale words (tile rows start anywhere, so they
+                // are gathered row by row), copied asynchronously: the stage's
+                // barrier completes only once they have landed
                 for (int sl = 0; sl < ns; ++sl) {
-                    const uint32_t sfs =
-                        smem_u32(sf_smem + stage * SF_STAGE_BYTES + sl * SF_SLAB_BYTES);
                     const int kw = 4 * (kb * SLABS + sl);  // scale byte of the slab's first block
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int m = lane + 32 * j;  // A row within the tile
                         const int grow = tl.row0 + m;
                         const bool in = grow < R;
-                        cp_async_word(sfs + (uint32_t)(lane * 4 + j) * 4u,
+                        cp_async_word(sfs + (uint32_t)(sl * SF_BLOCK + (lane * 4 + j) * 4),
                                       sfA + (size_t)(in ? grow : 0) * sf_row + kw, in ? 4u : 0u);
-                        const uint8_t* bsrc;
-                        if (SWIGLU) {
-                            bsrc = (m < 64 ? sfB0 + (size_t)(tl.n0 + m) * sf_row
-                                           : sfB1 + (size_t)(tl.n0 + m - 64) * sf_row);
-                        } else {
-                            bsrc = sfB0 + (size_t)(tl.n0 + m) * sf_row;
-                        }
-                        cp_async_word(sfs + 512u + (uint32_t)(lane * 4 + j) * 4u,
-                                      bsrc + (size_t)tl.e * sfb_expert_stride + kw, 4u);
                     }
                 }
                 cp_async_arrive(fb);
@@ -306,8 +301,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 for (int sl = 0; sl < ns; ++sl) {
-                    tmem_cp_sf(sfa_t + 8u * sl, sf_desc(sfs + sl * SF_SLAB_BYTES));
-                    tmem_cp_sf(sfb_t + 8u * sl, sf_desc(sfs + sl * SF_SLAB_BYTES + 512));
+                    tmem_cp_sf(sfa_t + 8u * sl, sf_desc(sfs + sl * SF_BLOCK));
+                    tmem_cp_sf(sfb_t + 8u * sl, sf_desc(sfs + (SLABS + sl) * SF_BLOCK));
                 }
                 for (int sl = 0; sl < ns; ++sl) {
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
@@ -434,10 +429,44 @@ __global__ void __launch_bounds__(256) mx_dispatch_kernel(const __nv_bfloat16* _
     }
 }
 
+// Weight scales packed for the tensor-core scale copy. For every expert,
+// 128-row B tile of the kernel (gate/up: rows n0..n0+63 of W1 then of W3,
+// n0 = 64 nb; down: rows n0..n0+127 of W2, n0 = 128 nb) and 128-element K
+// slab s, one 512-byte block holds the four scale bytes of each of the 128
+// rows in the 32-row x 16-byte order tcgen05.cp.32x128b.warpx4 copies:
+// row m's word at 16 (m % 32) + 4 (m / 32). Blocks are ordered (expert,
+// n-block, slab), so one stage's slabs are adjacent. One thread per word.
+__global__ void __launch_bounds__(256)
+    pack_scales_kernel(const uint8_t* __restrict__ Sa, const uint8_t* __restrict__ Sb,
+                       int64_t rows_per_expert, int64_t half_rows, int64_t sf_row, int nb_count,
+                       int ks_count, int64_t n_words, uint32_t* __restrict__ packed) {
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_words;
+         w += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t blk = w >> 7;          // 128 words per 512-byte block
+        const int pos = (int)(w & 127);      // word position in the block
+        const int m = (pos >> 2) + 32 * (pos & 3);  // tile row this word holds
+        const int slab = (int)(blk % ks_count);
+        const int64_t eb = blk / ks_count;
+        const int nb = (int)(eb % nb_count);
+        const int64_t e = eb / nb_count;
+        const uint8_t* src;
+        int64_t row;
+        if (Sb != nullptr) {  // gate/up: 64 rows of W1, then 64 of W3
+            src = m < half_rows ? Sa : Sb;
+            row = (int64_t)nb * half_rows + (m < half_rows ? m : m - half_rows);
+        } else {
+            src = Sa;
+            row = (int64_t)nb * 128 + m;
+        }
+        const uint8_t* p = src + (e * rows_per_expert + row) * sf_row + 4 * slab;
+        packed[w] = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
+                    ((uint32_t)p[3] << 24);
+    }
+}
+
 template <bool SWIGLU>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                  const uint8_t* sfA, const uint8_t* sfB0, const uint8_t* sfB1, int64_t sfb_stride,
-                  const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, uint8_t* oq,
+                  const uint8_t* sfA, const uint8_t* sfBp, const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, uint8_t* oq,
                   uint8_t* os, __nv_bfloat16* ob, int64_t ldo, cudaStream_t st) {
     auto kern = mx_gemm_kernel<SWIGLU>;
     static bool attr_done[64] = {false};
@@ -454,7 +483,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     const int64_t sms = num_sms();
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
-    kern<<<grid, THREADS, SMEM_BYTES, st>>>(a, b0, b1, sfA, sfB0, sfB1, sfb_stride, offsets, (int)E,
+    kern<<<grid, THREADS, SMEM_BYTES, st>>>(a, b0, b1, sfA, sfBp, offsets, (int)E,
                                            (int)R, (int)K, (int)N, oq, os, ob, ldo, status_ptr());
     return launch_status();
 }
@@ -482,28 +511,56 @@ extern "C" int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T,
     return launch_status();
 }
 
-static int mx_check(const void* A, const void* As, const void* B, const void* Bs,
+static int mx_check(const void* A, const void* As, const void* B, const void* Bp,
                     const int32_t* offsets, int64_t E, int64_t R, int64_t d, int64_t F) {
     if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
     if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (R > INT32_MAX - 2 * mxg::BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
-    if (!offsets || !A || !As || !B || !Bs) return MOE_ERR_INVALID;
-    if (!aligned16(A) || !aligned16(B)) return MOE_ERR_INVALID;
-    // scale words are read as aligned 32-bit loads
-    if ((reinterpret_cast<uintptr_t>(As) & 3u) || (reinterpret_cast<uintptr_t>(Bs) & 3u))
-        return MOE_ERR_INVALID;
+    if (!offsets || !A || !As || !B || !Bp) return MOE_ERR_INVALID;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(Bp)) return MOE_ERR_INVALID;
+    // activation scale words are read as aligned 32-bit loads
+    if (reinterpret_cast<uintptr_t>(As) & 3u) return MOE_ERR_INVALID;
     return MOE_OK;
 }
 
+extern "C" int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s,
+                                        const uint8_t* W2s, int64_t E, int64_t d, int64_t F,
+                                        uint8_t* Ps13, uint8_t* Ps2, void* stream) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || d <= 0 || F <= 0) return MOE_ERR_INVALID;
+    if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if ((W1s == nullptr) != (W3s == nullptr) || (W1s == nullptr) != (Ps13 == nullptr))
+        return MOE_ERR_INVALID;
+    if ((W2s == nullptr) != (Ps2 == nullptr)) return MOE_ERR_INVALID;
+    if ((Ps13 && !aligned16(Ps13)) || (Ps2 && !aligned16(Ps2))) return MOE_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (Ps13) {  // gate/up tiles: 64 rows of W1 + 64 of W3 per n-block, K = d
+        const int nb = (int)(F / 64), ks = (int)(d / 128);
+        const int64_t words = E * nb * ks * 128;
+        int64_t g = (words + 255) / 256;
+        if (g > cap) g = cap;
+        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W1s, W3s, F, 64, d / 32, nb, ks, words,
+                                                       reinterpret_cast<uint32_t*>(Ps13));
+    }
+    if (Ps2) {   // down tiles: 128 rows of W2 per n-block, K = F
+        const int nb = (int)(d / 128), ks = (int)(F / 128);
+        const int64_t words = E * nb * ks * 128;
+        int64_t g = (words + 255) / 256;
+        if (g > cap) g = cap;
+        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W2s, nullptr, d, 128, F / 32, nb, ks,
+                                                       words, reinterpret_cast<uint32_t*>(Ps2));
+    }
+    return launch_status();
+}
+
 extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
-                                         const uint8_t* W1s, const uint8_t* W3q,
-                                         const uint8_t* W3s, int64_t w13_expert_stride,
-                                         const int32_t* offsets, int64_t E, int64_t R, int64_t d,
-                                         int64_t F, uint8_t* Hq, uint8_t* Hs, void* stream) {
-    int rc = mx_check(Xq, Xs, W1q, W1s, offsets, E, R, d, F);
+                                         const uint8_t* W3q, const uint8_t* Ps13,
+                                         int64_t w13_expert_stride, const int32_t* offsets,
+                                         int64_t E, int64_t R, int64_t d, int64_t F, uint8_t* Hq,
+                                         uint8_t* Hs, void* stream) {
+    int rc = mx_check(Xq, Xs, W1q, Ps13, offsets, E, R, d, F);
     if (rc != MOE_OK) return rc;
-    if (!W3q || !W3s || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq)) return MOE_ERR_INVALID;
-    if ((reinterpret_cast<uintptr_t>(W3s) & 3u)) return MOE_ERR_INVALID;
+    if (!W3q || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq)) return MOE_ERR_INVALID;
     if ((w13_expert_stride < F * d && E > 1) || w13_expert_stride % 128 != 0) return MOE_ERR_INVALID;
     if (R == 0) return MOE_OK;
     CUtensorMap a, b0, b1;
@@ -511,15 +568,15 @@ extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, c
         !make_map_3d(&b0, W1q, mxg::U8, 1, d, F, E, w13_expert_stride, 64) ||
         !make_map_3d(&b1, W3q, mxg::U8, 1, d, F, E, w13_expert_stride, 64))
         return MOE_ERR_CUDA;
-    return mxg::launch<true>(a, b0, b1, Xs, W1s, W3s, w13_expert_stride / 32, offsets, E, R, d, F,
-                             Hq, Hs, nullptr, F, as_stream(stream));
+    return mxg::launch<true>(a, b0, b1, Xs, Ps13, offsets, E, R, d, F, Hq, Hs, nullptr, F,
+                             as_stream(stream));
 }
 
 extern "C" int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const uint8_t* W2q,
-                                      const uint8_t* W2s, int64_t w2_expert_stride,
+                                      const uint8_t* Ps2, int64_t w2_expert_stride,
                                       const int32_t* offsets, int64_t E, int64_t R, int64_t d,
                                       int64_t F, void* Ye, void* stream) {
-    int rc = mx_check(Hq, Hs, W2q, W2s, offsets, E, R, d, F);
+    int rc = mx_check(Hq, Hs, W2q, Ps2, offsets, E, R, d, F);
     if (rc != MOE_OK) return rc;
     if (!Ye || !aligned16(Ye)) return MOE_ERR_INVALID;
     if ((w2_expert_stride < F * d && E > 1) || w2_expert_stride % 128 != 0) return MOE_ERR_INVALID;
@@ -528,7 +585,6 @@ extern "C" int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, cons
     if (!make_map_2d(&a, Hq, mxg::U8, 1, F, R, mxg::BM) ||
         !make_map_3d(&b0, W2q, mxg::U8, 1, F, d, E, w2_expert_stride, mxg::MMA_N))
         return MOE_ERR_CUDA;
-    return mxg::launch<false>(a, b0, b0, Hs, W2s, W2s, w2_expert_stride / 32, offsets, E, R, F, d,
-                              nullptr, nullptr, static_cast<__nv_bfloat16*>(Ye), d,
-                              as_stream(stream));
+    return mxg::launch<false>(a, b0, b0, Hs, Ps2, offsets, E, R, F, d, nullptr, nullptr,
+                              static_cast<__nv_bfloat16*>(Ye), d, as_stream(stream));
 }

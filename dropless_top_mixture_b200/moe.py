@@ -85,7 +85,7 @@ class LayerMxArgs(ctypes.Structure):
         ("k", ctypes.c_int32), ("renorm", ctypes.c_int32), ("reserved0", ctypes.c_int32),
         ("reserved1", ctypes.c_int32),
         ("x", _p), ("logits", _p), ("Wr", _p),
-        ("W1q", _p), ("W1s", _p), ("W3q", _p), ("W3s", _p), ("W2q", _p), ("W2s", _p),
+        ("W1q", _p), ("W3q", _p), ("W2q", _p), ("Ps13", _p), ("Ps2", _p),
         ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
         ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
         ("workspace", _p), ("workspace_bytes", _sz),
@@ -114,7 +114,8 @@ _SIGS = {
     "mxfp8_quantize": (_i32, [_p, _i32, _i64, _i64, _i32, _p, _p, _p]),
     "mxfp8_dequantize": (_i32, [_p, _p, _i32, _i64, _i64, _p, _p]),
     "moe_dispatch_mxfp8": (_i32, [_p, _p, _i64, _i64, _i32, _p, _p, _p]),
-    "moe_grouped_gate_up_mxfp8": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64,
+    "mxfp8_pack_weight_scales": (_i32, [_p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
+    "moe_grouped_gate_up_mxfp8": (_i32, [_p, _p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64,
                                          _p, _p, _p]),
     "moe_grouped_down_mxfp8": (_i32, [_p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _p]),
     "moe_layer_mxfp8_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
@@ -671,24 +672,47 @@ def moe_version() -> str:
 
 @dataclass
 class MxWeights:
-    """E4M3 codes and UE8M0 scales of W1, W3 [E,F,d] and W2 [E,d,F]."""
+    """E4M3 codes and UE8M0 scales of W1, W3 [E,F,d] and W2 [E,d,F], and the
+    scales packed for the GEMMs (mxfp8_pack_weight_scales; filled by
+    mxfp8_quantize_weights, or on first use)."""
     W1q: torch.Tensor
     W1s: torch.Tensor
     W3q: torch.Tensor
     W3s: torch.Tensor
     W2q: torch.Tensor
     W2s: torch.Tensor
+    Ps13: Optional[torch.Tensor] = None
+    Ps2: Optional[torch.Tensor] = None
+
+
+def mxfp8_pack_weight_scales(w: MxWeights) -> MxWeights:
+    E, F, d = w.W1q.shape
+    dev = w.W1q.device
+    w.Ps13 = torch.empty(E * (F // 64) * (d // 128) * 512, dtype=torch.uint8, device=dev)
+    w.Ps2 = torch.empty(E * (d // 128) * (F // 128) * 512, dtype=torch.uint8, device=dev)
+    for t in (w.W1s, w.W3s, w.W2s):
+        _need(t, "weight scales")
+    rc = lib.mxfp8_pack_weight_scales(_ptr(w.W1s), _ptr(w.W3s), _ptr(w.W2s), E, d, F,
+                                      _ptr(w.Ps13), _ptr(w.Ps2), _stream(w.W1q))
+    _check("mxfp8_pack_weight_scales", rc)
+    return w
+
+
+def _packed(w: MxWeights) -> MxWeights:
+    return w if w.Ps13 is not None else mxfp8_pack_weight_scales(w)
 
 
 def mxfp8_quantize_weights(W1, W3, W2) -> MxWeights:
     """Offline quantisation of the expert weights along their contraction
-    dimension (d for W1/W3, F for W2) with UE8M0 block scales."""
+    dimension (d for W1/W3, F for W2) with UE8M0 block scales, plus the
+    scales packed for the GEMMs."""
     E, F, d = W1.shape
     q1, s1 = mxfp8_quantize(W1.reshape(E * F, d), MOE_SCALE_E8M0)
     q3, s3 = mxfp8_quantize(W3.reshape(E * F, d), MOE_SCALE_E8M0)
     q2, s2 = mxfp8_quantize(W2.reshape(E * d, F), MOE_SCALE_E8M0)
-    return MxWeights(q1.view(E, F, d), s1.view(E, F, d // 32), q3.view(E, F, d),
-                     s3.view(E, F, d // 32), q2.view(E, d, F), s2.view(E, d, F // 32))
+    w = MxWeights(q1.view(E, F, d), s1.view(E, F, d // 32), q3.view(E, F, d),
+                  s3.view(E, F, d // 32), q2.view(E, d, F), s2.view(E, d, F // 32))
+    return mxfp8_pack_weight_scales(w)
 
 
 def moe_dispatch_mxfp8(x, slot, Xq=None, Xs=None):
@@ -712,9 +736,10 @@ def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None):
         Hq = torch.empty((R, F), dtype=torch.uint8, device=Xq.device)
     if Hs is None:
         Hs = torch.empty((R, F // 32), dtype=torch.uint8, device=Xq.device)
-    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xs), _ptr(w.W1q), _ptr(w.W1s), _ptr(w.W3q),
-                                       _ptr(w.W3s), w.W1q.stride(0), _ptr(offsets), E, R, d, F,
-                                       _ptr(Hq), _ptr(Hs), _stream(Xq))
+    w = _packed(w)
+    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xs), _ptr(w.W1q), _ptr(w.W3q), _ptr(w.Ps13),
+                                       w.W1q.stride(0), _ptr(offsets), E, R, d, F, _ptr(Hq),
+                                       _ptr(Hs), _stream(Xq))
     _check("moe_grouped_gate_up_mxfp8", rc)
     return Hq, Hs
 
@@ -725,7 +750,8 @@ def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None):
     R = Hq.shape[0]
     if Ye is None:
         Ye = torch.empty((R, d), dtype=torch.bfloat16, device=Hq.device)
-    rc = lib.moe_grouped_down_mxfp8(_ptr(Hq), _ptr(Hs), _ptr(w.W2q), _ptr(w.W2s), w.W2q.stride(0),
+    w = _packed(w)
+    rc = lib.moe_grouped_down_mxfp8(_ptr(Hq), _ptr(Hs), _ptr(w.W2q), _ptr(w.Ps2), w.W2q.stride(0),
                                     _ptr(offsets), E, R, d, F, _ptr(Ye), _stream(Hq))
     _check("moe_grouped_down_mxfp8", rc)
     return Ye
@@ -734,6 +760,7 @@ def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None):
 def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm: bool = False,
                         out: Optional[LayerOut] = None) -> LayerOut:
     _need(x, "x")
+    w = _packed(w)
     T, d = x.shape
     E, F, _ = w.W1q.shape
     dev = x.device
@@ -746,8 +773,8 @@ def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm
                        counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
                        slot=torch.empty((T, k), **i32), workspace=ws)
     a = LayerMxArgs(T=T, d=d, E=E, F=F, k=k, renorm=int(renorm), reserved0=0, reserved1=0,
-                    x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1q=_ptr(w.W1q), W1s=_ptr(w.W1s),
-                    W3q=_ptr(w.W3q), W3s=_ptr(w.W3s), W2q=_ptr(w.W2q), W2s=_ptr(w.W2s),
+                    x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1q=_ptr(w.W1q), W3q=_ptr(w.W3q),
+                    W2q=_ptr(w.W2q), Ps13=_ptr(w.Ps13), Ps2=_ptr(w.Ps2),
                     w13_expert_stride=w.W1q.stride(0), w2_expert_stride=w.W2q.stride(0),
                     out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
                     counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),

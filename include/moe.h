@@ -299,20 +299,35 @@ MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mod
  *   Weights are E4M3 codes with UE8M0 scales along their contraction
  *   dimension (mxfp8_quantize of W1/W3 as [E*F, d] and W2 as [E*d, F]):
  *   W1q/W3q [E,F,d] + W1s/W3s [E,F,d/32]; W2q [E,d,F] + W2s [E,d,F/32];
- *   expert strides in elements of the code tensors (scale strides are /32).
+ *   expert strides in elements of the code tensors. The GEMMs take the
+ *   weight scales packed once by mxfp8_pack_weight_scales (below).
  *   gate/up writes H quantised from its fp32 value: Hq [R,F] + Hs [R,F/32];
  *   down writes Ye [R,d] bf16. Limits: d % 128 == 0, F % 128 == 0; code
- *   pointers 16-byte aligned, scale pointers 4-byte aligned.
+ *   and packed-scale pointers 16-byte aligned, Xs/Hs 4-byte aligned.
+ *
+ * mxfp8_pack_weight_scales: the weight scales in the order the GEMMs'
+ *   tensor-core scale copy reads them, so each pipeline stage fetches them
+ *   with one bulk copy. For every expert, every 128-row B tile (gate/up:
+ *   rows 64nb..64nb+63 of W1 then the same rows of W3; down: rows
+ *   128nb..128nb+127 of W2) and every 128-element K slab s, a 512-byte
+ *   block holds the four scale bytes (K blocks 4s..4s+3) of tile row m at
+ *   byte 16*(m % 32) + 4*(m / 32); blocks ordered (expert, n-block, slab).
+ *   Ps13: E*(F/64)*(d/128)*512 bytes (from W1s, W3s); Ps2:
+ *   E*(d/128)*(F/128)*512 bytes (from W2s). Either pair may be NULL.
+ *   Scale tensors contiguous as above; packed outputs 16-byte aligned.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T, int64_t d, int k,
                                uint8_t* Xq, uint8_t* Xs, void* stream);
+MOE_API int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s, const uint8_t* W2s,
+                                     int64_t E, int64_t d, int64_t F, uint8_t* Ps13,
+                                     uint8_t* Ps2, void* stream);
 MOE_API int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
-                                      const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                      const uint8_t* W3q, const uint8_t* Ps13,
                                       int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
                                       int64_t R, int64_t d, int64_t F, uint8_t* Hq, uint8_t* Hs,
                                       void* stream);
 MOE_API int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const uint8_t* W2q,
-                                   const uint8_t* W2s, int64_t w2_expert_stride,
+                                   const uint8_t* Ps2, int64_t w2_expert_stride,
                                    const int32_t* offsets, int64_t E, int64_t R, int64_t d,
                                    int64_t F, void* Ye, void* stream);
 
@@ -325,11 +340,10 @@ typedef struct moe_layer_mxfp8_args {
     const float* logits;    /* [T,E] fp32, or NULL to use Wr                  */
     const void* Wr;         /* [E,d] bf16                                     */
     const uint8_t* W1q;
-    const uint8_t* W1s;
     const uint8_t* W3q;
-    const uint8_t* W3s;
     const uint8_t* W2q;
-    const uint8_t* W2s;
+    const uint8_t* Ps13;    /* packed gate/up weight scales (mxfp8_pack_weight_scales) */
+    const uint8_t* Ps2;     /* packed down weight scales                      */
     int64_t w13_expert_stride, w2_expert_stride;
     void* out;              /* [T,d] bf16                                     */
     int32_t* idx;

@@ -137,3 +137,43 @@ def test_layer_mxfp8_full_size_sampled():
     print(f"\nMXFP8 layer vs bf16 oracle: rel-L2 {gap:.4f}; "
           f"MXFP8 oracle vs bf16 oracle: rel-L2 {rel_l2(ref['out'], bf):.4f}")
     assert gap < 0.1
+
+
+@pytest.mark.parametrize("E,d,F", [(3, 256, 128), (2, 128, 384)])
+def test_pack_weight_scales_layout(E, d, F):
+    """The packed weight scales are a permutation of the row-layout scale
+    bytes, as the header defines it: block (e, nb, s) of 512 bytes, tile row
+    m's four K-block bytes at 16*(m % 32) + 4*(m / 32)."""
+    moe = _moe()
+    g = torch.Generator().manual_seed(E + d + F)
+    s1 = torch.randint(0, 256, (E, F, d // 32), generator=g, dtype=torch.uint8)
+    s3 = torch.randint(0, 256, (E, F, d // 32), generator=g, dtype=torch.uint8)
+    s2 = torch.randint(0, 256, (E, d, F // 32), generator=g, dtype=torch.uint8)
+    z = lambda *sh: torch.zeros(*sh, dtype=torch.uint8, device="cuda")
+    w = moe.MxWeights(z(E, F, d), s1.cuda(), z(E, F, d), s3.cuda(), z(E, d, F), s2.cuda())
+    moe.mxfp8_pack_weight_scales(w)
+    got13 = w.Ps13.cpu().numpy()
+    got2 = w.Ps2.cpu().numpy()
+
+    def block(rows_bytes):            # rows_bytes: [128 rows, 4 bytes]
+        b = np.zeros(512, dtype=np.uint8)
+        for m in range(128):
+            o = 16 * (m % 32) + 4 * (m // 32)
+            b[o:o + 4] = rows_bytes[m]
+        return b
+
+    want13 = []
+    for e in range(E):
+        for nb in range(F // 64):
+            rows = np.concatenate([s1[e, 64 * nb:64 * nb + 64].numpy(),
+                                   s3[e, 64 * nb:64 * nb + 64].numpy()])
+            for s in range(d // 128):
+                want13.append(block(rows[:, 4 * s:4 * s + 4]))
+    want2 = []
+    for e in range(E):
+        for nb in range(d // 128):
+            rows = s2[e, 128 * nb:128 * nb + 128].numpy()
+            for s in range(F // 128):
+                want2.append(block(rows[:, 4 * s:4 * s + 4]))
+    assert np.array_equal(got13, np.concatenate(want13))
+    assert np.array_equal(got2, np.concatenate(want2))
