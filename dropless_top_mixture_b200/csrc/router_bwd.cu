@@ -36,8 +36,8 @@ constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int JB = 8;           // expert rows in flight per thread
 constexpr int EPL_MAX = MOE_MAX_EXPERTS / 32;  // logits per lane, aux kernel
-constexpr int AUX_MAX_BLOCKS = 512;
-constexpr int AUX_TOKENS_MIN = 32;
+constexpr int AUX_MAX_BLOCKS = 128;
+constexpr int AUX_TOKENS_MIN = 64;
 
 template <int DT>
 struct Vec;
@@ -241,28 +241,29 @@ __global__ void __launch_bounds__(THREADS)
     }
 }
 
-// aux = E * sum_e (counts[e]/T) * (P_sum[e]/T), P_sum[e] = sum over blocks of
-// partial[b][e] in block order; the expert terms are added in a fixed tree.
+// aux = E * sum_e (counts[e]/T) * (P_sum[e]/T). Warp w takes experts w,
+// w + WARPS, ...: lane l adds the partials of blocks l, l + 32, ... in order,
+// a fixed butterfly adds the lanes, and the expert terms are added in a
+// fixed tree, so the result is deterministic.
 __global__ void __launch_bounds__(THREADS)
     aux_final_kernel(const float* __restrict__ partial, int nblocks,
                      const int32_t* __restrict__ counts, int T, int E, float* __restrict__ aux) {
-    __shared__ float s_term[THREADS];
-    const int tid = threadIdx.x;
+    __shared__ float s_term[WARPS];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float term = 0.f;
-    for (int e = tid; e < E; e += THREADS) {
+    for (int e = warp; e < E; e += WARPS) {
         float P = 0.f;
-        for (int b = 0; b < nblocks; ++b) P += partial[(size_t)b * E + e];
+        for (int b = lane; b < nblocks; b += 32) P += partial[(size_t)b * E + e];
+        P = warp_sum(P);
         term += (float)counts[e] * P;
     }
-    s_term[tid] = term;
+    if (lane == 0) s_term[warp] = term;
     __syncthreads();
-    for (int w = THREADS / 2; w > 0; w >>= 1) {
-        if (tid < w) s_term[tid] += s_term[tid + w];
-        __syncthreads();
-    }
     if (tid == 0) {
+        float sum = 0.f;
+        for (int w = 0; w < WARPS; ++w) sum += s_term[w];
         const float invT = 1.0f / (float)T;
-        aux[0] = (float)E * s_term[0] * invT * invT;
+        aux[0] = (float)E * sum * invT * invT;
     }
 }
 
