@@ -599,7 +599,7 @@ def main(argv=None):
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide T and E by this factor (profiling a small case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=2,
+    ap.add_argument("--e2e-chunks", type=int, default=3,
                     help="token slices of the host-buffer forward (copies overlap compute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",

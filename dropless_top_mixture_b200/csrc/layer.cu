@@ -160,15 +160,26 @@ extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
     cudaStream_t sc = as_stream(stream), si = as_stream(stream_h2d), so = as_stream(stream_d2h);
     const size_t es = a->dtype == MOE_F32 ? 4 : 2;
     const int64_t T = a->T, d = a->d, E = a->E, k = a->k;
-    const int64_t Tc = (T + chunks - 1) / chunks;
+    // Slice boundaries: with three or more slices the first and the last are
+    // half the size of the others, so the copy-in before the first compute
+    // and the copy-out after the last one (the parts nothing overlaps) are
+    // short. bound(i) = T * w(i) / W, w = 0, 0.5, 1.5, ..., W - 0.5, W.
+    auto bound = [&](int i) -> int64_t {
+        if (i <= 0) return 0;
+        if (i >= chunks) return T;
+        if (chunks < 3) return T * i / chunks;
+        const int64_t W2 = 2 * (chunks - 1);  // total weight, in halves
+        return T * (2 * i - 1) / W2;
+    };
     // the staging buffers may still be in use by work enqueued on `stream`
     // before this call: the copy-ins wait for it
     if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS + 1], sc) != cudaSuccess ||
         cudaStreamWaitEvent(si, ev[2 * layer::MAX_CHUNKS + 1], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
     int n = 0;
-    for (int64_t t0 = 0; t0 < T; t0 += Tc, ++n) {
-        const int64_t tn = (T - t0 < Tc) ? T - t0 : Tc;
+    for (int i = 0; i < chunks; ++i) {
+        const int64_t t0 = bound(i), tn = bound(i + 1) - t0;
+        if (tn <= 0) continue;
         const size_t xoff = (size_t)t0 * d * es, xbytes = (size_t)tn * d * es;
         char* xd = static_cast<char*>(const_cast<void*>(a->x)) + xoff;
         if (cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + xoff, xbytes,
@@ -199,6 +210,7 @@ extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
         if (cudaMemcpyAsync(static_cast<char*>(out_host) + xoff, s.out, xbytes,
                             cudaMemcpyDeviceToHost, so) != cudaSuccess)
             return MOE_ERR_CUDA;
+        ++n;
     }
     if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS], so) != cudaSuccess ||
         cudaStreamWaitEvent(sc, ev[2 * layer::MAX_CHUNKS], 0) != cudaSuccess)

@@ -483,7 +483,7 @@ class HostLayer:
     repeated calls of one shape allocate nothing."""
 
     def __init__(self, T: int, d: int, E: int, F: int, k: int, dtype: torch.dtype, device,
-                 *, logits_given: bool, chunks: int = 2):
+                 *, logits_given: bool, chunks: int = 3):
         if not 1 <= chunks <= 64:
             raise ValueError("chunks must be in [1, 64]")
         dev = torch.device(device)

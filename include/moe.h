@@ -408,7 +408,10 @@ MOE_API int moe_layer_fwd(const moe_layer_args* args, void* stream);
  * cut into `chunks` consecutive token slices (<= 64): slice c is copied in
  * on `stream_h2d`, computed on `stream`, and copied out on `stream_d2h`, so
  * the copy-in of slice c+1 and the copy-out of slice c-1 run while slice c
- * computes. Every token's output equals moe_layer_fwd's bit for bit.
+ * computes. With three or more slices the first and the last hold half as
+ * many tokens as the others (slice i ends at token T*(2i+1)/(2(chunks-1)),
+ * the last at T), which shortens the copies nothing overlaps. Every token's
+ * output equals moe_layer_fwd's bit for bit.
  *   args        as for moe_layer_fwd; args->x (and args->logits) and
  *               args->out are device staging buffers for the whole batch
  *               ([T,d], [T,E], [T,d]); idx, gate and slot receive the

@@ -30,10 +30,21 @@ def _problem(T, d, F, E, k, dtype, seed):
     return x, W1, W3, W2, Wr, lg
 
 
+def _slice_bounds(T, chunks):
+    """Token slices of the host pipeline: equal for one or two slices; from
+    three on, the first and the last are half the size of the others."""
+    if chunks < 3:
+        return [T * i // chunks for i in range(chunks + 1)]
+    w2 = 2 * (chunks - 1)
+    return [0] + [T * (2 * i - 1) // w2 for i in range(1, chunks)] + [T]
+
+
 def _check_slices(slot, T, k, chunks):
-    Tc = -(-T // chunks)
-    for t0 in range(0, T, Tc):
-        s = slot[t0:t0 + Tc].reshape(-1)
+    b = _slice_bounds(T, chunks)
+    for t0, t1 in zip(b[:-1], b[1:]):
+        if t1 <= t0:
+            continue
+        s = slot[t0:t1].reshape(-1)
         assert np.array_equal(np.sort(s), np.arange(s.size))
 
 
