@@ -530,11 +530,15 @@ def _e2e(moe, w, inp, dev, world, args, backward):
     x_d = torch.empty_like(x)
     lg_d = torch.empty_like(logits) if logits is not None else None
     h2d = x.numel() * x.element_size() + (logits.numel() * 4 if logits is not None else 0)
+    if args.e2e_chunks <= 0:
+        wbytes = 3 * w.E * w.F * w.d * (1 if w.mxfp8 else x.element_size())
+        args.e2e_chunks = moe.choose_chunks(T, w.d, x.element_size(), wbytes)
     if w.mxfp8:
+        # token slices whose copies overlap the compute (moe_layer_fwd_mxfp8_host)
         mw = moe.mxfp8_quantize_weights(W1, W3, W2)
-        lo = moe.moe_layer_fwd_mxfp8(x, k, mw, logits=logits, Wr=Wr)
-        res = lo.out
-        run = lambda: moe.moe_layer_fwd_mxfp8(x_d, k, mw, logits=lg_d, Wr=Wr, out=lo)
+        hlm = moe.HostLayerMxfp8(T, w.d, w.E, w.F, k, dev, logits_given=logits is not None,
+                                 chunks=args.e2e_chunks)
+        res = hlm.res.out
     elif backward:
         dO_h = inp["dOut"].cpu().pin_memory()
         dO_d = torch.empty_like(inp["dOut"])
@@ -554,7 +558,10 @@ def _e2e(moe, w, inp, dev, world, args, backward):
         res = hl.res.out
     res_h = torch.empty(res.shape, dtype=res.dtype).pin_memory()
 
-    if not w.mxfp8 and not backward:
+    if w.mxfp8:
+        def e2e_step():
+            hlm(x_h, mw, logits_host=lg_h, Wr=Wr, out_host=res_h)
+    elif not backward:
         def e2e_step():
             hl(x_h, W1, W3, W2, logits_host=lg_h, Wr=Wr, out_host=res_h)
     else:
@@ -580,7 +587,7 @@ def _e2e(moe, w, inp, dev, world, args, backward):
     ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
     r = {"value": T * world * args.steps / (ms_e2e / 1e3), "unit": UNIT,
          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": res.numel() * res.element_size()}
-    if not w.mxfp8 and not backward:
+    if not backward:
         r["pipeline_chunks"] = args.e2e_chunks
     return r
 
@@ -599,8 +606,9 @@ def main(argv=None):
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide T and E by this factor (profiling a small case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=3,
-                    help="token slices of the host-buffer forward (copies overlap compute)")
+    ap.add_argument("--e2e-chunks", type=int, default=0,
+                    help="token slices of the host-buffer forward (copies overlap compute); "
+                         "0 = chosen from the copy and weight-streaming times (moe.choose_chunks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true",
                     help="skip nvidia-smi clock sampling (for runs under a profiler)")

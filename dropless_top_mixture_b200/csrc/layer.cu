@@ -143,6 +143,73 @@ static cudaEvent_t* pipeline_events() {
 }  // namespace layer
 }  // namespace moe
 
+namespace moe {
+namespace layer {
+
+// The copy / compute / copy pipeline over token slices shared by the bf16
+// and MXFP8 host entry points. run(t0, tn, x_slice, logits_slice, out_slice)
+// enqueues the layer for tokens t0..t0+tn-1 on `sc`. x and out rows are
+// row_bytes long. With three or more slices the first and the last are half
+// the size of the others, so the copy-in before the first compute and the
+// copy-out after the last one (the parts nothing overlaps) are short:
+// slice i ends at T * (2i + 1) / (2 (chunks - 1)), the last at T.
+template <typename Run>
+static int host_pipeline(int64_t T, int64_t E, size_t row_bytes, void* x_dev,
+                         const float* logits_dev, void* out_dev, const void* x_host,
+                         const float* logits_host, void* out_host, int chunks, cudaStream_t sc,
+                         cudaStream_t si, cudaStream_t so, Run&& run) {
+    cudaEvent_t* ev = pipeline_events();
+    if (!ev) return MOE_ERR_CUDA;
+    auto bound = [&](int i) -> int64_t {
+        if (i <= 0) return 0;
+        if (i >= chunks) return T;
+        if (chunks < 3) return T * i / chunks;
+        return T * (2 * i - 1) / (2 * (chunks - 1));
+    };
+    // the staging buffers may still be in use by work enqueued on `sc`
+    // before this call: the copy-ins wait for it
+    if (cudaEventRecord(ev[2 * MAX_CHUNKS + 1], sc) != cudaSuccess ||
+        cudaStreamWaitEvent(si, ev[2 * MAX_CHUNKS + 1], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int n = 0;
+    for (int i = 0; i < chunks; ++i) {
+        const int64_t t0 = bound(i), tn = bound(i + 1) - t0;
+        if (tn <= 0) continue;
+        const size_t off = (size_t)t0 * row_bytes, bytes = (size_t)tn * row_bytes;
+        char* xd = static_cast<char*>(x_dev) + off;
+        if (cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + off, bytes,
+                            cudaMemcpyHostToDevice, si) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        float* ld = nullptr;
+        if (logits_dev) {
+            ld = const_cast<float*>(logits_dev) + (size_t)t0 * E;
+            if (cudaMemcpyAsync(ld, logits_host + (size_t)t0 * E, (size_t)tn * E * sizeof(float),
+                                cudaMemcpyHostToDevice, si) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
+        if (cudaEventRecord(ev[2 * n], si) != cudaSuccess ||
+            cudaStreamWaitEvent(sc, ev[2 * n], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        char* od = static_cast<char*>(out_dev) + off;
+        const int rc = run(t0, tn, xd, ld, od);
+        if (rc != MOE_OK) return rc;
+        if (cudaEventRecord(ev[2 * n + 1], sc) != cudaSuccess ||
+            cudaStreamWaitEvent(so, ev[2 * n + 1], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaMemcpyAsync(static_cast<char*>(out_host) + off, od, bytes, cudaMemcpyDeviceToHost,
+                            so) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        ++n;
+    }
+    if (cudaEventRecord(ev[2 * MAX_CHUNKS], so) != cudaSuccess ||
+        cudaStreamWaitEvent(sc, ev[2 * MAX_CHUNKS], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // namespace layer
+}  // namespace moe
+
 extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
                                   const float* logits_host, void* out_host, int chunks,
                                   void* stream, void* stream_h2d, void* stream_d2h) {
@@ -155,67 +222,48 @@ extern "C" int moe_layer_fwd_host(const moe_layer_args* a, const void* x_host,
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->k < 1) return MOE_ERR_INVALID;
     if (a->dtype != MOE_BF16 && a->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
     if (a->T == 0) return moe_layer_fwd(a, stream);
-    cudaEvent_t* ev = layer::pipeline_events();
-    if (!ev) return MOE_ERR_CUDA;
-    cudaStream_t sc = as_stream(stream), si = as_stream(stream_h2d), so = as_stream(stream_d2h);
     const size_t es = a->dtype == MOE_F32 ? 4 : 2;
-    const int64_t T = a->T, d = a->d, E = a->E, k = a->k;
-    // Slice boundaries: with three or more slices the first and the last are
-    // half the size of the others, so the copy-in before the first compute
-    // and the copy-out after the last one (the parts nothing overlaps) are
-    // short. bound(i) = T * w(i) / W, w = 0, 0.5, 1.5, ..., W - 0.5, W.
-    auto bound = [&](int i) -> int64_t {
-        if (i <= 0) return 0;
-        if (i >= chunks) return T;
-        if (chunks < 3) return T * i / chunks;
-        const int64_t W2 = 2 * (chunks - 1);  // total weight, in halves
-        return T * (2 * i - 1) / W2;
-    };
-    // the staging buffers may still be in use by work enqueued on `stream`
-    // before this call: the copy-ins wait for it
-    if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS + 1], sc) != cudaSuccess ||
-        cudaStreamWaitEvent(si, ev[2 * layer::MAX_CHUNKS + 1], 0) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    int n = 0;
-    for (int i = 0; i < chunks; ++i) {
-        const int64_t t0 = bound(i), tn = bound(i + 1) - t0;
-        if (tn <= 0) continue;
-        const size_t xoff = (size_t)t0 * d * es, xbytes = (size_t)tn * d * es;
-        char* xd = static_cast<char*>(const_cast<void*>(a->x)) + xoff;
-        if (cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + xoff, xbytes,
-                            cudaMemcpyHostToDevice, si) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        float* ld = nullptr;
-        if (a->logits) {
-            ld = const_cast<float*>(a->logits) + (size_t)t0 * E;
-            if (cudaMemcpyAsync(ld, logits_host + (size_t)t0 * E, (size_t)tn * E * sizeof(float),
-                                cudaMemcpyHostToDevice, si) != cudaSuccess)
-                return MOE_ERR_CUDA;
-        }
-        if (cudaEventRecord(ev[2 * n], si) != cudaSuccess || cudaStreamWaitEvent(sc, ev[2 * n], 0) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        moe_layer_args s = *a;
-        s.T = tn;
-        s.x = xd;
-        s.logits = ld;
-        s.out = static_cast<char*>(a->out) + xoff;
-        s.idx = a->idx + (size_t)t0 * k;
-        s.gate = a->gate + (size_t)t0 * k;
-        s.slot = a->slot + (size_t)t0 * k;
-        const int rc = moe_layer_fwd(&s, stream);
-        if (rc != MOE_OK) return rc;
-        if (cudaEventRecord(ev[2 * n + 1], sc) != cudaSuccess ||
-            cudaStreamWaitEvent(so, ev[2 * n + 1], 0) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        if (cudaMemcpyAsync(static_cast<char*>(out_host) + xoff, s.out, xbytes,
-                            cudaMemcpyDeviceToHost, so) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        ++n;
-    }
-    if (cudaEventRecord(ev[2 * layer::MAX_CHUNKS], so) != cudaSuccess ||
-        cudaStreamWaitEvent(sc, ev[2 * layer::MAX_CHUNKS], 0) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    return MOE_OK;
+    const int64_t k = a->k;
+    return layer::host_pipeline(
+        a->T, a->E, (size_t)a->d * es, const_cast<void*>(a->x), a->logits, a->out, x_host,
+        logits_host, out_host, chunks, as_stream(stream), as_stream(stream_h2d),
+        as_stream(stream_d2h), [&](int64_t t0, int64_t tn, void* xs, float* ls, void* os) {
+            moe_layer_args s = *a;
+            s.T = tn;
+            s.x = xs;
+            s.logits = ls;
+            s.out = os;
+            s.idx = a->idx + (size_t)t0 * k;
+            s.gate = a->gate + (size_t)t0 * k;
+            s.slot = a->slot + (size_t)t0 * k;
+            return moe_layer_fwd(&s, stream);
+        });
+}
+
+extern "C" int moe_layer_fwd_mxfp8_host(const moe_layer_mxfp8_args* a, const void* x_host,
+                                        const float* logits_host, void* out_host, int chunks,
+                                        void* stream, void* stream_h2d, void* stream_d2h) {
+    if (!a || !x_host || !out_host || chunks < 1 || chunks > layer::MAX_CHUNKS) return MOE_ERR_INVALID;
+    if ((a->logits == nullptr) != (logits_host == nullptr)) return MOE_ERR_INVALID;
+    if (stream == stream_h2d || stream == stream_d2h || stream_h2d == stream_d2h)
+        return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->T == 0) return moe_layer_fwd_mxfp8(a, stream);
+    const int64_t k = a->k;
+    return layer::host_pipeline(
+        a->T, a->E, (size_t)a->d * 2, const_cast<void*>(a->x), a->logits, a->out, x_host,
+        logits_host, out_host, chunks, as_stream(stream), as_stream(stream_h2d),
+        as_stream(stream_d2h), [&](int64_t t0, int64_t tn, void* xs, float* ls, void* os) {
+            moe_layer_mxfp8_args s = *a;
+            s.T = tn;
+            s.x = xs;
+            s.logits = ls;
+            s.out = os;
+            s.idx = a->idx + (size_t)t0 * k;
+            s.gate = a->gate + (size_t)t0 * k;
+            s.slot = a->slot + (size_t)t0 * k;
+            return moe_layer_fwd_mxfp8(&s, stream);
+        });
 }
 
 extern "C" size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype) {

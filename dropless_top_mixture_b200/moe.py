@@ -120,6 +120,8 @@ _SIGS = {
     "moe_grouped_down_mxfp8": (_i32, [_p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _p]),
     "moe_layer_mxfp8_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
     "moe_layer_fwd_mxfp8": (_i32, [ctypes.POINTER(LayerMxArgs), _p]),
+    "moe_layer_fwd_mxfp8_host": (_i32, [ctypes.POINTER(LayerMxArgs), _p, _p, _p, _i32, _p, _p,
+                                        _p]),
     "moe_layer_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32, _i32]),
     "moe_layer_fwd": (_i32, [ctypes.POINTER(LayerArgs), _p]),
     "moe_layer_fwd_host": (_i32, [ctypes.POINTER(LayerArgs), _p, _p, _p, _i32, _p, _p, _p]),
@@ -475,6 +477,25 @@ def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool =
     return out
 
 
+# Nominal bandwidths for choosing the host pipeline's slice count: pinned
+# host <-> device copies over PCIe Gen5 x16, and HBM for re-streaming the
+# expert weights once per slice.
+PCIE_GBS = 55.0
+HBM_GBS = 6500.0
+
+
+def choose_chunks(T: int, d: int, act_esize: int, weight_bytes: int, max_chunks: int = 8) -> int:
+    """Slice count for the host pipeline. With c slices the time is about
+    compute + c * Wt + Ct * h(c): every slice streams the weights once (Wt),
+    and of the copies (Ct per direction) what nothing overlaps is 2 Ct for
+    one slice, Ct for two, and Ct / (c - 1) from three on (half-size first
+    and last slices). Returns the c that minimises c * Wt + Ct * h(c)."""
+    ct = T * d * act_esize / (PCIE_GBS * 1e9)
+    wt = weight_bytes / (HBM_GBS * 1e9)
+    h = lambda c: 2.0 if c == 1 else (1.0 if c == 2 else 1.0 / (c - 1))
+    return min(range(1, max_chunks + 1), key=lambda c: c * wt + ct * h(c))
+
+
 class HostLayer:
     """moe_layer_fwd_host: the layer from pinned host x (and logits) to
     pinned host out, cut into `chunks` token slices whose copy-in, compute
@@ -782,3 +803,58 @@ def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm
     rc = lib.moe_layer_fwd_mxfp8(ctypes.byref(a), _stream(x))
     _check("moe_layer_fwd_mxfp8", rc)
     return out
+
+
+class HostLayerMxfp8:
+    """moe_layer_fwd_mxfp8_host: the MXFP8 layer from pinned host x (bf16,
+    and logits) to pinned host out (bf16), in `chunks` token slices whose
+    copies overlap the compute. Holds the staging buffers, routing outputs,
+    workspace and copy streams, so repeated calls of one shape allocate
+    nothing."""
+
+    def __init__(self, T: int, d: int, E: int, F: int, k: int, device, *, logits_given: bool,
+                 chunks: int = 3):
+        if not 1 <= chunks <= 64:
+            raise ValueError("chunks must be in [1, 64]")
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.T, self.d, self.E, self.F, self.k = T, d, E, F, k
+        self.chunks = chunks
+        self.x = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_given else None
+        self.res = LayerOut(out=torch.empty((T, d), dtype=torch.bfloat16, device=dev),
+                            idx=torch.empty((T, k), **i32),
+                            gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                            counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+                            slot=torch.empty((T, k), **i32),
+                            workspace=_alloc_ws(lib.moe_layer_mxfp8_workspace_size(
+                                T, d, E, F, k, int(logits_given)), dev))
+        self.s_h2d = torch.cuda.Stream(dev)
+        self.s_d2h = torch.cuda.Stream(dev)
+
+    def __call__(self, x_host: torch.Tensor, w: MxWeights, *, logits_host=None, Wr=None,
+                 renorm: bool = False, out_host: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if x_host.is_cuda or tuple(x_host.shape) != (self.T, self.d) or x_host.dtype != torch.bfloat16:
+            raise ValueError("x_host must be a [T, d] bf16 host tensor")
+        if (logits_host is None) != (self.logits is None):
+            raise ValueError("logits_host must be given exactly when the layer was built for it")
+        if logits_host is not None and (logits_host.is_cuda or logits_host.dtype != torch.float32
+                                        or tuple(logits_host.shape) != (self.T, self.E)):
+            raise ValueError("logits_host must be a [T, E] fp32 host tensor")
+        if out_host is None:
+            out_host = torch.empty((self.T, self.d), dtype=torch.bfloat16, pin_memory=True)
+        w = _packed(w)
+        r = self.res
+        a = LayerMxArgs(T=self.T, d=self.d, E=self.E, F=self.F, k=self.k, renorm=int(renorm),
+                        reserved0=0, reserved1=0, x=_ptr(self.x), logits=_ptr(self.logits),
+                        Wr=_ptr(Wr), W1q=_ptr(w.W1q), W3q=_ptr(w.W3q), W2q=_ptr(w.W2q),
+                        Ps13=_ptr(w.Ps13), Ps2=_ptr(w.Ps2), w13_expert_stride=w.W1q.stride(0),
+                        w2_expert_stride=w.W2q.stride(0), out=_ptr(r.out), idx=_ptr(r.idx),
+                        gate=_ptr(r.gate), counts=_ptr(r.counts), offsets=_ptr(r.offsets),
+                        slot=_ptr(r.slot), workspace=_ptr(r.workspace),
+                        workspace_bytes=r.workspace.numel())
+        rc = lib.moe_layer_fwd_mxfp8_host(ctypes.byref(a), x_host.data_ptr(), _ptr(logits_host),
+                                          out_host.data_ptr(), self.chunks, _stream(self.x),
+                                          self.s_h2d.cuda_stream, self.s_d2h.cuda_stream)
+        _check("moe_layer_fwd_mxfp8_host", rc)
+        return out_host

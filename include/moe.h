@@ -358,6 +358,14 @@ typedef struct moe_layer_mxfp8_args {
 MOE_API size_t moe_layer_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
                                               int logits_given);
 MOE_API int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* args, void* stream);
+/* moe_layer_fwd_mxfp8_host — moe_layer_fwd_mxfp8 from and to host memory in
+ * token slices with the copies overlapped, exactly as moe_layer_fwd_host
+ * (x and out are bf16 [T,d] host buffers; args->x, ->logits, ->out are the
+ * device staging buffers). Every token's output equals the one-shot call's
+ * bit for bit. */
+MOE_API int moe_layer_fwd_mxfp8_host(const moe_layer_mxfp8_args* args, const void* x_host,
+                                     const float* logits_host, void* out_host, int chunks,
+                                     void* stream, void* stream_h2d, void* stream_d2h);
 
 /* ------------------------------------------------------------------------
  * moe_layer_fwd — the whole layer: route -> dispatch -> grouped SwiGLU ->

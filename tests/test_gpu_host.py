@@ -125,3 +125,20 @@ def test_host_pipeline_full_size():
     assert moe.moe_get_status() == 0
     assert torch.equal(out, ref.out.cpu())
     assert torch.equal(hl.res.idx.cpu(), ref.idx.cpu())
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 5])
+def test_mxfp8_host_pipeline_matches_device_call(chunks):
+    moe = _moe()
+    T, d, F, E, k = 700, 256, 256, 8, 2
+    x, W1, W3, W2, Wr, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=31 + chunks)
+    dev = "cuda"
+    w = moe.mxfp8_quantize_weights(W1.to(dev), W3.to(dev), W2.to(dev))
+    ref = moe.moe_layer_fwd_mxfp8(x.to(dev), k, w, logits=lg.to(dev))
+    hl = moe.HostLayerMxfp8(T, d, E, F, k, dev, logits_given=True, chunks=chunks)
+    out = hl(x.pin_memory(), w, logits_host=lg.pin_memory())
+    torch.cuda.current_stream().synchronize()
+    assert moe.moe_get_status() == 0
+    assert torch.equal(out, ref.out.cpu())
+    assert torch.equal(hl.res.idx.cpu(), ref.idx.cpu())
+    _check_slices(hl.res.slot.cpu().numpy(), T, k, chunks)
