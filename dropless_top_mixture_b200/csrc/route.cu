@@ -12,11 +12,13 @@
 //
 // Routing metadata is a stable counting sort of the token-major (t, j) list
 // by expert, built in three launches:
-//   1. topk_chunk: one warp per chunk of CHUNK consecutive tokens. It selects
-//      the k experts of each token in order and keeps, per expert, a running
-//      count inside the chunk; the count before a token's hit is that
-//      token's rank among the chunk's rows of the expert (stable by token).
-//      Per-chunk counts go to ws_count[e][c].
+//   1. topk_group: one CTA per chunk of 8 to 32 consecutive tokens (a group
+//      of 1 to 16 lanes per token, by E). It selects the k experts of each
+//      token in order, marks each selection in a per-expert bit mask over the
+//      chunk's tokens, and reads a token's rank among the chunk's rows of the
+//      expert (stable by token) off the mask. Per-chunk counts go to
+//      ws_count[e][c]. When the logits are computed, it also adds the router's
+//      four quarter planes (and writes the logits out if asked).
 //   2. scan: one block per expert scans ws_count[e][:] over chunks (exclusive,
 //      in place) and writes counts[e]; the last block to finish (ticket
 //      counter) scans counts into offsets and tile_offsets.
@@ -28,7 +30,6 @@
 namespace moe {
 namespace route {
 
-constexpr int CHUNK = 8;           // tokens per warp in topk_chunk
 constexpr int LOGIT_TT = 64;       // tokens per router-logits tile
 constexpr int LOGIT_TE = 64;       // experts per router-logits tile
 constexpr int LOGIT_TK = 32;       // contraction chunk staged in shared memory
@@ -71,7 +72,7 @@ struct Stage8<float> {
 // each from +0.0 in ascending j, their sums added in order ((c0 + c1) + c2)
 // + c3. One CTA (128 threads) computes one quarter's chains for a 64-token x
 // 64-expert tile (grid z = quarter) and writes them to that quarter's plane;
-// sum_quarters_kernel adds the four planes. Thread (ty, tx) owns tokens
+// the top-k kernel adds the four planes in order. Thread (ty, tx) owns tokens
 // 8ty..8ty+7 and experts 4tx..4tx+3, each with its own fp32 accumulator.
 // Rows of x and Wr are staged 32 columns at a time, transposed into k-major
 // shared memory (two buffers, one barrier per chunk; a warp writes 32
@@ -161,139 +162,169 @@ __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* 
     }
 }
 
-// logits[i] = ((p0[i] + p1[i]) + p2[i]) + p3[i] over the four quarter planes
-// (plane stride pstride floats, a multiple of 64; planes and logits 16-byte
-// aligned), four floats per thread step, the last n % 4 one at a time.
-__global__ void __launch_bounds__(256) sum_quarters_kernel(const float* __restrict__ planes,
-                                                           int64_t n, int64_t pstride,
-                                                           float* __restrict__ logits) {
-    const int64_t nv = n / 4, sv = pstride / 4;
-    const float4* p = reinterpret_cast<const float4*>(planes);
-    float4* o = reinterpret_cast<float4*>(logits);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float4 a = __ldcs(p + i);
-#pragma unroll
-        for (int q = 1; q < LOGIT_SPLIT; ++q) {
-            const float4 b = __ldcs(p + q * sv + i);
-            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-        }
-        o[i] = a;
-    }
-    for (int64_t i = nv * 4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float a = planes[i];
-#pragma unroll
-        for (int q = 1; q < LOGIT_SPLIT; ++q) a += planes[q * pstride + i];
-        logits[i] = a;
-    }
-}
-
 // ------------------------------------------------------------------ a1
 
-// Total order used by the top-k: larger logit first, then lower index.
-__device__ __forceinline__ bool beats(float av, int ai, float bv, int bi) {
-    if (ai < 0) return false;
-    if (bi < 0) return true;
-    return av > bv || (av == bv && ai < bi);
+// Top-k on G lanes per token. Lane g of a token's group holds the logits of
+// experts g*VPL .. g*VPL + VPL - 1 in registers; G is the smallest power of
+// two with 32*G >= E and VPL = ceil(E/G) rounded up to a multiple of 8, so
+// every lane holds at most 32. A token's k selections are k rounds of: a
+// tournament over the lane's untaken logits (lower expert first on equal
+// values), then a butterfly over the G lanes of the group. The order is
+// total (larger logit first, then lower index), so every lane of the group
+// agrees on the winner and the result is the stable descending sort's first
+// k. NaN stands for "taken or absent" inside the kernel; an input NaN is
+// read as -inf (ranks below every number).
+//
+// One CTA is one chunk of CH tokens (CH = 32 for E <= 128, 16 for E <= 256,
+// 8 above). Each selection sets the token's bit in a shared-memory mask of
+// its expert; after a barrier the rank of (t, e) within the chunk is the
+// count of the mask's bits below t, and popc of the whole mask is the chunk
+// count ws_count[e][chunk].
+//
+// The logits are read from nplanes planes pstride floats apart and added in
+// plane order ((p0 + p1) + p2) + p3 (nplanes = 4: the router's quarter
+// chains; 1: logits given by the caller); logits_out, when not null,
+// receives the sums.
+constexpr int topk_group_of(int E) {
+    int g = 1;
+    while (32 * g < E) g *= 2;
+    return g;
+}
+constexpr int topk_vpl_of(int E, int G) { return ((E + G - 1) / G + 7) / 8 * 8; }
+constexpr int topk_threads_of(int G) { return 32 * G < 128 ? 32 * G : 128; }
+
+__device__ __forceinline__ bool is_num(float a) { return a == a; }
+
+// (bv, be) <- the better of itself and (ov, oe); NaN never wins.
+__device__ __forceinline__ void keep_better(float ov, int oe, float& bv, int& be) {
+    const bool o_wins = is_num(ov) && (!is_num(bv) || ov > bv || (ov == bv && oe < be));
+    bv = o_wins ? ov : bv;
+    be = o_wins ? oe : be;
 }
 
-// EPL = experts per lane (ceil(E/32)); expert e lives in lane e%32, slot e/32.
-template <int EPL>
-__global__ void __launch_bounds__(128) topk_chunk_kernel(
-    const float* __restrict__ logits, int T, int E, int k, int renorm, int nchunks,
-    int32_t* __restrict__ idx, float* __restrict__ gate, int32_t* __restrict__ rank,
-    int32_t* __restrict__ ws_count) {
-    const int lane = threadIdx.x & 31;
-    const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (c >= nchunks) return;
-    int cnt[EPL];
-#pragma unroll
-    for (int q = 0; q < EPL; ++q) cnt[q] = 0;
+template <int G, int VPL>
+__global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
+    const float* __restrict__ src, int nplanes, int64_t pstride, int vec, int T, int E, int k,
+    int renorm, int nchunks, float* __restrict__ logits_out, int32_t* __restrict__ idx,
+    float* __restrict__ gate, int32_t* __restrict__ rank, int32_t* __restrict__ ws_count) {
+    constexpr int NT = topk_threads_of(G);
+    constexpr int CH = NT / G;  // tokens per chunk (<= 32: one mask word per expert)
+    __shared__ uint32_t hits[32 * G];
+    const int c = blockIdx.x;
+    const int g = threadIdx.x % G;
+    const int tl = threadIdx.x / G;
+    const int t = c * CH + tl;
+    const bool live = t < T;
+    for (int i = threadIdx.x; i < E; i += NT) hits[i] = 0u;
+    __syncthreads();
 
-    for (int i = 0; i < CHUNK; ++i) {
-        const int t = c * CHUNK + i;
-        if (t >= T) break;
-        const float* row = logits + (size_t)t * E;
-        float v[EPL];
-        float mx = -INFINITY;
+    const int e0 = g * VPL;
+    float v[VPL];
 #pragma unroll
-        for (int q = 0; q < EPL; ++q) {
-            const int e = lane + 32 * q;
-            float a = (e < E) ? __ldg(row + e) : -INFINITY;
-            if (isnan(a)) a = -INFINITY;
-            v[q] = a;
-            mx = fmaxf(mx, a);
-        }
-        mx = warp_max(mx);
-        float s = 0.f;
+    for (int q = 0; q < VPL; ++q) v[q] = __int_as_float(0x7fc00000);
+    if (live) {
+        const float* row = src + (size_t)t * E;
+        if (vec) {
 #pragma unroll
-        for (int q = 0; q < EPL; ++q) {
-            const int e = lane + 32 * q;
-            if (e < E) s += expf(v[q] - mx);
-        }
-        s = warp_sum(s);
-
-        uint32_t taken = 0;
-        int my_e = 0, my_r = 0;
-        float my_g = 0.f;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = -1;
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) {
-                const int e = lane + 32 * q;
-                if (e < E && !((taken >> q) & 1u) && beats(v[q], e, bv, be)) {
-                    bv = v[q];
-                    be = e;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (beats(ov, oe, bv, be)) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            // be is the same in every lane; its owner marks it and hands out
-            // the in-chunk rank (count before this hit).
-            int r = 0;
-            if ((be & 31) == lane) {
-                const int qq = be >> 5;
-#pragma unroll
-                for (int q = 0; q < EPL; ++q)
-                    if (q == qq) {
-                        r = cnt[q];
-                        cnt[q] = r + 1;
-                        taken |= 1u << q;
+            for (int q = 0; q < VPL; q += 4) {
+                if (e0 + q < E) {  // E % 4 == 0: the whole float4 is in the row
+                    float4 a = __ldg(reinterpret_cast<const float4*>(row + e0 + q));
+                    for (int p = 1; p < nplanes; ++p) {
+                        const float4 b =
+                            __ldg(reinterpret_cast<const float4*>(row + p * pstride + e0 + q));
+                        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
                     }
+                    v[q] = a.x; v[q + 1] = a.y; v[q + 2] = a.z; v[q + 3] = a.w;
+                    if (logits_out)
+                        *reinterpret_cast<float4*>(logits_out + (size_t)t * E + e0 + q) = a;
+                }
             }
-            r = __shfl_sync(0xffffffffu, r, be & 31);
-            const float g = expf(bv - mx) / s;
-            if (lane == j) {
-                my_e = be;
-                my_g = g;
-                my_r = r;
-            }
-        }
-        if (renorm) {
-            float gs = 0.f;
-            for (int j = 0; j < k; ++j) gs += __shfl_sync(0xffffffffu, my_g, j);
-            my_g = my_g / gs;
-        }
-        if (lane < k) {
-            idx[(size_t)t * k + lane] = my_e;
-            gate[(size_t)t * k + lane] = my_g;
-            rank[(size_t)t * k + lane] = my_r;
-        }
-    }
+        } else {
 #pragma unroll
-    for (int q = 0; q < EPL; ++q) {
-        const int e = lane + 32 * q;
-        if (e < E) ws_count[(size_t)e * nchunks + c] = cnt[q];
+            for (int q = 0; q < VPL; ++q) {
+                if (e0 + q < E) {
+                    float a = __ldg(row + e0 + q);
+                    for (int p = 1; p < nplanes; ++p) a += __ldg(row + p * pstride + e0 + q);
+                    v[q] = a;
+                    if (logits_out) logits_out[(size_t)t * E + e0 + q] = a;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < VPL; ++q)
+            if (e0 + q < E && !is_num(v[q])) v[q] = -INFINITY;
     }
+
+    // softmax denominator: max over the group, then a pairwise sum of the
+    // lane's exp terms and a butterfly over the group
+    float mx = v[0];
+#pragma unroll
+    for (int q = 1; q < VPL; ++q) mx = fmaxf(mx, v[q]);
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float ex[VPL];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) ex[q] = is_num(v[q]) ? expf(v[q] - mx) : 0.f;
+#pragma unroll
+    for (int w = 1; w < VPL; w <<= 1)
+#pragma unroll
+        for (int q = 0; q + w < VPL; q += 2 * w) ex[q] += ex[q + w];
+    float s = ex[0];
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+
+    float gsum = 0.f;
+    for (int j = 0; j < k; ++j) {
+        // tournament over the lane's logits; on equal values the lower slot
+        // (lower expert) is kept
+        float tv[VPL];
+        int tq[VPL];
+#pragma unroll
+        for (int q = 0; q < VPL; ++q) {
+            tv[q] = v[q];
+            tq[q] = q;
+        }
+#pragma unroll
+        for (int w = 1; w < VPL; w <<= 1)
+#pragma unroll
+            for (int q = 0; q + w < VPL; q += 2 * w) {
+                const bool r = is_num(tv[q + w]) && !(tv[q + w] <= tv[q]);
+                tv[q] = r ? tv[q + w] : tv[q];
+                tq[q] = r ? tq[q + w] : tq[q];
+            }
+        float bv = tv[0];
+        int be = e0 + tq[0];
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            keep_better(ov, oe, bv, be);
+        }
+        // the owner lane retires the winner
+        const int qq = be - e0;
+#pragma unroll
+        for (int q = 0; q < VPL; ++q)
+            if (q == qq) v[q] = __int_as_float(0x7fc00000);
+        const float gj = expf(bv - mx) / s;
+        gsum += gj;
+        if (live) {
+            if (g == j % G) {
+                idx[(size_t)t * k + j] = be;
+                gate[(size_t)t * k + j] = gj;
+            }
+            if (qq >= 0 && qq < VPL) atomicOr(&hits[be], 1u << tl);
+        }
+    }
+    __syncthreads();
+    if (live) {
+        const uint32_t below = (1u << tl) - 1u;
+        for (int j = g; j < k; j += G) {
+            const int e = idx[(size_t)t * k + j];  // this thread's own store above
+            rank[(size_t)t * k + j] = __popc(hits[e] & below);
+            if (renorm) gate[(size_t)t * k + j] = gate[(size_t)t * k + j] / gsum;
+        }
+    }
+    for (int e = threadIdx.x; e < E; e += NT) ws_count[(size_t)e * nchunks + c] = __popc(hits[e]);
 }
 
 // ------------------------------------------------------------------ a2
@@ -381,7 +412,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(int E, int nchunks,
     if (threadIdx.x == 0) *ticket = 0;
 }
 
-__global__ void finalize_kernel(int T, int k, int E, int nchunks, const int32_t* __restrict__ idx,
+__global__ void finalize_kernel(int T, int k, int E, int chunk, int nchunks,
+                                const int32_t* __restrict__ idx,
                                 const int32_t* __restrict__ offsets,
                                 const int32_t* __restrict__ ws_count, int32_t* __restrict__ slot,
                                 int* status) {
@@ -394,36 +426,33 @@ __global__ void finalize_kernel(int T, int k, int E, int nchunks, const int32_t*
         set_status(status, MOE_DEVERR_BAD_INDEX);
         return;
     }
-    const int c = t / CHUNK;
+    const int c = t / chunk;
     slot[i] = offsets[e] + ws_count[(size_t)e * nchunks + c] + slot[i];
 }
 
 // ------------------------------------------------------------------ host
 
-inline int64_t nchunks_of(int64_t T) { return (T + CHUNK - 1) / CHUNK; }
+// The chunk counts are sized for the smallest chunk (8 tokens, E > 256), so
+// the workspace is a function of (T, E, from_x) alone.
+constexpr int MIN_CHUNK = 8;
+inline int64_t max_chunks_of(int64_t T) { return (T + MIN_CHUNK - 1) / MIN_CHUNK; }
 
 inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 struct RouteWs {
     int32_t* count;
     int32_t* ticket;
-    float* logits;  // the [T,E] logits when computed and not returned
-    float* planes;  // the four [T,E] quarter planes when computed
+    float* planes;  // the four [T,E] quarter planes when the logits are computed
 };
 
-// from_x: the logits are computed from x and Wr. The workspace then holds the
-// four quarter planes and a [T,E] logits buffer (used when the caller does
-// not ask for the logits), whatever logits_out is, so the size is a function
-// of (T, E, from_x) alone.
+// from_x: the logits are computed from x and Wr; the workspace then also
+// holds the four quarter planes (the top-k adds them itself).
 inline int64_t plane_stride(int64_t T, int64_t E) { return (T * E + 63) / 64 * 64; }
 
 inline size_t workspace_bytes(int64_t T, int64_t E, bool from_x) {
-    size_t b = align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
+    size_t b = align256(sizeof(int32_t) * (size_t)E * (size_t)max_chunks_of(T));
     b += 256;  // ticket
-    if (from_x) {
-        b += align256(sizeof(float) * (size_t)T * (size_t)E);
-        b += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
-    }
+    if (from_x) b += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
     return b;
 }
 
@@ -431,23 +460,36 @@ inline RouteWs carve(void* ws, int64_t T, int64_t E, bool from_x) {
     char* p = static_cast<char*>(ws);
     RouteWs r;
     r.count = reinterpret_cast<int32_t*>(p);
-    p += align256(sizeof(int32_t) * (size_t)E * (size_t)nchunks_of(T));
+    p += align256(sizeof(int32_t) * (size_t)E * (size_t)max_chunks_of(T));
     r.ticket = reinterpret_cast<int32_t*>(p);
     p += 256;
-    r.logits = from_x ? reinterpret_cast<float*>(p) : nullptr;
-    p += from_x ? align256(sizeof(float) * (size_t)T * (size_t)E) : 0;
     r.planes = from_x ? reinterpret_cast<float*>(p) : nullptr;
     return r;
 }
 
-template <int EPL>
-static void launch_topk(const float* logits, int T, int E, int k, int renorm, int nch,
-                        int32_t* idx, float* gate, int32_t* rank, int32_t* wsc,
-                        cudaStream_t st) {
-    const int warps_per_block = 4;
-    const int blocks = (nch + warps_per_block - 1) / warps_per_block;
-    topk_chunk_kernel<EPL><<<blocks, 32 * warps_per_block, 0, st>>>(logits, T, E, k, renorm, nch,
-                                                                    idx, gate, rank, wsc);
+// Launches the top-k for E experts; returns the chunk size (tokens per
+// chunk) or 0 if E is outside 1..512.
+static int launch_topk(const float* src, int nplanes, int64_t pstride, int T, int E, int k,
+                       int renorm, float* logits_out, int32_t* idx, float* gate, int32_t* rank,
+                       int32_t* wsc, cudaStream_t st) {
+    const int G = topk_group_of(E);
+    const int V = topk_vpl_of(E, G);
+    const int nt = topk_threads_of(G);
+    const int ch = nt / G;
+    const int nch = (T + ch - 1) / ch;
+    const int vec = (E % 4 == 0) && aligned16(src) && (!logits_out || aligned16(logits_out));
+#define MOE_TOPK_CASE(g, v)                                                                    \
+    if (G == g && V == v) {                                                                    \
+        topk_group_kernel<g, v><<<nch, nt, 0, st>>>(src, nplanes, pstride, vec, T, E, k,      \
+                                                    renorm, nch, logits_out, idx, gate, rank, \
+                                                    wsc);                                      \
+        return ch;                                                                             \
+    }
+    MOE_TOPK_CASE(1, 8) MOE_TOPK_CASE(1, 16) MOE_TOPK_CASE(1, 24) MOE_TOPK_CASE(1, 32)
+    MOE_TOPK_CASE(2, 24) MOE_TOPK_CASE(2, 32) MOE_TOPK_CASE(4, 24) MOE_TOPK_CASE(4, 32)
+    MOE_TOPK_CASE(8, 24) MOE_TOPK_CASE(8, 32) MOE_TOPK_CASE(16, 24) MOE_TOPK_CASE(16, 32)
+#undef MOE_TOPK_CASE
+    return 0;
 }
 
 }  // namespace route
@@ -497,9 +539,7 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     cudaStream_t st = as_stream(stream);
     route::RouteWs ws = route::carve(workspace, T, E, from_x);
 
-    const float* lg = logits;
     if (from_x) {
-        float* dst = logits_out ? logits_out : ws.logits;
         dim3 grid((unsigned)((T + route::LOGIT_TT - 1) / route::LOGIT_TT),
                   (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE), route::LOGIT_SPLIT);
         if (dtype == MOE_BF16)
@@ -510,36 +550,20 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
             route::router_logits_kernel<float><<<grid, route::LOGIT_THREADS, 0, st>>>(
                 static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d,
                 (int)E, ws.planes, route::plane_stride(T, E));
-        const int64_t n = T * E;
-        int64_t g = (n / 4 + 255) / 256;
-        const int64_t cap = (int64_t)num_sms() * 8;
-        if (g > cap) g = cap;
-        if (g < 1) g = 1;
-        route::sum_quarters_kernel<<<(int)g, 256, 0, st>>>(ws.planes, n,
-                                                           route::plane_stride(T, E), dst);
-        lg = dst;
     }
-    const int nch = (int)route::nchunks_of(T);
     // the in-chunk ranks are parked in `slot` and completed by finalize_kernel
-    switch ((E + 31) / 32) {
-#define MOE_TOPK_CASE(n)                                                                       \
-    case n:                                                                                    \
-        route::launch_topk<n>(lg, (int)T, (int)E, k, renorm, nch, idx, gate, slot, ws.count, \
-                              st);                                                             \
-        break;
-        MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4)
-        MOE_TOPK_CASE(5) MOE_TOPK_CASE(6) MOE_TOPK_CASE(7) MOE_TOPK_CASE(8)
-        MOE_TOPK_CASE(9) MOE_TOPK_CASE(10) MOE_TOPK_CASE(11) MOE_TOPK_CASE(12)
-        MOE_TOPK_CASE(13) MOE_TOPK_CASE(14) MOE_TOPK_CASE(15) MOE_TOPK_CASE(16)
-#undef MOE_TOPK_CASE
-        default:
-            return MOE_ERR_UNSUPPORTED;
-    }
+    const int chunk = from_x ? route::launch_topk(ws.planes, route::LOGIT_SPLIT,
+                                                  route::plane_stride(T, E), (int)T, (int)E, k,
+                                                  renorm, logits_out, idx, gate, slot, ws.count, st)
+                             : route::launch_topk(logits, 1, 0, (int)T, (int)E, k, renorm,
+                                                  nullptr, idx, gate, slot, ws.count, st);
+    if (chunk == 0) return MOE_ERR_UNSUPPORTED;
+    const int nch = (int)((T + chunk - 1) / chunk);
     if (cudaMemsetAsync(ws.ticket, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     route::scan_kernel<<<(unsigned)E, route::SCAN_THREADS, 0, st>>>(
         (int)E, nch, ws.count, counts, offsets, tile_offsets, ws.ticket);
     const int64_t n = T * k;
     route::finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        (int)T, k, (int)E, nch, idx, offsets, ws.count, slot, status_ptr());
+        (int)T, k, (int)E, chunk, nch, idx, offsets, ws.count, slot, status_ptr());
     return launch_status();
 }

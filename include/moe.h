@@ -101,8 +101,8 @@ extern "C" {
  *   tile_offsets [E+1] int32 exclusive prefix sum of ceil(counts/128), or NULL
  * Workspace: `workspace_bytes` >= moe_route_workspace_size(T, E,
  *            logits == NULL); 256-byte aligned device memory (with logits
- *            computed it holds the four quarter sums and, when logits_out
- *            is NULL, the logits). Its contents need not be initialised.
+ *            computed it holds the four quarter sums, which the top-k adds
+ *            itself). Its contents need not be initialised.
  * Limits: 1 <= k <= min(E, 32), E <= 512; when computing logits d % 128 == 0
  *            and logits_out (if given) 16-byte aligned.
  * ---------------------------------------------------------------------- */
@@ -127,7 +127,7 @@ MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dt
  *   - Size limit: moe_route_workspace_size(T, E, logits == NULL) must not
  *     exceed MOE_ROUTE_NOALLOC_SCRATCH_BYTES, else MOE_ERR_UNSUPPORTED and
  *     nothing is launched. (E = 64 with logits computed from x fits up to
- *     T = 6,393 tokens; E = 128 with logits given up to T = 131,064; E = 384
+ *     T = 7,943 tokens; E = 128 with logits given up to T = 131,064; E = 384
  *     with logits given up to T = 43,688.)
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make

@@ -36,15 +36,17 @@ def gate_tolerance(logits: np.ndarray, idx: np.ndarray, renorm: bool) -> np.ndar
 
     exp(l - max) in fp32: the subtraction rounds (|l-max| * 2^-24 absolute in
     the exponent's argument), expf adds at most 2 ulp; the denominator is a
-    sum of E positive terms done as ceil(E/32) sequential adds per lane and a
-    5-level butterfly; one division. Each term contributes at most 2^-24
-    relative; the bound below doubles it for margin.
+    sum of E positive terms done as a pairwise tree over each lane's (at most
+    32) terms and a butterfly over the lanes of the token's group, so a term
+    passes through at most ceil(log2 E) + 1 roundings (adding an exact zero
+    for an absent expert is exact); one division. Each rounding contributes
+    at most 2^-24 relative; the bound below doubles it for margin.
     """
     T, E = logits.shape
     lg = logits.astype(np.float64)
     mx = lg.max(axis=1, keepdims=True)
     sel = np.take_along_axis(lg, idx.astype(np.int64), axis=1)
-    terms = np.abs(sel - mx) + math.ceil(E / 32) + 5 + 2 + 2
+    terms = np.abs(sel - mx) + math.ceil(math.log2(E)) + 1 + 2 + 2
     if renorm:
         terms = terms + idx.shape[1] + 2
     return terms * 2.0 ** -23

@@ -33,11 +33,29 @@ def _check_route(r, lg_np, k, E, renorm=False):
 
 @pytest.mark.parametrize("kind", ["normal", "dups", "constant", "signed_zero"])
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (7, 8, 8), (37, 33, 5), (300, 64, 8), (1000, 128, 4),
-                                   (257, 384, 8), (64, 512, 32), (50, 1, 1)])
+                                   (257, 384, 8), (64, 512, 32), (50, 1, 1),
+                                   # one case per (lanes per token, logits per lane) shape
+                                   # of the top-k: (1,16) (1,24) (1,32) (2,32) (4,24)
+                                   # (8,24) (8,32) (16,32) besides those above
+                                   (40, 16, 3), (129, 20, 6), (65, 32, 32), (70, 52, 7),
+                                   (100, 80, 8), (70, 160, 8), (90, 256, 16), (33, 500, 9)])
 def test_route_from_logits_bitexact(kind, T, E, k):
     moe = _moe()
     lg = adversarial_logits(T, E, kind, seed=T + E)
     r = moe.moe_route(k, logits=lg.cuda())
+    _check_route(r, lg.numpy(), k, E)
+
+
+def test_route_logits_not_16_byte_aligned():
+    """Logits whose rows are not 16-byte aligned take the scalar loads."""
+    moe = _moe()
+    T, E, k = 95, 64, 8
+    lg = adversarial_logits(T, E, "dups", seed=3)
+    flat = torch.empty(T * E + 1, device="cuda")
+    view = flat[1:].view(T, E)
+    view.copy_(lg.cuda())
+    assert view.data_ptr() % 16 != 0
+    r = moe.moe_route(k, logits=view)
     _check_route(r, lg.numpy(), k, E)
 
 
