@@ -32,115 +32,133 @@ namespace route {
 
 constexpr int LOGIT_TT = 64;       // tokens per router-logits tile
 constexpr int LOGIT_TE = 64;       // experts per router-logits tile
-constexpr int LOGIT_TK = 32;       // contraction chunk staged in shared memory
+constexpr int LOGIT_TK = 16;       // contraction chunk staged in shared memory
 constexpr int LOGIT_LD = 68;       // padded row of the staged chunk (floats)
+constexpr int LOGIT_D_ALIGN = 128; // d must be a multiple of this
 
 // ------------------------------------------------------------------ a0
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 template <typename TX>
-struct Stage8;  // loads 8 consecutive elements as fp32
+struct Landed16;  // 16 consecutive elements of a row in shared memory, as fp32
 
 template <>
-struct Stage8<__nv_bfloat16> {
-    __device__ static void load(const __nv_bfloat16* p, bool ok, float* f) {
-        if (ok) {
-            uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-            unpack8(u, f);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = 0.f;
-        }
+struct Landed16<__nv_bfloat16> {
+    __device__ static void to_f32(const uint4* p, float* f) {
+        unpack8(p[0], f);
+        unpack8(p[1], f + 8);
     }
 };
 
 template <>
-struct Stage8<float> {
-    __device__ static void load(const float* p, bool ok, float* f) {
-        if (ok) {
-            float4 a = __ldg(reinterpret_cast<const float4*>(p));
-            float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-            f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-        } else {
+struct Landed16<float> {
+    __device__ static void to_f32(const uint4* p, float* f) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = reinterpret_cast<const float4*>(p)[i];
+            f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
         }
     }
 };
 
 // The logit of (t, e) is four fmaf chains, one per contiguous quarter of j,
 // each from +0.0 in ascending j, their sums added in order ((c0 + c1) + c2)
-// + c3. One CTA (128 threads) computes one quarter's chains for a 64-token x
+// + c3. One CTA (64 threads) computes one quarter's chains for a 64-token x
 // 64-expert tile (grid z = quarter) and writes them to that quarter's plane;
-// the top-k kernel adds the four planes in order. Thread (ty, tx) owns tokens
-// 8ty..8ty+7 and experts 4tx..4tx+3, each with its own fp32 accumulator.
-// Rows of x and Wr are staged 32 columns at a time, transposed into k-major
-// shared memory (two buffers, one barrier per chunk; a warp writes 32
-// consecutive rows of one column, so the transposing stores do not conflict);
-// the next chunk is prefetched into registers while the current one is
-// consumed. Per column: 3 shared loads feed 32 FMAs.
-constexpr int LOGIT_THREADS = 128;
+// the top-k kernel adds the four planes in order. Eight CTAs are resident
+// per SM, so the 1024 CTAs of the OLMoE shape run as one wave.
+//   staging: thread i copies 16 consecutive elements of x row t0 + i and of
+//            Wr row e0 + i per chunk into its own landing slots with
+//            cp.async (one chunk ahead), then converts them to fp32 into
+//            k-major shared memory (a warp writes 32 consecutive floats of
+//            one k: no conflicts);
+//   compute: thread (ty, tx) = (i / 8, i % 8) owns tokens 4ty..4ty+3 and
+//            32+4ty..32+4ty+3 and experts 4tx..4tx+3 and 32+4tx..32+4tx+3:
+//            64 accumulators; per k, 4 shared float4 loads (the eight tx of a
+//            phase read 128 consecutive bytes) feed 64 FMAs.
+constexpr int LOGIT_THREADS = 64;
 constexpr int LOGIT_SPLIT = 4;  // quarter chains per logit
 
 template <typename TX>
-__global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* __restrict__ x,
-                                                                      const TX* __restrict__ Wr,
-                                                                      int T, int d, int E,
-                                                                      float* __restrict__ planes,
-                                                                      int64_t pstride) {
+__global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
+    const TX* __restrict__ x, const TX* __restrict__ Wr, int T, int d, int E,
+    float* __restrict__ planes, int64_t pstride) {
+    constexpr int PIECES = LOGIT_TK * (int)sizeof(TX) / 16;  // 16-byte pieces per row chunk
+    constexpr int PEL = 16 / (int)sizeof(TX);                // elements per piece
     __shared__ __align__(16) float xs[2][LOGIT_TK][LOGIT_LD];
     __shared__ __align__(16) float ws[2][LOGIT_TK][LOGIT_LD];
+    __shared__ __align__(16) uint4 land[2][LOGIT_THREADS][PIECES];  // [x | Wr][row][piece]
     const int tid = threadIdx.x;
     const int t0 = blockIdx.x * LOGIT_TT;
     const int e0 = blockIdx.y * LOGIT_TE;
     const int dq = d / LOGIT_SPLIT;
     const int kbeg = blockIdx.z * dq;
     float* __restrict__ logits = planes + (size_t)blockIdx.z * pstride;
-    // staging role: row = tid % 64 (token or expert), columns (tid / 64) * 16 .. +15
-    const int srow = tid & 63;
-    const int scol = (tid >> 6) * 16;
-    const bool xok = (t0 + srow) < T;
-    const bool wok = (e0 + srow) < E;
-    const TX* xp = x + (size_t)(t0 + srow) * d + kbeg + scol;
-    const TX* wp = Wr + (size_t)(e0 + srow) * d + kbeg + scol;
-    // compute role
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[8][4];
+    const bool xok = (t0 + tid) < T;
+    const bool wok = (e0 + tid) < E;
+    // rows past T or E are zero-filled; their source address stays row 0's
+    const TX* xp = x + (size_t)(xok ? t0 + tid : 0) * d + kbeg;
+    const TX* wp = Wr + (size_t)(wok ? e0 + tid : 0) * d + kbeg;
+    const uint32_t lx = (uint32_t)__cvta_generic_to_shared(&land[0][tid][0]);
+    const uint32_t lw = (uint32_t)__cvta_generic_to_shared(&land[1][tid][0]);
+    const int ty = tid >> 3, tx = tid & 7;
+    float acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-    float fx[16], fw[16];
-    Stage8<TX>::load(xp, xok, fx);
-    Stage8<TX>::load(xp + 8, xok, fx + 8);
-    Stage8<TX>::load(wp, wok, fw);
-    Stage8<TX>::load(wp + 8, wok, fw + 8);
+#pragma unroll
+    for (int p = 0; p < PIECES; ++p) {
+        cp_async16(lx + 16 * p, xp + p * PEL, xok ? 16 : 0);
+        cp_async16(lw + 16 * p, wp + p * PEL, wok ? 16 : 0);
+    }
+    cp_async_commit();
     int buf = 0;
     for (int k0 = 0; k0 < dq; k0 += LOGIT_TK, buf ^= 1) {
+        cp_async_wait_all();  // this thread's own copies of chunk k0
+        {
+            float f[16];
+            Landed16<TX>::to_f32(&land[0][tid][0], f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            xs[buf][scol + i][srow] = fx[i];
-            ws[buf][scol + i][srow] = fw[i];
+            for (int i = 0; i < 16; ++i) xs[buf][i][tid] = f[i];
+            Landed16<TX>::to_f32(&land[1][tid][0], f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ws[buf][i][tid] = f[i];
         }
         __syncthreads();
         if (k0 + LOGIT_TK < dq) {
-            Stage8<TX>::load(xp + k0 + LOGIT_TK, xok, fx);
-            Stage8<TX>::load(xp + k0 + LOGIT_TK + 8, xok, fx + 8);
-            Stage8<TX>::load(wp + k0 + LOGIT_TK, wok, fw);
-            Stage8<TX>::load(wp + k0 + LOGIT_TK + 8, wok, fw + 8);
+#pragma unroll
+            for (int p = 0; p < PIECES; ++p) {
+                cp_async16(lx + 16 * p, xp + k0 + LOGIT_TK + p * PEL, xok ? 16 : 0);
+                cp_async16(lw + 16 * p, wp + k0 + LOGIT_TK + p * PEL, wok ? 16 : 0);
+            }
+            cp_async_commit();
         }
-#pragma unroll 4
+#pragma unroll
         for (int kk = 0; kk < LOGIT_TK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8 + 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
+            const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][32 + 4 * ty]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][kk][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][kk][32 + 4 * tx]);
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float bv[4] = {b.x, b.y, b.z, b.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         // no second barrier: the next chunk goes to the other buffer, and the
         // barrier after that write keeps any thread from overwriting this
@@ -148,16 +166,20 @@ __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* 
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int t = t0 + ty * 8 + i;
+        const int t = t0 + (i < 4 ? 4 * ty + i : 32 + 4 * ty + (i - 4));
         if (t >= T) continue;
-        const int e = e0 + tx * 4;
-        if (e + 3 < E && (E & 3) == 0) {
-            *reinterpret_cast<float4*>(&logits[(size_t)t * E + e]) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (e + j < E) logits[(size_t)t * E + e + j] = acc[i][j];
+        for (int h = 0; h < 2; ++h) {
+            const int e = e0 + 32 * h + 4 * tx;
+            const float* a = &acc[i][4 * h];
+            if (e + 3 < E && (E & 3) == 0) {
+                *reinterpret_cast<float4*>(&logits[(size_t)t * E + e]) =
+                    make_float4(a[0], a[1], a[2], a[3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (e + j < E) logits[(size_t)t * E + e + j] = a[j];
+            }
         }
     }
 }
@@ -165,32 +187,31 @@ __global__ void __launch_bounds__(LOGIT_THREADS) router_logits_kernel(const TX* 
 // ------------------------------------------------------------------ a1
 
 // Top-k on G lanes per token. Lane g of a token's group holds the logits of
-// experts g*VPL .. g*VPL + VPL - 1 in registers; G is the smallest power of
-// two with 32*G >= E and VPL = ceil(E/G) rounded up to a multiple of 8, so
-// every lane holds at most 32. A token's k selections are k rounds of: a
-// tournament over the lane's untaken logits (lower expert first on equal
-// values), then a butterfly over the G lanes of the group. The order is
-// total (larger logit first, then lower index), so every lane of the group
-// agrees on the winner and the result is the stable descending sort's first
-// k. NaN stands for "taken or absent" inside the kernel; an input NaN is
-// read as -inf (ranks below every number).
+// experts g*VPL .. g*VPL + VPL - 1 in registers (VPL a multiple of 8, at
+// most 32). G starts at the smallest power of two with 32*G >= E and is
+// doubled, while each lane keeps at least 8 logits and G <= 16, until the
+// launch has about 1024 threads per SM: the selection is a chain of
+// dependent steps, so it is latency-bound and wants many warps. A token's k
+// selections are k rounds of: a tournament over the lane's untaken logits
+// (lower expert first on equal values), then a butterfly over the G lanes of
+// the group. The order is total (larger logit first, then lower index), so
+// every lane of the group agrees on the winner and the result is the stable
+// descending sort's first k. NaN stands for "taken or absent" inside the
+// kernel; an input NaN is read as -inf (ranks below every number).
 //
-// One CTA is one chunk of CH tokens (CH = 32 for E <= 128, 16 for E <= 256,
-// 8 above). Each selection sets the token's bit in a shared-memory mask of
-// its expert; after a barrier the rank of (t, e) within the chunk is the
+// One CTA is one chunk of CH tokens (CH = 32 for G <= 4, 16 for G = 8, 8 for
+// G = 16). The rounds only record (expert, logit) in shared memory; then
+// each lane takes the selections j = g, g + G, ...: it sets the token's bit
+// in the shared-memory mask of the expert, computes the gate and writes idx
+// and gate. After a barrier the rank of (t, e) within the chunk is the
 // count of the mask's bits below t, and popc of the whole mask is the chunk
 // count ws_count[e][chunk].
 //
-// The logits are read from nplanes planes pstride floats apart and added in
-// plane order ((p0 + p1) + p2) + p3 (nplanes = 4: the router's quarter
-// chains; 1: logits given by the caller); logits_out, when not null,
-// receives the sums.
-constexpr int topk_group_of(int E) {
-    int g = 1;
-    while (32 * g < E) g *= 2;
-    return g;
-}
-constexpr int topk_vpl_of(int E, int G) { return ((E + G - 1) / G + 7) / 8 * 8; }
+// The logits are read from NP planes pstride floats apart and added in
+// plane order ((p0 + p1) + p2) + p3 (NP = 4: the router's quarter chains;
+// 1: logits given by the caller); logits_out, when not null, receives the
+// sums.
+constexpr int TOPK_MAX_G = 16;
 constexpr int topk_threads_of(int G) { return 32 * G < 128 ? 32 * G : 128; }
 
 __device__ __forceinline__ bool is_num(float a) { return a == a; }
@@ -202,21 +223,22 @@ __device__ __forceinline__ void keep_better(float ov, int oe, float& bv, int& be
     be = o_wins ? oe : be;
 }
 
-template <int G, int VPL>
-__global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
-    const float* __restrict__ src, int nplanes, int64_t pstride, int vec, int T, int E, int k,
-    int renorm, int nchunks, float* __restrict__ logits_out, int32_t* __restrict__ idx,
+template <int G, int VPL, int NP>
+__global__ void __launch_bounds__(topk_threads_of(G), 1) topk_group_kernel(
+    const float* __restrict__ src, int64_t pstride, int vec, int T, int E, int k, int renorm,
+    int nchunks, float* __restrict__ logits_out, int32_t* __restrict__ idx,
     float* __restrict__ gate, int32_t* __restrict__ rank, int32_t* __restrict__ ws_count) {
     constexpr int NT = topk_threads_of(G);
     constexpr int CH = NT / G;  // tokens per chunk (<= 32: one mask word per expert)
     __shared__ uint32_t hits[32 * G];
+    __shared__ int32_t sel[CH][MOE_MAX_TOPK];  // selected expert of round j
+    __shared__ float sval[CH][MOE_MAX_TOPK];   // its logit, then its gate
     const int c = blockIdx.x;
     const int g = threadIdx.x % G;
     const int tl = threadIdx.x / G;
     const int t = c * CH + tl;
     const bool live = t < T;
     for (int i = threadIdx.x; i < E; i += NT) hits[i] = 0u;
-    __syncthreads();
 
     const int e0 = g * VPL;
     float v[VPL];
@@ -229,7 +251,8 @@ __global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
             for (int q = 0; q < VPL; q += 4) {
                 if (e0 + q < E) {  // E % 4 == 0: the whole float4 is in the row
                     float4 a = __ldg(reinterpret_cast<const float4*>(row + e0 + q));
-                    for (int p = 1; p < nplanes; ++p) {
+#pragma unroll
+                    for (int p = 1; p < NP; ++p) {
                         const float4 b =
                             __ldg(reinterpret_cast<const float4*>(row + p * pstride + e0 + q));
                         a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
@@ -244,7 +267,8 @@ __global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
             for (int q = 0; q < VPL; ++q) {
                 if (e0 + q < E) {
                     float a = __ldg(row + e0 + q);
-                    for (int p = 1; p < nplanes; ++p) a += __ldg(row + p * pstride + e0 + q);
+#pragma unroll
+                    for (int p = 1; p < NP; ++p) a += __ldg(row + p * pstride + e0 + q);
                     v[q] = a;
                     if (logits_out) logits_out[(size_t)t * E + e0 + q] = a;
                 }
@@ -262,18 +286,20 @@ __global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
     for (int q = 1; q < VPL; ++q) mx = fmaxf(mx, v[q]);
 #pragma unroll
     for (int o = 1; o < G; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float ex[VPL];
+    float s;
+    {
+        float ex[VPL];
 #pragma unroll
-    for (int q = 0; q < VPL; ++q) ex[q] = is_num(v[q]) ? expf(v[q] - mx) : 0.f;
+        for (int q = 0; q < VPL; ++q) ex[q] = is_num(v[q]) ? expf(v[q] - mx) : 0.f;
 #pragma unroll
-    for (int w = 1; w < VPL; w <<= 1)
+        for (int w = 1; w < VPL; w <<= 1)
 #pragma unroll
-        for (int q = 0; q + w < VPL; q += 2 * w) ex[q] += ex[q + w];
-    float s = ex[0];
+            for (int q = 0; q + w < VPL; q += 2 * w) ex[q] += ex[q + w];
+        s = ex[0];
+    }
 #pragma unroll
     for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
 
-    float gsum = 0.f;
     for (int j = 0; j < k; ++j) {
         // tournament over the lane's logits; on equal values the lower slot
         // (lower expert) is kept
@@ -300,32 +326,42 @@ __global__ void __launch_bounds__(topk_threads_of(G)) topk_group_kernel(
             const int oe = __shfl_xor_sync(0xffffffffu, be, o);
             keep_better(ov, oe, bv, be);
         }
-        // the owner lane retires the winner
+        // the owner lane retires the winner; lane j % G records it
         const int qq = be - e0;
 #pragma unroll
         for (int q = 0; q < VPL; ++q)
             if (q == qq) v[q] = __int_as_float(0x7fc00000);
-        const float gj = expf(bv - mx) / s;
-        gsum += gj;
-        if (live) {
-            if (g == j % G) {
-                idx[(size_t)t * k + j] = be;
-                gate[(size_t)t * k + j] = gj;
-            }
-            if (qq >= 0 && qq < VPL) atomicOr(&hits[be], 1u << tl);
+        if (g == (j & (G - 1))) {
+            sel[tl][j] = be;
+            sval[tl][j] = bv;
+        }
+    }
+    // each lane finishes its own selections j = g, g + G, ...; with renorm
+    // the gates are written after the barrier, divided by their sum
+    const uint32_t bit = 1u << tl;
+    if (live) {
+        for (int j = g; j < k; j += G) {
+            const int e = sel[tl][j];
+            const float gj = expf(sval[tl][j] - mx) / s;
+            sval[tl][j] = gj;
+            atomicOr(&hits[e], bit);
+            idx[(size_t)t * k + j] = e;
+            if (!renorm) gate[(size_t)t * k + j] = gj;
         }
     }
     __syncthreads();
     if (live) {
-        const uint32_t below = (1u << tl) - 1u;
+        float gsum = 0.f;
+        if (renorm)
+            for (int j = 0; j < k; ++j) gsum += sval[tl][j];
         for (int j = g; j < k; j += G) {
-            const int e = idx[(size_t)t * k + j];  // this thread's own store above
-            rank[(size_t)t * k + j] = __popc(hits[e] & below);
-            if (renorm) gate[(size_t)t * k + j] = gate[(size_t)t * k + j] / gsum;
+            rank[(size_t)t * k + j] = __popc(hits[sel[tl][j]] & (bit - 1u));
+            if (renorm) gate[(size_t)t * k + j] = sval[tl][j] / gsum;
         }
     }
     for (int e = threadIdx.x; e < E; e += NT) ws_count[(size_t)e * nchunks + c] = __popc(hits[e]);
 }
+
 
 // ------------------------------------------------------------------ a2
 
@@ -472,23 +508,31 @@ inline RouteWs carve(void* ws, int64_t T, int64_t E, bool from_x) {
 static int launch_topk(const float* src, int nplanes, int64_t pstride, int T, int E, int k,
                        int renorm, float* logits_out, int32_t* idx, float* gate, int32_t* rank,
                        int32_t* wsc, cudaStream_t st) {
-    const int G = topk_group_of(E);
-    const int V = topk_vpl_of(E, G);
+    int G = 1;
+    while (32 * G < E) G *= 2;
+    const int64_t want_threads = (int64_t)num_sms() * 1024;
+    while (G < TOPK_MAX_G && (int64_t)T * G < want_threads && E >= 16 * G) G *= 2;
+    const int V = ((E + G - 1) / G + 7) / 8 * 8;
     const int nt = topk_threads_of(G);
     const int ch = nt / G;
     const int nch = (T + ch - 1) / ch;
     const int vec = (E % 4 == 0) && aligned16(src) && (!logits_out || aligned16(logits_out));
+#define MOE_TOPK_NP(g, v, np)                                                                  \
+    topk_group_kernel<g, v, np><<<nch, nt, 0, st>>>(src, pstride, vec, T, E, k, renorm, nch,  \
+                                                    logits_out, idx, gate, rank, wsc)
 #define MOE_TOPK_CASE(g, v)                                                                    \
     if (G == g && V == v) {                                                                    \
-        topk_group_kernel<g, v><<<nch, nt, 0, st>>>(src, nplanes, pstride, vec, T, E, k,      \
-                                                    renorm, nch, logits_out, idx, gate, rank, \
-                                                    wsc);                                      \
+        if (nplanes == 4)                                                                      \
+            MOE_TOPK_NP(g, v, 4);                                                              \
+        else                                                                                   \
+            MOE_TOPK_NP(g, v, 1);                                                              \
         return ch;                                                                             \
     }
-    MOE_TOPK_CASE(1, 8) MOE_TOPK_CASE(1, 16) MOE_TOPK_CASE(1, 24) MOE_TOPK_CASE(1, 32)
-    MOE_TOPK_CASE(2, 24) MOE_TOPK_CASE(2, 32) MOE_TOPK_CASE(4, 24) MOE_TOPK_CASE(4, 32)
-    MOE_TOPK_CASE(8, 24) MOE_TOPK_CASE(8, 32) MOE_TOPK_CASE(16, 24) MOE_TOPK_CASE(16, 32)
+#define MOE_TOPK_G(g) MOE_TOPK_CASE(g, 8) MOE_TOPK_CASE(g, 16) MOE_TOPK_CASE(g, 24) MOE_TOPK_CASE(g, 32)
+    MOE_TOPK_G(1) MOE_TOPK_G(2) MOE_TOPK_G(4) MOE_TOPK_G(8) MOE_TOPK_G(16)
+#undef MOE_TOPK_G
 #undef MOE_TOPK_CASE
+#undef MOE_TOPK_NP
     return 0;
 }
 
@@ -525,7 +569,7 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     }
     const bool from_x = (logits == nullptr);
     if (from_x) {
-        if (!x || !Wr || d <= 0 || (d % (route::LOGIT_SPLIT * route::LOGIT_TK)) != 0)
+        if (!x || !Wr || d <= 0 || (d % route::LOGIT_D_ALIGN) != 0)
             return MOE_ERR_INVALID;
         if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
         if (!aligned16(x) || !aligned16(Wr)) return MOE_ERR_INVALID;

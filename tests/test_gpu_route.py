@@ -34,14 +34,26 @@ def _check_route(r, lg_np, k, E, renorm=False):
 @pytest.mark.parametrize("kind", ["normal", "dups", "constant", "signed_zero"])
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (7, 8, 8), (37, 33, 5), (300, 64, 8), (1000, 128, 4),
                                    (257, 384, 8), (64, 512, 32), (50, 1, 1),
-                                   # one case per (lanes per token, logits per lane) shape
-                                   # of the top-k: (1,16) (1,24) (1,32) (2,32) (4,24)
-                                   # (8,24) (8,32) (16,32) besides those above
+                                   # small batches: the lanes per token double up to
+                                   # 16 while each keeps >= 8 logits
                                    (40, 16, 3), (129, 20, 6), (65, 32, 32), (70, 52, 7),
-                                   (100, 80, 8), (70, 160, 8), (90, 256, 16), (33, 500, 9)])
+                                   (100, 80, 8), (70, 160, 8), (90, 256, 16), (33, 500, 9),
+                                   (20, 12, 4), (30, 129, 8)])
 def test_route_from_logits_bitexact(kind, T, E, k):
     moe = _moe()
     lg = adversarial_logits(T, E, kind, seed=T + E)
+    r = moe.moe_route(k, logits=lg.cuda())
+    _check_route(r, lg.numpy(), k, E)
+
+
+@pytest.mark.parametrize("T,E,k", [(160_000, 12, 2), (160_000, 20, 6), (160_000, 30, 8),
+                                   (80_000, 40, 8), (80_000, 60, 8), (40_000, 80, 8),
+                                   (40_000, 120, 4), (20_000, 160, 8), (20_000, 240, 8)])
+def test_route_large_batches(T, E, k):
+    """Batches large enough that the top-k keeps the fewest lanes per token
+    (up to 32 logits per lane; 148 SMs x 1024 threads reached)."""
+    moe = _moe()
+    lg = adversarial_logits(T, E, "dups", seed=T % 1000 + E)
     r = moe.moe_route(k, logits=lg.cuda())
     _check_route(r, lg.numpy(), k, E)
 
