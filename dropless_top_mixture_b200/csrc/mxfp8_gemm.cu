@@ -11,15 +11,22 @@
 //         output in the gate/up epilogue
 //   Ye = Hq W2q (block-scaled), fp32 accumulate, bf16 out; combine as in bf16.
 //
-// Kernel: tcgen05.mma kind::mxf8f6f4.block_scale, M = 128, N = 128, K = 32 per
+// Kernel: tcgen05.mma kind::mxf8f6f4.block_scale, M = 128, N = 256, K = 32 per
 // instruction, 128-byte K slabs staged by TMA with the same 128-byte swizzle
-// as the bf16 kernels, two slabs (8 MMAs) per pipeline stage so the per-stage
-// barrier wait, proxy fence and scale copies are paid once per 256 K. Per slab every row carries 4 UE8M0 scales (one 32-bit
-// word); the producer warp gathers the 128 A words and 128 B words (cp.async,
-// tracked by the stage's mbarrier) into the 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4 copies into TMEM
-// (lane m%32 of every sub-partition, column m/32, byte = K block), and the
-// MMA selects the byte with the scale-factor id of each of the 4 MMAs.
-// Accumulators: two 128-column TMEM buffers; the scale factors follow them.
+// as the bf16 kernels, one slab (4 MMAs) per stage, four stages. The wide N
+// halves the A traffic per flop against N = 128 and lets four 48 KB stages
+// be in flight: the operands of a 256-row expert come from DRAM (each weight
+// tile serves two row tiles), so bytes in flight bound the rate. Per slab
+// every row carries 4 UE8M0 scales (one 32-bit word); the producer warp
+// gathers the 128 A words (cp.async, tracked by the stage's mbarrier) and
+// fetches the B words pre-packed (mxfp8_pack_weight_scales) with one bulk
+// copy, both in the 32-row x 16-byte layout that tcgen05.cp.32x128b.warpx4
+// copies into TMEM (lane m%32 of every sub-partition, column m/32, byte = K
+// block); the MMA selects the byte with the scale-factor id of each of its
+// 4 MMAs. TMEM: one 256-column accumulator (two would leave no room for the
+// scale factors), then the scale factors. Eight epilogue warps first load
+// their 128 accumulator columns into registers and release the accumulator,
+// so the next tile's MMAs overlap the quantisation and stores.
 #include "mx_common.cuh"
 #include "tc_sm100.cuh"
 
@@ -29,23 +36,22 @@ namespace mxg {
 using namespace tc;
 
 constexpr int BM = 128;
-constexpr int MMA_N = 128;
-constexpr int BK = 128;  // e4m3 elements per 128-byte slab
-constexpr int SLABS = 2; // slabs per pipeline stage (8 MMAs per stage wait)
-constexpr int STAGES = 3;
-constexpr int THREADS = 192;
+constexpr int MMA_N = 256;
+constexpr int BK = 128;  // e4m3 elements per 128-byte slab (one slab per stage)
+constexpr int STAGES = 4;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int A_BYTES = BM * 128;
 constexpr int B_BYTES = MMA_N * 128;
-constexpr int SLAB_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGE_BYTES = SLABS * SLAB_BYTES;
-constexpr int SF_BLOCK = 512;         // one operand's scale words for one slab
-// per stage: A blocks of the SLABS slabs, then their B blocks (contiguous, so
-// one bulk copy brings the packed weight scales of the whole stage)
-constexpr int SF_STAGE_BYTES = 2 * SLABS * SF_BLOCK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SF_BLOCK = 512;  // scale words of 128 rows for one slab
+// per stage: the A block, then the two B blocks (contiguous, so one bulk copy
+// brings the packed weight scales of the stage)
+constexpr int SF_STAGE_BYTES = 3 * SF_BLOCK;
 constexpr int TMEM_ALLOC = 512;
-constexpr int SFA_COL = 2 * MMA_N;    // 256 (+8 per slab)
-constexpr int SFB_COL = SFA_COL + 4;  // 260 (+8 per slab)
-constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SFA_COL = MMA_N;        // 256..259
+constexpr int SFB_COL = SFA_COL + 4;  // 260..267
+constexpr int NUM_BARS = 2 * STAGES + 3;
 constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
 constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + META_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -116,9 +122,10 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// SWIGLU: B tile = 64 rows of W1 then 64 rows of W3 at the same n0; the
-// epilogue writes Hq/Hs (64 output columns per tile). Otherwise B = 128 rows
-// of W2 and the epilogue writes bf16 Ye (128 columns).
+// SWIGLU: B tile = 128 rows of W1 then 128 rows of W3 at the same n0; the
+// epilogue writes Hq/Hs (128 output columns per tile). Otherwise B = 256 rows
+// of W2 (rows past N read as zeros) and the epilogue writes bf16 Ye (256
+// columns, those past N skipped).
 template <bool SWIGLU>
 __global__ void __launch_bounds__(THREADS, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -170,27 +177,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
         return;
     }
-    const int NB = N / OUT_N;
+    const int NB = (N + OUT_N - 1) / OUT_N;
     const int total = s_toff[E] * NB;
     if ((int)blockIdx.x >= total) return;
-    const int KS = K / BK;                   // 128-byte slabs
-    const int KB = (KS + SLABS - 1) / SLABS;  // pipeline stages per tile
-    const int sf_row = K / 32;               // scale bytes per row
+    const int KS = K / BK;      // 128-byte slabs = pipeline stages per tile
+    const int sf_row = K / 32;  // scale bytes per row
 
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
     uint64_t* tfull = bars + 2 * STAGES;
-    uint64_t* tempty = bars + 2 * STAGES + 2;
-    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint64_t* tempty = bars + 2 * STAGES + 1;
+    uint64_t* drain = bars + 2 * STAGES + 2;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(full + s), 1 + 32);  // TMA bytes + each lane's scale words
             mbar_init(smem_u32(empty + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(tfull + b), 1);
-            mbar_init(smem_u32(tempty + b), 4);
-        }
+        mbar_init(smem_u32(tfull), 1);
+        mbar_init(smem_u32(tempty), EPI_WARPS);
         mbar_init(smem_u32(drain), 1);
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -215,46 +219,39 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < KS; ++kb) {
                 if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
                     ok = false;
                     break;
                 }
                 const uint32_t fb = smem_u32(full + stage);
-                const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 if (lane == 0) {
-                    mbar_expect_tx(fb, (uint32_t)(ns * (SLAB_BYTES + SF_BLOCK)));
-                    // packed B scales of this stage's slabs: one bulk copy
-                    const size_t blk = ((size_t)tl.e * NB + tl.n0 / OUT_N) * KS + kb * SLABS;
-                    bulk_load(sfs + SLABS * SF_BLOCK, sfBp + blk * SF_BLOCK,
-                              (uint32_t)(ns * SF_BLOCK), fb);
-                    for (int sl = 0; sl < ns; ++sl) {
-                        const int kc = (kb * SLABS + sl) * BK;
-                        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
-                        const uint32_t sb = sa + A_BYTES;
-                        tma_load_2d(sa, &tmA, fb, kc, tl.row0);
-                        if (SWIGLU) {
-                            tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
-                            tma_load_3d(sb + B_BYTES / 2, &tmB1, fb, kc, tl.n0, tl.e);
-                        } else {
-                            tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
-                        }
+                    mbar_expect_tx(fb, (uint32_t)(STAGE_BYTES + 2 * SF_BLOCK));
+                    // packed B scales of this slab (two 128-row blocks): one bulk copy
+                    const size_t blk = ((size_t)tl.e * NB + tl.n0 / OUT_N) * KS + kb;
+                    bulk_load(sfs + SF_BLOCK, sfBp + blk * (2 * SF_BLOCK), 2u * SF_BLOCK, fb);
+                    const int kc = kb * BK;
+                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    tma_load_2d(sa, &tmA, fb, kc, tl.row0);
+                    if (SWIGLU) {
+                        tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
+                        tma_load_3d(sb + B_BYTES / 2, &tmB1, fb, kc, tl.n0, tl.e);
+                    } else {
+                        tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
                     }
                 }
                 // activation scale words (tile rows start anywhere, so they
                 // are gathered row by row), copied asynchronously: the stage's
                 // barrier completes only once they have landed
-                for (int sl = 0; sl < ns; ++sl) {
-                    const int kw = 4 * (kb * SLABS + sl);  // scale byte of the slab's first block
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int m = lane + 32 * j;  // A row within the tile
-                        const int grow = tl.row0 + m;
-                        const bool in = grow < R;
-                        cp_async_word(sfs + (uint32_t)(sl * SF_BLOCK + (lane * 4 + j) * 4),
-                                      sfA + (size_t)(in ? grow : 0) * sf_row + kw, in ? 4u : 0u);
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    const int m = lane + 32 * j;  // A row within the tile
+                    const int grow = tl.row0 + m;
+                    const bool in = grow < R;
+                    cp_async_word(sfs + (uint32_t)((lane * 4 + j) * 4),
+                                  sfA + (size_t)(in ? grow : 0) * sf_row + 4 * kb, in ? 4u : 0u);
                 }
                 cp_async_arrive(fb);
                 issued_mask |= 1u << stage;
@@ -283,44 +280,39 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t sfa_t = tmem_base + SFA_COL;
         const uint32_t sfb_t = tmem_base + SFB_COL;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
-            const int buf = i & 1;
-            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+            // the epilogue has moved the previous tile's accumulator out
+            if (!mbar_wait(smem_u32(tempty), ((uint32_t)i & 1u) ^ 1u, s_abort, status,
+                           WAIT_LIMIT_NS)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < KS; ++kb) {
                 if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 fence_proxy_async_smem();  // scale words came through the generic proxy
-                const int ns = (KS - kb * SLABS < SLABS) ? KS - kb * SLABS : SLABS;
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
-                for (int sl = 0; sl < ns; ++sl) {
-                    tmem_cp_sf(sfa_t + 8u * sl, sf_desc(sfs + sl * SF_BLOCK));
-                    tmem_cp_sf(sfb_t + 8u * sl, sf_desc(sfs + (SLABS + sl) * SF_BLOCK));
-                }
-                for (int sl = 0; sl < ns; ++sl) {
-                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + sl * SLAB_BYTES);
-                    const uint64_t ad = sw128_desc(sa);
-                    const uint64_t bd = sw128_desc(sa + A_BYTES);
+                tmem_cp_sf(sfa_t, sf_desc(sfs));
+                tmem_cp_sf(sfb_t, sf_desc(sfs + SF_BLOCK));
+                tmem_cp_sf(sfb_t + 4u, sf_desc(sfs + 2 * SF_BLOCK));
+                const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+                const uint64_t ad = sw128_desc(sa);
+                const uint64_t bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_mx(dt, ad + 2 * ks, bd + 2 * ks, mx_idesc(ks),
-                               (sfa_t + 8u * sl) | ((uint32_t)ks << 30),
-                               (sfb_t + 8u * sl) | ((uint32_t)ks << 30), (kb | sl | ks) != 0);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_mx(tmem_base, ad + 2 * ks, bd + 2 * ks, mx_idesc(ks),
+                           sfa_t | ((uint32_t)ks << 30), sfb_t | ((uint32_t)ks << 30),
+                           (kb | ks) != 0);
                 tc_commit(smem_u32(empty + stage));
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
-            if (ok) tc_commit(smem_u32(tfull + buf));
+            if (ok) tc_commit(smem_u32(tfull));
         }
         if (!ok) {
             tc_commit(smem_u32(drain));
@@ -328,58 +320,70 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
         }
     } else if (warp >= 2) {
-        // ------------------------------------------------ epilogue
+        // ------------------------------------------------ epilogue: warp w
+        // reads TMEM lanes 32 (w % 4)..+31 (its rows) and column half h
         const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
         const int r_in_tile = q * 32 + lane;
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
-            const int buf = i & 1;
-            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            if (!mbar_wait(smem_u32(tfull), (uint32_t)i & 1u, s_abort, status, WAIT_LIMIT_NS))
+                break;
             tc_fence_after();
-            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
-            const int grow = tl.row0 + r_in_tile;
-            const bool valid = grow < tl.row_end;
-            const size_t grow_c = (size_t)(valid ? grow : 0);
-#pragma unroll 1
-            for (int c = 0; c < OUT_N / 32; ++c) {
-                uint32_t a[32];
-                float v[32];
-                tmem_ld32(ta + c * 32, a);
-                if constexpr (SWIGLU) {
-                    uint32_t b[32];
-                    tmem_ld32(ta + OUT_N + c * 32, b);
-                    tmem_wait_ld();
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);
+            uint32_t acc[128];
+            if constexpr (SWIGLU) {
+                // W1 columns 64h..64h+63 and the W3 columns 128 further on
+                tmem_ld32(ta + 64 * h, acc);
+                tmem_ld32(ta + 64 * h + 32, acc + 32);
+                tmem_ld32(ta + MMA_N / 2 + 64 * h, acc + 64);
+                tmem_ld32(ta + MMA_N / 2 + 64 * h + 32, acc + 96);
+            } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float g = __uint_as_float(a[j]);
-                        v[j] = g / (1.0f + __expf(-g)) * __uint_as_float(b[j]);
-                    }
-                    if (valid) {
+                for (int c = 0; c < 4; ++c) tmem_ld32(ta + 128 * h + 32 * c, acc + 32 * c);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(tempty));
+            const int grow = tl.row0 + r_in_tile;
+            if (grow < tl.row_end) {
+                const size_t gr = (size_t)grow;
+                if constexpr (SWIGLU) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float g = __uint_as_float(acc[32 * c + j]);
+                            v[j] = g / (1.0f + __expf(-g)) * __uint_as_float(acc[64 + 32 * c + j]);
+                        }
                         float sc;
                         const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
                         uint32_t w[8];
                         mxc::encode32(v, sc, w);
-                        uint4* dq = reinterpret_cast<uint4*>(out_q + grow_c * ldo + tl.n0 + c * 32);
+                        const int col = tl.n0 + 64 * h + 32 * c;
+                        uint4* dq = reinterpret_cast<uint4*>(out_q + gr * ldo + col);
                         dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
                         dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                        out_s[grow_c * (ldo / 32) + (tl.n0 + c * 32) / 32] = sbyte;
+                        out_s[gr * (ldo / 32) + col / 32] = sbyte;
                     }
                 } else {
-                    tmem_wait_ld();
-                    if (valid) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
-                        uint4* d = reinterpret_cast<uint4*>(out_bf16 + grow_c * ldo + tl.n0 + c * 32);
+                    for (int c = 0; c < 4; ++c) {
+                        const int col = tl.n0 + 128 * h + 32 * c;
+                        if (col < N) {
+                            float v[32];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) d[u] = pack8(v + 8 * u);
+                            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[32 * c + j]);
+                            uint4* d = reinterpret_cast<uint4*>(out_bf16 + gr * ldo + col);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) d[u] = pack8(v + 8 * u);
+                        }
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
         }
     }
 
@@ -430,37 +434,44 @@ __global__ void __launch_bounds__(256) mx_dispatch_kernel(const __nv_bfloat16* _
 }
 
 // Weight scales packed for the tensor-core scale copy. For every expert,
-// 128-row B tile of the kernel (gate/up: rows n0..n0+63 of W1 then of W3,
-// n0 = 64 nb; down: rows n0..n0+127 of W2, n0 = 128 nb) and 128-element K
-// slab s, one 512-byte block holds the four scale bytes of each of the 128
-// rows in the 32-row x 16-byte order tcgen05.cp.32x128b.warpx4 copies:
-// row m's word at 16 (m % 32) + 4 (m / 32). Blocks are ordered (expert,
-// n-block, slab), so one stage's slabs are adjacent. One thread per word.
+// 256-row B tile of the kernel (gate/up: rows n0..n0+127 of W1 then of W3,
+// n0 = 128 nb; down: rows n0..n0+255 of W2, n0 = 256 nb, rows past the
+// matrix zero) and 128-element K slab s, two 512-byte blocks (tile rows
+// 0..127, then 128..255) each hold the four scale bytes of their 128 rows in
+// the 32-row x 16-byte order tcgen05.cp.32x128b.warpx4 copies: row m's word
+// at 16 (m % 32) + 4 (m / 32). Blocks are ordered (expert, n-block, slab,
+// half), so one stage's blocks are adjacent. One thread per word.
 __global__ void __launch_bounds__(256)
     pack_scales_kernel(const uint8_t* __restrict__ Sa, const uint8_t* __restrict__ Sb,
-                       int64_t rows_per_expert, int64_t half_rows, int64_t sf_row, int nb_count,
-                       int ks_count, int64_t n_words, uint32_t* __restrict__ packed) {
+                       int64_t rows_per_expert, int64_t sf_row, int nb_count, int ks_count,
+                       int64_t n_words, uint32_t* __restrict__ packed) {
     for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_words;
          w += (int64_t)gridDim.x * blockDim.x) {
         const int64_t blk = w >> 7;          // 128 words per 512-byte block
         const int pos = (int)(w & 127);      // word position in the block
-        const int m = (pos >> 2) + 32 * (pos & 3);  // tile row this word holds
-        const int slab = (int)(blk % ks_count);
-        const int64_t eb = blk / ks_count;
+        const int m = (pos >> 2) + 32 * (pos & 3);  // row within the block
+        const int half = (int)(blk & 1);
+        const int64_t bs = blk >> 1;
+        const int slab = (int)(bs % ks_count);
+        const int64_t eb = bs / ks_count;
         const int nb = (int)(eb % nb_count);
         const int64_t e = eb / nb_count;
         const uint8_t* src;
         int64_t row;
-        if (Sb != nullptr) {  // gate/up: 64 rows of W1, then 64 of W3
-            src = m < half_rows ? Sa : Sb;
-            row = (int64_t)nb * half_rows + (m < half_rows ? m : m - half_rows);
+        if (Sb != nullptr) {  // gate/up: the W1 block, then the W3 block
+            src = half ? Sb : Sa;
+            row = (int64_t)nb * 128 + m;
         } else {
             src = Sa;
-            row = (int64_t)nb * 128 + m;
+            row = (int64_t)nb * 256 + half * 128 + m;
         }
-        const uint8_t* p = src + (e * rows_per_expert + row) * sf_row + 4 * slab;
-        packed[w] = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
-                    ((uint32_t)p[3] << 24);
+        uint32_t word = 0;
+        if (row < rows_per_expert) {
+            const uint8_t* p = src + (e * rows_per_expert + row) * sf_row + 4 * slab;
+            word = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
+                   ((uint32_t)p[3] << 24);
+        }
+        packed[w] = word;
     }
 }
 
@@ -479,7 +490,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
         attr_done[dev] = true;
     }
     const int out_n = SWIGLU ? MMA_N / 2 : MMA_N;
-    const int64_t max_tiles = (R / BM + E) * (N / out_n);
+    const int64_t max_tiles = (R / BM + E) * ((N + out_n - 1) / out_n);
     const int64_t sms = num_sms();
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
@@ -534,21 +545,21 @@ extern "C" int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s,
     if ((Ps13 && !aligned16(Ps13)) || (Ps2 && !aligned16(Ps2))) return MOE_ERR_INVALID;
     cudaStream_t st = as_stream(stream);
     const int64_t cap = (int64_t)num_sms() * 8;
-    if (Ps13) {  // gate/up tiles: 64 rows of W1 + 64 of W3 per n-block, K = d
-        const int nb = (int)(F / 64), ks = (int)(d / 128);
-        const int64_t words = E * nb * ks * 128;
+    if (Ps13) {  // gate/up tiles: 128 rows of W1 + 128 of W3 per n-block, K = d
+        const int nb = (int)(F / 128), ks = (int)(d / 128);
+        const int64_t words = E * nb * ks * 2 * 128;
         int64_t g = (words + 255) / 256;
         if (g > cap) g = cap;
-        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W1s, W3s, F, 64, d / 32, nb, ks, words,
+        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W1s, W3s, F, d / 32, nb, ks, words,
                                                        reinterpret_cast<uint32_t*>(Ps13));
     }
-    if (Ps2) {   // down tiles: 128 rows of W2 per n-block, K = F
-        const int nb = (int)(d / 128), ks = (int)(F / 128);
-        const int64_t words = E * nb * ks * 128;
+    if (Ps2) {   // down tiles: 256 rows of W2 per n-block, K = F
+        const int nb = (int)((d + 255) / 256), ks = (int)(F / 128);
+        const int64_t words = E * nb * ks * 2 * 128;
         int64_t g = (words + 255) / 256;
         if (g > cap) g = cap;
-        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W2s, nullptr, d, 128, F / 32, nb, ks,
-                                                       words, reinterpret_cast<uint32_t*>(Ps2));
+        mxg::pack_scales_kernel<<<(int)g, 256, 0, st>>>(W2s, nullptr, d, F / 32, nb, ks, words,
+                                                       reinterpret_cast<uint32_t*>(Ps2));
     }
     return launch_status();
 }
@@ -565,8 +576,8 @@ extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, c
     if (R == 0) return MOE_OK;
     CUtensorMap a, b0, b1;
     if (!make_map_2d(&a, Xq, mxg::U8, 1, d, R, mxg::BM) ||
-        !make_map_3d(&b0, W1q, mxg::U8, 1, d, F, E, w13_expert_stride, 64) ||
-        !make_map_3d(&b1, W3q, mxg::U8, 1, d, F, E, w13_expert_stride, 64))
+        !make_map_3d(&b0, W1q, mxg::U8, 1, d, F, E, w13_expert_stride, mxg::MMA_N / 2) ||
+        !make_map_3d(&b1, W3q, mxg::U8, 1, d, F, E, w13_expert_stride, mxg::MMA_N / 2))
         return MOE_ERR_CUDA;
     return mxg::launch<true>(a, b0, b1, Xs, Ps13, offsets, E, R, d, F, Hq, Hs, nullptr, F,
                              as_stream(stream));

@@ -709,8 +709,8 @@ class MxWeights:
 def mxfp8_pack_weight_scales(w: MxWeights) -> MxWeights:
     E, F, d = w.W1q.shape
     dev = w.W1q.device
-    w.Ps13 = torch.empty(E * (F // 64) * (d // 128) * 512, dtype=torch.uint8, device=dev)
-    w.Ps2 = torch.empty(E * (d // 128) * (F // 128) * 512, dtype=torch.uint8, device=dev)
+    w.Ps13 = torch.empty(E * (F // 128) * (d // 128) * 1024, dtype=torch.uint8, device=dev)
+    w.Ps2 = torch.empty(E * ((d + 255) // 256) * (F // 128) * 1024, dtype=torch.uint8, device=dev)
     for t in (w.W1s, w.W3s, w.W2s):
         _need(t, "weight scales")
     rc = lib.mxfp8_pack_weight_scales(_ptr(w.W1s), _ptr(w.W3s), _ptr(w.W2s), E, d, F,

@@ -307,13 +307,14 @@ MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mod
  *
  * mxfp8_pack_weight_scales: the weight scales in the order the GEMMs'
  *   tensor-core scale copy reads them, so each pipeline stage fetches them
- *   with one bulk copy. For every expert, every 128-row B tile (gate/up:
- *   rows 64nb..64nb+63 of W1 then the same rows of W3; down: rows
- *   128nb..128nb+127 of W2) and every 128-element K slab s, a 512-byte
- *   block holds the four scale bytes (K blocks 4s..4s+3) of tile row m at
- *   byte 16*(m % 32) + 4*(m / 32); blocks ordered (expert, n-block, slab).
- *   Ps13: E*(F/64)*(d/128)*512 bytes (from W1s, W3s); Ps2:
- *   E*(d/128)*(F/128)*512 bytes (from W2s). Either pair may be NULL.
+ *   with one bulk copy. For every expert, every 256-row B tile (gate/up:
+ *   rows 128nb..128nb+127 of W1 then the same rows of W3; down: rows
+ *   256nb..256nb+255 of W2, rows past d zero) and every 128-element K slab
+ *   s, two 512-byte blocks (tile rows 0..127, then 128..255) each hold the
+ *   four scale bytes (K blocks 4s..4s+3) of their row m at byte
+ *   16*(m % 32) + 4*(m / 32); blocks ordered (expert, n-block, slab, half).
+ *   Ps13: E*(F/128)*(d/128)*1024 bytes (from W1s, W3s); Ps2:
+ *   E*ceil(d/256)*(F/128)*1024 bytes (from W2s). Either pair may be NULL.
  *   Scale tensors contiguous as above; packed outputs 16-byte aligned.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T, int64_t d, int k,

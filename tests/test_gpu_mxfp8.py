@@ -56,7 +56,7 @@ def test_dispatch_mxfp8_bitexact():
 
 
 @pytest.mark.parametrize("T,d,F,E,k", [(300, 256, 256, 5, 2), (700, 512, 384, 16, 4),
-                                       (37, 128, 128, 4, 2)])
+                                       (37, 128, 128, 4, 2), (200, 384, 256, 6, 3)])
 def test_grouped_mxfp8_gemms(T, d, F, E, k):
     moe = _moe()
     x, W1, W3, W2, lg = _problem(T, d, F, E, k, seed=T + d + F)
@@ -139,11 +139,12 @@ def test_layer_mxfp8_full_size_sampled():
     assert gap < 0.1
 
 
-@pytest.mark.parametrize("E,d,F", [(3, 256, 128), (2, 128, 384)])
+@pytest.mark.parametrize("E,d,F", [(3, 256, 128), (2, 128, 384), (2, 384, 256)])
 def test_pack_weight_scales_layout(E, d, F):
     """The packed weight scales are a permutation of the row-layout scale
-    bytes, as the header defines it: block (e, nb, s) of 512 bytes, tile row
-    m's four K-block bytes at 16*(m % 32) + 4*(m / 32)."""
+    bytes, as the header defines it: for block (e, nb, s, half) of 512 bytes,
+    the row m of that half's 128 tile rows has its four K-block bytes at
+    16*(m % 32) + 4*(m / 32); rows past the matrix are zero."""
     moe = _moe()
     g = torch.Generator().manual_seed(E + d + F)
     s1 = torch.randint(0, 256, (E, F, d // 32), generator=g, dtype=torch.uint8)
@@ -155,25 +156,28 @@ def test_pack_weight_scales_layout(E, d, F):
     got13 = w.Ps13.cpu().numpy()
     got2 = w.Ps2.cpu().numpy()
 
-    def block(rows_bytes):            # rows_bytes: [128 rows, 4 bytes]
+    def block(rows_bytes):            # rows_bytes: [<= 128 rows, 4 bytes]
         b = np.zeros(512, dtype=np.uint8)
-        for m in range(128):
+        for m in range(rows_bytes.shape[0]):
             o = 16 * (m % 32) + 4 * (m // 32)
             b[o:o + 4] = rows_bytes[m]
         return b
 
     want13 = []
     for e in range(E):
-        for nb in range(F // 64):
-            rows = np.concatenate([s1[e, 64 * nb:64 * nb + 64].numpy(),
-                                   s3[e, 64 * nb:64 * nb + 64].numpy()])
+        for nb in range(F // 128):
+            halves = [s1[e, 128 * nb:128 * nb + 128].numpy(),
+                      s3[e, 128 * nb:128 * nb + 128].numpy()]
             for s in range(d // 128):
-                want13.append(block(rows[:, 4 * s:4 * s + 4]))
+                for rows in halves:
+                    want13.append(block(rows[:, 4 * s:4 * s + 4]))
     want2 = []
     for e in range(E):
-        for nb in range(d // 128):
-            rows = s2[e, 128 * nb:128 * nb + 128].numpy()
+        for nb in range((d + 255) // 256):
+            halves = [s2[e, 256 * nb:256 * nb + 128].numpy(),
+                      s2[e, 256 * nb + 128:256 * nb + 256].numpy()]
             for s in range(F // 128):
-                want2.append(block(rows[:, 4 * s:4 * s + 4]))
+                for rows in halves:
+                    want2.append(block(rows[:, 4 * s:4 * s + 4]))
     assert np.array_equal(got13, np.concatenate(want13))
     assert np.array_equal(got2, np.concatenate(want2))
