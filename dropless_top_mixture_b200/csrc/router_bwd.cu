@@ -241,29 +241,40 @@ __global__ void __launch_bounds__(THREADS)
     }
 }
 
-// aux = E * sum_e (counts[e]/T) * (P_sum[e]/T). Warp w takes experts w,
-// w + WARPS, ...: lane l adds the partials of blocks l, l + 32, ... in order,
-// a fixed butterfly adds the lanes, and the expert terms are added in a
-// fixed tree, so the result is deterministic.
-__global__ void __launch_bounds__(THREADS)
+// aux = E * sum_e (counts[e]/T) * (P_sum[e]/T). Thread e adds the partials
+// of expert e over the blocks in block order (loads issued 16 at a time,
+// coalesced across experts), then the expert terms are added in a fixed
+// shared-memory tree, so the result is deterministic.
+constexpr int AUX_FINAL_THREADS = MOE_MAX_EXPERTS;
+
+__global__ void __launch_bounds__(AUX_FINAL_THREADS)
     aux_final_kernel(const float* __restrict__ partial, int nblocks,
                      const int32_t* __restrict__ counts, int T, int E, float* __restrict__ aux) {
-    __shared__ float s_term[WARPS];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ float s_red[AUX_FINAL_THREADS];
+    const int e = threadIdx.x;
     float term = 0.f;
-    for (int e = warp; e < E; e += WARPS) {
+    if (e < E) {
         float P = 0.f;
-        for (int b = lane; b < nblocks; b += 32) P += partial[(size_t)b * E + e];
-        P = warp_sum(P);
-        term += (float)counts[e] * P;
+        int b = 0;
+        for (; b + 16 <= nblocks; b += 16) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = partial[(size_t)(b + i) * E + e];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) P += v[i];
+        }
+        for (; b < nblocks; ++b) P += partial[(size_t)b * E + e];
+        term = (float)counts[e] * P;
     }
-    if (lane == 0) s_term[warp] = term;
+    s_red[e] = term;
     __syncthreads();
-    if (tid == 0) {
-        float sum = 0.f;
-        for (int w = 0; w < WARPS; ++w) sum += s_term[w];
+    for (int w = AUX_FINAL_THREADS / 2; w > 0; w >>= 1) {
+        if (e < w) s_red[e] += s_red[e + w];
+        __syncthreads();
+    }
+    if (e == 0) {
         const float invT = 1.0f / (float)T;
-        aux[0] = (float)E * sum * invT * invT;
+        aux[0] = (float)E * s_red[0] * invT * invT;
     }
 }
 
@@ -457,7 +468,8 @@ extern "C" int moe_aux_loss(const float* logits, const int32_t* counts, int64_t 
     cudaStream_t st = as_stream(stream);
     float* part = static_cast<float*>(workspace);
     rb::aux_partial_kernel<<<used, rb::THREADS, 0, st>>>(logits, (int)T, (int)E, per, part);
-    rb::aux_final_kernel<<<1, rb::THREADS, 0, st>>>(part, used, counts, (int)T, (int)E, aux_out);
+    rb::aux_final_kernel<<<1, rb::AUX_FINAL_THREADS, 0, st>>>(part, used, counts, (int)T, (int)E,
+                                                               aux_out);
     return launch_status();
 }
 
