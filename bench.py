@@ -292,11 +292,22 @@ def _steps(moe, w, inp, dev, backward):
         Xq = torch.empty((R, d), dtype=torch.uint8, device=dev)
         Xs = torch.empty((R, d // 32), dtype=torch.uint8, device=dev)
         Hq = torch.empty((R, F), dtype=torch.uint8, device=dev)
-        Hs = torch.empty((R, F // 32), dtype=torch.uint8, device=dev)
+        # activation scales in the tile-packed layout the GEMMs copy
+        Xsp = torch.empty(moe.lib.mxfp8_act_scales_packed_size(E, R, d), dtype=torch.uint8,
+                          device=dev)
+        Hsp = torch.empty(moe.lib.mxfp8_act_scales_packed_size(E, R, F), dtype=torch.uint8,
+                          device=dev)
+
+        def mx_dispatch():
+            moe.moe_dispatch_mxfp8(x, rt.slot, Xq, Xs)
+            moe.mxfp8_pack_act_scales(Xs, rt.offsets, E, Xsp)
+
         fns = [("route", route),
-               ("dispatch", lambda: moe.moe_dispatch_mxfp8(x, rt.slot, Xq, Xs)),
-               ("gate_up", lambda: moe.moe_grouped_gate_up_mxfp8(Xq, Xs, mw, rt.offsets, Hq, Hs)),
-               ("down", lambda: moe.moe_grouped_down_mxfp8(Hq, Hs, mw, rt.offsets, Ye)),
+               ("dispatch", mx_dispatch),
+               ("gate_up", lambda: moe.moe_grouped_gate_up_mxfp8(Xq, Xsp, mw, rt.offsets, Hq, Hsp,
+                                                                 packed=True)),
+               ("down", lambda: moe.moe_grouped_down_mxfp8(Hq, Hsp, mw, rt.offsets, Ye,
+                                                           packed=True)),
                ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
         sx, sw, sh = 1 + 1 / 32, 1 + 1 / 32, 1 + 1 / 32
     else:
@@ -380,7 +391,7 @@ def _steps(moe, w, inp, dev, backward):
         # dx += dlogits Wr and dWr = dlogits^T x: two T x E x d products
         work["router_linear_bwd"] = (4.0 * T * E * d, T * E * 4 + E * d * es + 3 * T * d * es
                                      + E * d * es)
-    kernels = ((4 if use_router else 3) + 4
+    kernels = ((4 if use_router else 3) + (5 if w.mxfp8 else 4)
                + ((7 + 2 + 1 + (3 if use_router else 0)) if backward else 0))
     return [n for n, _ in fns], step, kernels, work, e_act
 

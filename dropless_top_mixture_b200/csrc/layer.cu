@@ -321,9 +321,10 @@ namespace layer {
 
 struct CarveMx {
     uint8_t* Xq;
-    uint8_t* Xs;
+    uint8_t* Xs;   // row layout, as the dispatch writes it
+    uint8_t* Xsp;  // tile-packed, as the gate/up GEMM reads it
     uint8_t* Hq;
-    uint8_t* Hs;
+    uint8_t* Hsp;  // tile-packed H scales (gate/up writes, down reads)
     void* Ye;
     void* route_ws;
     size_t route_bytes;
@@ -340,10 +341,12 @@ inline CarveMx carve_mx(void* base, int64_t T, int64_t d, int64_t E, int64_t F, 
     off += a256(R * d);
     c.Xs = reinterpret_cast<uint8_t*>(p + off);
     off += a256(R * d / 32);
+    c.Xsp = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(mxfp8_act_scales_packed_size(E, (int64_t)R, d));
     c.Hq = reinterpret_cast<uint8_t*>(p + off);
     off += a256(R * F);
-    c.Hs = reinterpret_cast<uint8_t*>(p + off);
-    off += a256(R * F / 32);
+    c.Hsp = reinterpret_cast<uint8_t*>(p + off);
+    off += a256(mxfp8_act_scales_packed_size(E, (int64_t)R, F));
     c.Ye = p + off;
     off += a256(R * d * 2);
     c.route_ws = p + off;
@@ -377,10 +380,12 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     const int64_t R = a->T * a->k;
     rc = moe_dispatch_mxfp8(a->x, a->slot, a->T, a->d, a->k, c.Xq, c.Xs, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xs, a->W1q, a->W3q, a->Ps13, a->w13_expert_stride,
-                                   a->offsets, a->E, R, a->d, a->F, c.Hq, c.Hs, stream);
+    rc = mxfp8_pack_act_scales(c.Xs, a->offsets, a->E, R, a->d, c.Xsp, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_down_mxfp8(c.Hq, c.Hs, a->W2q, a->Ps2, a->w2_expert_stride, a->offsets, a->E,
+    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xsp, a->W1q, a->W3q, a->Ps13, a->w13_expert_stride,
+                                   a->offsets, a->E, R, a->d, a->F, c.Hq, c.Hsp, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_grouped_down_mxfp8(c.Hq, c.Hsp, a->W2q, a->Ps2, a->w2_expert_stride, a->offsets, a->E,
                                 R, a->d, a->F, c.Ye, stream);
     if (rc != MOE_OK) return rc;
     return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, MOE_BF16, a->out, stream);

@@ -88,6 +88,7 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
 
 struct Tile {
     int e, row0, row_end, n0;
+    int tile;  // global row-tile index: s_toff[e] + row tile within the expert
 };
 
 __device__ __forceinline__ Tile decode_tile(int t, int NB, int E, int out_n, const int* s_toff,
@@ -107,50 +108,20 @@ __device__ __forceinline__ Tile decode_tile(int t, int NB, int E, int out_n, con
     tl.row0 = s_off[lo] + m * BM;
     tl.row_end = s_off[lo + 1];
     tl.n0 = nb * out_n;
+    tl.tile = s_toff[lo] + m;
     return tl;
 }
 
-// 4-byte asynchronous global->shared copy; src_bytes = 0 fills zeros.
-__device__ __forceinline__ void cp_async_word(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-// The mbarrier counts one arrival once all of this thread's earlier cp.async
-// copies have landed.
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// SWIGLU: B tile = 128 rows of W1 then 128 rows of W3 at the same n0; the
-// epilogue writes Hq/Hs (128 output columns per tile). Otherwise B = 256 rows
-// of W2 (rows past N read as zeros) and the epilogue writes bf16 Ye (256
-// columns, those past N skipped).
-template <bool SWIGLU>
-__global__ void __launch_bounds__(THREADS, 1)
-    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                   const __grid_constant__ CUtensorMap tmB0,
-                   const __grid_constant__ CUtensorMap tmB1, const uint8_t* __restrict__ sfA,
-                   const uint8_t* __restrict__ sfBp, const int32_t* __restrict__ offsets, int E, int R,
-                   int K, int N, uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_s,
-                   __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status) {
-    constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sf_smem = smem + STAGES * STAGE_BYTES;
-    uint8_t* meta = sf_smem + STAGES * SF_STAGE_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
-    int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
-    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+// Tile table of an offsets vector in shared memory: s_toff[e] = sum over
+// e' < e of ceil(count/128), s_toff[E] = row tiles in all. Returns false
+// (and sets MOE_DEVERR_BAD_OFFSETS once) when offsets are not monotone from
+// 0 to R. Whole block; E <= MOE_MAX_EXPERTS.
+__device__ bool block_tile_table(const int32_t* __restrict__ offsets, int E, int R, int* s_off,
+                                 int* s_toff, int* s_bad, int* status) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int e = tid; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
-    if (warp == 0) {
+    if (tid < 32) {
         int carry = 0;
         bool bad = false;
         for (int base = 0; base < E; base += 32) {
@@ -173,15 +144,52 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     __syncthreads();
-    if (*s_bad) {
-        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
-        return;
+    if (*s_bad && tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+    return !*s_bad;
+}
+
+// Expert whose tile range holds row tile g (s_toff ascending, g < s_toff[E]).
+__device__ __forceinline__ int expert_of_tile(const int* s_toff, int E, int g) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_toff[mid] <= g) lo = mid;
+        else hi = mid - 1;
     }
+    return lo;
+}
+
+// SWIGLU: B tile = 128 rows of W1 then 128 rows of W3 at the same n0; the
+// epilogue writes Hq/Hs (128 output columns per tile). Otherwise B = 256 rows
+// of W2 (rows past N read as zeros) and the epilogue writes bf16 Ye (256
+// columns, those past N skipped).
+template <bool SWIGLU>
+__global__ void __launch_bounds__(THREADS, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                   const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, const uint8_t* __restrict__ sfAp,
+                   const uint8_t* __restrict__ sfBp, const int32_t* __restrict__ offsets, int E, int R,
+                   int K, int N, uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sp,
+                   __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status) {
+    constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sf_smem = smem + STAGES * STAGE_BYTES;
+    uint8_t* meta = sf_smem + STAGES * SF_STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (!block_tile_table(offsets, E, R, s_off, s_toff, s_bad, status)) return;
     const int NB = (N + OUT_N - 1) / OUT_N;
     const int total = s_toff[E] * NB;
     if ((int)blockIdx.x >= total) return;
-    const int KS = K / BK;      // 128-byte slabs = pipeline stages per tile
-    const int sf_row = K / 32;  // scale bytes per row
+    const int KS = K / BK;  // 128-byte slabs = pipeline stages per tile
 
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
@@ -190,7 +198,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* drain = bars + 2 * STAGES + 2;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(full + s), 1 + 32);  // TMA bytes + each lane's scale words
+            mbar_init(smem_u32(full + s), 1);  // the stage's TMA and bulk bytes
             mbar_init(smem_u32(empty + s), 1);
         }
         mbar_init(smem_u32(tfull), 1);
@@ -212,8 +220,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tmem_base = *s_tmem;
 
     if (warp == 0) {
-        // ------------------------------------------------ producer warp:
-        // lane 0 issues the TMA copies, all lanes gather the scale words
+        // ------------------------------------------------ producer (lane 0)
         int stage = 0;
         uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
         bool ok = true;
@@ -227,8 +234,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t fb = smem_u32(full + stage);
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 if (lane == 0) {
-                    mbar_expect_tx(fb, (uint32_t)(STAGE_BYTES + 2 * SF_BLOCK));
-                    // packed B scales of this slab (two 128-row blocks): one bulk copy
+                    mbar_expect_tx(fb, (uint32_t)(STAGE_BYTES + 3 * SF_BLOCK));
+                    // packed scales of this slab: the A tile's block, then the
+                    // B tile's two 128-row blocks
+                    bulk_load(sfs, sfAp + ((size_t)tl.tile * KS + kb) * SF_BLOCK, SF_BLOCK, fb);
                     const size_t blk = ((size_t)tl.e * NB + tl.n0 / OUT_N) * KS + kb;
                     bulk_load(sfs + SF_BLOCK, sfBp + blk * (2 * SF_BLOCK), 2u * SF_BLOCK, fb);
                     const int kc = kb * BK;
@@ -242,18 +251,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_3d(sb, &tmB0, fb, kc, tl.n0, tl.e);
                     }
                 }
-                // activation scale words (tile rows start anywhere, so they
-                // are gathered row by row), copied asynchronously: the stage's
-                // barrier completes only once they have landed
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int m = lane + 32 * j;  // A row within the tile
-                    const int grow = tl.row0 + m;
-                    const bool in = grow < R;
-                    cp_async_word(sfs + (uint32_t)((lane * 4 + j) * 4),
-                                  sfA + (size_t)(in ? grow : 0) * sf_row + 4 * kb, in ? 4u : 0u);
-                }
-                cp_async_arrive(fb);
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) {
@@ -293,7 +290,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                fence_proxy_async_smem();  // scale words came through the generic proxy
                 const uint32_t sfs = smem_u32(sf_smem + stage * SF_STAGE_BYTES);
                 tmem_cp_sf(sfa_t, sf_desc(sfs));
                 tmem_cp_sf(sfb_t, sf_desc(sfs + SF_BLOCK));
@@ -348,39 +344,47 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(tempty));
             const int grow = tl.row0 + r_in_tile;
-            if (grow < tl.row_end) {
-                const size_t gr = (size_t)grow;
-                if constexpr (SWIGLU) {
+            const bool valid = grow < tl.row_end;
+            const size_t gr = (size_t)(valid ? grow : 0);
+            if constexpr (SWIGLU) {
+                // H scales go to the tile-packed layout the down GEMM copies
+                // (tile rows past the expert's rows get 0)
+                const uint32_t sp_word = 16u * (uint32_t)(r_in_tile & 31) + 4u * (uint32_t)(r_in_tile >> 5);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < 2; ++c) {
+                    const int col = tl.n0 + 64 * h + 32 * c;
+                    uint8_t* sp = out_sp + ((size_t)tl.tile * (ldo / BK) + col / BK) * SF_BLOCK +
+                                  sp_word + (col / 32) % 4;
+                    if (!valid) {
+                        *sp = 0;
+                        continue;
+                    }
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float g = __uint_as_float(acc[32 * c + j]);
+                        v[j] = g / (1.0f + __expf(-g)) * __uint_as_float(acc[64 + 32 * c + j]);
+                    }
+                    float sc;
+                    const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
+                    uint32_t w[8];
+                    mxc::encode32(v, sc, w);
+                    uint4* dq = reinterpret_cast<uint4*>(out_q + gr * ldo + col);
+                    dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    *sp = sbyte;
+                }
+            } else if (valid) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int col = tl.n0 + 128 * h + 32 * c;
+                    if (col < N) {
                         float v[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float g = __uint_as_float(acc[32 * c + j]);
-                            v[j] = g / (1.0f + __expf(-g)) * __uint_as_float(acc[64 + 32 * c + j]);
-                        }
-                        float sc;
-                        const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
-                        uint32_t w[8];
-                        mxc::encode32(v, sc, w);
-                        const int col = tl.n0 + 64 * h + 32 * c;
-                        uint4* dq = reinterpret_cast<uint4*>(out_q + gr * ldo + col);
-                        dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                        out_s[gr * (ldo / 32) + col / 32] = sbyte;
-                    }
-                } else {
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[32 * c + j]);
+                        uint4* d = reinterpret_cast<uint4*>(out_bf16 + gr * ldo + col);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int col = tl.n0 + 128 * h + 32 * c;
-                        if (col < N) {
-                            float v[32];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[32 * c + j]);
-                            uint4* d = reinterpret_cast<uint4*>(out_bf16 + gr * ldo + col);
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) d[u] = pack8(v + 8 * u);
-                        }
+                        for (int u = 0; u < 4; ++u) d[u] = pack8(v + 8 * u);
                     }
                 }
             }
@@ -475,6 +479,42 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Activation scales from rows ([R, K/32] bytes) to the tile-packed layout
+// the GEMMs copy: for every row tile g of the expert-sorted rows (experts in
+// order, ceil(count/128) tiles each) and 128-element K slab s, a 512-byte
+// block holds the word (four K-block bytes) of tile row m at 16 (m % 32) +
+// 4 (m / 32); blocks ordered (tile, slab); tile rows past the expert's rows
+// hold 0. One thread per word; unpack is the inverse for the expert rows.
+template <bool UNPACK>
+__global__ void __launch_bounds__(256)
+    act_scales_kernel(const int32_t* __restrict__ offsets, int E, int R, int ks_count,
+                      int64_t n_words, const uint32_t* __restrict__ src,
+                      uint32_t* __restrict__ dst, int* status) {
+    __shared__ int s_off[MOE_MAX_EXPERTS + 1];
+    __shared__ int s_toff[MOE_MAX_EXPERTS + 1];
+    __shared__ int s_bad;
+    if (!block_tile_table(offsets, E, R, s_off, s_toff, &s_bad, status)) return;
+    const int64_t used = (int64_t)s_toff[E] * ks_count * 128;
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_words;
+         w += (int64_t)gridDim.x * blockDim.x) {
+        if (w >= used) break;  // tiles past the table's end are not used
+        const int pos = (int)(w & 127);
+        const int64_t blk = w >> 7;
+        const int slab = (int)(blk % ks_count);
+        const int g = (int)(blk / ks_count);
+        const int m = (pos >> 2) + 32 * (pos & 3);
+        const int e = expert_of_tile(s_toff, E, g);
+        const int row = s_off[e] + (g - s_toff[e]) * BM + m;
+        const bool in = row < s_off[e + 1];
+        const int64_t rw = (int64_t)row * ks_count + slab;  // row-layout word
+        if (UNPACK) {
+            if (in) dst[rw] = src[w];
+        } else {
+            dst[w] = in ? src[rw] : 0u;
+        }
+    }
+}
+
 template <bool SWIGLU>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const uint8_t* sfA, const uint8_t* sfBp, const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, uint8_t* oq,
@@ -528,9 +568,7 @@ static int mx_check(const void* A, const void* As, const void* B, const void* Bp
     if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (R > INT32_MAX - 2 * mxg::BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
     if (!offsets || !A || !As || !B || !Bp) return MOE_ERR_INVALID;
-    if (!aligned16(A) || !aligned16(B) || !aligned16(Bp)) return MOE_ERR_INVALID;
-    // activation scale words are read as aligned 32-bit loads
-    if (reinterpret_cast<uintptr_t>(As) & 3u) return MOE_ERR_INVALID;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(Bp) || !aligned16(As)) return MOE_ERR_INVALID;
     return MOE_OK;
 }
 
@@ -564,6 +602,46 @@ extern "C" int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s,
     return launch_status();
 }
 
+static int act_scales(const uint8_t* src, const int32_t* offsets, int64_t E, int64_t R,
+                      int64_t K, uint8_t* dst, void* stream, bool unpack) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || K <= 0) return MOE_ERR_INVALID;
+    if (K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (R > INT32_MAX - 2 * mxg::BM) return MOE_ERR_UNSUPPORTED;
+    if (R == 0) return MOE_OK;
+    if (!src || !dst || !offsets) return MOE_ERR_INVALID;
+    if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID;
+    const int ks = (int)(K / 128);
+    const int64_t words = (R / mxg::BM + E) * ks * 128;
+    // about one word per thread: each word is a dependent load and store
+    int64_t g = (words + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 32;
+    if (g > cap) g = cap;
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+    uint32_t* d = reinterpret_cast<uint32_t*>(dst);
+    if (unpack)
+        mxg::act_scales_kernel<true><<<(int)g, 256, 0, as_stream(stream)>>>(
+            offsets, (int)E, (int)R, ks, words, s, d, status_ptr());
+    else
+        mxg::act_scales_kernel<false><<<(int)g, 256, 0, as_stream(stream)>>>(
+            offsets, (int)E, (int)R, ks, words, s, d, status_ptr());
+    return launch_status();
+}
+
+extern "C" size_t mxfp8_act_scales_packed_size(int64_t E, int64_t R, int64_t K) {
+    if (E < 1 || R < 0 || K <= 0 || K % 128 != 0) return 0;
+    return (size_t)(R / mxg::BM + E) * (size_t)(K / 128) * mxg::SF_BLOCK;
+}
+
+extern "C" int mxfp8_pack_act_scales(const uint8_t* S, const int32_t* offsets, int64_t E,
+                                     int64_t R, int64_t K, uint8_t* Sp, void* stream) {
+    return act_scales(S, offsets, E, R, K, Sp, stream, false);
+}
+
+extern "C" int mxfp8_unpack_act_scales(const uint8_t* Sp, const int32_t* offsets, int64_t E,
+                                       int64_t R, int64_t K, uint8_t* S, void* stream) {
+    return act_scales(Sp, offsets, E, R, K, S, stream, true);
+}
+
 extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
                                          const uint8_t* W3q, const uint8_t* Ps13,
                                          int64_t w13_expert_stride, const int32_t* offsets,
@@ -571,7 +649,8 @@ extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, c
                                          uint8_t* Hs, void* stream) {
     int rc = mx_check(Xq, Xs, W1q, Ps13, offsets, E, R, d, F);
     if (rc != MOE_OK) return rc;
-    if (!W3q || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq)) return MOE_ERR_INVALID;
+    if (!W3q || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq) || !aligned16(Hs))
+        return MOE_ERR_INVALID;
     if ((w13_expert_stride < F * d && E > 1) || w13_expert_stride % 128 != 0) return MOE_ERR_INVALID;
     if (R == 0) return MOE_OK;
     CUtensorMap a, b0, b1;

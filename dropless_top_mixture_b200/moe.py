@@ -115,6 +115,9 @@ _SIGS = {
     "mxfp8_dequantize": (_i32, [_p, _p, _i32, _i64, _i64, _p, _p]),
     "moe_dispatch_mxfp8": (_i32, [_p, _p, _i64, _i64, _i32, _p, _p, _p]),
     "mxfp8_pack_weight_scales": (_i32, [_p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
+    "mxfp8_act_scales_packed_size": (_sz, [_i64, _i64, _i64]),
+    "mxfp8_pack_act_scales": (_i32, [_p, _p, _i64, _i64, _i64, _p, _p]),
+    "mxfp8_unpack_act_scales": (_i32, [_p, _p, _i64, _i64, _i64, _p, _p]),
     "moe_grouped_gate_up_mxfp8": (_i32, [_p, _p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64,
                                          _p, _p, _p]),
     "moe_grouped_down_mxfp8": (_i32, [_p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _p]),
@@ -749,30 +752,63 @@ def moe_dispatch_mxfp8(x, slot, Xq=None, Xs=None):
     return Xq, Xs
 
 
-def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None):
+def mxfp8_pack_act_scales(S, offsets, E: int, Sp=None):
+    """Row-layout activation scales [R, K/32] -> the tile-packed layout the
+    MXFP8 GEMMs read (blocks of 512 bytes per 128-row tile and K slab)."""
+    _need(S, "S"); _need(offsets, "offsets")
+    R, kb = S.shape
+    if Sp is None:
+        Sp = torch.empty(lib.mxfp8_act_scales_packed_size(E, R, kb * 32), dtype=torch.uint8,
+                         device=S.device)
+    rc = lib.mxfp8_pack_act_scales(_ptr(S), _ptr(offsets), E, R, kb * 32, _ptr(Sp), _stream(S))
+    _check("mxfp8_pack_act_scales", rc)
+    return Sp
+
+
+def mxfp8_unpack_act_scales(Sp, offsets, E: int, R: int, K: int, S=None):
+    """Tile-packed activation scales -> row layout [R, K/32]."""
+    _need(Sp, "Sp"); _need(offsets, "offsets")
+    if S is None:
+        S = torch.empty((R, K // 32), dtype=torch.uint8, device=Sp.device)
+    rc = lib.mxfp8_unpack_act_scales(_ptr(Sp), _ptr(offsets), E, R, K, _ptr(S), _stream(Sp))
+    _check("mxfp8_unpack_act_scales", rc)
+    return S
+
+
+def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None, *,
+                              packed: bool = False):
+    """H = quantised SwiGLU of the block-scaled FP8 gate/up GEMMs. With
+    packed=False, Xs and the returned Hs are in row layout (packed and
+    unpacked here); with packed=True both are in the tile-packed layout."""
     _need(Xq, "Xq"); _need(Xs, "Xs"); _need(offsets, "offsets")
     E, F, d = w.W1q.shape
     R = Xq.shape[0]
+    dev = Xq.device
     if Hq is None:
-        Hq = torch.empty((R, F), dtype=torch.uint8, device=Xq.device)
-    if Hs is None:
-        Hs = torch.empty((R, F // 32), dtype=torch.uint8, device=Xq.device)
+        Hq = torch.empty((R, F), dtype=torch.uint8, device=dev)
+    Xsp = Xs if packed else mxfp8_pack_act_scales(Xs, offsets, E)
+    Hsp = Hs if (packed and Hs is not None) else torch.empty(
+        lib.mxfp8_act_scales_packed_size(E, R, F), dtype=torch.uint8, device=dev)
     w = _packed(w)
-    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xs), _ptr(w.W1q), _ptr(w.W3q), _ptr(w.Ps13),
+    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xsp), _ptr(w.W1q), _ptr(w.W3q), _ptr(w.Ps13),
                                        w.W1q.stride(0), _ptr(offsets), E, R, d, F, _ptr(Hq),
-                                       _ptr(Hs), _stream(Xq))
+                                       _ptr(Hsp), _stream(Xq))
     _check("moe_grouped_gate_up_mxfp8", rc)
-    return Hq, Hs
+    if packed:
+        return Hq, Hsp
+    return Hq, mxfp8_unpack_act_scales(Hsp, offsets, E, R, F, Hs)
 
 
-def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None):
+def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None, *, packed: bool = False):
+    """Ye = the block-scaled FP8 down GEMM; Hs in row layout unless packed."""
     _need(Hq, "Hq"); _need(Hs, "Hs"); _need(offsets, "offsets")
     E, d, F = w.W2q.shape
     R = Hq.shape[0]
     if Ye is None:
         Ye = torch.empty((R, d), dtype=torch.bfloat16, device=Hq.device)
+    Hsp = Hs if packed else mxfp8_pack_act_scales(Hs, offsets, E)
     w = _packed(w)
-    rc = lib.moe_grouped_down_mxfp8(_ptr(Hq), _ptr(Hs), _ptr(w.W2q), _ptr(w.Ps2), w.W2q.stride(0),
+    rc = lib.moe_grouped_down_mxfp8(_ptr(Hq), _ptr(Hsp), _ptr(w.W2q), _ptr(w.Ps2), w.W2q.stride(0),
                                     _ptr(offsets), E, R, d, F, _ptr(Ye), _stream(Hq))
     _check("moe_grouped_down_mxfp8", rc)
     return Ye

@@ -301,9 +301,12 @@ MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mod
  *   W1q/W3q [E,F,d] + W1s/W3s [E,F,d/32]; W2q [E,d,F] + W2s [E,d,F/32];
  *   expert strides in elements of the code tensors. The GEMMs take the
  *   weight scales packed once by mxfp8_pack_weight_scales (below).
- *   gate/up writes H quantised from its fp32 value: Hq [R,F] + Hs [R,F/32];
- *   down writes Ye [R,d] bf16. Limits: d % 128 == 0, F % 128 == 0; code
- *   and packed-scale pointers 16-byte aligned, Xs/Hs 4-byte aligned.
+ *   The activation scales they read (Xs for gate/up, Hs for down) are in the
+ *   tile-packed layout of mxfp8_pack_act_scales (below); gate/up writes H
+ *   quantised from its fp32 value: Hq [R,F] codes and its scales Hs in that
+ *   same tile-packed layout (K = F), ready for down; down writes Ye [R,d]
+ *   bf16. Limits: d % 128 == 0, F % 128 == 0; code and scale pointers
+ *   16-byte aligned.
  *
  * mxfp8_pack_weight_scales: the weight scales in the order the GEMMs'
  *   tensor-core scale copy reads them, so each pipeline stage fetches them
@@ -316,12 +319,32 @@ MOE_API int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_mod
  *   Ps13: E*(F/128)*(d/128)*1024 bytes (from W1s, W3s); Ps2:
  *   E*ceil(d/256)*(F/128)*1024 bytes (from W2s). Either pair may be NULL.
  *   Scale tensors contiguous as above; packed outputs 16-byte aligned.
+ *
+ * mxfp8_pack_act_scales / mxfp8_unpack_act_scales: activation scales between
+ *   the row layout S [R, K/32] (K-block bytes of each expert-sorted row, as
+ *   moe_dispatch_mxfp8 and mxfp8_quantize write them) and the tile-packed
+ *   layout Sp the GEMMs copy with one bulk copy per stage. The rows of
+ *   expert e (offsets[e]..offsets[e+1], device int32 [E+1]) form
+ *   ceil(count/128) row tiles, numbered over the experts in order; for row
+ *   tile g and 128-element K slab s, the 512-byte block at (g*(K/128) + s)*512
+ *   holds the word (four K-block bytes) of tile row m at 16*(m % 32) +
+ *   4*(m / 32); tile rows past the expert's rows hold 0 (pack writes them;
+ *   unpack ignores them). Sp takes mxfp8_act_scales_packed_size(E, R, K) =
+ *   (R/128 + E)*(K/128)*512 bytes (an upper bound on the tiles; blocks past
+ *   the last tile are not touched). K % 128 == 0; S and Sp 16-byte aligned;
+ *   offsets not monotone from 0 to R set MOE_DEVERR_BAD_OFFSETS and nothing
+ *   is written.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T, int64_t d, int k,
                                uint8_t* Xq, uint8_t* Xs, void* stream);
 MOE_API int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s, const uint8_t* W2s,
                                      int64_t E, int64_t d, int64_t F, uint8_t* Ps13,
                                      uint8_t* Ps2, void* stream);
+MOE_API size_t mxfp8_act_scales_packed_size(int64_t E, int64_t R, int64_t K);
+MOE_API int mxfp8_pack_act_scales(const uint8_t* S, const int32_t* offsets, int64_t E, int64_t R,
+                                  int64_t K, uint8_t* Sp, void* stream);
+MOE_API int mxfp8_unpack_act_scales(const uint8_t* Sp, const int32_t* offsets, int64_t E,
+                                    int64_t R, int64_t K, uint8_t* S, void* stream);
 MOE_API int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
                                       const uint8_t* W3q, const uint8_t* Ps13,
                                       int64_t w13_expert_stride, const int32_t* offsets, int64_t E,

@@ -181,3 +181,50 @@ def test_pack_weight_scales_layout(E, d, F):
                     want2.append(block(rows[:, 4 * s:4 * s + 4]))
     assert np.array_equal(got13, np.concatenate(want13))
     assert np.array_equal(got2, np.concatenate(want2))
+
+
+@pytest.mark.parametrize("counts,K", [([0, 130, 1, 256, 5], 256), ([300], 128), ([7, 0, 0, 129], 512)])
+def test_act_scales_pack_layout_and_roundtrip(counts, K):
+    """Tile-packed activation scales as the header defines them: row tiles
+    of 128 per expert (ceil(count/128) each, numbered in expert order), one
+    512-byte block per (tile, K slab), word of tile row m at
+    16*(m % 32) + 4*(m / 32), tile rows past the expert's rows zero; unpack
+    restores the rows."""
+    moe = _moe()
+    E = len(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offs[-1])
+    g = torch.Generator().manual_seed(R + K)
+    S = torch.randint(0, 256, (R, K // 32), generator=g, dtype=torch.uint8)
+    Sp = moe.mxfp8_pack_act_scales(S.cuda(), torch.from_numpy(offs).cuda(), E)
+    got = Sp.cpu().numpy()
+    ks = K // 128
+    want = []
+    for e in range(E):
+        rows = S[offs[e]:offs[e + 1]].numpy()
+        for mt in range((counts[e] + 127) // 128):
+            tile = rows[128 * mt:128 * mt + 128]
+            for s in range(ks):
+                b = np.zeros(512, dtype=np.uint8)
+                for m in range(tile.shape[0]):
+                    o = 16 * (m % 32) + 4 * (m // 32)
+                    b[o:o + 4] = tile[m, 4 * s:4 * s + 4]
+                want.append(b)
+    want = np.concatenate(want) if want else np.zeros(0, np.uint8)
+    assert np.array_equal(got[:want.size], want)
+    back = moe.mxfp8_unpack_act_scales(Sp, torch.from_numpy(offs).cuda(), E, R, K)
+    assert np.array_equal(back.cpu().numpy(), S.numpy())
+    assert moe.moe_get_status() == 0
+
+
+def test_act_scales_bad_offsets_flagged():
+    moe = _moe()
+    offs = torch.tensor([0, 40, 30, 64], dtype=torch.int32, device="cuda")  # not monotone
+    S = torch.zeros((64, 4), dtype=torch.uint8, device="cuda")
+    Sp = torch.full((moe.lib.mxfp8_act_scales_packed_size(3, 64, 128),), 7, dtype=torch.uint8,
+                    device="cuda")
+    moe.mxfp8_pack_act_scales(S, offs, 3, Sp)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status(clear=True) & moe.MOE_DEVERR_BAD_OFFSETS
+    assert (Sp.cpu() == 7).all()  # nothing written
+    assert moe.moe_get_status() == 0
