@@ -7,9 +7,11 @@
 One step = one pass of the whole layer over one batch: route (router logits,
 fp32 softmax + top-k, routing metadata) -> dispatch -> grouped gate/up GEMM
 with SwiGLU -> grouped down GEMM -> combine, each through the C ABI.
-`value` = tokens/s of the whole job with inputs resident in HBM; `e2e` = the
-same metric through moe_layer_fwd with the step's input copied from pinned
-host memory and the output copied back inside the timed region.
+`value` = tokens/s of the whole job with inputs resident in HBM, timed over
+replays of one step captured in a CUDA graph (the same library calls; eager
+steps with --no-graph, and the eager per-part breakdown is always reported);
+`e2e` = the same metric through moe_layer_fwd with the step's input copied
+from pinned host memory and the output copied back inside the timed region.
 
 Multi-GPU: the layer is run as independent replicas, one process per GPU
 (launched by torch.distributed.run); there is no data-path collective.
@@ -425,21 +427,53 @@ def run_ours(args):
     if moe.moe_get_status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-           for _ in range(args.steps)]
+    # Timed region: the step captured once in a CUDA graph and replayed K
+    # times (the library's calls are stream-ordered launches with no host
+    # synchronisation or allocation, so a replay runs exactly the eager
+    # launches without the per-call host overhead); the evented eager steps
+    # that follow give the per-part breakdown. With --no-graph, or if any rank
+    # fails to capture, the eager steps are the timed region.
+    graph, ms_graph = None, None
+    if not args.no_graph:
+        graph = _capture_step(step, dev)
+        if max_over_ranks(0.0 if graph is not None else 1.0, world, dev) > 0:
+            graph = None
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    if graph is not None:
+        for _ in range(args.warmup):
+            graph.replay()
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        w0 = time.monotonic()
+        start.record()
+        for _ in range(args.steps):
+            graph.replay()
+        end.record()
+        torch.cuda.synchronize(dev)
+        w1 = time.monotonic()
+        barrier(world)
+        ms_graph = max_over_ranks(start.elapsed_time(end), world, dev)
+        del graph
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+           for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    w0 = time.monotonic()
+    e0 = time.monotonic()
     start.record()
     for i in range(args.steps):
         step(evs[i])
     end.record()
     torch.cuda.synchronize(dev)
-    w1 = time.monotonic()
+    e1 = time.monotonic()
     barrier(world)
-    ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
+    ms_eager = max_over_ranks(start.elapsed_time(end), world, dev)
+    if ms_graph is None:
+        ms_total, launch = ms_eager, "eager (one host call per library entry)"
+        w0, w1 = e0, e1
+    else:
+        ms_total, launch = ms_graph, "CUDA graph of one step, replayed (same library calls)"
     ms_step = ms_total / args.steps
     value = T * world * args.steps / (ms_total / 1e3)
     per = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, p in enumerate(parts)}
@@ -520,6 +554,7 @@ def run_ours(args):
         "hbm": {"dispatch_frac": rates["dispatch"]["gbs"] / hbm,
                 "combine_frac": rates["combine"]["gbs"] / hbm, "peak_gbs": hbm},
         "e2e": e2e, "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
+        "launch": launch, "ms_per_step_eager": ms_eager / args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
         inp_cpu = {kk: v.cpu() for kk, v in inp.items()}
@@ -528,6 +563,26 @@ def run_ours(args):
         line["cpu_baseline"] = None
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _capture_step(step, dev):
+    """One step captured in a CUDA graph (after a warm call on the capture
+    stream), or None if capture is not possible here."""
+    try:
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        torch.cuda.synchronize(dev)
+        return g
+    except RuntimeError as ex:
+        print(f"bench: CUDA graph capture failed ({ex}); timing eager steps", file=sys.stderr)
+        return None
 
 
 def _e2e(moe, w, inp, dev, world, args, backward):
@@ -617,6 +672,8 @@ def main(argv=None):
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide T and E by this factor (profiling a small case of the same shape)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager steps instead of replays of one captured step")
     ap.add_argument("--e2e-chunks", type=int, default=0,
                     help="token slices of the host-buffer forward (copies overlap compute); "
                          "0 = chosen from the copy and weight-streaming times (moe.choose_chunks)")

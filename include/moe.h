@@ -5,7 +5,11 @@
  * memory; the library never allocates, frees or synchronises (except
  * moe_get_status, which reads the device status word). All work is enqueued
  * on the caller's stream, passed as a `void*` holding a cudaStream_t
- * (NULL = legacy default stream).
+ * (NULL = legacy default stream). So any sequence of calls other than
+ * moe_get_status and the *_host entries can be captured into a CUDA graph
+ * and replayed (the replay reads the buffers' current contents); make one
+ * call of each entry on the device before capturing, since the first call
+ * sets kernel attributes.
  *
  * Notation: T tokens, d hidden size, E experts, k experts per token, F expert
  * FFN width, R = T*k rows of the expert-sorted buffers.
