@@ -1,7 +1,8 @@
 // Route step of the dropless top-k MoE layer on sm_100a.
 //
-//   a0  router logits  logits[t,e] = four fmaf chains over the quarters of j
-//                      of x[t,j]*Wr[e,j], added in order
+//   a0  router logits  logits[t,e] = sum_j x[t,j]*Wr[e,j]: bf16 on the tensor
+//                      cores (fp32 accumulation); fp32 as four fmaf chains
+//                      over the quarters of j, added in order
 //   a1  fp32 softmax + top-k (ties to the lower expert index)
 //   a2  routing metadata: counts, offsets, slots, tile offsets
 //
@@ -17,15 +18,15 @@
 //      token in order, marks each selection in a per-expert bit mask over the
 //      chunk's tokens, and reads a token's rank among the chunk's rows of the
 //      expert (stable by token) off the mask. Per-chunk counts go to
-//      ws_count[e][c]. When the logits are computed, it also adds the router's
-//      four quarter planes (and writes the logits out if asked).
+//      ws_count[e][c]. For the fp32 router it also adds the four quarter
+//      planes (and writes the logits out if asked).
 //   2. scan: one block per expert scans ws_count[e][:] over chunks (exclusive,
 //      in place) and writes counts[e]; the last block to finish (ticket
 //      counter) scans counts into offsets and tile_offsets.
 //   3. finalize: slot = offsets[e] + chunk_base[e][c] + rank.
 // Integer work only after the top-k, so the result is bit-exact and
 // independent of scheduling.
-#include "common.cuh"
+#include "tc_sm100.cuh"
 
 namespace moe {
 namespace route {
@@ -51,39 +52,26 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-template <typename TX>
-struct Landed16;  // 16 consecutive elements of a row in shared memory, as fp32
-
-template <>
-struct Landed16<__nv_bfloat16> {
-    __device__ static void to_f32(const uint4* p, float* f) {
-        unpack8(p[0], f);
-        unpack8(p[1], f + 8);
-    }
-};
-
-template <>
-struct Landed16<float> {
-    __device__ static void to_f32(const uint4* p, float* f) {
+// 16 consecutive fp32 elements of a row landed in shared memory, to registers.
+__device__ __forceinline__ void landed16_to_f32(const uint4* p, float* f) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 v = reinterpret_cast<const float4*>(p)[i];
-            f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
-        }
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(p)[i];
+        f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
     }
-};
+}
 
-// The logit of (t, e) is four fmaf chains, one per contiguous quarter of j,
-// each from +0.0 in ascending j, their sums added in order ((c0 + c1) + c2)
-// + c3. One CTA (64 threads) computes one quarter's chains for a 64-token x
-// 64-expert tile (grid z = quarter) and writes them to that quarter's plane;
-// the top-k kernel adds the four planes in order. Eight CTAs are resident
-// per SM, so the 1024 CTAs of the OLMoE shape run as one wave.
+// fp32 router. The logit of (t, e) is four fmaf chains, one per contiguous
+// quarter of j, each from +0.0 in ascending j, their sums added in order
+// ((c0 + c1) + c2) + c3. One CTA (64 threads) computes one quarter's chains
+// for a 64-token x 64-expert tile (grid z = quarter) and writes them to that
+// quarter's plane; the top-k kernel adds the four planes in order. Eight
+// CTAs are resident per SM (127 registers).
 //   staging: thread i copies 16 consecutive elements of x row t0 + i and of
 //            Wr row e0 + i per chunk into its own landing slots with
-//            cp.async (one chunk ahead), then converts them to fp32 into
-//            k-major shared memory (a warp writes 32 consecutive floats of
-//            one k: no conflicts);
+//            cp.async (one chunk ahead), then stores them k-major into shared
+//            memory (a warp writes 32 consecutive floats of one k: no
+//            conflicts);
 //   compute: thread (ty, tx) = (i / 8, i % 8) owns tokens 4ty..4ty+3 and
 //            32+4ty..32+4ty+3 and experts 4tx..4tx+3 and 32+4tx..32+4tx+3:
 //            64 accumulators; per k, 4 shared float4 loads (the eight tx of a
@@ -91,12 +79,11 @@ struct Landed16<float> {
 constexpr int LOGIT_THREADS = 64;
 constexpr int LOGIT_SPLIT = 4;  // quarter chains per logit
 
-template <typename TX>
 __global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
-    const TX* __restrict__ x, const TX* __restrict__ Wr, int T, int d, int E,
+    const float* __restrict__ x, const float* __restrict__ Wr, int T, int d, int E,
     float* __restrict__ planes, int64_t pstride) {
-    constexpr int PIECES = LOGIT_TK * (int)sizeof(TX) / 16;  // 16-byte pieces per row chunk
-    constexpr int PEL = 16 / (int)sizeof(TX);                // elements per piece
+    constexpr int PIECES = LOGIT_TK * (int)sizeof(float) / 16;  // 16-byte pieces per row chunk
+    constexpr int PEL = 16 / (int)sizeof(float);                // elements per piece
     __shared__ __align__(16) float xs[2][LOGIT_TK][LOGIT_LD];
     __shared__ __align__(16) float ws[2][LOGIT_TK][LOGIT_LD];
     __shared__ __align__(16) uint4 land[2][LOGIT_THREADS][PIECES];  // [x | Wr][row][piece]
@@ -109,8 +96,8 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
     const bool xok = (t0 + tid) < T;
     const bool wok = (e0 + tid) < E;
     // rows past T or E are zero-filled; their source address stays row 0's
-    const TX* xp = x + (size_t)(xok ? t0 + tid : 0) * d + kbeg;
-    const TX* wp = Wr + (size_t)(wok ? e0 + tid : 0) * d + kbeg;
+    const float* xp = x + (size_t)(xok ? t0 + tid : 0) * d + kbeg;
+    const float* wp = Wr + (size_t)(wok ? e0 + tid : 0) * d + kbeg;
     const uint32_t lx = (uint32_t)__cvta_generic_to_shared(&land[0][tid][0]);
     const uint32_t lw = (uint32_t)__cvta_generic_to_shared(&land[1][tid][0]);
     const int ty = tid >> 3, tx = tid & 7;
@@ -131,10 +118,10 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
         cp_async_wait_all();  // this thread's own copies of chunk k0
         {
             float f[16];
-            Landed16<TX>::to_f32(&land[0][tid][0], f);
+            landed16_to_f32(&land[0][tid][0], f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) xs[buf][i][tid] = f[i];
-            Landed16<TX>::to_f32(&land[1][tid][0], f);
+            landed16_to_f32(&land[1][tid][0], f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) ws[buf][i][tid] = f[i];
         }
@@ -182,6 +169,200 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
             }
         }
     }
+}
+
+// ------------------------------------------------------------------ a0, bf16
+//
+// bf16 router: logits = x Wrᵀ on the tensor cores. The pages' router is a
+// bias-free linear layer in the model's dtype ("Transformers 中的 OLMoE" §2);
+// every bf16 x bf16 product is exact in fp32 and tcgen05 (kind::f16) sums
+// them into an fp32 TMEM accumulator, in the order the tensor core chooses.
+// One CTA computes a 128-token x EN-expert tile (EN = 64, 128 or 256 from E;
+// grid.y covers E > 256): warp 0 lane 0 streams 128-byte K slabs of x and Wr
+// with TMA through an RT_STAGES ring, warp 1 lane 0 issues 4 MMAs per slab,
+// warps 2..5 read the accumulator (one TMEM lane quarter each) and store fp32
+// rows, masked to T and E. Every wait is bounded as in the grouped GEMMs.
+constexpr int RT_BM = 128;
+constexpr int RT_THREADS = 192;
+
+template <int EN>
+struct RtCfg {
+    static constexpr int A_BYTES = RT_BM * 128;
+    static constexpr int B_BYTES = EN * 128;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = EN <= 128 ? 6 : 4;
+    static constexpr int NUM_BARS = 2 * STAGES + 2;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + NUM_BARS * 8 + 16;
+    static constexpr uint32_t IDESC = tc::make_idesc(1u, RT_BM, EN);
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+template <int EN>
+__global__ void __launch_bounds__(RT_THREADS, 1)
+    router_logits_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ CUtensorMap tmW, int T, int d, int E,
+                            float* __restrict__ logits, int vec, int* status) {
+    using namespace tc;
+    using C = RtCfg<EN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + C::STAGES;
+    uint64_t* done = bars + 2 * C::STAGES;
+    uint64_t* drain = done + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.x * RT_BM;
+    const int n0 = blockIdx.y * EN;
+    const int KS = d / 64;  // 128-byte slabs of bf16
+
+    if (tid == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        mbar_init(smem_u32(done), 1);
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmX);
+        prefetch_map(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s_tmem), EN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int kb = 0; kb < KS; ++kb) {
+            if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            const uint32_t fb = smem_u32(full + stage);
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+            mbar_expect_tx(fb, (uint32_t)C::STAGE_BYTES);
+            tma_load_2d(sa, &tmX, fb, kb * 64, m0);
+            tma_load_2d(sa + C::A_BYTES, &tmW, fb, kb * 64, n0);
+            issued_mask |= 1u << stage;
+            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) {  // no copy may still be landing when the CTA leaves
+            for (int s = 0; s < C::STAGES; ++s)
+                if ((issued_mask >> s) & 1u) {
+                    volatile int no_abort = 0;
+                    mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                              DRAIN_LIMIT_NS);
+                }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int kb = 0; kb < KS; ++kb) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+            const uint64_t ad = sw128_desc(sa);
+            const uint64_t bd = sw128_desc(sa + C::A_BYTES);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma<false>(tmem_base, ad + 2 * ks, bd + 2 * ks, C::IDESC, (kb | ks) != 0);
+            tc_commit(smem_u32(empty + stage));
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (ok) {
+            tc_commit(smem_u32(done));
+        } else {
+            tc_commit(smem_u32(drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        if (mbar_wait(smem_u32(done), 0, s_abort, status, WAIT_LIMIT_NS)) {
+            tc_fence_after();
+            const int t = m0 + q * 32 + lane;
+            const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < EN / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld32(ta + 32 * c, a);
+                tmem_wait_ld();
+                const int e0 = n0 + 32 * c;
+                if (t < T && e0 < E) {
+                    float* row = logits + (size_t)t * E + e0;
+                    if (vec && e0 + 32 <= E) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(row + j) =
+                                make_float4(__uint_as_float(a[j]), __uint_as_float(a[j + 1]),
+                                            __uint_as_float(a[j + 2]), __uint_as_float(a[j + 3]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (e0 + j < E) row[j] = __uint_as_float(a[j]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, EN);
+    }
+}
+
+template <int EN>
+static int launch_router_tc(const void* x, const void* Wr, int64_t T, int64_t d, int64_t E,
+                            float* logits, cudaStream_t st) {
+    using C = RtCfg<EN>;
+    auto kern = router_logits_tc_kernel<EN>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    CUtensorMap mx, mw;
+    if (!tc::make_map_2d(&mx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, T, RT_BM) ||
+        !tc::make_map_2d(&mw, Wr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, E, EN))
+        return MOE_ERR_CUDA;
+    const int vec = (E % 4 == 0) && aligned16(logits);
+    dim3 grid((unsigned)((T + RT_BM - 1) / RT_BM), (unsigned)((E + EN - 1) / EN));
+    kern<<<grid, RT_THREADS, C::SMEM_BYTES, st>>>(mx, mw, (int)T, (int)d, (int)E, logits, vec,
+                                                  status_ptr());
+    return MOE_OK;
 }
 
 // ------------------------------------------------------------------ a1
@@ -478,11 +659,13 @@ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 struct RouteWs {
     int32_t* count;
     int32_t* ticket;
-    float* planes;  // the four [T,E] quarter planes when the logits are computed
+    float* planes;  // four [T,E] planes when the logits are computed
 };
 
 // from_x: the logits are computed from x and Wr; the workspace then also
-// holds the four quarter planes (the top-k adds them itself).
+// holds four [T,E] planes: the fp32 router's quarter chains (the top-k adds
+// them), or in the first plane the bf16 router's logits when the caller does
+// not ask for them.
 inline int64_t plane_stride(int64_t T, int64_t E) { return (T * E + 63) / 64 * 64; }
 
 inline size_t workspace_bytes(int64_t T, int64_t E, bool from_x) {
@@ -583,24 +766,36 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     cudaStream_t st = as_stream(stream);
     route::RouteWs ws = route::carve(workspace, T, E, from_x);
 
-    if (from_x) {
+    int chunk = 0;
+    if (from_x && dtype == MOE_BF16) {
+        // tensor cores, fp32 accumulation; the top-k reads the one plane
+        float* dst = logits_out ? logits_out : ws.planes;
+        int rc = MOE_OK;
+        if (E <= 64)
+            rc = route::launch_router_tc<64>(x, Wr, T, d, E, dst, st);
+        else if (E <= 128)
+            rc = route::launch_router_tc<128>(x, Wr, T, d, E, dst, st);
+        else
+            rc = route::launch_router_tc<256>(x, Wr, T, d, E, dst, st);
+        if (rc != MOE_OK) return rc;
+        chunk = route::launch_topk(dst, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate, slot,
+                                   ws.count, st);
+    } else if (from_x) {
+        // fp32 router: four fixed-order fmaf chains per logit on the CUDA
+        // cores (tf32 tensor cores would round the inputs); the top-k adds
+        // the four quarter planes
         dim3 grid((unsigned)((T + route::LOGIT_TT - 1) / route::LOGIT_TT),
                   (unsigned)((E + route::LOGIT_TE - 1) / route::LOGIT_TE), route::LOGIT_SPLIT);
-        if (dtype == MOE_BF16)
-            route::router_logits_kernel<__nv_bfloat16><<<grid, route::LOGIT_THREADS, 0, st>>>(
-                static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
-                (int)T, (int)d, (int)E, ws.planes, route::plane_stride(T, E));
-        else
-            route::router_logits_kernel<float><<<grid, route::LOGIT_THREADS, 0, st>>>(
-                static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d,
-                (int)E, ws.planes, route::plane_stride(T, E));
+        route::router_logits_kernel<<<grid, route::LOGIT_THREADS, 0, st>>>(
+            static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d, (int)E,
+            ws.planes, route::plane_stride(T, E));
+        chunk = route::launch_topk(ws.planes, route::LOGIT_SPLIT, route::plane_stride(T, E),
+                                   (int)T, (int)E, k, renorm, logits_out, idx, gate, slot,
+                                   ws.count, st);
+    } else {
+        chunk = route::launch_topk(logits, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate,
+                                   slot, ws.count, st);
     }
-    // the in-chunk ranks are parked in `slot` and completed by finalize_kernel
-    const int chunk = from_x ? route::launch_topk(ws.planes, route::LOGIT_SPLIT,
-                                                  route::plane_stride(T, E), (int)T, (int)E, k,
-                                                  renorm, logits_out, idx, gate, slot, ws.count, st)
-                             : route::launch_topk(logits, 1, 0, (int)T, (int)E, k, renorm,
-                                                  nullptr, idx, gate, slot, ws.count, st);
     if (chunk == 0) return MOE_ERR_UNSUPPORTED;
     const int nch = (int)((T + chunk - 1) / chunk);
     if (cudaMemsetAsync(ws.ticket, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -86,12 +86,14 @@ extern "C" {
  *
  * Inputs (device):
  *   logits   [T,E] fp32 row-major, or NULL to compute logits = x·Wrᵀ from
- *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). The logit
- *            of (t,e) is four fp32 accumulators, one per contiguous quarter
- *            of j, each starting from +0.0 and updated by fused multiply-add
- *            in ascending j; the four are then added in order,
- *            ((c0 + c1) + c2) + c3. (The pages leave the order open; it is
- *            fixed because the top-k is taken on these bits.)
+ *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). bf16:
+ *            the tensor cores sum the exact bf16 products into fp32, in their
+ *            own order (the pages' router is a linear layer in the model
+ *            dtype). fp32: the logit of (t,e) is four fp32 accumulators, one
+ *            per contiguous quarter of j, each starting from +0.0 and updated
+ *            by fused multiply-add in ascending j, then added in order,
+ *            ((c0 + c1) + c2) + c3 (tf32 tensor cores would round the
+ *            inputs). The top-k is taken on the logits so computed.
  *   renorm   0: gates are the softmax probabilities; 1: divided by their sum.
  * Outputs (device, caller-allocated):
  *   logits_out  [T,E] fp32, or NULL (used only when logits == NULL)

@@ -63,3 +63,29 @@ def assert_close_scaled(got, ref, what="", max_abs=MAX_ABS, rel=REL_L2):
     rl = rel_l2(got, ref)
     assert ma <= max_abs and rl <= rel, f"{what}: scaled max-abs {ma:.3e} rel-L2 {rl:.3e}"
     return ma, rl
+
+
+def router_logits_checked(got, x: torch.Tensor, Wr: torch.Tensor) -> np.ndarray:
+    """Router logits from the GPU against the oracle's fixed-order fp32 logits,
+    returning the logits both sides route on (the GPU's).
+
+    fp32 inputs: the GPU runs the oracle's four in-order fmaf chains, so the
+    bits must agree. bf16 inputs: every product is exact in fp32 and both
+    sides are fp32 sums of the same d products, the tensor core in its own
+    order; a recursive fp32 sum of d terms errs by at most (d-1) 2^-24
+    sum|terms|, so the two differ by at most 2 (d-1) 2^-24 sum_j |x_j w_j|;
+    the bound doubles that for the tensor core's internal accumulation.
+    """
+    from oracle import moe_oracle as O
+    got = np.asarray(got, dtype=np.float32)
+    ref = O.router_logits(x, Wr)
+    if x.dtype == torch.float32:
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), "fp32 router logits"
+        return got
+    xa = np.abs(x.detach().cpu().double().numpy())
+    wa = np.abs(Wr.detach().cpu().double().numpy())
+    d = x.shape[1]
+    bound = 4.0 * (d - 1) * 2.0 ** -24 * (xa @ wa.T)
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= bound), f"bf16 router logits: worst err/bound {np.max(err / bound):.3e}"
+    return got

@@ -9,7 +9,7 @@ import torch
 
 from oracle import moe_oracle as O
 from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
-from tests._util import assert_close_layer, assert_close_scaled, np64
+from tests._util import assert_close_layer, assert_close_scaled, np64, router_logits_checked
 
 pytestmark = pytest.mark.gpu
 
@@ -154,8 +154,9 @@ def test_layer_backward_with_router(renorm, router_from_x):
                            Wr=kw.get("Wr"), aux_coef=0.01)
     torch.cuda.synchronize()
     assert moe.moe_get_status() == 0
-    ref = (O.moe_layer(x, k, W1, W3, W2, Wr=Wr, renorm=renorm) if router_from_x
-           else O.moe_layer(x, k, W1, W3, W2, logits=lg, renorm=renorm))
+    if router_from_x:  # route both sides on the GPU's logits (checked against the oracle's)
+        lg = router_logits_checked(fwd.logits.cpu().numpy(), x, Wr)
+    ref = O.moe_layer(x, k, W1, W3, W2, logits=lg, renorm=renorm)
     idx = ref["idx"]
     assert np.array_equal(gr.dgate.shape, (T, k))
     assert np.array_equal(fwd.idx.cpu().numpy(), idx)

@@ -7,7 +7,7 @@ import torch
 
 from oracle import moe_oracle as O
 from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
-from tests._util import assert_close_layer, assert_close_scaled, np64
+from tests._util import assert_close_layer, assert_close_scaled, np64, router_logits_checked
 
 pytestmark = pytest.mark.gpu
 
@@ -212,8 +212,9 @@ def test_layer_small_full_check(dtype):
     T, d, F, E, k = 777, 256, 384, 12, 3
     x, W1, W3, W2, lg = _problem(T, d, F, E, k, dtype, seed=99)
     Wr = (torch.randn(E, d, generator=torch.Generator().manual_seed(5)) * 0.05).to(dtype)
-    r = moe.moe_layer_fwd(x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda(), Wr=Wr.cuda())
-    ref = O.moe_layer(x, k, W1, W3, W2, Wr=Wr)
+    r = moe.moe_layer_fwd(x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda(), Wr=Wr.cuda(), save=True)
+    lg = router_logits_checked(r.logits.cpu().numpy(), x, Wr)
+    ref = O.moe_layer(x, k, W1, W3, W2, logits=lg)
     assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
     assert np.array_equal(r.slot.cpu().numpy(), ref["slot"])
     assert np.array_equal(r.offsets.cpu().numpy(), ref["offsets"])
@@ -242,12 +243,13 @@ def test_layer_full_size_sampled(name):
     moe = _moe()
     w = WORKLOADS[name]
     inp = make_inputs(w, "cuda")
-    kw = dict(Wr=inp["Wr"]) if w.logits == "router" else dict(logits=inp["logits"])
-    r = moe.moe_layer_fwd(inp["x"], w.k, inp["W1"], inp["W3"], inp["W2"], **kw)
+    router = w.logits == "router"
+    kw = dict(Wr=inp["Wr"]) if router else dict(logits=inp["logits"])
+    r = moe.moe_layer_fwd(inp["x"], w.k, inp["W1"], inp["W3"], inp["W2"], save=router, **kw)
     torch.cuda.synchronize()
     assert moe.moe_get_status() == 0
     x_cpu = inp["x"].cpu()
-    lg = (O.router_logits(x_cpu, inp["Wr"].cpu()) if w.logits == "router"
+    lg = (router_logits_checked(r.logits.cpu().numpy(), x_cpu, inp["Wr"].cpu()) if router
           else inp["logits"].cpu().numpy())
     idx, gate, _ = O.route(lg, w.k)
     meta = O.routing_metadata(idx, w.E)

@@ -10,7 +10,7 @@ import torch
 
 from oracle import moe_oracle as O
 from dropless_top_mixture_b200.workloads import WORKLOADS, make_inputs
-from tests._util import assert_close_layer, np64, rel_l2
+from tests._util import assert_close_layer, np64, rel_l2, router_logits_checked
 
 pytestmark = pytest.mark.gpu
 
@@ -151,7 +151,8 @@ def test_router_backward_chain_through_the_layer():
     dx = torch.zeros(T, d, dtype=torch.bfloat16, device="cuda")
     _, dWr = moe.moe_router_linear_bwd(r.dlogits, xd, Wrd, dx=dx)
     assert moe.moe_get_status() == 0
-    ref = O.moe_layer(x, k, W1, W3, W2, Wr=Wr)
+    lg = router_logits_checked(rt.logits.cpu().numpy(), x, Wr)
+    ref = O.moe_layer(x, k, W1, W3, W2, logits=lg)
     idx = ref["idx"]
     assert np.array_equal(rt.idx.cpu().numpy(), idx)
     Y = ref["Ye"][ref["slot"]]
