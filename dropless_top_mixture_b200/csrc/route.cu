@@ -520,6 +520,7 @@ __global__ void __launch_bounds__(topk_threads_of(G), 1) topk_group_kernel(
     // each lane finishes its own selections j = g, g + G, ...; with renorm
     // the gates are written after the barrier, divided by their sum
     const uint32_t bit = 1u << tl;
+    __syncthreads();  // every thread's share of the masks is zeroed
     if (live) {
         for (int j = g; j < k; j += G) {
             const int e = sel[tl][j];

@@ -107,8 +107,9 @@ extern "C" {
  *   tile_offsets [E+1] int32 exclusive prefix sum of ceil(counts/128), or NULL
  * Workspace: `workspace_bytes` >= moe_route_workspace_size(T, E,
  *            logits == NULL); 256-byte aligned device memory (with logits
- *            computed it holds the four quarter sums, which the top-k adds
- *            itself). Its contents need not be initialised.
+ *            computed it holds four [T,E] fp32 planes: the fp32 router's
+ *            quarter sums, or the bf16 router's logits when logits_out is
+ *            NULL). Its contents need not be initialised.
  * Limits: 1 <= k <= min(E, 32), E <= 512; when computing logits d % 128 == 0
  *            and logits_out (if given) 16-byte aligned.
  * ---------------------------------------------------------------------- */
@@ -381,7 +382,8 @@ typedef struct moe_layer_mxfp8_args {
     int32_t* counts;
     int32_t* offsets;
     int32_t* slot;
-    void* workspace;        /* Xq, Xs, Hq, Hs, Ye and the route workspace     */
+    void* workspace;        /* Xq, Xs (rows and tile-packed), Hq, Hs (packed),
+                               Ye and the route workspace                     */
     size_t workspace_bytes;
 } moe_layer_mxfp8_args;
 
