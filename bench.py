@@ -8,8 +8,9 @@ One step = one pass of the whole layer over one batch: route (router logits,
 fp32 softmax + top-k, routing metadata) -> dispatch -> grouped gate/up GEMM
 with SwiGLU -> grouped down GEMM -> combine, each through the C ABI.
 `value` = tokens/s of the whole job with inputs resident in HBM, timed over
-replays of one step captured in a CUDA graph (the same library calls; eager
-steps with --no-graph, and the eager per-part breakdown is always reported);
+one replay of the K steps captured in a CUDA graph (the same library calls,
+with CUDA events between the parts captured too, which give the breakdown);
+eager steps with --no-graph (their time is always reported as well);
 `e2e` = the same metric through moe_layer_fwd with the step's input copied
 from pinned host memory and the output copied back inside the timed region.
 
@@ -427,43 +428,52 @@ def run_ours(args):
     if moe.moe_get_status() != 0:
         raise RuntimeError("device status word set during warm-up")
 
-    # Timed region: the step captured once in a CUDA graph and replayed K
-    # times (the library's calls are stream-ordered launches with no host
+    # Timed region: the K steps captured once in a CUDA graph, with CUDA events
+    # between the parts of every step captured too (external events become
+    # event-record nodes), and the graph replayed once after an untimed warm
+    # replay. The library's calls are stream-ordered launches with no host
     # synchronisation or allocation, so a replay runs exactly the eager
-    # launches without the per-call host overhead); the evented eager steps
-    # that follow give the per-part breakdown. With --no-graph, or if any rank
-    # fails to capture, the eager steps are the timed region.
+    # launches without the per-call host overhead, and the part times come
+    # from the timed region itself. K eager steps follow (ms_per_step_eager);
+    # with --no-graph, or if any rank fails to capture, they are the timed
+    # region.
+    def make_events():
+        return [[torch.cuda.Event(enable_timing=True, external=True)
+                 for _ in range(len(parts) + 1)] for _ in range(args.steps)]
+
+    evs = make_events()
     graph, ms_graph = None, None
     if not args.no_graph:
-        graph = _capture_step(step, dev)
+        graph = _capture_step(lambda: [step(evs[i]) for i in range(args.steps)], dev)
         if max_over_ranks(0.0 if graph is not None else 1.0, world, dev) > 0:
             graph = None
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    per = None
     if graph is not None:
-        for _ in range(args.warmup):
-            graph.replay()
+        graph.replay()  # untimed: the K captured steps once more
+        torch.cuda.synchronize(dev)
         barrier(world)
         torch.cuda.synchronize(dev)
         w0 = time.monotonic()
         start.record()
-        for _ in range(args.steps):
-            graph.replay()
+        graph.replay()
         end.record()
         torch.cuda.synchronize(dev)
         w1 = time.monotonic()
         barrier(world)
         ms_graph = max_over_ranks(start.elapsed_time(end), world, dev)
+        per = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+               for j, p in enumerate(parts)}
         del graph
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-           for _ in range(args.steps)]
+    evs_e = make_events()
     barrier(world)
     torch.cuda.synchronize(dev)
     e0 = time.monotonic()
     start.record()
     for i in range(args.steps):
-        step(evs[i])
+        step(evs_e[i])
     end.record()
     torch.cuda.synchronize(dev)
     e1 = time.monotonic()
@@ -472,11 +482,13 @@ def run_ours(args):
     if ms_graph is None:
         ms_total, launch = ms_eager, "eager (one host call per library entry)"
         w0, w1 = e0, e1
+        per = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs_e)
+               for j, p in enumerate(parts)}
     else:
-        ms_total, launch = ms_graph, "CUDA graph of one step, replayed (same library calls)"
+        ms_total = ms_graph
+        launch = "CUDA graph of the K steps (same library calls), replayed once"
     ms_step = ms_total / args.steps
     value = T * world * args.steps / (ms_total / 1e3)
-    per = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, p in enumerate(parts)}
 
     # clocks: the timed window; if it held too few samples, keep running
     # untimed steps of the same workload while sampling
@@ -566,7 +578,7 @@ def run_ours(args):
 
 
 def _capture_step(step, dev):
-    """One step captured in a CUDA graph (after a warm call on the capture
+    """`step` captured in a CUDA graph (after a warm call on the capture
     stream), or None if capture is not possible here."""
     try:
         s = torch.cuda.Stream(dev)
