@@ -47,17 +47,23 @@ constexpr int BOX_BYTES = 64 * 128;  // one MN-major box: 64 K rows x 64 element
 constexpr int TMEM_ALLOC = 512;
 constexpr int STG_BYTES = 32 * 128;  // dW store staging: 32 rows x 64 bf16, one per buffer
 
-enum Mode { DH = 0, DX = 1, DW = 2 };
+// DXR and DWF serve the router GEMM backward (one row group, or token chunks
+// as groups): DXR is DH's operand layout with an epilogue that adds the
+// product into the existing out0 rows; DWF is DW with fp32 output tiles (the
+// partials of a split-K sum).
+enum Mode { DH = 0, DX = 1, DW = 2, DXR = 3, DWF = 4 };
+template <int MODE>
+constexpr bool is_dw() { return MODE == DW || MODE == DWF; }
 
 // DW tiles have a short K (an expert's rows) and a large output, so they use
 // fewer pipeline stages and spend the shared memory on store staging
 // (4 epilogue warps x 2 buffers) for TMA tensor stores.
 template <int MODE>
 struct ModeCfg {
-    static constexpr bool A_MN = (MODE == DW);
+    static constexpr bool A_MN = is_dw<MODE>();
     static constexpr uint32_t IDESC = make_idesc_major(1u, BM, MMA_N, A_MN, true);
-    static constexpr int STAGES = (MODE == DW) ? 3 : 4;
-    static constexpr int STAGING = (MODE == DW) ? EPI_WARPS * 2 * STG_BYTES : 0;
+    static constexpr int STAGES = is_dw<MODE>() ? 3 : 4;
+    static constexpr int STAGING = is_dw<MODE>() ? EPI_WARPS * 2 * STG_BYTES : 0;
     static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING + META_BYTES;
@@ -74,7 +80,7 @@ template <int MODE>
 __device__ __forceinline__ Tile decode(int t, int E, int NB, int MB, int K, const int* s_toff,
                                        const int* s_off) {
     Tile tl;
-    if (MODE == DW) {
+    if (is_dw<MODE>()) {
         const int tpe = MB * NB;
         const int e = t / tpe;
         const int l = t - e * tpe;
@@ -183,8 +189,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
     const int NB = Ndim / MMA_N;
-    const int MB = (MODE == DW) ? Mdim / BM : 1;
-    const int total = (MODE == DW) ? E * MB * NB : s_toff[E] * NB;
+    const int MB = is_dw<MODE>() ? Mdim / BM : 1;
+    const int total = is_dw<MODE>() ? E * MB * NB : s_toff[E] * NB;
     if ((int)blockIdx.x >= total) return;
     const int KF = K / 2 / BK;  // DX: slabs per operand pair
 
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                 const uint32_t sb = sa + A_BYTES;
                 mbar_expect_tx(fb, STAGE_BYTES);
-                if (MODE == DH) {
+                if (MODE == DH || MODE == DXR) {
                     tma_load_2d(sa, &tmA0, fb, kb * BK, tl.row0);
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sa = smem_u32(sa_p);
                 const uint32_t sb = sa + A_BYTES;
                 int nks = 4;  // 16-row K steps of this slab the MMAs consume
-                if (MODE == DW) {
+                if (is_dw<MODE>()) {
                     const int valid = tl.row_end - (tl.row0 + kb * BK);
                     if (valid < BK) {
                         // The slab ends inside the expert's last rows: only the K
@@ -364,7 +370,40 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
-            if (MODE == DW) {
+            if (MODE == DWF) {
+                // 32-column groups: TMEM -> fp32 -> 128-byte-swizzled staging
+                // (chunk c of row r at c ^ (r % 8)) -> TMA store of the warp's
+                // 32 x 32 fp32 box; two staging buffers per warp
+                const bool empty_k = tl.nkb == 0;
+                const int ybase = tl.e * Mdim + tl.m0 + q * 32;
+                uint8_t* stg = staging + (warp - 2) * 2 * STG_BYTES;
+#pragma unroll 1
+                for (int cc = col0 / 32; cc < (col0 + MMA_N / 2) / 32; ++cc) {
+                    uint8_t* sbuf = stg + (stg_count & 1) * STG_BYTES;
+                    ++stg_count;
+                    if (lane == 0) bulk_wait_read<1>();  // this buffer's previous store has read it
+                    __syncwarp();
+                    uint32_t a[32];
+                    if (!empty_k) {
+                        tmem_ld32(ta + cc * 32, a);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) a[j] = 0u;
+                    }
+#pragma unroll
+                    for (int chunk = 0; chunk < 8; ++chunk)
+                        *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                            make_uint4(a[4 * chunk], a[4 * chunk + 1], a[4 * chunk + 2],
+                                       a[4 * chunk + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmOut, smem_u32(sbuf), tl.n0 + cc * 32, ybase);
+                        bulk_commit();
+                    }
+                }
+            } else if (MODE == DW) {
                 // 64-column groups: TMEM -> bf16 -> 128-byte-swizzled staging
                 // (chunk c of row r at c ^ (r % 8), conflict-free) -> TMA store
                 // of the warp's 32 x 64 box; two staging buffers per warp
@@ -415,7 +454,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     float v[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
-                    if (MODE == DH) {
+                    if (MODE == DXR) {
+                        float old[32];
+                        load32_bf16(out0 + rowoff + c * 32, old);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] += old[j];
+                        store32_bf16(out0 + rowoff + c * 32, v);
+                    } else if (MODE == DH) {
                         float ga[32], ub[32], da[32], db[32];
                         load32_bf16(saveA + rowoff + c * 32, ga);
                         load32_bf16(saveB + rowoff + c * 32, ub);
@@ -438,7 +483,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(tempty + buf));
         }
-        if (MODE == DW && lane == 0) bulk_wait<0>();  // stores done before the CTA leaves
+        if (is_dw<MODE>() && lane == 0) bulk_wait<0>();  // stores done before the CTA leaves
         __syncwarp();
     }
 
@@ -468,7 +513,7 @@ static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMa
         attr_done[dev] = true;
     }
     const int64_t NB = Ndim / MMA_N;
-    const int64_t max_tiles = (MODE == DW) ? E * (Mdim / BM) * NB : (R / BM + E) * NB;
+    const int64_t max_tiles = is_dw<MODE>() ? E * (Mdim / BM) * NB : (R / BM + E) * NB;
     const int64_t sms = num_sms();
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
@@ -483,6 +528,42 @@ static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMa
 constexpr CUtensorMapDataType BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
 }  // namespace bwd
+}  // namespace moe
+
+namespace moe {
+
+// Router GEMM backward on the tensor cores, for router_bwd.cu. dl: dlogits in
+// bf16, [T, Ep] with Ep = E rounded up to 64 and zeros past E. dx (if not
+// null) += dl Wr: DXR over one row group (off_one = {0, T}), K = Ep, with Wr
+// [E, d] read MN-major (rows past E read as zeros). partial (if not null):
+// for token chunk g (off_chunks, G chunks), rows 0..Mp-1 of dlᵀ x over the
+// chunk's tokens, fp32 [G*Mp, d] (DWF, M = Mp = Ep rounded up to 128, columns
+// of dl past Ep read as zeros). d % 256 == 0.
+int router_linear_bwd_tc(const void* dl, int64_t Ep, const void* x, const void* Wr, int64_t T,
+                         int64_t d, int64_t E, const int32_t* off_one, const int32_t* off_chunks,
+                         int64_t G, int64_t Mp, void* dx, float* partial, cudaStream_t st) {
+    using namespace tc;
+    if (dx) {
+        CUtensorMap ma, mb;
+        if (!make_map_2d(&ma, dl, bwd::BF16, 2, Ep, T, bwd::BM) ||
+            !make_map_3d(&mb, Wr, bwd::BF16, 2, d, E, 1, E * d, 64))
+            return MOE_ERR_CUDA;
+        const int rc = bwd::launch<bwd::DXR>(ma, ma, mb, mb, ma, off_one, 1, T, Ep, 0, d, dx,
+                                             nullptr, d, nullptr, nullptr, st);
+        if (rc != MOE_OK) return rc;
+    }
+    if (partial) {
+        CUtensorMap ma, mb, mo;
+        if (!make_map_2d(&ma, dl, bwd::BF16, 2, Ep, T, 64) ||
+            !make_map_2d(&mb, x, bwd::BF16, 2, d, T, 64) ||
+            !make_map_2d(&mo, partial, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, G * Mp, 32))
+            return MOE_ERR_CUDA;
+        return bwd::launch<bwd::DWF>(ma, ma, mb, mb, mo, off_chunks, G, T, 0, Mp, d, nullptr,
+                                     nullptr, d, nullptr, nullptr, st);
+    }
+    return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;

@@ -446,7 +446,83 @@ inline DwrSplit dwr_split(int64_t T, int64_t d, int64_t E) {
     return s;
 }
 
+// ---------------------------------------------------------------- tensor-core path
+//
+// bf16 router GEMM backward on the tensor cores (the router is a linear
+// layer in the model's dtype, "Transformers 中的 OLMoE" §2, and its backward
+// runs in that dtype too): dlogits is rounded to bf16 once, then dx += dl Wr
+// and the partials of dWr = dlᵀ x over token chunks are tcgen05 GEMMs with
+// fp32 accumulation (backward.cu), and the chunks are summed in order as on
+// the CUDA-core path. Used when d % 256 == 0.
+constexpr int TC_CHUNK_MIN = 512;  // tokens per dWr chunk (at most MOE_MAX_EXPERTS chunks)
+
+struct TcLayout {
+    int64_t Ep, Mp, chunk, G;
+    size_t off_one, off_chunks, dl, partial, total;
+};
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+inline TcLayout tc_layout(int64_t T, int64_t d, int64_t E) {
+    TcLayout L;
+    L.Ep = (E + 63) / 64 * 64;
+    L.Mp = (E + 127) / 128 * 128;
+    int64_t chunk = (T + MOE_MAX_EXPERTS - 1) / MOE_MAX_EXPERTS;
+    chunk = (chunk + 63) / 64 * 64;
+    L.chunk = chunk < TC_CHUNK_MIN ? TC_CHUNK_MIN : chunk;
+    L.G = T > 0 ? (T + L.chunk - 1) / L.chunk : 1;
+    L.off_one = 0;
+    L.off_chunks = 256;
+    L.dl = L.off_chunks + align256(sizeof(int32_t) * (size_t)(MOE_MAX_EXPERTS + 1));
+    L.partial = L.dl + align256(sizeof(uint16_t) * (size_t)T * (size_t)L.Ep);
+    L.total = L.partial + sizeof(float) * (size_t)L.G * (size_t)L.Mp * (size_t)d;
+    return L;
+}
+
+// dl[t, e] = bf16(dlogits[t, e]) for e < E, 0 for E <= e < Ep; the row-group
+// offsets {0, T} and the chunk offsets {0, chunk, 2 chunk, ..., T}.
+__global__ void __launch_bounds__(THREADS)
+    dl_to_bf16_kernel(const float* __restrict__ dlogits, int64_t T, int E, int Ep, int G,
+                      int chunk, __nv_bfloat16* __restrict__ dl, int32_t* __restrict__ off_one,
+                      int32_t* __restrict__ off_chunks) {
+    const int64_t n = T * Ep;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / Ep;
+        const int e = (int)(i - t * Ep);
+        dl[i] = __float2bfloat16_rn(e < E ? dlogits[t * E + e] : 0.f);
+    }
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) {
+            off_one[0] = 0;
+            off_one[1] = (int32_t)T;
+        }
+        for (int g = threadIdx.x; g <= G; g += blockDim.x)
+            off_chunks[g] = (int32_t)((int64_t)g * chunk < T ? (int64_t)g * chunk : T);
+    }
+}
+
+// dWr[e, c] = round(sum over chunks, in order, of partial[g][e][c]), partial
+// rows Mp apart per chunk.
+__global__ void __launch_bounds__(THREADS)
+    dwr_reduce_pitched_kernel(const float* __restrict__ partial, int G, int64_t Mp, int E,
+                              int64_t d, __nv_bfloat16* __restrict__ dWr) {
+    const int64_t n = (int64_t)E * d;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = i / d, c = i - e * d;
+        float v = 0.f;
+        for (int g = 0; g < G; ++g) v += partial[((int64_t)g * Mp + e) * d + c];
+        dWr[i] = __float2bfloat16_rn(v);
+    }
+}
+
 }  // namespace rb
+
+int router_linear_bwd_tc(const void* dl, int64_t Ep, const void* x, const void* Wr, int64_t T,
+                         int64_t d, int64_t E, const int32_t* off_one, const int32_t* off_chunks,
+                         int64_t G, int64_t Mp, void* dx, float* partial, cudaStream_t st);
+
 }  // namespace moe
 
 using namespace moe;
@@ -528,7 +604,9 @@ extern "C" int moe_router_bwd(const void* dOut, const void* Ye, const int32_t* s
 extern "C" size_t moe_router_linear_bwd_workspace_size(int64_t T, int64_t d, int64_t E) {
     if (T < 0 || d <= 0 || E < 1) return 0;
     const rb::DwrSplit s = rb::dwr_split(T, d, E);
-    return sizeof(float) * (size_t)s.chunks * (size_t)E * (size_t)d;
+    const size_t cuda_core = sizeof(float) * (size_t)s.chunks * (size_t)E * (size_t)d;
+    const size_t tc = rb::tc_layout(T, d, E).total;
+    return cuda_core > tc ? cuda_core : tc;
 }
 
 extern "C" int moe_router_linear_bwd(const float* dlogits, const void* x, const void* Wr,
@@ -545,6 +623,35 @@ extern "C" int moe_router_linear_bwd(const float* dlogits, const void* x, const 
                 workspace_bytes < moe_router_linear_bwd_workspace_size(T, d, E)))
         return MOE_ERR_INVALID;
     cudaStream_t st = as_stream(stream);
+    const bool tc = dtype == MOE_BF16 && T > 0 && d % 256 == 0 && d <= (1 << 24) &&
+                    T <= INT32_MAX - 2 * 128 && (!dx || (aligned16(dx) && aligned16(Wr))) &&
+                    (!dWr || aligned16(x)) && workspace &&
+                    (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0 &&
+                    workspace_bytes >= moe_router_linear_bwd_workspace_size(T, d, E);
+    if (tc) {
+        const rb::TcLayout L = rb::tc_layout(T, d, E);
+        char* w = static_cast<char*>(workspace);
+        int32_t* off_one = reinterpret_cast<int32_t*>(w + L.off_one);
+        int32_t* off_chunks = reinterpret_cast<int32_t*>(w + L.off_chunks);
+        __nv_bfloat16* dl = reinterpret_cast<__nv_bfloat16*>(w + L.dl);
+        float* part = reinterpret_cast<float*>(w + L.partial);
+        int64_t g = (T * L.Ep + rb::THREADS - 1) / rb::THREADS;
+        const int64_t cap = (int64_t)num_sms() * 8;
+        if (g > cap) g = cap;
+        rb::dl_to_bf16_kernel<<<(int)g, rb::THREADS, 0, st>>>(dlogits, T, (int)E, (int)L.Ep,
+                                                              (int)L.G, (int)L.chunk, dl,
+                                                              off_one, off_chunks);
+        int rc = router_linear_bwd_tc(dl, L.Ep, x, Wr, T, d, E, off_one, off_chunks, L.G, L.Mp,
+                                      dx, dWr ? part : nullptr, st);
+        if (rc != MOE_OK) return rc;
+        if (dWr) {
+            int64_t rg = (E * d + rb::THREADS - 1) / rb::THREADS;
+            if (rg > cap) rg = cap;
+            rb::dwr_reduce_pitched_kernel<<<(int)rg, rb::THREADS, 0, st>>>(
+                part, (int)L.G, L.Mp, (int)E, d, static_cast<__nv_bfloat16*>(dWr));
+        }
+        return launch_status();
+    }
     if (dx && T > 0) {
         const dim3 grid((unsigned)((T + rb::LT - 1) / rb::LT), (unsigned)((d + rb::LC - 1) / rb::LC));
         if (dtype == MOE_BF16)

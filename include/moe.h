@@ -562,7 +562,11 @@ MOE_API int moe_layer_bwd(const moe_layer_bwd_args* args, void* stream);
  *   dWr[e,:] = round(sum_t dlogits[t,e] x[t,:])             (dWr NULL: skip)
  *   fp32 sums (dWr over fixed token chunks, then the chunks in order, in the
  *   workspace of moe_router_linear_bwd_workspace_size bytes). x [T,d],
- *   Wr [E,d], dx, dWr in `dtype`; d % 4 == 0.
+ *   Wr [E,d], dx, dWr in `dtype`; d % 4 == 0. With bf16 data, d % 256 == 0
+ *   and a 256-byte aligned workspace (16-byte aligned x, Wr, dx) the two
+ *   products run on the tensor cores, as the bf16 router's backward: dlogits
+ *   is rounded to bf16 once and the exact products are summed in fp32;
+ *   otherwise on the CUDA cores in fp32 from the fp32 dlogits.
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_aux_loss_workspace_size(int64_t T, int64_t E);
 MOE_API int moe_aux_loss(const float* logits, const int32_t* counts, int64_t T, int64_t E,
