@@ -92,7 +92,7 @@ def test_route_skewed_with_empty_experts():
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("T,d,E,k", [(5, 128, 8, 2), (130, 256, 64, 8), (77, 128, 33, 3),
                                      (64, 384, 17, 4), (300, 256, 100, 6), (257, 128, 300, 8),
-                                     (129, 512, 128, 4)])
+                                     (129, 512, 128, 4), (3, 128, 1, 1), (1, 256, 512, 32)])
 def test_router_logits_match_oracle(dtype, T, d, E, k):
     """fp32: the oracle's fixed-order chains bit for bit; bf16 (tensor cores):
     within the fp32 summation bound; routing on the GPU's logits bit-exact."""
