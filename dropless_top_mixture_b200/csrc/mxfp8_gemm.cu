@@ -479,12 +479,13 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Activation scales from rows ([R, K/32] bytes) to the tile-packed layout
-// the GEMMs copy: for every row tile g of the expert-sorted rows (experts in
-// order, ceil(count/128) tiles each) and 128-element K slab s, a 512-byte
-// block holds the word (four K-block bytes) of tile row m at 16 (m % 32) +
-// 4 (m / 32); blocks ordered (tile, slab); tile rows past the expert's rows
-// hold 0. One thread per word; unpack is the inverse for the expert rows.
+// Activation scales between rows ([R, K/32] bytes) and the tile-packed
+// layout the GEMMs copy: for every row tile g of the expert-sorted rows
+// (experts in order, ceil(count/128) tiles each) and 128-element K slab s, a
+// 512-byte block holds the word (four K-block bytes) of tile row m at
+// 16 (m % 32) + 4 (m / 32); blocks ordered (tile, slab); tile rows past the
+// expert's rows hold 0. This kernel: one thread per word (unpack uses it;
+// pack uses act_scales_pack_kernel below).
 template <bool UNPACK>
 __global__ void __launch_bounds__(256)
     act_scales_kernel(const int32_t* __restrict__ offsets, int E, int R, int ks_count,
@@ -511,6 +512,50 @@ __global__ void __launch_bounds__(256)
             if (in) dst[rw] = src[w];
         } else {
             dst[w] = in ? src[rw] : 0u;
+        }
+    }
+}
+
+// Packing, one CTA per row tile at a time (grid stride): the tile's 128 rows
+// x up to 32 slab words are read row by row (coalesced), held slab-major in
+// shared memory, and written block by block (coalesced 512-byte blocks).
+// Row m of a slab sits at m + 8 (m / 32) in its shared row (pitch 153
+// words), so both the column writes and the block-order reads hit 32
+// different banks.
+constexpr int PK_SLABS = 32;
+constexpr int PK_PITCH = 153;
+
+__global__ void __launch_bounds__(256)
+    act_scales_pack_kernel(const int32_t* __restrict__ offsets, int E, int R, int ks_count,
+                           const uint32_t* __restrict__ src, uint32_t* __restrict__ dst,
+                           int* status) {
+    __shared__ int s_off[MOE_MAX_EXPERTS + 1];
+    __shared__ int s_toff[MOE_MAX_EXPERTS + 1];
+    __shared__ int s_bad;
+    __shared__ uint32_t tile[PK_SLABS * PK_PITCH];
+    if (!block_tile_table(offsets, E, R, s_off, s_toff, &s_bad, status)) return;
+    const int tid = threadIdx.x;
+    const int ntiles = s_toff[E];
+    for (int g = blockIdx.x; g < ntiles; g += gridDim.x) {
+        const int e = expert_of_tile(s_toff, E, g);
+        const int row0 = s_off[e] + (g - s_toff[e]) * BM;
+        const int rend = s_off[e + 1];
+        for (int sc = 0; sc < ks_count; sc += PK_SLABS) {
+            const int nsl = ks_count - sc < PK_SLABS ? ks_count - sc : PK_SLABS;
+            __syncthreads();  // the previous chunk's words have been written out
+            for (int i = tid; i < BM * nsl; i += blockDim.x) {
+                const int r = i / nsl, j = i - r * nsl;
+                const int row = row0 + r;
+                tile[j * PK_PITCH + r + 8 * (r >> 5)] =
+                    row < rend ? src[(int64_t)row * ks_count + sc + j] : 0u;
+            }
+            __syncthreads();
+            for (int i = tid; i < nsl * BM; i += blockDim.x) {
+                const int j = i >> 7, pos = i & 127;
+                const int m = (pos >> 2) + 32 * (pos & 3);
+                dst[((int64_t)g * ks_count + sc + j) * BM + pos] =
+                    tile[j * PK_PITCH + m + 8 * (m >> 5)];
+            }
         }
     }
 }
@@ -618,12 +663,16 @@ static int act_scales(const uint8_t* src, const int32_t* offsets, int64_t E, int
     if (g > cap) g = cap;
     const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
     uint32_t* d = reinterpret_cast<uint32_t*>(dst);
-    if (unpack)
+    if (unpack) {
         mxg::act_scales_kernel<true><<<(int)g, 256, 0, as_stream(stream)>>>(
             offsets, (int)E, (int)R, ks, words, s, d, status_ptr());
-    else
-        mxg::act_scales_kernel<false><<<(int)g, 256, 0, as_stream(stream)>>>(
-            offsets, (int)E, (int)R, ks, words, s, d, status_ptr());
+    } else {
+        int64_t tiles = R / mxg::BM + E;
+        const int64_t tcap = (int64_t)num_sms() * 4;
+        if (tiles > tcap) tiles = tcap;
+        mxg::act_scales_pack_kernel<<<(int)tiles, 256, 0, as_stream(stream)>>>(
+            offsets, (int)E, (int)R, ks, s, d, status_ptr());
+    }
     return launch_status();
 }
 

@@ -183,7 +183,8 @@ def test_pack_weight_scales_layout(E, d, F):
     assert np.array_equal(got2, np.concatenate(want2))
 
 
-@pytest.mark.parametrize("counts,K", [([0, 130, 1, 256, 5], 256), ([300], 128), ([7, 0, 0, 129], 512)])
+@pytest.mark.parametrize("counts,K", [([0, 130, 1, 256, 5], 256), ([300], 128), ([7, 0, 0, 129], 512),
+                                      ([200, 57], 4352), ([128, 256], 4096)])
 def test_act_scales_pack_layout_and_roundtrip(counts, K):
     """Tile-packed activation scales as the header defines them: row tiles
     of 128 per expert (ceil(count/128) each, numbered in expert order), one
