@@ -127,3 +127,39 @@ def test_route_full_size_workloads(name):
         lg = inp["logits"].numpy()
     _check_route(r, lg, w.k, w.E)
     assert moe.moe_get_status() == 0
+
+
+@pytest.mark.slow
+def test_bf16_router_routing_against_oracle_logits_full_size():
+    """OLMoE-shaped layer (T=16384, d=2048, E=64, top-8), router from x·Wr on
+    the tensor cores, against the oracle routing on its own fixed-order fp32
+    logits: the indices must agree on every token except where two adjacent
+    logits among the oracle's top k + 1 lie within twice the largest
+    difference between the token's two logit vectors (a near-tie the two
+    roundings may break differently); there the GPU's choices must still
+    reach no lower than that band."""
+    moe = _moe()
+    w = WORKLOADS["olmoe_1b7b"]
+    inp = make_inputs(w, "cpu", weights=False)
+    x, Wr = inp["x"], inp["Wr"]
+    r = moe.moe_route(w.k, x=x.cuda(), Wr=Wr.cuda(), keep_logits=True)
+    got_lg = router_logits_checked(r.logits.cpu().numpy(), x, Wr).astype(np.float64)
+    ref_lg = O.router_logits(x, Wr).astype(np.float64)
+    idx_ref, _, _ = O.route(ref_lg.astype(np.float32), w.k)
+    idx_gpu = r.idx.cpu().numpy()
+    # the two logit vectors of a token differ by at most delta (checked above
+    # against the derived bound), so their orders can only differ between
+    # logits closer than 2 delta
+    srt = np.sort(ref_lg, axis=1)[:, ::-1]
+    kth = srt[:, w.k - 1]
+    band = 2.0 * np.abs(got_lg - ref_lg).max(axis=1)
+    # a near-tie anywhere among the top k + 1 can reorder or swap indices
+    near_tie = (np.diff(-srt[:, :w.k + 1], axis=1) <= band[:, None]).any(axis=1)
+    same = (idx_gpu == idx_ref).all(axis=1)
+    assert np.all(same | near_tie), f"{int((~same & ~near_tie).sum())} tokens differ without a near-tie"
+    for t in np.nonzero(~same)[0]:
+        lo = kth[t] - band[t]
+        # every expert the GPU chose is at least as large as the band's bottom
+        assert np.all(ref_lg[t, idx_gpu[t]] >= lo), t
+    print(f"\nnear-ties (adjacent top-{w.k + 1} logits within 2 delta): {int(near_tie.sum())} of {w.T} tokens; "
+          f"tokens whose index list differs: {int((~same).sum())}")
