@@ -561,6 +561,97 @@ def moe_layer_bwd_sampled(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W
 
 
 # --------------------------------------------------------------------------
+# f3: backward of the MXFP8 layer
+#     [NEWS "三招拆分、三项优化、一个精度开关": the MXFP8 switch speeds up
+#      training through the FFN and the expert data movement; OF capability
+#      table and "MXFP8 分块量化": 32-element blocks sharing one scale;
+#      REL "主要功能": bf16 weight gradients]
+# --------------------------------------------------------------------------
+
+def _qdq_rows(m: np.ndarray, mode: str) -> np.ndarray:
+    """Quantise-dequantise along the last axis (blocks of 32), float64 out."""
+    q, st = mxfp8_quantize(np.asarray(m, np.float32), mode)
+    return mxfp8_dequantize_f32(q, st, mode).astype(np.float64)
+
+
+def _bf16(m: np.ndarray) -> np.ndarray:
+    """fp32 value rounded to bf16 (round-to-nearest-even), as float64."""
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(m, np.float32)))
+    return t.to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def mxfp8_layer_bwd(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W2,
+                    logits: np.ndarray, mode: str = "e8m0", exact: bool = False,
+                    return_ops: bool = False) -> Dict[str, np.ndarray]:
+    """Backward of the MXFP8 layer (gates held constant). Reading (the pages
+    leave the backward's precision open): the forward is mxfp8_layer's; the
+    two input-gradient GEMMs quantise each operand along its contraction
+    dimension,
+        dH  = Q_d(dYe) Q_d(W2_e)                 (W2_e [d,F] quantised along d)
+        dXe = Q_F([dA | dB]) Q_F([W1_e; W3_e])   ([W1_e; W3_e] along F)
+    with dYe = gate * dOut[t] and dA = dH B silu'(A), dB = dH silu(A); the
+    weight gradients use the forward's dequantised operands without a
+    further quantisation: dW1 = dA^T Xd, dW3 = dB^T Xd, dW2 = dYe^T Hd.
+
+    Values that decide a quantised code are taken in the precision the
+    layer stores them in: dYe, dH and the pre-activations A, B are bf16
+    tensors (rounded once from their fp32 value); dA, dB are formed from
+    those and quantised from their fp32 value. Everything else is float64.
+
+    exact=True replaces every quantise-dequantise and bf16 rounding by the
+    identity, which must give moe_layer_bwd's gradients (a wiring check).
+    return_ops=True adds, per expert, the operands as quantised."""
+    qdq = (lambda m: np.asarray(m, np.float64)) if exact else (lambda m: _qdq_rows(m, mode))
+    rnd = (lambda m: np.asarray(m, np.float64)) if exact else _bf16
+    E, F, d = W1.shape
+    idx, gate, _ = route(logits, k)
+    meta = routing_metadata(idx, E)
+    slot, offsets = meta["slot"], meta["offsets"]
+    xd = qdq(to64(x))                              # token rows along d
+    Xd = dispatch(xd, slot)
+    dYe = rnd(dispatch(to64(dOut), slot, gate=gate))
+    R = Xd.shape[0]
+    dXe = np.zeros((R, d))
+    dW1 = np.zeros((E, F, d)); dW3 = np.zeros((E, F, d)); dW2 = np.zeros((E, d, F))
+    ops = {}
+    for e in range(E):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 == r0:
+            continue
+        w1, w3, w2 = to64(W1[e]), to64(W3[e]), to64(W2[e])
+        X = Xd[r0:r1]
+        # forward (mxfp8_layer): weights along d, H along F from its fp32 value
+        a_ex = X @ qdq(w1).T
+        b_ex = X @ qdq(w3).T
+        Hd = qdq(silu(a_ex) * b_ex)
+        A, B = rnd(a_ex), rnd(b_ex)
+        # backward
+        dy = dYe[r0:r1]
+        dyd = qdq(dy)                               # along d
+        w2t = w2.T                                  # [F, d]: row f = column f of W2_e
+        w2td = qdq(w2t)                             # along d
+        dH = rnd(dyd @ w2td.T)
+        da = dH * B * dsilu(A)
+        db = dH * silu(A)
+        dab = np.concatenate([da, db], axis=1)      # [rows, 2F]
+        dabd = qdq(dab)                             # along F
+        w13t = np.concatenate([w1.T, w3.T], axis=1)  # [d, 2F]: row i = W1_e[:, i] | W3_e[:, i]
+        w13td = qdq(w13t)                           # along F
+        dXe[r0:r1] = dabd @ w13td.T
+        dW1[e] = da.T @ X
+        dW3[e] = db.T @ X
+        dW2[e] = dy.T @ Hd
+        if return_ops:
+            ops[e] = dict(dy=dy, dyd=dyd, w2t=w2t, w2td=w2td, dH=dH, A=A, B=B, da=da, db=db,
+                          dab=dab, dabd=dabd, w13t=w13t, w13td=w13td, Hd=Hd, X=X)
+    dx = combine(dXe, slot, None)
+    res = dict(dx=dx, dW1=dW1, dW3=dW3, dW2=dW2, dXe=dXe, dYe=dYe, idx=idx, gate=gate, **meta)
+    if return_ops:
+        res["ops"] = ops
+    return res
+
+
+# --------------------------------------------------------------------------
 # f2: router backward and the load-balancing auxiliary loss
 #     [HF §2 router (fp32 softmax, top-k, optional norm_topk_prob);
 #      HF §4 "负载均衡辅助损失": Switch-Transformer-style loss from the

@@ -555,3 +555,100 @@ def test_router_linear_grad_finite_differences():
     for r, c in itertools.product(range(E), range(d)):
         e = np.zeros((E, d)); e[r, c] = 1.0
         assert dWr[r, c] == pytest.approx(L(x, Wr + e) - L(x, Wr), rel=1e-9, abs=1e-12)
+
+
+# ---------------------------------------------------------------- MXFP8 backward
+
+def _torch_qdq_rows(m):
+    """Quantise-dequantise along the last axis written independently of the
+    oracle's codec: torch's float8_e4m3fn cast of the fp32 quotient, the
+    scale 2^e with e = ceil(log2(fp32(amax / 448))) found by frexp (1 for an
+    all-zero block)."""
+    v = torch.as_tensor(np.ascontiguousarray(np.asarray(m, np.float32)))
+    rows, K = v.shape
+    b = v.reshape(rows, K // 32, 32)
+    amax = b.abs().amax(dim=2)
+    s32 = amax / 448.0
+    mant, ex = torch.frexp(s32)
+    e = torch.where(mant == 0.5, ex - 1, ex).clamp(-127, 127)
+    e = torch.where(amax == 0, torch.zeros_like(e), e)
+    scale = torch.ldexp(torch.ones_like(s32), e)
+    q = (b / scale[..., None]).to(torch.float8_e4m3fn).to(torch.float32)
+    return (q * scale[..., None]).reshape(rows, K).double().numpy()
+
+
+def _bf16_of(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def _mx_problem(seed, T=40, d=64, F=64, E=4, k=2, skew=False):
+    g = torch.Generator().manual_seed(seed)
+
+    def mod(shape):
+        # skew=True: magnitudes spread over 2^-3..2^3 along both of the last
+        # two axes, so 32-blocks along one axis and along the other get
+        # different scales (iid data would give the same scale either way)
+        if not skew:
+            return 1.0
+        r = torch.exp2(torch.randint(-3, 4, (shape[-2], 1), generator=g).float())
+        c = torch.exp2(torch.randint(-3, 4, (1, shape[-1]), generator=g).float())
+        return r * c
+
+    x = (torch.randn(T, d, generator=g) * mod((T, d))).to(torch.bfloat16)
+    W1 = (torch.randn(E, F, d, generator=g) * 0.15 * mod((F, d))).to(torch.bfloat16)
+    W3 = (torch.randn(E, F, d, generator=g) * 0.15 * mod((F, d))).to(torch.bfloat16)
+    W2 = (torch.randn(E, d, F, generator=g) * 0.15 * mod((d, F))).to(torch.bfloat16)
+    dOut = (torch.randn(T, d, generator=g) * mod((T, d))).to(torch.bfloat16)
+    lg = torch.randn(T, E, generator=g).numpy().astype(np.float32)
+    lg[:, E - 1] -= 30.0  # one expert with zero rows
+    return x, W1, W3, W2, lg, dOut
+
+
+def test_mxfp8_backward_exact_mode_is_the_backward():
+    # every quantisation and bf16 rounding replaced by the identity: the
+    # wiring (operands, transposes, gates, combine) must give the plain
+    # backward, itself pinned against torch autograd above
+    x, W1, W3, W2, lg, dOut = _mx_problem(61)
+    r = O.mxfp8_layer_bwd(x, dOut, 2, W1, W3, W2, lg, exact=True)
+    b = O.moe_layer_bwd(x, dOut, 2, W1, W3, W2, lg)
+    for name in ("dx", "dW1", "dW3", "dW2"):
+        assert np.allclose(r[name], b[name], rtol=1e-12, atol=1e-12), name
+    assert np.all(r["dW1"][3] == 0) and np.all(r["dW2"][3] == 0)
+
+
+def test_mxfp8_backward_operands_quantised_along_contraction():
+    # each quantised operand equals an independent torch restatement of the
+    # codec applied along the stated axis to the stated source
+    x, W1, W3, W2, lg, dOut = _mx_problem(62, skew=True)
+    k = 2
+    with np.errstate(over="ignore"):  # exp(-a) of large negative pre-activations: silu -> -0
+        r = O.mxfp8_layer_bwd(x, dOut, k, W1, W3, W2, lg, return_ops=True)
+    idx, gate = r["idx"], r["gate"]
+    assert set(r["ops"]) == {0, 1, 2}
+    x64, d64 = x.double().numpy(), dOut.double().numpy()
+    for e, op in r["ops"].items():
+        toks, js = np.nonzero(idx == e)     # token-major: the expert's row order
+        # forward operand: the token rows of x quantised along d
+        assert np.array_equal(op["X"], _torch_qdq_rows(x64[toks]))
+        w1, w3, w2 = (t[e].double().numpy() for t in (W1, W3, W2))
+        A = _bf16_of(op["X"] @ _torch_qdq_rows(w1).T)
+        assert np.array_equal(op["A"], A)
+        # dYe rows: bf16 of the fp32 product gate * dOut
+        dy = _bf16_of((gate[toks, js][:, None] * d64[toks]).astype(np.float32))
+        assert np.array_equal(op["dy"], dy)
+        assert np.array_equal(op["dyd"], _torch_qdq_rows(dy))          # along d
+        assert np.array_equal(op["w2td"], _torch_qdq_rows(w2.T))       # W2_e along d
+        both = np.concatenate([w1.T, w3.T], axis=1)                    # [d, 2F]
+        assert np.array_equal(op["w13td"], _torch_qdq_rows(both))      # along F
+        dab = np.concatenate([op["da"], op["db"]], axis=1)
+        assert np.array_equal(op["dabd"], _torch_qdq_rows(dab))        # along F
+
+
+def test_mxfp8_backward_error_against_exact_backward():
+    # the format's error: a few percent of relative L2, never a gross mistake
+    x, W1, W3, W2, lg, dOut = _mx_problem(63, T=96, d=128, F=128)
+    r = O.mxfp8_layer_bwd(x, dOut, 2, W1, W3, W2, lg)
+    b = O.moe_layer_bwd(x, dOut, 2, W1, W3, W2, lg)
+    for name in ("dx", "dW1", "dW3", "dW2"):
+        rel = np.linalg.norm(r[name] - b[name]) / np.linalg.norm(b[name])
+        assert 1e-3 < rel < 0.15, (name, rel)
