@@ -201,6 +201,12 @@ def oracle_sample(w, inp_cpu, S: int, backward: bool = False):
         lg = inp_cpu["logits"][:S].numpy()
     if w.mxfp8:
         O.mxfp8_layer(x, w.k, inp_cpu["W1"], inp_cpu["W3"], inp_cpu["W2"], lg)
+        if backward:
+            # the float64 input gradient of the sample (the oracle's MXFP8
+            # backward re-quantises whole expert weights per call, minutes
+            # per expert on the host, so it is not what the sample times)
+            O.moe_layer_bwd_sampled(x, inp_cpu["dOut"][:S], w.k, inp_cpu["W1"], inp_cpu["W3"],
+                                    inp_cpu["W2"], lg, list(range(S)), [])
         return time.perf_counter() - t0
     idx, gate, _ = O.route(lg, w.k)
     O.routing_metadata(idx, w.E)
@@ -219,7 +225,9 @@ def cpu_baseline(w, inp_cpu, target_s: float = 12.0, backward: bool = False):
         dt = oracle_sample(w, inp_cpu, S, backward)
     what = ("router logits, top-k, routing metadata and the per-token "
             + ("MXFP8 SwiGLU mixture" if w.mxfp8 else "SwiGLU mixture")
-            + (" plus the input gradient of those tokens (no weight gradients)" if backward else "")
+            + ((" plus the float64 input gradient of those tokens (no weight gradients)"
+                if w.mxfp8 else " plus the input gradient of those tokens (no weight gradients)")
+               if backward else "")
             + " in float64")
     return {"value": S / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"first {S} of {w.T} tokens of {w.name}: {what} ({dt:.1f} s)"}
@@ -305,14 +313,69 @@ def _steps(moe, w, inp, dev, backward):
             moe.moe_dispatch_mxfp8(x, rt.slot, Xq, Xs)
             moe.mxfp8_pack_act_scales(Xs, rt.offsets, E, Xsp)
 
+        A = torch.empty((R, F), dtype=torch.bfloat16, device=dev) if backward else None
+        B = torch.empty((R, F), dtype=torch.bfloat16, device=dev) if backward else None
         fns = [("route", route),
                ("dispatch", mx_dispatch),
                ("gate_up", lambda: moe.moe_grouped_gate_up_mxfp8(Xq, Xsp, mw, rt.offsets, Hq, Hsp,
-                                                                 packed=True)),
+                                                                 packed=True, A=A, B=B)),
                ("down", lambda: moe.moe_grouped_down_mxfp8(Hq, Hsp, mw, rt.offsets, Ye,
                                                            packed=True)),
                ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
         sx, sw, sh = 1 + 1 / 32, 1 + 1 / 32, 1 + 1 / 32
+        if backward:
+            # the backward weights, re-quantised along F (W1, W3) and d (W2):
+            # once per weight update, outside the timed region like mw
+            wb = moe.mxfp8_quantize_weights_bwd(W1, W3, W2)
+            dOut = inp["dOut"]
+            u8 = dict(dtype=torch.uint8, device=dev)
+            bf = dict(dtype=torch.bfloat16, device=dev)
+            dYe = torch.empty((R, d), **bf)
+            dYq, dYs = torch.empty((R, d), **u8), torch.empty((R, d // 32), **u8)
+            dYsp = torch.empty(moe.lib.mxfp8_act_scales_packed_size(E, R, d), **u8)
+            dH = torch.empty((R, F), **bf)
+            dA, dB = torch.empty((R, F), **bf), torch.empty((R, F), **bf)
+            dq, ds = torch.empty((R, 2 * F), **u8), torch.empty((R, 2 * F // 32), **u8)
+            dsp = torch.empty(moe.lib.mxfp8_act_scales_packed_size(E, R, 2 * F), **u8)
+            dXe, Xd = torch.empty((R, d), **bf), torch.empty((R, d), **bf)
+            Hs, Hd = torch.empty((R, F // 32), **u8), torch.empty((R, F), **bf)
+            dx = torch.empty((T, d), **bf)
+            dW = (torch.empty((E, F, d), **bf), torch.empty((E, F, d), **bf),
+                  torch.empty((E, d, F), **bf))
+
+            def bwd_dispatch():
+                moe.moe_dispatch(dOut, rt.slot, gate=rt.gate, out=dYe)
+                moe.mxfp8_quantize(dYe, q=dYq, scales=dYs)
+                moe.mxfp8_pack_act_scales(dYs, rt.offsets, E, dYsp)
+
+            def bwd_swiglu():
+                moe.moe_swiglu_bwd_mxfp8(dH, A, B, dA, dB, dq, ds)
+                moe.mxfp8_pack_act_scales(ds, rt.offsets, E, dsp)
+
+            def bwd_dequant():
+                moe.mxfp8_dequantize(Xq, Xs, out=Xd)
+                moe.mxfp8_unpack_act_scales(Hsp, rt.offsets, E, R, F, Hs)
+                moe.mxfp8_dequantize(Hq, Hs, out=Hd)
+
+            aux = torch.empty(1, dtype=torch.float32, device=dev)
+            aux_ws = torch.empty(moe.lib.moe_aux_loss_workspace_size(T, E), **u8)
+            rg = moe.RouterGrads(dgate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                                 dlogits=torch.empty((T, E), dtype=torch.float32, device=dev))
+            fns += [("bwd_dispatch", bwd_dispatch),
+                    ("bwd_dH", lambda: moe.moe_grouped_mxfp8_gemm(dYq, dYsp, wb.W2tq, wb.Ps2t,
+                                                                  rt.offsets, dH)),
+                    ("bwd_swiglu", bwd_swiglu),
+                    ("bwd_dX", lambda: moe.moe_grouped_mxfp8_gemm(dq, dsp, wb.W13tq, wb.Ps13t,
+                                                                  rt.offsets, dXe)),
+                    ("bwd_combine", lambda: moe.moe_combine(dXe, rt.slot, None, out=dx)),
+                    ("bwd_dequant", bwd_dequant),
+                    ("bwd_dW", lambda: moe.moe_grouped_swiglu_wgrad(Xd, dA, dB, dYe, Hd,
+                                                                    rt.offsets, out=dW)),
+                    ("aux_loss", lambda: moe.moe_aux_loss(logits, rt.counts, out=aux,
+                                                          workspace=aux_ws)),
+                    ("router_bwd", lambda: moe.moe_router_bwd(
+                        dOut, Ye, rt.slot, rt.idx, logits, rt.counts, aux_coef=0.01,
+                        dgate=rg.dgate, dlogits=rg.dlogits))]
     else:
         Xe = torch.empty((R, d), dtype=dt, device=dev)
         H = torch.empty((R, F), dtype=dt, device=dev)
@@ -385,7 +448,19 @@ def _steps(moe, w, inp, dev, backward):
         "down": (2.0 * R * d * F, R * F * sh + wbytes + R * d * 2),
         "combine": (0.0, R * d * 2 + T * d * 2 + R * 8),
     }
-    if backward:
+    if backward and w.mxfp8:
+        q8 = 1 + 1 / 32  # an E4M3 code and its share of a scale byte
+        wq = e_act * F * d * q8
+        work["bwd_dispatch"] = (0.0, T * d * 2 + R * d * 2 + R * 8 + R * d * 2 + R * d * q8)
+        work["bwd_dH"] = (2.0 * R * d * F, R * d * q8 + wq + R * F * 2)
+        work["bwd_swiglu"] = (0.0, 3 * R * F * 2 + 2 * R * F * 2 + 2 * R * F * q8)
+        work["bwd_dX"] = (4.0 * R * d * F, 2 * R * F * q8 + 2 * wq + R * d * 2)
+        work["bwd_combine"] = (0.0, R * d * 2 + T * d * 2 + R * 4)
+        work["bwd_dequant"] = (0.0, R * (d + F) * q8 + R * (d + F) * 2)
+        work["bwd_dW"] = (6.0 * R * d * F, 3 * e_act * F * d * 2 + R * (3 * d + 3 * F) * 2)
+        work["aux_loss"] = (0.0, T * E * 4 + E * 4)
+        work["router_bwd"] = (0.0, T * d * 2 + R * d * 2 + 2 * T * E * 4 + 3 * R * 4)
+    elif backward:
         work["bwd_dispatch"] = (0.0, T * d * es + R * d * es + R * 8)
         work["bwd_gemms"] = (12.0 * R * d * F, 6 * wbytes + R * (5 * d + 5 * F) * es)
         work["bwd_combine"] = (0.0, R * d * es + T * d * es + R * 4)
@@ -394,8 +469,13 @@ def _steps(moe, w, inp, dev, backward):
         # dx += dlogits Wr and dWr = dlogits^T x: two T x E x d products
         work["router_linear_bwd"] = (4.0 * T * E * d, T * E * 4 + E * d * es + 3 * T * d * es
                                      + E * d * es)
+    # backward: bf16 dispatch 1 + GEMMs 5 + combine 1; MXFP8 dispatch,
+    # quantise, pack 3 + dH 1 + SwiGLU, pack 2 + dX 1 + combine 1 +
+    # dequantise, unpack, dequantise 3 + dW 3; then the aux loss 2 and the
+    # router backward 1 (+3 for the router GEMM backward)
+    bwd_kernels = (14 if w.mxfp8 else 7) + 2 + 1 + (3 if use_router else 0)
     kernels = ((4 if use_router else 3) + (5 if w.mxfp8 else 4)
-               + ((7 + 2 + 1 + (3 if use_router else 0)) if backward else 0))
+               + (bwd_kernels if backward else 0))
     return [n for n, _ in fns], step, kernels, work, e_act
 
 
@@ -413,8 +493,8 @@ def run_ours(args):
         w = w.scaled(name=f"{w.name}/shrink{args.shrink}", T=max(1, w.T // args.shrink),
                      E=max(w.k, w.E // args.shrink))
     backward = bool(args.backward)
-    if backward and (w.mxfp8 or w.dtype != "bf16"):
-        raise SystemExit("--backward runs on the bf16 workloads")
+    if backward and not w.mxfp8 and w.dtype != "bf16":
+        raise SystemExit("--backward runs on the bf16 and MXFP8 workloads")
     if backward and not w.backward:
         w = w.scaled(name=w.name, backward=True)  # adds the upstream gradient dOut
     inp = make_inputs(w, dev)
@@ -537,11 +617,15 @@ def run_ours(args):
     gemm_parts = [p for p in parts if work[p][0] > 0]
     dom = max(gemm_parts, key=lambda p: per[p])
     flop, byts = work[dom]
-    ridge = peak_tf * 1e12 / (hbm * 1e9)
+    roof_tf, roof_src = peak_tf, tf_src
+    if dom == "bwd_dW":  # bf16 GEMMs inside the MXFP8 backward
+        roof_tf = bf16_tf
+        roof_src = f"{peak_src} bf16 sustained (kernel timed inside a long step)"
+    ridge = roof_tf * 1e12 / (hbm * 1e9)
     if flop / byts >= ridge:
-        roof = {"bound": "tensor", "achieved": rates[dom]["tflops"], "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": rates[dom]["tflops"] / peak_tf, "peak_source": tf_src,
-                "algorithmic_per_launch": f"{flop:.4g} flop"}
+        roof = {"bound": "tensor", "achieved": rates[dom]["tflops"], "peak": roof_tf,
+                "unit": "TFLOP/s", "frac": rates[dom]["tflops"] / roof_tf,
+                "peak_source": roof_src, "algorithmic_per_launch": f"{flop:.4g} flop"}
     else:
         roof = {"bound": "hbm", "achieved": rates[dom]["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": rates[dom]["gbs"] / hbm, "peak_source": f"{peak_src} HBM copy bandwidth",
@@ -549,6 +633,9 @@ def run_ours(args):
     roof["kernel"] = {"gate_up": "grouped gate_up GEMM + SwiGLU (tcgen05)",
                       "down": "grouped down GEMM (tcgen05)",
                       "bwd_gemms": "grouped backward GEMMs dH/dX/dW (tcgen05)",
+                      "bwd_dH": "MXFP8 grouped dH GEMM (tcgen05 block-scaled)",
+                      "bwd_dX": "MXFP8 grouped dX GEMM (tcgen05 block-scaled)",
+                      "bwd_dW": "bf16 weight-gradient GEMMs (tcgen05)",
                       "router_linear_bwd": "router GEMM backward (CUDA cores)"}[dom]
     roof["ridge_flop_per_byte"] = ridge
     roof["traffic"] = recorded_traffic(dom, w.name)
@@ -611,7 +698,21 @@ def _e2e(moe, w, inp, dev, world, args, backward):
     if args.e2e_chunks <= 0:
         wbytes = 3 * w.E * w.F * w.d * (1 if w.mxfp8 else x.element_size())
         args.e2e_chunks = moe.choose_chunks(T, w.d, x.element_size(), wbytes)
-    if w.mxfp8:
+    if w.mxfp8 and backward:
+        dO_h = inp["dOut"].cpu().pin_memory()
+        dO_d = torch.empty_like(inp["dOut"])
+        h2d += dO_d.numel() * dO_d.element_size()
+        mw = moe.mxfp8_quantize_weights(W1, W3, W2)
+        wb = moe.mxfp8_quantize_weights_bwd(W1, W3, W2)
+        lo = moe.moe_layer_fwd_mxfp8(x, k, mw, logits=logits, Wr=Wr, save=True)
+        gr = moe.moe_layer_bwd_mxfp8(lo, inp["dOut"], k, wb)
+        res = gr.dx
+
+        def run():
+            dO_d.copy_(dO_h, non_blocking=True)
+            moe.moe_layer_fwd_mxfp8(x_d, k, mw, logits=lg_d, Wr=Wr, out=lo, save=True)
+            moe.moe_layer_bwd_mxfp8(lo, dO_d, k, wb, out=gr)
+    elif w.mxfp8:
         # token slices whose copies overlap the compute (moe_layer_fwd_mxfp8_host)
         mw = moe.mxfp8_quantize_weights(W1, W3, W2)
         hlm = moe.HostLayerMxfp8(T, w.d, w.E, w.F, k, dev, logits_given=logits is not None,
@@ -636,7 +737,7 @@ def _e2e(moe, w, inp, dev, world, args, backward):
         res = hl.res.out
     res_h = torch.empty(res.shape, dtype=res.dtype).pin_memory()
 
-    if w.mxfp8:
+    if w.mxfp8 and not backward:
         def e2e_step():
             hlm(x_h, mw, logits_host=lg_h, Wr=Wr, out_host=res_h)
     elif not backward:

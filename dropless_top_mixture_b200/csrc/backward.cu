@@ -564,6 +564,37 @@ int router_linear_bwd_tc(const void* dl, int64_t Ep, const void* x, const void* 
     return MOE_OK;
 }
 
+
+// Weight gradients of the grouped SwiGLU FFN from bf16 rows: dW1_e = dAᵀ Xe,
+// dW3_e = dBᵀ Xe, dW2_e = dYeᵀ H over each expert's rows (every expert's
+// tiles run, so an expert with no rows gets zeros). Shared by the bf16 and
+// the MXFP8 backward (there Xe and H are the dequantised forward operands).
+int swiglu_wgrad(const void* Xe, const void* dA, const void* dB, const void* dYe, const void* H,
+                 const int32_t* offsets, int64_t E, int64_t R, int64_t d, int64_t F, void* dW1,
+                 void* dW3, void* dW2, cudaStream_t st) {
+    using namespace tc;
+    CUtensorMap gA, gB, gX, gY, gH;
+    const int64_t Rm = R > 0 ? R : 1;  // a map needs a non-empty extent; no rows are read when R == 0
+    if (!make_map_2d(&gA, dA, bwd::BF16, 2, F, Rm, 64) ||
+        !make_map_2d(&gB, dB, bwd::BF16, 2, F, Rm, 64) ||
+        !make_map_2d(&gX, Xe, bwd::BF16, 2, d, Rm, 64) ||
+        !make_map_2d(&gY, dYe, bwd::BF16, 2, d, Rm, 64) ||
+        !make_map_2d(&gH, H, bwd::BF16, 2, F, Rm, 64))
+        return MOE_ERR_CUDA;
+    CUtensorMap o1, o3, o2;  // the gradients as [E*M, N] for the TMA stores
+    if (!make_map_2d(&o1, dW1, bwd::BF16, 2, d, E * F, 32) ||
+        !make_map_2d(&o3, dW3, bwd::BF16, 2, d, E * F, 32) ||
+        !make_map_2d(&o2, dW2, bwd::BF16, 2, F, E * d, 32))
+        return MOE_ERR_CUDA;
+    int rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, o1, offsets, E, R, 0, F, d, dW1, nullptr, d,
+                                  nullptr, nullptr, st);
+    if (rc != MOE_OK) return rc;
+    rc = bwd::launch<bwd::DW>(gB, gB, gX, gX, o3, offsets, E, R, 0, F, d, dW3, nullptr, d, nullptr,
+                              nullptr, st);
+    if (rc != MOE_OK) return rc;
+    return bwd::launch<bwd::DW>(gY, gY, gH, gH, o2, offsets, E, R, 0, d, F, dW2, nullptr, F,
+                                nullptr, nullptr, st);
+}
 }  // namespace moe
 
 using namespace moe;
@@ -609,25 +640,20 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
         if (rc != MOE_OK) return rc;
     }
     // weight gradients (every expert's tile runs, so empty experts get zeros)
-    CUtensorMap gA, gB, gX, gY, gH;
-    const int64_t Rm = R > 0 ? R : 1;  // a map needs a non-empty extent; no rows are read when R == 0
-    if (!make_map_2d(&gA, dA, bwd::BF16, 2, F, Rm, 64) ||
-        !make_map_2d(&gB, dB, bwd::BF16, 2, F, Rm, 64) ||
-        !make_map_2d(&gX, Xe, bwd::BF16, 2, d, Rm, 64) ||
-        !make_map_2d(&gY, dYe, bwd::BF16, 2, d, Rm, 64) ||
-        !make_map_2d(&gH, H, bwd::BF16, 2, F, Rm, 64))
-        return MOE_ERR_CUDA;
-    CUtensorMap o1, o3, o2;  // the gradients as [E*M, N] for the TMA stores
-    if (!make_map_2d(&o1, dW1, bwd::BF16, 2, d, E * F, 32) ||
-        !make_map_2d(&o3, dW3, bwd::BF16, 2, d, E * F, 32) ||
-        !make_map_2d(&o2, dW2, bwd::BF16, 2, F, E * d, 32))
-        return MOE_ERR_CUDA;
-    rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, o1, offsets, E, R, 0, F, d, dW1, nullptr, d, nullptr,
-                              nullptr, st);
-    if (rc != MOE_OK) return rc;
-    rc = bwd::launch<bwd::DW>(gB, gB, gX, gX, o3, offsets, E, R, 0, F, d, dW3, nullptr, d, nullptr,
-                              nullptr, st);
-    if (rc != MOE_OK) return rc;
-    return bwd::launch<bwd::DW>(gY, gY, gH, gH, o2, offsets, E, R, 0, d, F, dW2, nullptr, F,
-                                nullptr, nullptr, st);
+    return swiglu_wgrad(Xe, dA, dB, dYe, H, offsets, E, R, d, F, dW1, dW3, dW2, st);
+}
+
+extern "C" int moe_grouped_swiglu_wgrad(const void* Xe, const void* dA, const void* dB,
+                                        const void* dYe, const void* H, const int32_t* offsets,
+                                        int64_t E, int64_t R, int64_t d, int64_t F, int dtype,
+                                        void* dW1, void* dW3, void* dW2, void* stream) {
+    if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
+    if (dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (d % 256 != 0 || F % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if (R > INT32_MAX - 2 * bwd::BM || d > (1 << 24) || F > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+    const void* ptrs[] = {Xe, dA, dB, dYe, H, dW1, dW3, dW2};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID;
+    if (!offsets) return MOE_ERR_INVALID;
+    return swiglu_wgrad(Xe, dA, dB, dYe, H, offsets, E, R, d, F, dW1, dW3, dW2, as_stream(stream));
 }

@@ -248,6 +248,8 @@ extern "C" int moe_layer_fwd_mxfp8_host(const moe_layer_mxfp8_args* a, const voi
     if (stream == stream_h2d || stream == stream_d2h || stream_h2d == stream_d2h)
         return MOE_ERR_INVALID;
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->save_Xq || a->save_Xs || a->save_Hq || a->save_Hsp || a->save_A || a->save_B)
+        return MOE_ERR_INVALID;  // the slices would overwrite one another's rows
     if (a->T == 0) return moe_layer_fwd_mxfp8(a, stream);
     const int64_t k = a->k;
     return layer::host_pipeline(
@@ -373,6 +375,19 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     const int logits_given = a->logits != nullptr;
     layer::CarveMx c = layer::carve_mx(a->workspace, a->T, a->d, a->E, a->F, a->k, logits_given);
     if (a->workspace_bytes < c.total) return MOE_ERR_INVALID;
+    const bool save = a->save_Xq != nullptr;
+    if (save) {
+        // the rows the backward reads go to the caller's buffers
+        const void* sv[] = {a->save_Xs, a->save_Hq, a->save_Hsp, a->save_A, a->save_B};
+        for (const void* q : sv)
+            if (!q) return MOE_ERR_INVALID;
+        c.Xq = a->save_Xq;
+        c.Xs = a->save_Xs;
+        c.Hq = a->save_Hq;
+        c.Hsp = a->save_Hsp;
+    } else if (a->save_Xs || a->save_Hq || a->save_Hsp || a->save_A || a->save_B) {
+        return MOE_ERR_INVALID;
+    }
     int rc = moe_route(a->logits, a->x, a->Wr, MOE_BF16, a->T, a->d, a->E, a->k, a->renorm,
                        nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
                        c.route_ws, c.route_bytes, stream);
@@ -382,8 +397,10 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     if (rc != MOE_OK) return rc;
     rc = mxfp8_pack_act_scales(c.Xs, a->offsets, a->E, R, a->d, c.Xsp, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_gate_up_mxfp8(c.Xq, c.Xsp, a->W1q, a->W3q, a->Ps13, a->w13_expert_stride,
-                                   a->offsets, a->E, R, a->d, a->F, c.Hq, c.Hsp, stream);
+    rc = moe_grouped_gate_up_mxfp8_save(c.Xq, c.Xsp, a->W1q, a->W3q, a->Ps13,
+                                        a->w13_expert_stride, a->offsets, a->E, R, a->d, a->F,
+                                        c.Hq, c.Hsp, save ? a->save_A : nullptr,
+                                        save ? a->save_B : nullptr, stream);
     if (rc != MOE_OK) return rc;
     rc = moe_grouped_down_mxfp8(c.Hq, c.Hsp, a->W2q, a->Ps2, a->w2_expert_stride, a->offsets, a->E,
                                 R, a->d, a->F, c.Ye, stream);

@@ -170,7 +170,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                    const __grid_constant__ CUtensorMap tmB1, const uint8_t* __restrict__ sfAp,
                    const uint8_t* __restrict__ sfBp, const int32_t* __restrict__ offsets, int E, int R,
                    int K, int N, uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sp,
-                   __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status) {
+                   __nv_bfloat16* __restrict__ out_bf16, int64_t ldo, int* status,
+                   __nv_bfloat16* __restrict__ save_a, __nv_bfloat16* __restrict__ save_b) {
     constexpr int OUT_N = SWIGLU ? MMA_N / 2 : MMA_N;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -360,6 +361,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                         continue;
                     }
                     float v[32];
+                    if (save_a != nullptr) {
+                        // pre-activations kept (bf16) for the backward pass
+                        uint4* da = reinterpret_cast<uint4*>(save_a + gr * ldo + col);
+                        uint4* db = reinterpret_cast<uint4*>(save_b + gr * ldo + col);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(acc[32 * c + 8 * u + j]);
+                            da[u] = pack8(v);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                v[j] = __uint_as_float(acc[64 + 32 * c + 8 * u + j]);
+                            db[u] = pack8(v);
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float g = __uint_as_float(acc[32 * c + j]);
@@ -563,7 +579,8 @@ __global__ void __launch_bounds__(256)
 template <bool SWIGLU>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const uint8_t* sfA, const uint8_t* sfBp, const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, uint8_t* oq,
-                  uint8_t* os, __nv_bfloat16* ob, int64_t ldo, cudaStream_t st) {
+                  uint8_t* os, __nv_bfloat16* ob, int64_t ldo, cudaStream_t st,
+                  void* save_a = nullptr, void* save_b = nullptr) {
     auto kern = mx_gemm_kernel<SWIGLU>;
     static bool attr_done[64] = {false};
     int dev = 0;
@@ -580,7 +597,9 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     const int grid = (int)(max_tiles < sms ? max_tiles : sms);
     if (grid <= 0) return MOE_OK;
     kern<<<grid, THREADS, SMEM_BYTES, st>>>(a, b0, b1, sfA, sfBp, offsets, (int)E,
-                                           (int)R, (int)K, (int)N, oq, os, ob, ldo, status_ptr());
+                                           (int)R, (int)K, (int)N, oq, os, ob, ldo, status_ptr(),
+                                           static_cast<__nv_bfloat16*>(save_a),
+                                           static_cast<__nv_bfloat16*>(save_b));
     return launch_status();
 }
 
@@ -691,15 +710,18 @@ extern "C" int mxfp8_unpack_act_scales(const uint8_t* Sp, const int32_t* offsets
     return act_scales(Sp, offsets, E, R, K, S, stream, true);
 }
 
-extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
-                                         const uint8_t* W3q, const uint8_t* Ps13,
-                                         int64_t w13_expert_stride, const int32_t* offsets,
-                                         int64_t E, int64_t R, int64_t d, int64_t F, uint8_t* Hq,
-                                         uint8_t* Hs, void* stream) {
+extern "C" int moe_grouped_gate_up_mxfp8_save(const uint8_t* Xq, const uint8_t* Xs,
+                                              const uint8_t* W1q, const uint8_t* W3q,
+                                              const uint8_t* Ps13, int64_t w13_expert_stride,
+                                              const int32_t* offsets, int64_t E, int64_t R,
+                                              int64_t d, int64_t F, uint8_t* Hq, uint8_t* Hs,
+                                              void* A_out, void* B_out, void* stream) {
     int rc = mx_check(Xq, Xs, W1q, Ps13, offsets, E, R, d, F);
     if (rc != MOE_OK) return rc;
     if (!W3q || !Hq || !Hs || !aligned16(W3q) || !aligned16(Hq) || !aligned16(Hs))
         return MOE_ERR_INVALID;
+    if ((A_out == nullptr) != (B_out == nullptr)) return MOE_ERR_INVALID;
+    if (A_out && (!aligned16(A_out) || !aligned16(B_out))) return MOE_ERR_INVALID;
     if ((w13_expert_stride < F * d && E > 1) || w13_expert_stride % 128 != 0) return MOE_ERR_INVALID;
     if (R == 0) return MOE_OK;
     CUtensorMap a, b0, b1;
@@ -708,7 +730,16 @@ extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, c
         !make_map_3d(&b1, W3q, mxg::U8, 1, d, F, E, w13_expert_stride, mxg::MMA_N / 2))
         return MOE_ERR_CUDA;
     return mxg::launch<true>(a, b0, b1, Xs, Ps13, offsets, E, R, d, F, Hq, Hs, nullptr, F,
-                             as_stream(stream));
+                             as_stream(stream), A_out, B_out);
+}
+
+extern "C" int moe_grouped_gate_up_mxfp8(const uint8_t* Xq, const uint8_t* Xs, const uint8_t* W1q,
+                                         const uint8_t* W3q, const uint8_t* Ps13,
+                                         int64_t w13_expert_stride, const int32_t* offsets,
+                                         int64_t E, int64_t R, int64_t d, int64_t F, uint8_t* Hq,
+                                         uint8_t* Hs, void* stream) {
+    return moe_grouped_gate_up_mxfp8_save(Xq, Xs, W1q, W3q, Ps13, w13_expert_stride, offsets, E,
+                                          R, d, F, Hq, Hs, nullptr, nullptr, stream);
 }
 
 extern "C" int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const uint8_t* W2q,

@@ -89,6 +89,21 @@ class LayerMxArgs(ctypes.Structure):
         ("w13_expert_stride", _i64), ("w2_expert_stride", _i64),
         ("out", _p), ("idx", _p), ("gate", _p), ("counts", _p), ("offsets", _p), ("slot", _p),
         ("workspace", _p), ("workspace_bytes", _sz),
+        ("save_Xq", _p), ("save_Xs", _p), ("save_Hq", _p), ("save_Hsp", _p), ("save_A", _p),
+        ("save_B", _p),
+    ]
+
+
+class LayerBwdMxArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", _i64), ("d", _i64), ("E", _i64), ("F", _i64),
+        ("k", ctypes.c_int32), ("reserved0", ctypes.c_int32), ("reserved1", ctypes.c_int32),
+        ("reserved2", ctypes.c_int32),
+        ("slot", _p), ("gate", _p), ("offsets", _p),
+        ("Xq", _p), ("Xs", _p), ("Hq", _p), ("Hsp", _p), ("A", _p), ("B", _p),
+        ("W13tq", _p), ("Ps13t", _p), ("W2tq", _p), ("Ps2t", _p),
+        ("dOut", _p), ("dx", _p), ("dW1", _p), ("dW3", _p), ("dW2", _p),
+        ("workspace", _p), ("workspace_bytes", _sz),
     ]
 
 
@@ -122,6 +137,15 @@ _SIGS = {
                                          _p, _p, _p]),
     "moe_grouped_down_mxfp8": (_i32, [_p, _p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _p, _p]),
     "moe_layer_mxfp8_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
+    "moe_grouped_gate_up_mxfp8_save": (_i32, [_p, _p, _p, _p, _p, _i64, _p, _i64, _i64, _i64,
+                                              _i64, _p, _p, _p, _p, _p]),
+    "mxfp8_quantize_weights_bwd": (_i32, [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _p, _p, _p,
+                                          _p, _p]),
+    "moe_swiglu_bwd_mxfp8": (_i32, [_p, _p, _p, _i64, _i64, _p, _p, _p, _p, _p]),
+    "moe_layer_bwd_mxfp8_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i32]),
+    "moe_layer_bwd_mxfp8": (_i32, [ctypes.POINTER(LayerBwdMxArgs), _p]),
+    "moe_grouped_swiglu_wgrad": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32, _p,
+                                        _p, _p, _p]),
     "moe_layer_fwd_mxfp8": (_i32, [ctypes.POINTER(LayerMxArgs), _p]),
     "moe_layer_fwd_mxfp8_host": (_i32, [ctypes.POINTER(LayerMxArgs), _p, _p, _p, _i32, _p, _p,
                                         _p]),
@@ -440,6 +464,10 @@ class LayerOut:
     Ye: Optional[torch.Tensor] = None   # expert outputs, for the router backward
     logits: Optional[torch.Tensor] = None  # fp32 logits (computed or given)
     renorm: bool = False
+    Xq: Optional[torch.Tensor] = None   # MXFP8 forward, save=True: codes and scales
+    Xs: Optional[torch.Tensor] = None   # the backward reads (row-layout Xs,
+    Hq: Optional[torch.Tensor] = None   # tile-packed Hsp)
+    Hsp: Optional[torch.Tensor] = None
 
 
 def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool = False,
@@ -776,10 +804,11 @@ def mxfp8_unpack_act_scales(Sp, offsets, E: int, R: int, K: int, S=None):
 
 
 def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None, *,
-                              packed: bool = False):
+                              packed: bool = False, A=None, B=None):
     """H = quantised SwiGLU of the block-scaled FP8 gate/up GEMMs. With
     packed=False, Xs and the returned Hs are in row layout (packed and
-    unpacked here); with packed=True both are in the tile-packed layout."""
+    unpacked here); with packed=True both are in the tile-packed layout.
+    A, B ([R,F] bf16, both or neither) receive the pre-activations."""
     _need(Xq, "Xq"); _need(Xs, "Xs"); _need(offsets, "offsets")
     E, F, d = w.W1q.shape
     R = Xq.shape[0]
@@ -790,9 +819,9 @@ def moe_grouped_gate_up_mxfp8(Xq, Xs, w: MxWeights, offsets, Hq=None, Hs=None, *
     Hsp = Hs if (packed and Hs is not None) else torch.empty(
         lib.mxfp8_act_scales_packed_size(E, R, F), dtype=torch.uint8, device=dev)
     w = _packed(w)
-    rc = lib.moe_grouped_gate_up_mxfp8(_ptr(Xq), _ptr(Xsp), _ptr(w.W1q), _ptr(w.W3q), _ptr(w.Ps13),
-                                       w.W1q.stride(0), _ptr(offsets), E, R, d, F, _ptr(Hq),
-                                       _ptr(Hsp), _stream(Xq))
+    rc = lib.moe_grouped_gate_up_mxfp8_save(_ptr(Xq), _ptr(Xsp), _ptr(w.W1q), _ptr(w.W3q),
+                                            _ptr(w.Ps13), w.W1q.stride(0), _ptr(offsets), E, R, d,
+                                            F, _ptr(Hq), _ptr(Hsp), _ptr(A), _ptr(B), _stream(Xq))
     _check("moe_grouped_gate_up_mxfp8", rc)
     if packed:
         return Hq, Hsp
@@ -814,8 +843,49 @@ def moe_grouped_down_mxfp8(Hq, Hs, w: MxWeights, offsets, Ye=None, *, packed: bo
     return Ye
 
 
+def moe_grouped_mxfp8_gemm(Aq, Asp, Bq, Pb, offsets, out=None):
+    """out[r] = A[r] · B_eᵀ for each expert e's rows on block-scaled FP8
+    (the down GEMM's kernel): Aq [R,K] E4M3 codes with tile-packed scales
+    Asp (K = the contraction), Bq [E,N,K] codes with scales packed as a W2
+    operand (mxfp8_pack_weight_scales); out [R,N] bf16."""
+    for t, n in ((Aq, "Aq"), (Asp, "Asp"), (Bq, "Bq"), (Pb, "Pb"), (offsets, "offsets")):
+        _need(t, n)
+    E, N, K = Bq.shape
+    R = Aq.shape[0]
+    if out is None:
+        out = torch.empty((R, N), dtype=torch.bfloat16, device=Aq.device)
+    rc = lib.moe_grouped_down_mxfp8(_ptr(Aq), _ptr(Asp), _ptr(Bq), _ptr(Pb), Bq.stride(0),
+                                    _ptr(offsets), E, R, N, K, _ptr(out), _stream(Aq))
+    _check("moe_grouped_down_mxfp8", rc)
+    return out
+
+
+def moe_grouped_swiglu_wgrad(Xe, dA, dB, dYe, H, offsets, out=None):
+    """dW1 = dAᵀ Xe, dW3 = dBᵀ Xe, dW2 = dYeᵀ H per expert (bf16); returns
+    (dW1, dW3, dW2), or fills `out` = (dW1, dW3, dW2)."""
+    for t, n in ((Xe, "Xe"), (dA, "dA"), (dB, "dB"), (dYe, "dYe"), (H, "H"),
+                 (offsets, "offsets")):
+        _need(t, n)
+    R, d = Xe.shape
+    F = dA.shape[1]
+    E = offsets.numel() - 1
+    if out is None:
+        kw = dict(dtype=Xe.dtype, device=Xe.device)
+        out = (torch.empty((E, F, d), **kw), torch.empty((E, F, d), **kw),
+               torch.empty((E, d, F), **kw))
+    dW1, dW3, dW2 = out
+    rc = lib.moe_grouped_swiglu_wgrad(_ptr(Xe), _ptr(dA), _ptr(dB), _ptr(dYe), _ptr(H),
+                                      _ptr(offsets), E, R, d, F, _dtype_code(Xe.dtype), _ptr(dW1),
+                                      _ptr(dW3), _ptr(dW2), _stream(Xe))
+    _check("moe_grouped_swiglu_wgrad", rc)
+    return out
+
+
 def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm: bool = False,
-                        out: Optional[LayerOut] = None) -> LayerOut:
+                        out: Optional[LayerOut] = None, save: bool = False) -> LayerOut:
+    """The MXFP8 layer. save=True keeps what moe_layer_bwd_mxfp8 reads:
+    Xq/Xs (dispatched codes, row-layout scales), Hq/Hsp (H codes, tile-packed
+    scales) and the bf16 pre-activations A, B."""
     _need(x, "x")
     w = _packed(w)
     T, d = x.shape
@@ -829,6 +899,17 @@ def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm
                        gate=torch.empty((T, k), dtype=torch.float32, device=dev),
                        counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
                        slot=torch.empty((T, k), **i32), workspace=ws)
+        if save:
+            R = T * k
+            u8 = dict(dtype=torch.uint8, device=dev)
+            out.Xq = torch.empty((R, d), **u8)
+            out.Xs = torch.empty((R, d // 32), **u8)
+            out.Hq = torch.empty((R, F), **u8)
+            out.Hsp = torch.empty(max(1, lib.mxfp8_act_scales_packed_size(E, R, F)), **u8)
+            out.A = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
+            out.B = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
+    if save and out.Xq is None:
+        raise ValueError("save=True needs an `out` made with save=True")
     a = LayerMxArgs(T=T, d=d, E=E, F=F, k=k, renorm=int(renorm), reserved0=0, reserved1=0,
                     x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1q=_ptr(w.W1q), W3q=_ptr(w.W3q),
                     W2q=_ptr(w.W2q), Ps13=_ptr(w.Ps13), Ps2=_ptr(w.Ps2),
@@ -836,8 +917,101 @@ def moe_layer_fwd_mxfp8(x, k: int, w: MxWeights, *, logits=None, Wr=None, renorm
                     out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
                     counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
                     workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    if save:
+        a.save_Xq, a.save_Xs, a.save_Hq = _ptr(out.Xq), _ptr(out.Xs), _ptr(out.Hq)
+        a.save_Hsp, a.save_A, a.save_B = _ptr(out.Hsp), _ptr(out.A), _ptr(out.B)
     rc = lib.moe_layer_fwd_mxfp8(ctypes.byref(a), _stream(x))
     _check("moe_layer_fwd_mxfp8", rc)
+    return out
+
+
+@dataclass
+class MxWeightsBwd:
+    """Backward weights of the MXFP8 layer: W13tq [E,d,2F] (row i = column i
+    of W1_e then of W3_e, blocks of 32 along F) and W2tq [E,F,d] (row f =
+    column f of W2_e, blocks along d), their UE8M0 scales and the scales
+    packed for the FP8 GEMMs."""
+    W13tq: torch.Tensor
+    W13ts: torch.Tensor
+    W2tq: torch.Tensor
+    W2ts: torch.Tensor
+    Ps13t: torch.Tensor
+    Ps2t: torch.Tensor
+
+
+def mxfp8_quantize_weights_bwd(W1, W3, W2) -> MxWeightsBwd:
+    """Re-quantise the bf16 expert weights along the contraction dimensions
+    of the backward's input-gradient GEMMs (F for W1/W3, d for W2) and pack
+    their scales; once per weight update."""
+    for t, n in ((W1, "W1"), (W3, "W3"), (W2, "W2")):
+        _need(t, n)
+    E, F, d, s13 = _w13(W1, W3)
+    if tuple(W2.shape) != (E, d, F) or W2.stride(1) != F or W2.stride(2) != 1:
+        raise ValueError("W2 must be [E,d,F] with rows contiguous")
+    dev = W1.device
+    u8 = dict(dtype=torch.uint8, device=dev)
+    wb = MxWeightsBwd(W13tq=torch.empty((E, d, 2 * F), **u8),
+                      W13ts=torch.empty((E, d, 2 * F // 32), **u8),
+                      W2tq=torch.empty((E, F, d), **u8), W2ts=torch.empty((E, F, d // 32), **u8),
+                      Ps13t=torch.empty(E * ((d + 255) // 256) * (2 * F // 128) * 1024, **u8),
+                      Ps2t=torch.empty(E * ((F + 255) // 256) * (d // 128) * 1024, **u8))
+    st = _stream(W1)
+    rc = lib.mxfp8_quantize_weights_bwd(_ptr(W1), _ptr(W3), _ptr(W2), s13, W2.stride(0), E, d, F,
+                                        _ptr(wb.W13tq), _ptr(wb.W13ts), _ptr(wb.W2tq),
+                                        _ptr(wb.W2ts), st)
+    _check("mxfp8_quantize_weights_bwd", rc)
+    # both packed as the down GEMM's W2 operand: [E, rows, K]
+    rc = lib.mxfp8_pack_weight_scales(None, None, _ptr(wb.W2ts), E, F, d, None, _ptr(wb.Ps2t), st)
+    _check("mxfp8_pack_weight_scales", rc)
+    rc = lib.mxfp8_pack_weight_scales(None, None, _ptr(wb.W13ts), E, d, 2 * F, None,
+                                      _ptr(wb.Ps13t), st)
+    _check("mxfp8_pack_weight_scales", rc)
+    return wb
+
+
+def moe_swiglu_bwd_mxfp8(dH, A, B, dA=None, dB=None, dABq=None, dABs=None):
+    """dA = dH*B*silu'(A), dB = dH*silu(A) (bf16) and the MXFP8 codes and
+    row-layout scales of [dA | dB] quantised from the fp32 values."""
+    for t, n in ((dH, "dH"), (A, "A"), (B, "B")):
+        _need(t, n)
+    R, F = dH.shape
+    dev = dH.device
+    dA = torch.empty_like(dH) if dA is None else dA
+    dB = torch.empty_like(dH) if dB is None else dB
+    dABq = torch.empty((R, 2 * F), dtype=torch.uint8, device=dev) if dABq is None else dABq
+    dABs = torch.empty((R, 2 * F // 32), dtype=torch.uint8, device=dev) if dABs is None else dABs
+    rc = lib.moe_swiglu_bwd_mxfp8(_ptr(dH), _ptr(A), _ptr(B), R, F, _ptr(dA), _ptr(dB),
+                                  _ptr(dABq), _ptr(dABs), _stream(dH))
+    _check("moe_swiglu_bwd_mxfp8", rc)
+    return dA, dB, dABq, dABs
+
+
+def moe_layer_bwd_mxfp8(fwd: LayerOut, dOut, k: int, wb: MxWeightsBwd,
+                        out: Optional[LayerGrads] = None) -> LayerGrads:
+    """Backward of moe_layer_fwd_mxfp8(save=True) with the gates held
+    constant: FP8 input-gradient GEMMs with wb's weights, bf16 weight
+    gradients on the forward's dequantised operands."""
+    _need(dOut, "dOut")
+    if fwd.Xq is None or fwd.A is None:
+        raise ValueError("moe_layer_bwd_mxfp8 needs the MXFP8 forward run with save=True")
+    T, d = dOut.shape
+    E, F = wb.W2tq.shape[0], wb.W2tq.shape[1]
+    dev = dOut.device
+    if out is None:
+        ws = _alloc_ws(lib.moe_layer_bwd_mxfp8_workspace_size(T, d, E, F, k), dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        out = LayerGrads(dx=torch.empty((T, d), **bf), dW1=torch.empty((E, F, d), **bf),
+                         dW3=torch.empty((E, F, d), **bf), dW2=torch.empty((E, d, F), **bf),
+                         workspace=ws)
+    a = LayerBwdMxArgs(T=T, d=d, E=E, F=F, k=k, reserved0=0, reserved1=0, reserved2=0,
+                       slot=_ptr(fwd.slot), gate=_ptr(fwd.gate), offsets=_ptr(fwd.offsets),
+                       Xq=_ptr(fwd.Xq), Xs=_ptr(fwd.Xs), Hq=_ptr(fwd.Hq), Hsp=_ptr(fwd.Hsp),
+                       A=_ptr(fwd.A), B=_ptr(fwd.B), W13tq=_ptr(wb.W13tq), Ps13t=_ptr(wb.Ps13t),
+                       W2tq=_ptr(wb.W2tq), Ps2t=_ptr(wb.Ps2t), dOut=_ptr(dOut), dx=_ptr(out.dx),
+                       dW1=_ptr(out.dW1), dW3=_ptr(out.dW3), dW2=_ptr(out.dW2),
+                       workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
+    rc = lib.moe_layer_bwd_mxfp8(ctypes.byref(a), _stream(dOut))
+    _check("moe_layer_bwd_mxfp8", rc)
     return out
 
 

@@ -261,6 +261,17 @@ MOE_API int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void* B,
                                    int64_t R, int64_t d, int64_t F, int dtype, void* dA, void* dB,
                                    void* dXe, void* dW1, void* dW3, void* dW2, void* stream);
 
+/* moe_grouped_swiglu_wgrad: the weight-gradient GEMMs of
+ * moe_grouped_swiglu_bwd alone (dW1_e = dAᵀ·Xe_e, dW3_e = dBᵀ·Xe_e,
+ * dW2_e = dYeᵀ·H_e over each expert's rows; zeros for an expert with no
+ * rows), from bf16 rows Xe, dYe [R,d] and dA, dB, H [R,F]. Same layouts and
+ * limits as moe_grouped_swiglu_bwd. The MXFP8 backward runs it on the
+ * forward's dequantised Xe and H. */
+MOE_API int moe_grouped_swiglu_wgrad(const void* Xe, const void* dA, const void* dB,
+                                     const void* dYe, const void* H, const int32_t* offsets,
+                                     int64_t E, int64_t R, int64_t d, int64_t F, int dtype,
+                                     void* dW1, void* dW3, void* dW2, void* stream);
+
 /* ------------------------------------------------------------------------
  * moe_combine — gate-weighted combine back to token order.
  *
@@ -361,6 +372,16 @@ MOE_API int moe_grouped_down_mxfp8(const uint8_t* Hq, const uint8_t* Hs, const u
                                    const uint8_t* Ps2, int64_t w2_expert_stride,
                                    const int32_t* offsets, int64_t E, int64_t R, int64_t d,
                                    int64_t F, void* Ye, void* stream);
+/* moe_grouped_gate_up_mxfp8_save: moe_grouped_gate_up_mxfp8 that also
+ * stores the pre-activations A = Xe·W1ᵀ and B = Xe·W3ᵀ (the fp32
+ * accumulators rounded to bf16, [R,F] each, 16-byte aligned) for the
+ * backward; A_out and B_out both NULL is the plain call. */
+MOE_API int moe_grouped_gate_up_mxfp8_save(const uint8_t* Xq, const uint8_t* Xs,
+                                           const uint8_t* W1q, const uint8_t* W3q,
+                                           const uint8_t* Ps13, int64_t w13_expert_stride,
+                                           const int32_t* offsets, int64_t E, int64_t R,
+                                           int64_t d, int64_t F, uint8_t* Hq, uint8_t* Hs,
+                                           void* A_out, void* B_out, void* stream);
 
 /* moe_layer_fwd_mxfp8 — route -> moe_dispatch_mxfp8 -> gate/up (MXFP8) ->
  * down (MXFP8) -> moe_combine (bf16), on one stream. x, Wr and out are bf16. */
@@ -385,6 +406,18 @@ typedef struct moe_layer_mxfp8_args {
     void* workspace;        /* Xq, Xs (rows and tile-packed), Hq, Hs (packed),
                                Ye and the route workspace                     */
     size_t workspace_bytes;
+    /* optional, all NULL or all set: the forward keeps what
+     * moe_layer_bwd_mxfp8 needs in these caller buffers instead of the
+     * workspace (R = T*k): Xq [R,d] codes, Xs [R,d/32] row-layout scales,
+     * Hq [R,F] codes, Hsp tile-packed H scales
+     * (mxfp8_act_scales_packed_size(E,R,F) bytes), A and B [R,F] bf16
+     * pre-activations. Not accepted by moe_layer_fwd_mxfp8_host. */
+    uint8_t* save_Xq;
+    uint8_t* save_Xs;
+    uint8_t* save_Hq;
+    uint8_t* save_Hsp;
+    void* save_A;
+    void* save_B;
 } moe_layer_mxfp8_args;
 
 MOE_API size_t moe_layer_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F, int k,
@@ -525,6 +558,80 @@ typedef struct moe_layer_bwd_args {
 
 MOE_API size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, int k, int dtype);
 MOE_API int moe_layer_bwd(const moe_layer_bwd_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 backward ["专家池 8→128 只慢 5%…", "三招拆分、三项优化、一个精度开关":
+ * the MXFP8 switch speeds up training through the FFN and the expert data
+ * movement; "olmoforge" README, "MXFP8 分块量化"]. Reading of the backward's
+ * precision (the pages leave it open): the two input-gradient GEMMs run on
+ * block-scaled FP8 with every operand quantised along its contraction
+ * dimension (UE8M0 scales, E4M3 codes), the weight gradients run as bf16
+ * GEMMs on the forward's dequantised operands:
+ *   dYe[slot[t,j]] = bf16(gate[t,j] * dOut[t])
+ *   dH  = Q_d(dYe) · Q_d(W2_e)             (contraction over d)
+ *   dA  = dH*B*silu'(A),  dB = dH*silu(A)   (fp32 from bf16 dH, A, B)
+ *   dXe = Q_F([dA|dB]) · Q_F([W1_e; W3_e])  (contraction over 2F)
+ *   dx[t] = sum_j dXe[slot[t,j]]
+ *   dW1_e = dAᵀ·deq(Xq),  dW3_e = dBᵀ·deq(Xq),  dW2_e = dYeᵀ·deq(Hq)
+ * with A, B, Xq, Hq the forward's (moe_layer_mxfp8_args.save_*).
+ *
+ * mxfp8_quantize_weights_bwd: the backward weights, once per weight update.
+ *   W1, W3 [E,F,d] and W2 [E,d,F] bf16 (expert strides in elements, rows
+ *   contiguous) -> W13tq [E,d,2F] codes with W13ts [E,d,2F/32] scales (row i:
+ *   column i of W1_e then column i of W3_e, blocks of 32 along F), and W2tq
+ *   [E,F,d] with W2ts [E,F,d/32] (row f: column f of W2_e, blocks along d).
+ *   Pack the scales with mxfp8_pack_weight_scales as a W2 operand: W2ts with
+ *   (d, F) = (F, d) -> Ps2t, W13ts with (d, F) = (d, 2F) -> Ps13t.
+ *   d % 128 == 0, F % 128 == 0; all pointers 16-byte aligned.
+ * moe_swiglu_bwd_mxfp8: the SwiGLU backward step alone: dH, A, B [R,F] bf16
+ *   -> dA, dB [R,F] bf16 and the codes of [dA|dB] dABq [R,2F] with scales
+ *   dABs [R,2F/32] (quantised from the fp32 values). F % 32 == 0.
+ * moe_layer_bwd_mxfp8: the whole chain on one stream (moe_dispatch,
+ *   mxfp8_quantize, mxfp8_pack_act_scales, moe_grouped_down_mxfp8 for dH
+ *   and dXe, moe_swiglu_bwd_mxfp8, moe_combine, mxfp8_dequantize and the
+ *   bf16 weight-gradient GEMMs of moe_grouped_swiglu_bwd). d % 256 == 0,
+ *   F % 256 == 0. Workspace: moe_layer_bwd_mxfp8_workspace_size bytes,
+ *   256-byte aligned. dx [T,d], dW1/dW3 [E,F,d], dW2 [E,d,F] bf16,
+ *   contiguous; an expert with no rows gets zero weight gradients. Router
+ *   and gate gradients are not part of it (use moe_router_bwd).
+ * ---------------------------------------------------------------------- */
+MOE_API int mxfp8_quantize_weights_bwd(const void* W1, const void* W3, const void* W2,
+                                       int64_t w13_expert_stride, int64_t w2_expert_stride,
+                                       int64_t E, int64_t d, int64_t F, uint8_t* W13tq,
+                                       uint8_t* W13ts, uint8_t* W2tq, uint8_t* W2ts,
+                                       void* stream);
+MOE_API int moe_swiglu_bwd_mxfp8(const void* dH, const void* A, const void* B, int64_t R,
+                                 int64_t F, void* dA, void* dB, uint8_t* dABq, uint8_t* dABs,
+                                 void* stream);
+
+typedef struct moe_layer_bwd_mxfp8_args {
+    int64_t T, d, E, F;
+    int32_t k, reserved0, reserved1, reserved2;
+    const int32_t* slot;    /* [T,k] from the forward                          */
+    const float* gate;      /* [T,k]                                          */
+    const int32_t* offsets; /* [E+1]                                          */
+    const uint8_t* Xq;      /* [R,d] the forward's dispatched codes            */
+    const uint8_t* Xs;      /* [R,d/32] their scales, row layout              */
+    const uint8_t* Hq;      /* [R,F] the forward's H codes                     */
+    const uint8_t* Hsp;     /* H scales, tile-packed (as gate/up wrote them)   */
+    const void* A;          /* [R,F] bf16 pre-activations                      */
+    const void* B;          /* [R,F] bf16                                      */
+    const uint8_t* W13tq;   /* [E,d,2F] (mxfp8_quantize_weights_bwd)           */
+    const uint8_t* Ps13t;   /* its packed scales                              */
+    const uint8_t* W2tq;    /* [E,F,d]                                        */
+    const uint8_t* Ps2t;    /* its packed scales                              */
+    const void* dOut;       /* [T,d] bf16 upstream gradient                   */
+    void* dx;               /* [T,d] bf16                                     */
+    void* dW1;              /* [E,F,d] bf16                                   */
+    void* dW3;              /* [E,F,d] bf16                                   */
+    void* dW2;              /* [E,d,F] bf16                                   */
+    void* workspace;
+    size_t workspace_bytes;
+} moe_layer_bwd_mxfp8_args;
+
+MOE_API size_t moe_layer_bwd_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E, int64_t F,
+                                                  int k);
+MOE_API int moe_layer_bwd_mxfp8(const moe_layer_bwd_mxfp8_args* args, void* stream);
 
 /* ------------------------------------------------------------------------
  * Router backward and the load-balancing auxiliary loss.

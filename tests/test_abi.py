@@ -79,6 +79,26 @@ def test_host_validation_rejects_without_launch(lib):
     assert L.moe_dispatch(p16, p16, None, 0, 64, 2, m.MOE_BF16, p16, None) == m.MOE_OK
     assert L.moe_row_token(p16, 0, 2, p16, None) == m.MOE_OK
     assert L.moe_layer_fwd(None, None) == m.MOE_ERR_INVALID
+    # MXFP8 backward: weights need d, F % 128; the SwiGLU step needs F % 32;
+    # the layer needs its arguments and d, F % 256
+    assert L.mxfp8_quantize_weights_bwd(p16, p16, p16, 96 * 128, 96 * 128, 2, 96, 128, p16, p16,
+                                        p16, p16, None) == m.MOE_ERR_UNSUPPORTED
+    assert L.mxfp8_quantize_weights_bwd(p16, None, p16, 128 * 128, 128 * 128, 2, 128, 128, p16,
+                                        p16, p16, p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_swiglu_bwd_mxfp8(p16, p16, p16, 4, 48, p16, p16, p16, p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_swiglu_bwd_mxfp8(p16, p16, p16, 0, 64, p16, p16, p16, p16, None) == m.MOE_OK
+    assert L.moe_layer_bwd_mxfp8(None, None) == m.MOE_ERR_INVALID
+    a = m.LayerBwdMxArgs(T=4, d=128, E=2, F=256, k=1, workspace=p16, workspace_bytes=1 << 15)
+    assert L.moe_layer_bwd_mxfp8(ctypes.byref(a), None) == m.MOE_ERR_UNSUPPORTED
+    a.d = 256
+    assert L.moe_layer_bwd_mxfp8(ctypes.byref(a), None) == m.MOE_ERR_INVALID  # no tensors
+    assert L.moe_grouped_swiglu_wgrad(p16, p16, p16, p16, p16, p16, 2, 8, 256, 256, m.MOE_F32,
+                                      p16, p16, p16, None) == m.MOE_ERR_UNSUPPORTED
+    # the MXFP8 forward's save buffers: all or none; not in the sliced host entry
+    f = m.LayerMxArgs(T=4, d=256, E=2, F=256, k=1, workspace=p16, workspace_bytes=1 << 15,
+                      save_A=p16)
+    assert L.moe_layer_fwd_mxfp8_host(ctypes.byref(f), p16, None, p16, 2, p16, p16 + 1,
+                                      p16 + 2) == m.MOE_ERR_INVALID
 
 
 def test_workspace_sizes_are_consistent(lib):
