@@ -944,8 +944,9 @@ def mxfp8_quantize_weights_bwd(W1, W3, W2) -> MxWeightsBwd:
     of the backward's input-gradient GEMMs (F for W1/W3, d for W2) and pack
     their scales; once per weight update."""
     for t, n in ((W1, "W1"), (W3, "W3"), (W2, "W2")):
-        _need(t, n)
-    E, F, d, s13 = _w13(W1, W3)
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+    E, F, d, s13 = _w13(W1, W3)  # views into a fused [E,2F,d] tensor are accepted
     if tuple(W2.shape) != (E, d, F) or W2.stride(1) != F or W2.stride(2) != 1:
         raise ValueError("W2 must be [E,d,F] with rows contiguous")
     dev = W1.device
