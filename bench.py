@@ -473,9 +473,11 @@ def _steps(moe, w, inp, dev, backward):
                                      + E * d * es)
     # backward: bf16 dispatch 1 + GEMMs 5 + combine 1; MXFP8 dispatch,
     # quantise, pack 3 + dH 1 + SwiGLU, pack 2 + dX 1 + combine 1 +
-    # dequantise, unpack, dequantise 3 + dW 3; then the aux loss 2 and the
-    # router backward 1 (+3 for the router GEMM backward)
-    bwd_kernels = (14 if w.mxfp8 else 7) + 2 + 1 + (3 if use_router else 0)
+    # dequantise, unpack, dequantise 3 + dW 3; then the aux loss 2 (partial
+    # sums, final sum) and the router backward 2 (gate gradients, softmax
+    # backward), + 4 for the router GEMM backward (dlogits to bf16, dx, dWr
+    # chunk partials, their ordered sum; the bf16 router workloads)
+    bwd_kernels = (14 if w.mxfp8 else 7) + 2 + 2 + (4 if use_router else 0)
     kernels = ((4 if use_router else 3) + (5 if w.mxfp8 else 4)
                + (bwd_kernels if backward else 0))
     return [n for n, _ in fns], step, kernels, work, e_act
