@@ -47,6 +47,12 @@ notes):
     payload = E4M3 with round-to-nearest-even and saturation to ±448 of the
     fp32 quotient v/scale. The sketch in [OF] rounds v/scale to an integer,
     which is not an E4M3 payload; the E4M3 reading is taken.
+  * MXFP8 backward (the pages leave its precision open): the input-gradient
+    GEMMs quantise each operand along its own contraction dimension (dYe
+    and W2 along d, [dA | dB] and [W1; W3] along F); the weight gradients
+    are exact GEMMs of the unquantised gradients with the forward's
+    dequantised operands. Values that decide a code are taken in the
+    precision the layer stores them in (bf16 dYe, dH, A, B).
 
 Where a function has no independent pin it says "parity unpinned"; every
 function below is pinned by tests/test_oracle.py.
