@@ -252,6 +252,13 @@ extern "C" int moe_layer_bwd_mxfp8(const moe_layer_bwd_mxfp8_args* a, void* stre
                           a->dW2};
     for (const void* p : need)
         if (!p) return MOE_ERR_INVALID;
+    // what the steps below check, checked before the first launch
+    const void* rows[] = {a->Xq, a->Hq, a->Hsp, a->A, a->B, a->W13tq, a->Ps13t, a->W2tq, a->Ps2t,
+                          a->dOut, a->dx, a->dW1, a->dW3, a->dW2};
+    for (const void* p : rows)
+        if (!aligned16(p)) return MOE_ERR_INVALID;
+    if (a->T * a->k > INT32_MAX - 256 || a->d > (1 << 24) || 2 * a->F > (1 << 24))
+        return MOE_ERR_UNSUPPORTED;
     const int64_t T = a->T, d = a->d, E = a->E, F = a->F, R = a->T * a->k;
     int rc;
     if (R > 0) {

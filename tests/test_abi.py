@@ -92,6 +92,11 @@ def test_host_validation_rejects_without_launch(lib):
     assert L.moe_layer_bwd_mxfp8(ctypes.byref(a), None) == m.MOE_ERR_UNSUPPORTED
     a.d = 256
     assert L.moe_layer_bwd_mxfp8(ctypes.byref(a), None) == m.MOE_ERR_INVALID  # no tensors
+    for f in ("slot", "gate", "offsets", "Xq", "Xs", "Hq", "Hsp", "A", "B", "W13tq", "Ps13t",
+              "W2tq", "Ps2t", "dOut", "dx", "dW1", "dW3", "dW2"):
+        setattr(a, f, p16)
+    a.dx = p16 + 2  # a misaligned output is caught before the first launch
+    assert L.moe_layer_bwd_mxfp8(ctypes.byref(a), None) == m.MOE_ERR_INVALID
     assert L.moe_grouped_swiglu_wgrad(p16, p16, p16, p16, p16, p16, 2, 8, 256, 256, m.MOE_F32,
                                       p16, p16, p16, None) == m.MOE_ERR_UNSUPPORTED
     # the MXFP8 forward's save buffers: all or none; not in the sliced host entry
