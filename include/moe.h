@@ -26,7 +26,12 @@
  *
  * Error behaviour (all calls): arguments are validated on the host before
  * anything is enqueued. MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED mean nothing was
- * launched. MOE_ERR_CUDA means a launch failed (the CUDA error is left for
+ * launched; for the whole-layer entries (moe_layer_*), which chain the
+ * single-step entries, this holds for the checks they make up front (their
+ * own arguments and workspace; moe_layer_bwd_mxfp8 checks every step's
+ * pointers and sizes too), while a step's own check that fails later, e.g. a
+ * weight pointer that is not 16-byte aligned, returns its code with the
+ * earlier steps already enqueued and the outputs incomplete. MOE_ERR_CUDA means a launch failed (the CUDA error is left for
  * cudaGetLastError). Faults found on the device (a metadata value out of
  * range, a pipeline wait that exceeded its time limit) set bits in a
  * per-process device status word instead of trapping; the kernel that finds
