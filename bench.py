@@ -240,6 +240,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = WORKLOADS[args.workload]
+    if args.backward and not w.backward:
+        w = w.scaled(name=w.name, backward=True)  # adds the upstream gradient dOut
     inp = make_inputs(w, "cpu")
     S = args.ref_tokens
     for _ in range(args.warmup):
@@ -252,7 +254,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": config_of(w, world),
+        "config": config_of(w, world, args.backward),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"each step: first {S} of {w.T} tokens of {w.name}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
