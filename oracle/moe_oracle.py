@@ -452,32 +452,54 @@ def mxfp8_dequantize(codes: np.ndarray, stored: np.ndarray, mode: str) -> torch.
 
 
 def mxfp8_layer(x: torch.Tensor, k: int, W1, W3, W2, logits: np.ndarray,
-                mode: str = "e8m0", tokens: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
-    """MXFP8 variant of the layer: x, W1, W3 quantised along d, W2 and H
-    along F; GEMMs on the dequantised values in float64; H quantised from
-    its fp32 value. ``tokens`` restricts the output to a sample."""
+                mode: str = "e8m0", tokens: Optional[np.ndarray] = None,
+                exact: bool = False, return_ops: bool = False) -> Dict[str, np.ndarray]:
+    """MXFP8 variant of the layer ([OF] capability table and "MXFP8 分块量化":
+    32-element blocks sharing one scale, E4M3 payload; [NEWS] "三招拆分、三项
+    优化、一个精度开关": the FFN runs on MXFP8 operands). Every GEMM operand
+    is quantised along its contraction dimension: the token rows of x and
+    the rows of W1_e, W3_e ([F, d]) along d; the rows of W2_e ([d, F]) and
+    H along F, H from its fp32 value silu(a) * b. The GEMMs then run on the
+    dequantised values in float64, per (token, choice) as in the per-token
+    formula out[t] = sum_j gate[t,j] W2_e(silu(W1_e x_t) * W3_e x_t).
+    ``tokens`` restricts the output to a sample.
+
+    exact=True replaces every quantise-dequantise (and the fp32 rounding of
+    H) by the identity, which must give the plain layer (a wiring check).
+    return_ops=True adds the operands as quantised: "xd" (the sampled token
+    rows), "w" {e: (w1d, w3d, w2d)}, "h" {(i, j): (H fp32 row, Hd row)}."""
+    if exact:
+        qdq = lambda m: np.asarray(m, np.float64)  # noqa: E731
+        h32 = lambda m: np.asarray(m, np.float64)  # noqa: E731
+    else:
+        qdq = lambda m: _qdq_rows(m, mode)  # noqa: E731
+        h32 = lambda m: np.asarray(m, np.float32).astype(np.float64)  # noqa: E731
     E = W1.shape[0]
     idx, gate, _ = route(logits, k)
     meta = routing_metadata(idx, E)
     T = x.shape[0]
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
-    xq, xs = mxfp8_quantize(x[torch.as_tensor(toks, dtype=torch.long)], mode)
-    xd = mxfp8_dequantize_f32(xq, xs, mode).astype(np.float64)
+    xd = qdq(to64(x[torch.as_tensor(toks, dtype=torch.long)]))      # along d
     out = np.zeros((len(toks), x.shape[1]))
-    cache = {}
+    wq = {}
+    hs = {}
     for i, t in enumerate(toks):
         for j in range(k):
             e = int(idx[t, j])
-            if e not in cache:
-                w1 = mxfp8_dequantize_f32(*mxfp8_quantize(W1[e], mode), mode).astype(np.float64)
-                w3 = mxfp8_dequantize_f32(*mxfp8_quantize(W3[e], mode), mode).astype(np.float64)
-                w2 = mxfp8_dequantize_f32(*mxfp8_quantize(W2[e], mode), mode).astype(np.float64)
-                cache[e] = (w1, w3, w2)
-            w1, w3, w2 = cache[e]
-            h = (silu(w1 @ xd[i]) * (w3 @ xd[i])).astype(np.float32)[None, :]
-            hd = mxfp8_dequantize_f32(*mxfp8_quantize(h, mode), mode).astype(np.float64)[0]
-            out[i] += gate[t, j] * (w2 @ hd)
-    return dict(out=out, idx=idx, gate=gate, tokens=toks, **meta)
+            if e not in wq:
+                wq[e] = (qdq(to64(W1[e])),   # [F, d] along d
+                         qdq(to64(W3[e])),   # [F, d] along d
+                         qdq(to64(W2[e])))   # [d, F] along F
+            w1d, w3d, w2d = wq[e]
+            h = h32(silu(w1d @ xd[i]) * (w3d @ xd[i]))
+            hd = qdq(h[None, :])[0]                                  # along F
+            out[i] += gate[t, j] * (w2d @ hd)
+            if return_ops:
+                hs[(i, j)] = (h, hd)
+    res = dict(out=out, idx=idx, gate=gate, tokens=toks, **meta)
+    if return_ops:
+        res["ops"] = dict(xd=xd, w=wq, h=hs)
+    return res
 
 
 # --------------------------------------------------------------------------

@@ -652,3 +652,64 @@ def test_mxfp8_backward_error_against_exact_backward():
     for name in ("dx", "dW1", "dW3", "dW2"):
         rel = np.linalg.norm(r[name] - b[name]) / np.linalg.norm(b[name])
         assert 1e-3 < rel < 0.15, (name, rel)
+
+
+# ---------------------------------------------------------------- MXFP8 forward
+
+def test_mxfp8_forward_exact_mode_is_the_layer():
+    # every quantise-dequantise (and the fp32 rounding of H) replaced by the
+    # identity: the wiring (which operand, gates, the per-token sum) must give
+    # the plain layer, itself pinned against torch above
+    x, W1, W3, W2, lg, _ = _mx_problem(71)
+    k = 2
+    r = O.mxfp8_layer(x, k, W1, W3, W2, lg, exact=True)
+    b = O.moe_layer(x, k, W1, W3, W2, logits=lg)
+    assert np.allclose(r["out"], b["out"], rtol=1e-12, atol=1e-12)
+    toks = np.array([0, 5, 17, 39])
+    rs = O.mxfp8_layer(x, k, W1, W3, W2, lg, tokens=toks, exact=True)
+    assert np.allclose(rs["out"], b["out"][toks], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(r["idx"], b["idx"]) and np.array_equal(r["slot"], b["slot"])
+
+
+def test_mxfp8_forward_operands_quantised_along_contraction():
+    # each quantised operand equals an independent torch restatement of the
+    # codec applied along the stated axis to the stated source; the skewed
+    # magnitudes make the other axis give other scales, which is checked too
+    x, W1, W3, W2, lg, _ = _mx_problem(72, skew=True)
+    k = 2
+    toks = np.arange(4, 36)  # 32 tokens, so blocks along the token axis exist too
+    with np.errstate(over="ignore"):
+        r = O.mxfp8_layer(x, k, W1, W3, W2, lg, tokens=toks, return_ops=True)
+    ops = r["ops"]
+    x64 = x.double().numpy()
+    assert np.array_equal(ops["xd"], _torch_qdq_rows(x64[toks]))            # x along d
+    assert not np.array_equal(ops["xd"], _torch_qdq_rows(x64[toks].T).T)
+    for e, (w1d, w3d, w2d) in ops["w"].items():
+        w1, w3, w2 = (t[e].double().numpy() for t in (W1, W3, W2))
+        assert np.array_equal(w1d, _torch_qdq_rows(w1))                    # [F, d] along d
+        assert np.array_equal(w3d, _torch_qdq_rows(w3))
+        assert np.array_equal(w2d, _torch_qdq_rows(w2))                    # [d, F] along F
+        # the other axis gives another result on these inputs
+        assert not np.array_equal(w1d, _torch_qdq_rows(w1.T).T)
+        assert not np.array_equal(w2d, _torch_qdq_rows(w2.T).T)
+    idx, gate = r["idx"], r["gate"]
+    out = np.zeros((len(toks), x.shape[1]))
+    for (i, j), (h, hd) in ops["h"].items():
+        e = int(idx[toks[i], j])
+        w1d, w3d, w2d = ops["w"][e]
+        xi = ops["xd"][i]
+        a, b = w1d @ xi, w3d @ xi
+        h_ref = (a / (1.0 + np.exp(-a)) * b).astype(np.float32).astype(np.float64)
+        assert np.array_equal(h, h_ref)                                    # H from its fp32 value
+        assert np.array_equal(hd, _torch_qdq_rows(h[None, :])[0])          # H along F
+        out[i] += gate[toks[i], j] * (w2d @ hd)
+    assert np.allclose(out, r["out"], rtol=1e-13, atol=1e-13)
+
+
+def test_mxfp8_forward_error_against_exact_layer():
+    # the format's error: a few percent of relative L2, never a gross mistake
+    x, W1, W3, W2, lg, _ = _mx_problem(73, T=96, d=128, F=128)
+    r = O.mxfp8_layer(x, 2, W1, W3, W2, lg)
+    b = O.moe_layer(x, 2, W1, W3, W2, logits=lg)
+    rel = np.linalg.norm(r["out"] - b["out"]) / np.linalg.norm(b["out"])
+    assert 1e-3 < rel < 0.15, rel
