@@ -15,6 +15,31 @@ namespace moe {
 // Address of this process's device status word on the current device.
 int* status_ptr();
 
+// While a whole-layer entry checks the arguments of every step it chains
+// before its first launch, the single-step entries it calls return MOE_OK
+// right after their host-side checks (tensor maps included) instead of
+// enqueuing work. The flag is per host thread.
+bool& check_only();
+struct CheckOnly {
+    CheckOnly() { check_only() = true; }
+    ~CheckOnly() { check_only() = false; }
+};
+
+// Runs `steps` (a chain of single-step entries) once with every step
+// stopping after its checks and, if all of them pass, once more for real, so
+// an invalid argument of any step is reported before anything is enqueued.
+// Inside an outer check pass it only checks.
+template <typename Steps>
+inline int checked(Steps&& steps) {
+    if (check_only()) return steps();
+    {
+        CheckOnly guard;
+        const int rc = steps();
+        if (rc != MOE_OK) return rc;
+    }
+    return steps();
+}
+
 inline int launch_status() {
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -185,6 +185,7 @@ extern "C" int moe_dispatch(const void* x, const int32_t* slot, const float* gat
     if (T == 0) return MOE_OK;
     if (!x || !slot || !Xe || !aligned16(x) || !aligned16(Xe)) return MOE_ERR_INVALID;
     if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     const int vpr = (int)(d * es / 16);
     const int64_t R = T * k;
     cudaStream_t st = as_stream(stream);
@@ -214,6 +215,7 @@ extern "C" int moe_combine(const void* Ye, const int32_t* slot, const float* gat
     if (T == 0) return MOE_OK;
     if (!Ye || !slot || !out || !aligned16(Ye) || !aligned16(out)) return MOE_ERR_INVALID;
     if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     const int vpr = (int)(d * es / 16);
     const int64_t R = T * k;
     cudaStream_t st = as_stream(stream);
@@ -240,6 +242,7 @@ extern "C" int moe_row_token(const int32_t* slot, int64_t T, int k, int32_t* row
     if (T == 0) return MOE_OK;
     if (!slot || !row_token) return MOE_ERR_INVALID;
     if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     const int64_t n = T * k;
     int64_t g = (n + dc::THREADS - 1) / dc::THREADS;
     const int64_t cap = (int64_t)num_sms() * 8;

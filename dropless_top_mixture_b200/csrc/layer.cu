@@ -13,6 +13,11 @@ namespace moe {
 
 __device__ int g_status_word;
 
+bool& check_only() {
+    thread_local bool flag = false;
+    return flag;
+}
+
 int* status_ptr() {
     static int* cached[64] = {nullptr};
     static std::mutex mu;
@@ -85,15 +90,11 @@ extern "C" size_t moe_layer_workspace_size(int64_t T, int64_t d, int64_t E, int6
     return layer::carve(nullptr, T, d, E, F, k, dtype, logits_given).total;
 }
 
-extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
-    if (!a) return MOE_ERR_INVALID;
-    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
-    if (a->dtype != MOE_BF16 && a->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
-    if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
-        return MOE_ERR_INVALID;
-    const int logits_given = a->logits != nullptr;
-    layer::Carve c = layer::carve(a->workspace, a->T, a->d, a->E, a->F, a->k, a->dtype, logits_given);
-    if (a->workspace_bytes < c.total) return MOE_ERR_INVALID;
+namespace moe {
+namespace layer {
+
+// The steps of moe_layer_fwd after its own checks.
+static int fwd_steps(const moe_layer_args* a, const Carve& c, void* stream) {
     if (a->T == 0) {
         return moe_route(a->logits, a->x, a->Wr, a->dtype, 0, a->d, a->E, a->k, a->renorm,
                          nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
@@ -118,25 +119,47 @@ extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
     return moe_combine(Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
 }
 
+}  // namespace layer
+}  // namespace moe
+
+extern "C" int moe_layer_fwd(const moe_layer_args* a, void* stream) {
+    if (!a) return MOE_ERR_INVALID;
+    if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
+    if (a->dtype != MOE_BF16 && a->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return MOE_ERR_INVALID;
+    const int logits_given = a->logits != nullptr;
+    const layer::Carve c =
+        layer::carve(a->workspace, a->T, a->d, a->E, a->F, a->k, a->dtype, logits_given);
+    if (a->workspace_bytes < c.total) return MOE_ERR_INVALID;
+    return checked([&] { return layer::fwd_steps(a, c, stream); });
+}
+
 namespace moe {
 namespace layer {
 
 constexpr int MAX_CHUNKS = 64;
+constexpr int NUM_EVENTS = 2 * MAX_CHUNKS + 3;
 
-// Events of the host pipeline, created once per device and kept.
-static cudaEvent_t* pipeline_events() {
-    static cudaEvent_t ev[64][2 * MAX_CHUNKS + 2];
+// Events of the host pipeline, created once per device and kept, and the
+// per-device lock that a call holds while it records and waits on them (the
+// record/wait pairs are consumed when they are enqueued, so holding the lock
+// for the enqueue loop keeps two host threads from interleaving on them).
+static cudaEvent_t* pipeline_events(std::mutex** mu_out) {
+    static cudaEvent_t ev[64][NUM_EVENTS];
     static bool made[64] = {false};
-    static std::mutex mu;
+    static std::mutex make_mu;
+    static std::mutex use_mu[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
+    std::lock_guard<std::mutex> lock(make_mu);
     if (!made[dev]) {
-        for (int i = 0; i < 2 * MAX_CHUNKS + 2; ++i)
+        for (int i = 0; i < NUM_EVENTS; ++i)
             if (cudaEventCreateWithFlags(&ev[dev][i], cudaEventDisableTiming) != cudaSuccess)
                 return nullptr;
         made[dev] = true;
     }
+    *mu_out = &use_mu[dev];
     return ev[dev];
 }
 
@@ -153,56 +176,88 @@ namespace layer {
 // the size of the others, so the copy-in before the first compute and the
 // copy-out after the last one (the parts nothing overlaps) are short:
 // slice i ends at T * (2i + 1) / (2 (chunks - 1)), the last at T.
+// Every slice's layer call is checked before the first copy is enqueued; if
+// an enqueue still fails, `sc` is made to wait for whatever the copy streams
+// already hold before the error is returned.
 template <typename Run>
 static int host_pipeline(int64_t T, int64_t E, size_t row_bytes, void* x_dev,
                          const float* logits_dev, void* out_dev, const void* x_host,
                          const float* logits_host, void* out_host, int chunks, cudaStream_t sc,
                          cudaStream_t si, cudaStream_t so, Run&& run) {
-    cudaEvent_t* ev = pipeline_events();
-    if (!ev) return MOE_ERR_CUDA;
     auto bound = [&](int i) -> int64_t {
         if (i <= 0) return 0;
         if (i >= chunks) return T;
         if (chunks < 3) return T * i / chunks;
         return T * (2 * i - 1) / (2 * (chunks - 1));
     };
+    auto slice = [&](int i, int64_t* t0, int64_t* tn, char** xd, float** ld, char** od) {
+        *t0 = bound(i);
+        *tn = bound(i + 1) - *t0;
+        const size_t off = (size_t)*t0 * row_bytes;
+        *xd = static_cast<char*>(x_dev) + off;
+        *ld = logits_dev ? const_cast<float*>(logits_dev) + (size_t)*t0 * E : nullptr;
+        *od = static_cast<char*>(out_dev) + off;
+    };
+    {
+        CheckOnly guard;
+        for (int i = 0; i < chunks; ++i) {
+            int64_t t0, tn;
+            char *xd, *od;
+            float* ld;
+            slice(i, &t0, &tn, &xd, &ld, &od);
+            if (tn <= 0) continue;
+            const int rc = run(t0, tn, xd, ld, od);
+            if (rc != MOE_OK) return rc;
+        }
+    }
+    std::mutex* mu = nullptr;
+    cudaEvent_t* ev = pipeline_events(&mu);
+    if (!ev) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(*mu);
+    const int JOIN_OUT = 2 * MAX_CHUNKS, START = 2 * MAX_CHUNKS + 1, JOIN_IN = 2 * MAX_CHUNKS + 2;
     // the staging buffers may still be in use by work enqueued on `sc`
     // before this call: the copy-ins wait for it
-    if (cudaEventRecord(ev[2 * MAX_CHUNKS + 1], sc) != cudaSuccess ||
-        cudaStreamWaitEvent(si, ev[2 * MAX_CHUNKS + 1], 0) != cudaSuccess)
+    if (cudaEventRecord(ev[START], sc) != cudaSuccess ||
+        cudaStreamWaitEvent(si, ev[START], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
+    auto fail = [&](int rc) {
+        // keep the promise that `sc` is ordered after every copy this call
+        // enqueued, so the caller may reuse its buffers once `sc` is done
+        cudaEventRecord(ev[JOIN_IN], si);
+        cudaStreamWaitEvent(sc, ev[JOIN_IN], 0);
+        cudaEventRecord(ev[JOIN_OUT], so);
+        cudaStreamWaitEvent(sc, ev[JOIN_OUT], 0);
+        return rc;
+    };
     int n = 0;
     for (int i = 0; i < chunks; ++i) {
-        const int64_t t0 = bound(i), tn = bound(i + 1) - t0;
+        int64_t t0, tn;
+        char *xd, *od;
+        float* ld;
+        slice(i, &t0, &tn, &xd, &ld, &od);
         if (tn <= 0) continue;
         const size_t off = (size_t)t0 * row_bytes, bytes = (size_t)tn * row_bytes;
-        char* xd = static_cast<char*>(x_dev) + off;
         if (cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + off, bytes,
                             cudaMemcpyHostToDevice, si) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        float* ld = nullptr;
-        if (logits_dev) {
-            ld = const_cast<float*>(logits_dev) + (size_t)t0 * E;
-            if (cudaMemcpyAsync(ld, logits_host + (size_t)t0 * E, (size_t)tn * E * sizeof(float),
-                                cudaMemcpyHostToDevice, si) != cudaSuccess)
-                return MOE_ERR_CUDA;
-        }
+            return fail(MOE_ERR_CUDA);
+        if (ld && cudaMemcpyAsync(ld, logits_host + (size_t)t0 * E, (size_t)tn * E * sizeof(float),
+                                  cudaMemcpyHostToDevice, si) != cudaSuccess)
+            return fail(MOE_ERR_CUDA);
         if (cudaEventRecord(ev[2 * n], si) != cudaSuccess ||
             cudaStreamWaitEvent(sc, ev[2 * n], 0) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        char* od = static_cast<char*>(out_dev) + off;
+            return fail(MOE_ERR_CUDA);
         const int rc = run(t0, tn, xd, ld, od);
-        if (rc != MOE_OK) return rc;
+        if (rc != MOE_OK) return fail(rc);
         if (cudaEventRecord(ev[2 * n + 1], sc) != cudaSuccess ||
             cudaStreamWaitEvent(so, ev[2 * n + 1], 0) != cudaSuccess)
-            return MOE_ERR_CUDA;
+            return fail(MOE_ERR_CUDA);
         if (cudaMemcpyAsync(static_cast<char*>(out_host) + off, od, bytes, cudaMemcpyDeviceToHost,
                             so) != cudaSuccess)
-            return MOE_ERR_CUDA;
+            return fail(MOE_ERR_CUDA);
         ++n;
     }
-    if (cudaEventRecord(ev[2 * MAX_CHUNKS], so) != cudaSuccess ||
-        cudaStreamWaitEvent(sc, ev[2 * MAX_CHUNKS], 0) != cudaSuccess)
+    if (cudaEventRecord(ev[JOIN_OUT], so) != cudaSuccess ||
+        cudaStreamWaitEvent(sc, ev[JOIN_OUT], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -275,6 +330,13 @@ extern "C" size_t moe_layer_bwd_workspace_size(int64_t T, int64_t d, int64_t F, 
     return 2 * layer::a256(R * d * es) + 2 * layer::a256(R * F * es);
 }
 
+namespace moe {
+namespace layer {
+static int bwd_steps(const moe_layer_bwd_args* a, int64_t R, void* dYe, void* dXe, void* dA,
+                     void* dB, void* stream);
+}  // namespace layer
+}  // namespace moe
+
 extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
     if (!a) return MOE_ERR_INVALID;
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
@@ -298,6 +360,16 @@ extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
     void* dA = p;
     p += layer::a256((size_t)R * a->F * 2);
     void* dB = p;
+    auto steps = [&]() { return layer::bwd_steps(a, R, dYe, dXe, dA, dB, stream); };
+    return checked(steps);
+}
+
+namespace moe {
+namespace layer {
+
+// The steps of moe_layer_bwd after its own checks.
+static int bwd_steps(const moe_layer_bwd_args* a, int64_t R, void* dYe, void* dXe, void* dA,
+                     void* dB, void* stream) {
     int rc;
     if (a->T > 0) {
         rc = moe_dispatch(a->dOut, a->slot, a->gate, a->T, a->d, a->k, a->dtype, dYe, stream);
@@ -317,6 +389,9 @@ extern "C" int moe_layer_bwd(const moe_layer_bwd_args* a, void* stream) {
     return moe_router_linear_bwd(a->dlogits, a->x, a->Wr, a->T, a->d, a->E, a->dtype, a->dx,
                                  a->dWr, a->router_workspace, a->router_workspace_bytes, stream);
 }
+
+}  // namespace layer
+}  // namespace moe
 
 namespace moe {
 namespace layer {
@@ -367,6 +442,13 @@ extern "C" size_t moe_layer_mxfp8_workspace_size(int64_t T, int64_t d, int64_t E
     return layer::carve_mx(nullptr, T, d, E, F, k, logits_given).total;
 }
 
+namespace moe {
+namespace layer {
+static int fwd_mxfp8_steps(const moe_layer_mxfp8_args* a, const CarveMx& c, bool save,
+                           void* stream);
+}  // namespace layer
+}  // namespace moe
+
 extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) {
     if (!a) return MOE_ERR_INVALID;
     if (a->T < 0 || a->d <= 0 || a->E < 1 || a->F <= 0 || a->k < 1) return MOE_ERR_INVALID;
@@ -388,6 +470,16 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     } else if (a->save_Xs || a->save_Hq || a->save_Hsp || a->save_A || a->save_B) {
         return MOE_ERR_INVALID;
     }
+    auto steps = [&]() { return layer::fwd_mxfp8_steps(a, c, save, stream); };
+    return checked(steps);
+}
+
+namespace moe {
+namespace layer {
+
+// The steps of moe_layer_fwd_mxfp8 after its own checks.
+static int fwd_mxfp8_steps(const moe_layer_mxfp8_args* a, const CarveMx& c, bool save,
+                           void* stream) {
     int rc = moe_route(a->logits, a->x, a->Wr, MOE_BF16, a->T, a->d, a->E, a->k, a->renorm,
                        nullptr, a->idx, a->gate, a->counts, a->offsets, a->slot, nullptr,
                        c.route_ws, c.route_bytes, stream);
@@ -407,3 +499,6 @@ extern "C" int moe_layer_fwd_mxfp8(const moe_layer_mxfp8_args* a, void* stream) 
     if (rc != MOE_OK) return rc;
     return moe_combine(c.Ye, a->slot, a->gate, a->T, a->d, a->k, MOE_BF16, a->out, stream);
 }
+
+}  // namespace layer
+}  // namespace moe

@@ -125,6 +125,7 @@ extern "C" int mxfp8_quantize(const void* in, int dtype, int64_t rows, int64_t c
     if (scale_mode != MOE_SCALE_F32 && scale_mode != MOE_SCALE_E8M0) return MOE_ERR_INVALID;
     if (rows == 0) return MOE_OK;
     if (!in || !q || !scales || !aligned16(in) || !aligned16(q)) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     const int64_t nb = rows * (cols / 32);
     cudaStream_t st = as_stream(stream);
     const int g = mx::grid_for(nb);
@@ -148,6 +149,7 @@ extern "C" int mxfp8_dequantize(const uint8_t* q, const void* scales, int scale_
     if (scale_mode != MOE_SCALE_F32 && scale_mode != MOE_SCALE_E8M0) return MOE_ERR_INVALID;
     if (rows == 0) return MOE_OK;
     if (!q || !scales || !out_bf16 || !aligned16(q) || !aligned16(out_bf16)) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     const int64_t nb = rows * (cols / 32);
     cudaStream_t st = as_stream(stream);
     const int g = mx::grid_for(nb);

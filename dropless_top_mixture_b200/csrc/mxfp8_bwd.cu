@@ -202,6 +202,7 @@ extern "C" int mxfp8_quantize_weights_bwd(const void* W1, const void* W3, const 
         if (!p || !aligned16(p)) return MOE_ERR_INVALID;
     if ((w13_expert_stride < F * d || w2_expert_stride < F * d) && E > 1) return MOE_ERR_INVALID;
     if (w13_expert_stride < 0 || w2_expert_stride < 0) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     cudaStream_t st = as_stream(stream);
     // W1_e, W3_e [F, d] -> rows i of [E, d, 2F]: (W1_e[:, i] | W3_e[:, i]) along F
     int rc = mxb::transpose_quant(W1, w13_expert_stride, E, F, d, W13tq, W13ts, 2 * F, 0, st);
@@ -224,6 +225,7 @@ extern "C" int moe_swiglu_bwd_mxfp8(const void* dH, const void* A, const void* B
     const int64_t n = R * (F / 32);
     const int64_t blocks = (n + 255) / 256;
     if (blocks > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     mxb::swiglu_bwd_quant_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(
         static_cast<const __nv_bfloat16*>(dH), static_cast<const __nv_bfloat16*>(A),
         static_cast<const __nv_bfloat16*>(B), R, (int)F, static_cast<__nv_bfloat16*>(dA),
@@ -236,6 +238,12 @@ extern "C" size_t moe_layer_bwd_mxfp8_workspace_size(int64_t T, int64_t d, int64
     if (T < 0 || d <= 0 || E <= 0 || F <= 0 || k <= 0) return 0;
     return mxb::carve(nullptr, T, d, E, F, k).total;
 }
+
+namespace moe {
+namespace mxb {
+static int bwd_steps(const moe_layer_bwd_mxfp8_args* a, const Carve& c, void* stream);
+}  // namespace mxb
+}  // namespace moe
 
 extern "C" int moe_layer_bwd_mxfp8(const moe_layer_bwd_mxfp8_args* a, void* stream) {
     if (!a) return MOE_ERR_INVALID;
@@ -259,6 +267,14 @@ extern "C" int moe_layer_bwd_mxfp8(const moe_layer_bwd_mxfp8_args* a, void* stre
         if (!aligned16(p)) return MOE_ERR_INVALID;
     if (a->T * a->k > INT32_MAX - 256 || a->d > (1 << 24) || 2 * a->F > (1 << 24))
         return MOE_ERR_UNSUPPORTED;
+    return checked([&] { return mxb::bwd_steps(a, c, stream); });
+}
+
+namespace moe {
+namespace mxb {
+
+// The steps of moe_layer_bwd_mxfp8 after its own checks.
+static int bwd_steps(const moe_layer_bwd_mxfp8_args* a, const Carve& c, void* stream) {
     const int64_t T = a->T, d = a->d, E = a->E, F = a->F, R = a->T * a->k;
     int rc;
     if (R > 0) {
@@ -294,3 +310,6 @@ extern "C" int moe_layer_bwd_mxfp8(const moe_layer_bwd_mxfp8_args* a, void* stre
     return swiglu_wgrad(c.dXe, c.dA, c.dB, c.dYe, c.dH, a->offsets, E, R, d, F, a->dW1, a->dW3,
                         a->dW2, as_stream(stream));
 }
+
+}  // namespace mxb
+}  // namespace moe

@@ -582,6 +582,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
                   uint8_t* os, __nv_bfloat16* ob, int64_t ldo, cudaStream_t st,
                   void* save_a = nullptr, void* save_b = nullptr) {
     auto kern = mx_gemm_kernel<SWIGLU>;
+    if (check_only()) return MOE_OK;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -617,6 +618,7 @@ extern "C" int moe_dispatch_mxfp8(const void* x, const int32_t* slot, int64_t T,
     if (T == 0) return MOE_OK;
     if (!x || !slot || !Xq || !Xs || !aligned16(x) || !aligned16(Xq)) return MOE_ERR_INVALID;
     if (T * k > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     const int64_t n = T * (d / 32);
     int64_t g = (n + 255) / 256;
     const int64_t cap = (int64_t)num_sms() * 16;
@@ -645,6 +647,7 @@ extern "C" int mxfp8_pack_weight_scales(const uint8_t* W1s, const uint8_t* W3s,
         return MOE_ERR_INVALID;
     if ((W2s == nullptr) != (Ps2 == nullptr)) return MOE_ERR_INVALID;
     if ((Ps13 && !aligned16(Ps13)) || (Ps2 && !aligned16(Ps2))) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     cudaStream_t st = as_stream(stream);
     const int64_t cap = (int64_t)num_sms() * 8;
     if (Ps13) {  // gate/up tiles: 128 rows of W1 + 128 of W3 per n-block, K = d
@@ -674,6 +677,7 @@ static int act_scales(const uint8_t* src, const int32_t* offsets, int64_t E, int
     if (R == 0) return MOE_OK;
     if (!src || !dst || !offsets) return MOE_ERR_INVALID;
     if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     const int ks = (int)(K / 128);
     const int64_t words = (R / mxg::BM + E) * ks * 128;
     // about one word per thread: each word is a dependent load and store

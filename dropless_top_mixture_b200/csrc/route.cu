@@ -51,6 +51,9 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async_wait_one() {  // all but the newest group
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // 16 consecutive fp32 elements of a row landed in shared memory, to registers.
 __device__ __forceinline__ void landed16_to_f32(const uint4* p, float* f) {
@@ -182,6 +185,15 @@ __global__ void __launch_bounds__(LOGIT_THREADS, 8) router_logits_kernel(
 // with TMA through an RT_STAGES ring, warp 1 lane 0 issues 4 MMAs per slab,
 // warps 2..5 read the accumulator (one TMEM lane quarter each) and store fp32
 // rows, masked to T and E. Every wait is bounded as in the grouped GEMMs.
+//
+// While the slabs sit in shared memory the four epilogue warps also sum the
+// squares of their rows: thread r of the A tile gives ||x_t||^2 for token
+// m0 + r (CTAs with blockIdx.y == 0), and in CTAs with blockIdx.x == 0 the
+// B tile's rows give ||w_e||^2. Each is an fp32 sum of exact squares in
+// ascending j, so it is at most d 2^-24 (relatively) below the true value;
+// the refinement below turns them into a bound on the logit error. A stage
+// is free again once the MMAs (one commit) and the four epilogue warps (one
+// arrival each) are done with it.
 constexpr int RT_BM = 128;
 constexpr int RT_THREADS = 192;
 
@@ -201,7 +213,8 @@ template <int EN>
 __global__ void __launch_bounds__(RT_THREADS, 1)
     router_logits_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                             const __grid_constant__ CUtensorMap tmW, int T, int d, int E,
-                            float* __restrict__ logits, int vec, int* status) {
+                            float* __restrict__ logits, int vec, float* __restrict__ xnorm2,
+                            float* __restrict__ wnorm2, int* status) {
     using namespace tc;
     using C = RtCfg<EN>;
     extern __shared__ uint8_t smem_raw[];
@@ -222,7 +235,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     if (tid == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(smem_u32(full + s), 1);
-            mbar_init(smem_u32(empty + s), 1);
+            mbar_init(smem_u32(empty + s), 1 + 4);  // MMA commit + 4 epilogue warps
         }
         mbar_init(smem_u32(done), 1);
         mbar_init(smem_u32(drain), 1);
@@ -303,7 +316,65 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;
-        if (mbar_wait(smem_u32(done), 0, s_abort, status, WAIT_LIMIT_NS)) {
+        const int r = q * 32 + lane;           // A row (token m0 + r)
+        const int er = (warp - 2) * 32 + lane;  // B rows er and er + 128
+        const bool do_x = blockIdx.y == 0, do_w = blockIdx.x == 0;
+        float sx = 0.f, sw0 = 0.f, sw1 = 0.f;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int kb = 0; kb < KS; ++kb) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* st_base = smem + stage * C::STAGE_BYTES;
+            // 128-byte rows with the 128-byte swizzle: logical 16-byte chunk c
+            // of row r sits at chunk c ^ (r & 7); the chunks are read in
+            // logical order, so the sums run in ascending j
+            if (do_x) {
+                const uint8_t* rowp = st_base + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4*>(rowp + 16 * (c ^ (r & 7))), f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sx = fmaf(f[i], f[i], sx);
+                }
+            }
+            if (do_w) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int br = er + 128 * h;
+                    if (br < EN) {
+                        const uint8_t* rowp = st_base + C::A_BYTES + br * 128;
+                        float acc = h ? sw1 : sw0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float f[8];
+                            unpack8(*reinterpret_cast<const uint4*>(rowp + 16 * (c ^ (br & 7))), f);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc = fmaf(f[i], f[i], acc);
+                        }
+                        if (h) sw1 = acc; else sw0 = acc;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(empty + stage));
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (ok) {
+            if (do_x && m0 + r < T) xnorm2[m0 + r] = sx;
+            if (do_w) {
+                if (er < EN && n0 + er < E) wnorm2[n0 + er] = sw0;
+                if (er + 128 < EN && n0 + er + 128 < E) wnorm2[n0 + er + 128] = sw1;
+            }
+        }
+        if (ok && mbar_wait(smem_u32(done), 0, s_abort, status, WAIT_LIMIT_NS)) {
             tc_fence_after();
             const int t = m0 + q * 32 + lane;
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -342,7 +413,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 
 template <int EN>
 static int launch_router_tc(const void* x, const void* Wr, int64_t T, int64_t d, int64_t E,
-                            float* logits, cudaStream_t st) {
+                            float* logits, float* xnorm2, float* wnorm2, cudaStream_t st) {
     using C = RtCfg<EN>;
     auto kern = router_logits_tc_kernel<EN>;
     static bool attr_done[64] = {false};
@@ -361,8 +432,341 @@ static int launch_router_tc(const void* x, const void* Wr, int64_t T, int64_t d,
     const int vec = (E % 4 == 0) && aligned16(logits);
     dim3 grid((unsigned)((T + RT_BM - 1) / RT_BM), (unsigned)((E + EN - 1) / EN));
     kern<<<grid, RT_THREADS, C::SMEM_BYTES, st>>>(mx, mw, (int)T, (int)d, (int)E, logits, vec,
-                                                  status_ptr());
+                                                  xnorm2, wnorm2, status_ptr());
     return MOE_OK;
+}
+
+// ------------------------------------------------------------------ a0, bf16: decisions in the fixed order
+//
+// The top-k must select exactly what it selects on the fixed-order logits f
+// (four fmaf chains over the quarters of j, added in order, as for the fp32
+// router). The tensor-core logit v of (t, e) and f are both fp32 sums of the
+// same d exact products, in different orders, so they differ by at most
+//     B_t = 2 d 2^-23 ||x_t|| max_e ||w_e||.
+// Reasoning: with P = sum_j |x_j w_j| <= ||x_t|| ||w_e|| (Cauchy-Schwarz),
+// four in-order fp32 chains of d/4 terms and three adds err by at most
+// (d/4 + 3) 2^-24 P; a tcgen05 kind::f16 instruction adds 16 exact products
+// to the fp32 accumulator losing at most one unit in the 2^-23 place of the
+// largest of its 17 addends for each addend, plus one rounding of the sum,
+// i.e. at most 18 2^-23 P per instruction over d/16 instructions; the total
+// 1.25 d 2^-23 P is rounded up to 2 d 2^-23 P, and the norms (fp32 sums of
+// exact squares) are enlarged by d 2^-23 before the square root.
+//
+// If |v_a - v_b| > 2 B_t, the order of a and b is the same under v and
+// under f. So the refinement writes f over v for every expert whose order
+// against another "candidate" of the token is not decided by v, where the
+// candidates are the experts with v >= (k-th largest v) - 2 B_t: every other
+// expert lies below each of the k experts that v ranks highest under both v
+// and f. Every comparison the top-k makes between the mixed values then
+// agrees with the one it makes on f (ties included, which can only occur
+// between two rewritten values), so idx, the order of j and therefore all
+// routing metadata equal those of the fixed-order logits. Gates are taken
+// from the mixed values. A token whose bound is not finite (an inf or NaN in
+// x or Wr) has all of its logits rewritten.
+//
+// One CTA handles RF_TOK tokens.
+// Phase 1: a group of G lanes per token (32/G tokens per warp at a time),
+// each lane holding the logits of experts g, g + G, ... in registers: k + 1
+// rounds of a group maximum give the k + 1 largest v in descending order;
+// listed are the winners among the first k whose neighbour in that order
+// lies within 2 B_t, and every other expert within 2 B_t below the k-th.
+// Phase 2: the tokens, ordered by the length of their lists so that a
+// warp's tokens carry similar counts, go to 8 threads each: (quarter q,
+// half h), the thread running the fmaf chains of quarter q for the listed
+// experts h, h + 2, ... (up to RF_NPT at once, in registers, sharing its x
+// values). The weight columns of each step (all experts, 4 quarters, RF_CK
+// columns) are staged in shared memory by coalesced cp.async, double
+// buffered; the four quarter sums of an expert meet by shuffles and are
+// added ((c0 + c1) + c2) + c3.
+constexpr int RF_TOK = 32;
+constexpr int RF_THREADS = 256;  // 8 per token in phase 2
+constexpr int RF_NPT = 8;        // listed experts per thread per pass (16 per token)
+
+__host__ __device__ constexpr int rf_group_of(int E) {
+    return E <= 8 ? 1 : E <= 16 ? 2 : E <= 32 ? 4 : E <= 64 ? 8 : E <= 128 ? 16 : 32;
+}
+// columns of each quarter staged per step, and the pitch of a staged row
+__host__ __device__ constexpr int rf_ck(int E) { return E <= 64 ? 32 : E <= 128 ? 16 : 8; }
+__host__ __device__ constexpr int rf_pitch(int E) { return 2 * rf_ck(E) + 16; }
+inline size_t rf_smem_bytes(int64_t E) {
+    return 2 * (size_t)E * 4 * (size_t)rf_pitch((int)E)       // phase 2 stages
+           + sizeof(int16_t) * (size_t)RF_TOK * (size_t)E;  // per-token lists
+}
+
+__device__ __forceinline__ float rf_key(float a) { return a == a ? a : -INFINITY; }
+
+// 8 bf16 (a 16-byte vector, element 0 in the low half of the first word)
+// to fp32: one shift or mask per element, exact.
+__device__ __forceinline__ void rf_unpack8(const uint4& u, float* f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// One staged step of NP chains (branch-free, so the chains interleave):
+// acc[p] runs fmaf over x[j] * w_p[j] for the step's CK columns in
+// ascending j; x comes from registers, w_p from the staged row at woff[p].
+template <int NP, int CK>
+__device__ __forceinline__ void rf_step(const uint4* xv, const unsigned char* wbase,
+                                        const uint32_t* woff, float* acc) {
+#pragma unroll
+    for (int j8 = 0; j8 < CK / 8; ++j8) {
+        float xf[8];
+        rf_unpack8(xv[j8], xf);
+        uint4 wv[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+            wv[p] = *reinterpret_cast<const uint4*>(wbase + woff[p] + 16 * j8);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            float wf[8];
+            rf_unpack8(wv[p], wf);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[p] = fmaf(xf[j], wf[j], acc[p]);
+        }
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(RF_THREADS, 3) refine_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr,
+    const float* __restrict__ xnorm2, const float* __restrict__ wnorm2, int T, int d, int E,
+    int k, float* __restrict__ logits) {
+    // logits per lane: rf_group_of gives G lanes to at most 8 G experts (16 G at G = 32)
+    constexpr int VPL = G == 32 ? MOE_MAX_EXPERTS / 32 : 8;
+    extern __shared__ __align__(16) unsigned char rf_smem[];
+    unsigned char* s_w = rf_smem;  // [2][E][4][pitch]: phase 2 stages
+    int16_t* s_list = reinterpret_cast<int16_t*>(
+        rf_smem + 2 * (size_t)E * 4 * rf_pitch(E));  // [RF_TOK][E]: listed experts
+    __shared__ int s_na[RF_TOK];
+    __shared__ int s_order[RF_TOK];
+    __shared__ int s_win_e[RF_TOK * (MOE_MAX_TOPK + 1)];
+    __shared__ float s_win_v[RF_TOK * (MOE_MAX_TOPK + 1)];
+    __shared__ int s_maxna;
+    __shared__ float s_wmax;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.x * RF_TOK;
+
+    if (warp == 0) {
+        float m = 0.f;
+        for (int e = lane; e < E; e += 32) {
+            const float v = wnorm2[e];
+            m = v == v ? fmaxf(m, v) : INFINITY;  // a NaN norm leaves no finite bound
+        }
+        m = warp_max(m);
+        if (lane == 0) s_wmax = m;
+    }
+    if (tid < RF_TOK) s_na[tid] = 0;
+    __syncthreads();
+    const float infl = 1.f + (float)d * 0x1p-23f;
+    const float wn = sqrtf(s_wmax * infl);
+
+    // ---------------------------------------------------------- phase 1
+    const int g = lane % G;
+    for (int tl = tid / G; tl < RF_TOK; tl += RF_THREADS / G) {
+        const int t = t0 + tl;
+        int16_t* lst = s_list + (size_t)tl * E;
+        const bool live = t < T;  // the same on every lane of the group
+        float v[VPL];
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = g + G * i;
+            v[i] = (live && e < E) ? rf_key(logits[(size_t)t * E + e]) : -INFINITY;
+        }
+        const float xn = live ? sqrtf(xnorm2[t] * infl) : 0.f;
+        const float gap = 4.f * (float)d * 0x1p-23f * xn * wn * (1.f + 0x1p-20f);  // 2 B_t
+        const bool all = live && !(gap <= 3.0e38f);  // no finite bound: every expert
+        // k + 1 rounds of a group maximum (lower expert first on ties), each
+        // retiring the winner: the k + 1 largest v in descending order
+        int* win_e = s_win_e + tl * (MOE_MAX_TOPK + 1);
+        float* win_v = s_win_v + tl * (MOE_MAX_TOPK + 1);
+        uint32_t taken = 0, top = 0;  // top: this lane's experts among the first k
+        const int rounds = k < E ? k + 1 : k;
+        for (int r = 0; r < rounds; ++r) {
+            if (r == k) top = taken;
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = g + G * i;
+                if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || v[i] > bv)) {
+                    bv = v[i];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            if (be < E && be % G == g) taken |= 1u << (be / G);
+            if (g == 0) {
+                win_e[r] = be;
+                win_v[r] = bv;
+            }
+        }
+        if (rounds == k) {  // k == E: nothing lies below the k-th
+            top = taken;
+            if (g == 0) win_v[k] = -INFINITY;
+        }
+        __syncwarp();
+        // Listed: every expert when there is no finite bound; else each of the
+        // k winners whose neighbour in the descending order lies within 2 B_t,
+        // and every other expert within 2 B_t below the k-th winner (which
+        // is then listed too). A difference of two nearby floats is exact,
+        // so the tests below round nothing that could move an expert across
+        // the 2 B_t line.
+        if (live) {
+            const float kth = win_v[k - 1];
+            for (int r = g; r < k; r += G) {
+                const float vr = win_v[r];
+                const bool a = all || (r > 0 && win_v[r - 1] - vr <= gap) ||
+                               (vr - win_v[r + 1] <= gap);
+                if (a) lst[atomicAdd(&s_na[tl], 1)] = (int16_t)win_e[r];
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = g + G * i;
+                if (e < E && !((top >> i) & 1u) && (all || kth - v[i] <= gap))
+                    lst[atomicAdd(&s_na[tl], 1)] = (int16_t)e;
+            }
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    if (tid < RF_TOK) {
+        // rank by descending count (ties by token): s_order[rank] = token
+        const int mine = s_na[tid];
+        int rank = 0;
+        for (int j = 0; j < RF_TOK; ++j) {
+            const int o = s_na[j];
+            rank += (o > mine) || (o == mine && j < tid);
+        }
+        s_order[rank] = tid;
+        if (rank == 0) s_maxna = mine;
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------- phase 2
+    const int maxna = s_maxna;
+    if (maxna == 0) return;
+    const int tl = s_order[tid >> 3];
+    const int q = (tid >> 1) & 3, h = tid & 1;
+    const int t = t0 + tl;
+    const int na = s_na[tl];
+    const int dq = d >> 2;
+    constexpr int CK = G <= 8 ? 32 : G == 16 ? 16 : 8;  // rf_ck(E) for the E this G serves
+    const int pitch = rf_pitch(E);
+    const int nsteps = dq / CK;
+    const int chunks = E * 4 * (CK / 8);  // 16-byte pieces of one stage
+    const uint32_t sw = smem_u32(s_w);
+    const uint32_t stage_bytes = (uint32_t)E * 4u * (uint32_t)pitch;
+    static_assert(RF_NPT == 8, "rf_step dispatch covers 1..8 chains");
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(t < T ? t : 0) * d + (size_t)q * dq);
+    auto stage = [&](int step, int buf) {
+        const int c0 = step * CK;
+        for (int i = tid; i < chunks; i += RF_THREADS) {
+            const int row = i / (CK / 8), part = i - row * (CK / 8);  // row = 4 e + quarter
+            const __nv_bfloat16* src =
+                Wr + (size_t)(row >> 2) * d + (size_t)(row & 3) * dq + c0 + 8 * part;
+            cp_async16(sw + buf * stage_bytes + row * pitch + 16 * part, src, 16);
+        }
+        cp_async_commit();
+    };
+    for (int pbase = 0; pbase < maxna; pbase += 2 * RF_NPT) {
+        int cnt = 0;
+        int ep[RF_NPT];
+        uint32_t woff[RF_NPT];
+#pragma unroll
+        for (int p = 0; p < RF_NPT; ++p) {
+            const int pi = pbase + 2 * p + h;
+            ep[p] = pi < na ? (int)s_list[(size_t)tl * E + pi] : 0;
+            woff[p] = (uint32_t)(ep[p] * 4 + q) * (uint32_t)pitch;  // expert 0 for unused slots
+            if (pi < na) cnt = p + 1;
+        }
+        // chains per thread in this warp (the rest compute and drop expert 0's)
+        const int npw = __reduce_max_sync(0xffffffffu, (unsigned)cnt);
+        float acc[RF_NPT];
+#pragma unroll
+        for (int p = 0; p < RF_NPT; ++p) acc[p] = 0.f;
+        __syncthreads();  // the previous pass is done with both stage buffers
+        stage(0, 0);
+        for (int st = 0; st < nsteps; ++st) {
+            uint4 xv[CK / 8];
+            if (npw > 0) {
+#pragma unroll
+                for (int u = 0; u < CK / 8; ++u) xv[u] = xr[(st * CK) / 8 + u];
+            }
+            if (st + 1 < nsteps) {
+                stage(st + 1, (st + 1) & 1);
+                cp_async_wait_one();
+            } else {
+                cp_async_wait_all();
+            }
+            __syncthreads();
+            const unsigned char* wb = s_w + (st & 1) * stage_bytes;
+            switch (npw) {
+                case 0: break;
+                case 1: rf_step<1, CK>(xv, wb, woff, acc); break;
+                case 2: rf_step<2, CK>(xv, wb, woff, acc); break;
+                case 3: rf_step<3, CK>(xv, wb, woff, acc); break;
+                case 4: rf_step<4, CK>(xv, wb, woff, acc); break;
+                case 5: rf_step<5, CK>(xv, wb, woff, acc); break;
+                case 6: rf_step<6, CK>(xv, wb, woff, acc); break;
+                case 7: rf_step<7, CK>(xv, wb, woff, acc); break;
+                default: rf_step<8, CK>(xv, wb, woff, acc); break;
+            }
+            __syncthreads();  // before the next stage overwrites this buffer
+        }
+        // quarters q = 0..3 of (token, h) are lanes 8m + 2q + h
+#pragma unroll
+        for (int p = 0; p < RF_NPT; ++p) {
+            const float c1 = __shfl_sync(0xffffffffu, acc[p], lane + 2);
+            const float c2 = __shfl_sync(0xffffffffu, acc[p], lane + 4);
+            const float c3 = __shfl_sync(0xffffffffu, acc[p], lane + 6);
+            if (q == 0 && p < cnt && t < T) logits[(size_t)t * E + ep[p]] = ((acc[p] + c1) + c2) + c3;
+        }
+    }
+}
+
+template <int G>
+static int launch_refine(const void* x, const void* Wr, const float* xnorm2, const float* wnorm2,
+                         int64_t T, int64_t d, int64_t E, int k, float* logits, cudaStream_t st) {
+    auto kern = refine_kernel<G>;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)rf_smem_bytes(MOE_MAX_EXPERTS)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const unsigned grid = (unsigned)((T + RF_TOK - 1) / RF_TOK);
+    kern<<<grid, RF_THREADS, rf_smem_bytes(E), st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr), xnorm2,
+        wnorm2, (int)T, (int)d, (int)E, k, logits);
+    return MOE_OK;
+}
+
+static int launch_refine_any(const void* x, const void* Wr, const float* xnorm2,
+                             const float* wnorm2, int64_t T, int64_t d, int64_t E, int k,
+                             float* logits, cudaStream_t st) {
+    switch (rf_group_of((int)E)) {
+        case 1: return launch_refine<1>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+        case 2: return launch_refine<2>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+        case 4: return launch_refine<4>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+        case 8: return launch_refine<8>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+        case 16: return launch_refine<16>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+        default: return launch_refine<32>(x, Wr, xnorm2, wnorm2, T, d, E, k, logits, st);
+    }
 }
 
 // ------------------------------------------------------------------ a1
@@ -661,6 +1065,8 @@ struct RouteWs {
     int32_t* count;
     int32_t* ticket;
     float* planes;  // four [T,E] planes when the logits are computed
+    float* xnorm2;  // [T] squared row norms of x (bf16 router)
+    float* wnorm2;  // [E] squared row norms of Wr (bf16 router)
 };
 
 // from_x: the logits are computed from x and Wr; the workspace then also
@@ -672,7 +1078,10 @@ inline int64_t plane_stride(int64_t T, int64_t E) { return (T * E + 63) / 64 * 6
 inline size_t workspace_bytes(int64_t T, int64_t E, bool from_x) {
     size_t b = align256(sizeof(int32_t) * (size_t)E * (size_t)max_chunks_of(T));
     b += 256;  // ticket
-    if (from_x) b += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
+    if (from_x) {
+        b += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
+        b += align256(sizeof(float) * (size_t)T) + align256(sizeof(float) * (size_t)E);
+    }
     return b;
 }
 
@@ -683,20 +1092,41 @@ inline RouteWs carve(void* ws, int64_t T, int64_t E, bool from_x) {
     p += align256(sizeof(int32_t) * (size_t)E * (size_t)max_chunks_of(T));
     r.ticket = reinterpret_cast<int32_t*>(p);
     p += 256;
-    r.planes = from_x ? reinterpret_cast<float*>(p) : nullptr;
+    r.planes = nullptr;
+    r.xnorm2 = r.wnorm2 = nullptr;
+    if (from_x) {
+        r.planes = reinterpret_cast<float*>(p);
+        p += align256(sizeof(float) * (size_t)LOGIT_SPLIT * (size_t)plane_stride(T, E));
+        r.xnorm2 = reinterpret_cast<float*>(p);
+        p += align256(sizeof(float) * (size_t)T);
+        r.wnorm2 = reinterpret_cast<float*>(p);
+    }
     return r;
 }
 
-// Launches the top-k for E experts; returns the chunk size (tokens per
-// chunk) or 0 if E is outside 1..512.
-static int launch_topk(const float* src, int nplanes, int64_t pstride, int T, int E, int k,
-                       int renorm, float* logits_out, int32_t* idx, float* gate, int32_t* rank,
-                       int32_t* wsc, cudaStream_t st) {
-    int G = 1;
-    while (32 * G < E) G *= 2;
+// Shape of the top-k launch for (T, E): lanes per token G, logits per lane
+// V and tokens per chunk; chunk = 0 if no instantiation serves E.
+struct TopkCfg {
+    int G, V, chunk;
+};
+static TopkCfg topk_config(int64_t T, int64_t E) {
+    TopkCfg c{1, 0, 0};
+    if (E < 1 || E > MOE_MAX_EXPERTS) return c;
+    while (32 * c.G < E) c.G *= 2;
     const int64_t want_threads = (int64_t)num_sms() * 1024;
-    while (G < TOPK_MAX_G && (int64_t)T * G < want_threads && E >= 16 * G) G *= 2;
-    const int V = ((E + G - 1) / G + 7) / 8 * 8;
+    while (c.G < TOPK_MAX_G && T * c.G < want_threads && E >= 16 * c.G) c.G *= 2;
+    c.V = (int)(((E + c.G - 1) / c.G + 7) / 8 * 8);
+    if (c.G > TOPK_MAX_G || c.V < 8 || c.V > 32) return c;
+    c.chunk = topk_threads_of(c.G) / c.G;
+    return c;
+}
+
+// Launches the top-k with the shape topk_config chose; returns the chunk
+// size (tokens per chunk).
+static int launch_topk(const TopkCfg& cfg, const float* src, int nplanes, int64_t pstride, int T,
+                       int E, int k, int renorm, float* logits_out, int32_t* idx, float* gate,
+                       int32_t* rank, int32_t* wsc, cudaStream_t st) {
+    const int G = cfg.G, V = cfg.V;
     const int nt = topk_threads_of(G);
     const int ch = nt / G;
     const int nch = (T + ch - 1) / ch;
@@ -742,6 +1172,7 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     if (T == 0) {
         // empty batch (an empty logits tensor may well be a null pointer): all
         // counts, offsets and tile offsets are zero
+        if (check_only()) return MOE_OK;
         cudaStream_t st0 = as_stream(stream);
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st0) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st0) != cudaSuccess)
@@ -757,6 +1188,7 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
             return MOE_ERR_INVALID;
         if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
         if (!aligned16(x) || !aligned16(Wr)) return MOE_ERR_INVALID;
+        if (d > (1 << 24)) return MOE_ERR_UNSUPPORTED;
     }
     if (T > 0 && (!idx || !gate || !slot)) return MOE_ERR_INVALID;
     if (!workspace || workspace_bytes < route::workspace_bytes(T, E, from_x))
@@ -764,23 +1196,29 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MOE_ERR_INVALID;
     if (from_x && logits_out && (reinterpret_cast<uintptr_t>(logits_out) & 15u) != 0)
         return MOE_ERR_INVALID;
+    const route::TopkCfg tk = route::topk_config(T, E);
+    if (tk.chunk == 0) return MOE_ERR_UNSUPPORTED;
+    if (check_only()) return MOE_OK;
     cudaStream_t st = as_stream(stream);
     route::RouteWs ws = route::carve(workspace, T, E, from_x);
 
-    int chunk = 0;
     if (from_x && dtype == MOE_BF16) {
-        // tensor cores, fp32 accumulation; the top-k reads the one plane
+        // tensor cores, fp32 accumulation, with the row norms of x and Wr;
+        // then the fixed-order logits of the experts whose order the tensor
+        // core sums cannot decide; the top-k reads the one plane
         float* dst = logits_out ? logits_out : ws.planes;
         int rc = MOE_OK;
         if (E <= 64)
-            rc = route::launch_router_tc<64>(x, Wr, T, d, E, dst, st);
+            rc = route::launch_router_tc<64>(x, Wr, T, d, E, dst, ws.xnorm2, ws.wnorm2, st);
         else if (E <= 128)
-            rc = route::launch_router_tc<128>(x, Wr, T, d, E, dst, st);
+            rc = route::launch_router_tc<128>(x, Wr, T, d, E, dst, ws.xnorm2, ws.wnorm2, st);
         else
-            rc = route::launch_router_tc<256>(x, Wr, T, d, E, dst, st);
+            rc = route::launch_router_tc<256>(x, Wr, T, d, E, dst, ws.xnorm2, ws.wnorm2, st);
         if (rc != MOE_OK) return rc;
-        chunk = route::launch_topk(dst, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate, slot,
-                                   ws.count, st);
+        rc = route::launch_refine_any(x, Wr, ws.xnorm2, ws.wnorm2, T, d, E, k, dst, st);
+        if (rc != MOE_OK) return rc;
+        route::launch_topk(tk, dst, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate, slot,
+                           ws.count, st);
     } else if (from_x) {
         // fp32 router: four fixed-order fmaf chains per logit on the CUDA
         // cores (tf32 tensor cores would round the inputs); the top-k adds
@@ -790,14 +1228,13 @@ extern "C" int moe_route(const float* logits, const void* x, const void* Wr, int
         route::router_logits_kernel<<<grid, route::LOGIT_THREADS, 0, st>>>(
             static_cast<const float*>(x), static_cast<const float*>(Wr), (int)T, (int)d, (int)E,
             ws.planes, route::plane_stride(T, E));
-        chunk = route::launch_topk(ws.planes, route::LOGIT_SPLIT, route::plane_stride(T, E),
-                                   (int)T, (int)E, k, renorm, logits_out, idx, gate, slot,
-                                   ws.count, st);
+        route::launch_topk(tk, ws.planes, route::LOGIT_SPLIT, route::plane_stride(T, E), (int)T,
+                           (int)E, k, renorm, logits_out, idx, gate, slot, ws.count, st);
     } else {
-        chunk = route::launch_topk(logits, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate,
-                                   slot, ws.count, st);
+        route::launch_topk(tk, logits, 1, 0, (int)T, (int)E, k, renorm, nullptr, idx, gate, slot,
+                           ws.count, st);
     }
-    if (chunk == 0) return MOE_ERR_UNSUPPORTED;
+    const int chunk = tk.chunk;
     const int nch = (int)((T + chunk - 1) / chunk);
     if (cudaMemsetAsync(ws.ticket, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     route::scan_kernel<<<(unsigned)E, route::SCAN_THREADS, 0, st>>>(

@@ -538,6 +538,7 @@ extern "C" int moe_aux_loss(const float* logits, const int32_t* counts, int64_t 
     if (!logits || !counts || !aux_out || !workspace) return MOE_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return MOE_ERR_INVALID;
     if (workspace_bytes < moe_aux_loss_workspace_size(T, E)) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     const int nb = rb::aux_blocks(T);
     const int per = (int)((T + nb - 1) / nb);
     const int used = (int)((T + per - 1) / per);
@@ -563,6 +564,7 @@ extern "C" int moe_router_bwd(const void* dOut, const void* Ye, const int32_t* s
     if (!dOut || !Ye || !slot || !idx || !logits || !dlogits) return MOE_ERR_INVALID;
     if (!aligned16(dOut) || !aligned16(Ye)) return MOE_ERR_INVALID;
     if (aux_coef != 0.f && !counts) return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     const double aux_scale = (double)aux_coef * (double)E / ((double)T * (double)T);
     const int vpr = (int)(d * es / 16);
     int64_t g = T;
@@ -622,6 +624,7 @@ extern "C" int moe_router_linear_bwd(const float* dlogits, const void* x, const 
     if (dWr && (!x || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0 ||
                 workspace_bytes < moe_router_linear_bwd_workspace_size(T, d, E)))
         return MOE_ERR_INVALID;
+    if (check_only()) return MOE_OK;
     cudaStream_t st = as_stream(stream);
     const bool tc = dtype == MOE_BF16 && T > 0 && d % 256 == 0 && d <= (1 << 24) &&
                     T <= INT32_MAX - 2 * 128 && (!dx || (aligned16(dx) && aligned16(Wr))) &&

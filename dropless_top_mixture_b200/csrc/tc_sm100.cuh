@@ -310,6 +310,7 @@ inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // 2-D map over a row-major [rows, cols] matrix; box = 128 bytes x box_rows.
 inline bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
                         uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    if (check_only()) return true;  // the check pass encodes no maps
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {cols, rows};
@@ -325,6 +326,7 @@ inline bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
 inline bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es,
                         uint64_t cols, uint64_t rows, uint64_t E, uint64_t estride,
                         uint32_t box_rows) {
+    if (check_only()) return true;  // the check pass encodes no maps
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[3] = {cols, rows, E};

@@ -26,17 +26,24 @@
  *
  * Error behaviour (all calls): arguments are validated on the host before
  * anything is enqueued. MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED mean nothing was
- * launched; for the whole-layer entries (moe_layer_*), which chain the
- * single-step entries, this holds for the checks they make up front (their
- * own arguments and workspace; moe_layer_bwd_mxfp8 checks every step's
- * pointers and sizes too), while a step's own check that fails later, e.g. a
- * weight pointer that is not 16-byte aligned, returns its code with the
- * earlier steps already enqueued and the outputs incomplete. MOE_ERR_CUDA means a launch failed (the CUDA error is left for
- * cudaGetLastError). Faults found on the device (a metadata value out of
- * range, a pipeline wait that exceeded its time limit) set bits in a
- * per-process device status word instead of trapping; the kernel that finds
- * one skips the bad access and returns. Read it with moe_get_status.
- * T == 0 is a valid no-op.
+ * launched. The whole-layer entries (moe_layer_*), which chain the
+ * single-step entries, first run every step's host checks without
+ * enqueuing anything (the *_host entries do so for every token slice), so
+ * an invalid argument of any step, such as a weight pointer of the last
+ * GEMM that is not 16-byte aligned, is reported before the first launch.
+ * MOE_ERR_CUDA means a CUDA call or launch failed (the CUDA error is left for
+ * cudaGetLastError); work enqueued before it stays enqueued. Faults found on
+ * the device (a metadata value out of range, a pipeline wait that exceeded
+ * its time limit) set bits in a per-process device status word instead of
+ * trapping; the kernel that finds one skips the bad access and returns. Read
+ * it with moe_get_status. T == 0 is a valid no-op.
+ *
+ * Per-device state: on its first use on a device the library looks up and
+ * keeps the device status word's address, sets kernel attributes, creates
+ * the host pipeline's events and (moe_route_noalloc) looks up its scratch
+ * array's address. A cudaDeviceReset, or any other teardown of the device's
+ * primary context, invalidates all of it: do not call the library on a
+ * device after resetting it.
  */
 #ifndef DROPLESS_TOP_MIXTURE_B200_MOE_H
 #define DROPLESS_TOP_MIXTURE_B200_MOE_H
@@ -91,14 +98,25 @@ extern "C" {
  *
  * Inputs (device):
  *   logits   [T,E] fp32 row-major, or NULL to compute logits = x·Wrᵀ from
- *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). bf16:
- *            the tensor cores sum the exact bf16 products into fp32, in their
- *            own order (the pages' router is a linear layer in the model
- *            dtype). fp32: the logit of (t,e) is four fp32 accumulators, one
- *            per contiguous quarter of j, each starting from +0.0 and updated
- *            by fused multiply-add in ascending j, then added in order,
- *            ((c0 + c1) + c2) + c3 (tf32 tensor cores would round the
- *            inputs). The top-k is taken on the logits so computed.
+ *   x        [T,d] and Wr [E,d] in `dtype` (MOE_F32 or MOE_BF16). The
+ *            routing is that of the fixed-order logits: the logit of (t,e)
+ *            is four fp32 accumulators, one per contiguous quarter of j,
+ *            each starting from +0.0 and updated by fused multiply-add in
+ *            ascending j, then added in order, ((c0 + c1) + c2) + c3.
+ *            fp32 inputs: computed that way on the CUDA cores (tf32 tensor
+ *            cores would round the inputs). bf16 inputs (the pages' router
+ *            is a linear layer in the model dtype): the tensor cores sum the
+ *            exact products into fp32 in their own order, which differs from
+ *            the fixed-order value by at most B_t = 2 d 2^-23 |x_t| max_e
+ *            |w_e|; every expert of a token whose order against another
+ *            candidate (an expert within 2 B_t of the k-th largest or above)
+ *            is closer than 2 B_t is recomputed in the fixed order, so idx,
+ *            the order of j and all metadata are exactly those of the
+ *            fixed-order logits (finite inputs; a token whose bound is not
+ *            finite has all E logits recomputed). The logits written out
+ *            are the fixed-order values for the recomputed experts and the
+ *            tensor-core sums for the others; the gates are computed from
+ *            them.
  *   renorm   0: gates are the softmax probabilities; 1: divided by their sum.
  * Outputs (device, caller-allocated):
  *   logits_out  [T,E] fp32, or NULL (used only when logits == NULL)
@@ -114,7 +132,8 @@ extern "C" {
  *            logits == NULL); 256-byte aligned device memory (with logits
  *            computed it holds four [T,E] fp32 planes: the fp32 router's
  *            quarter sums, or the bf16 router's logits when logits_out is
- *            NULL). Its contents need not be initialised.
+ *            NULL, and the squared row norms of x and Wr). Its contents need
+ *            not be initialised.
  * Limits: 1 <= k <= min(E, 32), E <= 512; when computing logits d % 128 == 0
  *            and logits_out (if given) 16-byte aligned.
  * ---------------------------------------------------------------------- */
@@ -139,7 +158,7 @@ MOE_API int moe_route(const float* logits, const void* x, const void* Wr, int dt
  *   - Size limit: moe_route_workspace_size(T, E, logits == NULL) must not
  *     exceed MOE_ROUTE_NOALLOC_SCRATCH_BYTES, else MOE_ERR_UNSUPPORTED and
  *     nothing is launched. (E = 64 with logits computed from x fits up to
- *     T = 7,943 tokens; E = 128 with logits given up to T = 131,064; E = 384
+ *     T = 7,913 tokens; E = 128 with logits given up to T = 131,064; E = 384
  *     with logits given up to T = 43,688.)
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
@@ -499,9 +518,13 @@ MOE_API int moe_layer_fwd(const moe_layer_args* args, void* stream);
  *   logits_host [T,E] fp32 host, or NULL when args->logits is NULL
  *   out_host    [T,d] host
  *   stream, stream_h2d, stream_d2h  three distinct streams; when the call
- *               returns, `stream` is ordered after the last copy-out.
+ *               returns, `stream` is ordered after the last copy-out (also
+ *               when it returns MOE_ERR_CUDA part-way: then after every copy
+ *               it had enqueued).
  * The first call on a device creates the events the pipeline uses (kept
- * for the life of the process). No save_* buffers in this mode.
+ * for the life of the process); calls from several host threads on one
+ * device take turns on them (a per-device lock held while a call enqueues).
+ * No save_* buffers in this mode.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_layer_fwd_host(const moe_layer_args* args, const void* x_host,
                                const float* logits_host, void* out_host, int chunks,

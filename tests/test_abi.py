@@ -115,3 +115,132 @@ def test_workspace_sizes_are_consistent(lib):
     ws = m.lib.moe_layer_workspace_size(T, d, E, F, k, m.MOE_BF16, 0)
     R = T * k
     assert ws >= 2 * (R * d * 2 + R * F * 2 // 2) + b
+
+
+def _aligned(nbytes, fill=0):
+    """A zero-offset-aligned (256-byte) numpy byte buffer and its address."""
+    import numpy as np
+    raw = np.full(nbytes + 512, fill, dtype=np.uint8)
+    off = (-raw.ctypes.data) % 256
+    return raw, raw.ctypes.data + off
+
+
+def test_layer_entries_check_every_step_before_launch(lib):
+    """A misaligned weight of a late step (W2 of the down GEMM, dW2 of the
+    weight gradients, W2 codes of the MXFP8 down GEMM) is reported as
+    MOE_ERR_INVALID before the first step is enqueued: the host buffers
+    passed as every output stay as they were (no GPU is touched: every
+    check runs on the host)."""
+    import numpy as np
+    from dropless_top_mixture_b200 import moe as m
+    L = m.lib
+    T, d, E, F, k = 64, 256, 8, 256, 2
+    R = T * k
+    keep = []
+
+    def buf(nbytes, fill=0):
+        raw, p = _aligned(nbytes, fill)
+        keep.append(raw)
+        return raw, p
+
+    _, x = buf(T * d * 2)
+    _, lg = buf(T * E * 4)
+    _, W1 = buf(E * F * d * 2)
+    _, W3 = buf(E * F * d * 2)
+    _, W2 = buf(E * d * F * 2 + 16)
+    outs = {n: buf(sz, 0xA5) for n, sz in (("out", T * d * 2), ("idx", R * 4), ("gate", R * 4),
+                                            ("counts", E * 4), ("offsets", (E + 1) * 4),
+                                            ("slot", R * 4))}
+    ws_bytes = L.moe_layer_workspace_size(T, d, E, F, k, m.MOE_BF16, 1)
+    _, ws = buf(ws_bytes)
+    a = m.LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=m.MOE_BF16, x=x, logits=lg, W1=W1, W3=W3,
+                    W2=W2 + 2, w13_expert_stride=F * d, w2_expert_stride=F * d,
+                    out=outs["out"][1], idx=outs["idx"][1], gate=outs["gate"][1],
+                    counts=outs["counts"][1], offsets=outs["offsets"][1], slot=outs["slot"][1],
+                    workspace=ws, workspace_bytes=ws_bytes)
+    assert L.moe_layer_fwd(ctypes.byref(a), None) == m.MOE_ERR_INVALID
+    for n, (raw, _) in outs.items():
+        assert (raw == 0xA5).all(), n
+    # the sliced host pipeline checks every slice's call before its first copy
+    xh_raw, xh = buf(T * d * 2, 0x11)
+    oh_raw, oh = buf(T * d * 2, 0x5A)
+    lh_raw, lh = buf(T * E * 4)
+    assert L.moe_layer_fwd_host(ctypes.byref(a), xh, lh, oh, 3, 1, 2, 3) == m.MOE_ERR_INVALID
+    assert (oh_raw == 0x5A).all()
+    for n, (raw, _) in outs.items():
+        assert (raw == 0xA5).all(), n
+    a.W2 = W2
+    a.w2_expert_stride = F * d + 3  # not a multiple of 8 elements: the down GEMM rejects it
+    assert L.moe_layer_fwd(ctypes.byref(a), None) == m.MOE_ERR_INVALID
+    for n, (raw, _) in outs.items():
+        assert (raw == 0xA5).all(), n
+
+    # backward: dW2 misaligned (the last GEMM of the chain)
+    grads = {n: buf(sz, 0xC3) for n, sz in (("dx", T * d * 2), ("dW1", E * F * d * 2),
+                                             ("dW3", E * F * d * 2), ("dW2", E * d * F * 2 + 16))}
+    bws = L.moe_layer_bwd_workspace_size(T, d, F, k, m.MOE_BF16)
+    _, bw = buf(bws)
+    _, tok = buf(R * d * 2)
+    _, rowsF = buf(R * F * 2)
+    b = m.LayerBwdArgs(T=T, d=d, E=E, F=F, k=k, dtype=m.MOE_BF16, slot=outs["slot"][1],
+                       gate=outs["gate"][1], offsets=outs["offsets"][1], Xe=tok, A=rowsF,
+                       B=rowsF, H=rowsF, W1=W1, W3=W3, W2=W2, w13_expert_stride=F * d,
+                       w2_expert_stride=F * d, dOut=x, dx=grads["dx"][1], dW1=grads["dW1"][1],
+                       dW3=grads["dW3"][1], dW2=grads["dW2"][1] + 2, workspace=bw,
+                       workspace_bytes=bws)
+    assert L.moe_layer_bwd(ctypes.byref(b), None) == m.MOE_ERR_INVALID
+    for n, (raw, _) in grads.items():
+        assert (raw == 0xC3).all(), n
+
+    # MXFP8 forward: the W2 codes misaligned
+    mws = L.moe_layer_mxfp8_workspace_size(T, d, E, F, k, 1)
+    _, mw = buf(mws)
+    _, q13 = buf(E * F * d)
+    _, q2 = buf(E * d * F + 16)
+    _, ps = buf(1 << 20)
+    f = m.LayerMxArgs(T=T, d=d, E=E, F=F, k=k, x=x, logits=lg, W1q=q13, W3q=q13, Ps13=ps,
+                      W2q=q2 + 1, Ps2=ps, w13_expert_stride=F * d, w2_expert_stride=F * d,
+                      out=outs["out"][1], idx=outs["idx"][1], gate=outs["gate"][1],
+                      counts=outs["counts"][1], offsets=outs["offsets"][1],
+                      slot=outs["slot"][1], workspace=mw, workspace_bytes=mws)
+    assert L.moe_layer_fwd_mxfp8(ctypes.byref(f), None) == m.MOE_ERR_INVALID
+    for n, (raw, _) in outs.items():
+        assert (raw == 0xA5).all(), n
+
+
+@pytest.mark.gpu
+def test_layer_entry_rejects_before_launch_on_device():
+    """The same on the GPU with device buffers: a misaligned W2 returns
+    MOE_ERR_INVALID and idx, the workspace's Xe rows and out keep their
+    sentinel bytes after the stream drains."""
+    import torch
+    from dropless_top_mixture_b200 import moe as m
+    T, d, E, F, k = 256, 256, 8, 256, 2
+    dev = "cuda"
+    x = torch.randn(T, d, device=dev).to(torch.bfloat16)
+    lg = torch.randn(T, E, device=dev)
+    W1 = torch.randn(E, F, d, device=dev).to(torch.bfloat16)
+    W3 = torch.randn(E, F, d, device=dev).to(torch.bfloat16)
+    W2 = torch.randn(E * d * F + 8, device=dev).to(torch.bfloat16)
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = torch.full((T, d), 7.0, dtype=torch.bfloat16, device=dev)
+    idx = torch.full((T, k), -5, **i32)
+    gate = torch.full((T, k), 3.0, device=dev)
+    counts = torch.full((E,), -5, **i32)
+    offsets = torch.full((E + 1,), -5, **i32)
+    slot = torch.full((T, k), -5, **i32)
+    ws_bytes = m.lib.moe_layer_workspace_size(T, d, E, F, k, m.MOE_BF16, 1)
+    ws = torch.full((ws_bytes,), 0x3C, dtype=torch.uint8, device=dev)
+    a = m.LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=m.MOE_BF16, x=x.data_ptr(),
+                    logits=lg.data_ptr(), W1=W1.data_ptr(), W3=W3.data_ptr(),
+                    W2=W2.data_ptr() + 2, w13_expert_stride=F * d, w2_expert_stride=F * d,
+                    out=out.data_ptr(), idx=idx.data_ptr(), gate=gate.data_ptr(),
+                    counts=counts.data_ptr(), offsets=offsets.data_ptr(), slot=slot.data_ptr(),
+                    workspace=ws.data_ptr(), workspace_bytes=ws_bytes)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert m.lib.moe_layer_fwd(ctypes.byref(a), stream) == m.MOE_ERR_INVALID
+    torch.cuda.synchronize()
+    assert (out == 7.0).all() and (idx == -5).all() and (gate == 3.0).all()
+    assert (counts == -5).all() and (offsets == -5).all() and (slot == -5).all()
+    assert (ws == 0x3C).all()  # Xe, H, Ye and the route workspace untouched
+    assert m.moe_get_status() == 0

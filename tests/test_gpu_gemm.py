@@ -7,7 +7,8 @@ import torch
 
 from oracle import moe_oracle as O
 from dropless_top_mixture_b200.workloads import WORKLOADS, adversarial_logits, make_inputs
-from tests._util import assert_close_layer, assert_close_scaled, np64, router_logits_checked
+from tests._util import (assert_close_layer, assert_close_scaled, np64,
+                         route_equals_oracle_own_logits, router_logits_checked)
 
 pytestmark = pytest.mark.gpu
 
@@ -214,6 +215,7 @@ def test_layer_small_full_check(dtype):
     Wr = (torch.randn(E, d, generator=torch.Generator().manual_seed(5)) * 0.05).to(dtype)
     r = moe.moe_layer_fwd(x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda(), Wr=Wr.cuda(), save=True)
     lg = router_logits_checked(r.logits.cpu().numpy(), x, Wr)
+    route_equals_oracle_own_logits(r, x, Wr, k, E)
     ref = O.moe_layer(x, k, W1, W3, W2, logits=lg)
     assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
     assert np.array_equal(r.slot.cpu().numpy(), ref["slot"])
@@ -251,6 +253,8 @@ def test_layer_full_size_sampled(name):
     x_cpu = inp["x"].cpu()
     lg = (router_logits_checked(r.logits.cpu().numpy(), x_cpu, inp["Wr"].cpu()) if router
           else inp["logits"].cpu().numpy())
+    if router:
+        route_equals_oracle_own_logits(r, x_cpu, inp["Wr"].cpu(), w.k, w.E)
     idx, gate, _ = O.route(lg, w.k)
     meta = O.routing_metadata(idx, w.E)
     assert np.array_equal(r.idx.cpu().numpy(), idx)
