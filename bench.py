@@ -2,17 +2,24 @@
 """Benchmark of the dropless top-k MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference]
+                    [--also NAMES] [--impl ours|reference]
 
 One step = one pass of the whole layer over one batch: route (router logits,
 fp32 softmax + top-k, routing metadata) -> dispatch -> grouped gate/up GEMM
 with SwiGLU -> grouped down GEMM -> combine, each through the C ABI.
+The default workload is the 128-expert layer of the expert-count sweep
+(T=8192, d=4096, E=128, top-4, ffn 2048, bf16, logits ~ N(0,1)), the
+configuration the layer's targets are stated on; the OLMoE-shaped layer
+(router from x·Wrᵀ) is timed the same way in the same run and reported
+under "also".
 `value` = tokens/s of the whole job with inputs resident in HBM, timed over
 one replay of the K steps captured in a CUDA graph (the same library calls,
 with CUDA events between the parts captured too, which give the breakdown);
 eager steps with --no-graph (their time is always reported as well);
 `e2e` = the same metric through moe_layer_fwd with the step's input copied
 from pinned host memory and the output copied back inside the timed region.
+`cpu_baseline` / `cpu_baseline_one_thread` = the CPU oracle on a bounded
+sample of the workload, on the host's BLAS threads / on one thread.
 
 Multi-GPU: the layer is run as independent replicas, one process per GPU
 (launched by torch.distributed.run); there is no data-path collective.
@@ -45,7 +52,8 @@ from dropless_top_mixture_b200.workloads import WORKLOADS, make_inputs  # noqa: 
 
 METRIC = "MoE-layer tokens/s and grouped-GEMM TFLOP/s (% of peak) on 1 B200; dispatch GB/s"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "olmoe_1b7b"
+DEFAULT_WORKLOAD = "sweep_e128"
+ALSO_WORKLOAD = "olmoe_1b7b"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -217,21 +225,33 @@ def oracle_sample(w, inp_cpu, S: int, backward: bool = False):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, inp_cpu, target_s: float = 12.0, backward: bool = False):
-    # the MXFP8 oracle quantises each routed expert's whole weights (seconds
-    # per expert on the host), so its sample is a couple of tokens
-    S = 2 if w.mxfp8 else (16 if backward else 64)
-    dt = oracle_sample(w, inp_cpu, S, backward)
-    if dt < target_s / 4 and S < w.T:
-        S = int(min(w.T, max(S + 1, S * target_s / max(dt, 1e-3))))
+def cpu_baseline(w, inp_cpu, target_s: float = 15.0, backward: bool = False, threads=None):
+    """The oracle as it stands on a bounded sample of the workload, on the
+    host's cores (BLAS and OpenMP threads as configured) or, with
+    ``threads``, limited to that many threads."""
+    import contextlib
+    lim = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=threads)
+    with lim:
+        # the MXFP8 oracle quantises each routed expert's whole weights
+        # (seconds per expert on the host), so its sample is a couple of tokens
+        S = 2 if w.mxfp8 else (16 if backward else 64)
+        if threads == 1 and not w.mxfp8:
+            S = max(4, S // 4)
         dt = oracle_sample(w, inp_cpu, S, backward)
+        if dt < target_s / 2 and S < w.T:
+            S = int(min(w.T, max(S + 1, S * target_s / max(dt, 1e-3))))
+            dt = oracle_sample(w, inp_cpu, S, backward)
+        cores = threads if threads is not None else blas_threads()
     what = ("router logits, top-k, routing metadata and the per-token "
             + ("MXFP8 SwiGLU mixture" if w.mxfp8 else "SwiGLU mixture")
             + ((" plus the float64 input gradient of those tokens (no weight gradients)"
                 if w.mxfp8 else " plus the input gradient of those tokens (no weight gradients)")
                if backward else "")
             + " in float64")
-    return {"value": S / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": S / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"first {S} of {w.T} tokens of {w.name}: {what} ({dt:.1f} s)"}
 
 
@@ -480,34 +500,36 @@ def _steps(moe, w, inp, dev, backward):
     # backward), + 4 for the router GEMM backward (dlogits to bf16, dx, dWr
     # chunk partials, their ordered sum; the bf16 router workloads)
     bwd_kernels = (14 if w.mxfp8 else 7) + 2 + 2 + (4 if use_router else 0)
-    kernels = ((4 if use_router else 3) + (5 if w.mxfp8 else 4)
+    # route: (tensor-core logits, fixed-order refinement) + top-k, scan,
+    # finalize
+    kernels = ((5 if use_router else 3) + (5 if w.mxfp8 else 4)
                + (bwd_kernels if backward else 0))
     return [n for n, _ in fns], step, kernels, work, e_act
 
 
-def run_ours(args):
-    rank, world, local = dist_env()
-    dist_init(world, "nccl")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    from dropless_top_mixture_b200 import moe
-
-    w = WORKLOADS[args.workload]
+def _workload(name, args):
+    w = WORKLOADS[name]
     if args.shrink > 1:
         # the same shape per expert (T and E divided together) on a smaller
         # problem, for profiler captures that must stay small
         w = w.scaled(name=f"{w.name}/shrink{args.shrink}", T=max(1, w.T // args.shrink),
                      E=max(w.k, w.E // args.shrink))
-    backward = bool(args.backward)
-    if backward and not w.mxfp8 and w.dtype != "bf16":
+    if args.backward and not w.mxfp8 and w.dtype != "bf16":
         raise SystemExit("--backward runs on the bf16 and MXFP8 workloads")
-    if backward and not w.backward:
+    if args.backward and not w.backward:
         w = w.scaled(name=w.name, backward=True)  # adds the upstream gradient dOut
+    return w
+
+
+def _measure(moe, w, args, rank, world, local, dev, full: bool):
+    """Warm up, time K steps of workload ``w`` (graph replay, else eager) and,
+    when ``full``, the clocks and the end-to-end run. Returns the raw
+    figures; the caller turns them into the JSON line."""
+    backward = bool(args.backward)
     inp = make_inputs(w, dev)
-    T, d, E, k, F, R = w.T, w.d, w.E, w.k, w.F, w.R
     parts, step, kernels_per_step, work, e_act = _steps(moe, w, inp, dev, backward)
 
-    sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    sampler = ClockSampler(local) if (full and rank == 0 and not args.no_clocks) else None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -536,6 +558,7 @@ def run_ours(args):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     per = None
+    w0 = w1 = None
     if graph is not None:
         graph.replay()  # untimed: the K captured steps once more
         torch.cuda.synchronize(dev)
@@ -573,8 +596,6 @@ def run_ours(args):
     else:
         ms_total = ms_graph
         launch = "CUDA graph of the K steps (same library calls), replayed once"
-    ms_step = ms_total / args.steps
-    value = T * world * args.steps / (ms_total / 1e3)
 
     # clocks: the timed window; if it held too few samples, keep running
     # untimed steps of the same workload while sampling
@@ -596,16 +617,24 @@ def run_ours(args):
 
     # end to end through the public layer calls with host buffers
     e2e = None
-    if not args.no_e2e:
+    if full and not args.no_e2e:
         e2e = _e2e(moe, w, inp, dev, world, args, backward)
 
     if moe.moe_get_status() != 0:
         raise RuntimeError("device status word set during the timed region")
     if sampler is not None:
         sampler.stop()
-    if rank != 0:
-        return 0
+    inp_cpu = ({kk: v.cpu() for kk, v in inp.items()}
+               if full and rank == 0 and world == 1 and not args.no_cpu_baseline else None)
+    return dict(parts=parts, per=per, work=work, e_act=e_act, ms_total=ms_total,
+                ms_eager=ms_eager, launch=launch, clocks=clocks, e2e=e2e,
+                kernels_per_step=kernels_per_step, inp_cpu=inp_cpu)
 
+
+def _rates(w, m):
+    """Per-part rates, the roofline of the dominant GEMM and the HBM
+    fractions of dispatch and combine."""
+    parts, per, work = m["parts"], m["per"], m["work"]
     peaks, peak_src = measured_peaks()
     hbm = peaks["hbm_gbs"]
     bf16_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -647,23 +676,65 @@ def run_ours(args):
     roof["traffic"] = recorded_traffic(dom, w.name)
     ffn_t = (per["gate_up"] + per["down"]) / 1e3
     ffn_tf = (work["gate_up"][0] + work["down"][0]) / ffn_t / 1e12
+    grouped = {"ffn_tflops": ffn_tf, "ffn_frac_of_peak": ffn_tf / peak_tf,
+               "peak_tflops": peak_tf, "experts_with_rows": m["e_act"]}
+    hbm_fr = {"dispatch_frac": rates["dispatch"]["gbs"] / hbm,
+              "combine_frac": rates["combine"]["gbs"] / hbm, "peak_gbs": hbm}
+    return rates, roof, grouped, hbm_fr
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    dist_init(world, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from dropless_top_mixture_b200 import moe
+
+    w = _workload(args.workload, args)
+    backward = bool(args.backward)
+    m = _measure(moe, w, args, rank, world, local, dev, full=True)
+    # a second workload, device-timed only (the same step, K and W)
+    also = {}
+    for name in ([] if args.also in ("", "none") else args.also.split(",")):
+        if name == args.workload:
+            continue
+        wa = _workload(name, args)
+        ma = _measure(moe, wa, args, rank, world, local, dev, full=False)
+        also[wa.name] = (wa, ma)
+    if rank != 0:
+        return 0
+
+    ms_step = m["ms_total"] / args.steps
+    value = w.T * world * args.steps / (m["ms_total"] / 1e3)
+    rates, roof, grouped, hbm_fr = _rates(w, m)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if w.mxfp8 else ("bf16" if w.dtype == "bf16" else "f32"),
         "data": "synthetic", "config": config_of(w, world, backward), "roofline": roof,
-        "breakdown": rates,
-        "grouped_gemm": {"ffn_tflops": ffn_tf, "ffn_frac_of_peak": ffn_tf / peak_tf,
-                         "peak_tflops": peak_tf, "experts_with_rows": e_act},
-        "hbm": {"dispatch_frac": rates["dispatch"]["gbs"] / hbm,
-                "combine_frac": rates["combine"]["gbs"] / hbm, "peak_gbs": hbm},
-        "e2e": e2e, "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
-        "launch": launch, "ms_per_step_eager": ms_eager / args.steps,
+        "breakdown": rates, "grouped_gemm": grouped, "hbm": hbm_fr,
+        "e2e": m["e2e"], "gpu_launches": m["kernels_per_step"] * args.steps,
+        "clocks": m["clocks"], "launch": m["launch"],
+        "ms_per_step_eager": m["ms_eager"] / args.steps,
     }
-    if world == 1 and not args.no_cpu_baseline:
-        inp_cpu = {kk: v.cpu() for kk, v in inp.items()}
-        line["cpu_baseline"] = cpu_baseline(w, inp_cpu, backward=backward)
+    if also:
+        line["also"] = {}
+        for name, (wa, ma) in also.items():
+            ra, rfa, ga, ha = _rates(wa, ma)
+            line["also"][name] = {
+                "value": wa.T * world * args.steps / (ma["ms_total"] / 1e3), "unit": UNIT,
+                "ms_per_step": ma["ms_total"] / args.steps, "config": config_of(wa, world, backward),
+                "roofline": rfa, "breakdown": ra, "grouped_gemm": ga, "hbm": ha,
+                "gpu_launches": ma["kernels_per_step"] * args.steps, "launch": ma["launch"],
+                "note": "device-timed like the headline, in the same run; no e2e or CPU baseline"}
+            line["gpu_launches"] += ma["kernels_per_step"] * args.steps
+            line["gpu_launches_note"] = ("headline steps plus the steps of the workloads under "
+                                         "'also', each timed in its own region")
+    if m["inp_cpu"] is not None:
+        line["cpu_baseline"] = cpu_baseline(w, m["inp_cpu"], backward=backward)
+        line["cpu_baseline_one_thread"] = cpu_baseline(w, m["inp_cpu"], backward=backward,
+                                                       threads=1)
     else:
         line["cpu_baseline"] = None
     print(json.dumps(line), flush=True)
@@ -783,6 +854,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--also", default=ALSO_WORKLOAD,
+                    help="comma-separated workloads also timed (device only) into the 'also' key; "
+                         "'none' to skip")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=64,
                     help="tokens per step of the CPU-oracle reference arm")

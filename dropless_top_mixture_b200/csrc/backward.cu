@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             for (int kb = 0; kb < tl.nkb; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
                     ok = false;
                     break;
                 }
@@ -292,14 +292,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wait_limit())) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
             for (int kb = 0; kb < tl.nkb; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
                     ok = false;
                     break;
                 }
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, WAIT_LIMIT_NS)) break;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wait_limit())) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
             if (MODE == DWF) {

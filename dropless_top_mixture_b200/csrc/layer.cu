@@ -18,6 +18,17 @@ bool& check_only() {
     return flag;
 }
 
+namespace tc {
+// Setters of the per-unit pipeline wait limits (filled during static
+// initialisation, before any call into the library).
+static int (*g_limit_setters[16])(uint64_t);
+static int g_num_limit_setters = 0;
+int register_wait_limit_setter(int (*set)(uint64_t ns)) {
+    if (g_num_limit_setters < 16) g_limit_setters[g_num_limit_setters++] = set;
+    return g_num_limit_setters;
+}
+}  // namespace tc
+
 int* status_ptr() {
     static int* cached[64] = {nullptr};
     static std::mutex mu;
@@ -71,6 +82,13 @@ inline Carve carve(void* base, int64_t T, int64_t d, int64_t E, int64_t F, int k
 using namespace moe;
 
 extern "C" const char* moe_version(void) { return "dropless_top_mixture_b200 0.1 sm_100a"; }
+
+extern "C" int moe_debug_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns ? ns : 2000000000ull;
+    for (int i = 0; i < tc::g_num_limit_setters; ++i)
+        if (tc::g_limit_setters[i](v) != 0) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
 
 extern "C" int moe_get_status(int32_t* host_status, int clear, void* stream) {
     if (!host_status) return MOE_ERR_INVALID;

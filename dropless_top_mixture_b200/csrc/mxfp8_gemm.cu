@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
             for (int kb = 0; kb < KS; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
                     ok = false;
                     break;
                 }
@@ -280,13 +280,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
             // the epilogue has moved the previous tile's accumulator out
             if (!mbar_wait(smem_u32(tempty), ((uint32_t)i & 1u) ^ 1u, s_abort, status,
-                           WAIT_LIMIT_NS)) {
+                           wait_limit())) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             for (int kb = 0; kb < KS; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
                     ok = false;
                     break;
                 }
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
-            if (!mbar_wait(smem_u32(tfull), (uint32_t)i & 1u, s_abort, status, WAIT_LIMIT_NS))
+            if (!mbar_wait(smem_u32(tfull), (uint32_t)i & 1u, s_abort, status, wait_limit()))
                 break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);

@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, WAIT_LIMIT_NS)) {
+            if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
                 ok = false;
                 break;
             }
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
                 ok = false;
                 break;
             }
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, WAIT_LIMIT_NS)) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
                 ok = false;
                 break;
             }
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 if (er + 128 < EN && n0 + er + 128 < E) wnorm2[n0 + er + 128] = sw1;
             }
         }
-        if (ok && mbar_wait(smem_u32(done), 0, s_abort, status, WAIT_LIMIT_NS)) {
+        if (ok && mbar_wait(smem_u32(done), 0, s_abort, status, wait_limit())) {
             tc_fence_after();
             const int t = m0 + q * 32 + lane;
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);

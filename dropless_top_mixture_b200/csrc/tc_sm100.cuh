@@ -15,6 +15,20 @@ namespace tc {
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // 0.1 s
 
+// Time limit of the pipeline waits in this compilation unit's kernels:
+// WAIT_LIMIT_NS unless moe_debug_set_wait_limit_ns lowered it (a test of
+// the abort path). The drain waits after an abort keep DRAIN_LIMIT_NS.
+static __device__ uint64_t g_wait_limit_ns = WAIT_LIMIT_NS;
+__device__ __forceinline__ uint64_t wait_limit() { return g_wait_limit_ns; }
+
+// Every compilation unit that includes this header registers a setter for
+// its own copy of the limit (layer.cu keeps the list).
+int register_wait_limit_setter(int (*set)(uint64_t ns));
+static int set_wait_limit_here(uint64_t ns) {
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof ns) == cudaSuccess ? 0 : -1;
+}
+static const int g_wait_limit_setter = register_wait_limit_setter(&set_wait_limit_here);
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
@@ -37,15 +51,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity. Returns false if the wait
 // timed out (status bit + abort flag set here) or another role aborted.
+// try_wait may suspend the thread for a while inside one poll, so the clock
+// and the abort flag are read every 64 polls. A limit below 1 ms (set for a
+// test of the abort path) polls with the non-blocking test_wait and reads
+// the clock at every poll, so that any wait not already complete gives up.
 __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                        int* status, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const bool quick = limit_ns < 1000000ull;
+    if (quick ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint32_t every = quick ? 1u : 64u;
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (quick ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (it % every == 0) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > limit_ns) {
                 set_status(status, MOE_DEVERR_TIMEOUT);

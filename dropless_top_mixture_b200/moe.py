@@ -161,6 +161,7 @@ _SIGS = {
     "moe_router_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64]),
     "moe_router_linear_bwd": (_i32, [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _p, _sz, _p]),
     "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
+    "moe_debug_set_wait_limit_ns": (_i32, [ctypes.c_uint64]),
     "moe_version": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -718,6 +719,15 @@ def moe_get_status(clear: bool = True, device=None) -> int:
 
 def moe_version() -> str:
     return lib.moe_version().decode()
+
+
+def moe_debug_set_wait_limit_ns(ns: int, device=None) -> None:
+    """Test-only: time limit of the kernels' pipeline waits on the device
+    (0 = the default 2 s)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        rc = lib.moe_debug_set_wait_limit_ns(int(ns))
+    _check("moe_debug_set_wait_limit_ns", rc)
 
 
 # ----------------------------------------------------------------- MXFP8 path

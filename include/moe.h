@@ -723,6 +723,20 @@ MOE_API int moe_router_linear_bwd(const float* dlogits, const void* x, const voi
  * ---------------------------------------------------------------------- */
 MOE_API int moe_get_status(int32_t* host_status, int clear, void* stream);
 
+/* ------------------------------------------------------------------------
+ * moe_debug_set_wait_limit_ns — for tests of the fault path only: sets the
+ * time limit of every bounded pipeline wait in the tensor-core kernels
+ * (grouped GEMMs, backward GEMMs, MXFP8 GEMMs, router) on the current
+ * device; 0 restores the default of 2 s. A wait that exceeds the limit sets
+ * MOE_DEVERR_TIMEOUT and an abort flag; every role of the kernel then stops
+ * issuing, waits (at most 0.1 s) for the copies and MMAs it already has in
+ * flight, the tensor memory is freed and the kernel returns with its outputs
+ * incomplete. With a limit of a few nanoseconds nearly every wait gives up,
+ * which exercises that path without any fault. Synchronous (a copy to device
+ * memory); do not change it while kernels of the library are running.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_debug_set_wait_limit_ns(uint64_t ns);
+
 /* library version string */
 MOE_API const char* moe_version(void);
 
