@@ -655,7 +655,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint64_t bd = sw128_desc(sa + pr::A_BYTES);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc_mma_pair(dt, ad + 2 * ks, bd + 2 * ks, IDESC, (kb | ks) != 0);
+                    tc_mma_pair<TF32>(dt, ad + 2 * ks, bd + 2 * ks, IDESC, (kb | ks) != 0);
                 tc_commit_pair(smem_u32(empty + stage), 0x3);
                 if (++stage == STAGES) {
                     stage = 0;

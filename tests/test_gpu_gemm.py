@@ -68,14 +68,23 @@ def test_grouped_swiglu_small(dtype, T, d, F, E, k):
 TAIL_COUNTS = [1, 15, 16, 17, 31, 33, 127, 128, 129, 200, 0, 255, 257, 64, 384, 3]
 
 
+# larger experts: after 0, 1 or 2 full 256-row chunks the last rows number
+# 1, 64, 127, 128, 129, 200, 255 or 256; an empty expert too
+LARGER_COUNTS = [1, 64, 127, 128, 129, 200, 255, 256, 257, 300, 384, 385, 511, 512, 0, 640]
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("d,F", [(256, 256), (384, 128), (512, 384)])
-def test_grouped_swiglu_every_tail_size(dtype, d, F):
+@pytest.mark.parametrize("which", ["small_experts", "larger_experts"])
+def test_grouped_swiglu_every_tail_size(dtype, d, F, which):
     """Expert segments given directly by offsets, so every ragged tail size
-    (the operand-swapped tail tiles) is met; A, B and H kept for the
-    backward are checked too."""
+    is met, with 16 experts averaging 104 rows and with experts averaging
+    259 rows (the gate/up GEMM on single-CTA tiles in both; the down GEMM
+    on CTA pairs where experts average 512 rows or more); A, B and H kept
+    for the backward are checked too."""
     moe = _moe()
-    counts = np.array(TAIL_COUNTS, dtype=np.int64)
+    counts = np.array(TAIL_COUNTS if which == "small_experts" else LARGER_COUNTS,
+                      dtype=np.int64)
     E, R = len(counts), int(counts.sum())
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     g = torch.Generator().manual_seed(d + F)
