@@ -51,21 +51,28 @@ constexpr int STG_BYTES = 32 * 128;  // dW store staging: 32 rows x 64 bf16, one
 // as groups): DXR is DH's operand layout with an epilogue that adds the
 // product into the existing out0 rows; DWF is DW with fp32 output tiles (the
 // partials of a split-K sum).
-enum Mode { DH = 0, DX = 1, DW = 2, DXR = 3, DWF = 4 };
+enum Mode { DH = 0, DX = 1, DW = 2, DXR = 3, DWF = 4, DWS = 5 };
 template <int MODE>
-constexpr bool is_dw() { return MODE == DW || MODE == DWF; }
+constexpr bool is_dw() { return MODE == DW || MODE == DWF || MODE == DWS; }
 
-// DW tiles have a short K (an expert's rows) and a large output, so they use
-// fewer pipeline stages and spend the shared memory on store staging
-// (4 epilogue warps x 2 buffers) for TMA tensor stores.
+// DW tiles have a short K (an expert's rows) and a large output. With 128
+// or more rows per expert, the load ring keeps 4 stages like the other modes
+// (a tile's K loop is a few slabs, so the ring's depth is what keeps bytes
+// in flight) and each epilogue warp has one staging buffer for its TMA
+// tensor stores; with fewer rows (DWS) a tile is one or two slabs and the
+// stores bound it, so 3 stages and 2 staging buffers per warp. The expert
+// offsets are read from global memory instead of a shared table.
 template <int MODE>
 struct ModeCfg {
     static constexpr bool A_MN = is_dw<MODE>();
     static constexpr uint32_t IDESC = make_idesc_major(1u, BM, MMA_N, A_MN, true);
-    static constexpr int STAGES = is_dw<MODE>() ? 3 : 4;
-    static constexpr int STAGING = is_dw<MODE>() ? EPI_WARPS * 2 * STG_BYTES : 0;
+    static constexpr int STAGES = MODE == DWS ? 3 : 4;
+    static constexpr int STG_BUFS = MODE == DWS ? 2 : (is_dw<MODE>() ? 1 : 0);  // per epilogue warp
+    static constexpr int STAGING = EPI_WARPS * STG_BUFS * STG_BYTES;
+    static constexpr bool TABLES = !is_dw<MODE>();  // shared offset and tile tables
     static constexpr int NUM_BARS = 2 * STAGES + 5;
-    static constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+    static constexpr int META_BYTES =
+        NUM_BARS * 8 + 16 + (TABLES ? 2 * 4 * (MOE_MAX_EXPERTS + 1) : 0);
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING + META_BYTES;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -154,12 +161,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + NUM_BARS * 8);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
-    int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
-    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    // DW: the offsets straight from global memory; the others: shared copies
+    // and the tile table
+    int* s_tab = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
+    const int* s_off = C::TABLES ? s_tab : offsets;
+    int* s_toff = C::TABLES ? s_tab + (MOE_MAX_EXPERTS + 1) : nullptr;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // --- routing offsets -> tile table (validated) -----------------------
-    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    if (C::TABLES)
+        for (int e = tid; e <= E; e += THREADS) s_tab[e] = offsets[e];
     __syncthreads();
     if (warp == 0) {
         int carry = 0;
@@ -174,12 +185,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             int tot;
             const int ex = warp_exclusive_scan(m, &tot);
-            if (e < E) s_toff[e] = carry + ex;
+            if (C::TABLES && e < E) s_toff[e] = carry + ex;
             carry += tot;
         }
         bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
         if (lane == 0) {
-            s_toff[E] = carry;
+            if (C::TABLES) s_toff[E] = carry;
             *s_bad = bad ? 1 : 0;
         }
     }
@@ -370,18 +381,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wait_limit())) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
-            if (MODE == DWF) {
+            if constexpr (MODE == DWF) {
                 // 32-column groups: TMEM -> fp32 -> 128-byte-swizzled staging
                 // (chunk c of row r at c ^ (r % 8)) -> TMA store of the warp's
-                // 32 x 32 fp32 box; two staging buffers per warp
+                // 32 x 32 fp32 box; one staging buffer per warp
                 const bool empty_k = tl.nkb == 0;
                 const int ybase = tl.e * Mdim + tl.m0 + q * 32;
-                uint8_t* stg = staging + (warp - 2) * 2 * STG_BYTES;
+                uint8_t* stg = staging + (warp - 2) * C::STG_BUFS * STG_BYTES;
 #pragma unroll 1
                 for (int cc = col0 / 32; cc < (col0 + MMA_N / 2) / 32; ++cc) {
-                    uint8_t* sbuf = stg + (stg_count & 1) * STG_BYTES;
+                    uint8_t* sbuf = stg + (stg_count % C::STG_BUFS) * STG_BYTES;
                     ++stg_count;
-                    if (lane == 0) bulk_wait_read<1>();  // this buffer's previous store has read it
+                    if (lane == 0) bulk_wait_read<C::STG_BUFS - 1>();  // its previous store has read it
                     __syncwarp();
                     uint32_t a[32];
                     if (!empty_k) {
@@ -403,18 +414,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                         bulk_commit();
                     }
                 }
-            } else if (MODE == DW) {
+            } else if constexpr (MODE == DW || MODE == DWS) {
                 // 64-column groups: TMEM -> bf16 -> 128-byte-swizzled staging
                 // (chunk c of row r at c ^ (r % 8), conflict-free) -> TMA store
-                // of the warp's 32 x 64 box; two staging buffers per warp
+                // of the warp's 32 x 64 box; one staging buffer per warp
                 const bool empty_k = tl.nkb == 0;
                 const int ybase = tl.e * Mdim + tl.m0 + q * 32;
-                uint8_t* stg = staging + (warp - 2) * 2 * STG_BYTES;
+                uint8_t* stg = staging + (warp - 2) * C::STG_BUFS * STG_BYTES;
 #pragma unroll 1
                 for (int cc = col0 / 64; cc < (col0 + MMA_N / 2) / 64; ++cc) {
-                    uint8_t* sbuf = stg + (stg_count & 1) * STG_BYTES;
+                    uint8_t* sbuf = stg + (stg_count % C::STG_BUFS) * STG_BYTES;
                     ++stg_count;
-                    if (lane == 0) bulk_wait_read<1>();  // this buffer's previous store has read it
+                    if (lane == 0) bulk_wait_read<C::STG_BUFS - 1>();  // its previous store has read it
                     __syncwarp();
                     uint32_t a[2][32];
                     if (!empty_k) {
@@ -587,6 +598,16 @@ int swiglu_wgrad(const void* Xe, const void* dA, const void* dB, const void* dYe
         !make_map_2d(&o3, dW3, bwd::BF16, 2, d, E * F, 32) ||
         !make_map_2d(&o2, dW2, bwd::BF16, 2, F, E * d, 32))
         return MOE_ERR_CUDA;
+    if (R < 128 * E) {  // experts average fewer than 128 rows: the store-bound form
+        int rc = bwd::launch<bwd::DWS>(gA, gA, gX, gX, o1, offsets, E, R, 0, F, d, dW1, nullptr,
+                                       d, nullptr, nullptr, st);
+        if (rc != MOE_OK) return rc;
+        rc = bwd::launch<bwd::DWS>(gB, gB, gX, gX, o3, offsets, E, R, 0, F, d, dW3, nullptr, d,
+                                   nullptr, nullptr, st);
+        if (rc != MOE_OK) return rc;
+        return bwd::launch<bwd::DWS>(gY, gY, gH, gH, o2, offsets, E, R, 0, d, F, dW2, nullptr, F,
+                                     nullptr, nullptr, st);
+    }
     int rc = bwd::launch<bwd::DW>(gA, gA, gX, gX, o1, offsets, E, R, 0, F, d, dW1, nullptr, d,
                                   nullptr, nullptr, st);
     if (rc != MOE_OK) return rc;

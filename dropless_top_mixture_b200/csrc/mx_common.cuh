@@ -45,6 +45,24 @@ __device__ __forceinline__ uint8_t e8m0_scale(const float* v, float* scale) {
     return (uint8_t)(e + 127);
 }
 
+// 32 values / 2^(sbyte - 127) -> 32 E4M3 codes packed in 8 words. The
+// division by a power of two is a multiplication by its exact reciprocal
+// 2^(127 - sbyte), which is rounded once to the same fp32 value.
+__device__ __forceinline__ void encode32_e8m0(const float* v, uint8_t sbyte, uint32_t* w) {
+    const float inv = exp2_exact(127 - (int)sbyte);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_fp8_storage_t c =
+                __nv_cvt_float_to_fp8(v[4 * i + j] * inv, __NV_SATFINITE, __NV_E4M3);
+            word |= (uint32_t)c << (8 * j);
+        }
+        w[i] = word;
+    }
+}
+
 // 32 values / scale -> 32 E4M3 codes packed in 8 words.
 __device__ __forceinline__ void encode32(const float* v, float scale, uint32_t* w) {
 #pragma unroll

@@ -49,13 +49,14 @@ __global__ void __launch_bounds__(THREADS) quantize_kernel(const void* __restric
 #pragma unroll
         for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
         const float s32 = __fdiv_rn(amax, 448.0f);
-        float s;
+        float s, inv = 1.f;
         if (MODE == MOE_SCALE_F32) {
             s = (amax == 0.f) ? 1.0f : s32;
             static_cast<float*>(scales)[b] = s;
         } else {
             const int e = (amax == 0.f) ? 0 : pow2_ceil_exp(s32);
             s = exp2_exact(e);
+            inv = exp2_exact(-e);
             static_cast<uint8_t*>(scales)[b] = (uint8_t)(e + 127);
         }
         uint32_t w[8];
@@ -64,8 +65,10 @@ __global__ void __launch_bounds__(THREADS) quantize_kernel(const void* __restric
             uint32_t word = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const __nv_fp8_storage_t c =
-                    __nv_cvt_float_to_fp8(__fdiv_rn(v[4 * i + j], s), __NV_SATFINITE, __NV_E4M3);
+                // a UE8M0 scale is a power of two: divide by multiplying by its
+                // exact reciprocal (the same rounded value)
+                const float qv = MODE == MOE_SCALE_E8M0 ? v[4 * i + j] * inv : __fdiv_rn(v[4 * i + j], s);
+                const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(qv, __NV_SATFINITE, __NV_E4M3);
                 word |= (uint32_t)c << (8 * j);
             }
             w[i] = word;

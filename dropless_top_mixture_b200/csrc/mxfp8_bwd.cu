@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(256)
     float sc;
     const uint8_t sb = mxc::e8m0_scale(v, &sc);
     uint32_t w[8];
-    mxc::encode32(v, sc, w);
+    mxc::encode32_e8m0(v, sb, w);
     const int64_t orow = (int64_t)e * cols + c;
     uint4* dq = reinterpret_cast<uint4*>(q + orow * ldq + col_off + r0);
     dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -85,60 +85,90 @@ static int transpose_quant(const void* in, int64_t in_es, int64_t E, int64_t row
 
 __device__ __forceinline__ float sigmoid_(float a) { return 1.0f / (1.0f + __expf(-a)); }
 
-// One thread per 32-column block of one row: the pairwise SwiGLU backward
-// dA = dH·B·silu'(A), dB = dH·silu(A) (silu'(a) = s(1 + a(1 - s)),
-// s = sigmoid(a)) in fp32; dA, dB stored in bf16 [R, F]; the fp32 values
-// quantised into Q [R, 2F] (dA in columns 0..F-1, dB in F..2F-1) with scale
-// bytes S [R, 2F/32].
+// The pairwise SwiGLU backward dA = dH·B·silu'(A), dB = dH·silu(A)
+// (silu'(a) = s(1 + a(1 - s)), s = sigmoid(a)) in fp32; dA, dB stored in
+// bf16 [R, F]; the fp32 values quantised into Q [R, 2F] (dA in columns
+// 0..F-1, dB in F..2F-1) with scale bytes S [R, 2F/32]. Four lanes share a
+// 32-column block, eight columns each: a warp reads and writes 512
+// contiguous bytes of a row per access, and the block's maximum is two
+// shuffles among the four lanes. F % 32 == 0, so a block's lanes are
+// consecutive lanes of one warp.
+// 8 values / 2^e -> 8 E4M3 codes, dividing by the power of two as a
+// multiplication by its exact reciprocal (the same rounded value)
+__device__ __forceinline__ uint2 encode8(const float* v, int e) {
+    const float inv = mxc::exp2_exact(-e);
+    uint32_t w[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_fp8_storage_t c =
+                __nv_cvt_float_to_fp8(v[4 * i + j] * inv, __NV_SATFINITE, __NV_E4M3);
+            word |= (uint32_t)c << (8 * j);
+        }
+        w[i] = word;
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+// UE8M0 scale exponent of a block whose 32 values are spread over 4
+// consecutive lanes (8 each); every lane of the four gets it.
+__device__ __forceinline__ int e8m0_exp_4lanes(const float* v) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    return (amax == 0.f) ? 0 : mxc::pow2_ceil_exp(__fdiv_rn(amax, 448.0f));
+}
+
 __global__ void __launch_bounds__(256)
     swiglu_bwd_quant_kernel(const __nv_bfloat16* __restrict__ dH,
                             const __nv_bfloat16* __restrict__ A,
                             const __nv_bfloat16* __restrict__ B, int64_t R, int F,
                             __nv_bfloat16* __restrict__ dA, __nv_bfloat16* __restrict__ dB,
                             uint8_t* __restrict__ q, uint8_t* __restrict__ s) {
+    const int per_row = F / 8;  // 8-column pieces per row (a multiple of 4)
     const int nb = F / 32;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= R * nb) return;
-    const int64_t r = i / nb;
-    const int b = (int)(i - r * nb);
-    const int64_t off = r * F + (int64_t)b * 32;
-    float da[32], db[32];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    // R * per_row is a multiple of 4, so the four lanes of a block are all
+    // live or all past the end; the dead ones still take part in the shuffles
+    const bool live = i < R * (int64_t)per_row;
+    const int64_t r = live ? i / per_row : 0;
+    const int c8 = live ? (int)(i - r * per_row) : 0;
+    const int64_t off = r * F + 8 * (int64_t)c8;
+    float da[8], db[8];
+    if (live) {
         float h[8], a[8], g[8];
-        unpack8(reinterpret_cast<const uint4*>(dH + off)[u], h);
-        unpack8(reinterpret_cast<const uint4*>(A + off)[u], a);
-        unpack8(reinterpret_cast<const uint4*>(B + off)[u], g);
+        unpack8(*reinterpret_cast<const uint4*>(dH + off), h);
+        unpack8(*reinterpret_cast<const uint4*>(A + off), a);
+        unpack8(*reinterpret_cast<const uint4*>(B + off), g);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float sg = sigmoid_(a[j]);
             const float silu = a[j] * sg;
             const float dsilu = sg * (1.0f + a[j] * (1.0f - sg));
-            da[8 * u + j] = h[j] * g[j] * dsilu;
-            db[8 * u + j] = h[j] * silu;
+            da[j] = h[j] * g[j] * dsilu;
+            db[j] = h[j] * silu;
         }
-    }
+        *reinterpret_cast<uint4*>(dA + off) = pack8(da);
+        *reinterpret_cast<uint4*>(dB + off) = pack8(db);
+    } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        reinterpret_cast<uint4*>(dA + off)[u] = pack8(da + 8 * u);
-        reinterpret_cast<uint4*>(dB + off)[u] = pack8(db + 8 * u);
+        for (int j = 0; j < 8; ++j) da[j] = db[j] = 0.f;
     }
+    const int ea = e8m0_exp_4lanes(da);
+    const int eb = e8m0_exp_4lanes(db);
+    if (!live) return;
     const int64_t qrow = r * 2 * F;
-    const int64_t srow = r * 2 * nb;
-    uint32_t w[8];
-    float sc;
-    uint8_t sb = mxc::e8m0_scale(da, &sc);
-    mxc::encode32(da, sc, w);
-    uint4* dq = reinterpret_cast<uint4*>(q + qrow + (int64_t)b * 32);
-    dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    s[srow + b] = sb;
-    sb = mxc::e8m0_scale(db, &sc);
-    mxc::encode32(db, sc, w);
-    dq = reinterpret_cast<uint4*>(q + qrow + F + (int64_t)b * 32);
-    dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    s[srow + nb + b] = sb;
+    *reinterpret_cast<uint2*>(q + qrow + 8 * c8) = encode8(da, ea);
+    *reinterpret_cast<uint2*>(q + qrow + F + 8 * c8) = encode8(db, eb);
+    if ((c8 & 3) == 0) {
+        const int64_t srow = r * 2 * nb;
+        s[srow + (c8 >> 2)] = (uint8_t)(ea + 127);
+        s[srow + nb + (c8 >> 2)] = (uint8_t)(eb + 127);
+    }
 }
 
 inline size_t a256(size_t n) { return (n + 255) & ~size_t(255); }
@@ -222,7 +252,7 @@ extern "C" int moe_swiglu_bwd_mxfp8(const void* dH, const void* A, const void* B
     for (const void* p : ptrs)
         if (!p || !aligned16(p)) return MOE_ERR_INVALID;
     if (!dABs) return MOE_ERR_INVALID;
-    const int64_t n = R * (F / 32);
+    const int64_t n = R * (F / 8);  // one thread per 8 columns
     const int64_t blocks = (n + 255) / 256;
     if (blocks > INT32_MAX) return MOE_ERR_UNSUPPORTED;
     if (check_only()) return MOE_OK;

@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     float sc;
                     const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
                     uint32_t w[8];
-                    mxc::encode32(v, sc, w);
+                    mxc::encode32_e8m0(v, sbyte, w);
                     uint4* dq = reinterpret_cast<uint4*>(out_q + gr * ldo + col);
                     dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
                     dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(256) mx_dispatch_kernel(const __nv_bfloat16* _
         float sc;
         const uint8_t sbyte = mxc::e8m0_scale(v, &sc);
         uint32_t w[8];
-        mxc::encode32(v, sc, w);
+        mxc::encode32_e8m0(v, sbyte, w);
         const uint4 c0 = make_uint4(w[0], w[1], w[2], w[3]);
         const uint4 c1 = make_uint4(w[4], w[5], w[6], w[7]);
         for (int j = 0; j < k; ++j) {

@@ -679,6 +679,59 @@ def mxfp8_layer_bwd(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W2,
     return res
 
 
+def mxfp8_layer_bwd_sampled(x: torch.Tensor, dOut: torch.Tensor, k: int, W1, W3, W2,
+                            logits: np.ndarray, tokens, experts,
+                            mode: str = "e8m0") -> Dict[str, np.ndarray]:
+    """mxfp8_layer_bwd's gradients restricted to a sample, for full-size
+    workloads: dx for the given tokens and dW1, dW3, dW2 for the given
+    experts (from all of that expert's rows). Every quantisation in that
+    reading is per row of an activation (the token rows of x, dYe, [dA | dB],
+    H) or per weight, so a (token, choice) row's chain needs only its own
+    row and its expert's weights, quantised once per expert here."""
+    E, F, d = W1.shape
+    idx, gate, _ = route(logits, k)
+    meta = routing_metadata(idx, E)
+    qdq = lambda m: _qdq_rows(m, mode)  # noqa: E731
+    cache = {}
+
+    def wq(e):
+        if e not in cache:
+            w1, w3, w2 = to64(W1[e]), to64(W3[e]), to64(W2[e])
+            cache[e] = dict(w1d=qdq(w1), w3d=qdq(w3), w2td=qdq(w2.T),
+                            w13td=qdq(np.concatenate([w1.T, w3.T], axis=1)))
+        return cache[e]
+
+    def rows(e, toks, js):
+        w = wq(e)
+        tt = torch.as_tensor(np.asarray(toks), dtype=torch.long)
+        X = qdq(to64(x[tt]))                                   # token rows along d
+        a, b = X @ w["w1d"].T, X @ w["w3d"].T
+        Hd = qdq(silu(a) * b)                                  # H along F
+        A, B = _bf16(a), _bf16(b)
+        dy = _bf16(gate[toks, js][:, None] * to64(dOut[tt]))   # bf16 of gate * dOut
+        dH = _bf16(qdq(dy) @ w["w2td"].T)                      # dYe along d
+        da = dH * B * dsilu(A)
+        db = dH * silu(A)
+        dXe = qdq(np.concatenate([da, db], axis=1)) @ w["w13td"].T  # [dA | dB] along F
+        return X, Hd, dy, da, db, dXe
+
+    tokens = np.asarray(tokens)
+    dx = np.zeros((len(tokens), d))
+    for i, t in enumerate(tokens):
+        for j in range(k):
+            dx[i] += rows(int(idx[t, j]), np.array([t]), np.array([j]))[5][0]
+    dW = {}
+    for e in experts:
+        e = int(e)
+        toks, js = np.nonzero(idx == e)  # token-major: the expert buffer's order
+        if len(toks) == 0:
+            dW[e] = (np.zeros((F, d)), np.zeros((F, d)), np.zeros((d, F)))
+            continue
+        X, Hd, dy, da, db, _ = rows(e, toks, js)
+        dW[e] = (da.T @ X, db.T @ X, dy.T @ Hd)
+    return dict(dx=dx, dW=dW, idx=idx, gate=gate, tokens=tokens, **meta)
+
+
 # --------------------------------------------------------------------------
 # f2: router backward and the load-balancing auxiliary loss
 #     [HF §2 router (fp32 softmax, top-k, optional norm_topk_prob);

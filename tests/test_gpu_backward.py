@@ -64,12 +64,14 @@ def test_layer_backward_small(T, d, F, E, k):
     _check_grads(g, ref, E)
 
 
-def test_expert_backward_ragged_segments():
-    """Counts 1, 63, 64, 65, 128, 129, 0 and a large expert: K slabs that end
-    inside, at, and just past a 64-row boundary."""
+@pytest.mark.parametrize("counts", [[1, 63, 64, 65, 128, 129, 0, 300],
+                                    [1, 63, 64, 65, 128, 129, 0, 300, 512, 257]])
+def test_expert_backward_ragged_segments(counts):
+    """Counts 1, 63, 64, 65, 128, 129, 0 and large experts: K slabs that end
+    inside, at, and just past a 64-row boundary; averaging under 128 rows
+    per expert (weight gradients in the store-bound form) and over it."""
     moe = _moe()
     d, F = 256, 256
-    counts = [1, 63, 64, 65, 128, 129, 0, 300]
     E = len(counts)
     R = sum(counts)
     g = torch.Generator().manual_seed(77)

@@ -195,3 +195,32 @@ def test_layer_bwd_mxfp8_rejects_bad_arguments():
         moe.moe_layer_bwd_mxfp8(fw, dOut.cuda(), k, wb, out=gr)
     torch.cuda.synchronize()
     assert moe.moe_get_status() == 0
+
+
+@pytest.mark.slow
+def test_layer_bwd_mxfp8_full_size_sampled():
+    """The MXFP8 backward of the 128-expert workload (T=8192, d=4096,
+    F=2048, top-4) at full size, in the launch configuration the benchmark
+    times, against the oracle's MXFP8 backward restricted to a sample: dx of
+    one token and the weight gradients of one of its experts (the oracle
+    re-quantises each expert's weights in numpy, about 18 s per expert)."""
+    from dropless_top_mixture_b200.workloads import WORKLOADS, make_inputs
+    moe = _moe()
+    wl = WORKLOADS["mxfp8_e128"].scaled(backward=True)
+    inp = make_inputs(wl, "cuda")
+    w = moe.mxfp8_quantize_weights(inp["W1"], inp["W3"], inp["W2"])
+    wb = moe.mxfp8_quantize_weights_bwd(inp["W1"], inp["W3"], inp["W2"])
+    fw = moe.moe_layer_fwd_mxfp8(inp["x"], wl.k, w, logits=inp["logits"], save=True)
+    gr = moe.moe_layer_bwd_mxfp8(fw, inp["dOut"], wl.k, wb)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == 0
+    lg = inp["logits"].cpu().numpy()
+    tok = wl.T // 2 + 17
+    e = int(fw.idx[tok, 0].item())
+    W1, W3, W2 = (inp[n].cpu() for n in ("W1", "W3", "W2"))
+    ref = O.mxfp8_layer_bwd_sampled(inp["x"].cpu(), inp["dOut"].cpu(), wl.k, W1, W3, W2, lg,
+                                    [tok], [e])
+    assert np.array_equal(fw.idx.cpu().numpy(), ref["idx"])
+    assert_close_scaled(np64(gr.dx[tok:tok + 1]), ref["dx"], "dx (sampled token)")
+    for name, r in zip(("dW1", "dW3", "dW2"), ref["dW"][e]):
+        assert_close_scaled(np64(getattr(gr, name)[e]), r, f"{name} of expert {e}")

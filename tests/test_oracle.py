@@ -713,3 +713,18 @@ def test_mxfp8_forward_error_against_exact_layer():
     b = O.moe_layer(x, 2, W1, W3, W2, logits=lg)
     rel = np.linalg.norm(r["out"] - b["out"]) / np.linalg.norm(b["out"])
     assert 1e-3 < rel < 0.15, rel
+
+
+def test_mxfp8_sampled_backward_matches_full_backward():
+    # the per-row restatement used at full size equals the whole-batch MXFP8
+    # backward on the sampled tokens and experts (empty expert included)
+    x, W1, W3, W2, lg, dOut = _mx_problem(64, T=60, d=64, F=64, E=4, k=2, skew=True)
+    with np.errstate(over="ignore"):
+        full = O.mxfp8_layer_bwd(x, dOut, 2, W1, W3, W2, lg)
+        toks = np.array([0, 7, 31, 59])
+        smp = O.mxfp8_layer_bwd_sampled(x, dOut, 2, W1, W3, W2, lg, toks, [0, 2, 3])
+    assert np.allclose(smp["dx"], full["dx"][toks], rtol=1e-12, atol=1e-12)
+    for e in (0, 2, 3):
+        for got, ref in zip(smp["dW"][e], (full["dW1"][e], full["dW3"][e], full["dW2"][e])):
+            assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), e
+    assert all(np.all(m == 0) for m in smp["dW"][3])  # expert 3 gets no rows
