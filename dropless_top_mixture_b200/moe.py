@@ -161,6 +161,10 @@ _SIGS = {
     "moe_router_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64]),
     "moe_router_linear_bwd": (_i32, [_p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _p, _sz, _p]),
     "moe_get_status": (_i32, [ctypes.POINTER(ctypes.c_int32), _i32, _p]),
+    "moe_ep_workspace_size": (_sz, [_i64]),
+    "moe_ep_plan": (_i32, [_p, _i32, _i32, _p, _p, _p, _i64, _i64, _i32, _p, _p, _p, _p, _sz, _p]),
+    "moe_dispatch_ep": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _i32, _i64, _p]),
+    "moe_combine_ep": (_i32, [_p, _p, _p, _p, _i64, _i64, _i32, _i32, _i32, _i64, _p, _p]),
     "moe_debug_set_wait_limit_ns": (_i32, [ctypes.c_uint64]),
     "moe_version": (ctypes.c_char_p, []),
 }
@@ -706,6 +710,69 @@ def moe_router_linear_bwd(dlogits, x, Wr, dx=None, want_dWr: bool = True, dWr=No
                                    0 if workspace is None else workspace.numel(), _stream(x))
     _check("moe_router_linear_bwd", rc)
     return dx, dWr
+
+
+# ----------------------------------------------------------------- expert parallelism
+
+@dataclass
+class EPPlan:
+    """Where this rank's (token, choice) rows live on their experts' ranks."""
+    dst_rank: torch.Tensor      # [T,k] int32
+    dst_row: torch.Tensor       # [T,k] int32
+    recv_offsets: torch.Tensor  # [E/G + 1] int32: this rank's receive buffer by local expert
+
+
+def moe_ep_plan(counts_all: torch.Tensor, me: int, route: "Route",
+                out: Optional[EPPlan] = None,
+                workspace: Optional[torch.Tensor] = None) -> EPPlan:
+    """counts_all [G,E] int32 (row s = rank s's per-expert counts); `route`
+    is this rank's moe_route result."""
+    _need(counts_all, "counts_all")
+    G, E = counts_all.shape
+    T, k = route.idx.shape
+    dev = counts_all.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = EPPlan(dst_rank=torch.empty((T, k), **i32), dst_row=torch.empty((T, k), **i32),
+                     recv_offsets=torch.empty(E // G + 1 if G and E % G == 0 else 1, **i32))
+    if workspace is None:
+        workspace = _alloc_ws(lib.moe_ep_workspace_size(E), dev)
+    rc = lib.moe_ep_plan(_ptr(counts_all), G, me, _ptr(route.idx), _ptr(route.slot),
+                         _ptr(route.offsets), T, E, k, _ptr(out.dst_rank), _ptr(out.dst_row),
+                         _ptr(out.recv_offsets), _ptr(workspace), workspace.numel(),
+                         _stream(counts_all))
+    _check("moe_ep_plan", rc)
+    return out
+
+
+def _ptr_table(bufs, dev) -> torch.Tensor:
+    return torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=dev)
+
+
+def moe_dispatch_ep(x: torch.Tensor, plan: EPPlan, recv_table: torch.Tensor,
+                    rows_max: int) -> None:
+    """Write every (token, choice) row of x into its owner's receive buffer;
+    recv_table is a device int64 tensor of the G buffers' addresses."""
+    _need(x, "x")
+    T, d = x.shape
+    k = plan.dst_rank.shape[1]
+    rc = lib.moe_dispatch_ep(_ptr(x), _ptr(plan.dst_rank), _ptr(plan.dst_row), T, d, k,
+                             _dtype_code(x.dtype), _ptr(recv_table), recv_table.numel(),
+                             rows_max, _stream(x))
+    _check("moe_dispatch_ep", rc)
+
+
+def moe_combine_ep(ye_table: torch.Tensor, plan: EPPlan, gate: torch.Tensor, d: int,
+                   dtype: torch.dtype, rows_max: int,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    T, k = plan.dst_rank.shape
+    if out is None:
+        out = torch.empty((T, d), dtype=dtype, device=gate.device)
+    rc = lib.moe_combine_ep(_ptr(ye_table), _ptr(plan.dst_rank), _ptr(plan.dst_row), _ptr(gate),
+                            T, d, k, _dtype_code(dtype), ye_table.numel(), rows_max, _ptr(out),
+                            _stream(gate))
+    _check("moe_combine_ep", rc)
+    return out
 
 
 def moe_get_status(clear: bool = True, device=None) -> int:

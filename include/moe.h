@@ -717,6 +717,53 @@ MOE_API int moe_router_linear_bwd(const float* dlogits, const void* x, const voi
                                   void* stream);
 
 /* ------------------------------------------------------------------------
+ * Expert parallelism over G ranks (one GPU each).
+ *
+ * ["olmoforge" README, capability table]: row-wise expert parallelism
+ * writes every token row straight into the input buffer of its expert, on
+ * whichever GPU holds it; [NEWS, "关键数字"]: experts are spread over the GPUs.
+ * Rank r owns experts r*El .. (r+1)*El - 1 (El = E / G). Each rank routes its
+ * own T tokens with moe_route; the ranks then gather their counts into
+ * counts_all [G, E] (row s = rank s's counts, e.g. one all-gather). Rank r's
+ * receive buffer holds the rows of its experts expert-major, and within an
+ * expert the rows of rank 0, then rank 1, ..., each in its sender's token
+ * order; it is the expert-sorted input of rank r's grouped GEMMs with
+ * offsets recv_offsets.
+ *
+ * moe_ep_plan — for this rank (`me`): dst_rank [T,k] and dst_row [T,k], the
+ *   owner and the row in the owner's receive buffer of every (t, j), and
+ *   recv_offsets [El+1] of this rank's receive buffer (recv_offsets[El] = its
+ *   rows). idx, slot, offsets from this rank's moe_route. Workspace:
+ *   moe_ep_workspace_size(E) bytes of device memory. Limits: E % G == 0,
+ *   1 <= G <= 64. A negative count or an expert index out of range sets
+ *   MOE_DEVERR_BAD_INDEX (the row gets dst_rank = dst_row = -1).
+ * moe_dispatch_ep — recv_bufs[dst_rank[t,j]][dst_row[t,j], :] = x[t, :].
+ *   recv_bufs: device array of G device pointers (8-byte aligned), each a
+ *   [rows_max, d] buffer in `dtype`, 16-byte aligned: on a multi-GPU node the
+ *   peers' receive buffers mapped into this process, so the rows travel over
+ *   NVLink as stores; a row outside [0, rows_max), a null or misaligned
+ *   pointer is skipped and sets MOE_DEVERR_BAD_INDEX.
+ * moe_combine_ep — out[t] = sum_j gate[t,j] * ye_bufs[dst_rank[t,j]][dst_row[t,j]]
+ *   (fp32 fused multiply-add in ascending j, rounded once to `dtype`): the
+ *   owners' expert outputs gathered back (peer loads on a multi-GPU node).
+ * The caller orders the steps across ranks: every rank's dispatch into a
+ * buffer completes before its owner's GEMMs read it, and the owner's GEMMs
+ * before any rank's combine reads the output (e.g. a stream-ordered barrier
+ * between the steps).
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_ep_workspace_size(int64_t E);
+MOE_API int moe_ep_plan(const int32_t* counts_all, int G, int me, const int32_t* idx,
+                        const int32_t* slot, const int32_t* offsets, int64_t T, int64_t E, int k,
+                        int32_t* dst_rank, int32_t* dst_row, int32_t* recv_offsets,
+                        void* workspace, size_t workspace_bytes, void* stream);
+MOE_API int moe_dispatch_ep(const void* x, const int32_t* dst_rank, const int32_t* dst_row,
+                            int64_t T, int64_t d, int k, int dtype, void* const* recv_bufs, int G,
+                            int64_t rows_max, void* stream);
+MOE_API int moe_combine_ep(const void* const* ye_bufs, const int32_t* dst_rank,
+                           const int32_t* dst_row, const float* gate, int64_t T, int64_t d, int k,
+                           int dtype, int G, int64_t rows_max, void* out, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_get_status — read (and optionally clear) the device status word of the
  * current device. Synchronises the given stream. *host_status receives an OR
  * of MOE_DEVERR_* bits (0 = no fault seen).

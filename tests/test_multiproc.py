@@ -59,3 +59,40 @@ def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
     bench.barrier(1)
     assert not torch.distributed.is_initialized()
+
+
+def _ep_worker(rank, world, port, E, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    from dropless_top_mixture_b200 import ep
+    g = torch.Generator().manual_seed(100 + rank)
+    counts = torch.randint(0, 50, (E,), generator=g, dtype=torch.int32)
+    allc = ep.exchange_counts(counts)
+    mine = list(ep.owned_experts(E, world, rank))
+    q.put((rank, allc.numpy().tolist(), mine, ep.receive_rows_max(300, 4, world)))
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+
+
+def test_expert_parallel_count_exchange_world3():
+    """Expert parallelism's host side over gloo: every rank receives every
+    rank's per-expert counts in rank order, the experts split into
+    contiguous blocks, and receive buffers are sized for every token of every
+    rank landing on one rank."""
+    E, world = 12, 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, E, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=5) for _ in range(world))
+    expect = [torch.randint(0, 50, (E,), generator=torch.Generator().manual_seed(100 + r),
+                            dtype=torch.int32).tolist() for r in range(world)]
+    for rank, allc, mine, rows_max in res:
+        assert allc == expect
+        assert mine == list(range(rank * 4, rank * 4 + 4))
+        assert rows_max == 3 * 300 * 4
