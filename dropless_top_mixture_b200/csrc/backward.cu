@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int* s_off = C::TABLES ? s_tab : offsets;
     int* s_toff = C::TABLES ? s_tab + (MOE_MAX_EXPERTS + 1) : nullptr;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
 
     // --- routing offsets -> tile table (validated) -----------------------
     if (C::TABLES)
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             for (int kb = 0; kb < tl.nkb; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -303,14 +304,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
             for (int kb = 0; kb < tl.nkb; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -378,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const Tile tl = decode<MODE>(t, E, NB, MB, K, s_toff, s_off);
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wait_limit())) break;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wl)) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
             if constexpr (MODE == DWF) {

@@ -36,7 +36,7 @@
 // The accumulator is double-buffered in TMEM (2 x MMA_N columns), so the
 // epilogue of tile i overlaps the main loop of tile i+1.
 //
-// Every wait is bounded: after wait_limit() the waiting thread sets
+// Every wait is bounded: after its time limit (2 s) the waiting thread sets
 // MOE_DEVERR_TIMEOUT and an abort flag, all roles leave their loops, the MMA
 // issuer drains its outstanding MMAs, the producer waits (again bounded) for
 // its copies in flight, and TMEM is released before the CTA exits.
@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
 
     // --- device-side tile table from the routing offsets (validated) -------
     for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 bool w = true;
                 if (lane == 0)
                     w = mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status,
-                                  wait_limit());
+                                  wl);
                 if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) {
                     ok = false;
                     break;
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -334,14 +335,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wait_limit())) break;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wl)) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * MMA_N);
             const int grow = tl.row0 + r_in_tile;
@@ -503,6 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     int* s_off = reinterpret_cast<int*>(meta + pr::NUM_BARS * 8 + 16);
     int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
     const uint32_t rank = cluster_ctarank();
     const int cid = (int)cluster_id_x(), ncl = (int)ncluster_x();
 
@@ -593,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int arow = s_off[lo] + m * pr::PM + (int)rank * BM;
             const int n0 = nb * OUT_N;
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -638,14 +640,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int t = cid; t < total && ok; t += ncl, ++i) {
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t dt = tmem_base + (uint32_t)(buf * MMA_N);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -691,7 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int n0 = nb * OUT_N;
             const int buf = i & 1;
             const uint32_t tp = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wait_limit())) break;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wl)) break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * MMA_N);
             const int grow = s_off[lo] + m * pr::PM + (int)rank * BM + r_in_tile;

@@ -185,6 +185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* s_off = reinterpret_cast<int*>(meta + NUM_BARS * 8 + 16);
     int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
 
     if (!block_tile_table(offsets, E, R, s_off, s_toff, s_bad, status)) return;
     const int NB = (N + OUT_N - 1) / OUT_N;
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
             for (int kb = 0; kb < KS; ++kb) {
-                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -280,13 +281,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
             // the epilogue has moved the previous tile's accumulator out
             if (!mbar_wait(smem_u32(tempty), ((uint32_t)i & 1u) ^ 1u, s_abort, status,
-                           wait_limit())) {
+                           wl)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             for (int kb = 0; kb < KS; ++kb) {
-                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                     ok = false;
                     break;
                 }
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const Tile tl = decode_tile(t, NB, E, OUT_N, s_toff, s_off);
-            if (!mbar_wait(smem_u32(tfull), (uint32_t)i & 1u, s_abort, status, wait_limit()))
+            if (!mbar_wait(smem_u32(tfull), (uint32_t)i & 1u, s_abort, status, wl))
                 break;
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);

@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
     const int m0 = blockIdx.x * RT_BM;
     const int n0 = blockIdx.y * EN;
     const int KS = d / 64;  // 128-byte slabs of bf16
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KS; ++kb) {
-            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wait_limit())) {
+            if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
                 ok = false;
                 break;
             }
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 if (er + 128 < EN && n0 + er + 128 < E) wnorm2[n0 + er + 128] = sw1;
             }
         }
-        if (ok && mbar_wait(smem_u32(done), 0, s_abort, status, wait_limit())) {
+        if (ok && mbar_wait(smem_u32(done), 0, s_abort, status, wl)) {
             tc_fence_after();
             const int t = m0 + q * 32 + lane;
             const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16);
