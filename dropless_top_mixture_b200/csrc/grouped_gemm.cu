@@ -766,12 +766,469 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
     return launch_status();
 }
 
+// ------------------------------------------------------ token-column tiles
+//
+// The same products with the operands' roles swapped: the 256 MMA rows of a
+// CTA pair are weight rows and its N columns are one expert's tokens, so a
+// tile covers N = 16 .. 256 tokens in steps of 16 rather than 128 or 256
+// rows. An expert of c rows is cut into chunks of 256 rows and a last chunk
+// of the remaining rows rounded up to 16, so the MMAs compute at most 15
+// masked rows per expert (experts of about 256 rows: 3% of the MMA work,
+// against 20% for 128-row tiles).
+//
+// Each pipeline stage holds two 128-byte K slabs, and each CTA fetches it
+// with two TMA copies (one of weights, one of tokens) of up to 32 KB: on
+// B200 the copy engine's rate depends on the number of copies far more than
+// on their size (two 16 KB copies per 32 KB stage stream about two thirds
+// as fast as one 32 KB copy), so the weight and token boxes each span both
+// slabs through a map whose last dimension steps 128 bytes along K.
+//
+// gate/up: a 5-D map over the W1 and W3 rows delivers, for each TMEM lane
+// quarter q of CTA r, 16 rows of the first tensor and then the same 16
+// features' rows of the second (features f0 + 64 r + 16 q ..), so lanes l
+// and l + 16 of an epilogue warp hold the gate and up pre-activations of
+// one feature and one shuffle pairs them for the SwiGLU; the pair covers 128
+// features of H. down: CTA r holds 128 rows of W2 (output features
+// f0 + 128 r ..); the pair covers 256. Tokens: CTA r copies rows
+// row0 + r N/2 .. with the smallest box of 8 .. 128 rows that covers N/2
+// (rows past the chunk are fetched and never multiplied). Accumulator column
+// c is token row0 + c and TMEM lane i is feature i of the CTA's rows, so the
+// epilogue writes each token's run of the quarter's features (32 or 64
+// contiguous bytes). Tiles run expert by expert, feature block major and
+// chunk minor, so the chunks that share a weight block run together.
+namespace sw {
+constexpr int STAGES = 3;
+constexpr int SLABS = 2;                    // 128-byte K slabs per stage
+constexpr int A_BYTES = SLABS * 128 * 128;  // 128 weight rows
+constexpr int B_BYTES = SLABS * 128 * 128;  // up to 128 token rows (half of N = 256)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int META_BYTES = NUM_BARS * 8 + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + META_BYTES;
+constexpr int NBOX = 5;                     // token boxes of 8, 16, 32, 64, 128 rows
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+struct TokenMaps {
+    CUtensorMap m[NBOX];
+};
+
+struct Chunk {
+    int e, fb, row0, row_end, n;
+};
+
+// Tile t -> (expert, feature block, token chunk); s_toff is the prefix of
+// the experts' chunk counts.
+__device__ __forceinline__ Chunk decode(int t, int FB, int E, const int* s_toff, const int* s_off) {
+    const int q = t / FB;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_toff[mid] <= q) lo = mid;
+        else hi = mid - 1;
+    }
+    const int ch = s_toff[lo + 1] - s_toff[lo];
+    const int l = t - s_toff[lo] * FB;
+    const int fb = l / ch, j = l - fb * ch;
+    Chunk c;
+    c.e = lo;
+    c.fb = fb;
+    c.row0 = s_off[lo] + 256 * j;
+    const int rows = min(256, s_off[lo + 1] - c.row0);
+    c.row_end = c.row0 + rows;
+    c.n = (rows + 15) & ~15;
+    return c;
+}
+
+// smallest token box (index into TokenMaps) covering `half` rows
+__device__ __forceinline__ int box_sel(int half) {
+    return half <= 8 ? 0 : half <= 16 ? 1 : half <= 32 ? 2 : half <= 64 ? 3 : 4;
+}
+
+template <typename T>
+__device__ __forceinline__ T to_out(float v);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ float to_out<float>(float v) {
+    return v;
+}
+}  // namespace sw
+
+template <typename TIn, bool SWIGLU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW,
+                             const __grid_constant__ sw::TokenMaps tmX,
+                             const int32_t* __restrict__ offsets, int E, int R, int K, int NOUT,
+                             int wpe, int second_is_gate, TIn* __restrict__ out, int64_t ldo,
+                             TIn* __restrict__ save_a, TIn* __restrict__ save_b, int* status) {
+    constexpr bool TF32 = std::is_same<TIn, float>::value;
+    constexpr int BK = 128 / (int)sizeof(TIn);
+    constexpr uint32_t IDESC_M = make_idesc(TF32 ? 2u : 1u, 256, 0);  // N filled per tile
+    constexpr int STAGES = sw::STAGES;
+    constexpr int FEAT = SWIGLU ? 128 : 256;  // output features per pair tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* meta = smem + STAGES * sw::STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + sw::NUM_BARS * 8);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    int* s_bad = reinterpret_cast<int*>(s_tmem + 2);
+    int* s_off = reinterpret_cast<int*>(meta + sw::NUM_BARS * 8 + 16);
+    int* s_toff = s_off + (MOE_MAX_EXPERTS + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t wl = wait_limit();  // the pipeline waits' time limit, read once
+    const uint32_t rank = cluster_ctarank();
+    const int cid = (int)cluster_id_x(), ncl = (int)ncluster_x();
+
+    // --- chunk table from the routing offsets (validated) ------------------
+    for (int e = tid; e <= E; e += THREADS) s_off[e] = offsets[e];
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int ch = 0;
+            if (e < E) {
+                const int cnt = s_off[e + 1] - s_off[e];
+                if (cnt < 0) bad = true;
+                else ch = (cnt + 255) >> 8;
+            }
+            int tot;
+            const int ex = warp_exclusive_scan(ch, &tot);
+            if (e < E) s_toff[e] = carry + ex;
+            carry += tot;
+        }
+        bad = __any_sync(0xffffffffu, bad) || s_off[0] != 0 || s_off[E] != R;
+        if (lane == 0) {
+            s_toff[E] = carry;
+            *s_bad = bad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    // both CTAs of a pair see the same offsets, so they leave here together
+    if (*s_bad) {
+        if (tid == 0 && blockIdx.x == 0) set_status(status, MOE_DEVERR_BAD_OFFSETS);
+        return;
+    }
+    const int FB = NOUT / FEAT;
+    const int total = s_toff[E] * FB;
+    if (cid >= total) return;
+    const int KS = K / (sw::SLABS * BK);  // stages per tile
+
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(tfull + b), 1);
+            mbar_init(smem_u32(tempty + b), 2 * EPI_WARPS);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmW);
+        for (int b = 0; b < sw::NBOX; ++b) prefetch_map(&tmX.m[b]);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(s_tmem), 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const uint32_t leader_full = map_to_cta(smem_u32(full), 0);
+    const uint32_t leader_tempty = map_to_cta(smem_u32(tempty), 0);
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+        bool ok = true;
+        for (int t = cid; t < total && ok; t += ncl) {
+            const sw::Chunk c = sw::decode(t, FB, E, s_toff, s_off);
+            const int half = c.n >> 1;  // token rows of this CTA (a multiple of 8)
+            const int bs = sw::box_sel(half);
+            const CUtensorMap* xm = &tmX.m[bs];
+            const int brow = c.row0 + (int)rank * half;
+            const uint32_t tx = 2u * (uint32_t)(sw::A_BYTES + (8 << bs) * 128 * sw::SLABS);
+            const int wcoord = SWIGLU ? c.e * wpe + c.fb * 8 + 4 * (int)rank
+                                      : c.e * wpe + c.fb * FEAT + 128 * (int)rank;
+            for (int ks = 0; ks < KS; ++ks) {
+                if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, s_abort, status, wl)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fbar = leader_full + (uint32_t)stage * 8u;
+                const uint32_t sa = smem_u32(smem + stage * sw::STAGE_BYTES);
+                if (rank == 0) mbar_expect_tx(smem_u32(full + stage), tx);
+                if (SWIGLU)
+                    tma_load_5d_pair(sa, &tmW, fbar, 0, 0, 0, wcoord, sw::SLABS * ks);
+                else
+                    tma_load_3d_pair(sa, &tmW, fbar, 0, wcoord, sw::SLABS * ks);
+                tma_load_3d_pair(sa + sw::A_BYTES, xm, fbar, 0, brow, sw::SLABS * ks);
+                issued_mask |= 1u << stage;
+                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            // the leader's stage barriers count both CTAs' copies: wait there
+            // (bounded); the partner gives its copies a bounded grace period
+            if (rank == 0) {
+                for (int s = 0; s < STAGES; ++s)
+                    if ((issued_mask >> s) & 1u) {
+                        volatile int no_abort = 0;
+                        mbar_wait(smem_u32(full + s), (issued_parity >> s) & 1u, &no_abort, nullptr,
+                                  DRAIN_LIMIT_NS);
+                    }
+            } else {
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 1000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------ MMA issuer (leader)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int i = 0;
+        for (int t = cid; t < total && ok; t += ncl, ++i) {
+            const sw::Chunk c = sw::decode(t, FB, E, s_toff, s_off);
+            const uint32_t idesc = IDESC_M | ((uint32_t)(c.n >> 3) << 17);
+            const uint32_t bslab = (uint32_t)(8 << sw::box_sel(c.n >> 1)) * 128u;  // B slab stride
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tempty + buf), tp ^ 1u, s_abort, status, wl)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem_base + (uint32_t)(buf * 256);
+            for (int ks = 0; ks < KS; ++ks) {
+                if (!mbar_wait(smem_u32(full + stage), phase, s_abort, status, wl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + stage * sw::STAGE_BYTES);
+#pragma unroll
+                for (int sl = 0; sl < sw::SLABS; ++sl) {
+                    const uint64_t ad = sw128_desc(sa + (uint32_t)sl * (128u * 128u));
+                    const uint64_t bd = sw128_desc(sa + sw::A_BYTES + (uint32_t)sl * bslab);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc_mma_pair<TF32>(dt, ad + 2 * k, bd + 2 * k, idesc, (ks | sl | k) != 0);
+                }
+                tc_commit_pair(smem_u32(empty + stage), 0x3);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit_pair(smem_u32(tfull + buf), 0x3);
+        }
+        if (!ok) {
+            tc_commit_pair(smem_u32(drain), 0x1);
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(drain), 0, &no_abort, nullptr, DRAIN_LIMIT_NS);
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (both CTAs)
+        // warp w reads TMEM lane quarter w % 4; the two warps of a quarter
+        // take alternate 32-column (token) chunks
+        const int qd = warp & 3;
+        const int h = (warp - 2) >> 2;
+        const bool lo = lane < 16;
+        const bool holds_gate = lo != (second_is_gate != 0);
+        int i = 0;
+        for (int t = cid; t < total; t += ncl, ++i) {
+            const sw::Chunk c = sw::decode(t, FB, E, s_toff, s_off);
+            const int buf = i & 1;
+            const uint32_t tp = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(smem_u32(tfull + buf), tp, s_abort, status, wl)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * 256);
+            const int f = SWIGLU ? c.fb * FEAT + 64 * (int)rank + 16 * qd + (lane & 15)
+                                 : c.fb * FEAT + 128 * (int)rank + 32 * qd + lane;
+            const int nch = (c.n + 31) >> 5;
+#pragma unroll 1
+            for (int ck = h; ck < nch; ck += 2) {
+                uint32_t a[32];
+                tmem_ld32(ta + (uint32_t)(ck * 32), a);
+                tmem_wait_ld();
+                const int tok0 = c.row0 + ck * 32;
+                if constexpr (SWIGLU) {
+                    if (save_a != nullptr) {
+                        // pre-activations kept for the backward pass
+                        TIn* dst = holds_gate ? save_a : save_b;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (tok0 + j < c.row_end)
+                                dst[(size_t)(tok0 + j) * ldo + f] =
+                                    sw::to_out<TIn>(__uint_as_float(a[j]));
+                    }
+                    // lane l < 16 finishes tokens 0..15 of the chunk with the
+                    // values of lane l + 16, which finishes tokens 16..31
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float mine_lo = __uint_as_float(a[j]);
+                        const float mine_hi = __uint_as_float(a[16 + j]);
+                        const float other =
+                            __shfl_xor_sync(0xffffffffu, lo ? mine_hi : mine_lo, 16);
+                        const float mine = lo ? mine_lo : mine_hi;
+                        const float g = holds_gate ? mine : other;
+                        const float u = holds_gate ? other : mine;
+                        const int tok = tok0 + (lo ? 0 : 16) + j;
+                        if (tok < c.row_end)
+                            out[(size_t)tok * ldo + f] = sw::to_out<TIn>(silu_mul(g, u));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (tok0 + j < c.row_end)
+                            out[(size_t)(tok0 + j) * ldo + f] = sw::to_out<TIn>(__uint_as_float(a[j]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty + (uint32_t)buf * 8u);
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+// Token maps over X [R, K]: dims (128-byte slab, rows, slabs), boxes of
+// 8 .. 128 rows spanning two slabs.
+inline bool make_token_maps(sw::TokenMaps* tm, const void* X, CUtensorMapDataType dt, int es,
+                            int64_t K, int64_t R) {
+    const uint64_t bk = 128 / es;
+    const uint64_t dims[3] = {bk, (uint64_t)R, (uint64_t)K / bk};
+    const uint64_t strides[2] = {(uint64_t)K * es, 128};
+    for (int b = 0; b < sw::NBOX; ++b) {
+        const uint32_t box[3] = {(uint32_t)bk, 8u << b, (uint32_t)sw::SLABS};
+        if (!make_map_nd(&tm->m[b], X, dt, 3, dims, strides, box)) return false;
+    }
+    return true;
+}
+
+// gate/up weight map: dims (slab, 16 rows, 2 tensors, 16-row groups, slabs)
+// over the W1 and W3 rows, the lower address first; needs the expert stride
+// to be a whole number of 16-row groups and the two tensors a multiple of 16
+// bytes apart. *second_is_gate tells which tensor is first.
+inline bool gate_up_map_fits(const void* W1, const void* W3, int64_t estride, int64_t E,
+                             int64_t d, int es) {
+    const int64_t diff = (int64_t)((const char*)W3 - (const char*)W1);
+    const int64_t ad = diff < 0 ? -diff : diff;
+    return ad > 0 && ad % 16 == 0 && ad < (int64_t(1) << 40) && (E == 1 || estride % (16 * d) == 0) &&
+           (int64_t)d * es < (int64_t(1) << 40);
+}
+inline bool make_gate_up_map(CUtensorMap* m, const void* W1, const void* W3, CUtensorMapDataType dt,
+                             int es, int64_t estride, int64_t E, int64_t d, int64_t F, int* wpe,
+                             int* second_is_gate) {
+    const bool w3_first = (const char*)W3 < (const char*)W1;
+    const void* base = w3_first ? W3 : W1;
+    const int64_t diff = w3_first ? (const char*)W1 - (const char*)W3 : (const char*)W3 - (const char*)W1;
+    const int64_t gpe = E == 1 ? F / 16 : estride / (16 * d);
+    const uint64_t bk = 128 / es;
+    const uint64_t dims[5] = {bk, 16, 2, (uint64_t)((E - 1) * gpe + F / 16), (uint64_t)d / bk};
+    const uint64_t strides[4] = {(uint64_t)d * es, (uint64_t)diff, (uint64_t)(16 * d * es), 128};
+    const uint32_t box[5] = {(uint32_t)bk, 16, 2, 4, (uint32_t)sw::SLABS};
+    *wpe = (int)gpe;
+    *second_is_gate = w3_first ? 1 : 0;
+    return make_map_nd(m, base, dt, 5, dims, strides, box);
+}
+// down weight map: dims (slab, rows of all experts, slabs) over W2 [E, d, F];
+// needs the expert stride to be a whole number of rows.
+inline bool down_map_fits(int64_t estride, int64_t E, int64_t F) {
+    return E == 1 || estride % F == 0;
+}
+inline bool make_down_map(CUtensorMap* m, const void* W2, CUtensorMapDataType dt, int es,
+                          int64_t estride, int64_t E, int64_t d, int64_t F, int* wpe) {
+    const int64_t rpe = E == 1 ? d : estride / F;
+    const uint64_t bk = 128 / es;
+    const uint64_t dims[3] = {bk, (uint64_t)((E - 1) * rpe + d), (uint64_t)F / bk};
+    const uint64_t strides[2] = {(uint64_t)F * es, 128};
+    const uint32_t box[3] = {(uint32_t)bk, 128, (uint32_t)sw::SLABS};
+    *wpe = (int)rpe;
+    return make_map_nd(m, W2, dt, 3, dims, strides, box);
+}
+
+template <typename TIn, bool SWIGLU>
+static int launch_swap(const CUtensorMap& w, const sw::TokenMaps& x, const int32_t* offsets,
+                       int64_t E, int64_t R, int64_t K, int64_t NOUT, int wpe, int second_is_gate,
+                       void* out, int64_t ldo, cudaStream_t st, void* save_a = nullptr,
+                       void* save_b = nullptr) {
+    auto kern = grouped_gemm_swap_kernel<TIn, SWIGLU>;
+    if (check_only()) return MOE_OK;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sw::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const int64_t feat = SWIGLU ? 128 : 256;
+    const int64_t max_tiles = (R / 256 + E) * (NOUT / feat);
+    const int64_t pairs = num_sms() / 2;
+    const int npairs = (int)(max_tiles < pairs ? max_tiles : pairs);
+    if (npairs <= 0) return MOE_OK;
+    kern<<<2 * npairs, THREADS, sw::SMEM_BYTES, st>>>(
+        w, x, offsets, (int)E, (int)R, (int)K, (int)NOUT, wpe, second_is_gate,
+        static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a), static_cast<TIn*>(save_b),
+        status_ptr());
+    return launch_status();
+}
+
 // Measured on B200: the pair tile speeds up the down GEMM (olmoe-shaped layer
 // 1071 -> 1143 TFLOP/s) but not gate/up, which already runs at the
 // power-capped clock; with about 256 rows per expert the pair's second half
 // computes many rows it then masks (128-expert sweep: slower). So it is
 // used for the down GEMM when experts average at least 512 rows.
 inline bool use_pair(int64_t R, int64_t E) { return R >= 512 * E; }
+
+// Tile form: 0 = chosen by shape, 1 = row tiles, 2 = token-column tiles
+// (where the weight strides allow them). Set by moe_debug_set_gemm_form.
+inline int& gemm_form() {
+    static int form = 0;
+    return form;
+}
+
+// Measured on B200 (bf16, power-capped layer steps and isolated calls):
+// token-column tiles run gate/up 8-12% and down up to 26% faster than row
+// tiles when experts average 512 rows or more (OLMoE-shaped layer, 8 and 32
+// experts of the sweep); at about 256 rows per expert (128-expert sweep) the
+// last chunk of each expert streams a whole weight block for a few tokens
+// and row tiles are about 4% faster; below that the two trade places from
+// run to run. So: token columns from 512 rows per expert on.
+inline bool use_swap(int64_t R, int64_t E) {
+    const int f = gemm_form();
+    if (f != 0) return f == 2;
+    return R >= 512 * E;
+}
 
 static int check_common(const void* A, const void* B, const int32_t* offsets, int64_t E,
                         int64_t R, int64_t d, int64_t F, int dtype) {
@@ -804,11 +1261,24 @@ extern "C" int moe_grouped_gate_up_save(const void* Xe, const void* W1, const vo
     const CUtensorMapDataType dt =
         dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap a, b0, b1;
+    cudaStream_t st = as_stream(stream);
+    if (gg::use_swap(R, E) && gg::gate_up_map_fits(W1, W3, w13_expert_stride, E, d, es)) {
+        gg::sw::TokenMaps xm;
+        int wpe = 0, second_is_gate = 0;
+        if (!gg::make_gate_up_map(&b0, W1, W3, dt, es, w13_expert_stride, E, d, F, &wpe,
+                                  &second_is_gate) ||
+            !gg::make_token_maps(&xm, Xe, dt, es, d, R))
+            return MOE_ERR_CUDA;
+        if (dtype == MOE_BF16)
+            return gg::launch_swap<__nv_bfloat16, true>(b0, xm, offsets, E, R, d, F, wpe,
+                                                         second_is_gate, H, F, st, A_out, B_out);
+        return gg::launch_swap<float, true>(b0, xm, offsets, E, R, d, F, wpe, second_is_gate, H, F,
+                                            st, A_out, B_out);
+    }
     if (!gg::make_map_2d(&a, Xe, dt, es, d, R, gg::BM) ||
         !gg::make_map_3d(&b0, W1, dt, es, d, F, E, w13_expert_stride, 128) ||
         !gg::make_map_3d(&b1, W3, dt, es, d, F, E, w13_expert_stride, 128))
         return MOE_ERR_CUDA;
-    cudaStream_t st = as_stream(stream);
     if (dtype == MOE_BF16)
         return gg::launch<__nv_bfloat16, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st,
                                                      A_out, B_out);
@@ -865,8 +1335,20 @@ extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert
     const CUtensorMapDataType dt =
         dtype == MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int mma_n = (d % 256 == 0) ? 256 : 128;
-    const bool pair = mma_n == 256 && gg::use_pair(R, E);
     CUtensorMap a, b0;
+    if (mma_n == 256 && gg::use_swap(R, E) && gg::down_map_fits(w2_expert_stride, E, F)) {
+        gg::sw::TokenMaps xm;
+        int wpe = 0;
+        if (!gg::make_down_map(&b0, W2, dt, es, w2_expert_stride, E, d, F, &wpe) ||
+            !gg::make_token_maps(&xm, H, dt, es, F, R))
+            return MOE_ERR_CUDA;
+        cudaStream_t st = as_stream(stream);
+        if (dtype == MOE_BF16)
+            return gg::launch_swap<__nv_bfloat16, false>(b0, xm, offsets, E, R, F, d, wpe, 0, Ye, d,
+                                                          st);
+        return gg::launch_swap<float, false>(b0, xm, offsets, E, R, F, d, wpe, 0, Ye, d, st);
+    }
+    const bool pair = mma_n == 256 && gg::use_pair(R, E);
     if (!gg::make_map_2d(&a, H, dt, es, F, R, gg::BM) ||
         !gg::make_map_3d(&b0, W2, dt, es, F, d, E, w2_expert_stride, pair ? 128 : mma_n))
         return MOE_ERR_CUDA;
@@ -883,6 +1365,12 @@ extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert
     }
     if (mma_n == 256) return gg::launch<float, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
     return gg::launch<float, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+}
+
+extern "C" int moe_debug_set_gemm_form(int form) {
+    if (form < 0 || form > 2) return MOE_ERR_INVALID;
+    gg::gemm_form() = form;
+    return MOE_OK;
 }
 
 extern "C" int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, const void* W2,

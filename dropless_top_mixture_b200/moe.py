@@ -166,6 +166,7 @@ _SIGS = {
     "moe_dispatch_ep": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _i32, _i64, _p]),
     "moe_combine_ep": (_i32, [_p, _p, _p, _p, _i64, _i64, _i32, _i32, _i32, _i64, _p, _p]),
     "moe_debug_set_wait_limit_ns": (_i32, [ctypes.c_uint64]),
+    "moe_debug_set_gemm_form": (_i32, [_i32]),
     "moe_version": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -377,20 +378,30 @@ def moe_grouped_swiglu_bwd(Xe, A, B, H, dYe, W1, W3, W2, offsets,
                           dA=torch.empty((R, F), dtype=dt, device=dev),
                           dB=torch.empty((R, F), dtype=dt, device=dev))
     rc = lib.moe_grouped_swiglu_bwd(_ptr(Xe), _ptr(A), _ptr(B), _ptr(H), _ptr(dYe), _ptr(W1),
-                                    _ptr(W3), _ptr(W2), s13, W2.stride(0), _ptr(offsets), E, R, d,
+                                    _ptr(W3), _ptr(W2), s13, _w2(W2)[3], _ptr(offsets), E, R, d,
                                     F, _dtype_code(dt), _ptr(out.dA), _ptr(out.dB), _ptr(out.dXe),
                                     _ptr(out.dW1), _ptr(out.dW3), _ptr(out.dW2), _stream(Xe))
     _check("moe_grouped_swiglu_bwd", rc)
     return out
 
 
-def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch.Tensor:
-    _need(H, "H"); _need(W2, "W2"); _need(offsets, "offsets")
+def _w2(W2: torch.Tensor):
+    # [E,d,F] with rows contiguous; experts any (multiple of 8) stride apart
+    if not W2.is_cuda:
+        raise ValueError("W2 must be a CUDA tensor")
     E, d, F = W2.shape
+    if W2.stride(2) != 1 or W2.stride(1) != F:
+        raise ValueError("W2 must be [E,d,F] with rows contiguous")
+    return E, d, F, W2.stride(0)
+
+
+def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(H, "H"); _need(offsets, "offsets")
+    E, d, F, s2 = _w2(W2)
     R = H.shape[0]
     if Ye is None:
         Ye = torch.empty((R, d), dtype=H.dtype, device=H.device)
-    rc = lib.moe_grouped_down(_ptr(H), _ptr(W2), W2.stride(0), _ptr(offsets), E, R, d, F,
+    rc = lib.moe_grouped_down(_ptr(H), _ptr(W2), s2, _ptr(offsets), E, R, d, F,
                               _dtype_code(H.dtype), _ptr(Ye), _stream(H))
     _check("moe_grouped_down", rc)
     return Ye
@@ -398,14 +409,14 @@ def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch
 
 def moe_grouped_swiglu(Xe, W1, W3, W2, offsets, H: Optional[torch.Tensor] = None,
                        Ye: Optional[torch.Tensor] = None):
-    _need(Xe, "Xe"); _need(W2, "W2"); _need(offsets, "offsets")
+    _need(Xe, "Xe"); _need(offsets, "offsets")
     E, F, d, s13 = _w13(W1, W3)
     R = Xe.shape[0]
     if H is None:
         H = torch.empty((R, F), dtype=Xe.dtype, device=Xe.device)
     if Ye is None:
         Ye = torch.empty((R, d), dtype=Xe.dtype, device=Xe.device)
-    rc = lib.moe_grouped_swiglu(_ptr(Xe), _ptr(W1), _ptr(W3), _ptr(W2), s13, W2.stride(0),
+    rc = lib.moe_grouped_swiglu(_ptr(Xe), _ptr(W1), _ptr(W3), _ptr(W2), s13, _w2(W2)[3],
                                 _ptr(offsets), E, R, d, F, _dtype_code(Xe.dtype), _ptr(H),
                                 _ptr(Ye), _stream(Xe))
     _check("moe_grouped_swiglu", rc)
@@ -502,7 +513,7 @@ def moe_layer_fwd(x, k: int, W1, W3, W2, *, logits=None, Wr=None, renorm: bool =
     save_logits = out.logits if (save and logits is None) else None
     a = LayerArgs(T=T, d=d, E=E, F=F, k=k, dtype=_dtype_code(x.dtype), renorm=int(renorm),
                   reserved0=0, x=_ptr(x), logits=_ptr(logits), Wr=_ptr(Wr), W1=_ptr(W1),
-                  W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13, w2_expert_stride=W2.stride(0),
+                  W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13, w2_expert_stride=_w2(W2)[3],
                   out=_ptr(out.out), idx=_ptr(out.idx), gate=_ptr(out.gate),
                   counts=_ptr(out.counts), offsets=_ptr(out.offsets), slot=_ptr(out.slot),
                   workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel(),
@@ -575,7 +586,7 @@ class HostLayer:
         a = LayerArgs(T=self.T, d=self.d, E=E, F=F, k=self.k, dtype=_dtype_code(self.dtype),
                       renorm=int(renorm), reserved0=0, x=_ptr(self.x), logits=_ptr(self.logits),
                       Wr=_ptr(Wr), W1=_ptr(W1), W3=_ptr(W3), W2=_ptr(W2),
-                      w13_expert_stride=s13, w2_expert_stride=W2.stride(0), out=_ptr(r.out),
+                      w13_expert_stride=s13, w2_expert_stride=_w2(W2)[3], out=_ptr(r.out),
                       idx=_ptr(r.idx), gate=_ptr(r.gate), counts=_ptr(r.counts),
                       offsets=_ptr(r.offsets), slot=_ptr(r.slot), workspace=_ptr(r.workspace),
                       workspace_bytes=r.workspace.numel(), save_Xe=None, save_H=None,
@@ -636,7 +647,7 @@ def moe_layer_bwd(fwd: LayerOut, dOut, k: int, W1, W3, W2,
                      slot=_ptr(fwd.slot), gate=_ptr(fwd.gate), offsets=_ptr(fwd.offsets),
                      Xe=_ptr(fwd.Xe), A=_ptr(fwd.A), B=_ptr(fwd.B), H=_ptr(fwd.H), W1=_ptr(W1),
                      W3=_ptr(W3), W2=_ptr(W2), w13_expert_stride=s13,
-                     w2_expert_stride=W2.stride(0), dOut=_ptr(dOut), dx=_ptr(out.dx),
+                     w2_expert_stride=_w2(W2)[3], dOut=_ptr(dOut), dx=_ptr(out.dx),
                      dW1=_ptr(out.dW1), dW3=_ptr(out.dW3), dW2=_ptr(out.dW2),
                      workspace=_ptr(out.workspace), workspace_bytes=out.workspace.numel())
     if router:
@@ -795,6 +806,15 @@ def moe_debug_set_wait_limit_ns(ns: int, device=None) -> None:
     with torch.cuda.device(dev):
         rc = lib.moe_debug_set_wait_limit_ns(int(ns))
     _check("moe_debug_set_wait_limit_ns", rc)
+
+
+GEMM_FORM_AUTO, GEMM_FORM_ROWS, GEMM_FORM_TOKENS = 0, 1, 2
+
+
+def moe_debug_set_gemm_form(form: int) -> None:
+    """Test-only: tile form of the grouped GEMMs (GEMM_FORM_AUTO by shape,
+    GEMM_FORM_ROWS, GEMM_FORM_TOKENS where the weight layout allows)."""
+    _check("moe_debug_set_gemm_form", lib.moe_debug_set_gemm_form(int(form)))
 
 
 # ----------------------------------------------------------------- MXFP8 path
@@ -1034,7 +1054,7 @@ def mxfp8_quantize_weights_bwd(W1, W3, W2) -> MxWeightsBwd:
                       Ps13t=torch.empty(E * ((d + 255) // 256) * (2 * F // 128) * 1024, **u8),
                       Ps2t=torch.empty(E * ((F + 255) // 256) * (d // 128) * 1024, **u8))
     st = _stream(W1)
-    rc = lib.mxfp8_quantize_weights_bwd(_ptr(W1), _ptr(W3), _ptr(W2), s13, W2.stride(0), E, d, F,
+    rc = lib.mxfp8_quantize_weights_bwd(_ptr(W1), _ptr(W3), _ptr(W2), s13, _w2(W2)[3], E, d, F,
                                         _ptr(wb.W13tq), _ptr(wb.W13ts), _ptr(wb.W2tq),
                                         _ptr(wb.W2ts), st)
     _check("mxfp8_quantize_weights_bwd", rc)

@@ -226,6 +226,14 @@ MOE_API int moe_row_token(const int32_t* slot, int64_t T, int k, int32_t* row_to
  *   H   [R,F] device output/workspace; Ye [R,d] device output.
  * Limits: d % 128 == 0, F % 128 == 0, E <= 512; every pointer 16-byte
  * aligned; strides multiples of 8 elements.
+ * Two tile forms compute the same sums in the same order (bit-identical
+ * results): row tiles (128 or, for the down GEMM of experts averaging 512+
+ * rows, 256 expert rows x 256 weight rows) and token-column tiles (256
+ * weight rows x up to 256 of one expert's tokens, in steps of 16), chosen
+ * by shape: token columns when experts average 512 rows or more and the
+ * weight layout allows their maps (gate/up: the expert stride a multiple of
+ * 16*d and W3 - W1 a nonzero multiple of 16 bytes; down: the expert stride
+ * a multiple of F and d % 256 == 0), row tiles otherwise.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
                                 int64_t w13_expert_stride, const int32_t* offsets, int64_t E,
@@ -783,6 +791,13 @@ MOE_API int moe_get_status(int32_t* host_status, int clear, void* stream);
  * memory); do not change it while kernels of the library are running.
  * ---------------------------------------------------------------------- */
 MOE_API int moe_debug_set_wait_limit_ns(uint64_t ns);
+
+/* moe_debug_set_gemm_form — for tests: the tile form of the bf16/fp32
+ * grouped GEMMs (moe_grouped_gate_up[_save], moe_grouped_down and the layer
+ * entries that call them): 0 = by shape (the default), 1 = row tiles, 2 =
+ * token-column tiles wherever the weight layout allows them. Process-wide;
+ * MOE_ERR_INVALID for any other value. */
+MOE_API int moe_debug_set_gemm_form(int form);
 
 /* library version string */
 MOE_API const char* moe_version(void);

@@ -1,6 +1,8 @@
 """Grouped SwiGLU GEMMs (tcgen05) and the whole layer on the GPU against the
 oracle: small shapes that span several tiles with ragged tails and empty
 experts, then every workload at full size on sampled tokens."""
+import contextlib
+
 import numpy as np
 import pytest
 import torch
@@ -16,6 +18,19 @@ pytestmark = pytest.mark.gpu
 def _moe():
     from dropless_top_mixture_b200 import moe
     return moe
+
+
+@contextlib.contextmanager
+def _gemm_form(form):
+    """Force the grouped GEMMs' tile form (rows / token columns) inside."""
+    moe = _moe()
+    code = {"auto": moe.GEMM_FORM_AUTO, "rows": moe.GEMM_FORM_ROWS,
+            "tokens": moe.GEMM_FORM_TOKENS}[form]
+    moe.moe_debug_set_gemm_form(code)
+    try:
+        yield
+    finally:
+        moe.moe_debug_set_gemm_form(moe.GEMM_FORM_AUTO)
 
 
 def _problem(T, d, F, E, k, dtype, seed, skew=True):
@@ -76,12 +91,20 @@ LARGER_COUNTS = [1, 64, 127, 128, 129, 200, 255, 256, 257, 300, 384, 385, 511, 5
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("d,F", [(256, 256), (384, 128), (512, 384)])
 @pytest.mark.parametrize("which", ["small_experts", "larger_experts"])
-def test_grouped_swiglu_every_tail_size(dtype, d, F, which):
+@pytest.mark.parametrize("form", ["rows", "tokens"])
+def test_grouped_swiglu_every_tail_size(dtype, d, F, which, form):
     """Expert segments given directly by offsets, so every ragged tail size
     is met, with 16 experts averaging 104 rows and with experts averaging
-    259 rows (the gate/up GEMM on single-CTA tiles in both; the down GEMM
-    on CTA pairs where experts average 512 rows or more); A, B and H kept
-    for the backward are checked too."""
+    259 rows, on row tiles (128-row single-CTA tiles; the down GEMM on CTA
+    pairs where experts average 512 rows or more) and on token-column tiles
+    (256-row chunks and a last chunk of 1 .. 256 rows; d = 384 keeps the
+    down GEMM on row tiles); A, B and H kept for the backward are checked
+    too."""
+    with _gemm_form(form):
+        _every_tail_size(dtype, d, F, which)
+
+
+def _every_tail_size(dtype, d, F, which):
     moe = _moe()
     counts = np.array(TAIL_COUNTS if which == "small_experts" else LARGER_COUNTS,
                       dtype=np.int64)
@@ -186,6 +209,96 @@ def test_grouped_gate_up_fused_gate_up_layout():
     H = moe.moe_grouped_gate_up(Xe, gate_up[:, :F], gate_up[:, F:],
                                 torch.from_numpy(meta["offsets"]).cuda())
     assert_close_scaled(np64(H), H_ref, "H")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_token_tiles_equal_row_tiles_bitwise(dtype):
+    """Both tile forms sum each output over K in the same order, so H, the
+    saved pre-activations and Ye agree bit for bit."""
+    moe = _moe()
+    counts = np.array(LARGER_COUNTS + TAIL_COUNTS, dtype=np.int64)
+    E, R, d, F = len(counts), int(counts.sum()), 512, 256
+    offs = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).cuda()
+    g = torch.Generator().manual_seed(5)
+    Xe = torch.randn(R, d, generator=g).to(dtype).cuda()
+    W1 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(dtype).cuda()
+    W3 = (torch.randn(E, F, d, generator=g) * d ** -0.5).to(dtype).cuda()
+    W2 = (torch.randn(E, d, F, generator=g) * F ** -0.5).to(dtype).cuda()
+    out = {}
+    for form in ("rows", "tokens"):
+        with _gemm_form(form):
+            H, A, B = moe.moe_grouped_gate_up_save(Xe, W1, W3, offs)
+            Ye = moe.moe_grouped_down(H, W2, offs)
+        out[form] = (H, A, B, Ye)
+    assert moe.moe_get_status() == 0
+    for a, b, name in zip(out["rows"], out["tokens"], "H A B Ye".split()):
+        assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("w3_first", [False, True])
+def test_token_tiles_fused_gate_up_either_order(w3_first):
+    """Token-column gate/up on the two halves of one [E, 2F, d] tensor, W1
+    the first half or the second (the map then starts at W3 and the
+    epilogue takes the gate from the upper lanes)."""
+    moe = _moe()
+    T, d, F, E, k = 900, 256, 256, 3, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=43)
+    meta, gate, Xe_ref, H_ref, Ye_ref = _expert_ref(x, W1, W3, W2, lg, k)
+    both = torch.cat([W3, W1] if w3_first else [W1, W3], dim=1).cuda()
+    w1 = both[:, F:] if w3_first else both[:, :F]
+    w3 = both[:, :F] if w3_first else both[:, F:]
+    Xe = torch.from_numpy(Xe_ref).to(torch.bfloat16).cuda()
+    offs = torch.from_numpy(meta["offsets"]).cuda()
+    with _gemm_form("tokens"):
+        H, A, B = moe.moe_grouped_gate_up_save(Xe, w1, w3, offs)
+    assert moe.moe_get_status() == 0
+    assert_close_scaled(np64(H), H_ref, "H")
+    with _gemm_form("rows"):
+        H2, A2, B2 = moe.moe_grouped_gate_up_save(Xe, w1, w3, offs)
+    assert torch.equal(H, H2) and torch.equal(A, A2) and torch.equal(B, B2)
+
+
+def test_token_form_falls_back_on_padded_expert_stride():
+    """An expert stride that is not a whole number of 16-row groups (gate/up)
+    or of rows (down) cannot be mapped for token columns: the row tiles run
+    instead, with the same results."""
+    moe = _moe()
+    T, d, F, E, k = 700, 256, 256, 4, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=44)
+    meta, gate, Xe_ref, H_ref, Ye_ref = _expert_ref(x, W1, W3, W2, lg, k)
+    pad13 = torch.zeros(E, F + 8, d, dtype=torch.bfloat16)
+    pad13[:, :F] = W1
+    w1 = pad13.cuda()[:, :F]
+    pad3 = torch.zeros(E, F + 8, d, dtype=torch.bfloat16)
+    pad3[:, :F] = W3
+    w3 = pad3.cuda()[:, :F]
+    pad2 = torch.zeros(E, d + 1, F, dtype=torch.bfloat16)
+    pad2[:, :d] = W2
+    w2 = pad2.cuda()[:, :d]
+    Xe = torch.from_numpy(Xe_ref).to(torch.bfloat16).cuda()
+    offs = torch.from_numpy(meta["offsets"]).cuda()
+    with _gemm_form("tokens"):
+        H = moe.moe_grouped_gate_up(Xe, w1, w3, offs)
+        Ye = moe.moe_grouped_down(H, w2, offs)
+    assert moe.moe_get_status() == 0
+    assert_close_scaled(np64(H), H_ref, "H")
+    assert_close_scaled(np64(Ye), Ye_ref, "Ye")
+
+
+@pytest.mark.parametrize("form", ["rows", "tokens"])
+def test_layer_fwd_save_either_tile_form(form):
+    """The whole layer forward (saving A, B and H for the backward) on each
+    tile form."""
+    moe = _moe()
+    T, d, F, E, k = 1500, 256, 256, 4, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=45)
+    ref = O.moe_layer(x, k, W1, W3, W2, logits=lg)
+    with _gemm_form(form):
+        r = moe.moe_layer_fwd(x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda(),
+                              logits=torch.from_numpy(lg).cuda(), save=True)
+    assert moe.moe_get_status() == 0
+    assert np.array_equal(r.idx.cpu().numpy(), ref["idx"])
+    assert_close_layer(np64(r.out), ref["out"], "out")
 
 
 def test_grouped_gemm_deterministic():
