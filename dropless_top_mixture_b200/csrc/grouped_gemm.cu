@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const int32_t* __restrict__ offsets, int E, int R, int K, int N,
                         TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
                         TIn* __restrict__ save_b, int* status,
-                        const int32_t* __restrict__ row_token, int x_rows) {
+                        const int32_t* __restrict__ row_token, int x_rows, int b_mode) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -262,8 +262,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sb = sa + C::A_BYTES;
                 if (lane == 0) {
                     mbar_expect_tx(fb, C::STAGE_BYTES);
-                    tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
-                    tma_load_3d(sb + C::B_BYTES / 2, &tmB1, fb, kb * C::BK, tl.n0, tl.e);
+                    if (b_mode) {
+                        tma_load_4d(sb, &tmB0, fb, kb * C::BK, tl.n0, 0, tl.e);
+                    } else {
+                        tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
+                        tma_load_3d(sb + C::B_BYTES / 2, &tmB1, fb, kb * C::BK, tl.n0, tl.e);
+                    }
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                 }
@@ -303,7 +307,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sb = sa + C::A_BYTES;
                 mbar_expect_tx(fb, C::STAGE_BYTES);
                 tma_load_2d(sa, &tmA, fb, kb * C::BK, tl.row0);
-                if (SWIGLU) {
+                if (SWIGLU && b_mode) {
+                    // W1 and W3 blocks in one copy (a map with both tensors
+                    // as its third dimension)
+                    tma_load_4d(sb, &tmB0, fb, kb * C::BK, tl.n0, 0, tl.e);
+                } else if (SWIGLU) {
                     tma_load_3d(sb, &tmB0, fb, kb * C::BK, tl.n0, tl.e);
                     tma_load_3d(sb + C::B_BYTES / 2, &tmB1, fb, kb * C::BK, tl.n0, tl.e);
                 } else {
@@ -373,6 +381,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int c_lo = ((warp - 2) >> 2) * (C::OUT_N / 64);  // this warp's half of the
         const int c_hi = c_lo + C::OUT_N / 64;                  // 32-column chunks
         const int r_in_tile = q * 32 + lane;
+        // accumulator columns of the gate and up halves (b_mode 2: the
+        // fused copy puts W3's block first)
+        const int gcol = b_mode == 2 ? C::OUT_N : 0;
+        const int ucol = b_mode == 2 ? 0 : C::OUT_N;
         int i = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
             const Tile tl = decode_tile(t, NB, E, C::OUT_N, s_toff, s_off);
@@ -388,10 +400,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t a[32];
                 float v[32];
-                tmem_ld32(ta + c * 32, a);
+                tmem_ld32(ta + (SWIGLU ? gcol : 0) + c * 32, a);
                 if constexpr (SWIGLU) {
                     uint32_t b[32];
-                    tmem_ld32(ta + C::OUT_N + c * 32, b);
+                    tmem_ld32(ta + ucol + c * 32, b);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
@@ -430,7 +442,7 @@ template <typename TIn, bool SWIGLU, int MMA_N, bool GATHER = false>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, void* out,
                   int64_t ldo, cudaStream_t st, void* save_a = nullptr, void* save_b = nullptr,
-                  const int32_t* row_token = nullptr, int64_t x_rows = 0) {
+                  const int32_t* row_token = nullptr, int64_t x_rows = 0, int b_mode = 0) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N, GATHER>;
     if (check_only()) return MOE_OK;
@@ -450,7 +462,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     kern<<<grid, THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K, (int)N,
                                               static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a),
                                               static_cast<TIn*>(save_b), status_ptr(), row_token,
-                                              (int)x_rows);
+                                              (int)x_rows, b_mode);
     return launch_status();
 }
 
@@ -1230,6 +1242,23 @@ inline bool use_swap(int64_t R, int64_t E) {
     return R >= 512 * E;
 }
 
+// Row-tile gate/up B map: dims (slab, F rows, 2 tensors, E) over W1 and W3,
+// the lower address first, so one copy fetches both 128-row blocks. Returns
+// the mode for the kernel (1: W1 first, 2: W3 first) or 0 when the two
+// tensors are not a multiple of 16 bytes apart (two maps then).
+inline int make_w13_map(CUtensorMap* m, const void* W1, const void* W3, CUtensorMapDataType dt,
+                        int es, int64_t estride, int64_t E, int64_t d, int64_t F) {
+    const int64_t diff = (int64_t)((const char*)W3 - (const char*)W1);
+    const int64_t ad = diff < 0 ? -diff : diff;
+    if (ad == 0 || ad % 16 != 0 || ad >= (int64_t(1) << 40)) return 0;
+    const uint64_t bk = 128 / es;
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)F, 2, (uint64_t)E};
+    const uint64_t strides[3] = {(uint64_t)d * es, (uint64_t)ad, (uint64_t)estride * es};
+    const uint32_t box[4] = {(uint32_t)bk, 128, 2, 1};
+    if (!make_map_nd(m, diff > 0 ? W1 : W3, dt, 4, dims, strides, box)) return -1;
+    return diff > 0 ? 1 : 2;
+}
+
 static int check_common(const void* A, const void* B, const int32_t* offsets, int64_t E,
                         int64_t R, int64_t d, int64_t F, int dtype) {
     if (E < 1 || E > MOE_MAX_EXPERTS || R < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID;
@@ -1275,14 +1304,18 @@ extern "C" int moe_grouped_gate_up_save(const void* Xe, const void* W1, const vo
         return gg::launch_swap<float, true>(b0, xm, offsets, E, R, d, F, wpe, second_is_gate, H, F,
                                             st, A_out, B_out);
     }
-    if (!gg::make_map_2d(&a, Xe, dt, es, d, R, gg::BM) ||
-        !gg::make_map_3d(&b0, W1, dt, es, d, F, E, w13_expert_stride, 128) ||
-        !gg::make_map_3d(&b1, W3, dt, es, d, F, E, w13_expert_stride, 128))
+    if (!gg::make_map_2d(&a, Xe, dt, es, d, R, gg::BM)) return MOE_ERR_CUDA;
+    const int b_mode = gg::make_w13_map(&b0, W1, W3, dt, es, w13_expert_stride, E, d, F);
+    if (b_mode < 0) return MOE_ERR_CUDA;
+    if (b_mode == 0 && (!gg::make_map_3d(&b0, W1, dt, es, d, F, E, w13_expert_stride, 128) ||
+                        !gg::make_map_3d(&b1, W3, dt, es, d, F, E, w13_expert_stride, 128)))
         return MOE_ERR_CUDA;
+    if (b_mode != 0) b1 = b0;
     if (dtype == MOE_BF16)
         return gg::launch<__nv_bfloat16, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st,
-                                                     A_out, B_out);
-    return gg::launch<float, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st, A_out, B_out);
+                                                     A_out, B_out, nullptr, 0, b_mode);
+    return gg::launch<float, true, 256>(a, b0, b1, offsets, E, R, d, F, H, F, st, A_out, B_out,
+                                        nullptr, 0, b_mode);
 }
 
 extern "C" int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
