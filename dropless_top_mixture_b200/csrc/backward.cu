@@ -61,7 +61,10 @@ constexpr bool is_dw() { return MODE == DW || MODE == DWF || MODE == DWS; }
 // in flight) and each epilogue warp has one staging buffer for its TMA
 // tensor stores; with fewer rows (DWS) a tile is one or two slabs and the
 // stores bound it, so 3 stages and 2 staging buffers per warp. The expert
-// offsets are read from global memory instead of a shared table.
+// offsets are read from global memory instead of a shared table. (One 8 KB
+// store per warp and tile instead of two 4 KB ones needs the room of a
+// load stage and measured slower on B200: the 4th stage is what lets the
+// next tile's loads run ahead.)
 template <int MODE>
 struct ModeCfg {
     static constexpr bool A_MN = is_dw<MODE>();
@@ -255,27 +258,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                 const uint32_t sb = sa + A_BYTES;
                 mbar_expect_tx(fb, STAGE_BYTES);
+                // one copy per operand: the MN-major operands' 64-column
+                // boxes come as the chunks of one box of a map whose third
+                // dimension steps 64 columns (few large copies stream faster
+                // than many small ones on B200)
                 if (MODE == DH || MODE == DXR) {
                     tma_load_2d(sa, &tmA0, fb, kb * BK, tl.row0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tma_load_3d(sb + j * BOX_BYTES, &tmB0, fb, tl.n0 + j * 64, kb * BK, tl.e);
+                    tma_load_4d(sb, &tmB0, fb, 0, kb * BK, tl.n0 / 64, tl.e);
                 } else if (MODE == DX) {
                     const bool second = kb >= KF;
                     const int kf = second ? kb - KF : kb;
                     tma_load_2d(sa, second ? &tmA1 : &tmA0, fb, kf * BK, tl.row0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tma_load_3d(sb + j * BOX_BYTES, second ? &tmB1 : &tmB0, fb,
-                                    tl.n0 + j * 64, kf * BK, tl.e);
+                    tma_load_4d(sb, second ? &tmB1 : &tmB0, fb, 0, kf * BK, tl.n0 / 64, tl.e);
                 } else {
                     const int r = tl.row0 + kb * BK;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        tma_load_2d(sa + i * BOX_BYTES, &tmA0, fb, tl.m0 + i * 64, r);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tma_load_2d(sb + j * BOX_BYTES, &tmB0, fb, tl.n0 + j * 64, r);
+                    tma_load_3d(sa, &tmA0, fb, 0, r, tl.m0 / 64);
+                    tma_load_3d(sb, &tmB0, fb, 0, r, tl.n0 / 64);
                 }
                 issued_mask |= 1u << stage;
                 issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -540,6 +538,18 @@ static int launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMa
 
 constexpr CUtensorMapDataType BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
+// MN-major operand map over bf16 [rows, cols] (E == 0) or E such matrices
+// `estride` elements apart: dims (64 columns, rows, cols / 64 chunks[, E]),
+// so one box of `chunks` chunks x 64 rows lands as `chunks` consecutive
+// 64-row x 128-byte tiles, the layout the MN-major MMA descriptors read.
+inline bool make_mn_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t E,
+                        int64_t estride, uint32_t chunks) {
+    const uint64_t dims[4] = {64, (uint64_t)rows, (uint64_t)cols / 64, (uint64_t)(E > 0 ? E : 1)};
+    const uint64_t strides[3] = {(uint64_t)cols * 2, 128, (uint64_t)(E > 0 ? estride : 0) * 2};
+    const uint32_t box[4] = {64, 64, chunks, 1};
+    return tc::make_map_nd(m, base, BF16, E > 0 ? 4 : 3, dims, strides, box);
+}
+
 }  // namespace bwd
 }  // namespace moe
 
@@ -559,7 +569,7 @@ int router_linear_bwd_tc(const void* dl, int64_t Ep, const void* x, const void* 
     if (dx) {
         CUtensorMap ma, mb;
         if (!make_map_2d(&ma, dl, bwd::BF16, 2, Ep, T, bwd::BM) ||
-            !make_map_3d(&mb, Wr, bwd::BF16, 2, d, E, 1, E * d, 64))
+            !bwd::make_mn_map(&mb, Wr, d, E, 1, E * d, 4))
             return MOE_ERR_CUDA;
         const int rc = bwd::launch<bwd::DXR>(ma, ma, mb, mb, ma, off_one, 1, T, Ep, 0, d, dx,
                                              nullptr, d, nullptr, nullptr, st);
@@ -567,8 +577,7 @@ int router_linear_bwd_tc(const void* dl, int64_t Ep, const void* x, const void* 
     }
     if (partial) {
         CUtensorMap ma, mb, mo;
-        if (!make_map_2d(&ma, dl, bwd::BF16, 2, Ep, T, 64) ||
-            !make_map_2d(&mb, x, bwd::BF16, 2, d, T, 64) ||
+        if (!bwd::make_mn_map(&ma, dl, Ep, T, 0, 0, 2) || !bwd::make_mn_map(&mb, x, d, T, 0, 0, 4) ||
             !make_map_2d(&mo, partial, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, G * Mp, 32))
             return MOE_ERR_CUDA;
         return bwd::launch<bwd::DWF>(ma, ma, mb, mb, mo, off_chunks, G, T, 0, Mp, d, nullptr,
@@ -588,11 +597,11 @@ int swiglu_wgrad(const void* Xe, const void* dA, const void* dB, const void* dYe
     using namespace tc;
     CUtensorMap gA, gB, gX, gY, gH;
     const int64_t Rm = R > 0 ? R : 1;  // a map needs a non-empty extent; no rows are read when R == 0
-    if (!make_map_2d(&gA, dA, bwd::BF16, 2, F, Rm, 64) ||
-        !make_map_2d(&gB, dB, bwd::BF16, 2, F, Rm, 64) ||
-        !make_map_2d(&gX, Xe, bwd::BF16, 2, d, Rm, 64) ||
-        !make_map_2d(&gY, dYe, bwd::BF16, 2, d, Rm, 64) ||
-        !make_map_2d(&gH, H, bwd::BF16, 2, F, Rm, 64))
+    // A operands (M side, 2 chunks = 128 columns) and B operands (N side, 4
+    // chunks = 256 columns) of the weight-gradient tiles
+    if (!bwd::make_mn_map(&gA, dA, F, Rm, 0, 0, 2) || !bwd::make_mn_map(&gB, dB, F, Rm, 0, 0, 2) ||
+        !bwd::make_mn_map(&gY, dYe, d, Rm, 0, 0, 2) || !bwd::make_mn_map(&gX, Xe, d, Rm, 0, 0, 4) ||
+        !bwd::make_mn_map(&gH, H, F, Rm, 0, 0, 4))
         return MOE_ERR_CUDA;
     CUtensorMap o1, o3, o2;  // the gradients as [E*M, N] for the TMA stores
     if (!make_map_2d(&o1, dW1, bwd::BF16, 2, d, E * F, 32) ||
@@ -646,7 +655,7 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
         // dH = dYe W2_e (+ pairwise SwiGLU backward) -> dA, dB
         CUtensorMap mA, mW2;
         if (!make_map_2d(&mA, dYe, bwd::BF16, 2, d, R, bwd::BM) ||
-            !make_map_3d(&mW2, W2, bwd::BF16, 2, F, d, E, w2_expert_stride, 64))
+            !bwd::make_mn_map(&mW2, W2, F, d, E, w2_expert_stride, 4))
             return MOE_ERR_CUDA;
         rc = bwd::launch<bwd::DH>(mA, mA, mW2, mW2, mA, offsets, E, R, d, 0, F, dA, dB, F, A, B,
                                   st);
@@ -655,8 +664,8 @@ extern "C" int moe_grouped_swiglu_bwd(const void* Xe, const void* A, const void*
         CUtensorMap mdA, mdB, mW1, mW3;
         if (!make_map_2d(&mdA, dA, bwd::BF16, 2, F, R, bwd::BM) ||
             !make_map_2d(&mdB, dB, bwd::BF16, 2, F, R, bwd::BM) ||
-            !make_map_3d(&mW1, W1, bwd::BF16, 2, d, F, E, w13_expert_stride, 64) ||
-            !make_map_3d(&mW3, W3, bwd::BF16, 2, d, F, E, w13_expert_stride, 64))
+            !bwd::make_mn_map(&mW1, W1, d, F, E, w13_expert_stride, 4) ||
+            !bwd::make_mn_map(&mW3, W3, d, F, E, w13_expert_stride, 4))
             return MOE_ERR_CUDA;
         rc = bwd::launch<bwd::DX>(mdA, mdB, mW1, mW3, mdA, offsets, E, R, 2 * F, 0, d, dXe,
                                   nullptr, d, nullptr, nullptr, st);
