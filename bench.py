@@ -5,8 +5,11 @@
                     [--also NAMES] [--impl ours|reference]
 
 One step = one pass of the whole layer over one batch: route (router logits,
-fp32 softmax + top-k, routing metadata) -> dispatch -> grouped gate/up GEMM
-with SwiGLU -> grouped down GEMM -> combine, each through the C ABI.
+fp32 softmax + top-k, routing metadata) -> dispatch (recording each row's
+gate) -> grouped gate/up GEMM with SwiGLU -> grouped down GEMM with the gates
+in its epilogue -> combine, each through the C ABI (the sequence
+moe_layer_fwd runs; with --backward the gates stay in the combine, since the
+router backward reads the expert rows unscaled).
 The default workload is the 128-expert layer of the expert-count sweep
 (T=8192, d=4096, E=128, top-4, ffn 2048, bf16, logits ~ N(0,1)), the
 configuration the layer's targets are stated on; the OLMoE-shaped layer
@@ -412,11 +415,23 @@ def _steps(moe, w, inp, dev, backward):
             else:
                 moe.moe_grouped_gate_up(Xe, W1, W3, rt.offsets, H=H)
 
-        fns = [("route", route),
-               ("dispatch", lambda: moe.moe_dispatch(x, rt.slot, out=Xe)),
-               ("gate_up", gate_up),
-               ("down", lambda: moe.moe_grouped_down(H, W2, rt.offsets, Ye=Ye)),
-               ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
+        if backward:
+            # the router backward reads Ye unscaled: gates in the combine
+            fns = [("route", route),
+                   ("dispatch", lambda: moe.moe_dispatch(x, rt.slot, out=Xe)),
+                   ("gate_up", gate_up),
+                   ("down", lambda: moe.moe_grouped_down(H, W2, rt.offsets, Ye=Ye)),
+                   ("combine", lambda: moe.moe_combine(Ye, rt.slot, rt.gate, out=out))]
+        else:
+            # as moe_layer_fwd runs it: the gates in the down GEMM's epilogue
+            row_gate = torch.empty(R, dtype=torch.float32, device=dev)
+            fns = [("route", route),
+                   ("dispatch", lambda: moe.moe_dispatch_gate(x, rt.slot, rt.gate, out=Xe,
+                                                              row_gate=row_gate)),
+                   ("gate_up", gate_up),
+                   ("down", lambda: moe.moe_grouped_down_gated(H, W2, rt.offsets, row_gate,
+                                                               Ye=Ye)),
+                   ("combine", lambda: moe.moe_combine(Ye, rt.slot, None, out=out))]
         sx, sw, sh = es, es, es
         if backward:
             dOut = inp["dOut"]
@@ -465,12 +480,15 @@ def _steps(moe, w, inp, dev, backward):
     torch.cuda.synchronize(dev)
     e_act = int((rt.counts > 0).sum().item())
     wbytes = e_act * F * d * sw
+    # the bf16/fp32 forward alone carries the gates from the dispatch (which
+    # records them per row) through the down epilogue, not to the combine
+    gated = not backward and not w.mxfp8
     work = {
         "route": (0.0, T * (d * es if use_router else E * 4) + R * 12),
-        "dispatch": (0.0, T * d * es + R * d * sx + R * 4),
+        "dispatch": (0.0, T * d * es + R * d * sx + R * 4 + (R * 8 if gated else 0)),
         "gate_up": (4.0 * R * d * F, R * d * sx + 2 * wbytes + R * F * sh),
-        "down": (2.0 * R * d * F, R * F * sh + wbytes + R * d * 2),
-        "combine": (0.0, R * d * 2 + T * d * 2 + R * 8),
+        "down": (2.0 * R * d * F, R * F * sh + wbytes + R * d * 2 + (R * 4 if gated else 0)),
+        "combine": (0.0, R * d * 2 + T * d * 2 + (R * 4 if gated else R * 8)),
     }
     if backward and w.mxfp8:
         q8 = 1 + 1 / 32  # an E4M3 code and its share of a scale byte

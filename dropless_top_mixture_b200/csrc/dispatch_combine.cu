@@ -42,13 +42,16 @@ struct Vec<MOE_F32> {
     }
 };
 
-// Xe[slot[t,j]] = x[t]   (SCALED: = round(gate[t,j] * x[t]))
+// Xe[slot[t,j]] = x[t]   (SCALED: = round(gate[t,j] * x[t]));
+// row_gate (if not null): row_gate[slot[t,j]] = gate[t,j], the gate of each
+// expert row for the down GEMM's epilogue
 template <int DT, bool SCALED>
 __global__ void __launch_bounds__(THREADS) dispatch_kernel(const uint4* __restrict__ x,
                                                            const int32_t* __restrict__ slot,
                                                            const float* __restrict__ gate,
                                                            int T, int k, int vpr, int64_t R,
-                                                           uint4* __restrict__ Xe, int* status) {
+                                                           uint4* __restrict__ Xe, int* status,
+                                                           float* __restrict__ row_gate) {
     __shared__ int s_slot[MOE_MAX_TOPK];
     __shared__ float s_gate[MOE_MAX_TOPK];
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
@@ -61,6 +64,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_kernel(const uint4* __restri
             }
             s_slot[threadIdx.x] = s;
             if (SCALED) s_gate[threadIdx.x] = gate[(size_t)t * k + threadIdx.x];
+            if (row_gate != nullptr && s >= 0) row_gate[s] = gate[(size_t)t * k + threadIdx.x];
         }
         __syncthreads();
         const uint4* src = x + (size_t)t * vpr;
@@ -176,8 +180,9 @@ inline int grid_for(int64_t T) {
 
 using namespace moe;
 
-extern "C" int moe_dispatch(const void* x, const int32_t* slot, const float* gate, int64_t T,
-                            int64_t d, int k, int dtype, void* Xe, void* stream) {
+static int dispatch_impl(const void* x, const int32_t* slot, const float* gate, bool scaled,
+                         int64_t T, int64_t d, int k, int dtype, void* Xe, float* row_gate,
+                         void* stream) {
     if (T < 0 || d <= 0 || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_INVALID;
     if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     const int es = dtype == MOE_F32 ? 4 : 2;
@@ -193,17 +198,29 @@ extern "C" int moe_dispatch(const void* x, const int32_t* slot, const float* gat
     const uint4* xs = static_cast<const uint4*>(x);
     uint4* xe = static_cast<uint4*>(Xe);
     if (dtype == MOE_BF16) {
-        if (gate)
-            dc::dispatch_kernel<MOE_BF16, true><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr());
+        if (scaled)
+            dc::dispatch_kernel<MOE_BF16, true><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr(), row_gate);
         else
-            dc::dispatch_kernel<MOE_BF16, false><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr());
+            dc::dispatch_kernel<MOE_BF16, false><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr(), row_gate);
     } else {
-        if (gate)
-            dc::dispatch_kernel<MOE_F32, true><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr());
+        if (scaled)
+            dc::dispatch_kernel<MOE_F32, true><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr(), row_gate);
         else
-            dc::dispatch_kernel<MOE_F32, false><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr());
+            dc::dispatch_kernel<MOE_F32, false><<<grid, dc::THREADS, 0, st>>>(xs, slot, gate, (int)T, k, vpr, R, xe, status_ptr(), row_gate);
     }
     return launch_status();
+}
+
+extern "C" int moe_dispatch(const void* x, const int32_t* slot, const float* gate, int64_t T,
+                            int64_t d, int k, int dtype, void* Xe, void* stream) {
+    return dispatch_impl(x, slot, gate, gate != nullptr, T, d, k, dtype, Xe, nullptr, stream);
+}
+
+extern "C" int moe_dispatch_gate(const void* x, const int32_t* slot, const float* gate, int64_t T,
+                                 int64_t d, int k, int dtype, void* Xe, float* row_gate,
+                                 void* stream) {
+    if (T > 0 && (!gate || !row_gate)) return MOE_ERR_INVALID;
+    return dispatch_impl(x, slot, gate, false, T, d, k, dtype, Xe, row_gate, stream);
 }
 
 extern "C" int moe_combine(const void* Ye, const int32_t* slot, const float* gate, int64_t T,

@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const int32_t* __restrict__ offsets, int E, int R, int K, int N,
                         TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
                         TIn* __restrict__ save_b, int* status,
-                        const int32_t* __restrict__ row_token, int x_rows, int b_mode) {
+                        const int32_t* __restrict__ row_token, int x_rows, int b_mode,
+                        const float* __restrict__ row_gate) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -396,6 +397,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int grow = tl.row0 + r_in_tile;
             const bool valid = grow < tl.row_end;
             TIn* orow = out + (size_t)(valid ? grow : 0) * ldo + tl.n0;
+            // down with gates: the row's gate scales its fp32 sums
+            const float g = (!SWIGLU && row_gate != nullptr && valid) ? __ldg(row_gate + grow) : 1.f;
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t a[32];
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 } else {
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                    for (int j = 0; j < 32; ++j) v[j] = g * __uint_as_float(a[j]);
                 }
                 if (valid) Store32<TIn>::run(orow + c * 32, v);
             }
@@ -442,7 +445,8 @@ template <typename TIn, bool SWIGLU, int MMA_N, bool GATHER = false>
 static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                   const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N, void* out,
                   int64_t ldo, cudaStream_t st, void* save_a = nullptr, void* save_b = nullptr,
-                  const int32_t* row_token = nullptr, int64_t x_rows = 0, int b_mode = 0) {
+                  const int32_t* row_token = nullptr, int64_t x_rows = 0, int b_mode = 0,
+                  const float* row_gate = nullptr) {
     using C = Cfg<TIn, SWIGLU, MMA_N>;
     auto kern = grouped_gemm_kernel<TIn, SWIGLU, MMA_N, GATHER>;
     if (check_only()) return MOE_OK;
@@ -462,7 +466,7 @@ static int launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap
     kern<<<grid, THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K, (int)N,
                                               static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a),
                                               static_cast<TIn*>(save_b), status_ptr(), row_token,
-                                              (int)x_rows, b_mode);
+                                              (int)x_rows, b_mode, row_gate);
     return launch_status();
 }
 
@@ -498,7 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                              const __grid_constant__ CUtensorMap tmB1,
                              const int32_t* __restrict__ offsets, int E, int R, int K, int N,
                              TIn* __restrict__ out, int64_t ldo, TIn* __restrict__ save_a,
-                             TIn* __restrict__ save_b, int* status) {
+                             TIn* __restrict__ save_b, int* status,
+                             const float* __restrict__ row_gate) {
     constexpr bool TF32 = std::is_same<TIn, float>::value;
     constexpr int BK = 128 / (int)sizeof(TIn);
     constexpr int MMA_N = 256;
@@ -711,6 +716,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int grow = s_off[lo] + m * pr::PM + (int)rank * BM + r_in_tile;
             const bool valid = grow < row_end;
             TIn* orow = out + (size_t)(valid ? grow : 0) * ldo + n0;
+            const float g = (!SWIGLU && row_gate != nullptr && valid) ? __ldg(row_gate + grow) : 1.f;
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c) {
                 uint32_t a[32];
@@ -731,7 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 } else {
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                    for (int j = 0; j < 32; ++j) v[j] = g * __uint_as_float(a[j]);
                 }
                 if (valid) Store32<TIn>::run(orow + c * 32, v);
             }
@@ -754,7 +760,7 @@ template <typename TIn, bool SWIGLU>
 static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const int32_t* offsets, int64_t E, int64_t R, int64_t K, int64_t N,
                        void* out, int64_t ldo, cudaStream_t st, void* save_a = nullptr,
-                       void* save_b = nullptr) {
+                       void* save_b = nullptr, const float* row_gate = nullptr) {
     auto kern = grouped_gemm_pair_kernel<TIn, SWIGLU>;
     if (check_only()) return MOE_OK;
     static bool attr_done[64] = {false};
@@ -774,7 +780,8 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
     kern<<<2 * npairs, THREADS, pr::SMEM_BYTES, st>>>(a, b0, b1, offsets, (int)E, (int)R, (int)K,
                                                       (int)N, static_cast<TIn*>(out), ldo,
                                                       static_cast<TIn*>(save_a),
-                                                      static_cast<TIn*>(save_b), status_ptr());
+                                                      static_cast<TIn*>(save_b), status_ptr(),
+                                                      row_gate);
     return launch_status();
 }
 
@@ -874,7 +881,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                              const __grid_constant__ sw::TokenMaps tmX,
                              const int32_t* __restrict__ offsets, int E, int R, int K, int NOUT,
                              int wpe, int second_is_gate, TIn* __restrict__ out, int64_t ldo,
-                             TIn* __restrict__ save_a, TIn* __restrict__ save_b, int* status) {
+                             TIn* __restrict__ save_a, TIn* __restrict__ save_b, int* status,
+                             const float* __restrict__ row_gate) {
     constexpr bool TF32 = std::is_same<TIn, float>::value;
     constexpr int BK = 128 / (int)sizeof(TIn);
     constexpr uint32_t IDESC_M = make_idesc(TF32 ? 2u : 1u, 256, 0);  // N filled per tile
@@ -1110,10 +1118,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             out[(size_t)tok * ldo + f] = sw::to_out<TIn>(silu_mul(g, u));
                     }
                 } else {
+                    // down with gates: column j is token row tok0 + j; lane j
+                    // fetches its gate and the shuffle hands it to every lane
+                    float gl = 1.f;
+                    if (row_gate != nullptr && tok0 + lane < c.row_end) gl = __ldg(row_gate + tok0 + lane);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
+                    for (int j = 0; j < 32; ++j) {
+                        const float gj = __shfl_sync(0xffffffffu, gl, j);
                         if (tok0 + j < c.row_end)
-                            out[(size_t)(tok0 + j) * ldo + f] = sw::to_out<TIn>(__uint_as_float(a[j]));
+                            out[(size_t)(tok0 + j) * ldo + f] =
+                                sw::to_out<TIn>(gj * __uint_as_float(a[j]));
+                    }
                 }
             }
             tc_fence_before();
@@ -1191,7 +1206,7 @@ template <typename TIn, bool SWIGLU>
 static int launch_swap(const CUtensorMap& w, const sw::TokenMaps& x, const int32_t* offsets,
                        int64_t E, int64_t R, int64_t K, int64_t NOUT, int wpe, int second_is_gate,
                        void* out, int64_t ldo, cudaStream_t st, void* save_a = nullptr,
-                       void* save_b = nullptr) {
+                       void* save_b = nullptr, const float* row_gate = nullptr) {
     auto kern = grouped_gemm_swap_kernel<TIn, SWIGLU>;
     if (check_only()) return MOE_OK;
     static bool attr_done[64] = {false};
@@ -1211,7 +1226,7 @@ static int launch_swap(const CUtensorMap& w, const sw::TokenMaps& x, const int32
     kern<<<2 * npairs, THREADS, sw::SMEM_BYTES, st>>>(
         w, x, offsets, (int)E, (int)R, (int)K, (int)NOUT, wpe, second_is_gate,
         static_cast<TIn*>(out), ldo, static_cast<TIn*>(save_a), static_cast<TIn*>(save_b),
-        status_ptr());
+        status_ptr(), row_gate);
     return launch_status();
 }
 
@@ -1355,9 +1370,9 @@ extern "C" int moe_grouped_gate_up_gather(const void* x, const int32_t* row_toke
                                               nullptr, row_token, T);
 }
 
-extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
-                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
-                                int64_t F, int dtype, void* Ye, void* stream) {
+static int grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
+                        const int32_t* offsets, const float* row_gate, int64_t E, int64_t R,
+                        int64_t d, int64_t F, int dtype, void* Ye, void* stream) {
     int rc = gg::check_common(H, W2, offsets, E, R, d, F, dtype);
     if (rc != MOE_OK) return rc;
     if (!Ye || !aligned16(Ye)) return MOE_ERR_INVALID;
@@ -1378,8 +1393,9 @@ extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert
         cudaStream_t st = as_stream(stream);
         if (dtype == MOE_BF16)
             return gg::launch_swap<__nv_bfloat16, false>(b0, xm, offsets, E, R, F, d, wpe, 0, Ye, d,
-                                                          st);
-        return gg::launch_swap<float, false>(b0, xm, offsets, E, R, F, d, wpe, 0, Ye, d, st);
+                                                          st, nullptr, nullptr, row_gate);
+        return gg::launch_swap<float, false>(b0, xm, offsets, E, R, F, d, wpe, 0, Ye, d, st,
+                                             nullptr, nullptr, row_gate);
     }
     const bool pair = mma_n == 256 && gg::use_pair(R, E);
     if (!gg::make_map_2d(&a, H, dt, es, F, R, gg::BM) ||
@@ -1388,16 +1404,37 @@ extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert
     cudaStream_t st = as_stream(stream);
     if (pair) {
         if (dtype == MOE_BF16)
-            return gg::launch_pair<__nv_bfloat16, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
-        return gg::launch_pair<float, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+            return gg::launch_pair<__nv_bfloat16, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st,
+                                                          nullptr, nullptr, row_gate);
+        return gg::launch_pair<float, false>(a, b0, b0, offsets, E, R, F, d, Ye, d, st, nullptr,
+                                             nullptr, row_gate);
     }
     if (dtype == MOE_BF16) {
         if (mma_n == 256)
-            return gg::launch<__nv_bfloat16, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
-        return gg::launch<__nv_bfloat16, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+            return gg::launch<__nv_bfloat16, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st,
+                                                          nullptr, nullptr, nullptr, 0, 0, row_gate);
+        return gg::launch<__nv_bfloat16, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st,
+                                                      nullptr, nullptr, nullptr, 0, 0, row_gate);
     }
-    if (mma_n == 256) return gg::launch<float, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
-    return gg::launch<float, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st);
+    if (mma_n == 256)
+        return gg::launch<float, false, 256>(a, b0, b0, offsets, E, R, F, d, Ye, d, st, nullptr,
+                                             nullptr, nullptr, 0, 0, row_gate);
+    return gg::launch<float, false, 128>(a, b0, b0, offsets, E, R, F, d, Ye, d, st, nullptr,
+                                         nullptr, nullptr, 0, 0, row_gate);
+}
+
+extern "C" int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
+                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
+                                int64_t F, int dtype, void* Ye, void* stream) {
+    return grouped_down(H, W2, w2_expert_stride, offsets, nullptr, E, R, d, F, dtype, Ye, stream);
+}
+
+extern "C" int moe_grouped_down_gated(const void* H, const void* W2, int64_t w2_expert_stride,
+                                      const int32_t* offsets, const float* row_gate, int64_t E,
+                                      int64_t R, int64_t d, int64_t F, int dtype, void* Ye,
+                                      void* stream) {
+    if (R > 0 && !row_gate) return MOE_ERR_INVALID;
+    return grouped_down(H, W2, w2_expert_stride, offsets, row_gate, E, R, d, F, dtype, Ye, stream);
 }
 
 extern "C" int moe_debug_set_gemm_form(int form) {

@@ -51,6 +51,7 @@ struct Carve {
     void* Xe;
     void* H;
     void* Ye;
+    float* row_gate;  // gate of each expert row, for the down GEMM's epilogue
     void* route_ws;
     size_t route_bytes;
     size_t total;
@@ -69,6 +70,8 @@ inline Carve carve(void* base, int64_t T, int64_t d, int64_t E, int64_t F, int k
     off += a256(R * F * es);
     c.Ye = p + off;
     off += a256(R * d * es);
+    c.row_gate = reinterpret_cast<float*>(p + off);
+    off += a256(R * sizeof(float));
     c.route_ws = p + off;
     c.route_bytes = moe_route_workspace_size(T, E, logits_given ? 0 : 1);
     off += a256(c.route_bytes);
@@ -126,15 +129,25 @@ static int fwd_steps(const moe_layer_args* a, const Carve& c, void* stream) {
     void* Xe = a->save_Xe ? a->save_Xe : c.Xe;
     void* H = a->save_H ? a->save_H : c.H;
     void* Ye = a->save_Ye ? a->save_Ye : c.Ye;
-    rc = moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, Xe, stream);
+    // Without a kept Ye (which the router backward reads unscaled) the gates
+    // go into the down GEMM's epilogue ("olmoforge" README, capability
+    // table: the expert path fused with the routing weights), the dispatch
+    // recording each row's gate, and the combine adds the k rows as they are.
+    const bool gated = a->save_Ye == nullptr;
+    rc = gated ? moe_dispatch_gate(a->x, a->slot, a->gate, a->T, a->d, a->k, a->dtype, Xe,
+                                   c.row_gate, stream)
+               : moe_dispatch(a->x, a->slot, nullptr, a->T, a->d, a->k, a->dtype, Xe, stream);
     if (rc != MOE_OK) return rc;
     rc = moe_grouped_gate_up_save(Xe, a->W1, a->W3, a->w13_expert_stride, a->offsets, a->E, R,
                                   a->d, a->F, a->dtype, H, a->save_A, a->save_B, stream);
     if (rc != MOE_OK) return rc;
-    rc = moe_grouped_down(H, a->W2, a->w2_expert_stride, a->offsets, a->E, R, a->d, a->F,
-                          a->dtype, Ye, stream);
+    rc = gated ? moe_grouped_down_gated(H, a->W2, a->w2_expert_stride, a->offsets, c.row_gate,
+                                        a->E, R, a->d, a->F, a->dtype, Ye, stream)
+               : moe_grouped_down(H, a->W2, a->w2_expert_stride, a->offsets, a->E, R, a->d, a->F,
+                                  a->dtype, Ye, stream);
     if (rc != MOE_OK) return rc;
-    return moe_combine(Ye, a->slot, a->gate, a->T, a->d, a->k, a->dtype, a->out, stream);
+    return moe_combine(Ye, a->slot, gated ? nullptr : a->gate, a->T, a->d, a->k, a->dtype,
+                       a->out, stream);
 }
 
 }  // namespace layer

@@ -114,6 +114,8 @@ _SIGS = {
     "moe_route_noalloc": (_i32, [_p, _p, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _p, _p, _p,
                                  _p, _p, _p, _p]),
     "moe_dispatch": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p]),
+    "moe_dispatch_gate": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _p, _p]),
+    "moe_grouped_down_gated": (_i32, [_p, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_grouped_gate_up": (_i32, [_p, _p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_grouped_down": (_i32, [_p, _p, _i64, _p, _i64, _i64, _i64, _i64, _i32, _p, _p]),
     "moe_row_token": (_i32, [_p, _i64, _i32, _p, _p]),
@@ -295,6 +297,24 @@ def moe_dispatch(x: torch.Tensor, slot: torch.Tensor, gate: Optional[torch.Tenso
     return out
 
 
+def moe_dispatch_gate(x: torch.Tensor, slot: torch.Tensor, gate: torch.Tensor,
+                      out: Optional[torch.Tensor] = None,
+                      row_gate: Optional[torch.Tensor] = None):
+    """Unscaled dispatch that also records row_gate[slot[t,j]] = gate[t,j];
+    returns (Xe, row_gate)."""
+    _need(x, "x"); _need(slot, "slot"); _need(gate, "gate")
+    T, d = x.shape
+    k = slot.shape[1]
+    if out is None:
+        out = torch.empty((T * k, d), dtype=x.dtype, device=x.device)
+    if row_gate is None:
+        row_gate = torch.empty(T * k, dtype=torch.float32, device=x.device)
+    rc = lib.moe_dispatch_gate(_ptr(x), _ptr(slot), _ptr(gate), T, d, k, _dtype_code(x.dtype),
+                               _ptr(out), _ptr(row_gate), _stream(x))
+    _check("moe_dispatch_gate", rc)
+    return out, row_gate
+
+
 def _w13(W1: torch.Tensor, W3: torch.Tensor):
     # [E,F,d] tensors, or views into a fused [E,2F,d] gate/up tensor
     E, F, d = W1.shape
@@ -404,6 +424,20 @@ def moe_grouped_down(H, W2, offsets, Ye: Optional[torch.Tensor] = None) -> torch
     rc = lib.moe_grouped_down(_ptr(H), _ptr(W2), s2, _ptr(offsets), E, R, d, F,
                               _dtype_code(H.dtype), _ptr(Ye), _stream(H))
     _check("moe_grouped_down", rc)
+    return Ye
+
+
+def moe_grouped_down_gated(H, W2, offsets, row_gate, Ye: Optional[torch.Tensor] = None):
+    """moe_grouped_down with each row's sums scaled by row_gate[r] before
+    rounding (the gates from moe_dispatch_gate)."""
+    _need(H, "H"); _need(offsets, "offsets"); _need(row_gate, "row_gate")
+    E, d, F, s2 = _w2(W2)
+    R = H.shape[0]
+    if Ye is None:
+        Ye = torch.empty((R, d), dtype=H.dtype, device=H.device)
+    rc = lib.moe_grouped_down_gated(_ptr(H), _ptr(W2), s2, _ptr(offsets), _ptr(row_gate), E, R,
+                                    d, F, _dtype_code(H.dtype), _ptr(Ye), _stream(H))
+    _check("moe_grouped_down_gated", rc)
     return Ye
 
 

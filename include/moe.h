@@ -190,6 +190,13 @@ MOE_API int moe_route_noalloc(const float* logits, const void* x, const void* Wr
  * ---------------------------------------------------------------------- */
 MOE_API int moe_dispatch(const void* x, const int32_t* slot, const float* gate, int64_t T,
                          int64_t d, int k, int dtype, void* Xe, void* stream);
+/* moe_dispatch_gate — the unscaled dispatch that also records each expert
+ * row's gate, row_gate[slot[t,j]] = gate[t,j] (fp32 [R], device), for
+ * moe_grouped_down_gated. gate [T,k] and row_gate must be non-NULL when
+ * T > 0; otherwise as moe_dispatch. */
+MOE_API int moe_dispatch_gate(const void* x, const int32_t* slot, const float* gate, int64_t T,
+                              int64_t d, int k, int dtype, void* Xe, float* row_gate,
+                              void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_row_token — the inverse of the slot map: row_token[slot[t,j]] = t,
@@ -242,6 +249,16 @@ MOE_API int moe_grouped_gate_up(const void* Xe, const void* W1, const void* W3,
 MOE_API int moe_grouped_down(const void* H, const void* W2, int64_t w2_expert_stride,
                              const int32_t* offsets, int64_t E, int64_t R, int64_t d, int64_t F,
                              int dtype, void* Ye, void* stream);
+/* moe_grouped_down with the routing weights in its epilogue ([OF]
+ * capability table; "Transformers 中的 OLMoE" §3 multiplies each expert's
+ * output by its top-k weight): Ye[r] = round_dtype(row_gate[r] *
+ * fp32(H[r]·W2_eᵀ)), so the combine adds the k rows of a token with unit
+ * gates (moe_combine with gate = NULL). row_gate [R] fp32 from
+ * moe_dispatch_gate, non-NULL when R > 0; otherwise as moe_grouped_down. */
+MOE_API int moe_grouped_down_gated(const void* H, const void* W2, int64_t w2_expert_stride,
+                                   const int32_t* offsets, const float* row_gate, int64_t E,
+                                   int64_t R, int64_t d, int64_t F, int dtype, void* Ye,
+                                   void* stream);
 MOE_API int moe_grouped_swiglu(const void* Xe, const void* W1, const void* W3, const void* W2,
                                int64_t w13_expert_stride, int64_t w2_expert_stride,
                                const int32_t* offsets, int64_t E, int64_t R, int64_t d,
@@ -486,7 +503,11 @@ typedef struct moe_layer_args {
     int32_t* counts;        /* [E]                                            */
     int32_t* offsets;       /* [E+1]                                          */
     int32_t* slot;          /* [T,k]                                          */
-    /* scratch (device): Xe [R,d], H [R,F], Ye [R,d] and the route workspace */
+    /* scratch (device): Xe [R,d], H [R,F], Ye [R,d], the rows' gates [R] and
+     * the route workspace. Without save_Ye the layer applies the gates in
+     * the down GEMM's epilogue (moe_dispatch_gate, moe_grouped_down_gated,
+     * unit-gate combine); with save_Ye it keeps Ye unscaled for the router
+     * backward and the combine applies the gates. */
     void* workspace;
     size_t workspace_bytes;
     /* optional (device, NULL = not kept): rows kept for moe_layer_bwd. When

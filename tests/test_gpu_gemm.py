@@ -212,6 +212,61 @@ def test_grouped_gate_up_fused_gate_up_layout():
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("counts,form", [(TAIL_COUNTS, "rows"), (TAIL_COUNTS, "tokens"),
+                                         (LARGER_COUNTS, "rows"), (LARGER_COUNTS, "tokens"),
+                                         ([600, 700, 0, 1300], "rows")])
+def test_grouped_down_gated_every_tail_size(dtype, counts, form):
+    """The down GEMM with each row's gate applied in the epilogue, on row
+    tiles (the last case on CTA-pair row tiles: experts averaging 650 rows)
+    and on token-column tiles: Ye[r] = gate[r] * (H[r] W2_e^T)."""
+    moe = _moe()
+    counts = np.array(counts, dtype=np.int64)
+    E, R, d, F = len(counts), int(counts.sum()), 512, 256
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    g = torch.Generator().manual_seed(R)
+    H = torch.randn(R, F, generator=g).to(dtype)
+    W2 = (torch.randn(E, d, F, generator=g) * F ** -0.5).to(dtype)
+    rg = torch.rand(R, generator=g) * 0.9 + 0.05
+    ref = np.empty((R, d))
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        ref[a:b] = np64(H[a:b]) @ np64(W2[e]).T
+    ref *= rg.double().numpy()[:, None]
+    offs = torch.from_numpy(offsets).cuda()
+    Ye = torch.full((R, d), float("nan"), dtype=dtype, device="cuda")
+    with _gemm_form(form):
+        moe.moe_grouped_down_gated(H.cuda(), W2.cuda(), offs, rg.cuda(), Ye=Ye)
+        plain = moe.moe_grouped_down(H.cuda(), W2.cuda(), offs)
+    assert moe.moe_get_status() == 0
+    assert torch.isfinite(Ye.float()).all()
+    assert_close_scaled(np64(Ye), ref, "Ye")
+    # the gate multiplies the fp32 sum once: within one rounding of the
+    # ungated row times the gate
+    unit = 2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -23
+    scaled = np64(plain) * rg.double().numpy()[:, None]
+    assert np.all(np.abs(np64(Ye) - scaled) <= 2.5 * unit * np.abs(scaled) + 1e-30)
+
+
+@pytest.mark.parametrize("form", ["rows", "tokens"])
+def test_layer_fwd_gates_in_down_epilogue(form):
+    """moe_layer_fwd without kept rows applies the gates in the down GEMM's
+    epilogue; with them (save) the combine applies them. Both match the
+    oracle, and the routing is the same."""
+    moe = _moe()
+    T, d, F, E, k = 1100, 256, 256, 4, 2
+    x, W1, W3, W2, lg = _problem(T, d, F, E, k, torch.bfloat16, seed=46)
+    ref = O.moe_layer(x, k, W1, W3, W2, logits=lg)
+    with _gemm_form(form):
+        args = (x.cuda(), k, W1.cuda(), W3.cuda(), W2.cuda())
+        gated = moe.moe_layer_fwd(*args, logits=torch.from_numpy(lg).cuda())
+        kept = moe.moe_layer_fwd(*args, logits=torch.from_numpy(lg).cuda(), save=True)
+    assert moe.moe_get_status() == 0
+    assert torch.equal(gated.idx, kept.idx) and torch.equal(gated.slot, kept.slot)
+    assert_close_layer(np64(gated.out), ref["out"], "out (gated)")
+    assert_close_layer(np64(kept.out), ref["out"], "out (kept)")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_token_tiles_equal_row_tiles_bitwise(dtype):
     """Both tile forms sum each output over K in the same order, so H, the
     saved pre-activations and Ye agree bit for bit."""

@@ -50,6 +50,35 @@ def test_dispatch_scaled_by_gate():
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,d,E,k", [(1, 8, 4, 2), (33, 136, 8, 3), (517, 2048, 64, 8)])
+def test_dispatch_gate_records_row_gates(dtype, T, d, E, k):
+    """The gate-recording dispatch writes the same rows as moe_dispatch, bit
+    for bit, and row_gate[slot[t,j]] = gate[t,j] exactly."""
+    moe = _moe()
+    gate, meta = _routing(T, E, k, seed=T + 7)
+    x = torch.randn(T, d, generator=torch.Generator().manual_seed(d + 1)).to(dtype).cuda()
+    slot = torch.from_numpy(meta["slot"]).cuda()
+    g32 = torch.from_numpy(gate).float().cuda()
+    Xe, row_gate = moe.moe_dispatch_gate(x, slot, g32)
+    assert moe.moe_get_status() == 0
+    assert torch.equal(Xe, moe.moe_dispatch(x, slot))
+    want = np.empty(T * k, dtype=np.float32)
+    want[meta["slot"].reshape(-1)] = gate.astype(np.float32).reshape(-1)
+    assert np.array_equal(row_gate.cpu().numpy(), want)
+
+
+def test_dispatch_gate_flags_bad_slot():
+    moe = _moe()
+    x = torch.ones(2, 64, dtype=torch.bfloat16, device="cuda")
+    slot = torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda")  # 9 >= R = 4
+    gate = torch.full((2, 2), 0.5, device="cuda")
+    row_gate = torch.full((4,), -1.0, device="cuda")
+    moe.moe_dispatch_gate(x, slot, gate, row_gate=row_gate)
+    assert moe.moe_get_status() == moe.MOE_DEVERR_BAD_INDEX
+    assert row_gate.tolist() == [0.5, 0.5, 0.5, -1.0]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("T,d,E,k", [(1, 8, 4, 2), (33, 136, 8, 3), (517, 2048, 64, 8),
                                      (64, 7168, 384, 8)])
 def test_combine(dtype, T, d, E, k):
