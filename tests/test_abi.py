@@ -75,6 +75,18 @@ def test_host_validation_rejects_without_launch(lib):
     assert L.moe_grouped_gate_up_gather(p16, p16, 0, p16, p16, 128 * 128, p16, 4, 20, 128, 128,
                                         m.MOE_BF16, p16, None) == m.MOE_ERR_INVALID
     assert L.moe_row_token(p16, 4, 0, p16, None) == m.MOE_ERR_INVALID
+    # the gate-recording dispatch needs the gates and somewhere to put them;
+    # the gated down GEMM needs the row gates
+    assert L.moe_dispatch_gate(p16, p16, None, 4, 64, 2, m.MOE_BF16, p16, p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_dispatch_gate(p16, p16, p16, 4, 64, 2, m.MOE_BF16, p16, None, None) == m.MOE_ERR_INVALID
+    assert L.moe_dispatch_gate(p16, p16, None, 0, 64, 2, m.MOE_BF16, p16, None, None) == m.MOE_OK
+    assert L.moe_grouped_down_gated(p16, p16, 128 * 128, p16, None, 2, 8, 128, 128, m.MOE_BF16,
+                                    p16, None) == m.MOE_ERR_INVALID
+    assert L.moe_grouped_down_gated(p16, p16, 128 * 128, p16, None, 2, 0, 128, 128, m.MOE_BF16,
+                                    p16, None) == m.MOE_OK
+    # tile-form hook: 0, 1, 2 only
+    assert L.moe_debug_set_gemm_form(3) == m.MOE_ERR_INVALID
+    assert L.moe_debug_set_gemm_form(0) == m.MOE_OK
     # T == 0 is a no-op
     assert L.moe_dispatch(p16, p16, None, 0, 64, 2, m.MOE_BF16, p16, None) == m.MOE_OK
     assert L.moe_row_token(p16, 0, 2, p16, None) == m.MOE_OK
