@@ -7,16 +7,11 @@
 // table built from the routing offsets, so the host never learns the
 // per-expert row counts.
 //
-// Two products, each in three tile forms:
+// Two instantiations:
 //   gate_up  H[r]  = silu(Xe[r] W1_eᵀ) * (Xe[r] W3_eᵀ)   B tile = [W1 rows; W3 rows]
-//   down     Ye[r] = H[r] W2_eᵀ   (optionally times the row's gate, g[r], in
-//                                   the epilogue)
-// Row tiles (grouped_gemm_kernel, below), CTA-pair row tiles
-// (grouped_gemm_pair_kernel, 256 rows) and token-column tiles
-// (grouped_gemm_swap_kernel: the weights as the MMA's M side, an expert's
-// tokens as N); the host picks one by shape.
+//   down     Ye[r] = H[r] W2_eᵀ
 //
-// Row tiles: 128 rows (one expert's rows; the last tile of an expert overlaps the
+// Tile = 128 rows (one expert's rows; the last tile of an expert overlaps the
 // next expert's rows, which are computed and masked at the store) x MMA_N
 // columns of B. One 128xMMA_Nx16 MMA per 32 bytes of K; K is staged 128
 // bytes at a time by TMA with the 128-byte swizzle the MMA descriptors read.
