@@ -96,3 +96,20 @@ def test_expert_parallel_count_exchange_world3():
         assert allc == expect
         assert mine == list(range(rank * 4, rank * 4 + 4))
         assert rows_max == 3 * 300 * 4
+
+
+def test_expert_parallel_split_and_sizing():
+    """The expert split is contiguous and covers every expert once; an
+    expert count that does not divide over the ranks is refused; receive
+    buffers hold the dropless worst case (every token of every rank)."""
+    from dropless_top_mixture_b200 import ep
+    for E, G in ((64, 8), (12, 3), (7, 1), (128, 4)):
+        seen = []
+        for r in range(G):
+            blk = list(ep.owned_experts(E, G, r))
+            assert blk == list(range(r * E // G, (r + 1) * E // G))
+            seen += blk
+        assert seen == list(range(E))
+    with pytest.raises(ValueError):
+        ep.owned_experts(10, 4, 0)
+    assert ep.receive_rows_max(T_max=300, k=4, G=3) == 3 * 300 * 4
